@@ -1,0 +1,391 @@
+"""Benchmark of the Sparse GQA hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path (merge -> index/top-k -> sparse
+attention) over one sequence of the workload: for the default ``prefill128k``
+that is a 131072-token prefill in 16 chunks of 8192 queries, every chunk one
+``sgqa_forward`` call.  Inputs are synthetic (``inputs.py``), resident in HBM
+before timing, and larger than L2 (one 8192-query Q chunk is 201 MB).  With
+N > 1 (torchrun, one process per GPU) every rank runs its own sequence: no
+data-path collective, weak scaling, time = max over ranks.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the CPU oracle on a
+bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_long_context_sgqa_b200 import inputs as I  # noqa: E402
+
+METRIC = {
+    "prefill128k": ("sparse_gqa_prefill_tokens_per_s_128k", "tokens/s"),
+    "prefill8k": ("sparse_gqa_prefill_tokens_per_s_8k", "tokens/s"),
+    "prefill1m": ("sparse_gqa_prefill_tokens_per_s_1m", "tokens/s"),
+    "prefill1m_b1": ("sparse_gqa_prefill_tokens_per_s_1m_b1", "tokens/s"),
+    "decode": ("sparse_gqa_decode_tokens_per_s", "tokens/s"),
+}
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work (what the method itself must do), per call
+# ---------------------------------------------------------------------------
+
+def attn_flops(cnt: torch.Tensor, q_pos0: int, wl) -> float:
+    """4 * D * Hg flops per attended (query, token, group): QK^T and PV, union waste excluded."""
+    nq = cnt.shape[1]
+    t = torch.arange(q_pos0, q_pos0 + nq, device=cnt.device, dtype=torch.int64)
+    cur = (t % wl.block + 1)[None, :, None]
+    tokens = cnt.to(torch.int64) * wl.block + cur
+    return float(tokens.sum().item()) * 4 * wl.head_dim * wl.heads_per_group
+
+
+def index_flops(q_pos0: int, nq: int, wl, num_seqs: int = 1) -> float:
+    t = np.arange(q_pos0, q_pos0 + nq, dtype=np.int64)
+    pairs = float((t // wl.block).sum()) * wl.groups * num_seqs
+    return pairs * wl.idx_heads * wl.idx_dim * 2
+
+
+def attn_bytes_decode(cnt: torch.Tensor, q_pos0: int, wl) -> float:
+    t = q_pos0
+    tokens = cnt.to(torch.int64) * wl.block + (t % wl.block + 1)
+    return float(tokens.sum().item()) * wl.head_dim * 2 * 2
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nme, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(nme)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the CUDA arm
+# ---------------------------------------------------------------------------
+
+def setup(wl, dev, seq):
+    from sparse_long_context_sgqa_b200.api import SparseGQA
+    from sparse_long_context_sgqa_b200.binding import Params
+    p = Params(num_kv_groups=wl.groups, heads_per_group=wl.heads_per_group, head_dim=wl.head_dim,
+               idx_heads=wl.idx_heads, idx_dim=wl.idx_dim, block_size=wl.block, topk=wl.topk,
+               merge_in_f32=1 if wl.fp32_inputs else 0)
+    S = wl.num_seqs
+    model = SparseGQA(p, S, wl.seq_len, min(wl.chunk, wl.nq), dev)
+    for s in range(S):
+        c = I.make_cache(wl, dev, seq=seq * S + s)
+        for name in ("kp", "c", "k", "v"):
+            getattr(model, name)[s].copy_(c[name])
+        del c
+    qs = [I.make_queries(wl, dev, wl.q_start, wl.nq, seq=seq * S + s) for s in range(S)]
+    q = {n: torch.stack([x[n] for x in qs]).contiguous() for n in qs[0]}
+    del qs
+    if wl.q_start // wl.block > 0:  # earlier blocks of a decode context: merged before the step
+        from sparse_long_context_sgqa_b200 import binding as Bd
+        Bd.sgqa_merge_blocks(p, S, wl.seq_len, model.kp, model.c, 0, wl.q_start // wl.block, None, model.store)
+    out = torch.empty((S, wl.nq, wl.n_heads, wl.head_dim), dtype=torch.bfloat16, device=dev)
+    sel = torch.empty((S, wl.nq, wl.groups, wl.topk), dtype=torch.int32, device=dev)
+    cnt = torch.empty((S, wl.nq, wl.groups), dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+    return p, model, q, out, sel, cnt
+
+
+def stage_times(wl, p, model, q, dev):
+    """One step with CUDA events between the stage calls; returns per-stage ms and work."""
+    from sparse_long_context_sgqa_b200 import binding as Bd
+    S, B, G, k = wl.num_seqs, wl.block, wl.groups, wl.topk
+    chunk = min(wl.chunk, wl.nq)
+    st = torch.cuda.current_stream()
+    ms = {"merge": 0.0, "index": 0.0, "attention": 0.0}
+    work = {"attn_flops": 0.0, "index_flops": 0.0, "attn_bytes": 0.0, "launches": 0}
+    for c0 in range(0, wl.nq, chunk):
+        n = min(chunk, wl.nq - c0)
+        q0 = wl.q_start + c0
+        sel = torch.empty((S, n, G, k), dtype=torch.int32, device=dev)
+        cnt = torch.empty((S, n, G), dtype=torch.int32, device=dev)
+        out = torch.empty((S, n, wl.n_heads, wl.head_dim), dtype=torch.bfloat16, device=dev)
+        qs = {nme: q[nme][:, c0:c0 + n].contiguous() for nme in q}
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(st)
+        Bd.sgqa_merge_blocks(p, S, wl.seq_len, model.kp, model.c, q0 // B, (q0 + n) // B, None, model.store)
+        ev[1].record(st)
+        Bd.sgqa_index_topk(p, S, q0, n, qs["idx_q"], qs["idx_w"], wl.seq_len, model.store, sel, cnt, model.ws)
+        ev[2].record(st)
+        Bd.sgqa_sparse_attn(p, S, q0, n, qs["q"], wl.seq_len, wl.seq_len, model.k, model.v, sel, cnt, out,
+                            model.ws)
+        ev[3].record(st)
+        torch.cuda.synchronize()
+        ms["merge"] += ev[0].elapsed_time(ev[1])
+        ms["index"] += ev[1].elapsed_time(ev[2])
+        ms["attention"] += ev[2].elapsed_time(ev[3])
+        work["attn_flops"] += attn_flops(cnt, q0, wl)
+        work["index_flops"] += index_flops(q0, n, wl, S)
+        if n <= 32:
+            work["attn_bytes"] += attn_bytes_decode(cnt, q0, wl)
+        work["launches"] += 1
+    return ms, work
+
+
+def cuda_arm(args, wl, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    p, model, q, out, sel, cnt = setup(wl, dev, seq=rank)
+    chunk = min(wl.chunk, wl.nq)
+    n_chunks = (wl.nq + chunk - 1) // chunk
+
+    def step():
+        if wl.nq <= 32:
+            model.forward(wl.q_start, q["q"], q["idx_q"], q["idx_w"], sel, cnt, out)
+        else:
+            model.prefill(q["q"], q["idx_q"], q["idx_w"], out, sel, cnt, q_pos0=wl.q_start)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ms_stage, work = stage_times(wl, p, model, q, dev)
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        step()
+    e1.record(st)
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    elapsed = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([elapsed], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed = float(t.item())
+        torch.distributed.barrier()
+    from sparse_long_context_sgqa_b200 import binding as Bd
+    Bd.sgqa_check()
+    ms_step = elapsed / args.steps
+    tokens_per_step = wl.nq * wl.num_seqs
+    value = tokens_per_step * world / (ms_step / 1e3)
+
+    # end to end from pinned host memory (prefill workloads)
+    e2e = None
+    if not args.no_e2e and rank == 0:
+        e2e = e2e_measure(wl, model, q, out, dev)
+
+    peaks = load_peaks()
+    per_launch_ms = {k: v / max(1, work["launches"]) for k, v in ms_stage.items()}
+    if wl.nq <= 32:
+        achieved = work["attn_bytes"] / work["launches"] / (per_launch_ms["attention"] / 1e3) / 1e9
+        roof = {"kernel": "sparse attention (decode gather)", "bound": "hbm", "achieved": achieved,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None}
+    else:
+        dom = "attention" if ms_stage["attention"] >= ms_stage["index"] else "index"
+        fl = work["attn_flops"] if dom == "attention" else work["index_flops"]
+        achieved = fl / work["launches"] / (per_launch_ms[dom] / 1e3) / 1e12
+        pk = peaks["bf16_tflops_sustained"]
+        roof = {"kernel": f"sparse {dom} stage", "bound": "tensor", "achieved": achieved, "peak": pk,
+                "unit": "TFLOP/s", "frac": achieved / pk, "traffic": None}
+    roof["peak_source"] = peaks["source"]
+
+    res = {
+        "metric": METRIC[wl.name][0], "value": value, "unit": METRIC[wl.name][1], "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "seq_len": wl.seq_len, "num_seqs": wl.num_seqs, "queries": wl.nq,
+                   "chunk": chunk, "groups": wl.groups, "heads": wl.n_heads, "head_dim": wl.head_dim,
+                   "idx_heads": wl.idx_heads, "block": wl.block, "topk": wl.topk,
+                   "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (no flush)"},
+        "stages_ms_per_step": ms_stage,
+        "stage_tflops": {"index": work["index_flops"] / (ms_stage["index"] / 1e3) / 1e12 if ms_stage["index"] else None,
+                         "attention": work["attn_flops"] / (ms_stage["attention"] / 1e3) / 1e12},
+        "roofline": roof,
+        "gpu_launches": args.steps * n_chunks * launches_per_call(wl),
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    return res
+
+
+def launches_per_call(wl):
+    # merge, widen, score, top-k, then plan + attention (prefill) or attention + combine (decode)
+    return 6
+
+
+def e2e_measure(wl, model, q, out, dev, steps=2):
+    host = {n: getattr(model, n).cpu().pin_memory() for n in ("kp", "c", "k", "v")}
+    for n in ("q", "idx_q", "idx_w"):
+        host[n] = q[n].cpu().pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    st = torch.cuda.current_stream()
+    if wl.nq <= 32:
+        return None
+    model.forward_host(host, out_host)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        h2d, d2h = model.forward_host(host, out_host)
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return {"value": wl.nq * wl.num_seqs / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle arm (reference / cpu_baseline)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(wl, budget_s: float = 20.0, max_rows: int = 64):
+    """Time the CPU oracle on a bounded sample of the workload's queries.
+
+    The per-sequence merge is timed in full; query rows (all groups each) are
+    drawn uniformly over the workload's query positions until the budget is
+    spent.  tokens/s = 1 / (merge_s / N + row_s / rows).
+    """
+    from oracle import sgqa_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([x.get("num_threads", 1) for x in threadpool_info()] + [1])
+    except Exception:
+        threads = os.cpu_count()
+    dev = "cpu"
+    L = wl.seq_len
+    cache = I.make_cache(wl, dev, seq=0)
+    kp, c = cache["kp"].double().numpy(), cache["c"].double().numpy()
+    K, V = cache["k"].float().numpy(), cache["v"].float().numpy()
+    t0 = time.perf_counter()
+    merged = O.merge_blocks(kp, c, wl.block)
+    keys = O.e4m3_decode(O.store_codes(merged))
+    merge_s = time.perf_counter() - t0
+    rng = np.random.default_rng(123)
+    rows = 0
+    row_s = 0.0
+    while rows < max_rows and row_s < budget_s:
+        t = int(rng.integers(wl.q_start, wl.q_start + wl.nq))
+        qs = I.make_queries(wl, dev, t, 1, seq=0)
+        args = {n: qs[n].double().numpy() for n in qs}
+        t1 = time.perf_counter()
+        O.forward_rows([(0, g) for g in range(wl.groups)], q=args["q"], k=K, v=V, idx_q=args["idx_q"],
+                       idx_w=args["idx_w"], keys=keys, block=wl.block, topk=wl.topk,
+                       heads_per_group=wl.heads_per_group, q_pos0=t)
+        row_s += time.perf_counter() - t1
+        rows += 1
+    per_token = merge_s / L + row_s / rows
+    value = 1.0 / per_token
+    return {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{rows} query positions x {wl.groups} groups uniform over the workload's queries "
+                      f"(oracle {row_s:.1f}s) + full merge of {L // wl.block} blocks ({merge_s:.1f}s); "
+                      f"tokens/s = 1/(merge_s/N + row_s/rows)"}
+
+
+def reference_arm(args, wl):
+    cb = oracle_sample(wl, budget_s=max(5.0, 15.0 / max(1, args.steps)))
+    ms = 1e3 / cb["value"]
+    return {"impl": "reference", "metric": METRIC[wl.name][0], "value": cb["value"], "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms * wl.nq,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": wl.name, "seq_len": wl.seq_len, "queries": wl.nq,
+                                            "block": wl.block, "topk": wl.topk},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="prefill128k", choices=sorted(METRIC))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    wl = I.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(reference_arm(args, wl)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    res = cuda_arm(args, wl, rank, world, local_rank)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = oracle_sample(wl)
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

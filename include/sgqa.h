@@ -1,0 +1,175 @@
+/*
+ * sgqa.h -- C ABI of the Sparse GQA global-attention hot path (sm_100a).
+ *
+ * The operation is the one described on the page "Step-5-Preview: Sparse
+ * Reads Are Not a Compressed KV Cache" (flozi.net): block-wise merging of
+ * proxy keys into a compressed search store, a per-KV-group weighted-ReLU
+ * indexer with causal top-k block selection, and exact softmax attention over
+ * the selected original K/V plus the query's current block.  Each entry point
+ * below cites the section of that page that defines it.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every tensor pointer is a DEVICE pointer owned by the caller.  The library
+ *   allocates no device memory: scratch space comes from a caller workspace
+ *   whose size sgqa_workspace_size() returns.  Tensors are C-contiguous in the
+ *   layouts stated below; "bf16" tensors hold IEEE bfloat16 bit patterns.
+ * - S = num_seqs independent sequences of equal length are processed per call.
+ *   Per-sequence cache tensors are strided by `cache_cap` tokens (the cache
+ *   capacity per sequence, >= cache_len).
+ * - G = num_kv_groups, Hg = heads_per_group (query heads per KV group),
+ *   D = head_dim, H = idx_heads (indexer heads per group), Di = idx_dim,
+ *   B = block_size, k = topk (historical blocks kept per query and group).
+ * - Query i of a call sits at absolute position t = q_pos0 + i (zero-based).
+ * - `stream` is a cudaStream_t (passed as void*).  Calls only enqueue work on
+ *   it and return; results are valid once the stream reaches that point.
+ * - Return value: SGQA_OK, or an error code with a message available from
+ *   sgqa_last_error() (thread-local).  Invalid arguments are rejected on the
+ *   host before anything is enqueued.  No C++ exception crosses the ABI.
+ * - Every wait inside the kernels is bounded in time.  A kernel that gives up
+ *   sets a device status word and returns; sgqa_check() reports it as
+ *   SGQA_ERR_TIMEOUT (or SGQA_ERR_DEVICE for a failed device-side check).
+ */
+#ifndef SGQA_H
+#define SGQA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SGQA_OK = 0,
+  SGQA_ERR_INVALID_ARGUMENT = 1, /* a pointer, size or layout the call cannot take */
+  SGQA_ERR_UNSUPPORTED = 2,      /* a valid shape this build has no kernel for   */
+  SGQA_ERR_WORKSPACE = 3,        /* workspace missing, misaligned or too small   */
+  SGQA_ERR_CUDA = 4,             /* a CUDA runtime/driver call or launch failed  */
+  SGQA_ERR_TIMEOUT = 5,          /* a kernel's bounded wait ran out              */
+  SGQA_ERR_DEVICE = 6            /* a kernel's own bounds check failed           */
+} sgqa_status;
+
+typedef struct {
+  int32_t num_kv_groups;    /* G: KV groups (4 for the global layer)                */
+  int32_t heads_per_group;  /* Hg: query heads sharing one KV group and selection  */
+  int32_t head_dim;         /* D: main Q/K/V head width (192)                       */
+  int32_t idx_heads;        /* H: indexer heads per group (4 or 8)                  */
+  int32_t idx_dim;          /* Di: proxy-key / indexer width (64)                   */
+  int32_t block_size;       /* B: tokens merged into one summary (8; 1, 2, 4 also)  */
+  int32_t topk;             /* k: historical blocks kept per (query, group)         */
+  int32_t merge_in_f32;     /* proxy keys / logits dtype: 0 = bf16, 1 = fp32        */
+  float scale;              /* softmax scale; <= 0 means 1/sqrt(D)                  */
+} sgqa_params;
+
+/* Supported by this build: Hg = 16, D = 192, Di = 64, H in {4, 8},
+ * B in {1, 2, 4, 8}, 1 <= k <= 2048, G >= 1.  Other values return
+ * SGQA_ERR_UNSUPPORTED. */
+
+/*
+ * Bytes of workspace a call with these sizes needs (for sgqa_index_topk,
+ * sgqa_sparse_attn and sgqa_forward alike).  nq = queries per sequence per
+ * call, max_ctx = the largest q_pos0 + nq the workspace will serve.  The
+ * workspace must be 256-byte aligned.  Pure host computation; no CUDA call.
+ */
+sgqa_status sgqa_workspace_size(const sgqa_params* p, int64_t num_seqs, int64_t nq,
+                                int64_t max_ctx, size_t* bytes);
+
+/*
+ * Block-wise token merging.  Page section "Eight tokens become one search
+ * key, coordinate by coordinate": for every completed block r in
+ * [blk_begin, blk_end) and every proxy coordinate d,
+ *     merged[r, d] = sum_j softmax_j(c[B r + j, d]) * kp[B r + j, d],
+ * the softmax taken over the block's B logits of that coordinate with their
+ * maximum subtracted, accumulated in FP32; the stored code is
+ *     store[r, d] = E4M3_satfinite(BF16_rne(merged[r, d]))  (OCP FP8 E4M3).
+ *
+ * proxy_k, comp_logits : [S, cache_cap, Di]   bf16 (or fp32 if merge_in_f32)
+ * merged_f32           : [S, cache_cap / B, Di] fp32, or NULL to skip
+ * store                : [S, cache_cap / B, Di] uint8 E4M3 codes
+ * Blocks must be complete: B * blk_end <= cache_cap.  Rows outside
+ * [blk_begin, blk_end) are not touched.
+ */
+sgqa_status sgqa_merge_blocks(const sgqa_params* p, int64_t num_seqs, int64_t cache_cap,
+                              const void* proxy_k, const void* comp_logits,
+                              int64_t blk_begin, int64_t blk_end,
+                              float* merged_f32, uint8_t* store, void* stream);
+
+/*
+ * Indexer score and causal top-k selection.  Page section "Selection is a
+ * weighted ReLU score, not attention softmax": for query t, group g and
+ * historical block r < floor(t / B),
+ *     I[t, g, r] = sum_i w[t, g, i] * max(0, q[t, g, i] . widen(store[r])),
+ * with no softmax; the k blocks with the largest I are kept, equal scores
+ * going to the smaller block id.  With fewer than k candidates all are kept.
+ *
+ * idx_q     : [S, nq, G, H, Di] bf16 indexer queries
+ * idx_w     : [S, nq, G, H]     fp32 signed head weights (prescale included)
+ * store     : [S, cache_cap / B, Di] uint8 E4M3 codes; blocks
+ *             [0, floor((q_pos0 + nq - 1) / B)) must be merged already
+ * sel       : [S, nq, G, k] int32 out: selected block ids in ascending order,
+ *             padded with -1
+ * sel_count : [S, nq, G]    int32 out: min(k, floor(t / B))
+ */
+sgqa_status sgqa_index_topk(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                            const void* idx_q, const float* idx_w,
+                            int64_t cache_cap, const uint8_t* store,
+                            int32_t* sel, int32_t* sel_count,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Sparse attention over the selected original K/V.  Page sections "Main
+ * attention still reads original K/V" and "Selection is a weighted ReLU
+ * score ...": query head h uses group g = floor(h / Hg); it attends, with
+ * ordinary scaled dot products and an exact softmax, to every token of the
+ * blocks in sel[t, g] plus the positions B*floor(t/B) .. t of its current
+ * block.  The Hg heads of a group share the selection.  The output is the
+ * pre-gate head vector.
+ *
+ * q        : [S, nq, G*Hg, D] bf16
+ * k_cache, v_cache : [S, cache_cap, G, D] bf16; tokens < cache_len are valid and
+ *            cache_len >= q_pos0 + nq (the call's own K/V are already written)
+ * sel, sel_count   : as produced by sgqa_index_topk (ids ascending, < floor(t/B))
+ * out      : [S, nq, G*Hg, D] bf16
+ */
+sgqa_status sgqa_sparse_attn(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                             const void* q, int64_t cache_cap, int64_t cache_len,
+                             const void* k_cache, const void* v_cache,
+                             const int32_t* sel, const int32_t* sel_count, void* out,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The whole hot path for one call: merge the blocks that this call's tokens
+ * complete (blocks [floor(q_pos0/B), floor((q_pos0+nq)/B))), then
+ * sgqa_index_topk, then sgqa_sparse_attn.  Arguments as above; the proxy keys,
+ * logits and K/V of positions [q_pos0, q_pos0 + nq) must already be in the
+ * caches, and blocks below floor(q_pos0/B) merged by earlier calls.  sel and
+ * sel_count are outputs too.  merged_f32 may be NULL.
+ */
+sgqa_status sgqa_forward(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                         const void* q, const void* idx_q, const float* idx_w,
+                         int64_t cache_cap, int64_t cache_len,
+                         const void* proxy_k, const void* comp_logits,
+                         const void* k_cache, const void* v_cache,
+                         float* merged_f32, uint8_t* store,
+                         int32_t* sel, int32_t* sel_count, void* out,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronise `stream` and report the device status word that bounded waits
+ * and device-side checks write (then clear it).  Returns SGQA_OK,
+ * SGQA_ERR_TIMEOUT, SGQA_ERR_DEVICE or SGQA_ERR_CUDA.
+ */
+sgqa_status sgqa_check(void* stream);
+
+/* Message of the last failed call on this thread ("" if none).  The pointer
+ * stays valid until the next call on this thread. */
+const char* sgqa_last_error(void);
+
+/* Library version string. */
+const char* sgqa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SGQA_H */

@@ -1,0 +1,78 @@
+"""User-facing API: one object that owns the caches and workspace of a batch of
+sequences and runs the hot path chunk by chunk through the C ABI.
+
+``SparseGQA.prefill`` / ``decode`` take device tensors; ``forward_host`` takes
+pinned host tensors and copies them in and the result out (the end-to-end
+path).  All arithmetic runs in ``libsgqa.so``.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as Bd
+
+
+class SparseGQA:
+    def __init__(self, params: Bd.Params, num_seqs: int, capacity: int, chunk: int, device,
+                 keep_merged_f32: bool = False):
+        self.p = params
+        self.S = num_seqs
+        self.cap = capacity
+        self.chunk = chunk
+        self.device = torch.device(device)
+        G, D, Di, B = params.num_kv_groups, params.head_dim, params.idx_dim, params.block_size
+        in_dt = torch.float32 if params.merge_in_f32 else torch.bfloat16
+        self.kp = torch.empty((num_seqs, capacity, Di), dtype=in_dt, device=device)
+        self.c = torch.empty((num_seqs, capacity, Di), dtype=in_dt, device=device)
+        self.k = torch.empty((num_seqs, capacity, G, D), dtype=torch.bfloat16, device=device)
+        self.v = torch.empty((num_seqs, capacity, G, D), dtype=torch.bfloat16, device=device)
+        self.store = torch.zeros((num_seqs, capacity // B, Di), dtype=torch.uint8, device=device)
+        self.merged = (torch.zeros((num_seqs, capacity // B, Di), dtype=torch.float32, device=device)
+                       if keep_merged_f32 else None)
+        self.ws = Bd.alloc_workspace(params, num_seqs, chunk, capacity, device)
+
+    def forward(self, q_pos0, q, idx_q, idx_w, sel, sel_count, out, cache_len=None, stream=None):
+        """One call of the hot path for queries [q_pos0, q_pos0 + nq) (nq <= chunk)."""
+        nq = q.shape[1]
+        Bd.sgqa_forward(self.p, self.S, q_pos0, nq, q, idx_q, idx_w, self.cap,
+                        self.cap if cache_len is None else cache_len, self.kp, self.c, self.k, self.v,
+                        self.merged, self.store, sel, sel_count, out, self.ws, stream)
+
+    def prefill(self, q, idx_q, idx_w, out, sel=None, sel_count=None, q_pos0=0, stream=None):
+        """Chunked prefill of all queries in q ([S, N, G*Hg, D]); caches already hold their K/V."""
+        S, N = q.shape[0], q.shape[1]
+        G, k = self.p.num_kv_groups, self.p.topk
+        for c0 in range(0, N, self.chunk):
+            n = min(self.chunk, N - c0)
+            s_sel = sel[:, c0:c0 + n] if sel is not None and S == 1 else torch.empty(
+                (S, n, G, k), dtype=torch.int32, device=self.device)
+            s_cnt = sel_count[:, c0:c0 + n] if sel_count is not None and S == 1 else torch.empty(
+                (S, n, G), dtype=torch.int32, device=self.device)
+            o = out[:, c0:c0 + n] if S == 1 else torch.empty((S, n) + tuple(out.shape[2:]),
+                                                             dtype=out.dtype, device=self.device)
+            self.forward(q_pos0 + c0, q[:, c0:c0 + n], idx_q[:, c0:c0 + n], idx_w[:, c0:c0 + n],
+                         s_sel, s_cnt, o, stream=stream)
+            if S != 1:
+                out[:, c0:c0 + n] = o
+                if sel is not None:
+                    sel[:, c0:c0 + n] = s_sel
+                if sel_count is not None:
+                    sel_count[:, c0:c0 + n] = s_cnt
+
+    def forward_host(self, host: dict, out_host: torch.Tensor, stream=None):
+        """End to end from pinned host memory: copy the inputs in, run, copy the output out.
+
+        host holds pinned tensors with the cache layouts (kp, c, k, v) and the query
+        layouts (q, idx_q, idx_w) of a full prefill; out_host receives [S, N, G*Hg, D].
+        Returns (bytes copied host->device, bytes copied device->host).
+        """
+        h2d = 0
+        for name in ("kp", "c", "k", "v"):
+            getattr(self, name).copy_(host[name], non_blocking=True)
+            h2d += host[name].numel() * host[name].element_size()
+        dq = {n: host[n].to(self.device, non_blocking=True) for n in ("q", "idx_q", "idx_w")}
+        h2d += sum(host[n].numel() * host[n].element_size() for n in ("q", "idx_q", "idx_w"))
+        out = torch.empty(out_host.shape, dtype=out_host.dtype, device=self.device)
+        self.prefill(dq["q"], dq["idx_q"], dq["idx_w"], out, stream=stream)
+        out_host.copy_(out, non_blocking=True)
+        return h2d, out_host.numel() * out_host.element_size()

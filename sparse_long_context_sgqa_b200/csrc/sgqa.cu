@@ -1,0 +1,407 @@
+// C ABI of the Sparse GQA hot path: argument validation, workspace carve-up
+// and kernel launches.  All kernels live in the headers included below; this
+// is the library's single translation unit (so the device status word is one
+// symbol per device).
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <string>
+
+#include "../../include/sgqa.h"
+#include "attn_mma.cuh"
+#include "common.cuh"
+#include "index_rows.cuh"
+#include "merge.cuh"
+
+namespace {
+
+thread_local std::string g_err;
+
+sgqa_status fail(sgqa_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+sgqa_status fail(sgqa_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
+sgqa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SGQA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define SGQA_LAUNCH_CHECK(what)                           \
+  do {                                                    \
+    cudaError_t e_ = cudaGetLastError();                  \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what);    \
+  } while (0)
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+sgqa_status check_params(const sgqa_params* p) {
+  if (p == nullptr) return fail(SGQA_ERR_INVALID_ARGUMENT, "params is NULL");
+  if (p->num_kv_groups < 1 || p->heads_per_group < 1 || p->head_dim < 1 || p->idx_heads < 1 ||
+      p->idx_dim < 1 || p->block_size < 1 || p->topk < 1)
+    return fail(SGQA_ERR_INVALID_ARGUMENT, "all sizes in sgqa_params must be >= 1");
+  if (p->heads_per_group != 16 || p->head_dim != 192 || p->idx_dim != 64)
+    return fail(SGQA_ERR_UNSUPPORTED, "this build supports heads_per_group=16, head_dim=192, idx_dim=64");
+  if (p->idx_heads != 4 && p->idx_heads != 8)
+    return fail(SGQA_ERR_UNSUPPORTED, "idx_heads must be 4 or 8");
+  const int B = p->block_size;
+  if (B != 1 && B != 2 && B != 4 && B != 8) return fail(SGQA_ERR_UNSUPPORTED, "block_size must be 1, 2, 4 or 8");
+  if (p->topk > 2048) return fail(SGQA_ERR_UNSUPPORTED, "topk must be <= 2048");
+  if (p->merge_in_f32 != 0 && p->merge_in_f32 != 1)
+    return fail(SGQA_ERR_INVALID_ARGUMENT, "merge_in_f32 must be 0 or 1");
+  return SGQA_OK;
+}
+
+float softmax_scale(const sgqa_params* p) {
+  return p->scale > 0.f ? p->scale : 1.0f / sqrtf(static_cast<float>(p->head_dim));
+}
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Queries per sequence below which attention runs split-K per query.
+constexpr int64_t kDecodeMaxNq = 32;
+
+int decode_splits(int64_t rows) {
+  int64_t s = (4 * 148 + rows - 1) / std::max<int64_t>(rows, 1);
+  return static_cast<int>(std::min<int64_t>(std::max<int64_t>(s, 1), 32));
+}
+
+int plan_pow2(int k) {
+  int p = 1;
+  while (p < 8 * k) p <<= 1;
+  return std::max(p, 2);
+}
+
+struct IndexWs {
+  int64_t rpad;
+  size_t keys_off, scores_off, bytes;
+};
+IndexWs index_ws(const sgqa_params* p, int64_t S, int64_t nq, int64_t max_ctx) {
+  IndexWs w;
+  const int64_t rneed = std::max<int64_t>((max_ctx - 1) / p->block_size, 1);
+  w.rpad = round_up(rneed, 64);
+  w.keys_off = 0;
+  size_t keys = align256(static_cast<size_t>(S * w.rpad * 64) * 2);
+  w.scores_off = keys;
+  size_t scores = align256(static_cast<size_t>(S * nq * p->num_kv_groups * w.rpad) * 4);
+  w.bytes = keys + scores;
+  return w;
+}
+
+struct AttnWs {
+  int nsplit;
+  size_t ids_off, mask_off, cnt_off, po_off, pml_off, bytes;
+};
+AttnWs attn_ws(const sgqa_params* p, int64_t S, int64_t nq) {
+  AttnWs w{};
+  const int64_t G = p->num_kv_groups;
+  if (nq <= kDecodeMaxNq) {
+    const int64_t rows = S * nq * G;
+    w.nsplit = decode_splits(rows);
+    w.po_off = 0;
+    size_t po = align256(static_cast<size_t>(rows * w.nsplit) * 16 * 192 * 4);
+    w.pml_off = po;
+    size_t pml = align256(static_cast<size_t>(rows * w.nsplit) * 16 * 2 * 4);
+    w.bytes = po + pml;
+  } else {
+    const int64_t units = S * ((nq + 7) / 8) * G;
+    const int64_t cap = 8 * static_cast<int64_t>(p->topk);
+    w.ids_off = 0;
+    size_t ids = align256(static_cast<size_t>(units * cap) * 4);
+    w.mask_off = ids;
+    size_t mask = align256(static_cast<size_t>(units * cap));
+    w.cnt_off = ids + mask;
+    size_t cnt = align256(static_cast<size_t>(units) * 4);
+    w.bytes = ids + mask + cnt;
+  }
+  return w;
+}
+
+template <typename T>
+T* ws_at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+sgqa_status check_ws(void* ws, size_t have, size_t need) {
+  if (need == 0) return SGQA_OK;
+  if (ws == nullptr) return fail(SGQA_ERR_WORKSPACE, "workspace is NULL (need %zu bytes)", need);
+  if (!aligned(ws, 256)) return fail(SGQA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (have < need) return fail(SGQA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", have, need);
+  return SGQA_OK;
+}
+
+template <int B>
+void launch_merge(bool f32, const void* kp, const void* c, int64_t cap, int64_t b0, int64_t nblk,
+                  int64_t S, float* merged, uint8_t* store, cudaStream_t st) {
+  const int64_t threads = S * nblk * 8;
+  const unsigned grid = static_cast<unsigned>((threads + sgqa::kMergeThreads - 1) / sgqa::kMergeThreads);
+  if (f32)
+    sgqa::merge_blocks_kernel<B, true><<<grid, sgqa::kMergeThreads, 0, st>>>(kp, c, cap, b0, nblk, S, merged, store);
+  else
+    sgqa::merge_blocks_kernel<B, false><<<grid, sgqa::kMergeThreads, 0, st>>>(kp, c, cap, b0, nblk, S, merged, store);
+}
+
+sgqa_status do_merge(const sgqa_params* p, int64_t S, int64_t cap, const void* kp, const void* c,
+                     int64_t b0, int64_t b1, float* merged, uint8_t* store, cudaStream_t st) {
+  const int64_t nblk = b1 - b0;
+  if (nblk <= 0) return SGQA_OK;
+  const bool f32 = p->merge_in_f32 != 0;
+  switch (p->block_size) {
+    case 1: launch_merge<1>(f32, kp, c, cap, b0, nblk, S, merged, store, st); break;
+    case 2: launch_merge<2>(f32, kp, c, cap, b0, nblk, S, merged, store, st); break;
+    case 4: launch_merge<4>(f32, kp, c, cap, b0, nblk, S, merged, store, st); break;
+    default: launch_merge<8>(f32, kp, c, cap, b0, nblk, S, merged, store, st); break;
+  }
+  SGQA_LAUNCH_CHECK("merge_blocks_kernel");
+  return SGQA_OK;
+}
+
+sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* idx_q,
+                     const float* idx_w, int64_t cap, const uint8_t* store, int32_t* sel,
+                     int32_t* sel_count, void* ws, cudaStream_t st) {
+  const int B = p->block_size, G = p->num_kv_groups, H = p->idx_heads;
+  const IndexWs w = index_ws(p, S, nq, q0 + nq);
+  const int64_t rneed = (q0 + nq - 1) / B;
+  __nv_bfloat16* keys = ws_at<__nv_bfloat16>(ws, w.keys_off);
+  float* scores = ws_at<float>(ws, w.scores_off);
+  if (rneed > 0) {
+    const int64_t threads = S * rneed * 8;
+    sgqa::widen_store_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(
+        store, cap / B, rneed, w.rpad, S, keys);
+    SGQA_LAUNCH_CHECK("widen_store_kernel");
+    const int qpc = 64 / H;
+    dim3 grid(static_cast<unsigned>((nq + qpc - 1) / qpc),
+              static_cast<unsigned>((rneed + sgqa::kScoreCandPerCta - 1) / sgqa::kScoreCandPerCta),
+              static_cast<unsigned>(S * G));
+    if (grid.y > 65535 || grid.z > 65535) return fail(SGQA_ERR_UNSUPPORTED, "index grid too large");
+    const __nv_bfloat16* iq = static_cast<const __nv_bfloat16*>(idx_q);
+    if (H == 8)
+      sgqa::index_score_kernel<8><<<grid, sgqa::kScoreWarps * 32, 0, st>>>(iq, idx_w, keys, scores, nq, G, q0, B, w.rpad);
+    else
+      sgqa::index_score_kernel<4><<<grid, sgqa::kScoreWarps * 32, 0, st>>>(iq, idx_w, keys, scores, nq, G, q0, B, w.rpad);
+    SGQA_LAUNCH_CHECK("index_score_kernel");
+  }
+  const int64_t rows = S * nq * G;
+  sgqa::topk_rows_kernel<<<static_cast<unsigned>(rows), sgqa::kSelThreads, 0, st>>>(
+      scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count);
+  SGQA_LAUNCH_CHECK("topk_rows_kernel");
+  return SGQA_OK;
+}
+
+template <int B>
+sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q,
+                        int64_t cap, int64_t clen, const void* kc, const void* vc, const int32_t* sel,
+                        const int32_t* sel_count, void* out, void* ws, cudaStream_t st) {
+  const int G = p->num_kv_groups, k = p->topk;
+  const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
+  const AttnWs w = attn_ws(p, S, nq);
+  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(kc);
+  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(vc);
+  __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(out);
+  if (nq <= kDecodeMaxNq) {
+    const int64_t rows = S * nq * G;
+    const size_t smem = sgqa::kDecWarps * sgqa::kDecStages * 2 * sgqa::kStageElems * 2;
+    cudaFuncSetAttribute(sgqa::attn_decode_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    float* po = ws_at<float>(ws, w.po_off);
+    float* pml = ws_at<float>(ws, w.pml_off);
+    sgqa::attn_decode_kernel<B><<<static_cast<unsigned>(rows * w.nsplit), sgqa::kDecWarps * 32, smem, st>>>(
+        qb, kb, vb, sel, sel_count, po, pml, nq, G, k, q0, cap, w.nsplit, scale_log2);
+    SGQA_LAUNCH_CHECK("attn_decode_kernel");
+    sgqa::attn_combine_kernel<<<static_cast<unsigned>(rows * 16), 64, 0, st>>>(po, pml, ob, rows, w.nsplit);
+    SGQA_LAUNCH_CHECK("attn_combine_kernel");
+    return SGQA_OK;
+  }
+  const int64_t units = S * ((nq + 7) / 8) * G;
+  const int pow2 = plan_pow2(k);
+  int32_t* ids = ws_at<int32_t>(ws, w.ids_off);
+  uint8_t* msk = ws_at<uint8_t>(ws, w.mask_off);
+  int32_t* cnt = ws_at<int32_t>(ws, w.cnt_off);
+  const size_t psmem = static_cast<size_t>(pow2) * 4;
+  cudaFuncSetAttribute(sgqa::attn_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
+  sgqa::attn_plan_kernel<<<static_cast<unsigned>(units), sgqa::kPlanThreads, psmem, st>>>(
+      sel, sel_count, nq, G, k, pow2, ids, msk, cnt);
+  SGQA_LAUNCH_CHECK("attn_plan_kernel");
+  const size_t smem = sgqa::kGroupedStages * 2 * sgqa::kStageElems * 2;
+  cudaFuncSetAttribute(sgqa::attn_grouped_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  sgqa::attn_grouped_kernel<B><<<static_cast<unsigned>(units), sgqa::kGroupedThreads, smem, st>>>(
+      qb, kb, vb, ids, msk, cnt, ob, nq, G, k, q0, cap, clen, scale_log2);
+  SGQA_LAUNCH_CHECK("attn_grouped_kernel");
+  return SGQA_OK;
+}
+
+sgqa_status do_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q,
+                    int64_t cap, int64_t clen, const void* kc, const void* vc, const int32_t* sel,
+                    const int32_t* sel_count, void* out, void* ws, cudaStream_t st) {
+  switch (p->block_size) {
+    case 1: return launch_attn<1>(p, S, q0, nq, q, cap, clen, kc, vc, sel, sel_count, out, ws, st);
+    case 2: return launch_attn<2>(p, S, q0, nq, q, cap, clen, kc, vc, sel, sel_count, out, ws, st);
+    case 4: return launch_attn<4>(p, S, q0, nq, q, cap, clen, kc, vc, sel, sel_count, out, ws, st);
+    default: return launch_attn<8>(p, S, q0, nq, q, cap, clen, kc, vc, sel, sel_count, out, ws, st);
+  }
+}
+
+sgqa_status check_common(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, int64_t cap) {
+  sgqa_status s = check_params(p);
+  if (s != SGQA_OK) return s;
+  if (S < 1) return fail(SGQA_ERR_INVALID_ARGUMENT, "num_seqs must be >= 1");
+  if (q0 < 0) return fail(SGQA_ERR_INVALID_ARGUMENT, "q_pos0 must be >= 0");
+  if (nq < 0) return fail(SGQA_ERR_INVALID_ARGUMENT, "nq must be >= 0");
+  if (cap < q0 + nq) return fail(SGQA_ERR_INVALID_ARGUMENT, "cache_cap (%lld) < q_pos0 + nq (%lld)",
+                                 (long long)cap, (long long)(q0 + nq));
+  if (cap > (int64_t(1) << 31) - 1) return fail(SGQA_ERR_UNSUPPORTED, "cache_cap must be < 2^31");
+  return SGQA_OK;
+}
+
+#define REQUIRE_PTR(ptr, align)                                                                 \
+  do {                                                                                          \
+    if ((ptr) == nullptr) return fail(SGQA_ERR_INVALID_ARGUMENT, #ptr " is NULL");             \
+    if (!aligned((ptr), (align))) return fail(SGQA_ERR_INVALID_ARGUMENT, #ptr " must be %d-byte aligned", (int)(align)); \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* sgqa_version(void) { return "sgqa-b200 0.1 (sm_100a)"; }
+
+const char* sgqa_last_error(void) { return g_err.c_str(); }
+
+sgqa_status sgqa_workspace_size(const sgqa_params* p, int64_t num_seqs, int64_t nq, int64_t max_ctx,
+                                size_t* bytes) {
+  g_err.clear();
+  sgqa_status s = check_params(p);
+  if (s != SGQA_OK) return s;
+  if (bytes == nullptr) return fail(SGQA_ERR_INVALID_ARGUMENT, "bytes is NULL");
+  if (num_seqs < 1 || nq < 0 || max_ctx < nq) return fail(SGQA_ERR_INVALID_ARGUMENT, "bad sizes");
+  const IndexWs iw = index_ws(p, num_seqs, nq, std::max<int64_t>(max_ctx, 1));
+  const AttnWs aw = attn_ws(p, num_seqs, nq);
+  *bytes = std::max(iw.bytes, aw.bytes);
+  return SGQA_OK;
+}
+
+sgqa_status sgqa_merge_blocks(const sgqa_params* p, int64_t num_seqs, int64_t cache_cap,
+                              const void* proxy_k, const void* comp_logits, int64_t blk_begin,
+                              int64_t blk_end, float* merged_f32, uint8_t* store, void* stream) {
+  g_err.clear();
+  sgqa_status s = check_params(p);
+  if (s != SGQA_OK) return s;
+  if (num_seqs < 1 || cache_cap < 0) return fail(SGQA_ERR_INVALID_ARGUMENT, "bad num_seqs/cache_cap");
+  if (blk_begin < 0 || blk_end < blk_begin || blk_end * p->block_size > cache_cap)
+    return fail(SGQA_ERR_INVALID_ARGUMENT, "block range [%lld, %lld) not complete within cache_cap %lld",
+                (long long)blk_begin, (long long)blk_end, (long long)cache_cap);
+  if (blk_end == blk_begin) return SGQA_OK;
+  REQUIRE_PTR(proxy_k, 16);
+  REQUIRE_PTR(comp_logits, 16);
+  REQUIRE_PTR(store, 8);
+  if (merged_f32 != nullptr && !aligned(merged_f32, 16))
+    return fail(SGQA_ERR_INVALID_ARGUMENT, "merged_f32 must be 16-byte aligned");
+  return do_merge(p, num_seqs, cache_cap, proxy_k, comp_logits, blk_begin, blk_end, merged_f32, store,
+                  static_cast<cudaStream_t>(stream));
+}
+
+sgqa_status sgqa_index_topk(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                            const void* idx_q, const float* idx_w, int64_t cache_cap,
+                            const uint8_t* store, int32_t* sel, int32_t* sel_count, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  g_err.clear();
+  sgqa_status s = check_common(p, num_seqs, q_pos0, nq, cache_cap);
+  if (s != SGQA_OK) return s;
+  if (nq == 0) return SGQA_OK;
+  REQUIRE_PTR(idx_q, 16);
+  REQUIRE_PTR(idx_w, 8);
+  REQUIRE_PTR(store, 16);
+  REQUIRE_PTR(sel, 4);
+  REQUIRE_PTR(sel_count, 4);
+  const IndexWs w = index_ws(p, num_seqs, nq, q_pos0 + nq);
+  if ((s = check_ws(workspace, workspace_bytes, w.bytes)) != SGQA_OK) return s;
+  return do_index(p, num_seqs, q_pos0, nq, idx_q, idx_w, cache_cap, store, sel, sel_count, workspace,
+                  static_cast<cudaStream_t>(stream));
+}
+
+sgqa_status sgqa_sparse_attn(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                             const void* q, int64_t cache_cap, int64_t cache_len, const void* k_cache,
+                             const void* v_cache, const int32_t* sel, const int32_t* sel_count,
+                             void* out, void* workspace, size_t workspace_bytes, void* stream) {
+  g_err.clear();
+  sgqa_status s = check_common(p, num_seqs, q_pos0, nq, cache_cap);
+  if (s != SGQA_OK) return s;
+  if (cache_len < q_pos0 + nq || cache_len > cache_cap)
+    return fail(SGQA_ERR_INVALID_ARGUMENT, "need q_pos0 + nq <= cache_len <= cache_cap");
+  if (nq == 0) return SGQA_OK;
+  REQUIRE_PTR(q, 16);
+  REQUIRE_PTR(k_cache, 16);
+  REQUIRE_PTR(v_cache, 16);
+  REQUIRE_PTR(sel, 4);
+  REQUIRE_PTR(sel_count, 4);
+  REQUIRE_PTR(out, 16);
+  const AttnWs w = attn_ws(p, num_seqs, nq);
+  if ((s = check_ws(workspace, workspace_bytes, w.bytes)) != SGQA_OK) return s;
+  return do_attn(p, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k_cache, v_cache, sel, sel_count, out,
+                 workspace, static_cast<cudaStream_t>(stream));
+}
+
+sgqa_status sgqa_forward(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                         const void* q, const void* idx_q, const float* idx_w, int64_t cache_cap,
+                         int64_t cache_len, const void* proxy_k, const void* comp_logits,
+                         const void* k_cache, const void* v_cache, float* merged_f32, uint8_t* store,
+                         int32_t* sel, int32_t* sel_count, void* out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  g_err.clear();
+  sgqa_status s = check_common(p, num_seqs, q_pos0, nq, cache_cap);
+  if (s != SGQA_OK) return s;
+  if (cache_len < q_pos0 + nq || cache_len > cache_cap)
+    return fail(SGQA_ERR_INVALID_ARGUMENT, "need q_pos0 + nq <= cache_len <= cache_cap");
+  if (nq == 0) return SGQA_OK;
+  REQUIRE_PTR(q, 16);
+  REQUIRE_PTR(idx_q, 16);
+  REQUIRE_PTR(idx_w, 8);
+  REQUIRE_PTR(proxy_k, 16);
+  REQUIRE_PTR(comp_logits, 16);
+  REQUIRE_PTR(k_cache, 16);
+  REQUIRE_PTR(v_cache, 16);
+  REQUIRE_PTR(store, 16);
+  REQUIRE_PTR(sel, 4);
+  REQUIRE_PTR(sel_count, 4);
+  REQUIRE_PTR(out, 16);
+  if (merged_f32 != nullptr && !aligned(merged_f32, 16))
+    return fail(SGQA_ERR_INVALID_ARGUMENT, "merged_f32 must be 16-byte aligned");
+  size_t need = 0;
+  if ((s = sgqa_workspace_size(p, num_seqs, nq, q_pos0 + nq, &need)) != SGQA_OK) return s;
+  if ((s = check_ws(workspace, workspace_bytes, need)) != SGQA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int B = p->block_size;
+  if ((s = do_merge(p, num_seqs, cache_cap, proxy_k, comp_logits, q_pos0 / B, (q_pos0 + nq) / B,
+                    merged_f32, store, st)) != SGQA_OK)
+    return s;
+  if ((s = do_index(p, num_seqs, q_pos0, nq, idx_q, idx_w, cache_cap, store, sel, sel_count, workspace,
+                    st)) != SGQA_OK)
+    return s;
+  return do_attn(p, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k_cache, v_cache, sel, sel_count, out,
+                 workspace, st);
+}
+
+sgqa_status sgqa_check(void* stream) {
+  g_err.clear();
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int code = 0;
+  e = cudaMemcpyFromSymbol(&code, sgqa::g_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read device status");
+  if (code == 0) return SGQA_OK;
+  const int zero = 0;
+  cudaMemcpyToSymbol(sgqa::g_status, &zero, sizeof(int));
+  if (code == sgqa::kDevTimeout) return fail(SGQA_ERR_TIMEOUT, "a kernel's bounded wait ran out");
+  return fail(SGQA_ERR_DEVICE, "a kernel's device-side check failed (code %d)", code);
+}
+
+}  // extern "C"

@@ -201,3 +201,38 @@ def make_queries(wl: Workload, device, pos0: int, n: int, seq: int = 0):
         iq[a - pos0:b - pos0] = iq_[lo:hi].to(dt)
         iw[a - pos0:b - pos0] = iw_[lo:hi]
     return {"q": q, "idx_q": iq, "idx_w": iw}
+
+
+def make_selection(wl: Workload, device, pos0: int, n: int, num_seqs: int = 1, seed: int = 0):
+    """A random valid selection input (for exercising attention on its own).
+
+    For query t and group g: min(k, floor(t/B)) distinct block ids < floor(t/B),
+    ascending, padded with -1; counts [S, n, G].  Queries of one 64-token
+    segment rank blocks by a shared random preference plus their own noise,
+    so adjacent queries overlap as real selections do.
+    """
+    G, k, B = wl.groups, wl.topk, wl.block
+    sel = torch.full((num_seqs, n, G, k), -1, dtype=torch.int32, device=device)
+    cnt = torch.empty((num_seqs, n, G), dtype=torch.int32, device=device)
+    tmax = pos0 + n - 1
+    rmax = max(tmax // B, 1)
+    for s in range(num_seqs):
+        for r0 in range(0, n, 256):
+            r1 = min(n, r0 + 256)
+            t = torch.arange(pos0 + r0, pos0 + r1, device=device)
+            ncand = t // B
+            seg = t // QUERY_SEGMENT
+            pref = _randn((int(seg.max() - seg.min()) + 1, G, rmax), device, wl.seed, seed, s, "selpref", r0)
+            noise = _randn((r1 - r0, G, rmax), device, wl.seed, seed, s, "selnoise", r0)
+            sc = pref[seg - seg.min()] + 0.5 * noise
+            valid = torch.arange(rmax, device=device)[None, None, :] < ncand[:, None, None]
+            sc = torch.where(valid, sc, torch.full_like(sc, -float("inf")))
+            kk = min(k, rmax)
+            top = torch.topk(sc, kk, dim=-1).indices
+            take = torch.arange(kk, device=device)[None, None, :] < torch.clamp(ncand, max=k)[:, None, None]
+            ids = torch.where(take, top, torch.full_like(top, 1 << 30))
+            ids = torch.sort(ids, dim=-1).values
+            ids = torch.where(ids == (1 << 30), torch.full_like(ids, -1), ids)
+            sel[s, r0:r1, :, :kk] = ids.to(torch.int32)
+            cnt[s, r0:r1] = torch.clamp(ncand, max=k).to(torch.int32)[:, None]
+    return sel, cnt

@@ -1,0 +1,246 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Tolerances: merged keys 1e-3 relative (1e-6 absolute floor) in FP32; store
+codes bit-exact except where FP32 rounding of the exact merged value decides a
+boundary; selections bit-exact except swaps between scores within 1e-5
+relative of the k-th score; attention outputs 2e-2 max-abs on bf16 outputs.
+"""
+import dataclasses
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import sgqa_oracle as O
+from sparse_long_context_sgqa_b200 import inputs as I
+from tests import _harness as Hn
+
+pytestmark = pytest.mark.gpu
+
+WL = I.WORKLOADS
+SMALL8 = dataclasses.replace(WL["prefill8k"], name="prefill2k", seq_len=2048)
+
+
+def _bd():
+    from sparse_long_context_sgqa_b200 import binding
+    return binding
+
+
+def test_library_loads(cuda_device):
+    assert "sm_100a" in _bd().version()
+
+
+def test_e4m3_store_exhaustive_over_bf16(cuda_device):
+    """B=1 merge is the identity, so the store path sees every BF16 value."""
+    bits = (np.arange(2 ** 16, dtype=np.uint32) << np.uint32(16)).view(np.float32)
+    vals = bits[np.isfinite(bits)]
+    n = (len(vals) + 63) // 64 * 64
+    x = np.zeros(n, dtype=np.float32)
+    x[:len(vals)] = vals
+    kp = torch.from_numpy(x.reshape(-1, 64)).to(cuda_device)
+    c = torch.zeros_like(kp)
+    p = _bd().Params(num_kv_groups=1, idx_heads=4, block_size=1, topk=8, merge_in_f32=1)
+    L = kp.shape[0]
+    store = torch.zeros((L, 64), dtype=torch.uint8, device=cuda_device)
+    merged = torch.zeros((L, 64), dtype=torch.float32, device=cuda_device)
+    _bd().sgqa_merge_blocks(p, 1, L, kp, c, 0, L, merged, store)
+    torch.cuda.synchronize()
+    assert torch.equal(merged.cpu(), kp.cpu())
+    ref = O.e4m3_encode(O.round_e4m3(x.astype(np.float64)))
+    got = store.cpu().numpy().reshape(-1)
+    bad = np.nonzero(got != ref)[0]
+    detail = [(float(x[j]), int(got[j]), int(ref[j])) for j in bad[:12]]
+    assert len(bad) == 0, f"{len(bad)} codes differ (value, gpu, oracle): {detail}"
+
+
+
+@pytest.mark.parametrize("wl", [WL["tiny"], SMALL8,
+                                dataclasses.replace(SMALL8, block=4, name="b4"),
+                                dataclasses.replace(SMALL8, block=1, name="b1"),
+                                WL["prefill8k"]], ids=lambda w: w.name)
+def test_merge_parity(cuda_device, wl):
+    cache, _ = Hn.make_inputs(wl, cuda_device)
+    p = Hn.params_for(wl)
+    L, B = wl.seq_len, wl.block
+    store = torch.zeros((1, L // B, 64), dtype=torch.uint8, device=cuda_device)
+    merged = torch.zeros((1, L // B, 64), dtype=torch.float32, device=cuda_device)
+    # two calls: [0, a) then [a, L/B) -- ranges must not disturb other rows
+    a = (L // B) // 3
+    _bd().sgqa_merge_blocks(p, 1, L, cache["kp"], cache["c"], 0, a, merged, store)
+    _bd().sgqa_merge_blocks(p, 1, L, cache["kp"], cache["c"], a, L // B, merged, store)
+    torch.cuda.synchronize()
+    exact = O.merge_blocks(Hn.to_np(cache["kp"][0]), Hn.to_np(cache["c"][0]), B)
+    got = merged[0].cpu().double().numpy()
+    assert np.all(np.abs(got - exact) <= Hn.MERGE_RTOL * np.abs(exact) + Hn.MERGE_ATOL)
+    codes = store[0].cpu().numpy()
+    ok = Hn.store_mismatch_ok(codes, exact)
+    assert ok.all(), f"{(~ok).sum()} store codes differ beyond FP32 rounding"
+    flips = (codes != O.store_codes(exact)).sum()
+    assert flips <= max(2, 1e-4 * codes.size)
+
+
+def _index_isolated(wl, device, q_pos0, nq, rows):
+    cache, _ = Hn.make_inputs(wl, device)
+    qs = I.make_queries(wl, device, q_pos0, nq)
+    if wl.fp32_inputs:
+        qs["idx_q"] = qs["idx_q"].to(torch.bfloat16)
+    _, codes, keys = Hn.oracle_keys(Hn.to_np(cache["kp"][0]), Hn.to_np(cache["c"][0]), wl.block)
+    L = wl.seq_len
+    store = torch.from_numpy(codes).to(device)[None].contiguous()
+    p = Hn.params_for(wl)
+    sel = torch.full((1, nq, wl.groups, wl.topk), -7, dtype=torch.int32, device=device)
+    cnt = torch.full((1, nq, wl.groups), -7, dtype=torch.int32, device=device)
+    ws = _bd().alloc_workspace(p, 1, nq, q_pos0 + nq, device)
+    _bd().sgqa_index_topk(p, 1, q_pos0, nq, qs["idx_q"][None].contiguous(), qs["idx_w"][None].contiguous(),
+                          L, store, sel, cnt, ws)
+    _bd().sgqa_check()
+    sel, cnt = sel[0].cpu().numpy(), cnt[0].cpu().numpy()
+    t = q_pos0 + np.arange(nq)
+    assert np.array_equal(cnt, np.minimum(wl.topk, t // wl.block)[:, None].repeat(wl.groups, 1))
+    iq, iw = Hn.to_np(qs["idx_q"]), Hn.to_np(qs["idx_w"])
+    ties = 0
+    for i in rows:
+        for g in range(wl.groups):
+            tt = q_pos0 + i
+            sc = O.index_scores(iq[i, g], iw[i, g], keys[:tt // wl.block])
+            c = cnt[i, g]
+            assert np.all(sel[i, g, c:] == -1)
+            ties += Hn.check_selection(sel[i, g, :c], sc, wl.topk)
+    return ties
+
+
+@pytest.mark.parametrize("case", ["tiny", "prefill8k", "unaligned_chunk", "b1", "b4_k64"])
+def test_index_topk_parity(cuda_device, case):
+    if case == "tiny":
+        wl = WL["tiny"]; q0, nq = 0, 256; rows = range(256)
+    elif case == "prefill8k":
+        wl = WL["prefill8k"]; q0, nq = 0, 8192; rows = Hn.sample_rows(wl, 48)
+    elif case == "unaligned_chunk":
+        wl = SMALL8; q0, nq = 1029, 611; rows = list(range(0, nq, 13)) + [nq - 1]
+    elif case == "b1":
+        wl = dataclasses.replace(SMALL8, block=1, topk=256); q0, nq = 0, 2048; rows = list(range(0, 2048, 37)) + [2047]
+    else:
+        wl = dataclasses.replace(SMALL8, block=4, topk=64); q0, nq = 512, 1536; rows = list(range(0, nq, 29)) + [nq - 1]
+    ties = _index_isolated(wl, cuda_device, q0, nq, rows)
+    assert ties <= 2 * len(rows)
+
+
+def _attn_isolated(wl, device, q_pos0, nq, rows, num_seqs=1, groups=None):
+    cache, _ = Hn.make_inputs(wl, device, seqs=range(num_seqs))
+    qs = [I.make_queries(wl, device, q_pos0, nq, seq=s) for s in range(num_seqs)]
+    q = torch.stack([x["q"] for x in qs]).to(torch.bfloat16).contiguous()
+    sel, cnt = I.make_selection(wl, device, q_pos0, nq, num_seqs=num_seqs)
+    p = Hn.params_for(wl)
+    L = wl.seq_len
+    out = torch.zeros((num_seqs, nq, wl.n_heads, wl.head_dim), dtype=torch.bfloat16, device=device)
+    ws = _bd().alloc_workspace(p, num_seqs, nq, q_pos0 + nq, device)
+    _bd().sgqa_sparse_attn(p, num_seqs, q_pos0, nq, q, L, L, cache["k"], cache["v"], sel, cnt, out, ws)
+    _bd().sgqa_check()
+    worst = 0.0
+    for s in range(num_seqs):
+        K, V = Hn.to_np(cache["k"][s]), Hn.to_np(cache["v"][s])
+        qn = Hn.to_np(q[s])
+        seln, cntn = sel[s].cpu().numpy(), cnt[s].cpu().numpy()
+        on = out[s].float().cpu().numpy()
+        for i in rows:
+            for g in (range(wl.groups) if groups is None else groups):
+                t = q_pos0 + i
+                ids = seln[i, g, :cntn[i, g]]
+                pos = O.attended_positions(t, ids, wl.block)
+                hs = slice(g * 16, (g + 1) * 16)
+                ref = O.sparse_attention(qn[i, hs], K[pos, g], V[pos, g], Hn.scale_of(wl))
+                worst = max(worst, float(np.abs(on[i, hs] - ref).max()))
+    assert worst <= Hn.ATTN_ATOL, worst
+    return worst
+
+
+@pytest.mark.parametrize("case", ["tiny", "prefill8k", "unaligned_chunk", "decode_path", "b1", "b2"])
+def test_sparse_attn_parity(cuda_device, case):
+    if case == "tiny":
+        _attn_isolated(WL["tiny"], cuda_device, 0, 256, range(256))
+    elif case == "prefill8k":
+        _attn_isolated(WL["prefill8k"], cuda_device, 0, 8192, Hn.sample_rows(WL["prefill8k"], 40))
+    elif case == "unaligned_chunk":
+        _attn_isolated(SMALL8, cuda_device, 1029, 611, list(range(0, 611, 7)) + [610])
+    elif case == "decode_path":
+        wl = dataclasses.replace(SMALL8, seq_len=20000, name="dec")
+        _attn_isolated(wl, cuda_device, 19990, 10, range(10), num_seqs=3)
+    elif case == "b1":
+        wl = dataclasses.replace(SMALL8, block=1, topk=2048)
+        _attn_isolated(wl, cuda_device, 0, 2048, list(range(0, 2048, 41)) + [2047])
+    else:
+        wl = dataclasses.replace(SMALL8, block=2, topk=100)
+        _attn_isolated(wl, cuda_device, 0, 2048, list(range(0, 2048, 41)) + [2047])
+
+
+def _e2e(wl, device, rows, seqs=(0,)):
+    run = Hn.run_forward(wl, device)
+    B = wl.block
+    stats = {"rows": 0, "tie_rows": 0, "flip_rows": 0, "worst": 0.0}
+    for s in seqs:
+        exact = O.merge_blocks(Hn.to_np(run.cache["kp"][s]), Hn.to_np(run.cache["c"][s]), B)
+        codes = O.store_codes(exact)
+        gpu_codes = run.store[s].cpu().numpy()
+        assert Hn.store_mismatch_ok(gpu_codes, exact).all()
+        flipped = set(np.nonzero((gpu_codes != codes).any(axis=1))[0].tolist())
+        keys = O.e4m3_decode(codes)
+        K, V = Hn.to_np(run.cache["k"][s]), Hn.to_np(run.cache["v"][s])
+        q, iq, iw = (Hn.to_np(run.queries[x][s]) for x in ("q", "idx_q", "idx_w"))
+        sel, cnt = run.sel[s].cpu().numpy(), run.cnt[s].cpu().numpy()
+        out = run.out[s].float().cpu().numpy()
+        for i in rows:
+            t = wl.q_start + i
+            for g in range(wl.groups):
+                stats["rows"] += 1
+                sc = O.index_scores(iq[i, g], iw[i, g], keys[:t // B])
+                ref_sel = O.select_topk(sc, wl.topk)
+                gsel = sel[i, g, :cnt[i, g]]
+                assert cnt[i, g] == len(ref_sel)
+                if not np.array_equal(gsel, ref_sel):
+                    diff = set(np.setxor1d(gsel, ref_sel).tolist())
+                    if diff & flipped:
+                        stats["flip_rows"] += 1
+                        continue
+                    Hn.check_selection(gsel, sc, wl.topk)
+                    stats["tie_rows"] += 1
+                    continue
+                pos = O.attended_positions(t, ref_sel, B)
+                hs = slice(g * 16, (g + 1) * 16)
+                ref = O.sparse_attention(q[i, hs], K[pos, g], V[pos, g], Hn.scale_of(wl))
+                stats["worst"] = max(stats["worst"], float(np.abs(out[i, hs] - ref).max()))
+    assert stats["worst"] <= Hn.ATTN_ATOL, stats
+    assert stats["flip_rows"] + stats["tie_rows"] <= max(2, 0.05 * stats["rows"]), stats
+    return stats
+
+
+def test_forward_tiny_all_rows(cuda_device):
+    _e2e(WL["tiny"], cuda_device, range(256))
+
+
+def test_forward_prefill8k_sampled(cuda_device):
+    _e2e(WL["prefill8k"], cuda_device, Hn.sample_rows(WL["prefill8k"], 40))
+
+
+def test_full_topk_equals_dense_causal_attention(cuda_device):
+    """k >= number of blocks: the sparse path is textbook causal attention."""
+    wl = dataclasses.replace(WL["tiny"], topk=32, name="tiny_dense")
+    run = Hn.run_forward(wl, cuda_device)
+    q = Hn.to_np(run.queries["q"][0]).transpose(1, 0, 2)       # [16, N, D]
+    k = Hn.to_np(run.cache["k"][0, :, 0])[None].repeat(16, 0)
+    v = Hn.to_np(run.cache["v"][0, :, 0])[None].repeat(16, 0)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), is_causal=True).numpy()
+    got = run.out[0].float().cpu().numpy().transpose(1, 0, 2)
+    assert np.abs(got - ref).max() <= Hn.ATTN_ATOL
+
+
+def test_forward_decode_workload_full_size(cuda_device):
+    """16 sequences x 262144 cached tokens, one query each; two sequences checked."""
+    wl = WL["decode"]
+    _e2e(wl, cuda_device, [0], seqs=(0, 11))
+
+
+def test_forward_prefill128k_last_chunk(cuda_device):
+    wl = dataclasses.replace(WL["prefill128k"], q_start=131072 - 8192)
+    _e2e(wl, cuda_device, Hn.sample_rows(wl, 24))
