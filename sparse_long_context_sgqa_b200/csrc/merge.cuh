@@ -61,9 +61,12 @@ merge_blocks_kernel(const void* __restrict__ kp, const void* __restrict__ logits
     float m = c[0][d];
 #pragma unroll
     for (int j = 1; j < B; ++j) m = fmaxf(m, c[j][d]);
-    float num = 0.f, den = 0.f;
+    // The sums start from the first term (not from +0), so a block whose
+    // terms are all -0 keeps the sign of zero, as a plain sum does.
+    float den = expf(c[0][d] - m);
+    float num = den * k[0][d];
 #pragma unroll
-    for (int j = 0; j < B; ++j) {
+    for (int j = 1; j < B; ++j) {
       const float e = expf(c[j][d] - m);
       den += e;
       num = fmaf(e, k[j][d], num);
