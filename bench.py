@@ -184,7 +184,22 @@ def stage_times(wl, p, model, q, dev):
         if n <= 32:
             work["attn_bytes"] += attn_bytes_decode(cnt, q0, wl)
         work["launches"] += 1
+        if n > 32 and c0 + chunk >= wl.nq:
+            work["union"] = union_stats(sel, cnt, wl)
     return ms, work
+
+
+def union_stats(sel, cnt, wl):
+    """Blocks per 8-query unit (the attention kernel's work) against blocks per query."""
+    S, n, G, k = sel.shape
+    nb = n // 8
+    u = sel[:, :nb * 8].reshape(S, nb, 8, G, k).permute(0, 1, 3, 2, 4).reshape(-1, 8 * k)
+    u = torch.sort(u, dim=-1).values
+    distinct = ((u[:, 1:] != u[:, :-1]) & (u[:, 1:] >= 0)).sum(-1) + (u[:, 0] >= 0).to(torch.int64)
+    per_unit = float(distinct.double().mean())
+    per_query = float(cnt.double().mean())
+    return {"blocks_per_unit": per_unit, "blocks_per_query": per_query,
+            "inflation": per_unit / max(per_query, 1e-9)}
 
 
 def cuda_arm(args, wl, rank, world, local_rank):
@@ -258,6 +273,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
                    "idx_heads": wl.idx_heads, "block": wl.block, "topk": wl.topk,
                    "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (no flush)"},
         "stages_ms_per_step": ms_stage,
+        "union": work.get("union"),
         "stage_tflops": {"index": work["index_flops"] / (ms_stage["index"] / 1e3) / 1e12 if ms_stage["index"] else None,
                          "attention": work["attn_flops"] / (ms_stage["attention"] / 1e3) / 1e12},
         "roofline": roof,

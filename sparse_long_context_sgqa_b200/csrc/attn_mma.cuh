@@ -34,10 +34,95 @@ constexpr int kStageElems = kStepTok * kRowPad;  // one K or V stage
 // the 8 queries' selected blocks, each with an 8-bit mask of the queries that
 // selected it.
 // ---------------------------------------------------------------------------
-constexpr int kPlanThreads = 1024;
+constexpr int kPlanThreads = 512;
 
+// The candidate ids of a unit are < floor(t_last / B); a bitmap over that range
+// (one bit per block, in shared memory) turns the union into set-bit order:
+// set bits, prefix-popcount the words, then every (query, id) finds its union
+// position from the prefix and ORs its query bit into that entry's mask.
 __global__ void __launch_bounds__(kPlanThreads)
 attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ sel_count,
+                 int64_t nq, int G, int k, int nwords, int32_t* __restrict__ plan_ids,
+                 uint8_t* __restrict__ plan_mask, int32_t* __restrict__ plan_count) {
+  extern __shared__ uint32_t sm_words[];      // [nwords] bitmap, then [nwords] prefix
+  uint32_t* bm = sm_words;
+  uint32_t* pre = sm_words + nwords;
+  __shared__ int warp_sums[kPlanThreads / 32];
+  __shared__ int s_total;
+  const int64_t nqb = (nq + 7) / 8;
+  const int64_t unit = blockIdx.x;  // (seq * nqb + qb) * G + g
+  const int g = static_cast<int>(unit % G);
+  const int64_t qb = (unit / G) % nqb;
+  const int64_t seq = unit / (G * nqb);
+  const int tid = threadIdx.x;
+  for (int w = tid; w < nwords; w += kPlanThreads) bm[w] = 0;
+  __syncthreads();
+  const int nq_here = static_cast<int>(nq - qb * 8 < 8 ? nq - qb * 8 : 8);
+  const int64_t row0 = (seq * nq + qb * 8) * G + g;
+  const int nbits = nwords * 32;
+  for (int q = 0; q < nq_here; ++q) {
+    const int64_t row = row0 + static_cast<int64_t>(q) * G;
+    const int cnt = min(max(sel_count[row], 0), k);
+    for (int j = tid; j < cnt; j += kPlanThreads) {
+      const int id = sel[row * k + j];
+      if (id >= 0 && id < nbits) atomicOr(&bm[id >> 5], 1u << (id & 31));
+      else report(kDevBounds);
+    }
+  }
+  __syncthreads();
+  // exclusive prefix of popcounts, words split into contiguous per-thread runs
+  const int per = (nwords + kPlanThreads - 1) / kPlanThreads;
+  const int w0 = tid * per, w1 = min(nwords, w0 + per);
+  int local = 0;
+  for (int w = w0; w < w1; ++w) local += __popc(bm[w]);
+  const int lane = tid & 31, warp = tid >> 5;
+  int x = local;
+  for (int o = 1; o < 32; o <<= 1) { int y = __shfl_up_sync(0xffffffffu, x, o); if (lane >= o) x += y; }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kPlanThreads / 32 ? warp_sums[lane] : 0;
+    for (int o = 1; o < 32; o <<= 1) { int y = __shfl_up_sync(0xffffffffu, w, o); if (lane >= o) w += y; }
+    if (lane < kPlanThreads / 32) warp_sums[lane] = w;
+    if (lane == kPlanThreads / 32 - 1) s_total = w;
+  }
+  __syncthreads();
+  int run = (warp > 0 ? warp_sums[warp - 1] : 0) + x - local;
+  const int64_t obase = unit * (8 * static_cast<int64_t>(k));
+  for (int w = w0; w < w1; ++w) {
+    pre[w] = run;
+    uint32_t bits = bm[w];
+    int pos = run;
+    while (bits) {
+      const int b = __ffs(bits) - 1;
+      bits &= bits - 1;
+      plan_ids[obase + pos] = w * 32 + b;
+      plan_mask[obase + pos] = 0;
+      ++pos;
+    }
+    run = pos;
+  }
+  __syncthreads();
+  uint32_t* mask32 = reinterpret_cast<uint32_t*>(plan_mask + obase);  // 8k-byte aligned per unit
+  for (int q = 0; q < nq_here; ++q) {
+    const int64_t row = row0 + static_cast<int64_t>(q) * G;
+    const int cnt = min(max(sel_count[row], 0), k);
+    for (int j = tid; j < cnt; j += kPlanThreads) {
+      const int id = sel[row * k + j];
+      if (id < 0 || id >= nbits) continue;
+      const int pos = pre[id >> 5] + __popc(bm[id >> 5] & ((1u << (id & 31)) - 1u));
+      atomicOr(&mask32[pos >> 2], (1u << q) << (8 * (pos & 3)));
+    }
+  }
+  if (tid == 0) plan_count[unit] = s_total;
+}
+
+constexpr int kPlanSortThreads = 1024;
+
+// Same plan by a bitonic sort of the 8 lists' (id, query) keys; used when the
+// id range is too wide for a shared-memory bitmap (B = 1 at very long contexts).
+__global__ void __launch_bounds__(kPlanSortThreads)
+attn_plan_sort_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ sel_count,
                  int64_t nq, int G, int k, int pow2, int32_t* __restrict__ plan_ids,
                  uint8_t* __restrict__ plan_mask, int32_t* __restrict__ plan_count) {
   extern __shared__ uint32_t sk[];  // pow2 keys
@@ -48,20 +133,20 @@ attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ se
   const int64_t qb = (unit / G) % nqb;
   const int64_t seq = unit / (G * nqb);
   const int tid = threadIdx.x;
-  for (int j = tid; j < pow2; j += kPlanThreads) sk[j] = 0xFFFFFFFFu;
+  for (int j = tid; j < pow2; j += kPlanSortThreads) sk[j] = 0xFFFFFFFFu;
   __syncthreads();
   for (int q = 0; q < 8; ++q) {
     const int64_t i = qb * 8 + q;
     if (i >= nq) break;
     const int64_t row = (seq * nq + i) * G + g;
     const int cnt = min(max(sel_count[row], 0), k);
-    for (int j = tid; j < cnt; j += kPlanThreads)
+    for (int j = tid; j < cnt; j += kPlanSortThreads)
       sk[q * k + j] = (static_cast<uint32_t>(sel[row * k + j]) << 3) | q;
   }
   __syncthreads();
   for (int size = 2; size <= pow2; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int c = tid; c < pow2 / 2; c += kPlanThreads) {
+      for (int c = tid; c < pow2 / 2; c += kPlanSortThreads) {
         const int lo = 2 * stride * (c / stride) + (c % stride);
         const int hi = lo + stride;
         const bool asc = (lo & size) == 0;
@@ -72,7 +157,7 @@ attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ se
     }
   }
   // Dedup: a run of equal ids becomes one entry whose mask ORs the run.
-  const int per = pow2 / kPlanThreads > 0 ? pow2 / kPlanThreads : 1;
+  const int per = pow2 / kPlanSortThreads > 0 ? pow2 / kPlanSortThreads : 1;
   const int beg = tid * per;
   int heads = 0;
   for (int j = beg; j < beg + per && j < pow2; ++j) {
@@ -102,7 +187,7 @@ attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ se
     plan_mask[obase + pos] = static_cast<uint8_t>(m);
     ++pos;
   }
-  if (tid == kPlanThreads - 1) plan_count[unit] = pos;
+  if (tid == kPlanSortThreads - 1) plan_count[unit] = pos;
 }
 
 // ---------------------------------------------------------------------------

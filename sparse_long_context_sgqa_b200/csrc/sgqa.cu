@@ -5,13 +5,16 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
+#include <cudaTypedefs.h>
 #include <string>
 
 #include "../../include/sgqa.h"
 #include "attn_mma.cuh"
+#include "attn_tc.cuh"
 #include "common.cuh"
 #include "index_rows.cuh"
 #include "merge.cuh"
@@ -75,6 +78,12 @@ int decode_splits(int64_t rows) {
   return static_cast<int>(std::min<int64_t>(std::max<int64_t>(s, 1), 32));
 }
 
+// Prefill attention path for B = 8: tcgen05 kernel unless SGQA_ATTN_PATH=mma.
+bool use_tc_attention() {
+  const char* e = getenv("SGQA_ATTN_PATH");
+  return !(e != nullptr && strcmp(e, "mma") == 0);
+}
+
 int plan_pow2(int k) {
   int p = 1;
   while (p < 8 * k) p <<= 1;
@@ -118,7 +127,7 @@ AttnWs attn_ws(const sgqa_params* p, int64_t S, int64_t nq) {
     w.ids_off = 0;
     size_t ids = align256(static_cast<size_t>(units * cap) * 4);
     w.mask_off = ids;
-    size_t mask = align256(static_cast<size_t>(units * cap));
+    size_t mask = align256(static_cast<size_t>(units * cap) + 64);
     w.cnt_off = ids + mask;
     size_t cnt = align256(static_cast<size_t>(units) * 4);
     w.bytes = ids + mask + cnt;
@@ -197,6 +206,61 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
   return SGQA_OK;
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims/strides innermost first, strides in bytes for dims >= 1.
+sgqa_status encode_bf16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                        const cuuint64_t* strides, const cuuint32_t* box, const char* what) {
+  auto enc = tmap_encoder();
+  if (enc == nullptr) return fail(SGQA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SGQA_ERR_CUDA, "tensor map for %s: CUresult %d", what, (int)r);
+  return SGQA_OK;
+}
+
+sgqa_status launch_attn_tc(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q,
+                           int64_t cap, int64_t clen, const void* kc, const void* vc, const int32_t* ids,
+                           const uint8_t* msk, const int32_t* cnt, void* out, int64_t units, cudaStream_t st) {
+  const int G = p->num_kv_groups;
+  const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
+  CUtensorMap qm, km, vm;
+  sgqa_status s;
+  {
+    cuuint64_t dims[2] = {192, static_cast<cuuint64_t>(S * nq * G * 16)};
+    cuuint64_t strides[1] = {192 * 2};
+    cuuint32_t box[2] = {64, 16};
+    if ((s = encode_bf16(&qm, q, 2, dims, strides, box, "q")) != SGQA_OK) return s;
+  }
+  {
+    // (64 elements, token rows < cache_len, 3 column chunks, group, sequence)
+    cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(clen), 3, static_cast<cuuint64_t>(G), static_cast<cuuint64_t>(S)};
+    cuuint64_t strides[4] = {static_cast<cuuint64_t>(G) * 384, 128, 384, static_cast<cuuint64_t>(cap) * G * 384};
+    cuuint32_t box[5] = {64, 8, 3, 1, 1};
+    if ((s = encode_bf16(&km, kc, 5, dims, strides, box, "k_cache")) != SGQA_OK) return s;
+    if ((s = encode_bf16(&vm, vc, 5, dims, strides, box, "v_cache")) != SGQA_OK) return s;
+  }
+  static_assert(sizeof(sgqa::AttnTcSmem) + 1024 <= 232448, "attention tile exceeds shared memory");
+  const size_t smem = sizeof(sgqa::AttnTcSmem) + 1024;
+  cudaFuncSetAttribute(sgqa::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  sgqa::attn_tc_kernel<<<static_cast<unsigned>(units), sgqa::kTcThreads, smem, st>>>(
+      qm, km, vm, ids, msk, cnt, static_cast<__nv_bfloat16*>(out), nq, G, p->topk, q0, scale_log2);
+  SGQA_LAUNCH_CHECK("attn_tc_kernel");
+  return SGQA_OK;
+}
+
 template <int B>
 sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q,
                         int64_t cap, int64_t clen, const void* kc, const void* vc, const int32_t* sel,
@@ -222,15 +286,27 @@ sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq,
     return SGQA_OK;
   }
   const int64_t units = S * ((nq + 7) / 8) * G;
-  const int pow2 = plan_pow2(k);
+  const int64_t nbits = std::max<int64_t>((q0 + nq - 1) / B, 1);
+  const int nwords = static_cast<int>((nbits + 31) / 32);
   int32_t* ids = ws_at<int32_t>(ws, w.ids_off);
   uint8_t* msk = ws_at<uint8_t>(ws, w.mask_off);
   int32_t* cnt = ws_at<int32_t>(ws, w.cnt_off);
-  const size_t psmem = static_cast<size_t>(pow2) * 4;
-  cudaFuncSetAttribute(sgqa::attn_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
-  sgqa::attn_plan_kernel<<<static_cast<unsigned>(units), sgqa::kPlanThreads, psmem, st>>>(
-      sel, sel_count, nq, G, k, pow2, ids, msk, cnt);
-  SGQA_LAUNCH_CHECK("attn_plan_kernel");
+  const size_t psmem = static_cast<size_t>(nwords) * 8;
+  if (psmem <= 96 * 1024) {
+    cudaFuncSetAttribute(sgqa::attn_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
+    sgqa::attn_plan_kernel<<<static_cast<unsigned>(units), sgqa::kPlanThreads, psmem, st>>>(
+        sel, sel_count, nq, G, k, nwords, ids, msk, cnt);
+    SGQA_LAUNCH_CHECK("attn_plan_kernel");
+  } else {
+    const int pow2 = plan_pow2(k);
+    const size_t ssmem = static_cast<size_t>(pow2) * 4;
+    cudaFuncSetAttribute(sgqa::attn_plan_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
+    sgqa::attn_plan_sort_kernel<<<static_cast<unsigned>(units), sgqa::kPlanSortThreads, ssmem, st>>>(
+        sel, sel_count, nq, G, k, pow2, ids, msk, cnt);
+    SGQA_LAUNCH_CHECK("attn_plan_sort_kernel");
+  }
+  if (B == 8 && use_tc_attention())
+    return launch_attn_tc(p, S, q0, nq, q, cap, clen, kc, vc, ids, msk, cnt, out, units, st);
   const size_t smem = sgqa::kGroupedStages * 2 * sgqa::kStageElems * 2;
   cudaFuncSetAttribute(sgqa::attn_grouped_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   sgqa::attn_grouped_kernel<B><<<static_cast<unsigned>(units), sgqa::kGroupedThreads, smem, st>>>(
