@@ -159,11 +159,12 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int& total, int* warp
 __global__ void __launch_bounds__(kSelThreads)
 topk_rows_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int G,
                  int64_t q_pos0, int B, int k, int32_t* __restrict__ sel,
-                 int32_t* __restrict__ sel_count) {
+                 int32_t* __restrict__ sel_count, const int32_t* __restrict__ only_if) {
   __shared__ uint32_t hist[2048];
   __shared__ int warp_sums[32];
   __shared__ uint32_t s_prefix, s_rem;
   const int64_t row = blockIdx.x;  // (seq * nq + i) * G + g
+  if (only_if != nullptr && only_if[row] == 0) return;  // row already selected
   const int64_t i = (row / G) % nq;
   const int64_t t = q_pos0 + i;
   const int64_t n = t / B;

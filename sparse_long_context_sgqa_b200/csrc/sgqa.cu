@@ -17,6 +17,7 @@
 #include "attn_tc.cuh"
 #include "common.cuh"
 #include "index_rows.cuh"
+#include "index_tc.cuh"
 #include "merge.cuh"
 
 namespace {
@@ -90,19 +91,35 @@ int plan_pow2(int k) {
   return std::max(p, 2);
 }
 
+// Staging capacity per (query, group) list of the streaming top-k: room for k
+// kept entries plus at least two candidate tiles of appends.
+int staging_cap(int k) {
+  const int64_t c = std::max<int64_t>(4 * static_cast<int64_t>(k), k + 2 * sgqa::kIdxCand);
+  return static_cast<int>(round_up(c, 32));
+}
+
 struct IndexWs {
   int64_t rpad;
-  size_t keys_off, scores_off, bytes;
+  int cap;
+  size_t keys_off, scores_off, flags_off, staging_off, staged_off, bytes;
 };
 IndexWs index_ws(const sgqa_params* p, int64_t S, int64_t nq, int64_t max_ctx) {
   IndexWs w;
   const int64_t rneed = std::max<int64_t>((max_ctx - 1) / p->block_size, 1);
-  w.rpad = round_up(rneed, 64);
+  w.rpad = round_up(rneed, 128);
+  w.cap = staging_cap(p->topk);
   w.keys_off = 0;
-  size_t keys = align256(static_cast<size_t>(S * w.rpad * 64) * 2);
+  const size_t keys = align256(static_cast<size_t>(S * w.rpad * 64) * 2);
+  const int64_t rows = S * nq * p->num_kv_groups;
+  // materialised scores (few queries) or staging lists (prefill) share one region
   w.scores_off = keys;
-  size_t scores = align256(static_cast<size_t>(S * nq * p->num_kv_groups * w.rpad) * 4);
-  w.bytes = keys + scores;
+  const size_t scores = align256(static_cast<size_t>(rows * w.rpad) * 4) + align256(static_cast<size_t>(rows) * 4);
+  w.flags_off = keys + align256(static_cast<size_t>(rows * w.rpad) * 4);
+  w.staging_off = keys;
+  const size_t staging = align256(static_cast<size_t>(rows) * w.cap * 8);
+  w.staged_off = keys + staging;
+  const size_t staged = align256(static_cast<size_t>(rows) * 4);
+  w.bytes = keys + std::max(scores, staging + staged);
   return w;
 }
 
@@ -174,38 +191,6 @@ sgqa_status do_merge(const sgqa_params* p, int64_t S, int64_t cap, const void* k
   return SGQA_OK;
 }
 
-sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* idx_q,
-                     const float* idx_w, int64_t cap, const uint8_t* store, int32_t* sel,
-                     int32_t* sel_count, void* ws, cudaStream_t st) {
-  const int B = p->block_size, G = p->num_kv_groups, H = p->idx_heads;
-  const IndexWs w = index_ws(p, S, nq, q0 + nq);
-  const int64_t rneed = (q0 + nq - 1) / B;
-  __nv_bfloat16* keys = ws_at<__nv_bfloat16>(ws, w.keys_off);
-  float* scores = ws_at<float>(ws, w.scores_off);
-  if (rneed > 0) {
-    const int64_t threads = S * rneed * 8;
-    sgqa::widen_store_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(
-        store, cap / B, rneed, w.rpad, S, keys);
-    SGQA_LAUNCH_CHECK("widen_store_kernel");
-    const int qpc = 64 / H;
-    dim3 grid(static_cast<unsigned>((nq + qpc - 1) / qpc),
-              static_cast<unsigned>((rneed + sgqa::kScoreCandPerCta - 1) / sgqa::kScoreCandPerCta),
-              static_cast<unsigned>(S * G));
-    if (grid.y > 65535 || grid.z > 65535) return fail(SGQA_ERR_UNSUPPORTED, "index grid too large");
-    const __nv_bfloat16* iq = static_cast<const __nv_bfloat16*>(idx_q);
-    if (H == 8)
-      sgqa::index_score_kernel<8><<<grid, sgqa::kScoreWarps * 32, 0, st>>>(iq, idx_w, keys, scores, nq, G, q0, B, w.rpad);
-    else
-      sgqa::index_score_kernel<4><<<grid, sgqa::kScoreWarps * 32, 0, st>>>(iq, idx_w, keys, scores, nq, G, q0, B, w.rpad);
-    SGQA_LAUNCH_CHECK("index_score_kernel");
-  }
-  const int64_t rows = S * nq * G;
-  sgqa::topk_rows_kernel<<<static_cast<unsigned>(rows), sgqa::kSelThreads, 0, st>>>(
-      scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count);
-  SGQA_LAUNCH_CHECK("topk_rows_kernel");
-  return SGQA_OK;
-}
-
 PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = []() {
     void* f = nullptr;
@@ -258,6 +243,135 @@ sgqa_status launch_attn_tc(const sgqa_params* p, int64_t S, int64_t q0, int64_t 
   sgqa::attn_tc_kernel<<<static_cast<unsigned>(units), sgqa::kTcThreads, smem, st>>>(
       qm, km, vm, ids, msk, cnt, static_cast<__nv_bfloat16*>(out), nq, G, p->topk, q0, scale_log2);
   SGQA_LAUNCH_CHECK("attn_tc_kernel");
+  return SGQA_OK;
+}
+
+// Index path for many queries: tcgen05 score rows + two-pass top-k by default;
+// SGQA_INDEX_PATH=stream selects the fused streaming top-k kernel instead.
+bool use_stream_index() {
+  const char* e = getenv("SGQA_INDEX_PATH");
+  return e != nullptr && strcmp(e, "stream") == 0;
+}
+
+sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* idx_q,
+                     const float* idx_w, int64_t cap, const uint8_t* store, int32_t* sel,
+                     int32_t* sel_count, void* ws, cudaStream_t st) {
+  const int B = p->block_size, G = p->num_kv_groups, H = p->idx_heads;
+  const IndexWs w = index_ws(p, S, nq, q0 + nq);
+  const int64_t rneed = (q0 + nq - 1) / B;
+  __nv_bfloat16* keys = ws_at<__nv_bfloat16>(ws, w.keys_off);
+  if (rneed > 0) {
+    const int64_t threads = S * rneed * 8;
+    sgqa::widen_store_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(
+        store, cap / B, rneed, w.rpad, S, keys);
+    SGQA_LAUNCH_CHECK("widen_store_kernel");
+  }
+  const __nv_bfloat16* iq = static_cast<const __nv_bfloat16*>(idx_q);
+  if (nq > kDecodeMaxNq && use_stream_index()) {
+    uint2* staging = ws_at<uint2>(ws, w.staging_off);
+    int32_t* staged = ws_at<int32_t>(ws, w.staged_off);
+    const int Q = sgqa::kIdxCols / H;
+    sgqa_status s;
+    CUtensorMap km, qm;
+    {
+      cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(S * w.rpad)};
+      cuuint64_t strides[1] = {128};
+      cuuint32_t box[2] = {64, static_cast<cuuint32_t>(sgqa::kIdxCand)};
+      if ((s = encode_bf16(&km, keys, 2, dims, strides, box, "indexer keys")) != SGQA_OK) return s;
+    }
+    {
+      cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(G),
+                            static_cast<cuuint64_t>(S * nq)};
+      cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(H) * 128, static_cast<cuuint64_t>(G) * H * 128};
+      cuuint32_t box[4] = {64, static_cast<cuuint32_t>(H), 1, static_cast<cuuint32_t>(Q)};
+      if ((s = encode_bf16(&qm, iq, 4, dims, strides, box, "idx_q")) != SGQA_OK) return s;
+    }
+    const int64_t ntq = (nq + Q - 1) / Q;
+    const int64_t grid = static_cast<int64_t>(G) * S * ntq;
+    static_assert(sizeof(sgqa::IndexTcSmem) + 1024 <= 232448, "index tile exceeds shared memory");
+    const size_t smem = sizeof(sgqa::IndexTcSmem) + 1024;
+    if (H == 8) {
+      cudaFuncSetAttribute(sgqa::index_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      sgqa::index_tc_kernel<8><<<static_cast<unsigned>(grid), sgqa::kIdxThreads, smem, st>>>(
+          km, qm, idx_w, staging, staged, nq, G, q0, B, w.rpad, p->topk, w.cap);
+    } else {
+      cudaFuncSetAttribute(sgqa::index_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      sgqa::index_tc_kernel<4><<<static_cast<unsigned>(grid), sgqa::kIdxThreads, smem, st>>>(
+          km, qm, idx_w, staging, staged, nq, G, q0, B, w.rpad, p->topk, w.cap);
+    }
+    SGQA_LAUNCH_CHECK("index_tc_kernel");
+    const int buf_entries = std::min(w.cap, 2048);
+    const size_t fsmem = static_cast<size_t>(sgqa::kFinalWarps) * buf_entries * 8;
+    cudaFuncSetAttribute(sgqa::topk_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem);
+    const int64_t rows = S * nq * G;
+    sgqa::topk_final_kernel<<<static_cast<unsigned>((rows + sgqa::kFinalWarps - 1) / sgqa::kFinalWarps),
+                              sgqa::kFinalWarps * 32, fsmem, st>>>(staging, staged, rows, nq, G, q0, B, p->topk,
+                                                                   w.cap, buf_entries, sel, sel_count);
+    SGQA_LAUNCH_CHECK("topk_final_kernel");
+    return SGQA_OK;
+  }
+  float* scores = ws_at<float>(ws, w.scores_off);
+  int32_t* flags = ws_at<int32_t>(ws, w.flags_off);
+  if (rneed > 0 && nq > kDecodeMaxNq) {
+    // tcgen05 scores: 256 (query, head) columns per CTA, 128 candidates per MMA
+    const int Q = sgqa::kIdxCols / H;
+    sgqa_status s;
+    CUtensorMap km, qm;
+    {
+      cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(S * w.rpad)};
+      cuuint64_t strides[1] = {128};
+      cuuint32_t box[2] = {64, static_cast<cuuint32_t>(sgqa::kIdxCand)};
+      if ((s = encode_bf16(&km, keys, 2, dims, strides, box, "indexer keys")) != SGQA_OK) return s;
+    }
+    {
+      cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(G),
+                            static_cast<cuuint64_t>(S * nq)};
+      cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(H) * 128, static_cast<cuuint64_t>(G) * H * 128};
+      cuuint32_t box[4] = {64, static_cast<cuuint32_t>(H), 1, static_cast<cuuint32_t>(Q)};
+      if ((s = encode_bf16(&qm, iq, 4, dims, strides, box, "idx_q")) != SGQA_OK) return s;
+    }
+    const int64_t grid = static_cast<int64_t>(G) * S * ((nq + Q - 1) / Q);
+    const size_t smem = sizeof(sgqa::IndexTcSmem) + 1024;
+    if (H == 8) {
+      cudaFuncSetAttribute(sgqa::index_score_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      sgqa::index_score_tc_kernel<8><<<static_cast<unsigned>(grid), sgqa::kIdxThreads, smem, st>>>(
+          km, qm, idx_w, scores, nq, G, q0, B, w.rpad);
+    } else {
+      cudaFuncSetAttribute(sgqa::index_score_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      sgqa::index_score_tc_kernel<4><<<static_cast<unsigned>(grid), sgqa::kIdxThreads, smem, st>>>(
+          km, qm, idx_w, scores, nq, G, q0, B, w.rpad);
+    }
+    SGQA_LAUNCH_CHECK("index_score_tc_kernel");
+  } else if (rneed > 0) {
+    const int qpc = 64 / H;
+    dim3 grid(static_cast<unsigned>((nq + qpc - 1) / qpc),
+              static_cast<unsigned>((rneed + sgqa::kScoreCandPerCta - 1) / sgqa::kScoreCandPerCta),
+              static_cast<unsigned>(S * G));
+    if (grid.y > 65535 || grid.z > 65535) return fail(SGQA_ERR_UNSUPPORTED, "index grid too large");
+    if (H == 8)
+      sgqa::index_score_kernel<8><<<grid, sgqa::kScoreWarps * 32, 0, st>>>(iq, idx_w, keys, scores, nq, G, q0, B, w.rpad);
+    else
+      sgqa::index_score_kernel<4><<<grid, sgqa::kScoreWarps * 32, 0, st>>>(iq, idx_w, keys, scores, nq, G, q0, B, w.rpad);
+    SGQA_LAUNCH_CHECK("index_score_kernel");
+  }
+  const int64_t rows = S * nq * G;
+  const int nwords = static_cast<int>((std::max<int64_t>(rneed, 1) + 31) / 32);
+  const size_t ssmem = (static_cast<size_t>(sgqa::kRows2Bins) + 2 * sgqa::kRows2Cand + nwords) * 4;
+  // The histogram + gather variant is opt-in (SGQA_TOPK_PATH=hist2); the
+  // three-pass radix select is the default.
+  const char* tp = getenv("SGQA_TOPK_PATH");
+  const bool hist2 = tp != nullptr && strcmp(tp, "hist2") == 0;
+  if (hist2 && ssmem <= 200 * 1024) {
+    cudaFuncSetAttribute(sgqa::topk_rows2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
+    sgqa::topk_rows2_kernel<<<static_cast<unsigned>(rows), sgqa::kRows2Threads, ssmem, st>>>(
+        scores, w.rpad, nq, G, q0, B, p->topk, nwords, sel, sel_count, flags);
+    SGQA_LAUNCH_CHECK("topk_rows2_kernel");
+  } else {
+    flags = nullptr;  // too wide for the bitmap: the radix kernel takes every row
+  }
+  sgqa::topk_rows_kernel<<<static_cast<unsigned>(rows), sgqa::kSelThreads, 0, st>>>(
+      scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, flags);
+  SGQA_LAUNCH_CHECK("topk_rows_kernel");
   return SGQA_OK;
 }
 
