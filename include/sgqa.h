@@ -156,6 +156,32 @@ sgqa_status sgqa_forward(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0,
                          void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Sparse attention for decode-sized calls without a caller workspace.  The
+ * pages have no counterpart: this entry point exists for callers that cannot
+ * allocate device memory when they call -- a host runtime that fixed its
+ * device memory at start-up, or a plugin reached through a plain C interface
+ * with no allocator handle -- and cudaMalloc may also synchronise the device,
+ * which a latency-bound decode step must avoid.
+ *
+ * Same computation and arguments as sgqa_sparse_attn, minus the workspace.
+ * It takes only calls with nq <= 32 queries per sequence (the split-K decode
+ * path) whose split partials fit the library's static scratch array of
+ * SGQA_NOALLOC_SCRATCH_BYTES (16 MiB) per device; larger calls return
+ * SGQA_ERR_UNSUPPORTED with a message.  The array is a file-scope __device__
+ * variable that every GPU loading the library holds until exit.  The first
+ * call on a device looks up the array's device address (set-up); make that
+ * first call before any stream capture.  All calls share the array, so calls
+ * that overlap on the GPU (other streams, other host threads) race; order
+ * them on one stream.  Nothing in the array needs clearing: every call writes
+ * each partial it reads.  No cudaMalloc, cudaFree or allocating routine.
+ */
+#define SGQA_NOALLOC_SCRATCH_BYTES (16u << 20)
+sgqa_status sgqa_sparse_attn_noalloc(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                                     const void* q, int64_t cache_cap, int64_t cache_len,
+                                     const void* k_cache, const void* v_cache,
+                                     const int32_t* sel, const int32_t* sel_count, void* out, void* stream);
+
+/*
  * Synchronise `stream` and report the device status word that bounded waits
  * and device-side checks write (then clear it).  Returns SGQA_OK,
  * SGQA_ERR_TIMEOUT, SGQA_ERR_DEVICE or SGQA_ERR_CUDA.

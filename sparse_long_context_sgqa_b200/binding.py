@@ -25,7 +25,7 @@ STATUS = {0: "SGQA_OK", 1: "SGQA_ERR_INVALID_ARGUMENT", 2: "SGQA_ERR_UNSUPPORTED
           3: "SGQA_ERR_WORKSPACE", 4: "SGQA_ERR_CUDA", 5: "SGQA_ERR_TIMEOUT", 6: "SGQA_ERR_DEVICE"}
 
 EXPORTED = ["sgqa_workspace_size", "sgqa_merge_blocks", "sgqa_index_topk", "sgqa_sparse_attn",
-            "sgqa_forward", "sgqa_check", "sgqa_last_error", "sgqa_version"]
+            "sgqa_forward", "sgqa_sparse_attn_noalloc", "sgqa_check", "sgqa_last_error", "sgqa_version"]
 
 
 class SgqaError(RuntimeError):
@@ -67,6 +67,7 @@ _lib.sgqa_sparse_attn.argtypes = [_P, _i64, _i64, _i64, _vp, _i64, _i64, _vp, _v
                                   _vp, _sz, _vp]
 _lib.sgqa_forward.argtypes = [_P, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp,
                               _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.sgqa_sparse_attn_noalloc.argtypes = [_P, _i64, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.sgqa_check.argtypes = [_vp]
 _lib.sgqa_last_error.restype = ctypes.c_char_p
 _lib.sgqa_version.restype = ctypes.c_char_p
@@ -133,6 +134,15 @@ def sgqa_forward(p: Params, num_seqs, q_pos0, nq, q, idx_q, idx_w, cache_cap, ca
                           _ptr(v_cache), _ptr(merged_f32), _ptr(store), _ptr(sel), _ptr(sel_count),
                           _ptr(out), _ptr(workspace), workspace.numel() if workspace is not None else 0,
                           _stream(stream)))
+
+
+def sgqa_sparse_attn_noalloc(p: Params, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k_cache, v_cache, sel,
+                             sel_count, out, stream=None):
+    """sgqa_sparse_attn for decode-sized calls (nq <= 32) using the library's
+    static scratch instead of a workspace; for callers that cannot allocate."""
+    _ok(_lib.sgqa_sparse_attn_noalloc(ctypes.byref(p.c()), num_seqs, q_pos0, nq, _ptr(q), cache_cap, cache_len,
+                                      _ptr(k_cache), _ptr(v_cache), _ptr(sel), _ptr(sel_count), _ptr(out),
+                                      _stream(stream)))
 
 
 def sgqa_check(stream=None):

@@ -9,6 +9,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cudaTypedefs.h>
 #include <string>
 
@@ -458,6 +459,29 @@ sgqa_status check_common(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq
     if (!aligned((ptr), (align))) return fail(SGQA_ERR_INVALID_ARGUMENT, #ptr " must be %d-byte aligned", (int)(align)); \
   } while (0)
 
+// Scratch for sgqa_sparse_attn_noalloc: a file-scope device array (one per
+// device that loads the library).  Host code needs its device address, looked
+// up once per device with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SGQA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+
+sgqa_status noalloc_scratch(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SGQA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    g_noalloc_ptr[dev].store(p, std::memory_order_release);
+  }
+  *ptr = p;
+  return SGQA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -578,6 +602,35 @@ sgqa_status sgqa_forward(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0,
     return s;
   return do_attn(p, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k_cache, v_cache, sel, sel_count, out,
                  workspace, st);
+}
+
+sgqa_status sgqa_sparse_attn_noalloc(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                                     const void* q, int64_t cache_cap, int64_t cache_len, const void* k_cache,
+                                     const void* v_cache, const int32_t* sel, const int32_t* sel_count,
+                                     void* out, void* stream) {
+  g_err.clear();
+  sgqa_status s = check_common(p, num_seqs, q_pos0, nq, cache_cap);
+  if (s != SGQA_OK) return s;
+  if (cache_len < q_pos0 + nq || cache_len > cache_cap)
+    return fail(SGQA_ERR_INVALID_ARGUMENT, "need q_pos0 + nq <= cache_len <= cache_cap");
+  if (nq == 0) return SGQA_OK;
+  if (nq > kDecodeMaxNq)
+    return fail(SGQA_ERR_UNSUPPORTED, "sgqa_sparse_attn_noalloc takes at most %d queries per sequence (got %lld)",
+                (int)kDecodeMaxNq, (long long)nq);
+  REQUIRE_PTR(q, 16);
+  REQUIRE_PTR(k_cache, 16);
+  REQUIRE_PTR(v_cache, 16);
+  REQUIRE_PTR(sel, 4);
+  REQUIRE_PTR(sel_count, 4);
+  REQUIRE_PTR(out, 16);
+  const AttnWs w = attn_ws(p, num_seqs, nq);
+  if (w.bytes > SGQA_NOALLOC_SCRATCH_BYTES)
+    return fail(SGQA_ERR_UNSUPPORTED, "call needs %zu bytes of scratch; the static array holds %u",
+                w.bytes, (unsigned)SGQA_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != SGQA_OK) return s;
+  return do_attn(p, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k_cache, v_cache, sel, sel_count, out,
+                 scratch, static_cast<cudaStream_t>(stream));
 }
 
 sgqa_status sgqa_check(void* stream) {
