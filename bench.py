@@ -209,11 +209,27 @@ def cuda_arm(args, wl, rank, world, local_rank):
     chunk = min(wl.chunk, wl.nq)
     n_chunks = (wl.nq + chunk - 1) // chunk
 
-    def step():
+    def eager_step():
         if wl.nq <= 32:
             model.forward(wl.q_start, q["q"], q["idx_q"], q["idx_w"], sel, cnt, out)
         else:
             model.prefill(q["q"], q["idx_q"], q["idx_w"], out, sel, cnt, q_pos0=wl.q_start)
+
+    graph = None
+    if wl.nq <= 32 and not args.no_graph:
+        # a decode step is a handful of short kernels: replay it as one CUDA graph
+        eager_step()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            eager_step()
+        torch.cuda.synchronize()
+
+    def step():
+        if graph is not None:
+            graph.replay()
+        else:
+            eager_step()
 
     for _ in range(args.warmup):
         step()
@@ -278,6 +294,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
                          "attention": work["attn_flops"] / (ms_stage["attention"] / 1e3) / 1e12},
         "roofline": roof,
         "gpu_launches": args.steps * n_chunks * launches_per_call(wl),
+        "cuda_graph": graph is not None,
         "clocks": clocks,
         "e2e": e2e,
     }
@@ -378,8 +395,16 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="decode: launch eagerly instead of replaying a CUDA graph")
+    ap.add_argument("--seq-len", type=int, default=0, help="override the workload's context length")
+    ap.add_argument("--num-seqs", type=int, default=0, help="override the workload's sequence count")
     args = ap.parse_args()
     wl = I.WORKLOADS[args.workload]
+    if args.seq_len or args.num_seqs:
+        import dataclasses
+        L = args.seq_len or wl.seq_len
+        qs = L - 1 if wl.n_queries == 1 else wl.q_start
+        wl = dataclasses.replace(wl, seq_len=L, num_seqs=args.num_seqs or wl.num_seqs, q_start=qs)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -128,13 +128,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             rows[e] = (e == 0 || (e == 1 && c0 + 8 <= t_last)) ? static_cast<int32_t>(c0 + 8 * e) : -64;
         }
       };
-      int32_t rows[8];
+      int32_t rows[8], next[8];
       tile_rows(0, rows);
+      if (n_tiles > 1) tile_rows(1, next);
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % kTcStages;
         const uint32_t ph = ((j / kTcStages) - 1) & 1;
-        int32_t next[8];
-        if (j + 1 < n_tiles) tile_rows(j + 1, next);
+        int32_t next2[8];
+        if (j + 2 < n_tiles) tile_rows(j + 2, next2);
         if (j >= kTcStages && !tc::mbar_wait(bar(sm.k_empty[s]), ph, abort)) break;
         tc::mbar_expect_tx(bar(sm.k_full[s]), 8 * 3 * 1024);
 #pragma unroll
@@ -149,7 +150,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                           bar(sm.v_full[s]));
         issued = j + 1;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) rows[e] = next[e];
+        for (int e = 0; e < 8; ++e) {
+          rows[e] = next[e];
+          next[e] = next2[e];
+        }
       }
       if (*abort) {
         // Let the copies already issued land before the CTA's shared memory goes away.
@@ -346,6 +350,287 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     tc::fence_after();
     tc::tmem_dealloc(tmem, 512);
   }
+}
+
+}  // namespace sgqa
+
+namespace sgqa {
+
+// ---------------------------------------------------------------------------
+// Decode attention (few queries, long context): HBM-bound gather of the
+// selected 8-token blocks.  One CTA takes a contiguous range of one (query,
+// group)'s blocks (split-K); a single producer thread streams each block's K
+// and V (one 5-D TMA box each, 3 KB, 128-byte swizzled) into a 16-slot ring,
+// and four compute warps consume two blocks (16 tokens) per step with the
+// warp-level MMA formulation (16 heads = the m16 rows).  Each split writes
+// its (max, sum, unnormalised O); the last split of a row to finish (atomic
+// ticket) combines them into the bf16 output and re-arms the ticket.
+// ---------------------------------------------------------------------------
+constexpr int kDecSlots = 16;
+constexpr int kDecThreads = 160;  // warp 0 producer, warps 1-4 compute
+
+struct __align__(1024) DecSmem {
+  uint8_t kv[kDecSlots][2][3 * 1024];   // [slot][K|V][chunk][8 rows x 128 B]
+  int32_t rows[2049];                   // first token row of each of this CTA's blocks
+  uint64_t full[kDecSlots], empty[kDecSlots];
+  int abort;
+  int last;
+};
+
+// byte offset of (token row r in 0..7, 16-byte piece j in 0..23) in a swizzled block tile
+__device__ __forceinline__ uint32_t blk_off(uint32_t r, uint32_t j) {
+  return (j >> 3) * 1024u + r * 128u + (((j & 7u) ^ r) << 4);
+}
+
+__global__ void __launch_bounds__(kDecThreads, 2)
+attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                       const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ sel,
+                       const int32_t* __restrict__ sel_count, float* __restrict__ part_o,
+                       float* __restrict__ part_ml, int32_t* __restrict__ tickets,
+                       __nv_bfloat16* __restrict__ out, int64_t nq, int G, int k, int64_t q_pos0, int nsplit,
+                       float scale_log2) {
+  extern __shared__ uint8_t smem_raw[];
+  DecSmem& sm = *reinterpret_cast<DecSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x % nsplit;
+  const int64_t row = blockIdx.x / nsplit;  // (seq * nq + i) * G + g
+  const int g = static_cast<int>(row % G);
+  const int64_t i = (row / G) % nq;
+  const int64_t seq = row / (G * nq);
+  const int64_t t = q_pos0 + i;
+  const int cnt = min(max(sel_count[row], 0), k);
+  const int32_t* ids = sel + row * k;
+  const int nblk = cnt + 1;  // selected blocks, then the current block
+  const int per = (nblk + nsplit - 1) / nsplit;
+  const int b0 = min(nblk, split * per), b1 = min(nblk, b0 + per);
+  const int nb = b1 - b0;
+  const int64_t cur0 = 8 * (t / 8);
+  volatile int* abort = &sm.abort;
+  auto bar = [](uint64_t& b) { return smem_u32(&b); };
+  if (threadIdx.x == 0) {
+    sm.abort = 0;
+    for (int s = 0; s < kDecSlots; ++s) {
+      tc::mbar_init(bar(sm.full[s]), 1);
+      tc::mbar_init(bar(sm.empty[s]), 1);
+    }
+    tc::mbar_fence_init();
+  }
+  // stage the block rows (one coalesced read instead of a dependent load per TMA issue)
+  for (int b = threadIdx.x; b < nb; b += kDecThreads) {
+    const int e = b0 + b;
+    sm.rows[b] = e < cnt ? ids[e] * 8 : static_cast<int32_t>(cur0);
+  }
+  // per-warp attention state (warps 1..4); Q loads overlap the staging
+  WarpAttn st;
+  if (warp >= 1) warp_load_q(st, q + ((seq * nq + i) * G + g) * kHg * kD, lane);
+  __syncthreads();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::prefetch_tmap(&kmap);
+      tc::prefetch_tmap(&vmap);
+      // blocks in pairs: step s uses slots 2s, 2s+1 (mod kDecSlots); an odd tail gets a zero block
+      const int nsteps = (nb + 1) / 2;
+      int issued = 0;
+      for (int b = 0; b < 2 * nsteps; ++b) {
+        const int slot = b % kDecSlots;
+        if (b >= kDecSlots && !tc::mbar_wait(bar(sm.empty[slot]), ((b / kDecSlots) - 1) & 1, abort)) break;
+        const int32_t r = b < nb ? sm.rows[b] : -64;  // -64: zero-filled tail block
+        tc::mbar_expect_tx(bar(sm.full[slot]), 2 * 3 * 1024);
+        tc::tma_load_5d(smem_u32(&sm.kv[slot][0][0]), &kmap, 0, r, 0, g, static_cast<int32_t>(seq), bar(sm.full[slot]));
+        tc::tma_load_5d(smem_u32(&sm.kv[slot][1][0]), &vmap, 0, r, 0, g, static_cast<int32_t>(seq), bar(sm.full[slot]));
+        issued = b + 1;
+      }
+      if (*abort) {
+        for (int b = issued > kDecSlots ? issued - kDecSlots : 0; b < issued; ++b) {
+          const uint64_t t0 = globaltimer_ns();
+          while (!tc::mbar_try(bar(sm.full[b % kDecSlots]), (b / kDecSlots) & 1) && globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+      }
+    }
+  } else {
+    const int cw = warp - 1;  // compute warp 0..3
+    const int nsteps = (nb + 1) / 2;
+    const int mrow = lane & 7, mat = lane >> 3;
+    for (int s = cw; s < nsteps; s += 4) {
+      const int ba = 2 * s, bb = 2 * s + 1;
+      const int sa = ba % kDecSlots, sb2 = bb % kDecSlots;
+      if (!tc::mbar_wait(bar(sm.full[sa]), (ba / kDecSlots) & 1, abort)) break;
+      if (!tc::mbar_wait(bar(sm.full[sb2]), (bb / kDecSlots) & 1, abort)) break;
+      // token mask: 8 tokens per block; the current block only up to t; zero blocks none
+      uint32_t tm = 0;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int b = 2 * s + h;
+        if (b < nb) {
+          const int e = b0 + b;
+          uint32_t m8 = 0xFFu;
+          if (e >= cnt) m8 = (t - cur0 >= 7) ? 0xFFu : ((1u << (t - cur0 + 1)) - 1u);
+          tm |= m8 << (8 * h);
+        }
+      }
+      const uint32_t ka = smem_u32(&sm.kv[sa][0][0]), kb = smem_u32(&sm.kv[sb2][0][0]);
+      const uint32_t va = smem_u32(&sm.kv[sa][1][0]), vb = smem_u32(&sm.kv[sb2][1][0]);
+      // S = Q K^T: matrices (tok 0-7 = block a | 8-15 = block b) x (dims 16ks | 16ks+8)
+      float sc[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+      const uint32_t kblk = (mat >> 1) ? kb : ka;
+#pragma unroll
+      for (int ks = 0; ks < 12; ++ks) {
+        uint32_t bf[4];
+        ldmatrix_x4(bf, kblk + blk_off(mrow, 2 * ks + (mat & 1)));
+        mma_bf16_16816(sc[0], st.qf[ks], bf[0], bf[1]);
+        mma_bf16_16816(sc[1], st.qf[ks], bf[2], bf[3]);
+      }
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int tok = 8 * nt + 2 * (lane & 3) + (e & 1);
+          sc[nt][e] = ((tm >> tok) & 1u) ? sc[nt][e] * scale_log2 : -INFINITY;
+          mx[e >> 1] = fmaxf(mx[e >> 1], sc[nt][e]);
+        }
+      }
+      // lazy rescale: the reference max moves only when the new max exceeds it
+      // by more than 2^8 (P stays <= 256, exact in the final normalisation)
+      float alpha[2], muse[2];
+      bool need = false;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+        alpha[r] = 1.f;
+        if (st.m[r] == -INFINITY) {
+          st.m[r] = mx[r];
+        } else if (mx[r] > st.m[r] + 8.f) {
+          alpha[r] = exp2f(st.m[r] - mx[r]);
+          st.m[r] = mx[r];
+          need = true;
+        }
+        muse[r] = st.m[r] == -INFINITY ? 0.f : st.m[r];
+      }
+      float p[2][4], psum[2] = {0.f, 0.f};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          p[nt][e] = exp2f(sc[nt][e] - muse[e >> 1]);
+          psum[e >> 1] += p[nt][e];
+        }
+      st.l[0] = st.l[0] * alpha[0] + psum[0];
+      st.l[1] = st.l[1] * alpha[1] + psum[1];
+      if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int j = 0; j < 24; ++j) {
+          st.o[j][0] *= alpha[0]; st.o[j][1] *= alpha[0];
+          st.o[j][2] *= alpha[1]; st.o[j][3] *= alpha[1];
+        }
+      }
+      uint32_t pa[4];
+      pa[0] = pack_bf16x2(p[0][0], p[0][1]);
+      pa[1] = pack_bf16x2(p[0][2], p[0][3]);
+      pa[2] = pack_bf16x2(p[1][0], p[1][1]);
+      pa[3] = pack_bf16x2(p[1][2], p[1][3]);
+      // PV: trans matrices (tok 0-7 = a | 8-15 = b) x (dims 16jj | 16jj+8)
+      const uint32_t vblk = (mat & 1) ? vb : va;
+#pragma unroll
+      for (int jj = 0; jj < 12; ++jj) {
+        uint32_t bf[4];
+        ldmatrix_x4_trans(bf, vblk + blk_off(mrow, 2 * jj + (mat >> 1)));
+        mma_bf16_16816(st.o[2 * jj], pa, bf[0], bf[1]);
+        mma_bf16_16816(st.o[2 * jj + 1], pa, bf[2], bf[3]);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        tc::mbar_arrive(bar(sm.empty[sa]));
+        tc::mbar_arrive(bar(sm.empty[sb2]));
+      }
+    }
+  }
+  __syncthreads();
+  // combine the four compute warps (shared memory reused), write this split's partial
+  constexpr int kCoStride = kD + 4;                       // padded rows: no bank conflicts
+  float* cm = reinterpret_cast<float*>(&sm.kv[0][0][0]);  // [4][16]
+  float* cl = cm + 4 * kHg;                               // [4][16]
+  float* co = cl + 4 * kHg;                               // [4][16][196]
+  if (warp >= 1) {
+    const int cw = warp - 1;
+    float l0 = st.l[0], l1 = st.l[1];
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    const int h0 = lane >> 2, h1 = h0 + 8;
+    if ((lane & 3) == 0) {
+      cm[cw * kHg + h0] = st.m[0]; cm[cw * kHg + h1] = st.m[1];
+      cl[cw * kHg + h0] = l0;      cl[cw * kHg + h1] = l1;
+    }
+#pragma unroll
+    for (int j = 0; j < 24; ++j) {
+      const int d = 8 * j + 2 * (lane & 3);
+      *reinterpret_cast<float2*>(&co[(cw * kHg + h0) * kCoStride + d]) = make_float2(st.o[j][0], st.o[j][1]);
+      *reinterpret_cast<float2*>(&co[(cw * kHg + h1) * kCoStride + d]) = make_float2(st.o[j][2], st.o[j][3]);
+    }
+  }
+  __syncthreads();
+  float* po = part_o + (row * nsplit + split) * kHg * kD;
+  float* pml = part_ml + (row * nsplit + split) * kHg * 2;
+  for (int idx = threadIdx.x; idx < kHg * kD; idx += kDecThreads) {
+    const int h = idx / kD;
+    float mm = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) mm = fmaxf(mm, cm[w * kHg + h]);
+    const float mu = mm == -INFINITY ? 0.f : mm;
+    float acc = 0.f, ls = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float a = exp2f(cm[w * kHg + h] - mu);
+      acc += a * co[(w * kHg + h) * kCoStride + (idx % kD)];
+      ls += a * cl[w * kHg + h];
+    }
+    po[idx] = acc;
+    if (idx % kD == 0) { pml[2 * h] = mm; pml[2 * h + 1] = ls; }
+  }
+  // the last split of this row combines all partials
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int old = atomicAdd(&tickets[row], 1);
+    sm.last = (old == nsplit - 1);
+  }
+  __syncthreads();
+  if (!sm.last) return;
+  __threadfence();
+  // scale factor of every (split, head) partial, computed once
+  float* fac = co;  // [nsplit][16] (the combine buffers are free again)
+  float* inv = co + 32 * kHg;  // [16]
+  if (threadIdx.x < kHg) {
+    const int h = threadIdx.x;
+    float mm = -INFINITY;
+    for (int s2 = 0; s2 < nsplit; ++s2) mm = fmaxf(mm, __ldcg(&part_ml[((row * nsplit + s2) * kHg + h) * 2]));
+    const float mu = mm == -INFINITY ? 0.f : mm;
+    float ls = 0.f;
+    for (int s2 = 0; s2 < nsplit; ++s2) {
+      const float* ml = part_ml + ((row * nsplit + s2) * kHg + h) * 2;
+      const float a = exp2f(__ldcg(&ml[0]) - mu);
+      fac[s2 * kHg + h] = a;
+      ls += a * __ldcg(&ml[1]);
+    }
+    inv[h] = 1.f / ls;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < kHg * kD; idx += kDecThreads) {
+    const int h = idx / kD;
+    const float* src = part_o + (row * nsplit) * kHg * kD + idx;
+    float acc = 0.f;
+    for (int s2 = 0; s2 < nsplit; ++s2) acc += fac[s2 * kHg + h] * __ldcg(src + static_cast<int64_t>(s2) * kHg * kD);
+    out[row * kHg * kD + idx] = __float2bfloat16_rn(acc * inv[h]);
+  }
+  if (threadIdx.x == 0) tickets[row] = 0;
 }
 
 }  // namespace sgqa

@@ -47,11 +47,13 @@ constexpr int kScoreCandPerCta = 1024;
 // Grid: x = query tiles of 64/H queries, y = candidate chunks of 1024,
 // z = seq * G + g.  Each warp takes 16-candidate strips; the 64 columns of the
 // B operand are (query, head) pairs of the tile.
-template <int H>
+// E4M3 = true: keys are the E4M3 store itself ([S, store_rows, 64] bytes),
+// widened to BF16 in registers (decode reads the store once, no BF16 copy).
+template <int H, bool E4M3>
 __global__ void __launch_bounds__(kScoreWarps * 32)
 index_score_kernel(const __nv_bfloat16* __restrict__ idx_q, const float* __restrict__ idx_w,
-                   const __nv_bfloat16* __restrict__ keys, float* __restrict__ scores,
-                   int64_t nq, int G, int64_t q_pos0, int B, int64_t rpad) {
+                   const void* __restrict__ keys_any, float* __restrict__ scores,
+                   int64_t nq, int G, int64_t q_pos0, int B, int64_t rpad, int64_t key_rows) {
   constexpr int QPC = 64 / H;  // queries per CTA tile
   constexpr int Di = 64;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -91,17 +93,33 @@ index_score_kernel(const __nv_bfloat16* __restrict__ idx_q, const float* __restr
     wv[j][0] = qok[j] ? wr[0] : 0.f;
     wv[j][1] = qok[j] ? wr[1] : 0.f;
   }
-  const __nv_bfloat16* kbase = keys + seq * rpad * Di;
   for (int64_t r0 = c0 + 16 * warp; r0 < c1; r0 += 16 * kScoreWarps) {
     uint32_t af[4][4];
-    const __nv_bfloat16* ra = kbase + (r0 + (lane >> 2)) * Di + 2 * (lane & 3);
-    const __nv_bfloat16* rb = ra + 8 * Di;
+    if constexpr (E4M3) {
+      // rows past the store's end read as zero (their scores are never selected)
+      const uint8_t* kb = static_cast<const uint8_t*>(keys_any) + seq * key_rows * Di;
+      const int64_t ra_row = r0 + (lane >> 2), rb_row = ra_row + 8;
+      const uint8_t* ra = kb + ra_row * Di + 2 * (lane & 3);
+      const uint8_t* rb = kb + rb_row * Di + 2 * (lane & 3);
+      const bool oka = ra_row < key_rows, okb = rb_row < key_rows;
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      af[s][0] = *reinterpret_cast<const uint32_t*>(ra + 16 * s);
-      af[s][1] = *reinterpret_cast<const uint32_t*>(rb + 16 * s);
-      af[s][2] = *reinterpret_cast<const uint32_t*>(ra + 16 * s + 8);
-      af[s][3] = *reinterpret_cast<const uint32_t*>(rb + 16 * s + 8);
+      for (int s = 0; s < 4; ++s) {
+        af[s][0] = oka ? e4m3x2_to_bf16x2(*reinterpret_cast<const uint16_t*>(ra + 16 * s)) : 0u;
+        af[s][1] = okb ? e4m3x2_to_bf16x2(*reinterpret_cast<const uint16_t*>(rb + 16 * s)) : 0u;
+        af[s][2] = oka ? e4m3x2_to_bf16x2(*reinterpret_cast<const uint16_t*>(ra + 16 * s + 8)) : 0u;
+        af[s][3] = okb ? e4m3x2_to_bf16x2(*reinterpret_cast<const uint16_t*>(rb + 16 * s + 8)) : 0u;
+      }
+    } else {
+      const __nv_bfloat16* kbase = static_cast<const __nv_bfloat16*>(keys_any) + seq * rpad * Di;
+      const __nv_bfloat16* ra = kbase + (r0 + (lane >> 2)) * Di + 2 * (lane & 3);
+      const __nv_bfloat16* rb = ra + 8 * Di;
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        af[s][0] = *reinterpret_cast<const uint32_t*>(ra + 16 * s);
+        af[s][1] = *reinterpret_cast<const uint32_t*>(rb + 16 * s);
+        af[s][2] = *reinterpret_cast<const uint32_t*>(ra + 16 * s + 8);
+        af[s][3] = *reinterpret_cast<const uint32_t*>(rb + 16 * s + 8);
+      }
     }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -155,11 +173,17 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int& total, int* warp
   return before;
 }
 
-// One CTA per (seq, query, group) row of scores.
+// One CTA per (seq, query, group) row of scores.  STAGE = true copies the row
+// into shared memory first (rows of up to kSelStageMax scores), so the radix
+// passes read SRAM instead of HBM.
+constexpr int kSelStageMax = 40960;
+
+template <bool STAGE>
 __global__ void __launch_bounds__(kSelThreads)
 topk_rows_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int G,
                  int64_t q_pos0, int B, int k, int32_t* __restrict__ sel,
                  int32_t* __restrict__ sel_count, const int32_t* __restrict__ only_if) {
+  extern __shared__ float staged_row[];
   __shared__ uint32_t hist[2048];
   __shared__ int warp_sums[32];
   __shared__ uint32_t s_prefix, s_rem;
@@ -171,6 +195,13 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int
   const float* srow = scores + row * rpad;
   int32_t* out = sel + row * k;
   const int tid = threadIdx.x;
+  if (STAGE && n > k) {
+    const float4* src4 = reinterpret_cast<const float4*>(srow);
+    float4* dst4 = reinterpret_cast<float4*>(staged_row);
+    for (int64_t j = tid; j < (n + 3) / 4; j += kSelThreads) dst4[j] = src4[j];
+    __syncthreads();
+    srow = staged_row;
+  }
   if (n <= k) {
     for (int j = tid; j < k; j += kSelThreads) out[j] = j < n ? j : -1;
     if (tid == 0) sel_count[row] = static_cast<int32_t>(n);
@@ -184,9 +215,14 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int
     const uint32_t nb = 1u << widths[p];
     for (uint32_t b = tid; b < 2048; b += kSelThreads) hist[b] = 0;
     __syncthreads();
-    for (int64_t j = tid; j < n; j += kSelThreads) {
-      const uint32_t key = score_key(srow[j]);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+    for (int64_t j0 = 0; j0 < n; j0 += kSelThreads) {
+      // lanes with equal bins add once: the keys share their top bits
+      const int64_t j = j0 + tid;
+      const uint32_t key = j < n ? score_key(srow[j]) : 0u;
+      const bool in = j < n && (key & mask) == prefix;
+      const uint32_t bin = in ? ((key >> shift) & (nb - 1)) : (4096u + (tid & 31));
+      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+      if (in && (peers & ((1u << (tid & 31)) - 1u)) == 0u) atomicAdd(&hist[bin], __popc(peers));
     }
     __syncthreads();
     // Find the bin, counted from the top, that holds the rem-th largest key.
@@ -237,6 +273,198 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int
     eq_seen += eq_total;
   }
   if (tid == 0) sel_count[row] = k;
+}
+
+}  // namespace sgqa
+
+namespace sgqa {
+
+// Decode scores: one CTA per (sequence, 128 candidates) scores that query's
+// four groups at once (B operand = 4 groups x 8 heads = 32 columns, resident in
+// registers), reading the E4M3 store directly; each warp takes 32 candidates.
+constexpr int kDecScoreWarps = 4;
+
+__global__ void __launch_bounds__(kDecScoreWarps * 32)
+index_score_decode_kernel(const __nv_bfloat16* __restrict__ idx_q, const float* __restrict__ idx_w,
+                          const uint8_t* __restrict__ store, float* __restrict__ scores, int64_t nq,
+                          int64_t q_pos0, int B, int64_t rpad, int64_t key_rows) {
+  constexpr int G = 4, H = 8, Di = 64;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t sq = blockIdx.y;  // seq * nq + i
+  const int64_t i = sq % nq, seq = sq / nq;
+  const int64_t ncand = (q_pos0 + i) / B;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 128 + 32 * warp;
+  if (c0 >= ncand) return;
+  // B fragments: column n = 8g + head (lane/4 within an n-tile)
+  uint32_t bf[G][4][2];
+  float wv[G][2];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const __nv_bfloat16* row = idx_q + ((sq * G + g) * H + (lane >> 2)) * Di;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int k0 = 16 * s + 2 * (lane & 3);
+      bf[g][s][0] = *reinterpret_cast<const uint32_t*>(row + k0);
+      bf[g][s][1] = *reinterpret_cast<const uint32_t*>(row + k0 + 8);
+    }
+    const float* wr = idx_w + (sq * G + g) * H + 2 * (lane & 3);
+    wv[g][0] = wr[0];
+    wv[g][1] = wr[1];
+  }
+  const uint8_t* kb = store + seq * key_rows * Di;
+#pragma unroll
+  for (int strip = 0; strip < 2; ++strip) {
+    const int64_t r0 = c0 + 16 * strip;
+    const int64_t ra_row = r0 + (lane >> 2), rb_row = ra_row + 8;
+    const bool oka = ra_row < key_rows, okb = rb_row < key_rows;
+    const uint8_t* ra = kb + ra_row * Di + 2 * (lane & 3);
+    const uint8_t* rb = kb + rb_row * Di + 2 * (lane & 3);
+    uint32_t af[4][4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      af[s][0] = oka ? e4m3x2_to_bf16x2(*reinterpret_cast<const uint16_t*>(ra + 16 * s)) : 0u;
+      af[s][1] = okb ? e4m3x2_to_bf16x2(*reinterpret_cast<const uint16_t*>(rb + 16 * s)) : 0u;
+      af[s][2] = oka ? e4m3x2_to_bf16x2(*reinterpret_cast<const uint16_t*>(ra + 16 * s + 8)) : 0u;
+      af[s][3] = okb ? e4m3x2_to_bf16x2(*reinterpret_cast<const uint16_t*>(rb + 16 * s + 8)) : 0u;
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < 4; ++s) mma_bf16_16816(acc, af[s], bf[g][s][0], bf[g][s][1]);
+      float pa = wv[g][0] * fmaxf(acc[0], 0.f) + wv[g][1] * fmaxf(acc[1], 0.f);
+      float pb = wv[g][0] * fmaxf(acc[2], 0.f) + wv[g][1] * fmaxf(acc[3], 0.f);
+      pa += __shfl_xor_sync(0xffffffffu, pa, 1);
+      pa += __shfl_xor_sync(0xffffffffu, pa, 2);
+      pb += __shfl_xor_sync(0xffffffffu, pb, 1);
+      pb += __shfl_xor_sync(0xffffffffu, pb, 2);
+      if ((lane & 3) == 0) {
+        float* srow = scores + (sq * G + g) * rpad;
+        srow[ra_row] = pa;
+        srow[rb_row] = pb;
+      }
+    }
+  }
+}
+
+// Exact top-k of rows of at most 32768 scores: 1024 threads hold 32 keys each
+// in registers; four 8-bit radix passes with a private histogram per warp
+// (no cross-warp contention on the few bins that clustered keys share); the
+// kept ids are marked in a bitmap and read out in id order (ascending).
+constexpr int kRegSelThreads = 1024;
+constexpr int kRegSelPer = 32;
+
+__global__ void __launch_bounds__(kRegSelThreads)
+topk_rows_reg_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int G, int64_t q_pos0, int B,
+                     int k, int32_t* __restrict__ sel, int32_t* __restrict__ sel_count) {
+  __shared__ uint32_t wh[32][256];
+  __shared__ uint32_t keep_bits[1024];
+  __shared__ uint32_t tie_bits[1024];
+  __shared__ int sums[32];
+  __shared__ uint32_t s_pick, s_rem;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t row = blockIdx.x;
+  const int64_t i = (row / G) % nq;
+  const int n = static_cast<int>((q_pos0 + i) / B);
+  const float* srow = scores + row * rpad;
+  int32_t* out = sel + row * k;
+  if (n <= k) {
+    for (int j = tid; j < k; j += kRegSelThreads) out[j] = j < n ? j : -1;
+    if (tid == 0) sel_count[row] = n;
+    return;
+  }
+  uint32_t key[kRegSelPer];
+#pragma unroll
+  for (int u = 0; u < kRegSelPer; ++u) {
+    const int j = tid + u * kRegSelThreads;
+    key[u] = j < n ? score_key(srow[j]) : 0u;  // 0 sorts below every real key
+  }
+  keep_bits[tid] = 0;
+  tie_bits[tid] = 0;
+  uint32_t prefix = 0, mask = 0, rem = static_cast<uint32_t>(k);
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = lane; b < 256; b += 32) wh[warp][b] = 0;
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < kRegSelPer; ++u) {
+      const bool in = (key[u] & mask) == prefix && (tid + u * kRegSelThreads) < n;
+      if (in) atomicAdd(&wh[warp][(key[u] >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    // bins from the top: thread b < 256 sums bin 255-b over the warps
+    uint32_t c = 0;
+    if (tid < 256) {
+      const int b = 255 - tid;
+#pragma unroll 8
+      for (int w = 0; w < 32; ++w) c += wh[w][b];
+    }
+    // inclusive scan over the 256 descending bins (8 warps)
+    uint32_t x = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) { uint32_t y = __shfl_up_sync(0xffffffffu, x, o); if (lane >= o) x += y; }
+    if (tid < 256 && lane == 31) sums[warp] = static_cast<int>(x);
+    __syncthreads();
+    if (tid < 256) {
+      uint32_t before = x - c;
+      for (int w = 0; w < warp; ++w) before += sums[w];
+      if (before < rem && rem <= before + c) { s_pick = 255 - tid; s_rem = rem - before; }
+    }
+    __syncthreads();
+    prefix |= s_pick << shift;
+    mask |= 255u << shift;
+    rem = s_rem;
+    __syncthreads();
+  }
+  const uint32_t theta = prefix;  // the k-th largest key; rem of its ties are kept
+#pragma unroll
+  for (int u = 0; u < kRegSelPer; ++u) {
+    const int j = tid + u * kRegSelThreads;
+    if (j < n && key[u] > theta) atomicOr(&keep_bits[j >> 5], 1u << (j & 31));
+    if (j < n && key[u] == theta) atomicOr(&tie_bits[j >> 5], 1u << (j & 31));
+  }
+  __syncthreads();
+  // ties in id order: thread w owns word w; keep the first rem tie bits overall
+  {
+    const uint32_t tb = tie_bits[tid];
+    uint32_t cnt = __popc(tb), x = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) { uint32_t y = __shfl_up_sync(0xffffffffu, x, o); if (lane >= o) x += y; }
+    if (lane == 31) sums[warp] = static_cast<int>(x);
+    __syncthreads();
+    uint32_t before = x - cnt;
+    for (int w = 0; w < warp; ++w) before += sums[w];
+    uint32_t take = tb;
+    if (before >= rem) take = 0;
+    else if (before + cnt > rem) {
+      uint32_t need = rem - before, t2 = 0, b = tb;
+      while (need--) { t2 |= b & (~b + 1u); b &= b - 1u; }
+      take = t2;
+    }
+    keep_bits[tid] |= take;
+    __syncthreads();
+  }
+  // read out in id order
+  const uint32_t kb = keep_bits[tid];
+  const uint32_t cnt = __popc(kb);
+  uint32_t x = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) { uint32_t y = __shfl_up_sync(0xffffffffu, x, o); if (lane >= o) x += y; }
+  __syncthreads();
+  if (lane == 31) sums[warp] = static_cast<int>(x);
+  __syncthreads();
+  uint32_t pos = x - cnt;
+  for (int w = 0; w < warp; ++w) pos += sums[w];
+  uint32_t b = kb;
+  while (b) {
+    const int t = __ffs(b) - 1;
+    b &= b - 1;
+    if (pos < static_cast<uint32_t>(k)) out[pos] = tid * 32 + t;
+    ++pos;
+  }
+  if (tid == kRegSelThreads - 1) {
+    sel_count[row] = k;
+    if (pos != static_cast<uint32_t>(k)) report(kDevBounds);
+  }
 }
 
 }  // namespace sgqa

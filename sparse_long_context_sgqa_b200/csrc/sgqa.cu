@@ -75,8 +75,12 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 // Queries per sequence below which attention runs split-K per query.
 constexpr int64_t kDecodeMaxNq = 32;
 
+// Split-K factor for decode attention: one wave of two CTAs per SM.  On the
+// 16 x 262144 decode workload this beat both two waves of shorter CTAs (their
+// fixed costs -- staging, first loads, cross-warp combine -- add up) and one
+// CTA per SM (four compute warps cannot keep an SM's share of HBM busy).
 int decode_splits(int64_t rows) {
-  int64_t s = (4 * 148 + rows - 1) / std::max<int64_t>(rows, 1);
+  int64_t s = (2 * 148) / std::max<int64_t>(rows, 1);
   return static_cast<int>(std::min<int64_t>(std::max<int64_t>(s, 1), 32));
 }
 
@@ -126,7 +130,7 @@ IndexWs index_ws(const sgqa_params* p, int64_t S, int64_t nq, int64_t max_ctx) {
 
 struct AttnWs {
   int nsplit;
-  size_t ids_off, mask_off, cnt_off, po_off, pml_off, bytes;
+  size_t ids_off, mask_off, cnt_off, po_off, pml_off, tick_off, bytes;
 };
 AttnWs attn_ws(const sgqa_params* p, int64_t S, int64_t nq) {
   AttnWs w{};
@@ -138,7 +142,9 @@ AttnWs attn_ws(const sgqa_params* p, int64_t S, int64_t nq) {
     size_t po = align256(static_cast<size_t>(rows * w.nsplit) * 16 * 192 * 4);
     w.pml_off = po;
     size_t pml = align256(static_cast<size_t>(rows * w.nsplit) * 16 * 2 * 4);
-    w.bytes = po + pml;
+    w.tick_off = po + pml;
+    size_t tick = align256(static_cast<size_t>(rows) * 4);
+    w.bytes = po + pml + tick;
   } else {
     const int64_t units = S * ((nq + 7) / 8) * G;
     const int64_t cap = 8 * static_cast<int64_t>(p->topk);
@@ -261,7 +267,7 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
   const IndexWs w = index_ws(p, S, nq, q0 + nq);
   const int64_t rneed = (q0 + nq - 1) / B;
   __nv_bfloat16* keys = ws_at<__nv_bfloat16>(ws, w.keys_off);
-  if (rneed > 0) {
+  if (rneed > 0 && nq > kDecodeMaxNq) {
     const int64_t threads = S * rneed * 8;
     sgqa::widen_store_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(
         store, cap / B, rneed, w.rpad, S, keys);
@@ -343,19 +349,34 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
           km, qm, idx_w, scores, nq, G, q0, B, w.rpad);
     }
     SGQA_LAUNCH_CHECK("index_score_tc_kernel");
+  } else if (rneed > 0 && G == 4 && H == 8) {
+    // few queries: one CTA per (query, 128 candidates) scores all four groups from the E4M3 store
+    dim3 grid(static_cast<unsigned>((rneed + 127) / 128), static_cast<unsigned>(S * nq));
+    sgqa::index_score_decode_kernel<<<grid, sgqa::kDecScoreWarps * 32, 0, st>>>(iq, idx_w, store, scores, nq, q0, B,
+                                                                                 w.rpad, cap / B);
+    SGQA_LAUNCH_CHECK("index_score_decode_kernel");
   } else if (rneed > 0) {
+    // few queries: warp-MMA scores straight from the E4M3 store
     const int qpc = 64 / H;
     dim3 grid(static_cast<unsigned>((nq + qpc - 1) / qpc),
               static_cast<unsigned>((rneed + sgqa::kScoreCandPerCta - 1) / sgqa::kScoreCandPerCta),
               static_cast<unsigned>(S * G));
     if (grid.y > 65535 || grid.z > 65535) return fail(SGQA_ERR_UNSUPPORTED, "index grid too large");
     if (H == 8)
-      sgqa::index_score_kernel<8><<<grid, sgqa::kScoreWarps * 32, 0, st>>>(iq, idx_w, keys, scores, nq, G, q0, B, w.rpad);
+      sgqa::index_score_kernel<8, true><<<grid, sgqa::kScoreWarps * 32, 0, st>>>(iq, idx_w, store, scores, nq, G,
+                                                                                  q0, B, w.rpad, cap / B);
     else
-      sgqa::index_score_kernel<4><<<grid, sgqa::kScoreWarps * 32, 0, st>>>(iq, idx_w, keys, scores, nq, G, q0, B, w.rpad);
+      sgqa::index_score_kernel<4, true><<<grid, sgqa::kScoreWarps * 32, 0, st>>>(iq, idx_w, store, scores, nq, G,
+                                                                                  q0, B, w.rpad, cap / B);
     SGQA_LAUNCH_CHECK("index_score_kernel");
   }
   const int64_t rows = S * nq * G;
+  if (nq <= kDecodeMaxNq && rneed <= sgqa::kRegSelThreads * sgqa::kRegSelPer) {
+    sgqa::topk_rows_reg_kernel<<<static_cast<unsigned>(rows), sgqa::kRegSelThreads, 0, st>>>(
+        scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count);
+    SGQA_LAUNCH_CHECK("topk_rows_reg_kernel");
+    return SGQA_OK;
+  }
   const int nwords = static_cast<int>((std::max<int64_t>(rneed, 1) + 31) / 32);
   const size_t ssmem = (static_cast<size_t>(sgqa::kRows2Bins) + 2 * sgqa::kRows2Cand + nwords) * 4;
   // The histogram + gather variant is opt-in (SGQA_TOPK_PATH=hist2); the
@@ -370,8 +391,15 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
   } else {
     flags = nullptr;  // too wide for the bitmap: the radix kernel takes every row
   }
-  sgqa::topk_rows_kernel<<<static_cast<unsigned>(rows), sgqa::kSelThreads, 0, st>>>(
-      scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, flags);
+  if (rneed <= sgqa::kSelStageMax) {
+    const size_t rsmem = static_cast<size_t>((rneed + 3) / 4 * 4) * 4;
+    cudaFuncSetAttribute(sgqa::topk_rows_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem);
+    sgqa::topk_rows_kernel<true><<<static_cast<unsigned>(rows), sgqa::kSelThreads, rsmem, st>>>(
+        scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, flags);
+  } else {
+    sgqa::topk_rows_kernel<false><<<static_cast<unsigned>(rows), sgqa::kSelThreads, 0, st>>>(
+        scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, flags);
+  }
   SGQA_LAUNCH_CHECK("topk_rows_kernel");
   return SGQA_OK;
 }
@@ -387,6 +415,28 @@ sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq,
   const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(kc);
   const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(vc);
   __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(out);
+  if (nq <= kDecodeMaxNq && B == 8) {
+    // TMA-fed gather; the last split of each row combines (tickets start at zero)
+    const int64_t rows = S * nq * G;
+    CUtensorMap km, vm;
+    cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(clen), 3, static_cast<cuuint64_t>(G), static_cast<cuuint64_t>(S)};
+    cuuint64_t strides[4] = {static_cast<cuuint64_t>(G) * 384, 128, 384, static_cast<cuuint64_t>(cap) * G * 384};
+    cuuint32_t box[5] = {64, 8, 3, 1, 1};
+    sgqa_status s;
+    if ((s = encode_bf16(&km, kc, 5, dims, strides, box, "k_cache")) != SGQA_OK) return s;
+    if ((s = encode_bf16(&vm, vc, 5, dims, strides, box, "v_cache")) != SGQA_OK) return s;
+    float* po = ws_at<float>(ws, w.po_off);
+    float* pml = ws_at<float>(ws, w.pml_off);
+    int32_t* tick = ws_at<int32_t>(ws, w.tick_off);
+    cudaError_t e = cudaMemsetAsync(tick, 0, static_cast<size_t>(rows) * 4, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(tickets)");
+    const size_t smem = sizeof(sgqa::DecSmem) + 1024;
+    cudaFuncSetAttribute(sgqa::attn_decode_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    sgqa::attn_decode_tma_kernel<<<static_cast<unsigned>(rows * w.nsplit), sgqa::kDecThreads, smem, st>>>(
+        km, vm, qb, sel, sel_count, po, pml, tick, ob, nq, G, k, q0, w.nsplit, scale_log2);
+    SGQA_LAUNCH_CHECK("attn_decode_tma_kernel");
+    return SGQA_OK;
+  }
   if (nq <= kDecodeMaxNq) {
     const int64_t rows = S * nq * G;
     const size_t smem = sgqa::kDecWarps * sgqa::kDecStages * 2 * sgqa::kStageElems * 2;
