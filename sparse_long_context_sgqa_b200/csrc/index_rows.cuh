@@ -215,14 +215,9 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int
     const uint32_t nb = 1u << widths[p];
     for (uint32_t b = tid; b < 2048; b += kSelThreads) hist[b] = 0;
     __syncthreads();
-    for (int64_t j0 = 0; j0 < n; j0 += kSelThreads) {
-      // lanes with equal bins add once: the keys share their top bits
-      const int64_t j = j0 + tid;
-      const uint32_t key = j < n ? score_key(srow[j]) : 0u;
-      const bool in = j < n && (key & mask) == prefix;
-      const uint32_t bin = in ? ((key >> shift) & (nb - 1)) : (4096u + (tid & 31));
-      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (in && (peers & ((1u << (tid & 31)) - 1u)) == 0u) atomicAdd(&hist[bin], __popc(peers));
+    for (int64_t j = tid; j < n; j += kSelThreads) {
+      const uint32_t key = score_key(srow[j]);
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
     }
     __syncthreads();
     // Find the bin, counted from the top, that holds the rem-th largest key.

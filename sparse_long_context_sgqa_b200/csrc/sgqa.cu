@@ -371,6 +371,8 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
     SGQA_LAUNCH_CHECK("index_score_kernel");
   }
   const int64_t rows = S * nq * G;
+  // few long rows (decode): the register-resident select; many rows (prefill):
+  // the 512-thread radix select, which keeps more rows in flight per SM
   if (nq <= kDecodeMaxNq && rneed <= sgqa::kRegSelThreads * sgqa::kRegSelPer) {
     sgqa::topk_rows_reg_kernel<<<static_cast<unsigned>(rows), sgqa::kRegSelThreads, 0, st>>>(
         scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count);
@@ -391,15 +393,8 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
   } else {
     flags = nullptr;  // too wide for the bitmap: the radix kernel takes every row
   }
-  if (rneed <= sgqa::kSelStageMax) {
-    const size_t rsmem = static_cast<size_t>((rneed + 3) / 4 * 4) * 4;
-    cudaFuncSetAttribute(sgqa::topk_rows_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem);
-    sgqa::topk_rows_kernel<true><<<static_cast<unsigned>(rows), sgqa::kSelThreads, rsmem, st>>>(
-        scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, flags);
-  } else {
-    sgqa::topk_rows_kernel<false><<<static_cast<unsigned>(rows), sgqa::kSelThreads, 0, st>>>(
-        scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, flags);
-  }
+  sgqa::topk_rows_kernel<false><<<static_cast<unsigned>(rows), sgqa::kSelThreads, 0, st>>>(
+      scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, flags);
   SGQA_LAUNCH_CHECK("topk_rows_kernel");
   return SGQA_OK;
 }
