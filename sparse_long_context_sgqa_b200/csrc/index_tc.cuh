@@ -57,15 +57,9 @@ __device__ __noinline__ void warp_select(const uint2* buf, int n, int k, uint32_
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int b = lane; b < 256; b += 32) hist[b] = 0;
     __syncwarp();
-    // lanes that hit the same bin add once (their count): keys share their top
-    // bits, so plain per-lane atomics would serialise on a few bins
-    for (int i0 = 0; i0 < n; i0 += 32) {
-      const int i = i0 + lane;
-      const uint32_t key = i < n ? buf[i].x : 0u;
-      const bool in = i < n && (key & mask) == prefix;
-      const uint32_t bin = in ? ((key >> shift) & 255u) : (256u + lane);
-      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (in && (peers & ((1u << lane) - 1u)) == 0u) atomicAdd(&hist[bin], __popc(peers));
+    for (int i = lane; i < n; i += 32) {
+      const uint32_t key = buf[i].x;
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
     }
     __syncwarp();
     uint32_t loc[8], sum = 0;
@@ -103,13 +97,9 @@ __device__ __noinline__ void warp_select(const uint2* buf, int n, int k, uint32_
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int b = lane; b < 256; b += 32) hist[b] = 0;
       __syncwarp();
-      for (int i0 = 0; i0 < n; i0 += 32) {
-        const int i = i0 + lane;
-        const uint2 e = i < n ? buf[i] : make_uint2(0u, 0u);
-        const bool in = i < n && e.x == theta && (e.y & imask) == ipre;
-        const uint32_t bin = in ? ((e.y >> shift) & 255u) : (256u + lane);
-        const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-        if (in && (peers & ((1u << lane) - 1u)) == 0u) atomicAdd(&hist[bin], __popc(peers));
+      for (int i = lane; i < n; i += 32) {
+        const uint2 e = buf[i];
+        if (e.x == theta && (e.y & imask) == ipre) atomicAdd(&hist[(e.y >> shift) & 255u], 1u);
       }
       __syncwarp();
       uint32_t loc[8], sum = 0;
@@ -530,27 +520,29 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
   }
 }
 
-// Exact top-k of materialised score rows in two passes over the row: a
-// 4096-bin histogram of the top 12 bits of the order-preserving key finds the
-// bin holding the k-th score; the second pass marks every entry of a higher
-// bin in a bitmap and gathers the boundary bin's (key, id) pairs, of which a
-// warp radix-selects the remainder (ties to the smaller id).  The bitmap is
-// read out in id order, so the output is ascending.  One CTA per row.  Rows
-// whose boundary bin exceeds the gather buffer report failure in `overflow`
-// (the caller then runs topk_rows_kernel on them).
+// Exact top-k of materialised score rows in two passes over the row.  Pass 1
+// counts the top 11 bits of every order-preserving key into a private
+// histogram per warp (two 16-bit counters per word: warps never contend);
+// their sum locates the bin holding the k-th score.  Pass 2 marks every
+// entry of a higher bin in a bitmap and gathers the boundary bin's (key, id)
+// pairs, of which one warp radix-selects the remainder (ties to the smaller
+// id).  The bitmap is read out in id order, so the output is ascending.  One
+// CTA per row; a row whose boundary bin overflows the gather buffer is flagged
+// in `overflow` for topk_rows_kernel.
 constexpr int kRows2Threads = 512;
-constexpr int kRows2Bins = 4096;
+constexpr int kRows2Warps = kRows2Threads / 32;
+constexpr int kRows2Bins = 2048;
 constexpr int kRows2Cand = 4096;
 
-__global__ void __launch_bounds__(kRows2Threads)
+__global__ void __launch_bounds__(kRows2Threads, 2)
 topk_rows2_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int G, int64_t q_pos0, int B,
                   int k, int nwords, int32_t* __restrict__ sel, int32_t* __restrict__ sel_count,
                   int32_t* __restrict__ overflow) {
   extern __shared__ uint32_t sm2[];
-  uint32_t* hist = sm2;                                   // [4096]
-  uint2* cand = reinterpret_cast<uint2*>(sm2 + kRows2Bins);  // [kRows2Cand]
-  uint32_t* bits = sm2 + kRows2Bins + 2 * kRows2Cand;     // [nwords]
-  __shared__ int warp_sums[kRows2Threads / 32];
+  uint32_t* wh = sm2;                                                     // [16][1024] packed u16 pairs
+  uint2* cand = reinterpret_cast<uint2*>(sm2 + kRows2Warps * kRows2Bins / 2);  // [kRows2Cand]
+  uint32_t* bits = sm2 + kRows2Warps * kRows2Bins / 2 + 2 * kRows2Cand;       // [nwords]
+  __shared__ int warp_sums[kRows2Warps];
   __shared__ uint32_t s_bin, s_rem, s_nc;
   const int64_t row = blockIdx.x;
   const int64_t i = (row / G) % nq;
@@ -563,34 +555,39 @@ topk_rows2_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, in
     if (tid == 0) { sel_count[row] = static_cast<int32_t>(n); overflow[row] = 0; }
     return;
   }
-  for (int b = tid; b < kRows2Bins; b += kRows2Threads) hist[b] = 0;
+  uint32_t* myh = wh + warp * (kRows2Bins / 2);
+  for (int b = lane; b < kRows2Bins / 2; b += 32) myh[b] = 0;
   const int nw = static_cast<int>((n + 31) / 32);
   for (int w = tid; w < nw; w += kRows2Threads) bits[w] = 0;
   if (tid == 0) s_nc = 0;
-  __syncthreads();
-  for (int64_t j0 = 0; j0 < n; j0 += kRows2Threads) {
-    const int64_t j = j0 + tid;
-    const bool in = j < n;
-    const uint32_t bin = in ? (score_key(srow[j]) >> 20) : (kRows2Bins + lane);
-    const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-    if (in && (peers & ((1u << lane) - 1u)) == 0u) atomicAdd(&hist[bin], __popc(peers));
+  __syncwarp();
+  for (int64_t j = tid; j < n; j += kRows2Threads) {
+    const uint32_t bin = score_key(srow[j]) >> 21;
+    atomicAdd(&myh[bin >> 1], 1u << (16 * (bin & 1)));
   }
   __syncthreads();
-  // bin holding the k-th largest, scanning from the top (8 bins per thread)
+  // 4 bins per thread, from the top
   {
-    uint32_t loc[8], sum = 0;
+    uint32_t loc[4], sum = 0;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) { loc[q] = hist[kRows2Bins - 1 - (tid * 8 + q)]; sum += loc[q]; }
+    for (int q = 0; q < 4; ++q) {
+      const int b = kRows2Bins - 1 - (tid * 4 + q);
+      uint32_t c = 0;
+#pragma unroll 4
+      for (int w = 0; w < kRows2Warps; ++w) c += (wh[w * (kRows2Bins / 2) + (b >> 1)] >> (16 * (b & 1))) & 0xFFFFu;
+      loc[q] = c;
+      sum += c;
+    }
     uint32_t x = sum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) { uint32_t y = __shfl_up_sync(0xffffffffu, x, o); if (lane >= o) x += y; }
     if (lane == 31) warp_sums[warp] = static_cast<int>(x);
     __syncthreads();
     if (warp == 0) {
-      int w = lane < kRows2Threads / 32 ? warp_sums[lane] : 0;
+      int w = lane < kRows2Warps ? warp_sums[lane] : 0;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) { int y = __shfl_up_sync(0xffffffffu, w, o); if (lane >= o) w += y; }
-      if (lane < kRows2Threads / 32) warp_sums[lane] = w;
+      if (lane < kRows2Warps) warp_sums[lane] = w;
     }
     __syncthreads();
     const uint32_t before = (warp > 0 ? warp_sums[warp - 1] : 0) + x - sum;
@@ -598,23 +595,31 @@ topk_rows2_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, in
     if (before < kk && kk <= before + sum) {
       uint32_t acc = before;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (acc < kk && kk <= acc + loc[q]) { s_bin = kRows2Bins - 1 - (tid * 8 + q); s_rem = kk - acc; }
+      for (int q = 0; q < 4; ++q) {
+        if (acc < kk && kk <= acc + loc[q]) { s_bin = kRows2Bins - 1 - (tid * 4 + q); s_rem = kk - acc; }
         acc += loc[q];
       }
     }
     __syncthreads();
   }
   const uint32_t bstar = s_bin, rem = s_rem;
-  // second pass: higher bins straight into the bitmap, boundary bin gathered
-  for (int64_t j = tid; j < n; j += kRows2Threads) {
-    const uint32_t key = score_key(srow[j]);
-    const uint32_t bin = key >> 20;
-    if (bin > bstar) {
-      atomicOr(&bits[j >> 5], 1u << (j & 31));
-    } else if (bin == bstar) {
-      const uint32_t pos = atomicAdd(&s_nc, 1u);
-      if (pos < kRows2Cand) cand[pos] = make_uint2(key, static_cast<uint32_t>(j));
+  // pass 2: higher bins into the bitmap, the boundary bin gathered (one atomic per warp)
+  for (int64_t j0 = 0; j0 < n; j0 += kRows2Threads) {
+    const int64_t j = j0 + tid;
+    uint32_t key = 0, bin = 0;
+    if (j < n) {
+      key = score_key(srow[j]);
+      bin = key >> 21;
+      if (bin > bstar) atomicOr(&bits[j >> 5], 1u << (j & 31));
+    }
+    const bool g2 = j < n && bin == bstar;
+    const uint32_t bal = __ballot_sync(0xffffffffu, g2);
+    if (bal) {
+      uint32_t base = 0;
+      if (lane == __ffs(bal) - 1) base = atomicAdd(&s_nc, __popc(bal));
+      base = __shfl_sync(0xffffffffu, base, __ffs(bal) - 1);
+      const uint32_t pos = base + __popc(bal & ((1u << lane) - 1u));
+      if (g2 && pos < kRows2Cand) cand[pos] = make_uint2(key, static_cast<uint32_t>(j));
     }
   }
   __syncthreads();
@@ -625,7 +630,7 @@ topk_rows2_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, in
   }
   if (warp == 0) {
     uint32_t theta = 0, id_cut = 0xFFFFFFFFu;
-    if (nc > rem) warp_select(cand, static_cast<int>(nc), static_cast<int>(rem), hist, theta, id_cut);
+    if (nc > rem) warp_select(cand, static_cast<int>(nc), static_cast<int>(rem), wh, theta, id_cut);
     for (uint32_t c = lane; c < nc; c += 32) {
       const uint2 e = cand[c];
       if (nc <= rem || kept(e, theta, id_cut)) atomicOr(&bits[e.y >> 5], 1u << (e.y & 31));
@@ -644,10 +649,10 @@ topk_rows2_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, in
   if (lane == 31) warp_sums[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int w = lane < kRows2Threads / 32 ? warp_sums[lane] : 0;
+    int w = lane < kRows2Warps ? warp_sums[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) { int y = __shfl_up_sync(0xffffffffu, w, o); if (lane >= o) w += y; }
-    if (lane < kRows2Threads / 32) warp_sums[lane] = w;
+    if (lane < kRows2Warps) warp_sums[lane] = w;
   }
   __syncthreads();
   int pos = (warp > 0 ? warp_sums[warp - 1] : 0) + x - local;

@@ -380,18 +380,18 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
     return SGQA_OK;
   }
   const int nwords = static_cast<int>((std::max<int64_t>(rneed, 1) + 31) / 32);
-  const size_t ssmem = (static_cast<size_t>(sgqa::kRows2Bins) + 2 * sgqa::kRows2Cand + nwords) * 4;
-  // The histogram + gather variant is opt-in (SGQA_TOPK_PATH=hist2); the
-  // three-pass radix select is the default.
-  const char* tp = getenv("SGQA_TOPK_PATH");
-  const bool hist2 = tp != nullptr && strcmp(tp, "hist2") == 0;
-  if (hist2 && ssmem <= 200 * 1024) {
+  const size_t ssmem = (static_cast<size_t>(sgqa::kRows2Warps) * sgqa::kRows2Bins / 2 + 2 * sgqa::kRows2Cand + nwords) * 4;
+  // Long rows (>= 32768 candidates): two passes over the row (histogram, then
+  // gather); rows it cannot finish (boundary-bin overflow) go to the radix
+  // kernel.  Shorter rows: the four-pass radix kernel, whose smaller per-row
+  // set-up wins there (measured at 8K and 128K contexts).
+  if (rneed >= 32768 && ssmem <= 112 * 1024) {
     cudaFuncSetAttribute(sgqa::topk_rows2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
     sgqa::topk_rows2_kernel<<<static_cast<unsigned>(rows), sgqa::kRows2Threads, ssmem, st>>>(
         scores, w.rpad, nq, G, q0, B, p->topk, nwords, sel, sel_count, flags);
     SGQA_LAUNCH_CHECK("topk_rows2_kernel");
   } else {
-    flags = nullptr;  // too wide for the bitmap: the radix kernel takes every row
+    flags = nullptr;  // the radix kernel takes every row
   }
   sgqa::topk_rows_kernel<false><<<static_cast<unsigned>(rows), sgqa::kSelThreads, 0, st>>>(
       scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, flags);
