@@ -18,7 +18,7 @@
 //   O += P V      4 tcgen05.mma (M128 N192 K16), V as an MN-major operand.
 // Warp roles: warp 0 issues TMA (one 5-D box per 8-token block gathers all
 // 192 dims of K or V: 3 KB), warp 1 allocates TMEM and issues the MMAs from
-// one thread, warps 2-5 run the softmax and the epilogue.  Every mbarrier
+// one thread, warps 2-9 run the softmax and the epilogue.  Every mbarrier
 // wait is bounded (tc::mbar_wait).
 #pragma once
 #include "attn_mma.cuh"
@@ -26,19 +26,21 @@
 
 namespace sgqa {
 
-constexpr int kTcStages = 3;      // K ring and V ring depth (K freed after QK^T, V after PV)
-constexpr int kTcThreads = 192;
+constexpr int kTcStages = 3;      // K ring depth (K freed after QK^T)
+constexpr int kTcVStages = 2;     // V ring depth (V freed after PV)
+constexpr int kTcThreads = 320;  // producer, MMA, 8 softmax warps
 constexpr int kTcTileTok = 64;    // tokens per KV tile = 8 blocks of 8
 
 struct __align__(1024) AttnTcSmem {
   uint8_t q[3][128 * 128];                 // Q: 3 column chunks x 128 rows x 128 B (SW128)
   uint8_t k[kTcStages][8][3][1024];        // K tile: [block][chunk][8 rows x 128 B]
-  uint8_t v[kTcStages][8][3][1024];        // V tile, same layout (MN-major operand)
+  uint8_t v[kTcVStages][8][3][1024];       // V tile, same layout (MN-major operand)
   uint8_t p[2][128 * 128];                 // P: 128 rows x 64 tokens bf16 (SW128)
   uint64_t q_full;
-  uint64_t k_full[kTcStages], k_empty[kTcStages], v_full[kTcStages], v_empty[kTcStages];
+  uint64_t k_full[kTcStages], k_empty[kTcStages], v_full[kTcVStages], v_empty[kTcVStages];
   uint64_t s_full[3], s_free[3], p_full[2], p_empty[2];
   uint64_t o_done, o_final, drain;
+  float pmax[2][2][128];                   // row maxima of each half, by tile parity
   uint32_t tmem;
   int abort;
 };
@@ -78,15 +80,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     for (int s = 0; s < kTcStages; ++s) {
       tc::mbar_init(bar(sm.k_full[s]), 1);
       tc::mbar_init(bar(sm.k_empty[s]), 1);
+    }
+    for (int s = 0; s < kTcVStages; ++s) {
       tc::mbar_init(bar(sm.v_full[s]), 1);
       tc::mbar_init(bar(sm.v_empty[s]), 1);
     }
     for (int b = 0; b < 3; ++b) {
       tc::mbar_init(bar(sm.s_full[b]), 1);
-      tc::mbar_init(bar(sm.s_free[b]), 128);
+      tc::mbar_init(bar(sm.s_free[b]), 256);
     }
     for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(bar(sm.p_full[b]), 128);
+      tc::mbar_init(bar(sm.p_full[b]), 256);
       tc::mbar_init(bar(sm.p_empty[b]), 1);
     }
     tc::mbar_init(bar(sm.o_done), 1);
@@ -102,24 +106,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   const uint32_t tS0 = tmem + 256;    // S buffers at [256, 320), [320, 384), [384, 448)
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tc::prefetch_tmap(&qmap);
-      tc::prefetch_tmap(&kmap);
-      tc::prefetch_tmap(&vmap);
-      tc::mbar_expect_tx(bar(sm.q_full), 3 * 128 * 128);
-      const int32_t qrow0 = static_cast<int32_t>(((seq * nq + qb * 8) * G + g) * 16);
-      const int32_t qstride = G * 16;
-      for (int c = 0; c < 3; ++c)
-        for (int i = 0; i < 8; ++i)
-          tc::tma_load_2d(smem_u32(&sm.q[c][i * 16 * 128]), &qmap, 64 * c, qrow0 + i * qstride, bar(sm.q_full));
-      int issued = 0;
-      // block ids of the next union tile, fetched one tile ahead
+    // ------------------------------------------------------------ producers
+    // lane 0 streams Q and K, lane 1 streams V: the rings drain at different
+    // points (K after QK^T, V after PV), so each gets its own issuer.
+    if (lane < 2) {
+      const bool is_k = lane == 0;
+      const int nst = is_k ? kTcStages : kTcVStages;
+      if (is_k) {
+        tc::prefetch_tmap(&qmap);
+        tc::prefetch_tmap(&kmap);
+        tc::mbar_expect_tx(bar(sm.q_full), 3 * 128 * 128);
+        const int32_t qrow0 = static_cast<int32_t>(((seq * nq + qb * 8) * G + g) * 16);
+        const int32_t qstride = G * 16;
+        for (int c = 0; c < 3; ++c)
+          for (int i = 0; i < 8; ++i)
+            tc::tma_load_2d(smem_u32(&sm.q[c][i * 16 * 128]), &qmap, 64 * c, qrow0 + i * qstride, bar(sm.q_full));
+      } else {
+        tc::prefetch_tmap(&vmap);
+      }
+      // block ids of upcoming union tiles, fetched two tiles ahead
       auto tile_rows = [&](int j, int32_t (&rows)[8]) {
         if (j < n_union_tiles) {
-          const int4 a = *reinterpret_cast<const int4*>(uid + 8 * j);
-          const int4 b = *reinterpret_cast<const int4*>(uid + 8 * j + 4);
-          const int32_t ids[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+          const int4 a4 = *reinterpret_cast<const int4*>(uid + 8 * j);
+          const int4 b4 = *reinterpret_cast<const int4*>(uid + 8 * j + 4);
+          const int32_t ids[8] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
           for (int e = 0; e < 8; ++e) rows[e] = (8 * j + e < U) ? ids[e] * 8 : -64;
         } else {
@@ -131,23 +141,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       int32_t rows[8], next[8];
       tile_rows(0, rows);
       if (n_tiles > 1) tile_rows(1, next);
+      int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % kTcStages;
-        const uint32_t ph = ((j / kTcStages) - 1) & 1;
+        const int s = j % nst;
         int32_t next2[8];
         if (j + 2 < n_tiles) tile_rows(j + 2, next2);
-        if (j >= kTcStages && !tc::mbar_wait(bar(sm.k_empty[s]), ph, abort)) break;
-        tc::mbar_expect_tx(bar(sm.k_full[s]), 8 * 3 * 1024);
+        uint64_t* empty = is_k ? &sm.k_empty[s] : &sm.v_empty[s];
+        uint64_t* full = is_k ? &sm.k_full[s] : &sm.v_full[s];
+        if (j >= nst && !tc::mbar_wait(bar(*empty), ((j / nst) - 1) & 1, abort)) break;
+        tc::mbar_expect_tx(bar(*full), 8 * 3 * 1024);
+        const CUtensorMap* map = is_k ? &kmap : &vmap;
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          tc::tma_load_5d(smem_u32(&sm.k[s][e][0][0]), &kmap, 0, rows[e], 0, g, static_cast<int32_t>(seq),
-                          bar(sm.k_full[s]));
-        if (j >= kTcStages && !tc::mbar_wait(bar(sm.v_empty[s]), ph, abort)) { issued = -(j + 1); break; }
-        tc::mbar_expect_tx(bar(sm.v_full[s]), 8 * 3 * 1024);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          tc::tma_load_5d(smem_u32(&sm.v[s][e][0][0]), &vmap, 0, rows[e], 0, g, static_cast<int32_t>(seq),
-                          bar(sm.v_full[s]));
+        for (int e = 0; e < 8; ++e) {
+          const uint32_t dst = is_k ? smem_u32(&sm.k[s][e][0][0]) : smem_u32(&sm.v[s][e][0][0]);
+          tc::tma_load_5d(dst, map, 0, rows[e], 0, g, static_cast<int32_t>(seq), bar(*full));
+        }
         issued = j + 1;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -157,19 +165,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       }
       if (*abort) {
         // Let the copies already issued land before the CTA's shared memory goes away.
-        const bool k_only = issued < 0;
-        const int n_iss = k_only ? -issued : issued;
         const uint64_t t0 = globaltimer_ns();
-        while (!tc::mbar_try(bar(sm.q_full), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-        }
-        for (int j = n_iss > kTcStages ? n_iss - kTcStages : 0; j < n_iss; ++j) {
-          const uint64_t t1 = globaltimer_ns();
-          while (!tc::mbar_try(bar(sm.k_full[j % kTcStages]), (j / kTcStages) & 1) &&
-                 globaltimer_ns() - t1 < kWaitLimitNs) {
+        if (is_k)
+          while (!tc::mbar_try(bar(sm.q_full), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
           }
-          if (k_only && j == n_iss - 1) break;
-          while (!tc::mbar_try(bar(sm.v_full[j % kTcStages]), (j / kTcStages) & 1) &&
-                 globaltimer_ns() - t1 < kWaitLimitNs) {
+        for (int j = issued > nst ? issued - nst : 0; j < issued; ++j) {
+          const uint64_t t1 = globaltimer_ns();
+          uint64_t* full = is_k ? &sm.k_full[j % nst] : &sm.v_full[j % nst];
+          while (!tc::mbar_try(bar(*full), (j / nst) & 1) && globaltimer_ns() - t1 < kWaitLimitNs) {
           }
         }
       }
@@ -180,8 +183,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       const uint32_t id_qk = tc::idesc_bf16(128, 64, false);
       const uint32_t id_pv = tc::idesc_bf16(128, 192, true);
       auto pv = [&](int i) -> bool {
-        const int pb = i & 1, s = i % kTcStages;
-        if (!tc::mbar_wait(bar(sm.v_full[s]), (i / kTcStages) & 1, abort)) return false;
+        const int pb = i & 1, s = i % kTcVStages;
+        if (!tc::mbar_wait(bar(sm.v_full[s]), (i / kTcVStages) & 1, abort)) return false;
         if (!tc::mbar_wait(bar(sm.p_full[pb]), (i >> 1) & 1, abort)) return false;
         tc::fence_after();
 #pragma unroll
@@ -226,7 +229,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    // Eight warps, two per TMEM lane quadrant: both own the same 32 rows and
+    // split each tile's 64 tokens (and O's 192 columns) in halves, exchanging
+    // the row maxima through shared memory, so two warps per SM sub-partition
+    // hide each other's latency.  A failed wait clears `ok` but keeps the pair
+    // in step (every pair barrier is still reached).
+    const int sw = warp - 2;                 // 0..7
     const int quad = warp & 3;
+    const int half = sw >> 2;                // tokens [32 half, 32 half + 32)
+    const int pair_bar = 1 + quad;           // named barrier of the two warps of this quadrant
     const int m = quad * 32 + lane;          // TMEM lane = row = (query slot, head)
     const int qs = m >> 4;
     const int64_t qi = qb * 8 + qs;
@@ -236,54 +247,56 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    uint2 mb_next = n_union_tiles > 0 ? *reinterpret_cast<const uint2*>(umask) : make_uint2(0, 0);
+    uint32_t mb_next = n_union_tiles > 0 ? *reinterpret_cast<const uint32_t*>(umask + 4 * half) : 0u;
     for (int j = 0; j < n_tiles; ++j) {
       const int sb = j % 3, pb = j & 1;
-      const uint2 mb = mb_next;
-      if (j + 1 < n_union_tiles) mb_next = *reinterpret_cast<const uint2*>(umask + 8 * (j + 1));
-      // which of the 64 tokens this row attends
-      uint64_t tok_mask = 0;
+      const uint32_t mb = mb_next;
+      if (j + 1 < n_union_tiles) mb_next = *reinterpret_cast<const uint32_t*>(umask + 8 * (j + 1) + 4 * half);
+      // which of this half's 32 tokens the row attends
+      uint32_t tok_mask = 0;
       if (j < n_union_tiles) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint32_t byte = ((e < 4 ? mb.x : mb.y) >> (8 * (e & 3))) & 0xFFu;
-          if (8 * j + e < U && ((byte >> qs) & 1u)) tok_mask |= 0xFFull << (8 * e);
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t byte = (mb >> (8 * e)) & 0xFFu;
+          if (8 * j + 4 * half + e < U && ((byte >> qs) & 1u)) tok_mask |= 0xFFu << (8 * e);
         }
-      } else {
+      } else if (half == 0) {
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
           const int64_t tok = c0 + jj;
-          if (tok >= cur_lo && tok <= t) tok_mask |= 1ull << jj;
+          if (tok >= cur_lo && tok <= t) tok_mask |= 1u << jj;
         }
       }
-      if (!tc::mbar_wait(bar(sm.s_full[sb]), (j / 3) & 1, abort)) { ok = false; break; }
+      ok = ok && tc::mbar_wait(bar(sm.s_full[sb]), (j / 3) & 1, abort);
       tc::fence_after();
-      uint32_t sr[64];
-      tc::tmem_ld32(tS0 + 64 * sb + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tc::tmem_ld32(tS0 + 64 * sb + 32 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      uint32_t sr[32];
+      tc::tmem_ld32(tS0 + 64 * sb + 32 * half + lane_off, sr);
       tc::tmem_ld_wait();
       tc::fence_before();
       tc::mbar_arrive(bar(sm.s_free[sb]));
-      // masked scores (raw), their max; the scale is positive so it commutes with max
+      // masked raw scores and this half's max (the scale is positive: it commutes with max)
       float mraw = -INFINITY;
 #pragma unroll
-      for (int jj = 0; jj < 64; ++jj) {
-        const float x = ((tok_mask >> jj) & 1ull) ? __uint_as_float(sr[jj]) : -INFINITY;
+      for (int jj = 0; jj < 32; ++jj) {
+        const float x = ((tok_mask >> jj) & 1u) ? __uint_as_float(sr[jj]) : -INFINITY;
         sr[jj] = __float_as_uint(x);
         mraw = fmaxf(mraw, x);
       }
+      sm.pmax[pb][half][m] = mraw;
+      asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+      mraw = fmaxf(mraw, sm.pmax[pb][half ^ 1][m]);
       const float mt = mraw * scale_log2;
       const float m_new = fmaxf(m_used, mt);
       const bool need = (m_used != -INFINITY) && (m_new > m_used + 8.0f);
       if (m_used == -INFINITY) m_used = m_new;
       // P buffer pb is free once PV(j-2) has completed
-      if (j >= 2 && !tc::mbar_wait(bar(sm.p_empty[pb]), ((j >> 1) - 1) & 1, abort)) { ok = false; break; }
+      if (j >= 2) ok = ok && tc::mbar_wait(bar(sm.p_empty[pb]), ((j >> 1) - 1) & 1, abort);
       if (__any_sync(0xffffffffu, need)) {
-        if (j >= 1 && !tc::mbar_wait(bar(sm.o_done), (j - 1) & 1, abort)) { ok = false; break; }
+        if (j >= 1) ok = ok && tc::mbar_wait(bar(sm.o_done), (j - 1) & 1, abort);
         tc::fence_after();
         const float alpha = need ? exp2f(m_used - m_new) : 1.f;
 #pragma unroll 1
-        for (int h = 0; h < 6; ++h) {
+        for (int h = 3 * half; h < 3 * half + 3; ++h) {
           uint32_t o[32];
           tc::tmem_ld32(tO + lane_off + 32 * h, o);
           tc::tmem_ld_wait();
@@ -297,16 +310,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           m_used = m_new;
         }
       }
-      // P = 2^(s * scale - m_used) in BF16 (masked -> exp2(-inf) = 0)
+      // P = 2^(s * scale - m_used) in BF16 (masked -> exp2(-inf) = 0), 4 chunks of 8 tokens
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
       uint8_t* prow = &sm.p[pb][0];
       float lsum = 0.f;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int cc = 0; cc < 4; ++cc) {
         float pv8[8];
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
-          pv8[x] = exp2f(fmaf(__uint_as_float(sr[8 * c + x]), scale_log2, neg_m));
+          pv8[x] = exp2f(fmaf(__uint_as_float(sr[8 * cc + x]), scale_log2, neg_m));
           lsum += pv8[x];
         }
         uint4 w;
@@ -314,19 +327,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         w.y = pack_bf16x2(pv8[2], pv8[3]);
         w.z = pack_bf16x2(pv8[4], pv8[5]);
         w.w = pack_bf16x2(pv8[6], pv8[7]);
-        *reinterpret_cast<uint4*>(prow + tc::sw128_offset(static_cast<uint32_t>(m), static_cast<uint32_t>(c))) = w;
+        *reinterpret_cast<uint4*>(prow + tc::sw128_offset(static_cast<uint32_t>(m), static_cast<uint32_t>(4 * half + cc))) = w;
       }
       l += lsum;
       tc::fence_proxy_async_smem();
       tc::fence_before();
       tc::mbar_arrive(bar(sm.p_full[pb]));
     }
-    if (ok && tc::mbar_wait(bar(sm.o_final), 0, abort)) {
+    ok = ok && tc::mbar_wait(bar(sm.o_final), 0, abort);
+    // full row sum from both halves (the parity slot the last tile did not use)
+    sm.pmax[n_tiles & 1][half][m] = l;
+    asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+    const float ltot = l + sm.pmax[n_tiles & 1][half ^ 1][m];
+    if (ok) {
       tc::fence_after();
-      const float inv = 1.f / l;
+      const float inv = 1.f / ltot;
       __nv_bfloat16* orow = out + (((seq * nq + (qvalid ? qi : 0)) * G + g) * kHg + (m & 15)) * kD;
 #pragma unroll 1
-      for (int h = 0; h < 6; ++h) {
+      for (int h = 3 * half; h < 3 * half + 3; ++h) {
         uint32_t o[32];
         tc::tmem_ld32(tO + lane_off + 32 * h, o);
         tc::tmem_ld_wait();

@@ -32,12 +32,19 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 // Wait for the phase with the given parity to complete; gives up after
 // kWaitLimitNs, records kDevTimeout and returns false.  `abort` (shared)
 // short-cuts every later wait of the CTA once one has given up.
+// A wait also gives up at once when any CTA of any kernel has already
+// recorded a failure (device status word set), so a broken launch ends after
+// one bounded wait instead of one per CTA.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (true) {
+  for (uint32_t it = 0;; ++it) {
     if (mbar_try(bar, parity)) return true;
     if (*abort) return false;
+    if ((it & 1023u) == 1023u && *reinterpret_cast<volatile int*>(&g_status) != 0) {
+      *abort = 1;
+      return false;
+    }
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       *abort = 1;
       report(kDevTimeout);
