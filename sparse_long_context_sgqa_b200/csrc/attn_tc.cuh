@@ -37,9 +37,10 @@ struct __align__(1024) AttnTcSmem {
   uint8_t v[kTcVStages][8][3][1024];       // V tile, same layout (MN-major operand)
   uint8_t p[2][128 * 128];                 // P: 128 rows x 64 tokens bf16 (SW128)
   uint64_t q_full;
-  uint64_t k_full[kTcStages], k_empty[kTcStages], v_full[kTcVStages], v_empty[kTcVStages];
-  uint64_t s_full[3], s_free[3], p_full[2], p_empty[2];
-  uint64_t o_done, o_final, drain;
+  uint64_t k_full[kTcStages], k_empty[kTcStages], v_full[kTcVStages];
+  uint64_t s_full[3], s_free[3], p_full[2];
+  uint64_t pv_done[2];                     // PV(i) complete: V stage, P buffer and O free (i % 2)
+  uint64_t o_final, drain;
   float pmax[2][2][128];                   // row maxima of each half, by tile parity
   uint32_t tmem;
   int abort;
@@ -81,19 +82,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       tc::mbar_init(bar(sm.k_full[s]), 1);
       tc::mbar_init(bar(sm.k_empty[s]), 1);
     }
-    for (int s = 0; s < kTcVStages; ++s) {
-      tc::mbar_init(bar(sm.v_full[s]), 1);
-      tc::mbar_init(bar(sm.v_empty[s]), 1);
-    }
+    for (int s = 0; s < kTcVStages; ++s) tc::mbar_init(bar(sm.v_full[s]), 1);
     for (int b = 0; b < 3; ++b) {
       tc::mbar_init(bar(sm.s_full[b]), 1);
       tc::mbar_init(bar(sm.s_free[b]), 256);
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(bar(sm.p_full[b]), 256);
-      tc::mbar_init(bar(sm.p_empty[b]), 1);
+      tc::mbar_init(bar(sm.pv_done[b]), 1);
     }
-    tc::mbar_init(bar(sm.o_done), 1);
     tc::mbar_init(bar(sm.o_final), 1);
     tc::mbar_init(bar(sm.drain), 1);
     tc::mbar_fence_init();
@@ -146,7 +143,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         const int s = j % nst;
         int32_t next2[8];
         if (j + 2 < n_tiles) tile_rows(j + 2, next2);
-        uint64_t* empty = is_k ? &sm.k_empty[s] : &sm.v_empty[s];
+        uint64_t* empty = is_k ? &sm.k_empty[s] : &sm.pv_done[s];
         uint64_t* full = is_k ? &sm.k_full[s] : &sm.v_full[s];
         if (j >= nst && !tc::mbar_wait(bar(*empty), ((j / nst) - 1) & 1, abort)) break;
         tc::mbar_expect_tx(bar(*full), 8 * 3 * 1024);
@@ -182,20 +179,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     if (lane == 0) {
       const uint32_t id_qk = tc::idesc_bf16(128, 64, false);
       const uint32_t id_pv = tc::idesc_bf16(128, 192, true);
+      // Base descriptors once per unit; each MMA adds a constant offset (in
+      // 16-byte units, the descriptor's address field) to one of them.
+      const uint64_t dq = tc::sdesc_sw128(smem_u32(&sm.q[0][0]), 16, 1024);
+      // stages are contiguous: stage x starts x * 24 KB (1536 units) after stage 0; P buffers 16 KB apart
+      const uint64_t dk0 = tc::sdesc_sw128(smem_u32(&sm.k[0][0][0][0]), 16, 3072);
+      const uint64_t dv0 = tc::sdesc_sw128(smem_u32(&sm.v[0][0][0][0]), 1024, 3072);
+      const uint64_t dp0 = tc::sdesc_sw128(smem_u32(&sm.p[0][0]), 16, 1024);
       auto pv = [&](int i) -> bool {
         const int pb = i & 1, s = i % kTcVStages;
         if (!tc::mbar_wait(bar(sm.v_full[s]), (i / kTcVStages) & 1, abort)) return false;
         if (!tc::mbar_wait(bar(sm.p_full[pb]), (i >> 1) & 1, abort)) return false;
         tc::fence_after();
+        const uint64_t a0 = dp0 + 1024 * pb, b0 = dv0 + 1536 * s;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t a = tc::sdesc_sw128(smem_u32(&sm.p[pb][0]) + kk * 32, 16, 1024);
-          const uint64_t b = tc::sdesc_sw128(smem_u32(&sm.v[s][2 * kk][0][0]), 1024, 3072);
-          tc::mma_f16(tO, a, b, id_pv, (i > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc::mma_commit(bar(sm.v_empty[s]));
-        tc::mma_commit(bar(sm.p_empty[pb]));
-        tc::mma_commit(bar(sm.o_done));
+        for (int kk = 0; kk < 4; ++kk)  // P: +32 B per 16 tokens; V: +2 blocks (6144 B)
+          tc::mma_f16(tO, a0 + 2 * kk, b0 + 384 * kk, id_pv, (i > 0 || kk > 0) ? 1u : 0u);
+        tc::mma_commit(bar(sm.pv_done[pb]));
         return true;
       };
       bool ok = tc::mbar_wait(bar(sm.q_full), 0, abort);
@@ -206,12 +206,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         if (!tc::mbar_wait(bar(sm.k_full[s]), (j / kTcStages) & 1, abort)) { ok = false; break; }
         if (j >= 3 && !tc::mbar_wait(bar(sm.s_free[sb]), ((j / 3) - 1) & 1, abort)) { ok = false; break; }
         tc::fence_after();
+        const uint64_t b0 = dk0 + 1536 * s;
 #pragma unroll
-        for (int kk = 0; kk < 12; ++kk) {
-          const uint64_t a = tc::sdesc_sw128(smem_u32(&sm.q[kk >> 2][0]) + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = tc::sdesc_sw128(smem_u32(&sm.k[s][0][kk >> 2][0]) + (kk & 3) * 32, 16, 3072);
-          tc::mma_f16(tS0 + 64 * sb, a, b, id_qk, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 12; ++kk)  // Q: +16 KB per 64 dims, +32 B per 16; K: +1 KB per 64 dims
+          tc::mma_f16(tS0 + 64 * sb, dq + (kk >> 2) * 1024 + (kk & 3) * 2, b0 + (kk >> 2) * 64 + (kk & 3) * 2,
+                      id_qk, kk > 0 ? 1u : 0u);
         tc::mma_commit(bar(sm.k_empty[s]));
         tc::mma_commit(bar(sm.s_full[sb]));
         if (j >= 2 && !pv(j - 2)) { ok = false; break; }
@@ -290,9 +289,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       const bool need = (m_used != -INFINITY) && (m_new > m_used + 8.0f);
       if (m_used == -INFINITY) m_used = m_new;
       // P buffer pb is free once PV(j-2) has completed
-      if (j >= 2) ok = ok && tc::mbar_wait(bar(sm.p_empty[pb]), ((j >> 1) - 1) & 1, abort);
+      if (j >= 2) ok = ok && tc::mbar_wait(bar(sm.pv_done[pb]), ((j >> 1) - 1) & 1, abort);
       if (__any_sync(0xffffffffu, need)) {
-        if (j >= 1) ok = ok && tc::mbar_wait(bar(sm.o_done), (j - 1) & 1, abort);
+        // O must hold PV(j-1): pv_done[(j-1)&1] completes for the ((j-1)/2)-th time
+        if (j >= 1) ok = ok && tc::mbar_wait(bar(sm.pv_done[(j - 1) & 1]), ((j - 1) >> 1) & 1, abort);
         tc::fence_after();
         const float alpha = need ? exp2f(m_used - m_new) : 1.f;
 #pragma unroll 1
