@@ -8,46 +8,58 @@
 // The MMA M dimension is the 8 queries x 16 heads = 128 rows, all sharing the
 // group's K/V; the unit walks the sorted union of the 8 queries' selected
 // 8-token blocks (built by attn_plan_kernel) 64 tokens (8 blocks) at a time,
-// then one tile holding the current-block tokens.  Per 64-token tile:
-//   S = Q K^T     12 tcgen05.mma (M128 N64 K16) into TMEM, Q and K from SMEM
-//   softmax       4 warps, one TMEM lane (= one (query, head) row) per thread:
-//                 per-row block mask (the row's query must have selected the
-//                 block) and causal mask on the current block, running max
-//                 in log2 units with lazy rescaling of O (only when the max
-//                 grows by more than 2^8), P rounded to BF16 into SMEM
-//   O += P V      4 tcgen05.mma (M128 N192 K16), V as an MN-major operand.
-// Warp roles: warp 0 issues TMA (one 5-D box per 8-token block gathers all
-// 192 dims of K or V: 3 KB), warp 1 allocates TMEM and issues the MMAs from
-// one thread, warps 2-9 run the softmax and the epilogue.  Every mbarrier
-// wait is bounded (tc::mbar_wait).
+// then one tile holding the current-block tokens.
+//
+// Tensor memory (512 columns, one row per TMEM lane):
+//   [0, 192)    O accumulator, FP32
+//   [192, 384)  three S buffers of 64 FP32 columns; the softmax overwrites the
+//               first 32 columns of a buffer with its P (two BF16 per column)
+//   [384, 480)  Q, two BF16 per column, written once per unit by the softmax warps
+// Per 64-token tile j (buffer b = j % 3):
+//   S = Q K^T   12 tcgen05.mma (M128 N64 K16), A = Q from TMEM, B = K (SMEM, K-major)
+//   softmax     per-row block mask (the row's query must have selected the
+//               block) and causal mask on the current block, running max in
+//               log2 units with lazy rescaling of O (only when the max grows
+//               by more than 2^8), P rounded to BF16 and stored over S
+//   O += P V    4 tcgen05.mma (M128 N192 K16), A = P from TMEM, B = V (SMEM, MN-major)
+// The MMA thread issues S(j+1) before O += P(j) V(j), so the tensor pipe
+// computes the next scores while the softmax works on the current ones; the
+// softmax waits on an O update only for the (rare) rescale.
+// Warp roles: warp 0 streams K and warp 10 streams V by TMA (one 5-D box per
+// 8-token block gathers all 192 dims: 3 KB), warp 1 allocates TMEM and issues
+// the MMAs, warps 2-9 run the softmax and the epilogue.  The producer and MMA
+// warps run converged and hand each TMA or MMA batch to one elected lane:
+// issuing from a lone divergent lane costs the tensor pipe several hundred
+// cycles per tile in synchronisation stalls.  Every mbarrier wait is bounded
+// (tc::mbar_wait / tc::warp_wait).
 #pragma once
 #include "attn_mma.cuh"
 #include "tc.cuh"
 
 namespace sgqa {
 
-constexpr int kTcStages = 3;      // K ring depth (K freed after QK^T)
-constexpr int kTcVStages = 2;     // V ring depth (V freed after PV)
-constexpr int kTcThreads = 320;  // producer, MMA, 8 softmax warps
+constexpr int kTcStages = 4;      // K ring depth (K freed after QK^T)
+constexpr int kTcVStages = 4;     // V ring depth (V freed after PV)
+constexpr int kTcThreads = 352;   // K producer, MMA, 8 softmax warps, V producer
 constexpr int kTcTileTok = 64;    // tokens per KV tile = 8 blocks of 8
 
 struct __align__(1024) AttnTcSmem {
-  uint8_t q[3][128 * 128];                 // Q: 3 column chunks x 128 rows x 128 B (SW128)
-  uint8_t k[kTcStages][8][3][1024];        // K tile: [block][chunk][8 rows x 128 B]
+  uint8_t k[kTcStages][8][3][1024];        // K tile: [block][chunk][8 rows x 128 B] (SW128)
   uint8_t v[kTcVStages][8][3][1024];       // V tile, same layout (MN-major operand)
-  uint8_t p[2][128 * 128];                 // P: 128 rows x 64 tokens bf16 (SW128)
-  uint64_t q_full;
-  uint64_t k_full[kTcStages], k_empty[kTcStages], v_full[kTcVStages];
-  uint64_t s_full[3], s_free[3], p_full[2];
-  uint64_t pv_done[2];                     // PV(i) complete: V stage, P buffer and O free (i % 2)
+  uint64_t q_full;                         // Q written to TMEM (256 softmax threads)
+  uint64_t k_full[kTcStages], k_empty[kTcStages];
+  uint64_t v_full[kTcVStages], v_empty[kTcVStages];
+  uint64_t s_full[3];                      // S(j) in buffer j % 3
+  uint64_t p_full[3];                      // P(j) over S(j) (256 softmax threads)
+  uint64_t pv_done[3];                     // O += P(j) V(j) complete: buffer j % 3 free, O current
   uint64_t o_final, drain;
-  float pmax[2][2][128];                   // row maxima of each half, by tile parity
+  float pmax[2][2][128];                   // row maxima (and final sums) of each half, by tile parity
   uint32_t tmem;
   int abort;
 };
 
 __global__ void __launch_bounds__(kTcThreads, 1)
-attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUtensorMap kmap,
                const __grid_constant__ CUtensorMap vmap, const int32_t* __restrict__ plan_ids,
                const uint8_t* __restrict__ plan_mask, const int32_t* __restrict__ plan_count,
                __nv_bfloat16* __restrict__ out, int64_t nq, int G, int k, int64_t q_pos0,
@@ -77,17 +89,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   auto bar = [](uint64_t& b) { return smem_u32(&b); };
   if (threadIdx.x == 0) {
     sm.abort = 0;
-    tc::mbar_init(bar(sm.q_full), 1);
+    tc::mbar_init(bar(sm.q_full), 256);
     for (int s = 0; s < kTcStages; ++s) {
       tc::mbar_init(bar(sm.k_full[s]), 1);
       tc::mbar_init(bar(sm.k_empty[s]), 1);
     }
-    for (int s = 0; s < kTcVStages; ++s) tc::mbar_init(bar(sm.v_full[s]), 1);
+    for (int s = 0; s < kTcVStages; ++s) {
+      tc::mbar_init(bar(sm.v_full[s]), 1);
+      tc::mbar_init(bar(sm.v_empty[s]), 1);
+    }
     for (int b = 0; b < 3; ++b) {
       tc::mbar_init(bar(sm.s_full[b]), 1);
-      tc::mbar_init(bar(sm.s_free[b]), 256);
-    }
-    for (int b = 0; b < 2; ++b) {
       tc::mbar_init(bar(sm.p_full[b]), 256);
       tc::mbar_init(bar(sm.pv_done[b]), 1);
     }
@@ -100,52 +112,43 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   tc::fence_after();
   const uint32_t tmem = sm.tmem;
   const uint32_t tO = tmem;           // columns [0, 192)
-  const uint32_t tS0 = tmem + 256;    // S buffers at [256, 320), [320, 384), [384, 448)
+  const uint32_t tS0 = tmem + 192;    // S/P buffers at [192, 256), [256, 320), [320, 384)
+  const uint32_t tQ = tmem + 384;     // Q at [384, 480)
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 10) {
     // ------------------------------------------------------------ producers
-    // lane 0 streams Q and K, lane 1 streams V: the rings drain at different
-    // points (K after QK^T, V after PV), so each gets its own issuer.
-    if (lane < 2) {
-      const bool is_k = lane == 0;
-      const int nst = is_k ? kTcStages : kTcVStages;
-      if (is_k) {
-        tc::prefetch_tmap(&qmap);
-        tc::prefetch_tmap(&kmap);
-        tc::mbar_expect_tx(bar(sm.q_full), 3 * 128 * 128);
-        const int32_t qrow0 = static_cast<int32_t>(((seq * nq + qb * 8) * G + g) * 16);
-        const int32_t qstride = G * 16;
-        for (int c = 0; c < 3; ++c)
-          for (int i = 0; i < 8; ++i)
-            tc::tma_load_2d(smem_u32(&sm.q[c][i * 16 * 128]), &qmap, 64 * c, qrow0 + i * qstride, bar(sm.q_full));
+    // warp 0 streams K, warp 10 streams V: the rings drain at different points
+    // (K after QK^T, V after PV), so each gets its own issuer.
+    const bool is_k = warp == 0;
+    const int nst = is_k ? kTcStages : kTcVStages;
+    if (tc::elect_one()) tc::prefetch_tmap(is_k ? &kmap : &vmap);
+    __syncwarp();
+    // block ids of upcoming union tiles, fetched two tiles ahead
+    auto tile_rows = [&](int j, int32_t (&rows)[8]) {
+      if (j < n_union_tiles) {
+        const int4 a4 = *reinterpret_cast<const int4*>(uid + 8 * j);
+        const int4 b4 = *reinterpret_cast<const int4*>(uid + 8 * j + 4);
+        const int32_t ids[8] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) rows[e] = (8 * j + e < U) ? ids[e] * 8 : -64;
       } else {
-        tc::prefetch_tmap(&vmap);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          rows[e] = (e == 0 || (e == 1 && c0 + 8 <= t_last)) ? static_cast<int32_t>(c0 + 8 * e) : -64;
       }
-      // block ids of upcoming union tiles, fetched two tiles ahead
-      auto tile_rows = [&](int j, int32_t (&rows)[8]) {
-        if (j < n_union_tiles) {
-          const int4 a4 = *reinterpret_cast<const int4*>(uid + 8 * j);
-          const int4 b4 = *reinterpret_cast<const int4*>(uid + 8 * j + 4);
-          const int32_t ids[8] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-          for (int e = 0; e < 8; ++e) rows[e] = (8 * j + e < U) ? ids[e] * 8 : -64;
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            rows[e] = (e == 0 || (e == 1 && c0 + 8 <= t_last)) ? static_cast<int32_t>(c0 + 8 * e) : -64;
-        }
-      };
-      int32_t rows[8], next[8];
-      tile_rows(0, rows);
-      if (n_tiles > 1) tile_rows(1, next);
-      int issued = 0;
-      for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % nst;
-        int32_t next2[8];
-        if (j + 2 < n_tiles) tile_rows(j + 2, next2);
-        uint64_t* empty = is_k ? &sm.k_empty[s] : &sm.pv_done[s];
-        uint64_t* full = is_k ? &sm.k_full[s] : &sm.v_full[s];
-        if (j >= nst && !tc::mbar_wait(bar(*empty), ((j / nst) - 1) & 1, abort)) break;
+    };
+    int32_t rows[8], next[8];
+    tile_rows(0, rows);
+    if (n_tiles > 1) tile_rows(1, next);
+    int issued = 0;
+    for (int j = 0; j < n_tiles; ++j) {
+      const int s = j % nst;
+      int32_t next2[8];
+      if (j + 2 < n_tiles) tile_rows(j + 2, next2);
+      uint64_t* empty = is_k ? &sm.k_empty[s] : &sm.v_empty[s];
+      uint64_t* full = is_k ? &sm.k_full[s] : &sm.v_full[s];
+      if (j >= nst && !tc::warp_wait(bar(*empty), ((j / nst) - 1) & 1, abort)) break;
+      if (tc::elect_one()) {
         tc::mbar_expect_tx(bar(*full), 8 * 3 * 1024);
         const CUtensorMap* map = is_k ? &kmap : &vmap;
 #pragma unroll
@@ -153,86 +156,92 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           const uint32_t dst = is_k ? smem_u32(&sm.k[s][e][0][0]) : smem_u32(&sm.v[s][e][0][0]);
           tc::tma_load_5d(dst, map, 0, rows[e], 0, g, static_cast<int32_t>(seq), bar(*full));
         }
-        issued = j + 1;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          rows[e] = next[e];
-          next[e] = next2[e];
-        }
       }
-      if (*abort) {
-        // Let the copies already issued land before the CTA's shared memory goes away.
-        const uint64_t t0 = globaltimer_ns();
-        if (is_k)
-          while (!tc::mbar_try(bar(sm.q_full), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-          }
-        for (int j = issued > nst ? issued - nst : 0; j < issued; ++j) {
-          const uint64_t t1 = globaltimer_ns();
-          uint64_t* full = is_k ? &sm.k_full[j % nst] : &sm.v_full[j % nst];
-          while (!tc::mbar_try(bar(*full), (j / nst) & 1) && globaltimer_ns() - t1 < kWaitLimitNs) {
-          }
+      __syncwarp();
+      issued = j + 1;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        rows[e] = next[e];
+        next[e] = next2[e];
+      }
+    }
+    if (*abort) {
+      // Let the copies already issued land before the CTA's shared memory goes away.
+      for (int j = issued > nst ? issued - nst : 0; j < issued; ++j) {
+        const uint64_t t1 = globaltimer_ns();
+        uint64_t* full = is_k ? &sm.k_full[j % nst] : &sm.v_full[j % nst];
+        while (!tc::mbar_try(bar(*full), (j / nst) & 1) && globaltimer_ns() - t1 < kWaitLimitNs) {
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t id_qk = tc::idesc_bf16(128, 64, false);
-      const uint32_t id_pv = tc::idesc_bf16(128, 192, true);
-      // Base descriptors once per unit; each MMA adds a constant offset (in
-      // 16-byte units, the descriptor's address field) to one of them.
-      const uint64_t dq = tc::sdesc_sw128(smem_u32(&sm.q[0][0]), 16, 1024);
-      // stages are contiguous: stage x starts x * 24 KB (1536 units) after stage 0; P buffers 16 KB apart
-      const uint64_t dk0 = tc::sdesc_sw128(smem_u32(&sm.k[0][0][0][0]), 16, 3072);
-      const uint64_t dv0 = tc::sdesc_sw128(smem_u32(&sm.v[0][0][0][0]), 1024, 3072);
-      const uint64_t dp0 = tc::sdesc_sw128(smem_u32(&sm.p[0][0]), 16, 1024);
-      auto pv = [&](int i) -> bool {
-        const int pb = i & 1, s = i % kTcVStages;
-        if (!tc::mbar_wait(bar(sm.v_full[s]), (i / kTcVStages) & 1, abort)) return false;
-        if (!tc::mbar_wait(bar(sm.p_full[pb]), (i >> 1) & 1, abort)) return false;
-        tc::fence_after();
-        const uint64_t a0 = dp0 + 1024 * pb, b0 = dv0 + 1536 * s;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // P: +32 B per 16 tokens; V: +2 blocks (6144 B)
-          tc::mma_f16(tO, a0 + 2 * kk, b0 + 384 * kk, id_pv, (i > 0 || kk > 0) ? 1u : 0u);
-        tc::mma_commit(bar(sm.pv_done[pb]));
-        return true;
-      };
-      bool ok = tc::mbar_wait(bar(sm.q_full), 0, abort);
-      // QK^T runs two tiles ahead of PV, so the tensor pipe has work queued
-      // while the softmax of the older tile is still running.
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j % kTcStages, sb = j % 3;
-        if (!tc::mbar_wait(bar(sm.k_full[s]), (j / kTcStages) & 1, abort)) { ok = false; break; }
-        if (j >= 3 && !tc::mbar_wait(bar(sm.s_free[sb]), ((j / 3) - 1) & 1, abort)) { ok = false; break; }
-        tc::fence_after();
+    const uint32_t id_qk = tc::idesc_bf16(128, 64, false);
+    const uint32_t id_pv = tc::idesc_bf16(128, 192, true);
+    // Base descriptors once per unit; each MMA adds a constant offset (in
+    // 16-byte units, the descriptor's address field).  Stages are contiguous:
+    // stage x starts x * 24 KB (1536 units) after stage 0.
+    const uint64_t dk0 = tc::sdesc_sw128(smem_u32(&sm.k[0][0][0][0]), 16, 3072);
+    const uint64_t dv0 = tc::sdesc_sw128(smem_u32(&sm.v[0][0][0][0]), 1024, 3072);
+    auto qk = [&](int j) -> bool {
+      const int s = j % kTcStages, b = j % 3;
+      if (!tc::warp_wait(bar(sm.k_full[s]), (j / kTcStages) & 1, abort)) return false;
+      // buffer b still holds P(j-3) until O += P(j-3) V(j-3) has read it
+      if (j >= 3 && !tc::warp_wait(bar(sm.pv_done[b]), ((j / 3) - 1) & 1, abort)) return false;
+      tc::fence_after();
+      if (tc::elect_one()) {
         const uint64_t b0 = dk0 + 1536 * s;
 #pragma unroll
-        for (int kk = 0; kk < 12; ++kk)  // Q: +16 KB per 64 dims, +32 B per 16; K: +1 KB per 64 dims
-          tc::mma_f16(tS0 + 64 * sb, dq + (kk >> 2) * 1024 + (kk & 3) * 2, b0 + (kk >> 2) * 64 + (kk & 3) * 2,
-                      id_qk, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 12; ++kk)  // Q: 8 columns per 16 dims; K: +1 KB per 64 dims, +32 B per 16
+          tc::mma_f16_tmem_a(tS0 + 64 * b, tQ + 8 * kk, b0 + (kk >> 2) * 64 + (kk & 3) * 2, id_qk,
+                             kk > 0 ? 1u : 0u);
         tc::mma_commit(bar(sm.k_empty[s]));
-        tc::mma_commit(bar(sm.s_full[sb]));
-        if (j >= 2 && !pv(j - 2)) { ok = false; break; }
+        tc::mma_commit(bar(sm.s_full[b]));
       }
-      for (int i = n_tiles >= 2 ? n_tiles - 2 : 0; ok && i < n_tiles; ++i) ok = pv(i);
-      if (ok) {
-        tc::mma_commit(bar(sm.o_final));
-      } else {
-        // Let the MMAs already issued finish before TMEM is released.
-        tc::mma_commit(bar(sm.drain));
-        const uint64_t t0 = globaltimer_ns();
-        while (!tc::mbar_try(bar(sm.drain), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-        }
+      __syncwarp();
+      return true;
+    };
+    auto pv = [&](int j) -> bool {
+      const int s = j % kTcVStages, b = j % 3;
+      if (!tc::warp_wait(bar(sm.v_full[s]), (j / kTcVStages) & 1, abort)) return false;
+      if (!tc::warp_wait(bar(sm.p_full[b]), (j / 3) & 1, abort)) return false;
+      tc::fence_after();
+      if (tc::elect_one()) {
+        const uint64_t b0 = dv0 + 1536 * s;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // P: 8 columns per 16 tokens; V: +2 blocks (6144 B) per 16 tokens
+          tc::mma_f16_tmem_a(tO, tS0 + 64 * b + 8 * kk, b0 + 384 * kk, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        tc::mma_commit(bar(sm.v_empty[s]));
+        tc::mma_commit(bar(sm.pv_done[b]));
+      }
+      __syncwarp();
+      return true;
+    };
+    bool ok = tc::warp_wait(bar(sm.q_full), 0, abort);
+    tc::fence_after();
+    ok = ok && qk(0);
+    for (int j = 0; ok && j < n_tiles; ++j) {
+      if (j + 1 < n_tiles) ok = qk(j + 1);
+      ok = ok && pv(j);
+    }
+    if (ok) {
+      if (tc::elect_one()) tc::mma_commit(bar(sm.o_final));
+      __syncwarp();
+    } else {
+      // Let the MMAs already issued finish before TMEM is released.
+      if (tc::elect_one()) tc::mma_commit(bar(sm.drain));
+      __syncwarp();
+      const uint64_t t0 = globaltimer_ns();
+      while (!tc::mbar_try(bar(sm.drain), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
       }
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     // Eight warps, two per TMEM lane quadrant: both own the same 32 rows and
-    // split each tile's 64 tokens (and O's 192 columns) in halves, exchanging
-    // the row maxima through shared memory, so two warps per SM sub-partition
-    // hide each other's latency.  A failed wait clears `ok` but keeps the pair
-    // in step (every pair barrier is still reached).
+    // split each tile's 64 tokens (and Q's and O's columns) in halves,
+    // exchanging the row maxima through shared memory, so two warps per SM
+    // sub-partition hide each other's latency.  A failed wait clears `ok` but
+    // keeps the pair in step (every pair barrier is still reached).
     const int sw = warp - 2;                 // 0..7
     const int quad = warp & 3;
     const int half = sw >> 2;                // tokens [32 half, 32 half + 32)
@@ -244,11 +253,33 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     const int64_t t = q_pos0 + (qvalid ? qi : qb * 8);
     const int64_t cur_lo = 8 * (t / 8);
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const int64_t orow_idx = ((seq * nq + (qvalid ? qi : 0)) * G + g) * kHg + (m & 15);
+    // Q row m, dims [96 half, 96 half + 96), into TMEM columns tQ + 48 half ...
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(q + orow_idx * kD + 96 * half);
+#pragma unroll
+      for (int c = 0; c < 3; ++c) {
+        uint32_t r[16];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const uint4 w = qvalid ? src[4 * c + x] : make_uint4(0u, 0u, 0u, 0u);
+          r[4 * x + 0] = w.x;
+          r[4 * x + 1] = w.y;
+          r[4 * x + 2] = w.z;
+          r[4 * x + 3] = w.w;
+        }
+        tc::tmem_st16(tQ + lane_off + 48 * half + 16 * c, r);
+      }
+      tc::tmem_st_wait();
+      tc::fence_before();
+      tc::mbar_arrive(bar(sm.q_full));
+    }
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     uint32_t mb_next = n_union_tiles > 0 ? *reinterpret_cast<const uint32_t*>(umask + 4 * half) : 0u;
     for (int j = 0; j < n_tiles; ++j) {
-      const int sb = j % 3, pb = j & 1;
+      const int b = j % 3;
+      const uint32_t tS = tS0 + 64 * b + lane_off;
       const uint32_t mb = mb_next;
       if (j + 1 < n_union_tiles) mb_next = *reinterpret_cast<const uint32_t*>(umask + 8 * (j + 1) + 4 * half);
       // which of this half's 32 tokens the row attends
@@ -266,13 +297,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           if (tok >= cur_lo && tok <= t) tok_mask |= 1u << jj;
         }
       }
-      ok = ok && tc::mbar_wait(bar(sm.s_full[sb]), (j / 3) & 1, abort);
+      ok = ok && tc::mbar_wait(bar(sm.s_full[b]), (j / 3) & 1, abort);
       tc::fence_after();
       uint32_t sr[32];
-      tc::tmem_ld32(tS0 + 64 * sb + 32 * half + lane_off, sr);
+      tc::tmem_ld32(tS + 32 * half, sr);
       tc::tmem_ld_wait();
-      tc::fence_before();
-      tc::mbar_arrive(bar(sm.s_free[sb]));
       // masked raw scores and this half's max (the scale is positive: it commutes with max)
       float mraw = -INFINITY;
 #pragma unroll
@@ -281,18 +310,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         sr[jj] = __float_as_uint(x);
         mraw = fmaxf(mraw, x);
       }
-      sm.pmax[pb][half][m] = mraw;
+      sm.pmax[j & 1][half][m] = mraw;
+      // both halves have read their S columns before either writes P over them
       asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
-      mraw = fmaxf(mraw, sm.pmax[pb][half ^ 1][m]);
+      mraw = fmaxf(mraw, sm.pmax[j & 1][half ^ 1][m]);
       const float mt = mraw * scale_log2;
       const float m_new = fmaxf(m_used, mt);
       const bool need = (m_used != -INFINITY) && (m_new > m_used + 8.0f);
       if (m_used == -INFINITY) m_used = m_new;
-      // P buffer pb is free once PV(j-2) has completed
-      if (j >= 2) ok = ok && tc::mbar_wait(bar(sm.pv_done[pb]), ((j >> 1) - 1) & 1, abort);
       if (__any_sync(0xffffffffu, need)) {
-        // O must hold PV(j-1): pv_done[(j-1)&1] completes for the ((j-1)/2)-th time
-        if (j >= 1) ok = ok && tc::mbar_wait(bar(sm.pv_done[(j - 1) & 1]), ((j - 1) >> 1) & 1, abort);
+        // O must hold P(j-1) V(j-1) before it is rescaled
+        if (j >= 1) ok = ok && tc::mbar_wait(bar(sm.pv_done[(j - 1) % 3]), ((j - 1) / 3) & 1, abort);
         tc::fence_after();
         const float alpha = need ? exp2f(m_used - m_new) : 1.f;
 #pragma unroll 1
@@ -304,35 +332,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
           tc::tmem_st32(tO + lane_off + 32 * h, o);
         }
-        tc::tmem_st_wait();
         if (need) {
           l *= alpha;
           m_used = m_new;
         }
       }
-      // P = 2^(s * scale - m_used) in BF16 (masked -> exp2(-inf) = 0), 4 chunks of 8 tokens
+      // P = 2^(s * scale - m_used) in BF16 (masked -> exp2(-inf) = 0), packed
+      // two tokens per column over this half's part of columns [0, 32)
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
-      uint8_t* prow = &sm.p[pb][0];
       float lsum = 0.f;
+      uint32_t pk[16];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        float pv8[8];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          pv8[x] = exp2f(fmaf(__uint_as_float(sr[8 * cc + x]), scale_log2, neg_m));
-          lsum += pv8[x];
-        }
-        uint4 w;
-        w.x = pack_bf16x2(pv8[0], pv8[1]);
-        w.y = pack_bf16x2(pv8[2], pv8[3]);
-        w.z = pack_bf16x2(pv8[4], pv8[5]);
-        w.w = pack_bf16x2(pv8[6], pv8[7]);
-        *reinterpret_cast<uint4*>(prow + tc::sw128_offset(static_cast<uint32_t>(m), static_cast<uint32_t>(4 * half + cc))) = w;
+      for (int x = 0; x < 16; ++x) {
+        const float p0 = exp2f(fmaf(__uint_as_float(sr[2 * x]), scale_log2, neg_m));
+        const float p1 = exp2f(fmaf(__uint_as_float(sr[2 * x + 1]), scale_log2, neg_m));
+        lsum += p0 + p1;
+        pk[x] = pack_bf16x2(p0, p1);
       }
+      tc::tmem_st16(tS + 16 * half, pk);
       l += lsum;
-      tc::fence_proxy_async_smem();
+      tc::tmem_st_wait();
       tc::fence_before();
-      tc::mbar_arrive(bar(sm.p_full[pb]));
+      tc::mbar_arrive(bar(sm.p_full[b]));
     }
     ok = ok && tc::mbar_wait(bar(sm.o_final), 0, abort);
     // full row sum from both halves (the parity slot the last tile did not use)
@@ -342,7 +363,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     if (ok) {
       tc::fence_after();
       const float inv = 1.f / ltot;
-      __nv_bfloat16* orow = out + (((seq * nq + (qvalid ? qi : 0)) * G + g) * kHg + (m & 15)) * kD;
+      __nv_bfloat16* orow = out + orow_idx * kD;
 #pragma unroll 1
       for (int h = 3 * half; h < 3 * half + 3; ++h) {
         uint32_t o[32];

@@ -228,14 +228,8 @@ sgqa_status launch_attn_tc(const sgqa_params* p, int64_t S, int64_t q0, int64_t 
                            const uint8_t* msk, const int32_t* cnt, void* out, int64_t units, cudaStream_t st) {
   const int G = p->num_kv_groups;
   const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
-  CUtensorMap qm, km, vm;
+  CUtensorMap km, vm;
   sgqa_status s;
-  {
-    cuuint64_t dims[2] = {192, static_cast<cuuint64_t>(S * nq * G * 16)};
-    cuuint64_t strides[1] = {192 * 2};
-    cuuint32_t box[2] = {64, 16};
-    if ((s = encode_bf16(&qm, q, 2, dims, strides, box, "q")) != SGQA_OK) return s;
-  }
   {
     // (64 elements, token rows < cache_len, 3 column chunks, group, sequence)
     cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(clen), 3, static_cast<cuuint64_t>(G), static_cast<cuuint64_t>(S)};
@@ -248,7 +242,8 @@ sgqa_status launch_attn_tc(const sgqa_params* p, int64_t S, int64_t q0, int64_t 
   const size_t smem = sizeof(sgqa::AttnTcSmem) + 1024;
   cudaFuncSetAttribute(sgqa::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   sgqa::attn_tc_kernel<<<static_cast<unsigned>(units), sgqa::kTcThreads, smem, st>>>(
-      qm, km, vm, ids, msk, cnt, static_cast<__nv_bfloat16*>(out), nq, G, p->topk, q0, scale_log2);
+      static_cast<const __nv_bfloat16*>(q), km, vm, ids, msk, cnt, static_cast<__nv_bfloat16*>(out), nq, G,
+      p->topk, q0, scale_log2);
   SGQA_LAUNCH_CHECK("attn_tc_kernel");
   return SGQA_OK;
 }
