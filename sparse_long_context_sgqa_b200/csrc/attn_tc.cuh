@@ -50,10 +50,11 @@ struct __align__(1024) AttnTcSmem {
   uint64_t k_full[kTcStages], k_empty[kTcStages];
   uint64_t v_full[kTcVStages], v_empty[kTcVStages];
   uint64_t s_full[3];                      // S(j) in buffer j % 3
-  uint64_t p_full[3];                      // P(j) over S(j) (256 softmax threads)
+  uint64_t p_full[3];                      // P(j) over S(j) (the 128 threads of tile j's warps)
   uint64_t pv_done[3];                     // O += P(j) V(j) complete: buffer j % 3 free, O current
   uint64_t o_final, drain;
-  float pmax[2][2][128];                   // row maxima (and final sums) of each half, by tile parity
+  float mchain[128];                       // running reference max after the latest tile, per row
+  float lsum[2][128];                      // partial row sums of the two warps of a quadrant
   uint32_t tmem;
   int abort;
 };
@@ -100,7 +101,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     }
     for (int b = 0; b < 3; ++b) {
       tc::mbar_init(bar(sm.s_full[b]), 1);
-      tc::mbar_init(bar(sm.p_full[b]), 256);
+      tc::mbar_init(bar(sm.p_full[b]), 128);
       tc::mbar_init(bar(sm.pv_done[b]), 1);
     }
     tc::mbar_init(bar(sm.o_final), 1);
@@ -237,15 +238,20 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    // Eight warps, two per TMEM lane quadrant: both own the same 32 rows and
-    // split each tile's 64 tokens (and Q's and O's columns) in halves,
-    // exchanging the row maxima through shared memory, so two warps per SM
-    // sub-partition hide each other's latency.  A failed wait clears `ok` but
-    // keeps the pair in step (every pair barrier is still reached).
+    // Eight warps, two per TMEM lane quadrant (both own the same 32 rows).  The
+    // two take alternate tiles, so one warp's exponentials overlap the other's
+    // TMEM load and row max on the same SM sub-partition.  The running
+    // reference max is handed from tile to tile through shared memory: the
+    // warp of tile j publishes it (bar.arrive) right after its row max, the
+    // warp of tile j+1 picks it up (bar.sync) before computing P.  Each warp
+    // keeps its own partial row sum; the two are combined in the epilogue.  A
+    // failed wait clears `ok` but keeps every barrier step in place.
     const int sw = warp - 2;                 // 0..7
     const int quad = warp & 3;
-    const int half = sw >> 2;                // tokens [32 half, 32 half + 32)
-    const int pair_bar = 1 + quad;           // named barrier of the two warps of this quadrant
+    const int half = sw >> 2;                // this warp takes tiles j with j % 2 == half
+    const int pair_bar = 1 + quad;           // both warps of this quadrant
+    const int pub_mine = 5 + 2 * quad + half;         // this warp -> the other
+    const int pub_other = 5 + 2 * quad + (half ^ 1);  // the other warp -> this one
     const int m = quad * 32 + lane;          // TMEM lane = row = (query slot, head)
     const int qs = m >> 4;
     const int64_t qi = qb * 8 + qs;
@@ -274,57 +280,84 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       tc::fence_before();
       tc::mbar_arrive(bar(sm.q_full));
     }
-    float m_used = -INFINITY, l = 0.f;
+    float m_l = -INFINITY, l = 0.f;          // this warp's partial row sum, relative to 2^m_l
     bool ok = true;
-    uint32_t mb_next = n_union_tiles > 0 ? *reinterpret_cast<const uint32_t*>(umask + 4 * half) : 0u;
-    for (int j = 0; j < n_tiles; ++j) {
+    // mask bytes of this warp's next tile, loaded one own tile (two tiles) ahead
+    uint2 mb_next = half < n_union_tiles ? *reinterpret_cast<const uint2*>(umask + 8 * half) : make_uint2(0u, 0u);
+    for (int j = half; j < n_tiles; j += 2) {
       const int b = j % 3;
       const uint32_t tS = tS0 + 64 * b + lane_off;
-      const uint32_t mb = mb_next;
-      if (j + 1 < n_union_tiles) mb_next = *reinterpret_cast<const uint32_t*>(umask + 8 * (j + 1) + 4 * half);
-      // which of this half's 32 tokens the row attends
-      uint32_t tok_mask = 0;
+      const uint2 mb = mb_next;
+      if (j + 2 < n_union_tiles) mb_next = *reinterpret_cast<const uint2*>(umask + 8 * (j + 2));
+      // blocks (8 tokens each) of this tile the row attends: the row's query
+      // selected the block, or (current tile) causal positions of its own block
+      uint32_t bmask = 0;
       if (j < n_union_tiles) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t byte = (mb >> (8 * e)) & 0xFFu;
-          if (8 * j + 4 * half + e < U && ((byte >> qs) & 1u)) tok_mask |= 0xFFu << (8 * e);
+        for (int e = 0; e < 8; ++e) {
+          const uint32_t byte = ((e < 4 ? mb.x : mb.y) >> (8 * (e & 3))) & 0xFFu;
+          if (8 * j + e < U && ((byte >> qs) & 1u)) bmask |= 1u << e;
         }
-      } else if (half == 0) {
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int64_t tok = c0 + jj;
-          if (tok >= cur_lo && tok <= t) tok_mask |= 1u << jj;
-        }
+      } else {
+        bmask = 3u;
       }
       ok = ok && tc::mbar_wait(bar(sm.s_full[b]), (j / 3) & 1, abort);
       tc::fence_after();
-      uint32_t sr[32];
-      tc::tmem_ld32(tS + 32 * half, sr);
+      uint32_t sr[64];
+      tc::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tc::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tc::tmem_ld_wait();
-      // masked raw scores and this half's max (the scale is positive: it commutes with max)
-      float mraw = -INFINITY;
+      // masked raw scores and their max (the scale is positive: it commutes with max)
+      float bm[8];
+      if (j < n_union_tiles) {
+        // one decision per 8-token block
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {
-        const float x = ((tok_mask >> jj) & 1u) ? __uint_as_float(sr[jj]) : -INFINITY;
-        sr[jj] = __float_as_uint(x);
-        mraw = fmaxf(mraw, x);
+        for (int e = 0; e < 8; ++e) {
+          const bool keep = (bmask >> e) & 1u;
+          bm[e] = -INFINITY;
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            const float v = keep ? __uint_as_float(sr[8 * e + x]) : -INFINITY;
+            sr[8 * e + x] = __float_as_uint(v);
+            bm[e] = fmaxf(bm[e], v);
+          }
+        }
+      } else {
+        // current tile: tokens c0 .. c0 + 15, of which the row attends cur_lo .. t
+        const int lo = static_cast<int>(cur_lo - c0), hi = static_cast<int>(t - c0);  // 0 <= lo <= hi <= 15
+        const uint32_t tm = ((2u << hi) - 1u) & ~((1u << lo) - 1u);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          bm[e] = -INFINITY;
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            const bool keep = e < 2 && ((tm >> (8 * e + x)) & 1u);
+            const float v = keep ? __uint_as_float(sr[8 * e + x]) : -INFINITY;
+            sr[8 * e + x] = __float_as_uint(v);
+            bm[e] = fmaxf(bm[e], v);
+          }
+        }
       }
-      sm.pmax[j & 1][half][m] = mraw;
-      // both halves have read their S columns before either writes P over them
-      asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
-      mraw = fmaxf(mraw, sm.pmax[j & 1][half ^ 1][m]);
-      const float mt = mraw * scale_log2;
-      const float m_new = fmaxf(m_used, mt);
-      const bool need = (m_used != -INFINITY) && (m_new > m_used + 8.0f);
-      if (m_used == -INFINITY) m_used = m_new;
+      const float mraw = fmaxf(fmaxf(fmaxf(bm[0], bm[1]), fmaxf(bm[2], bm[3])),
+                               fmaxf(fmaxf(bm[4], bm[5]), fmaxf(bm[6], bm[7])));
+      // reference after tile j-1 (published by the other warp)
+      float m_prev = -INFINITY;
+      if (j > 0) {
+        asm volatile("bar.sync %0, 64;" ::"r"(pub_other) : "memory");
+        m_prev = sm.mchain[m];
+      }
+      const float m_new = fmaxf(m_prev, mraw * scale_log2);
+      const bool need = (m_prev != -INFINITY) && (m_new > m_prev + 8.0f);
+      const float m_use = (m_prev == -INFINITY || need) ? m_new : m_prev;
+      sm.mchain[m] = m_use;
+      if (j + 1 < n_tiles) asm volatile("bar.arrive %0, 64;" ::"r"(pub_mine) : "memory");
       if (__any_sync(0xffffffffu, need)) {
         // O must hold P(j-1) V(j-1) before it is rescaled
-        if (j >= 1) ok = ok && tc::mbar_wait(bar(sm.pv_done[(j - 1) % 3]), ((j - 1) / 3) & 1, abort);
+        ok = ok && tc::mbar_wait(bar(sm.pv_done[(j - 1) % 3]), ((j - 1) / 3) & 1, abort);
         tc::fence_after();
-        const float alpha = need ? exp2f(m_used - m_new) : 1.f;
+        const float alpha = need ? exp2f(m_prev - m_use) : 1.f;
 #pragma unroll 1
-        for (int h = 3 * half; h < 3 * half + 3; ++h) {
+        for (int h = 0; h < 6; ++h) {
           uint32_t o[32];
           tc::tmem_ld32(tO + lane_off + 32 * h, o);
           tc::tmem_ld_wait();
@@ -332,34 +365,46 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
           for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
           tc::tmem_st32(tO + lane_off + 32 * h, o);
         }
-        if (need) {
-          l *= alpha;
-          m_used = m_new;
+      }
+      if (m_l != m_use) {
+        l = m_l == -INFINITY ? 0.f : l * exp2f(m_l - m_use);
+        m_l = m_use;
+      }
+      // P = 2^(s * scale - m_use) in BF16 (masked -> 0), packed two tokens per
+      // column over columns [0, 32) of the buffer; blocks that no row of this
+      // warp attends skip their exponentials
+      const float neg_m = m_use == -INFINITY ? 0.f : -m_use;
+      float lsum = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (__any_sync(0xffffffffu, (bmask >> e) & 1u)) {
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sr[8 * e + 2 * x]), scale_log2, neg_m));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sr[8 * e + 2 * x + 1]), scale_log2, neg_m));
+            lsum += p0 + p1;
+            pk[4 * e + x] = pack_bf16x2(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int x = 0; x < 4; ++x) pk[4 * e + x] = 0u;
         }
       }
-      // P = 2^(s * scale - m_used) in BF16 (masked -> exp2(-inf) = 0), packed
-      // two tokens per column over this half's part of columns [0, 32)
-      const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
-      float lsum = 0.f;
-      uint32_t pk[16];
-#pragma unroll
-      for (int x = 0; x < 16; ++x) {
-        const float p0 = exp2f(fmaf(__uint_as_float(sr[2 * x]), scale_log2, neg_m));
-        const float p1 = exp2f(fmaf(__uint_as_float(sr[2 * x + 1]), scale_log2, neg_m));
-        lsum += p0 + p1;
-        pk[x] = pack_bf16x2(p0, p1);
-      }
-      tc::tmem_st16(tS + 16 * half, pk);
+      tc::tmem_st32(tS, pk);
       l += lsum;
       tc::tmem_st_wait();
       tc::fence_before();
       tc::mbar_arrive(bar(sm.p_full[b]));
     }
     ok = ok && tc::mbar_wait(bar(sm.o_final), 0, abort);
-    // full row sum from both halves (the parity slot the last tile did not use)
-    sm.pmax[n_tiles & 1][half][m] = l;
+    // both loops done: the final reference is in mchain; combine the two partial sums
     asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
-    const float ltot = l + sm.pmax[n_tiles & 1][half ^ 1][m];
+    const float m_fin = sm.mchain[m];
+    const float l_adj = (m_l == -INFINITY) ? 0.f : (m_l == m_fin ? l : l * exp2f(m_l - m_fin));
+    sm.lsum[half][m] = l_adj;
+    asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+    const float ltot = l_adj + sm.lsum[half ^ 1][m];
     if (ok) {
       tc::fence_after();
       const float inv = 1.f / ltot;
