@@ -184,12 +184,8 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     // stage x starts x * 24 KB (1536 units) after stage 0.
     const uint64_t dk0 = tc::sdesc_sw128(smem_u32(&sm.k[0][0][0][0]), 16, 3072);
     const uint64_t dv0 = tc::sdesc_sw128(smem_u32(&sm.v[0][0][0][0]), 1024, 3072);
-    auto qk = [&](int j) -> bool {
+    auto issue_qk = [&](int j) {
       const int s = j % kTcStages, b = j % 3;
-      if (!tc::warp_wait(bar(sm.k_full[s]), (j / kTcStages) & 1, abort)) return false;
-      // buffer b still holds P(j-3) until O += P(j-3) V(j-3) has read it
-      if (j >= 3 && !tc::warp_wait(bar(sm.pv_done[b]), ((j / 3) - 1) & 1, abort)) return false;
-      tc::fence_after();
       if (tc::elect_one()) {
         const uint64_t b0 = dk0 + 1536 * s;
 #pragma unroll
@@ -200,13 +196,9 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
         tc::mma_commit(bar(sm.s_full[b]));
       }
       __syncwarp();
-      return true;
     };
-    auto pv = [&](int j) -> bool {
+    auto issue_pv = [&](int j) {
       const int s = j % kTcVStages, b = j % 3;
-      if (!tc::warp_wait(bar(sm.v_full[s]), (j / kTcVStages) & 1, abort)) return false;
-      if (!tc::warp_wait(bar(sm.p_full[b]), (j / 3) & 1, abort)) return false;
-      tc::fence_after();
       if (tc::elect_one()) {
         const uint64_t b0 = dv0 + 1536 * s;
 #pragma unroll
@@ -216,14 +208,35 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
         tc::mma_commit(bar(sm.pv_done[b]));
       }
       __syncwarp();
-      return true;
     };
-    bool ok = tc::warp_wait(bar(sm.q_full), 0, abort);
+    bool ok = tc::warp_wait(bar(sm.q_full), 0, abort) && tc::warp_wait(bar(sm.k_full[0]), 0, abort);
     tc::fence_after();
-    ok = ok && qk(0);
+    if (ok) issue_qk(0);
     for (int j = 0; ok && j < n_tiles; ++j) {
-      if (j + 1 < n_tiles) ok = qk(j + 1);
-      ok = ok && pv(j);
+      // Iteration j issues S(j+1) = Q K(j+1)^T, then O += P(j) V(j).  Three of
+      // its four conditions are nearly always met by now (K(j+1) and V(j)
+      // landed, S buffer (j+1) % 3 released by PV(j-2)): one combined test,
+      // bounded waits only for what it found missing; then wait for P(j).
+      const int jn = j + 1, sk = jn % kTcStages, sv = j % kTcVStages, bn = jn % 3;
+      const bool has_next = jn < n_tiles;
+      const uint32_t ready = tc::mbar_test3(bar(sm.k_full[sk]), (jn / kTcStages) & 1, bar(sm.v_full[sv]),
+                                            (j / kTcVStages) & 1, bar(sm.pv_done[bn]), ((jn / 3) - 1) & 1);
+      const uint32_t need = (has_next ? 1u : 0u) | 2u | (has_next && jn >= 3 ? 4u : 0u);
+      if (!__all_sync(0xffffffffu, (ready & need) == need)) {
+        if (has_next) ok = tc::warp_wait(bar(sm.k_full[sk]), (jn / kTcStages) & 1, abort);
+        ok = ok && tc::warp_wait(bar(sm.v_full[sv]), (j / kTcVStages) & 1, abort);
+        // buffer (j+1) % 3 still holds P(j-2) until O += P(j-2) V(j-2) has read it
+        if (has_next && jn >= 3) ok = ok && tc::warp_wait(bar(sm.pv_done[bn]), ((jn / 3) - 1) & 1, abort);
+        if (!ok) break;
+      }
+      tc::fence_after();
+      if (has_next) issue_qk(jn);
+      if (!tc::warp_wait(bar(sm.p_full[j % 3]), (j / 3) & 1, abort)) {
+        ok = false;
+        break;
+      }
+      tc::fence_after();
+      issue_pv(j);
     }
     if (ok) {
       if (tc::elect_one()) tc::mma_commit(bar(sm.o_final));

@@ -29,6 +29,35 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking completion test of the phase with the given parity.  Its
+// result is consumed later, so the shared-memory round trip can overlap
+// other work of the thread.
+__device__ __forceinline__ uint32_t mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok;
+}
+// Three completion tests issued back to back (one shared-memory round trip
+// instead of three); bit i of the result is barrier i's test.
+__device__ __forceinline__ uint32_t mbar_test3(uint32_t b0, uint32_t p0, uint32_t b1, uint32_t p1, uint32_t b2,
+                                               uint32_t p2) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred q0, q1, q2;\n .reg .b32 r0, r1, r2;\n"
+      " mbarrier.test_wait.parity.shared::cta.b64 q0, [%1], %2;\n"
+      " mbarrier.test_wait.parity.shared::cta.b64 q1, [%3], %4;\n"
+      " mbarrier.test_wait.parity.shared::cta.b64 q2, [%5], %6;\n"
+      " selp.u32 r0, 1, 0, q0;\n selp.u32 r1, 2, 0, q1;\n selp.u32 r2, 4, 0, q2;\n"
+      " or.b32 r0, r0, r1;\n or.b32 %0, r0, r2;\n}"
+      : "=r"(ok)
+      : "r"(b0), "r"(p0), "r"(b1), "r"(p1), "r"(b2), "r"(p2)
+      : "memory");
+  return ok;
+}
 // Wait for the phase with the given parity to complete; gives up after
 // kWaitLimitNs, records kDevTimeout and returns false.  `abort` (shared)
 // short-cuts every later wait of the CTA once one has given up.
