@@ -12,19 +12,21 @@
 //
 // Tensor memory (512 columns, one row per TMEM lane):
 //   [0, 192)    O accumulator, FP32
-//   [192, 384)  three S buffers of 64 FP32 columns; the softmax overwrites the
-//               first 32 columns of a buffer with its P (two BF16 per column)
+//   [192, 320)  two S buffers of 64 FP32 columns
+//   [320, 384)  two P buffers of 32 columns, two BF16 per column
 //   [384, 480)  Q, two BF16 per column, written once per unit by the softmax warps
-// Per 64-token tile j (buffer b = j % 3):
+// An S buffer is free again as soon as the softmax has loaded it, a P buffer
+// once O += P V has read it.
+// Per 64-token tile j (buffers j % 2):
 //   S = Q K^T   12 tcgen05.mma (M128 N64 K16), A = Q from TMEM, B = K (SMEM, K-major)
 //   softmax     per-row block mask (the row's query must have selected the
 //               block) and causal mask on the current block, running max in
 //               log2 units with lazy rescaling of O (only when the max grows
-//               by more than 2^8), P rounded to BF16 and stored over S
+//               by more than 2^8), P rounded to BF16 into its P buffer
 //   O += P V    4 tcgen05.mma (M128 N192 K16), A = P from TMEM, B = V (SMEM, MN-major)
-// The MMA thread issues S(j+1) before O += P(j) V(j), so the tensor pipe
-// computes the next scores while the softmax works on the current ones; the
-// softmax waits on an O update only for the (rare) rescale.
+// The MMA warp issues S(j+2) before O += P(j) V(j), so the softmax always
+// finds the next scores computed; it waits on an O update only for the
+// (rare) rescale.
 // Warp roles: warp 0 streams K and warp 10 streams V by TMA (one 5-D box per
 // 8-token block gathers all 192 dims: 3 KB), warp 1 allocates TMEM and issues
 // the MMAs, warps 2-9 run the softmax and the epilogue.  The producer and MMA
@@ -49,9 +51,10 @@ struct __align__(1024) AttnTcSmem {
   uint64_t q_full;                         // Q written to TMEM (256 softmax threads)
   uint64_t k_full[kTcStages], k_empty[kTcStages];
   uint64_t v_full[kTcVStages], v_empty[kTcVStages];
-  uint64_t s_full[3];                      // S(j) in buffer j % 3
-  uint64_t p_full[3];                      // P(j) over S(j) (the 128 threads of tile j's warps)
-  uint64_t pv_done[3];                     // O += P(j) V(j) complete: buffer j % 3 free, O current
+  uint64_t s_full[2];                      // S(j) in S buffer j % 2
+  uint64_t s_free[2];                      // S(j) loaded by the softmax (the 128 threads of tile j's warps)
+  uint64_t p_full[2];                      // P(j) in P buffer j % 2 (the 128 threads of tile j's warps)
+  uint64_t pv_done[2];                     // O += P(j) V(j) complete: P buffer j % 2 free, O current
   uint64_t o_final, drain;
   float mchain[128];                       // running reference max after the latest tile, per row
   float lsum[2][128];                      // partial row sums of the two warps of a quadrant
@@ -99,8 +102,9 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       tc::mbar_init(bar(sm.v_full[s]), 1);
       tc::mbar_init(bar(sm.v_empty[s]), 1);
     }
-    for (int b = 0; b < 3; ++b) {
+    for (int b = 0; b < 2; ++b) {
       tc::mbar_init(bar(sm.s_full[b]), 1);
+      tc::mbar_init(bar(sm.s_free[b]), 128);
       tc::mbar_init(bar(sm.p_full[b]), 128);
       tc::mbar_init(bar(sm.pv_done[b]), 1);
     }
@@ -113,7 +117,8 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
   tc::fence_after();
   const uint32_t tmem = sm.tmem;
   const uint32_t tO = tmem;           // columns [0, 192)
-  const uint32_t tS0 = tmem + 192;    // S/P buffers at [192, 256), [256, 320), [320, 384)
+  const uint32_t tS0 = tmem + 192;    // S buffers at [192, 256), [256, 320)
+  const uint32_t tP0 = tmem + 320;    // P buffers at [320, 352), [352, 384)
   const uint32_t tQ = tmem + 384;     // Q at [384, 480)
 
   if (warp == 0 || warp == 10) {
@@ -185,7 +190,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     const uint64_t dk0 = tc::sdesc_sw128(smem_u32(&sm.k[0][0][0][0]), 16, 3072);
     const uint64_t dv0 = tc::sdesc_sw128(smem_u32(&sm.v[0][0][0][0]), 1024, 3072);
     auto issue_qk = [&](int j) {
-      const int s = j % kTcStages, b = j % 3;
+      const int s = j % kTcStages, b = j % 2;
       if (tc::elect_one()) {
         const uint64_t b0 = dk0 + 1536 * s;
 #pragma unroll
@@ -198,12 +203,12 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       __syncwarp();
     };
     auto issue_pv = [&](int j) {
-      const int s = j % kTcVStages, b = j % 3;
+      const int s = j % kTcVStages, b = j % 2;
       if (tc::elect_one()) {
         const uint64_t b0 = dv0 + 1536 * s;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // P: 8 columns per 16 tokens; V: +2 blocks (6144 B) per 16 tokens
-          tc::mma_f16_tmem_a(tO, tS0 + 64 * b + 8 * kk, b0 + 384 * kk, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_f16_tmem_a(tO, tP0 + 32 * b + 8 * kk, b0 + 384 * kk, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
         tc::mma_commit(bar(sm.v_empty[s]));
         tc::mma_commit(bar(sm.pv_done[b]));
       }
@@ -212,26 +217,31 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     bool ok = tc::warp_wait(bar(sm.q_full), 0, abort) && tc::warp_wait(bar(sm.k_full[0]), 0, abort);
     tc::fence_after();
     if (ok) issue_qk(0);
+    if (ok && n_tiles > 1) {
+      ok = tc::warp_wait(bar(sm.k_full[1]), 0, abort);
+      tc::fence_after();
+      if (ok) issue_qk(1);
+    }
     for (int j = 0; ok && j < n_tiles; ++j) {
-      // Iteration j issues S(j+1) = Q K(j+1)^T, then O += P(j) V(j).  Three of
-      // its four conditions are nearly always met by now (K(j+1) and V(j)
-      // landed, S buffer (j+1) % 3 released by PV(j-2)): one combined test,
-      // bounded waits only for what it found missing; then wait for P(j).
-      const int jn = j + 1, sk = jn % kTcStages, sv = j % kTcVStages, bn = jn % 3;
+      // Iteration j issues S(j+2) = Q K(j+2)^T, then O += P(j) V(j), so the
+      // softmax always has the next tile's scores waiting.  Three of its four
+      // conditions are usually met by now (K(j+2) and V(j) landed, S buffer
+      // j % 2 loaded by the softmax of tile j): one combined test, bounded
+      // waits only for what it found missing; then wait for P(j).
+      const int jn = j + 2, sk = jn % kTcStages, sv = j % kTcVStages, bn = j % 2;
       const bool has_next = jn < n_tiles;
       const uint32_t ready = tc::mbar_test3(bar(sm.k_full[sk]), (jn / kTcStages) & 1, bar(sm.v_full[sv]),
-                                            (j / kTcVStages) & 1, bar(sm.pv_done[bn]), ((jn / 3) - 1) & 1);
-      const uint32_t need = (has_next ? 1u : 0u) | 2u | (has_next && jn >= 3 ? 4u : 0u);
+                                            (j / kTcVStages) & 1, bar(sm.s_free[bn]), (j / 2) & 1);
+      const uint32_t need = has_next ? 7u : 2u;
       if (!__all_sync(0xffffffffu, (ready & need) == need)) {
         if (has_next) ok = tc::warp_wait(bar(sm.k_full[sk]), (jn / kTcStages) & 1, abort);
         ok = ok && tc::warp_wait(bar(sm.v_full[sv]), (j / kTcVStages) & 1, abort);
-        // buffer (j+1) % 3 still holds P(j-2) until O += P(j-2) V(j-2) has read it
-        if (has_next && jn >= 3) ok = ok && tc::warp_wait(bar(sm.pv_done[bn]), ((jn / 3) - 1) & 1, abort);
+        if (has_next) ok = ok && tc::warp_wait(bar(sm.s_free[bn]), (j / 2) & 1, abort);
         if (!ok) break;
       }
       tc::fence_after();
       if (has_next) issue_qk(jn);
-      if (!tc::warp_wait(bar(sm.p_full[j % 3]), (j / 3) & 1, abort)) {
+      if (!tc::warp_wait(bar(sm.p_full[j % 2]), (j / 2) & 1, abort)) {
         ok = false;
         break;
       }
@@ -298,8 +308,9 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     // mask bytes of this warp's next tile, loaded one own tile (two tiles) ahead
     uint2 mb_next = half < n_union_tiles ? *reinterpret_cast<const uint2*>(umask + 8 * half) : make_uint2(0u, 0u);
     for (int j = half; j < n_tiles; j += 2) {
-      const int b = j % 3;
+      const int b = j % 2;
       const uint32_t tS = tS0 + 64 * b + lane_off;
+      const uint32_t tP = tP0 + 32 * b + lane_off;
       const uint2 mb = mb_next;
       if (j + 2 < n_union_tiles) mb_next = *reinterpret_cast<const uint2*>(umask + 8 * (j + 2));
       // blocks (8 tokens each) of this tile the row attends: the row's query
@@ -314,12 +325,14 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       } else {
         bmask = 3u;
       }
-      ok = ok && tc::mbar_wait(bar(sm.s_full[b]), (j / 3) & 1, abort);
+      ok = ok && tc::mbar_wait(bar(sm.s_full[b]), (j / 2) & 1, abort);
       tc::fence_after();
       uint32_t sr[64];
       tc::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       tc::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tc::tmem_ld_wait();
+      tc::fence_before();
+      tc::mbar_arrive(bar(sm.s_free[b]));
       // masked raw scores and their max (the scale is positive: it commutes with max)
       float bm[8];
       if (j < n_union_tiles) {
@@ -366,7 +379,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       if (j + 1 < n_tiles) asm volatile("bar.arrive %0, 64;" ::"r"(pub_mine) : "memory");
       if (__any_sync(0xffffffffu, need)) {
         // O must hold P(j-1) V(j-1) before it is rescaled
-        ok = ok && tc::mbar_wait(bar(sm.pv_done[(j - 1) % 3]), ((j - 1) / 3) & 1, abort);
+        ok = ok && tc::mbar_wait(bar(sm.pv_done[(j - 1) % 2]), ((j - 1) / 2) & 1, abort);
         tc::fence_after();
         const float alpha = need ? exp2f(m_prev - m_use) : 1.f;
 #pragma unroll 1
@@ -384,8 +397,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
         m_l = m_use;
       }
       // P = 2^(s * scale - m_use) in BF16 (masked -> 0), packed two tokens per
-      // column over columns [0, 32) of the buffer; blocks that no row of this
-      // warp attends skip their exponentials
+      // column; blocks that no row of this warp attends skip their exponentials
       const float neg_m = m_use == -INFINITY ? 0.f : -m_use;
       float lsum = 0.f;
       uint32_t pk[32];
@@ -404,7 +416,10 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
           for (int x = 0; x < 4; ++x) pk[4 * e + x] = 0u;
         }
       }
-      tc::tmem_st32(tS, pk);
+      // P buffer b is free once O += P(j-2) V(j-2) has read it
+      if (j >= 2) ok = ok && tc::mbar_wait(bar(sm.pv_done[b]), ((j / 2) - 1) & 1, abort);
+      tc::fence_after();
+      tc::tmem_st32(tP, pk);
       l += lsum;
       tc::tmem_st_wait();
       tc::fence_before();
