@@ -723,4 +723,181 @@ topk_final_kernel(const uint2* __restrict__ staging, const int32_t* __restrict__
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Top-k for rows of at most kWinThreads * kWinPer candidates (every prefill
+// row up to a 131072-token context): the row is read from HBM once into
+// registers (thread t holds candidates t, t + 512, ...).  A 256-bin histogram
+// of the scores, linear between the row's minimum and maximum, finds the bin
+// b* holding the k-th largest; a linear bin is a monotone function of the
+// score, so every candidate of a higher bin beats every candidate of b*, and
+// only b* needs an exact (score, then smaller id) selection.  The selection is
+// a bitmap built with one ballot per warp and iteration (a warp's 32 lanes
+// hold 32 consecutive ids = one bitmap word), read out in ascending id order.
+// A row whose boundary bin holds more than kWinCand candidates (massive exact
+// ties) is flagged in `overflow` and left to the radix kernel.
+// ---------------------------------------------------------------------------
+constexpr int kWinThreads = 512;
+constexpr int kWinWarps = kWinThreads / 32;
+constexpr int kWinPer = 32;
+constexpr int kWinMaxCand = kWinThreads * kWinPer;  // 16384
+constexpr int kWinBins = 256;
+constexpr int kWinCand = 2048;
+
+struct WinSmem {
+  uint32_t wh[kWinWarps][kWinBins];   // per-warp histograms (also warp_select scratch)
+  uint2 cand[kWinCand];               // (key, id) of the boundary bin
+  uint32_t bits[kWinMaxCand / 32];    // selection bitmap
+  float rmax[kWinWarps], rmin[kWinWarps];
+  uint32_t wsum[kWinWarps];
+  uint32_t bstar, rem, nc;
+};
+
+__global__ void __launch_bounds__(kWinThreads, 2)
+topk_rows_win_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int G, int64_t q_pos0, int B,
+                     int k, int32_t* __restrict__ sel, int32_t* __restrict__ sel_count,
+                     int32_t* __restrict__ overflow) {
+  __shared__ WinSmem sm;
+  const int64_t row = blockIdx.x;  // (seq * nq + i) * G + g
+  const int64_t i = (row / G) % nq;
+  const int n = static_cast<int>((q_pos0 + i) / B);
+  const float* srow = scores + row * rpad;
+  int32_t* out = sel + row * k;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (n <= k) {
+    for (int j = tid; j < k; j += kWinThreads) out[j] = j < n ? j : -1;
+    if (tid == 0) {
+      sel_count[row] = n;
+      overflow[row] = 0;
+    }
+    return;
+  }
+  const int nper = (n + kWinThreads - 1) / kWinThreads;  // iterations that hold real candidates
+  float v[kWinPer];
+#pragma unroll
+  for (int e = 0; e < kWinPer; ++e) {
+    const int id = tid + kWinThreads * e;
+    v[e] = (e < nper && id < n) ? __ldcs(srow + id) : -INFINITY;
+  }
+  for (int b = tid; b < kWinWarps * kWinBins; b += kWinThreads) (&sm.wh[0][0])[b] = 0u;
+  if (tid == 0) sm.nc = 0;
+  // row maximum and minimum (over real candidates)
+  float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+  for (int e = 0; e < kWinPer; ++e) {
+    if (e >= nper) break;
+    mx = fmaxf(mx, v[e]);
+    if (tid + kWinThreads * e < n) mn = fminf(mn, v[e]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+  }
+  if (lane == 0) {
+    sm.rmax[warp] = mx;
+    sm.rmin[warp] = mn;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kWinWarps; ++w) {
+    mx = fmaxf(mx, sm.rmax[w]);
+    mn = fminf(mn, sm.rmin[w]);
+  }
+  // bin = floor((max - s) * scale), 0 for the maximum, at most 255 for the minimum
+  const float width = mx - mn;
+  const float scale = width > 0.f ? 255.5f / width : 0.f;
+  auto bin_of = [&](float x) -> int { return min(static_cast<int>((mx - x) * scale), kWinBins - 1); };
+  uint32_t* myh = sm.wh[warp];
+#pragma unroll
+  for (int e = 0; e < kWinPer; ++e) {
+    if (e >= nper) break;
+    if (tid + kWinThreads * e < n) atomicAdd(&myh[bin_of(v[e])], 1u);
+  }
+  __syncthreads();
+  // bin counts from the top; the bin where the running count reaches k
+  if (tid < kWinBins) {
+    uint32_t c = 0;
+#pragma unroll
+    for (int w = 0; w < kWinWarps; ++w) c += sm.wh[w][tid];
+    uint32_t inc = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    if (lane == 31) sm.wsum[warp] = inc;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    uint32_t before = inc - c;
+    for (int w = 0; w < warp; ++w) before += sm.wsum[w];
+    const uint32_t kk = static_cast<uint32_t>(k);
+    if (before < kk && kk <= before + c) {
+      sm.bstar = static_cast<uint32_t>(tid);
+      sm.rem = kk - before;
+    }
+  }
+  __syncthreads();
+  const int bstar = static_cast<int>(sm.bstar);
+  const uint32_t rem = sm.rem;
+  // higher bins straight into the bitmap; the boundary bin gathered
+  // bitmap words past the last iteration hold no candidate
+  if (tid >= nper * kWinWarps) sm.bits[tid] = 0u;
+#pragma unroll
+  for (int e = 0; e < kWinPer; ++e) {
+    if (e >= nper) break;
+    const bool real = tid + kWinThreads * e < n;
+    const int b = real ? bin_of(v[e]) : kWinBins;
+    const uint32_t above = __ballot_sync(0xffffffffu, b < bstar);
+    if (lane == 0) sm.bits[warp + kWinWarps * e] = above;
+    const bool eq = b == bstar;
+    const uint32_t bal = __ballot_sync(0xffffffffu, eq);
+    if (bal) {
+      uint32_t base = 0;
+      if (lane == 0) base = atomicAdd(&sm.nc, static_cast<uint32_t>(__popc(bal)));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      const uint32_t pos = base + __popc(bal & ((1u << lane) - 1u));
+      if (eq && pos < kWinCand) sm.cand[pos] = make_uint2(score_key(v[e]), static_cast<uint32_t>(tid + kWinThreads * e));
+    }
+  }
+  __syncthreads();
+  const uint32_t nc = sm.nc;
+  if (nc > kWinCand) {
+    if (tid == 0) overflow[row] = 1;
+    return;
+  }
+  if (warp == 0) {
+    uint32_t theta = 0, id_cut = 0xFFFFFFFFu;
+    if (nc > rem) warp_select(sm.cand, static_cast<int>(nc), static_cast<int>(rem), sm.wh[0], theta, id_cut);
+    for (uint32_t c = lane; c < nc; c += 32) {
+      const uint2 e = sm.cand[c];
+      if (nc <= rem || kept(e, theta, id_cut)) atomicOr(&sm.bits[e.y >> 5], 1u << (e.y & 31));
+    }
+  }
+  __syncthreads();
+  // ascending readout: thread t owns bitmap word t (ids 32 t .. 32 t + 31)
+  const uint32_t word = sm.bits[tid];
+  const uint32_t cnt = __popc(word);
+  uint32_t inc = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) sm.wsum[warp] = inc;
+  __syncthreads();
+  uint32_t pos = inc - cnt;
+  for (int w = 0; w < warp; ++w) pos += sm.wsum[w];
+  uint32_t wb = word;
+  while (wb) {
+    const int bit = __ffs(wb) - 1;
+    wb &= wb - 1;
+    if (pos < static_cast<uint32_t>(k)) out[pos] = 32 * tid + bit;
+    ++pos;
+  }
+  if (tid == 0) {
+    sel_count[row] = k;
+    overflow[row] = 0;
+  }
+}
+
 }  // namespace sgqa

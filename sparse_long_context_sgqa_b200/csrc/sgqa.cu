@@ -376,11 +376,16 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
   }
   const int nwords = static_cast<int>((std::max<int64_t>(rneed, 1) + 31) / 32);
   const size_t ssmem = (static_cast<size_t>(sgqa::kRows2Warps) * sgqa::kRows2Bins / 2 + 2 * sgqa::kRows2Cand + nwords) * 4;
-  // Long rows (>= 32768 candidates): two passes over the row (histogram, then
-  // gather); rows it cannot finish (boundary-bin overflow) go to the radix
-  // kernel.  Shorter rows: the four-pass radix kernel, whose smaller per-row
-  // set-up wins there (measured at 8K and 128K contexts).
-  if (rneed >= 32768 && ssmem <= 112 * 1024) {
+  // Rows of 2048 .. 16384 candidates: one HBM read into registers, a linear
+  // histogram and an exact boundary-bin select.  Long rows (>= 32768
+  // candidates): two passes over the row (histogram, then gather).  Rows either
+  // cannot finish (boundary-bin overflow) go to the radix kernel, which also
+  // takes the rows in between and short rows (its per-row set-up is smaller).
+  if (rneed >= 2048 && rneed <= sgqa::kWinMaxCand) {
+    sgqa::topk_rows_win_kernel<<<static_cast<unsigned>(rows), sgqa::kWinThreads, 0, st>>>(
+        scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, flags);
+    SGQA_LAUNCH_CHECK("topk_rows_win_kernel");
+  } else if (rneed >= 32768 && ssmem <= 112 * 1024) {
     cudaFuncSetAttribute(sgqa::topk_rows2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
     sgqa::topk_rows2_kernel<<<static_cast<unsigned>(rows), sgqa::kRows2Threads, ssmem, st>>>(
         scores, w.rpad, nq, G, q0, B, p->topk, nwords, sel, sel_count, flags);

@@ -126,6 +126,42 @@ def test_index_topk_parity(cuda_device, case):
     assert ties <= 2 * len(rows)
 
 
+def test_index_topk_exact_ties(cuda_device):
+    """Zero head weights make every score exactly 0: the only valid selection
+    is the k smallest block ids.  Rows of 600..2048 candidates resolve the tie
+    inside one histogram bin; rows of 2049..2903 candidates overflow the
+    boundary buffer and are redone by the radix kernel.  Every other query keeps its
+    weights and is checked against the oracle as usual."""
+    wl = dataclasses.replace(WL["prefill8k"], name="ties", seq_len=24576, topk=512)
+    cache, _ = Hn.make_inputs(wl, cuda_device)
+    q0, nq = 4800, 16384 + 2048  # candidates 600 .. 2903 per query (B = 8)
+    qs = I.make_queries(wl, cuda_device, q0, nq)
+    zero = torch.zeros(nq, dtype=torch.bool, device=cuda_device)
+    zero[::3] = True
+    qs["idx_w"][zero] = 0.0
+    _, codes, keys = Hn.oracle_keys(Hn.to_np(cache["kp"][0]), Hn.to_np(cache["c"][0]), wl.block)
+    store = torch.from_numpy(codes).to(cuda_device)[None].contiguous()
+    p = Hn.params_for(wl)
+    sel = torch.full((1, nq, wl.groups, wl.topk), -7, dtype=torch.int32, device=cuda_device)
+    cnt = torch.full((1, nq, wl.groups), -7, dtype=torch.int32, device=cuda_device)
+    ws = _bd().alloc_workspace(p, 1, nq, q0 + nq, cuda_device)
+    _bd().sgqa_index_topk(p, 1, q0, nq, qs["idx_q"][None].contiguous(), qs["idx_w"][None].contiguous(),
+                          wl.seq_len, store, sel, cnt, ws)
+    _bd().sgqa_check()
+    sel, cnt = sel[0].cpu().numpy(), cnt[0].cpu().numpy()
+    assert np.all(cnt == wl.topk)
+    zero_np = zero.cpu().numpy()
+    assert np.all(sel[zero_np] == np.arange(wl.topk, dtype=np.int32))
+    iq, iw = Hn.to_np(qs["idx_q"]), Hn.to_np(qs["idx_w"])
+    ties = 0
+    rows = [i for i in range(1, nq, 397) if not zero_np[i]] + [nq - 1]
+    for i in rows:
+        for g in range(wl.groups):
+            sc = O.index_scores(iq[i, g], iw[i, g], keys[:(q0 + i) // wl.block])
+            ties += Hn.check_selection(sel[i, g], sc, wl.topk)
+    assert ties <= 2 * len(rows)
+
+
 def _attn_isolated(wl, device, q_pos0, nq, rows, num_seqs=1, groups=None):
     cache, _ = Hn.make_inputs(wl, device, seqs=range(num_seqs))
     qs = [I.make_queries(wl, device, q_pos0, nq, seq=s) for s in range(num_seqs)]
