@@ -333,20 +333,16 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       tc::tmem_ld_wait();
       tc::fence_before();
       tc::mbar_arrive(bar(sm.s_free[b]));
-      // masked raw scores and their max (the scale is positive: it commutes with max)
+      // row max over the attended scores (the scale is positive: it commutes
+      // with max).  Union tiles mask whole blocks: a block the row does not
+      // attend gets the exponent offset -inf below instead of masked scores.
       float bm[8];
       if (j < n_union_tiles) {
-        // one decision per 8-token block
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const bool keep = (bmask >> e) & 1u;
-          bm[e] = -INFINITY;
-#pragma unroll
-          for (int x = 0; x < 8; ++x) {
-            const float v = keep ? __uint_as_float(sr[8 * e + x]) : -INFINITY;
-            sr[8 * e + x] = __float_as_uint(v);
-            bm[e] = fmaxf(bm[e], v);
-          }
+          const float* x = reinterpret_cast<const float*>(&sr[8 * e]);
+          const float mb = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])), fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
+          bm[e] = ((bmask >> e) & 1u) ? mb : -INFINITY;
         }
       } else {
         // current tile: tokens c0 .. c0 + 15, of which the row attends cur_lo .. t
@@ -396,26 +392,30 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
         l = m_l == -INFINITY ? 0.f : l * exp2f(m_l - m_use);
         m_l = m_use;
       }
-      // P = 2^(s * scale - m_use) in BF16 (masked -> 0), packed two tokens per
-      // column; blocks that no row of this warp attends skip their exponentials
+      // P = 2^(s * scale - m_use) in BF16, packed two tokens per column.  A
+      // block the row does not attend has offset -inf (P = 0); blocks no row
+      // of this warp attends skip their exponentials.
       const float neg_m = m_use == -INFINITY ? 0.f : -m_use;
-      float lsum = 0.f;
+      const uint32_t wmask = __reduce_or_sync(0xffffffffu, bmask);
+      float ls[8];
       uint32_t pk[32];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        if (__any_sync(0xffffffffu, (bmask >> e) & 1u)) {
+        ls[e] = 0.f;
+        if ((wmask >> e) & 1u) {
+          const float off = ((bmask >> e) & 1u) ? neg_m : -INFINITY;
+          float pe[8];
 #pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(sr[8 * e + 2 * x]), scale_log2, neg_m));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(sr[8 * e + 2 * x + 1]), scale_log2, neg_m));
-            lsum += p0 + p1;
-            pk[4 * e + x] = pack_bf16x2(p0, p1);
-          }
+          for (int x = 0; x < 8; ++x) pe[x] = fast_exp2(fmaf(__uint_as_float(sr[8 * e + x]), scale_log2, off));
+          ls[e] = ((pe[0] + pe[1]) + (pe[2] + pe[3])) + ((pe[4] + pe[5]) + (pe[6] + pe[7]));
+#pragma unroll
+          for (int x = 0; x < 4; ++x) pk[4 * e + x] = pack_bf16x2(pe[2 * x], pe[2 * x + 1]);
         } else {
 #pragma unroll
           for (int x = 0; x < 4; ++x) pk[4 * e + x] = 0u;
         }
       }
+      const float lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       // P buffer b is free once O += P(j-2) V(j-2) has read it
       if (j >= 2) ok = ok && tc::mbar_wait(bar(sm.pv_done[b]), ((j / 2) - 1) & 1, abort);
       tc::fence_after();

@@ -58,6 +58,27 @@ __device__ __forceinline__ uint32_t mbar_test3(uint32_t b0, uint32_t p0, uint32_
       : "memory");
   return ok;
 }
+// Six completion tests issued back to back; bit i of the result is barrier
+// i's test.
+__device__ __forceinline__ uint32_t mbar_test6(const uint32_t (&b)[6], const uint32_t (&p)[6]) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred q0, q1, q2, q3, q4, q5;\n .reg .b32 r0, r1, r2, r3, r4, r5;\n"
+      " mbarrier.test_wait.parity.shared::cta.b64 q0, [%1], %2;\n"
+      " mbarrier.test_wait.parity.shared::cta.b64 q1, [%3], %4;\n"
+      " mbarrier.test_wait.parity.shared::cta.b64 q2, [%5], %6;\n"
+      " mbarrier.test_wait.parity.shared::cta.b64 q3, [%7], %8;\n"
+      " mbarrier.test_wait.parity.shared::cta.b64 q4, [%9], %10;\n"
+      " mbarrier.test_wait.parity.shared::cta.b64 q5, [%11], %12;\n"
+      " selp.u32 r0, 1, 0, q0;\n selp.u32 r1, 2, 0, q1;\n selp.u32 r2, 4, 0, q2;\n"
+      " selp.u32 r3, 8, 0, q3;\n selp.u32 r4, 16, 0, q4;\n selp.u32 r5, 32, 0, q5;\n"
+      " or.b32 r0, r0, r1;\n or.b32 r2, r2, r3;\n or.b32 r4, r4, r5;\n or.b32 r0, r0, r2;\n or.b32 %0, r0, r4;\n}"
+      : "=r"(ok)
+      : "r"(b[0]), "r"(p[0]), "r"(b[1]), "r"(p[1]), "r"(b[2]), "r"(p[2]), "r"(b[3]), "r"(p[3]), "r"(b[4]),
+        "r"(p[4]), "r"(b[5]), "r"(p[5])
+      : "memory");
+  return ok;
+}
 // Wait for the phase with the given parity to complete; gives up after
 // kWaitLimitNs, records kDevTimeout and returns false.  `abort` (shared)
 // short-cuts every later wait of the CTA once one has given up.
