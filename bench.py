@@ -40,6 +40,18 @@ METRIC = {
 }
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+# dominant kernel, from one ncu capture of the current kernels (the files under
+# profiles/ give the commands and figures); None where no capture of the
+# current kernel exists.
+TRAFFIC = {
+    "prefill8k": 396573696,      # attn_tc_kernel, one launch (one 8192-query chunk)
+    "prefill128k": 2100310640,   # attn_tc_kernel, mean over the 16 chunk launches of one step
+    "prefill1m": None,
+    "decode": 236933632,         # attn_decode_tma_kernel, one launch (16 sequences)
+}
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -215,14 +227,18 @@ def cuda_arm(args, wl, rank, world, local_rank):
         else:
             model.prefill(q["q"], q["idx_q"], q["idx_w"], out, sel, cnt, q_pos0=wl.q_start)
 
+    from sparse_long_context_sgqa_b200 import binding as Bd
     graph = None
+    graph_launches = 0
     if wl.nq <= 32 and not args.no_graph:
         # a decode step is a handful of short kernels: replay it as one CUDA graph
         eager_step()
         torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()
+        n0 = Bd.launch_count()
         with torch.cuda.graph(graph):
             eager_step()
+        graph_launches = Bd.launch_count() - n0
         torch.cuda.synchronize()
 
     def step():
@@ -242,19 +258,22 @@ def cuda_arm(args, wl, rank, world, local_rank):
     sampler = ClockSampler(local_rank) if rank == 0 else None
     st = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_launch0 = Bd.launch_count()
     e0.record(st)
     for _ in range(args.steps):
         step()
     e1.record(st)
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
+    # kernels launched in the timed region: counted by the library (a graph
+    # replay launches the kernels captured once per step)
+    gpu_launches = graph_launches * args.steps if graph is not None else Bd.launch_count() - n_launch0
     elapsed = e0.elapsed_time(e1)
     if world > 1:
         t = torch.tensor([elapsed], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         elapsed = float(t.item())
         torch.distributed.barrier()
-    from sparse_long_context_sgqa_b200 import binding as Bd
     Bd.sgqa_check()
     ms_step = elapsed / args.steps
     tokens_per_step = wl.nq * wl.num_seqs
@@ -267,17 +286,25 @@ def cuda_arm(args, wl, rank, world, local_rank):
 
     peaks = load_peaks()
     per_launch_ms = {k: v / max(1, work["launches"]) for k, v in ms_stage.items()}
+    traffic = TRAFFIC.get(wl.name)
     if wl.nq <= 32:
         achieved = work["attn_bytes"] / work["launches"] / (per_launch_ms["attention"] / 1e3) / 1e9
-        roof = {"kernel": "sparse attention (decode gather)", "bound": "hbm", "achieved": achieved,
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None}
+        roof = {"kernel": "sparse attention (decode gather: attn_decode_tma_kernel)", "bound": "hbm",
+                "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                "traffic": traffic}
     else:
         dom = "attention" if ms_stage["attention"] >= ms_stage["index"] else "index"
         fl = work["attn_flops"] if dom == "attention" else work["index_flops"]
         achieved = fl / work["launches"] / (per_launch_ms[dom] / 1e3) / 1e12
         pk = peaks["bf16_tflops_sustained"]
-        roof = {"kernel": f"sparse {dom} stage", "bound": "tensor", "achieved": achieved, "peak": pk,
-                "unit": "TFLOP/s", "frac": achieved / pk, "traffic": None}
+        kname = "sparse attention stage (attn_plan_kernel + attn_tc_kernel)" if dom == "attention" else \
+            "index stage (score + top-k kernels)"
+        roof = {"kernel": kname, "bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
+                "frac": achieved / pk, "traffic": traffic if dom == "attention" else None}
+        if dom == "attention" and work.get("union"):
+            # the tensor cores run QK^T and PV over each 8-query unit's block union
+            infl = work["union"]["inflation"]
+            roof["mma_work"] = {"tflops": achieved * infl, "frac": achieved * infl / pk, "union_inflation": infl}
     roof["peak_source"] = peaks["source"]
 
     res = {
@@ -293,17 +320,12 @@ def cuda_arm(args, wl, rank, world, local_rank):
         "stage_tflops": {"index": work["index_flops"] / (ms_stage["index"] / 1e3) / 1e12 if ms_stage["index"] else None,
                          "attention": work["attn_flops"] / (ms_stage["attention"] / 1e3) / 1e12},
         "roofline": roof,
-        "gpu_launches": args.steps * n_chunks * launches_per_call(wl),
+        "gpu_launches": gpu_launches,
         "cuda_graph": graph is not None,
         "clocks": clocks,
         "e2e": e2e,
     }
     return res
-
-
-def launches_per_call(wl):
-    # merge, widen, score, top-k, then plan + attention (prefill) or attention + combine (decode)
-    return 6
 
 
 def e2e_measure(wl, model, q, out, dev, steps=2):

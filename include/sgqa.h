@@ -195,6 +195,14 @@ const char* sgqa_last_error(void);
 /* Library version string. */
 const char* sgqa_version(void);
 
+/* Number of kernels the library has launched in this process since it was
+ * loaded (all host threads and devices together); a call that fails before a
+ * launch adds nothing.  Launches issued while a stream is being captured into
+ * a CUDA graph are counted once, at capture: replays of the graph add nothing.
+ * Meant for counting GPU work, e.g. kernels per call in a benchmark.  Pure host
+ * read; never fails. */
+uint64_t sgqa_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -25,7 +25,8 @@ STATUS = {0: "SGQA_OK", 1: "SGQA_ERR_INVALID_ARGUMENT", 2: "SGQA_ERR_UNSUPPORTED
           3: "SGQA_ERR_WORKSPACE", 4: "SGQA_ERR_CUDA", 5: "SGQA_ERR_TIMEOUT", 6: "SGQA_ERR_DEVICE"}
 
 EXPORTED = ["sgqa_workspace_size", "sgqa_merge_blocks", "sgqa_index_topk", "sgqa_sparse_attn",
-            "sgqa_forward", "sgqa_sparse_attn_noalloc", "sgqa_check", "sgqa_last_error", "sgqa_version"]
+            "sgqa_forward", "sgqa_sparse_attn_noalloc", "sgqa_check", "sgqa_last_error", "sgqa_version",
+            "sgqa_launch_count"]
 
 
 class SgqaError(RuntimeError):
@@ -71,7 +72,8 @@ _lib.sgqa_sparse_attn_noalloc.argtypes = [_P, _i64, _i64, _i64, _vp, _i64, _i64,
 _lib.sgqa_check.argtypes = [_vp]
 _lib.sgqa_last_error.restype = ctypes.c_char_p
 _lib.sgqa_version.restype = ctypes.c_char_p
-for _f in EXPORTED[:-2]:
+_lib.sgqa_launch_count.restype = ctypes.c_uint64
+for _f in EXPORTED[:-3]:
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -92,6 +94,11 @@ def _stream(stream):
 
 def version() -> str:
     return _lib.sgqa_version().decode()
+
+
+def launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(_lib.sgqa_launch_count())
 
 
 def sgqa_workspace_size(p: Params, num_seqs: int, nq: int, max_ctx: int) -> int:

@@ -40,10 +40,14 @@ sgqa_status cuda_fail(cudaError_t e, const char* what) {
   return fail(SGQA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+// Kernels launched by this library (all threads), read by sgqa_launch_count().
+std::atomic<uint64_t> g_launches{0};
+
 #define SGQA_LAUNCH_CHECK(what)                           \
   do {                                                    \
     cudaError_t e_ = cudaGetLastError();                  \
     if (e_ != cudaSuccess) return cuda_fail(e_, what);    \
+    g_launches.fetch_add(1, std::memory_order_relaxed);   \
   } while (0)
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -532,6 +536,8 @@ sgqa_status noalloc_scratch(void** ptr) {
 extern "C" {
 
 const char* sgqa_version(void) { return "sgqa-b200 0.1 (sm_100a)"; }
+
+uint64_t sgqa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char* sgqa_last_error(void) { return g_err.c_str(); }
 
