@@ -24,6 +24,7 @@
 namespace sgqa {
 
 constexpr int kIdxThreads = 192;
+constexpr int kScoreTcThreads = 320;  // score kernel: producer, MMA, 8 epilogue warps
 constexpr int kIdxStages = 4;
 constexpr int kIdxCand = 128;    // candidates per tile (MMA M)
 constexpr int kIdxCols = 256;    // (query, head) columns per CTA (MMA N)
@@ -376,7 +377,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_constan
 // epilogue that writes I[t, g, r] as FP32 rows (one 128-byte coalesced store
 // per warp and query).  topk_rows_kernel then selects from the rows.
 template <int H>
-__global__ void __launch_bounds__(kIdxThreads, 1)
+__global__ void __launch_bounds__(kScoreTcThreads, 1)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_constant__ CUtensorMap qmap,
                       const float* __restrict__ idx_w, float* __restrict__ scores, int64_t nq, int G,
                       int64_t q_pos0, int B, int64_t rpad) {
@@ -406,12 +407,12 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(bar(sm.acc_full[b]), 1);
-      tc::mbar_init(bar(sm.acc_empty[b]), 128);
+      tc::mbar_init(bar(sm.acc_empty[b]), 256);
     }
     tc::mbar_init(bar(sm.drain), 1);
     tc::mbar_fence_init();
   }
-  for (int c = threadIdx.x; c < kIdxCols; c += kIdxThreads) {
+  for (int c = threadIdx.x; c < kIdxCols; c += kScoreTcThreads) {
     const int qs = c / H;
     sm.w[c] = qs < nq_here ? idx_w[((seq * nq + q0 + qs) * G + g) * H + (c % H)] : 0.f;
   }
@@ -421,59 +422,69 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
   const uint32_t tmem = sm.tmem;
   if (n_tiles > 0) {
     if (warp == 0) {
-      if (lane == 0) {
+      // producer: queries once, then the candidate tiles through the ring (converged warp, one elected issuer)
+      if (tc::elect_one()) {
         tc::prefetch_tmap(&keymap);
         tc::prefetch_tmap(&qmap);
         tc::mbar_expect_tx(bar(sm.b_full), kIdxCols * 128);
         tc::tma_load_4d(smem_u32(&sm.b[0]), &qmap, 0, 0, g, static_cast<int32_t>(seq * nq + q0), bar(sm.b_full));
-        int issued = 0;
-        for (int c = 0; c < n_tiles; ++c) {
-          const int s = c % kIdxStages;
-          if (c >= kIdxStages && !tc::mbar_wait(bar(sm.a_empty[s]), ((c / kIdxStages) - 1) & 1, abort)) break;
+      }
+      __syncwarp();
+      int issued = 0;
+      for (int c = 0; c < n_tiles; ++c) {
+        const int s = c % kIdxStages;
+        if (c >= kIdxStages && !tc::warp_wait(bar(sm.a_empty[s]), ((c / kIdxStages) - 1) & 1, abort)) break;
+        if (tc::elect_one()) {
           tc::mbar_expect_tx(bar(sm.a_full[s]), kIdxCand * 128);
           tc::tma_load_2d(smem_u32(&sm.a[s][0]), &keymap, 0, static_cast<int32_t>(seq * rpad + c * kIdxCand),
                           bar(sm.a_full[s]));
-          issued = c + 1;
         }
-        if (*abort) {
-          const uint64_t t0 = globaltimer_ns();
-          while (!tc::mbar_try(bar(sm.b_full), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-          }
-          for (int c = issued > kIdxStages ? issued - kIdxStages : 0; c < issued; ++c) {
-            const uint64_t t1 = globaltimer_ns();
-            while (!tc::mbar_try(bar(sm.a_full[c % kIdxStages]), (c / kIdxStages) & 1) &&
-                   globaltimer_ns() - t1 < kWaitLimitNs) {
-            }
+        __syncwarp();
+        issued = c + 1;
+      }
+      if (*abort) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!tc::mbar_try(bar(sm.b_full), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+        }
+        for (int c = issued > kIdxStages ? issued - kIdxStages : 0; c < issued; ++c) {
+          const uint64_t t1 = globaltimer_ns();
+          while (!tc::mbar_try(bar(sm.a_full[c % kIdxStages]), (c / kIdxStages) & 1) &&
+                 globaltimer_ns() - t1 < kWaitLimitNs) {
           }
         }
       }
     } else if (warp == 1) {
-      if (lane == 0) {
-        const uint32_t idesc = tc::idesc_bf16(kIdxCand, kIdxCols, false);
-        bool ok = tc::mbar_wait(bar(sm.b_full), 0, abort);
-        for (int c = 0; ok && c < n_tiles; ++c) {
-          const int s = c % kIdxStages, ab = c & 1;
-          if (!tc::mbar_wait(bar(sm.a_full[s]), (c / kIdxStages) & 1, abort)) { ok = false; break; }
-          if (c >= 2 && !tc::mbar_wait(bar(sm.acc_empty[ab]), ((c >> 1) - 1) & 1, abort)) { ok = false; break; }
-          tc::fence_after();
+      // MMA issuer (converged warp, one elected issuer per tile)
+      const uint32_t idesc = tc::idesc_bf16(kIdxCand, kIdxCols, false);
+      const uint64_t da0 = tc::sdesc_sw128(smem_u32(&sm.a[0][0]), 16, 1024);
+      const uint64_t db0 = tc::sdesc_sw128(smem_u32(&sm.b[0]), 16, 1024);
+      constexpr uint32_t kStageUnits = kIdxCand * 128 / 16;  // one key stage in 16-byte units
+      bool ok = tc::warp_wait(bar(sm.b_full), 0, abort);
+      for (int c = 0; ok && c < n_tiles; ++c) {
+        const int s = c % kIdxStages, ab = c & 1;
+        if (!tc::warp_wait(bar(sm.a_full[s]), (c / kIdxStages) & 1, abort)) { ok = false; break; }
+        if (c >= 2 && !tc::warp_wait(bar(sm.acc_empty[ab]), ((c >> 1) - 1) & 1, abort)) { ok = false; break; }
+        tc::fence_after();
+        if (tc::elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t a = tc::sdesc_sw128(smem_u32(&sm.a[s][0]) + kk * 32, 16, 1024);
-            const uint64_t b = tc::sdesc_sw128(smem_u32(&sm.b[0]) + kk * 32, 16, 1024);
-            tc::mma_f16(tmem + ab * kIdxCols, a, b, idesc, kk > 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < 4; ++kk)  // +32 B per 16 dims in both operands
+            tc::mma_f16(tmem + ab * kIdxCols, da0 + s * kStageUnits + 2 * kk, db0 + 2 * kk, idesc, kk > 0 ? 1u : 0u);
           tc::mma_commit(bar(sm.a_empty[s]));
           tc::mma_commit(bar(sm.acc_full[ab]));
         }
-        if (!ok) {
-          tc::mma_commit(bar(sm.drain));
-          const uint64_t t0 = globaltimer_ns();
-          while (!tc::mbar_try(bar(sm.drain), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-          }
+        __syncwarp();
+      }
+      if (!ok) {
+        if (tc::elect_one()) tc::mma_commit(bar(sm.drain));
+        __syncwarp();
+        const uint64_t t0 = globaltimer_ns();
+        while (!tc::mbar_try(bar(sm.drain), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
         }
       }
     } else {
+      // epilogue: eight warps, two per TMEM lane quadrant, each taking half of the 256 columns
       const int quad = warp & 3;
+      const int half = (warp - 2) >> 2;
       const int m = quad * 32 + lane;
       const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
       float* srow0 = scores + ((seq * nq + q0) * G + g) * rpad;
@@ -484,12 +495,13 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
         tc::fence_after();
         const int64_t r = static_cast<int64_t>(c) * kIdxCand + m;
 #pragma unroll
-        for (int ch2 = 0; ch2 < kIdxCols / 64; ++ch2) {
+        for (int h2 = 0; h2 < kIdxCols / 128; ++h2) {
+          const int ch2 = half * (kIdxCols / 128) + h2;
           uint32_t d2[64];
           tc::tmem_ld32(tmem + ab * kIdxCols + 64 * ch2 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&d2[0]));
           tc::tmem_ld32(tmem + ab * kIdxCols + 64 * ch2 + 32 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&d2[32]));
           tc::tmem_ld_wait();
-          if (ch2 == kIdxCols / 64 - 1) {
+          if (h2 == kIdxCols / 128 - 1) {
             tc::fence_before();
             tc::mbar_arrive(bar(sm.acc_empty[ab]));
           }

@@ -340,11 +340,11 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
     const size_t smem = sizeof(sgqa::IndexTcSmem) + 1024;
     if (H == 8) {
       cudaFuncSetAttribute(sgqa::index_score_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      sgqa::index_score_tc_kernel<8><<<static_cast<unsigned>(grid), sgqa::kIdxThreads, smem, st>>>(
+      sgqa::index_score_tc_kernel<8><<<static_cast<unsigned>(grid), sgqa::kScoreTcThreads, smem, st>>>(
           km, qm, idx_w, scores, nq, G, q0, B, w.rpad);
     } else {
       cudaFuncSetAttribute(sgqa::index_score_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      sgqa::index_score_tc_kernel<4><<<static_cast<unsigned>(grid), sgqa::kIdxThreads, smem, st>>>(
+      sgqa::index_score_tc_kernel<4><<<static_cast<unsigned>(grid), sgqa::kScoreTcThreads, smem, st>>>(
           km, qm, idx_w, scores, nq, G, q0, B, w.rpad);
     }
     SGQA_LAUNCH_CHECK("index_score_tc_kernel");
