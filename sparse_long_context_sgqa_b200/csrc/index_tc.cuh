@@ -373,13 +373,33 @@ index_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_constan
   }
 }
 
-// Scores only: the same TMA/tcgen05 pipeline as index_tc_kernel, with an
-// epilogue that writes I[t, g, r] as FP32 rows (one 128-byte coalesced store
-// per warp and query).  topk_rows_kernel then selects from the rows.
-template <int H>
+// Indexer scores I[t, g, r] on the tensor cores: the same TMA/tcgen05 pipeline
+// as index_tc_kernel (one CTA = 256 (query, head) columns of one group, all
+// candidates in tiles of 128), with one of three epilogues:
+//   kScoreRows    every score as FP32 rows [row, rpad] (one 128-byte store per
+//                 warp and query); a top-k kernel then selects from the rows;
+//   kScoreSample  only every kSampleStride-th candidate tile, compacted into
+//                 rows [row, ld] (for the per-row threshold estimate);
+//   kScoreFilter  every score, but only those at or above the row's threshold
+//                 are kept, as (order-preserving key, block id) pairs in the
+//                 row's staging list; the row's count (which may exceed the
+//                 list's capacity) is written at the end.  A CTA owns its rows,
+//                 so the counters live in shared memory.
+constexpr int kScoreRows = 0, kScoreSample = 1, kScoreFilter = 2;
+constexpr int kSampleStride = 16;
+struct ScoreOut {
+  float* scores;            // kScoreRows: [rows, ld] = [rows, rpad]; kScoreSample: [rows, ld]
+  int64_t ld;
+  const float* thr;         // kScoreFilter: per-row threshold
+  uint2* staging;           // kScoreFilter: [rows, cap] (key, id)
+  int32_t* staged;          // kScoreFilter: [rows] scores at or above the threshold
+  int cap;
+};
+
+template <int H, int MODE>
 __global__ void __launch_bounds__(kScoreTcThreads, 1)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_constant__ CUtensorMap qmap,
-                      const float* __restrict__ idx_w, float* __restrict__ scores, int64_t nq, int G,
+                      const float* __restrict__ idx_w, ScoreOut o, int64_t nq, int G,
                       int64_t q_pos0, int B, int64_t rpad) {
   constexpr int Q = kIdxCols / H;
   extern __shared__ uint8_t smem_raw[];
@@ -396,6 +416,9 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
   const int nq_here = static_cast<int>(nq - q0 < Q ? nq - q0 : Q);
   const int64_t ncand_max = (q_pos0 + q0 + nq_here - 1) / B;
   const int n_tiles = static_cast<int>((ncand_max + kIdxCand - 1) / kIdxCand);
+  // tiles this launch computes (the sample takes every kSampleStride-th) and the tile behind loop index c
+  const int n_loop = MODE == kScoreSample ? (n_tiles + kSampleStride - 1) / kSampleStride : n_tiles;
+  auto tile_of = [](int c) { return MODE == kScoreSample ? c * kSampleStride : c; };
   volatile int* abort = &sm.abort;
   auto bar = [](uint64_t& b) { return smem_u32(&b); };
   if (threadIdx.x == 0) {
@@ -416,6 +439,14 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
     const int qs = c / H;
     sm.w[c] = qs < nq_here ? idx_w[((seq * nq + q0 + qs) * G + g) * H + (c % H)] : 0.f;
   }
+  if (MODE == kScoreFilter) {
+    for (int qs = threadIdx.x; qs < Q; qs += kScoreTcThreads) {
+      const bool real = qs < nq_here;
+      sm.cnt[qs] = 0;
+      sm.thr[qs] = __float_as_uint(real ? o.thr[(seq * nq + q0 + qs) * G + g] : INFINITY);
+      sm.ncand[qs] = real ? static_cast<int>((q_pos0 + q0 + qs) / B) : 0;
+    }
+  }
   if (warp == 1) tc::tmem_alloc(smem_u32(&sm.tmem), 512);
   __syncthreads();
   tc::fence_after();
@@ -431,12 +462,13 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
       }
       __syncwarp();
       int issued = 0;
-      for (int c = 0; c < n_tiles; ++c) {
+      for (int c = 0; c < n_loop; ++c) {
         const int s = c % kIdxStages;
         if (c >= kIdxStages && !tc::warp_wait(bar(sm.a_empty[s]), ((c / kIdxStages) - 1) & 1, abort)) break;
         if (tc::elect_one()) {
           tc::mbar_expect_tx(bar(sm.a_full[s]), kIdxCand * 128);
-          tc::tma_load_2d(smem_u32(&sm.a[s][0]), &keymap, 0, static_cast<int32_t>(seq * rpad + c * kIdxCand),
+          tc::tma_load_2d(smem_u32(&sm.a[s][0]), &keymap, 0,
+                          static_cast<int32_t>(seq * rpad + static_cast<int64_t>(tile_of(c)) * kIdxCand),
                           bar(sm.a_full[s]));
         }
         __syncwarp();
@@ -460,7 +492,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
       const uint64_t db0 = tc::sdesc_sw128(smem_u32(&sm.b[0]), 16, 1024);
       constexpr uint32_t kStageUnits = kIdxCand * 128 / 16;  // one key stage in 16-byte units
       bool ok = tc::warp_wait(bar(sm.b_full), 0, abort);
-      for (int c = 0; ok && c < n_tiles; ++c) {
+      for (int c = 0; ok && c < n_loop; ++c) {
         const int s = c % kIdxStages, ab = c & 1;
         if (!tc::warp_wait(bar(sm.a_full[s]), (c / kIdxStages) & 1, abort)) { ok = false; break; }
         if (c >= 2 && !tc::warp_wait(bar(sm.acc_empty[ab]), ((c >> 1) - 1) & 1, abort)) { ok = false; break; }
@@ -487,13 +519,15 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
       const int half = (warp - 2) >> 2;
       const int m = quad * 32 + lane;
       const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-      float* srow0 = scores + ((seq * nq + q0) * G + g) * rpad;
-      const int64_t qstride = static_cast<int64_t>(G) * rpad;
-      for (int c = 0; c < n_tiles; ++c) {
+      const int64_t row0 = (seq * nq + q0) * G + g;  // row of query slot 0; slot qs is row0 + qs * G
+      // the CTA's smallest candidate count: tiles below it need no per-row bound check
+      const int64_t ncand_min = (q_pos0 + q0) / B;
+      for (int c = 0; c < n_loop; ++c) {
         const int ab = c & 1;
         if (!tc::mbar_wait(bar(sm.acc_full[ab]), (c >> 1) & 1, abort)) break;
         tc::fence_after();
-        const int64_t r = static_cast<int64_t>(c) * kIdxCand + m;
+        const int64_t r = static_cast<int64_t>(tile_of(c)) * kIdxCand + m;  // candidate block id
+        const bool tail = static_cast<int64_t>(tile_of(c) + 1) * kIdxCand > ncand_min;
 #pragma unroll
         for (int h2 = 0; h2 < kIdxCols / 128; ++h2) {
           const int ch2 = half * (kIdxCols / 128) + h2;
@@ -504,6 +538,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
           if (h2 == kIdxCols / 128 - 1) {
             tc::fence_before();
             tc::mbar_arrive(bar(sm.acc_empty[ab]));
+          }
+          float thr_q[64 / H];
+          if (MODE == kScoreFilter) {
+#pragma unroll
+            for (int qq = 0; qq < 64 / H; ++qq) thr_q[qq] = __uint_as_float(sm.thr[ch2 * (64 / H) + qq]);
           }
 #pragma unroll
           for (int qq = 0; qq < 64 / H; ++qq) {
@@ -518,11 +557,32 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
             float acc = 0.f;
 #pragma unroll
             for (int i = 0; i < H; ++i) acc = fmaf(wv[i], fmaxf(__uint_as_float(d2[qq * H + i]), 0.f), acc);
-            if (qs < nq_here) srow0[qs * qstride + r] = acc;
+            const int64_t row = row0 + static_cast<int64_t>(qs) * G;
+            if (MODE == kScoreRows) {
+              if (qs < nq_here) o.scores[row * o.ld + r] = acc;
+            } else if (MODE == kScoreSample) {
+              if (qs < nq_here) o.scores[row * o.ld + static_cast<int64_t>(c) * kIdxCand + m] = acc;
+            } else {
+              // keep the score if it reaches the row's threshold (rows past the
+              // call's queries have threshold +inf)
+              bool pass = acc >= thr_q[qq];
+              if (tail) pass = pass && r < sm.ncand[qs];
+              if (pass) {
+                const int pos = atomicAdd(&sm.cnt[qs], 1);
+                if (pos < o.cap) o.staging[row * o.cap + pos] = make_uint2(score_key(acc), static_cast<uint32_t>(r));
+              }
+            }
           }
         }
       }
+      if (MODE == kScoreFilter) {
+        asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight epilogue warps
+        if (warp == 2)
+          for (int qs = lane; qs < nq_here; qs += 32) o.staged[row0 + static_cast<int64_t>(qs) * G] = sm.cnt[qs];
+      }
     }
+  } else if (MODE == kScoreFilter && warp == 2) {
+    for (int qs = lane; qs < nq_here; qs += 32) o.staged[((seq * nq + q0 + qs) * G + g)] = 0;
   }
   tc::fence_before();
   __syncthreads();
@@ -909,6 +969,301 @@ topk_rows_win_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq,
   if (tid == 0) {
     sel_count[row] = k;
     overflow[row] = 0;
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// Filtered selection for long rows (no FP32 score rows in HBM).  A sample of
+// the scores (every kSampleStride-th candidate tile) gives each row a
+// threshold below its kThrRank-th largest sampled score, so about
+// kThrRank * kSampleStride candidates are expected to reach it; the full
+// score pass then keeps only the (key, id) pairs at or above the threshold.
+// The selection stays exact: every candidate at or above the threshold is in
+// the list, so if at least k are, the k largest are among them.  A row with
+// fewer than k or more than kFilterCap kept entries is flagged and redone from
+// recomputed scores by the radix kernel.
+// ---------------------------------------------------------------------------
+constexpr int kThrRank = 64;
+constexpr int kFilterCap = 4096;
+constexpr int kThrThreads = 256;
+constexpr int kThrPer = 32;  // samples per thread: rows of up to 131072 candidates
+
+__global__ void __launch_bounds__(kThrThreads)
+index_threshold_kernel(const float* __restrict__ sample, int64_t ld, int64_t nq, int G, int64_t q_pos0, int B,
+                       float* __restrict__ thr) {
+  __shared__ uint32_t wh[kThrThreads / 32][256];
+  __shared__ float rmax[kThrThreads / 32], rmin[kThrThreads / 32];
+  __shared__ uint32_t wsum[kThrThreads / 32];
+  __shared__ int s_bstar;
+  const int64_t row = blockIdx.x;
+  const int64_t i = (row / G) % nq;
+  const int64_t n = (q_pos0 + i) / B;
+  const float* srow = sample + row * ld;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // sample entry j = c * 128 + m is candidate (c * kSampleStride) * 128 + m
+  auto cand_of = [](int j) -> int64_t { return static_cast<int64_t>(j / kIdxCand) * kSampleStride * kIdxCand + j % kIdxCand; };
+  const int nsamp_tiles = static_cast<int>(((n + kIdxCand - 1) / kIdxCand + kSampleStride - 1) / kSampleStride);
+  const int nj = min(nsamp_tiles * kIdxCand, kThrThreads * kThrPer);
+  float v[kThrPer];
+  int nvalid = 0;
+#pragma unroll
+  for (int e = 0; e < kThrPer; ++e) {
+    const int j = tid + kThrThreads * e;
+    const bool ok = j < nj && cand_of(j) < n;
+    v[e] = ok ? srow[j] : -INFINITY;
+    nvalid += ok;
+  }
+  for (int b = tid; b < (kThrThreads / 32) * 256; b += kThrThreads) (&wh[0][0])[b] = 0u;
+  float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+  for (int e = 0; e < kThrPer; ++e) {
+    mx = fmaxf(mx, v[e]);
+    if (v[e] != -INFINITY) mn = fminf(mn, v[e]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    nvalid += __shfl_xor_sync(0xffffffffu, nvalid, o);
+  }
+  if (lane == 0) {
+    rmax[warp] = mx;
+    rmin[warp] = mn;
+    wsum[warp] = static_cast<uint32_t>(nvalid);
+  }
+  __syncthreads();
+  int total = 0;
+#pragma unroll
+  for (int w = 0; w < kThrThreads / 32; ++w) {
+    mx = fmaxf(mx, rmax[w]);
+    mn = fminf(mn, rmin[w]);
+    total += static_cast<int>(wsum[w]);
+  }
+  if (total <= kThrRank) {  // too few samples to estimate: keep everything
+    if (tid == 0) thr[row] = -INFINITY;
+    return;
+  }
+  const float width = mx - mn;
+  const float scale = width > 0.f ? 255.5f / width : 0.f;
+  auto bin_of = [&](float x) -> int { return min(static_cast<int>((mx - x) * scale), 255); };
+#pragma unroll
+  for (int e = 0; e < kThrPer; ++e)
+    if (v[e] != -INFINITY) atomicAdd(&wh[warp][bin_of(v[e])], 1u);
+  __syncthreads();
+  {
+    uint32_t c = 0;
+#pragma unroll
+    for (int w = 0; w < kThrThreads / 32; ++w) c += wh[w][tid];  // tid < 256: one bin per thread
+    uint32_t inc = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    __syncthreads();
+    if (lane == 31) wsum[warp] = inc;
+    __syncthreads();
+    uint32_t before = inc - c;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    if (before < static_cast<uint32_t>(kThrRank) && static_cast<uint32_t>(kThrRank) <= before + c) s_bstar = tid;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    // every sample of bin b* (and above) lies strictly above mx - (b* + 1) / scale
+    float t = scale > 0.f ? mx - static_cast<float>(s_bstar + 1) / scale : mx;
+    t -= fabsf(t) * 1e-6f + 1e-30f;
+    thr[row] = t;
+  }
+}
+
+// Exact top-k of a row's staged (key, id) list; ascending ids.  Rows with too
+// few or too many kept entries are flagged for the fallback.
+constexpr int kStagedThreads = 256;
+constexpr int kStagedPer = kFilterCap / kStagedThreads;  // 16
+
+__global__ void __launch_bounds__(kStagedThreads)
+topk_staged_kernel(const uint2* __restrict__ staging, const int32_t* __restrict__ staged, int64_t nq, int G,
+                   int64_t q_pos0, int B, int k, int cap, int nwords_max, int32_t* __restrict__ sel,
+                   int32_t* __restrict__ sel_count, int32_t* __restrict__ flags) {
+  extern __shared__ uint32_t dyn[];
+  uint2* cand = reinterpret_cast<uint2*>(dyn);                 // [kFilterCap]
+  uint32_t* bits = dyn + 2 * kFilterCap;                       // [nwords_max]
+  __shared__ uint32_t wh[kStagedThreads / 32][256];
+  __shared__ float rmax[kStagedThreads / 32], rmin[kStagedThreads / 32];
+  __shared__ uint32_t wsum[kStagedThreads / 32];
+  __shared__ uint32_t s_bstar, s_rem, s_nc;
+  const int64_t row = blockIdx.x;
+  const int64_t i = (row / G) % nq;
+  const int n = static_cast<int>((q_pos0 + i) / B);
+  int32_t* out = sel + row * k;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (n <= k) {
+    for (int j = tid; j < k; j += kStagedThreads) out[j] = j < n ? j : -1;
+    if (tid == 0) {
+      sel_count[row] = n;
+      flags[row] = 0;
+    }
+    return;
+  }
+  const int cnt = staged[row];
+  if (cnt < k || cnt > cap) {
+    if (tid == 0) flags[row] = 1;
+    return;
+  }
+  const uint2* list = staging + row * static_cast<int64_t>(cap);
+  const int nw = (n + 31) / 32;
+  for (int w = tid; w < nw; w += kStagedThreads) bits[w] = 0u;
+  for (int b = tid; b < (kStagedThreads / 32) * 256; b += kStagedThreads) (&wh[0][0])[b] = 0u;
+  if (tid == 0) s_nc = 0;
+  uint2 e[kStagedPer];
+  float v[kStagedPer];
+  float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+  for (int x = 0; x < kStagedPer; ++x) {
+    const int j = tid + kStagedThreads * x;
+    e[x] = j < cnt ? list[j] : make_uint2(0u, 0xFFFFFFFFu);
+    v[x] = j < cnt ? key_score(e[x].x) : -INFINITY;
+    mx = fmaxf(mx, v[x]);
+    if (j < cnt) mn = fminf(mn, v[x]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+  }
+  if (lane == 0) {
+    rmax[warp] = mx;
+    rmin[warp] = mn;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kStagedThreads / 32; ++w) {
+    mx = fmaxf(mx, rmax[w]);
+    mn = fminf(mn, rmin[w]);
+  }
+  const float width = mx - mn;
+  const float scale = width > 0.f ? 255.5f / width : 0.f;
+  auto bin_of = [&](float x) -> int { return min(static_cast<int>((mx - x) * scale), 255); };
+#pragma unroll
+  for (int x = 0; x < kStagedPer; ++x)
+    if (tid + kStagedThreads * x < cnt) atomicAdd(&wh[warp][bin_of(v[x])], 1u);
+  __syncthreads();
+  {
+    uint32_t c = 0;
+#pragma unroll
+    for (int w = 0; w < kStagedThreads / 32; ++w) c += wh[w][tid];
+    uint32_t inc = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    if (lane == 31) wsum[warp] = inc;
+    __syncthreads();
+    uint32_t before = inc - c;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    const uint32_t kk = static_cast<uint32_t>(k);
+    if (before < kk && kk <= before + c) {
+      s_bstar = static_cast<uint32_t>(tid);
+      s_rem = kk - before;
+    }
+  }
+  __syncthreads();
+  const int bstar = static_cast<int>(s_bstar);
+  const uint32_t rem = s_rem;
+  // higher bins into the bitmap, the boundary bin gathered
+#pragma unroll
+  for (int x = 0; x < kStagedPer; ++x) {
+    if (tid + kStagedThreads * x >= cnt) continue;
+    const int b = bin_of(v[x]);
+    if (b < bstar) {
+      atomicOr(&bits[e[x].y >> 5], 1u << (e[x].y & 31));
+    } else if (b == bstar) {
+      const uint32_t pos = atomicAdd(&s_nc, 1u);
+      cand[pos] = e[x];
+    }
+  }
+  __syncthreads();
+  const uint32_t nc = s_nc;
+  if (warp == 0) {
+    uint32_t theta = 0, id_cut = 0xFFFFFFFFu;
+    if (nc > rem) warp_select(cand, static_cast<int>(nc), static_cast<int>(rem), wh[0], theta, id_cut);
+    for (uint32_t c = lane; c < nc; c += 32) {
+      const uint2 x = cand[c];
+      if (nc <= rem || kept(x, theta, id_cut)) atomicOr(&bits[x.y >> 5], 1u << (x.y & 31));
+    }
+  }
+  __syncthreads();
+  // ascending readout: thread t owns words [t * per, t * per + per)
+  const int per = (nw + kStagedThreads - 1) / kStagedThreads;
+  uint32_t cntw = 0;
+  for (int w = tid * per; w < min(nw, tid * per + per); ++w) cntw += __popc(bits[w]);
+  uint32_t inc = cntw;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) wsum[warp] = inc;
+  __syncthreads();
+  uint32_t pos = inc - cntw;
+  for (int w = 0; w < warp; ++w) pos += wsum[w];
+  for (int w = tid * per; w < min(nw, tid * per + per); ++w) {
+    uint32_t wb = bits[w];
+    while (wb) {
+      const int bit = __ffs(wb) - 1;
+      wb &= wb - 1;
+      if (pos < static_cast<uint32_t>(k)) out[pos] = 32 * w + bit;
+      ++pos;
+    }
+  }
+  if (tid == 0) {
+    sel_count[row] = k;
+    flags[row] = 0;
+  }
+}
+
+// Flagged rows only: the row's scores recomputed on the CUDA cores (FP32 dot
+// products of the row's indexer queries with the widened keys) into the score
+// rows, for the radix kernel.
+__global__ void __launch_bounds__(256)
+index_score_fallback_kernel(const __nv_bfloat16* __restrict__ idx_q, const float* __restrict__ idx_w,
+                            const __nv_bfloat16* __restrict__ keys, const int32_t* __restrict__ flags,
+                            float* __restrict__ scores, int64_t nq, int G, int H, int64_t q_pos0, int B,
+                            int64_t rpad) {
+  const int64_t row = blockIdx.x;
+  if (flags[row] == 0) return;
+  __shared__ float qf[8][64];
+  __shared__ float wf[8];
+  const int64_t i = (row / G) % nq;
+  const int64_t seq = row / (static_cast<int64_t>(G) * nq);
+  const int64_t n = (q_pos0 + i) / B;
+  for (int x = threadIdx.x; x < H * 64; x += blockDim.x) qf[x / 64][x % 64] = __bfloat162float(idx_q[row * H * 64 + x]);
+  if (threadIdx.x < H) wf[threadIdx.x] = idx_w[row * H + threadIdx.x];
+  __syncthreads();
+  const __nv_bfloat16* kb = keys + seq * rpad * 64;
+  for (int64_t r = threadIdx.x; r < n; r += blockDim.x) {
+    float kv[64];
+    const uint4* src = reinterpret_cast<const uint4*>(kb + r * 64);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 u = src[c];
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        kv[8 * c + 2 * x] = __uint_as_float(w4[x] << 16);
+        kv[8 * c + 2 * x + 1] = __uint_as_float(w4[x] & 0xFFFF0000u);
+      }
+    }
+    float acc = 0.f;
+    for (int h = 0; h < H; ++h) {
+      float d = 0.f;
+#pragma unroll
+      for (int x = 0; x < 64; ++x) d = fmaf(qf[h][x], kv[x], d);
+      acc = fmaf(wf[h], fmaxf(d, 0.f), acc);
+    }
+    scores[row * rpad + r] = acc;
   }
 }
 

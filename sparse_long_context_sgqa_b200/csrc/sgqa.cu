@@ -107,28 +107,32 @@ int staging_cap(int k) {
   return static_cast<int>(round_up(c, 32));
 }
 
+// Index workspace: widened keys, then one region that holds, one after the
+// other within a call, the sampled scores, the filtered staging lists and the
+// FP32 score rows (the stages that use them run in that order), then three
+// per-row arrays.
 struct IndexWs {
-  int64_t rpad;
+  int64_t rpad, nsamp;
   int cap;
-  size_t keys_off, scores_off, flags_off, staging_off, staged_off, bytes;
+  size_t keys_off, scores_off, sample_off, staging_off, flags_off, staged_off, thr_off, bytes;
 };
 IndexWs index_ws(const sgqa_params* p, int64_t S, int64_t nq, int64_t max_ctx) {
   IndexWs w;
   const int64_t rneed = std::max<int64_t>((max_ctx - 1) / p->block_size, 1);
   w.rpad = round_up(rneed, 128);
+  w.nsamp = round_up(w.rpad, sgqa::kIdxCand * sgqa::kSampleStride) / sgqa::kSampleStride;
   w.cap = staging_cap(p->topk);
   w.keys_off = 0;
   const size_t keys = align256(static_cast<size_t>(S * w.rpad * 64) * 2);
-  const int64_t rows = S * nq * p->num_kv_groups;
-  // materialised scores (few queries) or staging lists (prefill) share one region
-  w.scores_off = keys;
-  const size_t scores = align256(static_cast<size_t>(rows * w.rpad) * 4) + align256(static_cast<size_t>(rows) * 4);
-  w.flags_off = keys + align256(static_cast<size_t>(rows * w.rpad) * 4);
-  w.staging_off = keys;
-  const size_t staging = align256(static_cast<size_t>(rows) * w.cap * 8);
-  w.staged_off = keys + staging;
-  const size_t staged = align256(static_cast<size_t>(rows) * 4);
-  w.bytes = keys + std::max(scores, staging + staged);
+  const size_t rows = static_cast<size_t>(S * nq * p->num_kv_groups);
+  const size_t big = align256(std::max({rows * static_cast<size_t>(w.rpad) * 4, rows * static_cast<size_t>(w.cap) * 8,
+                                        rows * static_cast<size_t>(sgqa::kFilterCap) * 8,
+                                        rows * static_cast<size_t>(w.nsamp) * 4}));
+  w.scores_off = w.sample_off = w.staging_off = keys;
+  w.flags_off = keys + big;
+  w.staged_off = w.flags_off + align256(rows * 4);
+  w.thr_off = w.staged_off + align256(rows * 4);
+  w.bytes = w.thr_off + align256(rows * 4);
   return w;
 }
 
@@ -254,6 +258,11 @@ sgqa_status launch_attn_tc(const sgqa_params* p, int64_t S, int64_t q0, int64_t 
 
 // Index path for many queries: tcgen05 score rows + two-pass top-k by default;
 // SGQA_INDEX_PATH=stream selects the fused streaming top-k kernel instead.
+// Rows longer than the register-resident top-k takes (16384 candidates) use
+// the filtered path; shorter rows are cheaper to materialise and select
+// (measured at 128K and 1M contexts).
+constexpr int64_t kFilterMinCand = 16385;
+
 bool use_stream_index() {
   const char* e = getenv("SGQA_INDEX_PATH");
   return e != nullptr && strcmp(e, "stream") == 0;
@@ -338,15 +347,55 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
     }
     const int64_t grid = static_cast<int64_t>(G) * S * ((nq + Q - 1) / Q);
     const size_t smem = sizeof(sgqa::IndexTcSmem) + 1024;
-    if (H == 8) {
-      cudaFuncSetAttribute(sgqa::index_score_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      sgqa::index_score_tc_kernel<8><<<static_cast<unsigned>(grid), sgqa::kScoreTcThreads, smem, st>>>(
-          km, qm, idx_w, scores, nq, G, q0, B, w.rpad);
-    } else {
-      cudaFuncSetAttribute(sgqa::index_score_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      sgqa::index_score_tc_kernel<4><<<static_cast<unsigned>(grid), sgqa::kScoreTcThreads, smem, st>>>(
-          km, qm, idx_w, scores, nq, G, q0, B, w.rpad);
+    auto launch_score = [&](int mode, sgqa::ScoreOut o) {
+#define SGQA_SCORE(HH, MM)                                                                                       \
+  do {                                                                                                           \
+    cudaFuncSetAttribute(sgqa::index_score_tc_kernel<HH, MM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    sgqa::index_score_tc_kernel<HH, MM><<<static_cast<unsigned>(grid), sgqa::kScoreTcThreads, smem, st>>>(       \
+        km, qm, idx_w, o, nq, G, q0, B, w.rpad);                                                                 \
+  } while (0)
+      if (H == 8) {
+        if (mode == sgqa::kScoreRows) SGQA_SCORE(8, sgqa::kScoreRows);
+        else if (mode == sgqa::kScoreSample) SGQA_SCORE(8, sgqa::kScoreSample);
+        else SGQA_SCORE(8, sgqa::kScoreFilter);
+      } else {
+        if (mode == sgqa::kScoreRows) SGQA_SCORE(4, sgqa::kScoreRows);
+        else if (mode == sgqa::kScoreSample) SGQA_SCORE(4, sgqa::kScoreSample);
+        else SGQA_SCORE(4, sgqa::kScoreFilter);
+      }
+#undef SGQA_SCORE
+    };
+    if (rneed >= kFilterMinCand) {
+      // Long rows: sampled threshold, filtered score pass, exact select from the
+      // kept lists; rows the filter could not settle are recomputed and go to
+      // the radix kernel.  No FP32 score row is written for the others.
+      const int64_t rows = S * nq * G;
+      float* sample = ws_at<float>(ws, w.sample_off);
+      float* thr = ws_at<float>(ws, w.thr_off);
+      uint2* staging = ws_at<uint2>(ws, w.staging_off);
+      int32_t* staged = ws_at<int32_t>(ws, w.staged_off);
+      launch_score(sgqa::kScoreSample, sgqa::ScoreOut{sample, w.nsamp, nullptr, nullptr, nullptr, 0});
+      SGQA_LAUNCH_CHECK("index_score_tc_kernel (sample)");
+      sgqa::index_threshold_kernel<<<static_cast<unsigned>(rows), sgqa::kThrThreads, 0, st>>>(sample, w.nsamp, nq, G,
+                                                                                           q0, B, thr);
+      SGQA_LAUNCH_CHECK("index_threshold_kernel");
+      launch_score(sgqa::kScoreFilter, sgqa::ScoreOut{nullptr, 0, thr, staging, staged, sgqa::kFilterCap});
+      SGQA_LAUNCH_CHECK("index_score_tc_kernel (filter)");
+      const int nwords_max = static_cast<int>((rneed + 31) / 32);
+      const size_t dsmem = static_cast<size_t>(2 * sgqa::kFilterCap + nwords_max) * 4;
+      cudaFuncSetAttribute(sgqa::topk_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsmem);
+      sgqa::topk_staged_kernel<<<static_cast<unsigned>(rows), sgqa::kStagedThreads, dsmem, st>>>(
+          staging, staged, nq, G, q0, B, p->topk, sgqa::kFilterCap, nwords_max, sel, sel_count, flags);
+      SGQA_LAUNCH_CHECK("topk_staged_kernel");
+      sgqa::index_score_fallback_kernel<<<static_cast<unsigned>(rows), 256, 0, st>>>(iq, idx_w, keys, flags, scores, nq,
+                                                                                   G, H, q0, B, w.rpad);
+      SGQA_LAUNCH_CHECK("index_score_fallback_kernel");
+      sgqa::topk_rows_kernel<false><<<static_cast<unsigned>(rows), sgqa::kSelThreads, 0, st>>>(
+          scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, flags);
+      SGQA_LAUNCH_CHECK("topk_rows_kernel");
+      return SGQA_OK;
     }
+    launch_score(sgqa::kScoreRows, sgqa::ScoreOut{scores, w.rpad, nullptr, nullptr, nullptr, 0});
     SGQA_LAUNCH_CHECK("index_score_tc_kernel");
   } else if (rneed > 0 && G == 4 && H == 8) {
     // few queries: one CTA per (query, 128 candidates) scores all four groups from the E4M3 store

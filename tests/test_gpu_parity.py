@@ -126,15 +126,23 @@ def test_index_topk_parity(cuda_device, case):
     assert ties <= 2 * len(rows)
 
 
-def test_index_topk_exact_ties(cuda_device):
+@pytest.mark.parametrize("case", ["short_rows", "filtered_rows"])
+def test_index_topk_exact_ties(cuda_device, case):
     """Zero head weights make every score exactly 0: the only valid selection
-    is the k smallest block ids.  Rows of 600..2048 candidates resolve the tie
-    inside one histogram bin; rows of 2049..2903 candidates overflow the
-    boundary buffer and are redone by the radix kernel.  Every other query keeps its
-    weights and is checked against the oracle as usual."""
-    wl = dataclasses.replace(WL["prefill8k"], name="ties", seq_len=24576, topk=512)
+    is the k smallest block ids.  short_rows: 600..2903 candidates per row,
+    where rows up to 2048 resolve the tie inside one histogram bin and longer
+    rows overflow the boundary buffer and are redone by the radix kernel.
+    filtered_rows: 16384..16895 candidates, the sampled-threshold path; every
+    zero row keeps all of its candidates, overflows the kept list and is
+    recomputed for the radix kernel.  The other queries keep their weights
+    and are checked against the oracle as usual."""
+    if case == "short_rows":
+        wl = dataclasses.replace(WL["prefill8k"], name="ties", seq_len=24576, topk=512)
+        q0, nq = 4800, 16384 + 2048  # candidates 600 .. 2903 per query (B = 8)
+    else:
+        wl = dataclasses.replace(WL["prefill8k"], name="ties_long", seq_len=139264, topk=512)
+        q0, nq = 131072, 4096  # candidates 16384 .. 16895 per query
     cache, _ = Hn.make_inputs(wl, cuda_device)
-    q0, nq = 4800, 16384 + 2048  # candidates 600 .. 2903 per query (B = 8)
     qs = I.make_queries(wl, cuda_device, q0, nq)
     zero = torch.zeros(nq, dtype=torch.bool, device=cuda_device)
     zero[::3] = True
@@ -154,7 +162,7 @@ def test_index_topk_exact_ties(cuda_device):
     assert np.all(sel[zero_np] == np.arange(wl.topk, dtype=np.int32))
     iq, iw = Hn.to_np(qs["idx_q"]), Hn.to_np(qs["idx_w"])
     ties = 0
-    rows = [i for i in range(1, nq, 397) if not zero_np[i]] + [nq - 1]
+    rows = [i for i in range(1, nq, 97 if case != "short_rows" else 397) if not zero_np[i]] + [nq - 1]
     for i in rows:
         for g in range(wl.groups):
             sc = O.index_scores(iq[i, g], iw[i, g], keys[:(q0 + i) // wl.block])
