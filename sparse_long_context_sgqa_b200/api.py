@@ -64,15 +64,52 @@ class SparseGQA:
 
         host holds pinned tensors with the cache layouts (kp, c, k, v) and the query
         layouts (q, idx_q, idx_w) of a full prefill; out_host receives [S, N, G*Hg, D].
-        Returns (bytes copied host->device, bytes copied device->host).
+        The copies are pipelined with the chunks: chunk c needs only the cache
+        positions before its last query and its own queries, so while chunk c
+        runs, chunk c+1's inputs are copied in on one stream and chunk c-1's
+        output is copied out on another (the two PCIe directions run at once).
+        Work is enqueued only; the given stream (default: the current one) waits
+        for the last copy out.  Returns (bytes copied host->device, bytes copied
+        device->host).
         """
-        h2d = 0
-        for name in ("kp", "c", "k", "v"):
-            getattr(self, name).copy_(host[name], non_blocking=True)
-            h2d += host[name].numel() * host[name].element_size()
-        dq = {n: host[n].to(self.device, non_blocking=True) for n in ("q", "idx_q", "idx_w")}
-        h2d += sum(host[n].numel() * host[n].element_size() for n in ("q", "idx_q", "idx_w"))
+        cur = torch.cuda.current_stream(self.device) if stream is None else stream
+        if not hasattr(self, "_copy_streams"):
+            self._copy_streams = (torch.cuda.Stream(device=self.device), torch.cuda.Stream(device=self.device))
+        h2d_s, d2h_s = self._copy_streams
+        S, N = host["q"].shape[0], host["q"].shape[1]
+        dq = {n: torch.empty(host[n].shape, dtype=host[n].dtype, device=self.device) for n in ("q", "idx_q", "idx_w")}
         out = torch.empty(out_host.shape, dtype=out_host.dtype, device=self.device)
-        self.prefill(dq["q"], dq["idx_q"], dq["idx_w"], out, stream=stream)
-        out_host.copy_(out, non_blocking=True)
+        G, k = self.p.num_kv_groups, self.p.topk
+        sel = torch.empty((S, self.chunk, G, k), dtype=torch.int32, device=self.device)
+        cnt = torch.empty((S, self.chunk, G), dtype=torch.int32, device=self.device)
+        h2d_s.wait_stream(cur)
+        d2h_s.wait_stream(cur)
+        for c0 in range(0, N, self.chunk):
+            n = min(self.chunk, N - c0)
+            with torch.cuda.stream(h2d_s):
+                for s in range(S):
+                    for name in ("kp", "c", "k", "v"):
+                        getattr(self, name)[s, c0:c0 + n].copy_(host[name][s, c0:c0 + n], non_blocking=True)
+                    for name in ("q", "idx_q", "idx_w"):
+                        dq[name][s, c0:c0 + n].copy_(host[name][s, c0:c0 + n], non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(h2d_s)
+            cur.wait_event(ready)
+            o = out[:, c0:c0 + n] if S == 1 else torch.empty((S, n) + tuple(out.shape[2:]), dtype=out.dtype,
+                                                             device=self.device)
+            self.forward(c0, dq["q"][:, c0:c0 + n], dq["idx_q"][:, c0:c0 + n], dq["idx_w"][:, c0:c0 + n],
+                         sel[:, :n], cnt[:, :n], o, stream=cur)
+            if S != 1:
+                out[:, c0:c0 + n] = o
+            done = torch.cuda.Event()
+            done.record(cur)
+            d2h_s.wait_event(done)
+            with torch.cuda.stream(d2h_s):
+                for s in range(S):
+                    out_host[s, c0:c0 + n].copy_(out[s, c0:c0 + n], non_blocking=True)
+        for t in list(dq.values()) + [out, sel, cnt]:
+            t.record_stream(h2d_s)
+            t.record_stream(d2h_s)
+        cur.wait_stream(d2h_s)
+        h2d = sum(host[n].numel() * host[n].element_size() for n in ("kp", "c", "k", "v", "q", "idx_q", "idx_w"))
         return h2d, out_host.numel() * out_host.element_size()

@@ -258,6 +258,28 @@ def _e2e(wl, device, rows, seqs=(0,)):
     return stats
 
 
+def test_forward_host_pipelined_matches_device_path(cuda_device):
+    """SparseGQA.forward_host copies each chunk's inputs in and output out on
+    side streams while other chunks run; its output must equal the chunked
+    device-resident path bit for bit (same kernels on the same inputs)."""
+    from sparse_long_context_sgqa_b200.api import SparseGQA
+    wl = dataclasses.replace(WL["prefill8k"], name="e2e", seq_len=3072, chunk=1024)
+    run = Hn.run_forward(wl, cuda_device)
+    p = Hn.params_for(wl)
+    model = SparseGQA(p, 1, wl.seq_len, wl.chunk, cuda_device)
+    host = {n: run.cache[n].cpu().pin_memory() for n in ("kp", "c", "k", "v")}
+    for n in ("q", "idx_q", "idx_w"):
+        host[n] = run.queries[n].cpu().pin_memory()
+    out_host = torch.empty(run.out.shape, dtype=run.out.dtype).pin_memory()
+    h2d, d2h = model.forward_host(host, out_host)
+    torch.cuda.synchronize()
+    _bd().sgqa_check()
+    assert h2d == sum(host[n].numel() * host[n].element_size() for n in host)
+    assert d2h == out_host.numel() * out_host.element_size()
+    assert torch.equal(out_host, run.out.cpu())
+    assert torch.equal(model.store.cpu(), run.store.cpu())
+
+
 def test_forward_tiny_all_rows(cuda_device):
     _e2e(WL["tiny"], cuda_device, range(256))
 
