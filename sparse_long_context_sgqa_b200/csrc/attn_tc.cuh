@@ -35,6 +35,8 @@
 // cycles per tile in synchronisation stalls.  Every mbarrier wait is bounded
 // (tc::mbar_wait / tc::warp_wait).
 #pragma once
+#include <cooperative_groups.h>
+
 #include "attn_mma.cuh"
 #include "tc.cuh"
 
@@ -474,9 +476,11 @@ namespace sgqa {
 // group)'s blocks (split-K); a single producer thread streams each block's K
 // and V (one 5-D TMA box each, 3 KB, 128-byte swizzled) into a 16-slot ring,
 // and four compute warps consume two blocks (16 tokens) per step with the
-// warp-level MMA formulation (16 heads = the m16 rows).  Each split writes
-// its (max, sum, unnormalised O); the last split of a row to finish (atomic
-// ticket) combines them into the bf16 output and re-arms the ticket.
+// warp-level MMA formulation (16 heads = the m16 rows).  The splits of a row
+// form one thread-block cluster: each keeps its (max, sum, unnormalised O) in
+// shared memory and, after a cluster barrier, finalises a slice of the row's
+// output by reading every split's partial through distributed shared memory
+// (no global partials, fences or tickets).
 // ---------------------------------------------------------------------------
 constexpr int kDecSlots = 16;
 constexpr int kDecThreads = 160;  // warp 0 producer, warps 1-4 compute
@@ -494,13 +498,13 @@ __device__ __forceinline__ uint32_t blk_off(uint32_t r, uint32_t j) {
   return (j >> 3) * 1024u + r * 128u + (((j & 7u) ^ r) << 4);
 }
 
+constexpr int kDecMaxSplit = 8;  // splits of a row = one (portable) cluster
+
 __global__ void __launch_bounds__(kDecThreads, 2)
 attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                        const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ sel,
-                       const int32_t* __restrict__ sel_count, float* __restrict__ part_o,
-                       float* __restrict__ part_ml, int32_t* __restrict__ tickets,
-                       __nv_bfloat16* __restrict__ out, int64_t nq, int G, int k, int64_t q_pos0, int nsplit,
-                       float scale_log2) {
+                       const int32_t* __restrict__ sel_count, __nv_bfloat16* __restrict__ out, int64_t nq, int G,
+                       int k, int64_t q_pos0, int nsplit, float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
   DecSmem& sm = *reinterpret_cast<DecSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
@@ -664,11 +668,18 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     }
   }
   __syncthreads();
-  // combine the four compute warps (shared memory reused), write this split's partial
+  // combine the four compute warps into this split's partial (shared memory
+  // of the ring reused): per-head factors once, then four FMAs per output
   constexpr int kCoStride = kD + 4;                       // padded rows: no bank conflicts
   float* cm = reinterpret_cast<float*>(&sm.kv[0][0][0]);  // [4][16]
   float* cl = cm + 4 * kHg;                               // [4][16]
   float* co = cl + 4 * kHg;                               // [4][16][196]
+  float* fw = co + 4 * kHg * kCoStride;                   // [4][16] warp factors
+  float* pm = reinterpret_cast<float*>(&sm.kv[0][0][0] + 65536);  // this split: max [16]
+  float* pl = pm + kHg;                                           //             sum [16]
+  float* pacc = pl + kHg;                                         //             O [16][192]
+  float* gf = pacc + kHg * kD;                                    // row factors [kDecMaxSplit][16]
+  float* ginv = gf + kDecMaxSplit * kHg;                          // [16]
   if (warp >= 1) {
     const int cw = warp - 1;
     float l0 = st.l[0], l1 = st.l[1];
@@ -689,60 +700,60 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     }
   }
   __syncthreads();
-  float* po = part_o + (row * nsplit + split) * kHg * kD;
-  float* pml = part_ml + (row * nsplit + split) * kHg * 2;
-  for (int idx = threadIdx.x; idx < kHg * kD; idx += kDecThreads) {
-    const int h = idx / kD;
+  if (threadIdx.x < kHg) {
+    const int h = threadIdx.x;
     float mm = -INFINITY;
 #pragma unroll
     for (int w = 0; w < 4; ++w) mm = fmaxf(mm, cm[w * kHg + h]);
     const float mu = mm == -INFINITY ? 0.f : mm;
-    float acc = 0.f, ls = 0.f;
+    float ls = 0.f;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       const float a = exp2f(cm[w * kHg + h] - mu);
-      acc += a * co[(w * kHg + h) * kCoStride + (idx % kD)];
+      fw[w * kHg + h] = a;
       ls += a * cl[w * kHg + h];
     }
-    po[idx] = acc;
-    if (idx % kD == 0) { pml[2 * h] = mm; pml[2 * h + 1] = ls; }
-  }
-  // the last split of this row combines all partials
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int old = atomicAdd(&tickets[row], 1);
-    sm.last = (old == nsplit - 1);
-  }
-  __syncthreads();
-  if (!sm.last) return;
-  __threadfence();
-  // scale factor of every (split, head) partial, computed once
-  float* fac = co;  // [nsplit][16] (the combine buffers are free again)
-  float* inv = co + 32 * kHg;  // [16]
-  if (threadIdx.x < kHg) {
-    const int h = threadIdx.x;
-    float mm = -INFINITY;
-    for (int s2 = 0; s2 < nsplit; ++s2) mm = fmaxf(mm, __ldcg(&part_ml[((row * nsplit + s2) * kHg + h) * 2]));
-    const float mu = mm == -INFINITY ? 0.f : mm;
-    float ls = 0.f;
-    for (int s2 = 0; s2 < nsplit; ++s2) {
-      const float* ml = part_ml + ((row * nsplit + s2) * kHg + h) * 2;
-      const float a = exp2f(__ldcg(&ml[0]) - mu);
-      fac[s2 * kHg + h] = a;
-      ls += a * __ldcg(&ml[1]);
-    }
-    inv[h] = 1.f / ls;
+    pm[h] = mm;
+    pl[h] = ls;
   }
   __syncthreads();
   for (int idx = threadIdx.x; idx < kHg * kD; idx += kDecThreads) {
-    const int h = idx / kD;
-    const float* src = part_o + (row * nsplit) * kHg * kD + idx;
+    const int h = idx / kD, d = idx % kD;
     float acc = 0.f;
-    for (int s2 = 0; s2 < nsplit; ++s2) acc += fac[s2 * kHg + h] * __ldcg(src + static_cast<int64_t>(s2) * kHg * kD);
-    out[row * kHg * kD + idx] = __float2bfloat16_rn(acc * inv[h]);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) acc = fmaf(fw[w * kHg + h], co[(w * kHg + h) * kCoStride + d], acc);
+    pacc[idx] = acc;
   }
-  if (threadIdx.x == 0) tickets[row] = 0;
+  // every split's partial is in its shared memory: combine across the cluster
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  cluster.sync();
+  if (threadIdx.x < kHg) {
+    const int h = threadIdx.x;
+    float mm = -INFINITY;
+    for (int r = 0; r < nsplit; ++r) mm = fmaxf(mm, cluster.map_shared_rank(pm, r)[h]);
+    const float mu = mm == -INFINITY ? 0.f : mm;
+    float ls = 0.f;
+    for (int r = 0; r < nsplit; ++r) {
+      const float a = exp2f(cluster.map_shared_rank(pm, r)[h] - mu);
+      gf[r * kHg + h] = a;
+      ls += a * cluster.map_shared_rank(pl, r)[h];
+    }
+    ginv[h] = 1.f / ls;
+  }
+  __syncthreads();
+  {
+    // this split finalises outputs [split * per, split * per + per) of the row's 16 x 192
+    const int per = (kHg * kD + nsplit - 1) / nsplit;
+    const int i0 = split * per, i1 = min(kHg * kD, i0 + per);
+    for (int idx = i0 + threadIdx.x; idx < i1; idx += kDecThreads) {
+      const int h = idx / kD;
+      float acc = 0.f;
+      for (int r = 0; r < nsplit; ++r) acc = fmaf(gf[r * kHg + h], cluster.map_shared_rank(pacc, r)[idx], acc);
+      out[row * kHg * kD + idx] = __float2bfloat16_rn(acc * ginv[h]);
+    }
+  }
+  cluster.sync();  // no split leaves while others still read its shared memory
 }
 
 }  // namespace sgqa

@@ -464,7 +464,7 @@ sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq,
   const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(vc);
   __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(out);
   if (nq <= kDecodeMaxNq && B == 8) {
-    // TMA-fed gather; the last split of each row combines (tickets start at zero)
+    // TMA-fed gather, the splits of a row combined inside their cluster
     const int64_t rows = S * nq * G;
     CUtensorMap km, vm;
     cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(clen), 3, static_cast<cuuint64_t>(G), static_cast<cuuint64_t>(S)};
@@ -473,15 +473,25 @@ sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq,
     sgqa_status s;
     if ((s = encode_bf16(&km, kc, 5, dims, strides, box, "k_cache")) != SGQA_OK) return s;
     if ((s = encode_bf16(&vm, vc, 5, dims, strides, box, "v_cache")) != SGQA_OK) return s;
-    float* po = ws_at<float>(ws, w.po_off);
-    float* pml = ws_at<float>(ws, w.pml_off);
-    int32_t* tick = ws_at<int32_t>(ws, w.tick_off);
-    cudaError_t e = cudaMemsetAsync(tick, 0, static_cast<size_t>(rows) * 4, st);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(tickets)");
+    // the splits of a row run as one cluster (combined through distributed shared memory)
+    const int nsplit = std::min(w.nsplit, sgqa::kDecMaxSplit);
     const size_t smem = sizeof(sgqa::DecSmem) + 1024;
     cudaFuncSetAttribute(sgqa::attn_decode_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    sgqa::attn_decode_tma_kernel<<<static_cast<unsigned>(rows * w.nsplit), sgqa::kDecThreads, smem, st>>>(
-        km, vm, qb, sel, sel_count, po, pml, tick, ob, nq, G, k, q0, w.nsplit, scale_log2);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(rows * nsplit));
+    cfg.blockDim = dim3(sgqa::kDecThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(nsplit);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, sgqa::attn_decode_tma_kernel, km, vm, qb, sel, sel_count, ob, nq, G, k,
+                                       q0, nsplit, scale_log2);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_decode_tma_kernel launch");
     SGQA_LAUNCH_CHECK("attn_decode_tma_kernel");
     return SGQA_OK;
   }
