@@ -24,7 +24,7 @@
 namespace sgqa {
 
 constexpr int kIdxThreads = 192;
-constexpr int kScoreTcThreads = 320;  // score kernel: producer, MMA, 8 epilogue warps
+constexpr int kScoreTcThreads = 576;  // score kernel: producer, MMA, 16 epilogue warps
 constexpr int kIdxStages = 4;
 constexpr int kIdxCand = 128;    // candidates per tile (MMA M)
 constexpr int kIdxCols = 256;    // (query, head) columns per CTA (MMA N)
@@ -391,9 +391,9 @@ struct ScoreOut {
   float* scores;            // kScoreRows: [rows, ld] = [rows, rpad]; kScoreSample: [rows, ld]
   int64_t ld;
   const float* thr;         // kScoreFilter: per-row threshold
-  uint2* staging;           // kScoreFilter: [rows, cap] (key, id)
-  int32_t* staged;          // kScoreFilter: [rows] scores at or above the threshold
-  int cap;
+  uint2* staging;           // kScoreFilter: [rows, 4, cap] (key, id), one list per TMEM lane quadrant
+  int32_t* staged;          // kScoreFilter: [rows, 4] scores at or above the threshold per list
+  int cap;                  // entries per list
 };
 
 template <int H, int MODE>
@@ -430,7 +430,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(bar(sm.acc_full[b]), 1);
-      tc::mbar_init(bar(sm.acc_empty[b]), 256);
+      tc::mbar_init(bar(sm.acc_empty[b]), 512);
     }
     tc::mbar_init(bar(sm.drain), 1);
     tc::mbar_fence_init();
@@ -514,14 +514,19 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
         }
       }
     } else {
-      // epilogue: eight warps, two per TMEM lane quadrant, each taking half of the 256 columns
+      // epilogue: sixteen warps, four per TMEM lane quadrant (= 32 candidates),
+      // each taking 64 of the 256 (query, head) columns, read 32 at a time
+      constexpr int QW = 32 / H;  // query slots per 32 columns
       const int quad = warp & 3;
-      const int half = (warp - 2) >> 2;
+      const int part = (warp - 2) >> 2;
       const int m = quad * 32 + lane;
       const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
       const int64_t row0 = (seq * nq + q0) * G + g;  // row of query slot 0; slot qs is row0 + qs * G
       // the CTA's smallest candidate count: tiles below it need no per-row bound check
       const int64_t ncand_min = (q_pos0 + q0) / B;
+      int kept[2 * QW];  // filter: this warp's kept entries per query slot (the same in every lane)
+#pragma unroll
+      for (int x = 0; x < 2 * QW; ++x) kept[x] = 0;
       for (int c = 0; c < n_loop; ++c) {
         const int ab = c & 1;
         if (!tc::mbar_wait(bar(sm.acc_full[ab]), (c >> 1) & 1, abort)) break;
@@ -529,24 +534,18 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
         const int64_t r = static_cast<int64_t>(tile_of(c)) * kIdxCand + m;  // candidate block id
         const bool tail = static_cast<int64_t>(tile_of(c) + 1) * kIdxCand > ncand_min;
 #pragma unroll
-        for (int h2 = 0; h2 < kIdxCols / 128; ++h2) {
-          const int ch2 = half * (kIdxCols / 128) + h2;
-          uint32_t d2[64];
-          tc::tmem_ld32(tmem + ab * kIdxCols + 64 * ch2 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&d2[0]));
-          tc::tmem_ld32(tmem + ab * kIdxCols + 64 * ch2 + 32 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&d2[32]));
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int col0 = 64 * part + 32 * h2;
+          uint32_t d[32];
+          tc::tmem_ld32(tmem + ab * kIdxCols + col0 + lane_off, d);
           tc::tmem_ld_wait();
-          if (h2 == kIdxCols / 128 - 1) {
+          if (h2 == 1) {
             tc::fence_before();
             tc::mbar_arrive(bar(sm.acc_empty[ab]));
           }
-          float thr_q[64 / H];
-          if (MODE == kScoreFilter) {
 #pragma unroll
-            for (int qq = 0; qq < 64 / H; ++qq) thr_q[qq] = __uint_as_float(sm.thr[ch2 * (64 / H) + qq]);
-          }
-#pragma unroll
-          for (int qq = 0; qq < 64 / H; ++qq) {
-            const int qs = ch2 * (64 / H) + qq;
+          for (int qq = 0; qq < QW; ++qq) {
+            const int qs = col0 / H + qq;
             const float4 w0 = *reinterpret_cast<const float4*>(&sm.w[qs * H]);
             float wv[H];
             wv[0] = w0.x; wv[1] = w0.y; wv[2] = w0.z; wv[3] = w0.w;
@@ -556,7 +555,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
             }
             float acc = 0.f;
 #pragma unroll
-            for (int i = 0; i < H; ++i) acc = fmaf(wv[i], fmaxf(__uint_as_float(d2[qq * H + i]), 0.f), acc);
+            for (int i = 0; i < H; ++i) acc = fmaf(wv[i], fmaxf(__uint_as_float(d[qq * H + i]), 0.f), acc);
             const int64_t row = row0 + static_cast<int64_t>(qs) * G;
             if (MODE == kScoreRows) {
               if (qs < nq_here) o.scores[row * o.ld + r] = acc;
@@ -564,25 +563,33 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
               if (qs < nq_here) o.scores[row * o.ld + static_cast<int64_t>(c) * kIdxCand + m] = acc;
             } else {
               // keep the score if it reaches the row's threshold (rows past the
-              // call's queries have threshold +inf)
-              bool pass = acc >= thr_q[qq];
+              // call's queries have threshold +inf); each (row, quadrant) has its
+              // own list, filled in ballot order: no shared counters
+              bool pass = acc >= __uint_as_float(sm.thr[qs]);
               if (tail) pass = pass && r < sm.ncand[qs];
-              if (pass) {
-                const int pos = atomicAdd(&sm.cnt[qs], 1);
-                if (pos < o.cap) o.staging[row * o.cap + pos] = make_uint2(score_key(acc), static_cast<uint32_t>(r));
+              const uint32_t bal = __ballot_sync(0xffffffffu, pass);
+              if (bal) {
+                const int pos = kept[h2 * QW + qq] + __popc(bal & ((1u << lane) - 1u));
+                if (pass && pos < o.cap)
+                  o.staging[(row * 4 + quad) * o.cap + pos] = make_uint2(score_key(acc), static_cast<uint32_t>(r));
+                kept[h2 * QW + qq] += __popc(bal);
               }
             }
           }
         }
       }
-      if (MODE == kScoreFilter) {
-        asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight epilogue warps
-        if (warp == 2)
-          for (int qs = lane; qs < nq_here; qs += 32) o.staged[row0 + static_cast<int64_t>(qs) * G] = sm.cnt[qs];
+      if (MODE == kScoreFilter && lane == 0) {
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+          for (int qq = 0; qq < QW; ++qq) {
+            const int qs = (64 * part + 32 * h2) / H + qq;
+            if (qs < nq_here) o.staged[(row0 + static_cast<int64_t>(qs) * G) * 4 + quad] = kept[h2 * QW + qq];
+          }
       }
     }
-  } else if (MODE == kScoreFilter && warp == 2) {
-    for (int qs = lane; qs < nq_here; qs += 32) o.staged[((seq * nq + q0 + qs) * G + g)] = 0;
+  } else if (MODE == kScoreFilter && warp >= 2 && warp < 6) {
+    for (int qs = lane; qs < nq_here; qs += 32) o.staged[((seq * nq + q0 + qs) * G + g) * 4 + (warp & 3)] = 0;
   }
   tc::fence_before();
   __syncthreads();
@@ -985,7 +992,8 @@ topk_rows_win_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq,
 // recomputed scores by the radix kernel.
 // ---------------------------------------------------------------------------
 constexpr int kThrRank = 64;
-constexpr int kFilterCap = 4096;
+constexpr int kFilterCap = 4096;             // kept entries per row: four lists of kFilterCap / 4
+constexpr int kFilterSubCap = kFilterCap / 4;
 constexpr int kThrThreads = 256;
 constexpr int kThrPer = 32;  // samples per thread: rows of up to 131072 candidates
 
@@ -1106,12 +1114,20 @@ topk_staged_kernel(const uint2* __restrict__ staging, const int32_t* __restrict_
     }
     return;
   }
-  const int cnt = staged[row];
-  if (cnt < k || cnt > cap) {
+  // the row's four lists (one per candidate quadrant of the score kernel)
+  const int4 c4 = *reinterpret_cast<const int4*>(staged + row * 4);
+  const int cnt = c4.x + c4.y + c4.z + c4.w;
+  if (cnt < k || c4.x > cap || c4.y > cap || c4.z > cap || c4.w > cap) {
     if (tid == 0) flags[row] = 1;
     return;
   }
-  const uint2* list = staging + row * static_cast<int64_t>(cap);
+  const int p1 = c4.x, p2 = p1 + c4.y, p3 = p2 + c4.z;
+  const uint2* lists = staging + row * 4 * static_cast<int64_t>(cap);
+  auto entry = [&](int j) -> uint2 {
+    const int q = (j >= p1) + (j >= p2) + (j >= p3);
+    const int off = j - (q == 0 ? 0 : q == 1 ? p1 : q == 2 ? p2 : p3);
+    return lists[q * static_cast<int64_t>(cap) + off];
+  };
   const int nw = (n + 31) / 32;
   for (int w = tid; w < nw; w += kStagedThreads) bits[w] = 0u;
   for (int b = tid; b < (kStagedThreads / 32) * 256; b += kStagedThreads) (&wh[0][0])[b] = 0u;
@@ -1122,7 +1138,7 @@ topk_staged_kernel(const uint2* __restrict__ staging, const int32_t* __restrict_
 #pragma unroll
   for (int x = 0; x < kStagedPer; ++x) {
     const int j = tid + kStagedThreads * x;
-    e[x] = j < cnt ? list[j] : make_uint2(0u, 0xFFFFFFFFu);
+    e[x] = j < cnt ? entry(j) : make_uint2(0u, 0xFFFFFFFFu);
     v[x] = j < cnt ? key_score(e[x].x) : -INFINITY;
     mx = fmaxf(mx, v[x]);
     if (j < cnt) mn = fminf(mn, v[x]);

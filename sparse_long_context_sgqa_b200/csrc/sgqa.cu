@@ -131,7 +131,7 @@ IndexWs index_ws(const sgqa_params* p, int64_t S, int64_t nq, int64_t max_ctx) {
   w.scores_off = w.sample_off = w.staging_off = keys;
   w.flags_off = keys + big;
   w.staged_off = w.flags_off + align256(rows * 4);
-  w.thr_off = w.staged_off + align256(rows * 4);
+  w.thr_off = w.staged_off + align256(rows * 4 * 4);  // staged: [rows, 4] counts
   w.bytes = w.thr_off + align256(rows * 4);
   return w;
 }
@@ -379,13 +379,13 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
       sgqa::index_threshold_kernel<<<static_cast<unsigned>(rows), sgqa::kThrThreads, 0, st>>>(sample, w.nsamp, nq, G,
                                                                                            q0, B, thr);
       SGQA_LAUNCH_CHECK("index_threshold_kernel");
-      launch_score(sgqa::kScoreFilter, sgqa::ScoreOut{nullptr, 0, thr, staging, staged, sgqa::kFilterCap});
+      launch_score(sgqa::kScoreFilter, sgqa::ScoreOut{nullptr, 0, thr, staging, staged, sgqa::kFilterSubCap});
       SGQA_LAUNCH_CHECK("index_score_tc_kernel (filter)");
       const int nwords_max = static_cast<int>((rneed + 31) / 32);
       const size_t dsmem = static_cast<size_t>(2 * sgqa::kFilterCap + nwords_max) * 4;
       cudaFuncSetAttribute(sgqa::topk_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsmem);
       sgqa::topk_staged_kernel<<<static_cast<unsigned>(rows), sgqa::kStagedThreads, dsmem, st>>>(
-          staging, staged, nq, G, q0, B, p->topk, sgqa::kFilterCap, nwords_max, sel, sel_count, flags);
+          staging, staged, nq, G, q0, B, p->topk, sgqa::kFilterSubCap, nwords_max, sel, sel_count, flags);
       SGQA_LAUNCH_CHECK("topk_staged_kernel");
       sgqa::index_score_fallback_kernel<<<static_cast<unsigned>(rows), 256, 0, st>>>(iq, idx_w, keys, flags, scores, nq,
                                                                                    G, H, q0, B, w.rpad);
