@@ -553,9 +553,18 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
               const float4 w1 = *reinterpret_cast<const float4*>(&sm.w[qs * H + 4]);
               wv[4] = w1.x; wv[5] = w1.y; wv[6] = w1.z; wv[7] = w1.w;
             }
-            float acc = 0.f;
+            // sum_i w_i * max(0, s_i): even and odd heads accumulate in the two
+            // halves of a packed FP32 pair (fma.rn.f32x2), added at the end
+            uint64_t acc2 = 0;
 #pragma unroll
-            for (int i = 0; i < H; ++i) acc = fmaf(wv[i], fmaxf(__uint_as_float(d[qq * H + i]), 0.f), acc);
+            for (int i = 0; i < H; i += 2) {
+              const uint64_t x2 = pack_f32x2(fmaxf(__uint_as_float(d[qq * H + i]), 0.f),
+                                             fmaxf(__uint_as_float(d[qq * H + i + 1]), 0.f));
+              const uint64_t w2 = pack_f32x2(wv[i], wv[i + 1]);
+              asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc2) : "l"(x2), "l"(w2));
+            }
+            const float acc = __uint_as_float(static_cast<uint32_t>(acc2)) +
+                              __uint_as_float(static_cast<uint32_t>(acc2 >> 32));
             const int64_t row = row0 + static_cast<int64_t>(qs) * G;
             if (MODE == kScoreRows) {
               if (qs < nq_here) o.scores[row * o.ld + r] = acc;
