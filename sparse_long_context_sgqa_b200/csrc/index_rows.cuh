@@ -178,17 +178,15 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int& total, int* warp
 // passes read SRAM instead of HBM.
 constexpr int kSelStageMax = 40960;
 
+// The selection of one row by the whole CTA (every thread calls it with the same row).
 template <bool STAGE>
-__global__ void __launch_bounds__(kSelThreads)
-topk_rows_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int G,
-                 int64_t q_pos0, int B, int k, int32_t* __restrict__ sel,
-                 int32_t* __restrict__ sel_count, const int32_t* __restrict__ only_if) {
+__device__ __forceinline__ void topk_row_radix(int64_t row, const float* __restrict__ scores, int64_t rpad,
+                                               int64_t nq, int G, int64_t q_pos0, int B, int k,
+                                               int32_t* __restrict__ sel, int32_t* __restrict__ sel_count) {
   extern __shared__ float staged_row[];
   __shared__ uint32_t hist[2048];
   __shared__ int warp_sums[32];
   __shared__ uint32_t s_prefix, s_rem;
-  const int64_t row = blockIdx.x;  // (seq * nq + i) * G + g
-  if (only_if != nullptr && only_if[row] == 0) return;  // row already selected
   const int64_t i = (row / G) % nq;
   const int64_t t = q_pos0 + i;
   const int64_t n = t / B;
@@ -268,6 +266,31 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int
     eq_seen += eq_total;
   }
   if (tid == 0) sel_count[row] = k;
+}
+
+// one CTA per row; only_if (optional) restricts the work to flagged rows
+template <bool STAGE>
+__global__ void __launch_bounds__(kSelThreads)
+topk_rows_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int G,
+                 int64_t q_pos0, int B, int k, int32_t* __restrict__ sel,
+                 int32_t* __restrict__ sel_count, const int32_t* __restrict__ only_if) {
+  const int64_t row = blockIdx.x;  // (seq * nq + i) * G + g
+  if (only_if != nullptr && only_if[row] == 0) return;  // row already selected
+  topk_row_radix<STAGE>(row, scores, rpad, nq, G, q_pos0, B, k, sel, sel_count);
+}
+
+// The rows another select kernel listed as unsettled (list[0 .. *count)),
+// a fixed grid striding over them: a launch with an empty list costs one
+// wave of CTAs that exit at once.
+__global__ void __launch_bounds__(kSelThreads)
+topk_rows_list_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int G, int64_t q_pos0, int B,
+                      int k, int32_t* __restrict__ sel, int32_t* __restrict__ sel_count,
+                      const int32_t* __restrict__ list, const int32_t* __restrict__ count) {
+  const int n = *count;
+  for (int x = blockIdx.x; x < n; x += gridDim.x) {
+    topk_row_radix<false>(list[x], scores, rpad, nq, G, q_pos0, B, k, sel, sel_count);
+    __syncthreads();  // the next row reuses the shared arrays
+  }
 }
 
 }  // namespace sgqa

@@ -625,7 +625,7 @@ constexpr int kRows2Cand = 4096;
 __global__ void __launch_bounds__(kRows2Threads, 2)
 topk_rows2_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int G, int64_t q_pos0, int B,
                   int k, int nwords, int32_t* __restrict__ sel, int32_t* __restrict__ sel_count,
-                  int32_t* __restrict__ overflow) {
+                  int32_t* __restrict__ overflow, int32_t* __restrict__ list, int32_t* __restrict__ list_count) {
   extern __shared__ uint32_t sm2[];
   uint32_t* wh = sm2;                                                     // [16][1024] packed u16 pairs
   uint2* cand = reinterpret_cast<uint2*>(sm2 + kRows2Warps * kRows2Bins / 2);  // [kRows2Cand]
@@ -713,7 +713,10 @@ topk_rows2_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, in
   __syncthreads();
   const uint32_t nc = s_nc;
   if (nc > kRows2Cand) {  // boundary bin too large for the gather buffer
-    if (tid == 0) overflow[row] = 1;
+    if (tid == 0) {
+      overflow[row] = 1;
+      list[atomicAdd(list_count, 1)] = static_cast<int32_t>(row);
+    }
     return;
   }
   if (warp == 0) {
@@ -844,7 +847,7 @@ struct WinSmem {
 __global__ void __launch_bounds__(kWinThreads, 2)
 topk_rows_win_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int G, int64_t q_pos0, int B,
                      int k, int32_t* __restrict__ sel, int32_t* __restrict__ sel_count,
-                     int32_t* __restrict__ overflow) {
+                     int32_t* __restrict__ overflow, int32_t* __restrict__ list, int32_t* __restrict__ list_count) {
   __shared__ WinSmem sm;
   const int64_t row = blockIdx.x;  // (seq * nq + i) * G + g
   const int64_t i = (row / G) % nq;
@@ -950,7 +953,10 @@ topk_rows_win_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq,
   __syncthreads();
   const uint32_t nc = sm.nc;
   if (nc > kWinCand) {
-    if (tid == 0) overflow[row] = 1;
+    if (tid == 0) {
+      overflow[row] = 1;
+      list[atomicAdd(list_count, 1)] = static_cast<int32_t>(row);
+    }
     return;
   }
   if (warp == 0) {
@@ -1021,13 +1027,16 @@ index_threshold_kernel(const float* __restrict__ sample, int64_t ld, int64_t nq,
   // sample entry j = c * 128 + m is candidate (c * kSampleStride) * 128 + m
   auto cand_of = [](int j) -> int64_t { return static_cast<int64_t>(j / kIdxCand) * kSampleStride * kIdxCand + j % kIdxCand; };
   const int nsamp_tiles = static_cast<int>(((n + kIdxCand - 1) / kIdxCand + kSampleStride - 1) / kSampleStride);
-  const int nj = min(nsamp_tiles * kIdxCand, kThrThreads * kThrPer);
+  const int nj_all = nsamp_tiles * kIdxCand;
+  // rows with more samples than the registers hold (contexts beyond 1M) use every step-th one
+  const int step = (nj_all + kThrThreads * kThrPer - 1) / (kThrThreads * kThrPer);
+  const int nj = (nj_all + step - 1) / step;
   float v[kThrPer];
   int nvalid = 0;
 #pragma unroll
   for (int e = 0; e < kThrPer; ++e) {
-    const int j = tid + kThrThreads * e;
-    const bool ok = j < nj && cand_of(j) < n;
+    const int j = (tid + kThrThreads * e) * step;
+    const bool ok = tid + kThrThreads * e < nj && cand_of(j) < n;
     v[e] = ok ? srow[j] : -INFINITY;
     nvalid += ok;
   }
@@ -1057,7 +1066,9 @@ index_threshold_kernel(const float* __restrict__ sample, int64_t ld, int64_t nq,
     mn = fminf(mn, rmin[w]);
     total += static_cast<int>(wsum[w]);
   }
-  if (total <= kThrRank) {  // too few samples to estimate: keep everything
+  // the threshold sits below the (kThrRank / step)-th largest of the samples read
+  const int rank = max(kThrRank / step, 1);
+  if (total <= rank) {  // too few samples to estimate: keep everything
     if (tid == 0) thr[row] = -INFINITY;
     return;
   }
@@ -1083,7 +1094,7 @@ index_threshold_kernel(const float* __restrict__ sample, int64_t ld, int64_t nq,
     __syncthreads();
     uint32_t before = inc - c;
     for (int w = 0; w < warp; ++w) before += wsum[w];
-    if (before < static_cast<uint32_t>(kThrRank) && static_cast<uint32_t>(kThrRank) <= before + c) s_bstar = tid;
+    if (before < static_cast<uint32_t>(rank) && static_cast<uint32_t>(rank) <= before + c) s_bstar = tid;
   }
   __syncthreads();
   if (tid == 0) {
@@ -1102,7 +1113,8 @@ constexpr int kStagedPer = kFilterCap / kStagedThreads;  // 16
 __global__ void __launch_bounds__(kStagedThreads)
 topk_staged_kernel(const uint2* __restrict__ staging, const int32_t* __restrict__ staged, int64_t nq, int G,
                    int64_t q_pos0, int B, int k, int cap, int nwords_max, int32_t* __restrict__ sel,
-                   int32_t* __restrict__ sel_count, int32_t* __restrict__ flags) {
+                   int32_t* __restrict__ sel_count, int32_t* __restrict__ flags, int32_t* __restrict__ list,
+                   int32_t* __restrict__ list_count) {
   extern __shared__ uint32_t dyn[];
   uint2* cand = reinterpret_cast<uint2*>(dyn);                 // [kFilterCap]
   uint32_t* bits = dyn + 2 * kFilterCap;                       // [nwords_max]
@@ -1127,7 +1139,10 @@ topk_staged_kernel(const uint2* __restrict__ staging, const int32_t* __restrict_
   const int4 c4 = *reinterpret_cast<const int4*>(staged + row * 4);
   const int cnt = c4.x + c4.y + c4.z + c4.w;
   if (cnt < k || c4.x > cap || c4.y > cap || c4.z > cap || c4.w > cap) {
-    if (tid == 0) flags[row] = 1;
+    if (tid == 0) {
+      flags[row] = 1;
+      list[atomicAdd(list_count, 1)] = static_cast<int32_t>(row);
+    }
     return;
   }
   const int p1 = c4.x, p2 = p1 + c4.y, p3 = p2 + c4.z;
@@ -1249,18 +1264,13 @@ topk_staged_kernel(const uint2* __restrict__ staging, const int32_t* __restrict_
   }
 }
 
-// Flagged rows only: the row's scores recomputed on the CUDA cores (FP32 dot
-// products of the row's indexer queries with the widened keys) into the score
-// rows, for the radix kernel.
-__global__ void __launch_bounds__(256)
-index_score_fallback_kernel(const __nv_bfloat16* __restrict__ idx_q, const float* __restrict__ idx_w,
-                            const __nv_bfloat16* __restrict__ keys, const int32_t* __restrict__ flags,
-                            float* __restrict__ scores, int64_t nq, int G, int H, int64_t q_pos0, int B,
-                            int64_t rpad) {
-  const int64_t row = blockIdx.x;
-  if (flags[row] == 0) return;
-  __shared__ float qf[8][64];
-  __shared__ float wf[8];
+// One flagged row's scores, recomputed by the whole CTA.
+__device__ __forceinline__ void index_score_fallback_row(int64_t row, const __nv_bfloat16* __restrict__ idx_q,
+                                                         const float* __restrict__ idx_w,
+                                                         const __nv_bfloat16* __restrict__ keys,
+                                                         float* __restrict__ scores, int64_t nq, int G, int H,
+                                                         int64_t q_pos0, int B, int64_t rpad, float (*qf)[64],
+                                                         float* wf) {
   const int64_t i = (row / G) % nq;
   const int64_t seq = row / (static_cast<int64_t>(G) * nq);
   const int64_t n = (q_pos0 + i) / B;
@@ -1291,5 +1301,23 @@ index_score_fallback_kernel(const __nv_bfloat16* __restrict__ idx_q, const float
     scores[row * rpad + r] = acc;
   }
 }
+
+// Listed rows only: the row's scores recomputed on the CUDA cores (FP32 dot
+// products of the row's indexer queries with the widened keys) into the score
+// rows, for the radix kernel; a fixed grid strides over the list.
+__global__ void __launch_bounds__(256)
+index_score_fallback_kernel(const __nv_bfloat16* __restrict__ idx_q, const float* __restrict__ idx_w,
+                            const __nv_bfloat16* __restrict__ keys, const int32_t* __restrict__ list,
+                            const int32_t* __restrict__ list_count, float* __restrict__ scores, int64_t nq, int G,
+                            int H, int64_t q_pos0, int B, int64_t rpad) {
+  __shared__ float qf[8][64];
+  __shared__ float wf[8];
+  const int nlist = *list_count;
+  for (int x = blockIdx.x; x < nlist; x += gridDim.x) {
+    __syncthreads();  // qf / wf of the previous row are no longer read
+    index_score_fallback_row(list[x], idx_q, idx_w, keys, scores, nq, G, H, q_pos0, B, rpad, qf, wf);
+  }
+}
+
 
 }  // namespace sgqa

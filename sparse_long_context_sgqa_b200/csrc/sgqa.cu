@@ -114,7 +114,7 @@ int staging_cap(int k) {
 struct IndexWs {
   int64_t rpad, nsamp;
   int cap;
-  size_t keys_off, scores_off, sample_off, staging_off, flags_off, staged_off, thr_off, bytes;
+  size_t keys_off, scores_off, sample_off, staging_off, flags_off, staged_off, thr_off, list_off, bytes;
 };
 IndexWs index_ws(const sgqa_params* p, int64_t S, int64_t nq, int64_t max_ctx) {
   IndexWs w;
@@ -132,7 +132,8 @@ IndexWs index_ws(const sgqa_params* p, int64_t S, int64_t nq, int64_t max_ctx) {
   w.flags_off = keys + big;
   w.staged_off = w.flags_off + align256(rows * 4);
   w.thr_off = w.staged_off + align256(rows * 4 * 4);  // staged: [rows, 4] counts
-  w.bytes = w.thr_off + align256(rows * 4);
+  w.list_off = w.thr_off + align256(rows * 4);       // unsettled rows [rows], then their count
+  w.bytes = w.list_off + align256(rows * 4) + 256;
   return w;
 }
 
@@ -260,7 +261,8 @@ sgqa_status launch_attn_tc(const sgqa_params* p, int64_t S, int64_t q0, int64_t 
 // SGQA_INDEX_PATH=stream selects the fused streaming top-k kernel instead.
 // Rows longer than the register-resident top-k takes (16384 candidates) use
 // the filtered path; shorter rows are cheaper to materialise and select
-// (measured at 128K and 1M contexts).
+// (measured at 128K and 1M contexts).  The kept lists are sized for k <= 512
+// (about 2k entries expected per row, 8k room).
 constexpr int64_t kFilterMinCand = 16385;
 
 bool use_stream_index() {
@@ -327,6 +329,9 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
   }
   float* scores = ws_at<float>(ws, w.scores_off);
   int32_t* flags = ws_at<int32_t>(ws, w.flags_off);
+  // rows a select kernel could not settle, for the radix kernel (count after the list)
+  int32_t* list = ws_at<int32_t>(ws, w.list_off);
+  int32_t* list_count = list + align256(static_cast<size_t>(S * nq * G) * 4) / 4;
   if (rneed > 0 && nq > kDecodeMaxNq) {
     // tcgen05 scores: 256 (query, head) columns per CTA, 128 candidates per MMA
     const int Q = sgqa::kIdxCols / H;
@@ -365,7 +370,7 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
       }
 #undef SGQA_SCORE
     };
-    if (rneed >= kFilterMinCand) {
+    if (rneed >= kFilterMinCand && p->topk * 8 <= sgqa::kFilterCap) {
       // Long rows: sampled threshold, filtered score pass, exact select from the
       // kept lists; rows the filter could not settle are recomputed and go to
       // the radix kernel.  No FP32 score row is written for the others.
@@ -384,15 +389,19 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
       const int nwords_max = static_cast<int>((rneed + 31) / 32);
       const size_t dsmem = static_cast<size_t>(2 * sgqa::kFilterCap + nwords_max) * 4;
       cudaFuncSetAttribute(sgqa::topk_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsmem);
+      cudaError_t e = cudaMemsetAsync(list_count, 0, 4, st);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(list count)");
       sgqa::topk_staged_kernel<<<static_cast<unsigned>(rows), sgqa::kStagedThreads, dsmem, st>>>(
-          staging, staged, nq, G, q0, B, p->topk, sgqa::kFilterSubCap, nwords_max, sel, sel_count, flags);
+          staging, staged, nq, G, q0, B, p->topk, sgqa::kFilterSubCap, nwords_max, sel, sel_count, flags, list,
+          list_count);
       SGQA_LAUNCH_CHECK("topk_staged_kernel");
-      sgqa::index_score_fallback_kernel<<<static_cast<unsigned>(rows), 256, 0, st>>>(iq, idx_w, keys, flags, scores, nq,
-                                                                                   G, H, q0, B, w.rpad);
+      const unsigned fb_grid = static_cast<unsigned>(std::min<int64_t>(rows, 2 * 148));
+      sgqa::index_score_fallback_kernel<<<fb_grid, 256, 0, st>>>(iq, idx_w, keys, list, list_count, scores, nq, G, H,
+                                                                 q0, B, w.rpad);
       SGQA_LAUNCH_CHECK("index_score_fallback_kernel");
-      sgqa::topk_rows_kernel<false><<<static_cast<unsigned>(rows), sgqa::kSelThreads, 0, st>>>(
-          scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, flags);
-      SGQA_LAUNCH_CHECK("topk_rows_kernel");
+      sgqa::topk_rows_list_kernel<<<fb_grid, sgqa::kSelThreads, 0, st>>>(scores, w.rpad, nq, G, q0, B, p->topk, sel,
+                                                                         sel_count, list, list_count);
+      SGQA_LAUNCH_CHECK("topk_rows_list_kernel");
       return SGQA_OK;
     }
     launch_score(sgqa::kScoreRows, sgqa::ScoreOut{scores, w.rpad, nullptr, nullptr, nullptr, 0});
@@ -435,19 +444,30 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
   // cannot finish (boundary-bin overflow) go to the radix kernel, which also
   // takes the rows in between and short rows (its per-row set-up is smaller).
   if (rneed >= 2048 && rneed <= sgqa::kWinMaxCand) {
+    cudaError_t e = cudaMemsetAsync(list_count, 0, 4, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(list count)");
     sgqa::topk_rows_win_kernel<<<static_cast<unsigned>(rows), sgqa::kWinThreads, 0, st>>>(
-        scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, flags);
+        scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, flags, list, list_count);
     SGQA_LAUNCH_CHECK("topk_rows_win_kernel");
+    sgqa::topk_rows_list_kernel<<<static_cast<unsigned>(std::min<int64_t>(rows, 2 * 148)), sgqa::kSelThreads, 0, st>>>(
+        scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, list, list_count);
+    SGQA_LAUNCH_CHECK("topk_rows_list_kernel");
+    return SGQA_OK;
   } else if (rneed >= 32768 && ssmem <= 112 * 1024) {
     cudaFuncSetAttribute(sgqa::topk_rows2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
+    cudaError_t e = cudaMemsetAsync(list_count, 0, 4, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(list count)");
     sgqa::topk_rows2_kernel<<<static_cast<unsigned>(rows), sgqa::kRows2Threads, ssmem, st>>>(
-        scores, w.rpad, nq, G, q0, B, p->topk, nwords, sel, sel_count, flags);
+        scores, w.rpad, nq, G, q0, B, p->topk, nwords, sel, sel_count, flags, list, list_count);
     SGQA_LAUNCH_CHECK("topk_rows2_kernel");
-  } else {
-    flags = nullptr;  // the radix kernel takes every row
+    sgqa::topk_rows_list_kernel<<<static_cast<unsigned>(std::min<int64_t>(rows, 2 * 148)), sgqa::kSelThreads, 0, st>>>(
+        scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, list, list_count);
+    SGQA_LAUNCH_CHECK("topk_rows_list_kernel");
+    return SGQA_OK;
   }
+  // the radix kernel takes every row
   sgqa::topk_rows_kernel<false><<<static_cast<unsigned>(rows), sgqa::kSelThreads, 0, st>>>(
-      scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, flags);
+      scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, nullptr);
   SGQA_LAUNCH_CHECK("topk_rows_kernel");
   return SGQA_OK;
 }
