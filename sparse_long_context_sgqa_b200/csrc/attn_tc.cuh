@@ -24,12 +24,13 @@
 //               log2 units with lazy rescaling of O (only when the max grows
 //               by more than 2^8), P rounded to BF16 into its P buffer
 //   O += P V    4 tcgen05.mma (M128 N192 K16), A = P from TMEM, B = V (SMEM, MN-major)
-// The MMA warp issues S(j+2) before O += P(j) V(j), so the softmax always
-// finds the next scores computed; it waits on an O update only for the
-// (rare) rescale.
+// The QK^T warp runs up to two tiles ahead of the PV warp (as far as the S
+// buffers the softmax releases allow), so the softmax always finds the next
+// scores computed; it waits on an O update only for the (rare) rescale.
 // Warp roles: warp 0 streams K and warp 10 streams V by TMA (one 5-D box per
 // 8-token block gathers all 192 dims: 3 KB), warp 1 allocates TMEM and issues
-// the MMAs, warps 2-9 run the softmax and the epilogue.  The producer and MMA
+// the QK^T MMAs, warp 11 issues the PV MMAs, warps 2-9 run the softmax and
+// the epilogue.  The producer and MMA
 // warps run converged and hand each TMA or MMA batch to one elected lane:
 // issuing from a lone divergent lane costs the tensor pipe several hundred
 // cycles per tile in synchronisation stalls.  Every mbarrier wait is bounded
@@ -44,7 +45,7 @@ namespace sgqa {
 
 constexpr int kTcStages = 4;      // K ring depth (K freed after QK^T)
 constexpr int kTcVStages = 4;     // V ring depth (V freed after PV)
-constexpr int kTcThreads = 352;   // K producer, MMA, 8 softmax warps, V producer
+constexpr int kTcThreads = 384;   // K producer, QK issuer, 8 softmax warps, V producer, PV issuer
 constexpr int kTcTileTok = 64;    // tokens per KV tile = 8 blocks of 8
 
 struct __align__(1024) AttnTcSmem {
@@ -57,7 +58,7 @@ struct __align__(1024) AttnTcSmem {
   uint64_t s_free[2];                      // S(j) loaded by the softmax (the 128 threads of tile j's warps)
   uint64_t p_full[2];                      // P(j) in P buffer j % 2 (the 128 threads of tile j's warps)
   uint64_t pv_done[2];                     // O += P(j) V(j) complete: P buffer j % 2 free, O current
-  uint64_t o_final, drain;
+  uint64_t o_final, drain, drain_pv;
   float mchain[128];                       // running reference max after the latest tile, per row
   float lsum[2][128];                      // partial row sums of the two warps of a quadrant
   uint32_t tmem;
@@ -112,6 +113,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     }
     tc::mbar_init(bar(sm.o_final), 1);
     tc::mbar_init(bar(sm.drain), 1);
+    tc::mbar_init(bar(sm.drain_pv), 1);
     tc::mbar_fence_init();
   }
   if (warp == 1) tc::tmem_alloc(smem_u32(&sm.tmem), 512);
@@ -131,28 +133,31 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     const int nst = is_k ? kTcStages : kTcVStages;
     if (tc::elect_one()) tc::prefetch_tmap(is_k ? &kmap : &vmap);
     __syncwarp();
-    // block ids of upcoming union tiles, fetched two tiles ahead
-    auto tile_rows = [&](int j, int32_t (&rows)[8]) {
-      if (j < n_union_tiles) {
-        const int4 a4 = *reinterpret_cast<const int4*>(uid + 8 * j);
-        const int4 b4 = *reinterpret_cast<const int4*>(uid + 8 * j + 4);
-        const int32_t ids[8] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) rows[e] = (8 * j + e < U) ? ids[e] * 8 : -64;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          rows[e] = (e == 0 || (e == 1 && c0 + 8 <= t_last)) ? static_cast<int32_t>(c0 + 8 * e) : -64;
-      }
+    // Block ids of the union, one per lane in batches of four tiles (32 ids),
+    // loaded a whole batch ahead: the id fetch (an L2 round trip) never sits
+    // between two tiles' copies.  Lane 8 t + e holds block e of tile 4 b + t.
+    auto load_batch = [&](int bt) -> int32_t {
+      const int idx = 32 * bt + lane;
+      return idx < U ? uid[idx] : -1;
     };
-    int32_t rows[8], next[8];
-    tile_rows(0, rows);
-    if (n_tiles > 1) tile_rows(1, next);
+    int32_t ids_cur = load_batch(0), ids_next = n_union_tiles > 4 ? load_batch(1) : -1;
     int issued = 0;
     for (int j = 0; j < n_tiles; ++j) {
       const int s = j % nst;
-      int32_t next2[8];
-      if (j + 2 < n_tiles) tile_rows(j + 2, next2);
+      if (j > 0 && (j & 3) == 0) {
+        ids_cur = ids_next;
+        if (4 * (j / 4 + 1) < n_union_tiles) ids_next = load_batch(j / 4 + 1);
+      }
+      // this tile's eight token rows (-64: a zero-filled box)
+      int32_t rows[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int32_t id = __shfl_sync(0xffffffffu, ids_cur, 8 * (j & 3) + e);
+        if (j < n_union_tiles)
+          rows[e] = id >= 0 ? id * 8 : -64;
+        else  // the current block and, when the unit spans two blocks, the next
+          rows[e] = (e == 0 || (e == 1 && c0 + 8 <= t_last)) ? static_cast<int32_t>(c0 + 8 * e) : -64;
+      }
       uint64_t* empty = is_k ? &sm.k_empty[s] : &sm.v_empty[s];
       uint64_t* full = is_k ? &sm.k_full[s] : &sm.v_full[s];
       if (j >= nst && !tc::warp_wait(bar(*empty), ((j / nst) - 1) & 1, abort)) break;
@@ -167,11 +172,6 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       }
       __syncwarp();
       issued = j + 1;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        rows[e] = next[e];
-        next[e] = next2[e];
-      }
     }
     if (*abort) {
       // Let the copies already issued land before the CTA's shared memory goes away.
@@ -182,8 +182,14 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 11) {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp 1 issues S(j) = Q K(j)^T, warp 11 issues O += P(j) V(j).  They
+    // touch disjoint TMEM (S buffers / O and P buffers) and each commit tracks
+    // its own warp's MMAs, so neither waits on the other: the scores run up
+    // to two tiles ahead (bounded by the S buffers the softmax releases) while
+    // PV follows the softmax.
+    const bool is_qk = warp == 1;
     const uint32_t id_qk = tc::idesc_bf16(128, 64, false);
     const uint32_t id_pv = tc::idesc_bf16(128, 192, true);
     // Base descriptors once per unit; each MMA adds a constant offset (in
@@ -191,74 +197,56 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     // stage x starts x * 24 KB (1536 units) after stage 0.
     const uint64_t dk0 = tc::sdesc_sw128(smem_u32(&sm.k[0][0][0][0]), 16, 3072);
     const uint64_t dv0 = tc::sdesc_sw128(smem_u32(&sm.v[0][0][0][0]), 1024, 3072);
-    auto issue_qk = [&](int j) {
-      const int s = j % kTcStages, b = j % 2;
-      if (tc::elect_one()) {
-        const uint64_t b0 = dk0 + 1536 * s;
-#pragma unroll
-        for (int kk = 0; kk < 12; ++kk)  // Q: 8 columns per 16 dims; K: +1 KB per 64 dims, +32 B per 16
-          tc::mma_f16_tmem_a(tS0 + 64 * b, tQ + 8 * kk, b0 + (kk >> 2) * 64 + (kk & 3) * 2, id_qk,
-                             kk > 0 ? 1u : 0u);
-        tc::mma_commit(bar(sm.k_empty[s]));
-        tc::mma_commit(bar(sm.s_full[b]));
-      }
-      __syncwarp();
-    };
-    auto issue_pv = [&](int j) {
-      const int s = j % kTcVStages, b = j % 2;
-      if (tc::elect_one()) {
-        const uint64_t b0 = dv0 + 1536 * s;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // P: 8 columns per 16 tokens; V: +2 blocks (6144 B) per 16 tokens
-          tc::mma_f16_tmem_a(tO, tP0 + 32 * b + 8 * kk, b0 + 384 * kk, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        tc::mma_commit(bar(sm.v_empty[s]));
-        tc::mma_commit(bar(sm.pv_done[b]));
-      }
-      __syncwarp();
-    };
-    bool ok = tc::warp_wait(bar(sm.q_full), 0, abort) && tc::warp_wait(bar(sm.k_full[0]), 0, abort);
-    tc::fence_after();
-    if (ok) issue_qk(0);
-    if (ok && n_tiles > 1) {
-      ok = tc::warp_wait(bar(sm.k_full[1]), 0, abort);
-      tc::fence_after();
-      if (ok) issue_qk(1);
-    }
-    for (int j = 0; ok && j < n_tiles; ++j) {
-      // Iteration j issues S(j+2) = Q K(j+2)^T, then O += P(j) V(j), so the
-      // softmax always has the next tile's scores waiting.  Three of its four
-      // conditions are usually met by now (K(j+2) and V(j) landed, S buffer
-      // j % 2 loaded by the softmax of tile j): one combined test, bounded
-      // waits only for what it found missing; then wait for P(j).
-      const int jn = j + 2, sk = jn % kTcStages, sv = j % kTcVStages, bn = j % 2;
-      const bool has_next = jn < n_tiles;
-      const uint32_t ready = tc::mbar_test3(bar(sm.k_full[sk]), (jn / kTcStages) & 1, bar(sm.v_full[sv]),
-                                            (j / kTcVStages) & 1, bar(sm.s_free[bn]), (j / 2) & 1);
-      const uint32_t need = has_next ? 7u : 2u;
-      if (!__all_sync(0xffffffffu, (ready & need) == need)) {
-        if (has_next) ok = tc::warp_wait(bar(sm.k_full[sk]), (jn / kTcStages) & 1, abort);
-        ok = ok && tc::warp_wait(bar(sm.v_full[sv]), (j / kTcVStages) & 1, abort);
-        if (has_next) ok = ok && tc::warp_wait(bar(sm.s_free[bn]), (j / 2) & 1, abort);
+    bool ok = true;
+    if (is_qk) {
+      ok = tc::warp_wait(bar(sm.q_full), 0, abort);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int s = j % kTcStages, b = j % 2;
+        ok = tc::warp_wait(bar(sm.k_full[s]), (j / kTcStages) & 1, abort);
+        // S buffer b is free once the softmax of tile j-2 has loaded it
+        if (ok && j >= 2) ok = tc::warp_wait(bar(sm.s_free[b]), ((j / 2) - 1) & 1, abort);
         if (!ok) break;
+        tc::fence_after();
+        if (tc::elect_one()) {
+          const uint64_t b0 = dk0 + 1536 * s;
+#pragma unroll
+          for (int kk = 0; kk < 12; ++kk)  // Q: 8 columns per 16 dims; K: +1 KB per 64 dims, +32 B per 16
+            tc::mma_f16_tmem_a(tS0 + 64 * b, tQ + 8 * kk, b0 + (kk >> 2) * 64 + (kk & 3) * 2, id_qk,
+                               kk > 0 ? 1u : 0u);
+          tc::mma_commit(bar(sm.k_empty[s]));
+          tc::mma_commit(bar(sm.s_full[b]));
+        }
+        __syncwarp();
       }
-      tc::fence_after();
-      if (has_next) issue_qk(jn);
-      if (!tc::warp_wait(bar(sm.p_full[j % 2]), (j / 2) & 1, abort)) {
-        ok = false;
-        break;
-      }
-      tc::fence_after();
-      issue_pv(j);
-    }
-    if (ok) {
-      if (tc::elect_one()) tc::mma_commit(bar(sm.o_final));
-      __syncwarp();
     } else {
-      // Let the MMAs already issued finish before TMEM is released.
-      if (tc::elect_one()) tc::mma_commit(bar(sm.drain));
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int s = j % kTcVStages, b = j % 2;
+        ok = tc::warp_wait(bar(sm.v_full[s]), (j / kTcVStages) & 1, abort) &&
+             tc::warp_wait(bar(sm.p_full[b]), (j / 2) & 1, abort);
+        if (!ok) break;
+        tc::fence_after();
+        if (tc::elect_one()) {
+          const uint64_t b0 = dv0 + 1536 * s;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // P: 8 columns per 16 tokens; V: +2 blocks (6144 B) per 16 tokens
+            tc::mma_f16_tmem_a(tO, tP0 + 32 * b + 8 * kk, b0 + 384 * kk, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_commit(bar(sm.v_empty[s]));
+          tc::mma_commit(bar(sm.pv_done[b]));
+        }
+        __syncwarp();
+      }
+      if (ok) {
+        if (tc::elect_one()) tc::mma_commit(bar(sm.o_final));
+        __syncwarp();
+      }
+    }
+    if (!ok) {
+      // Let this warp's MMAs already issued finish before TMEM is released.
+      uint64_t& d = is_qk ? sm.drain : sm.drain_pv;
+      if (tc::elect_one()) tc::mma_commit(bar(d));
       __syncwarp();
       const uint64_t t0 = globaltimer_ns();
-      while (!tc::mbar_try(bar(sm.drain), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+      while (!tc::mbar_try(bar(d), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
       }
     }
   } else {
