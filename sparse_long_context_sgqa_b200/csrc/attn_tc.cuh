@@ -65,6 +65,10 @@ struct __align__(1024) AttnTcSmem {
   int abort;
 };
 
+// SKIP_PAIRS: skip the exponentials of block pairs that no row of a warp
+// attends (pays when selections cover a small part of the context); otherwise
+// all 64 exponentials of a tile run as one branch-free block.
+template <bool SKIP_PAIRS>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUtensorMap kmap,
                const __grid_constant__ CUtensorMap vmap, const int32_t* __restrict__ plan_ids,
@@ -383,26 +387,33 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
         m_l = m_use;
       }
       // P = 2^(s * scale - m_use) in BF16, packed two tokens per column.  A
-      // block the row does not attend has offset -inf (P = 0); blocks no row
-      // of this warp attends skip their exponentials.
+      // block the row does not attend has offset -inf (P = 0).  Exponentials
+      // run in pairs of blocks (16 per branch-free chunk, so their latencies
+      // overlap); with SKIP_PAIRS a pair no row of this warp attends is skipped.
       const float neg_m = m_use == -INFINITY ? 0.f : -m_use;
-      const uint32_t wmask = __reduce_or_sync(0xffffffffu, bmask);
+      const uint32_t wmask = SKIP_PAIRS ? __reduce_or_sync(0xffffffffu, bmask) : 0xFFu;
       float ls[8];
       uint32_t pk[32];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        ls[e] = 0.f;
-        if ((wmask >> e) & 1u) {
-          const float off = ((bmask >> e) & 1u) ? neg_m : -INFINITY;
-          float pe[8];
+      for (int e2 = 0; e2 < 8; e2 += 2) {
+        if (!SKIP_PAIRS || ((wmask >> e2) & 3u)) {
 #pragma unroll
-          for (int x = 0; x < 8; ++x) pe[x] = fast_exp2(fmaf(__uint_as_float(sr[8 * e + x]), scale_log2, off));
-          ls[e] = ((pe[0] + pe[1]) + (pe[2] + pe[3])) + ((pe[4] + pe[5]) + (pe[6] + pe[7]));
+          for (int e = e2; e < e2 + 2; ++e) {
+            const float off = ((bmask >> e) & 1u) ? neg_m : -INFINITY;
+            float pe[8];
 #pragma unroll
-          for (int x = 0; x < 4; ++x) pk[4 * e + x] = pack_bf16x2(pe[2 * x], pe[2 * x + 1]);
+            for (int x = 0; x < 8; ++x) pe[x] = fast_exp2(fmaf(__uint_as_float(sr[8 * e + x]), scale_log2, off));
+            ls[e] = ((pe[0] + pe[1]) + (pe[2] + pe[3])) + ((pe[4] + pe[5]) + (pe[6] + pe[7]));
+#pragma unroll
+            for (int x = 0; x < 4; ++x) pk[4 * e + x] = pack_bf16x2(pe[2 * x], pe[2 * x + 1]);
+          }
         } else {
 #pragma unroll
-          for (int x = 0; x < 4; ++x) pk[4 * e + x] = 0u;
+          for (int e = e2; e < e2 + 2; ++e) {
+            ls[e] = 0.f;
+#pragma unroll
+            for (int x = 0; x < 4; ++x) pk[4 * e + x] = 0u;
+          }
         }
       }
       const float lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));

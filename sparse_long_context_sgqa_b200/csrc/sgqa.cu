@@ -249,8 +249,12 @@ sgqa_status launch_attn_tc(const sgqa_params* p, int64_t S, int64_t q0, int64_t 
   }
   static_assert(sizeof(sgqa::AttnTcSmem) + 1024 <= 232448, "attention tile exceeds shared memory");
   const size_t smem = sizeof(sgqa::AttnTcSmem) + 1024;
-  cudaFuncSetAttribute(sgqa::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  sgqa::attn_tc_kernel<<<static_cast<unsigned>(units), sgqa::kTcThreads, smem, st>>>(
+  // Selections covering under a quarter of the candidates leave many block
+  // pairs unattended by both queries of a warp: skip their exponentials.
+  const bool skip_pairs = (q0 + nq - 1) / p->block_size > 4 * static_cast<int64_t>(p->topk);
+  auto kern = skip_pairs ? sgqa::attn_tc_kernel<true> : sgqa::attn_tc_kernel<false>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  kern<<<static_cast<unsigned>(units), sgqa::kTcThreads, smem, st>>>(
       static_cast<const __nv_bfloat16*>(q), km, vm, ids, msk, cnt, static_cast<__nv_bfloat16*>(out), nq, G,
       p->topk, q0, scale_log2);
   SGQA_LAUNCH_CHECK("attn_tc_kernel");
