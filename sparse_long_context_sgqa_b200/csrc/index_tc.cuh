@@ -50,12 +50,33 @@ struct __align__(1024) IndexTcSmem {
 // (id_cut), so that {key > theta} + {key == theta, id <= id_cut} is exactly k
 // entries -- every key above the k-th and the smallest ids among its ties.
 // Radix select on the 32-bit order-preserving keys, 8 bits per pass from the
-// top; ties by a second radix select on the (distinct) ids.
+// top; ties by a second radix select on the (distinct) ids.  The passes start
+// at the highest byte in which the entries differ: the bits above it are
+// common to all of them, so the passes over those would pick them with the
+// count unchanged.
+__device__ __forceinline__ void common_high_bits(uint32_t and_all, uint32_t or_all, uint32_t& prefix,
+                                                 uint32_t& mask, int& shift) {
+  const uint32_t diff = and_all ^ or_all;
+  shift = diff ? (31 - __clz(static_cast<int>(diff))) / 8 * 8 : -8;
+  mask = shift >= 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+  prefix = and_all & mask;
+}
 __device__ __noinline__ void warp_select(const uint2* buf, int n, int k, uint32_t* hist, uint32_t& theta,
                                          uint32_t& id_cut) {
   const int lane = threadIdx.x & 31;
   uint32_t prefix = 0, mask = 0, rem = static_cast<uint32_t>(k);
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  int shift0;
+  {
+    uint32_t a = 0xFFFFFFFFu, o = 0u;
+    for (int i = lane; i < n; i += 32) {
+      a &= buf[i].x;
+      o |= buf[i].x;
+    }
+    a = __reduce_and_sync(0xffffffffu, a);
+    o = __reduce_or_sync(0xffffffffu, o);
+    common_high_bits(a, o, prefix, mask, shift0);
+  }
+  for (int shift = shift0; shift >= 0; shift -= 8) {
     for (int b = lane; b < 256; b += 32) hist[b] = 0;
     __syncwarp();
     for (int i = lane; i < n; i += 32) {
@@ -95,7 +116,21 @@ __device__ __noinline__ void warp_select(const uint2* buf, int n, int k, uint32_
   id_cut = 0xFFFFFFFFu;
   if (static_cast<uint32_t>(ties) > rem) {
     uint32_t ipre = 0, imask = 0, irem = rem;
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    int ishift0;
+    {
+      uint32_t a = 0xFFFFFFFFu, o = 0u;
+      for (int i = lane; i < n; i += 32) {
+        const uint2 e = buf[i];
+        if (e.x == theta) {
+          a &= e.y;
+          o |= e.y;
+        }
+      }
+      a = __reduce_and_sync(0xffffffffu, a);
+      o = __reduce_or_sync(0xffffffffu, o);
+      common_high_bits(a, o, ipre, imask, ishift0);
+    }
+    for (int shift = ishift0; shift >= 0; shift -= 8) {
       for (int b = lane; b < 256; b += 32) hist[b] = 0;
       __syncwarp();
       for (int i = lane; i < n; i += 32) {
@@ -816,70 +851,97 @@ topk_final_kernel(const uint2* __restrict__ staging, const int32_t* __restrict__
 
 
 // ---------------------------------------------------------------------------
-// Top-k for rows of at most kWinThreads * kWinPer candidates (every prefill
-// row up to a 131072-token context): the row is read from HBM once into
-// registers (thread t holds candidates t, t + 512, ...).  A 256-bin histogram
-// of the scores, linear between the row's minimum and maximum, finds the bin
-// b* holding the k-th largest; a linear bin is a monotone function of the
-// score, so every candidate of a higher bin beats every candidate of b*, and
-// only b* needs an exact (score, then smaller id) selection.  The selection is
-// a bitmap built with one ballot per warp and iteration (a warp's 32 lanes
-// hold 32 consecutive ids = one bitmap word), read out in ascending id order.
-// A row whose boundary bin holds more than kWinCand candidates (massive exact
-// ties) is flagged in `overflow` and left to the radix kernel.
+// Top-k for rows of 2048 .. kHistMaxCand candidates (every prefill row up to a
+// 131072-token context).  One 128-thread CTA per row, about 22 KB of shared
+// memory, so many rows are in flight per SM; the row streams through
+// registers.
+//
+// Survivor filter (rows of more than 4k candidates): a sample of an eighth of
+// the row (every eighth float4) gives a threshold T expected to pass about 2k
+// candidates; one pass over the row appends the survivors (score >= T) as
+// (score, id) to a shared list, one atomic per warp and batch.  If at least k
+// survive, the k largest of the row are all among them; otherwise (or if too
+// many survive) the exact step below runs over the whole row instead.
+//
+// Exact step (over the survivors, or the whole row): a 256-bin histogram of
+// the scores, linear between their minimum and maximum, finds the bin b*
+// holding the k-th largest.  Every step of the bin function rounds
+// monotonically, so the bin never decreases as the score falls: each entry of
+// a lower bin beats each entry of b*, and only b* needs the exact (score, then
+// smaller id) order.  When b* holds more entries than the boundary buffer, a
+// second 256-bin level splits b* the same way.  Selected ids are set in a
+// bitmap read out in ascending id order.  A row whose boundary still
+// overflows (massive exact ties) is flagged and listed for the radix kernel.
 // ---------------------------------------------------------------------------
-constexpr int kWinThreads = 512;
-constexpr int kWinWarps = kWinThreads / 32;
-constexpr int kWinPer = 32;
-constexpr int kWinMaxCand = kWinThreads * kWinPer;  // 16384
-constexpr int kWinBins = 256;
-constexpr int kWinCand = 2048;
+constexpr int kHistThreads = 128;
+constexpr int kHistWarps = kHistThreads / 32;
+constexpr int kHistBins = 256;         // 16-bit counters, two per word
+constexpr int kHistBnd = 256;          // boundary entries resolved in the kernel
+constexpr int kHistSurv = 2048;        // survivors of the sampled threshold
+constexpr int kHistMaxCand = 16384;
+constexpr int kHistSampPer = kHistMaxCand / 32 / kHistThreads;  // sample float4s per thread
+constexpr int kHistBatch = 8;          // float4s per thread in flight in the survivor pass
+constexpr uint32_t kHistRankMax = 64;  // boundary sets up to this size are ranked by all threads at once
+static_assert(kHistBins == 2 * kHistThreads, "one histogram word (two bins) per thread in the bin scan");
+static_assert(kHistMaxCand < 65536, "per-warp bin counts fit 16 bits");
 
-struct WinSmem {
-  uint32_t wh[kWinWarps][kWinBins];   // per-warp histograms (also warp_select scratch)
-  uint2 cand[kWinCand];               // (key, id) of the boundary bin
-  uint32_t bits[kWinMaxCand / 32];    // selection bitmap
-  float rmax[kWinWarps], rmin[kWinWarps];
-  uint32_t wsum[kWinWarps];
-  uint32_t bstar, rem, nc;
+struct HistSmem {
+  uint32_t wh[kHistWarps][kHistBins / 2];  // per-warp histograms (also warp_select scratch)
+  uint2 bnd[kHistBnd];                     // (key, id) of the boundary bin
+  uint2 surv[kHistSurv];                   // survivors as (score bits, id)
+  uint32_t bits[kHistMaxCand / 32];        // selection bitmap
+  float rmax[kHistWarps], rmin[kHistWarps];
+  uint32_t wsum[kHistWarps];
+  uint32_t bstar, rem, cstar, nc, nsurv;
 };
 
-__global__ void __launch_bounds__(kWinThreads, 2)
-topk_rows_win_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int G, int64_t q_pos0, int B,
-                     int k, int32_t* __restrict__ sel, int32_t* __restrict__ sel_count,
-                     int32_t* __restrict__ overflow, int32_t* __restrict__ list, int32_t* __restrict__ list_count) {
-  __shared__ WinSmem sm;
-  const int64_t row = blockIdx.x;  // (seq * nq + i) * G + g
-  const int64_t i = (row / G) % nq;
-  const int n = static_cast<int>((q_pos0 + i) / B);
-  const float* srow = scores + row * rpad;
-  int32_t* out = sel + row * k;
+// A float in [2^23, 2^24) is an integer (ulp 1); adding 1.5 * 2^23 to a value
+// in [0, 2^22) rounds it to the nearest integer, readable as the bit pattern
+// minus that of 1.5 * 2^23.
+constexpr float kRoundBase = 12582912.0f;
+constexpr int kRoundBits = 0x4B400000;
+
+__device__ __forceinline__ void hist_add(uint32_t* h, int b) { atomicAdd(&h[b >> 1], 1u << ((b & 1) * 16)); }
+
+// Bins are ordered best first.  Finds the bin of sm.wh in which the running
+// count reaches `need` (1 <= need <= total), its count, and the rank of `need`
+// inside it (sm.bstar, sm.cstar, sm.rem).  Called by every thread of the CTA.
+__device__ __forceinline__ void hist_boundary(HistSmem& sm, uint32_t need) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (n <= k) {
-    for (int j = tid; j < k; j += kWinThreads) out[j] = j < n ? j : -1;
-    if (tid == 0) {
-      sel_count[row] = n;
-      overflow[row] = 0;
-    }
-    return;
-  }
-  const int nper = (n + kWinThreads - 1) / kWinThreads;  // iterations that hold real candidates
-  float v[kWinPer];
+  uint32_t c0 = 0, c1 = 0;
 #pragma unroll
-  for (int e = 0; e < kWinPer; ++e) {
-    const int id = tid + kWinThreads * e;
-    v[e] = (e < nper && id < n) ? __ldcs(srow + id) : -INFINITY;
+  for (int w = 0; w < kHistWarps; ++w) {
+    const uint32_t pr = sm.wh[w][tid];
+    c0 += pr & 0xFFFFu;
+    c1 += pr >> 16;
   }
-  for (int b = tid; b < kWinWarps * kWinBins; b += kWinThreads) (&sm.wh[0][0])[b] = 0u;
-  if (tid == 0) sm.nc = 0;
-  // row maximum and minimum (over real candidates)
-  float mx = -INFINITY, mn = INFINITY;
+  const uint32_t c = c0 + c1;
+  uint32_t inc = c;
 #pragma unroll
-  for (int e = 0; e < kWinPer; ++e) {
-    if (e >= nper) break;
-    mx = fmaxf(mx, v[e]);
-    if (tid + kWinThreads * e < n) mn = fminf(mn, v[e]);
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
   }
+  if (lane == 31) sm.wsum[warp] = inc;
+  __syncthreads();
+  uint32_t before = inc - c;
+  for (int w = 0; w < warp; ++w) before += sm.wsum[w];
+  if (before < need && need <= before + c0) {
+    sm.bstar = 2 * tid;
+    sm.rem = need - before;
+    sm.cstar = c0;
+  } else if (before + c0 < need && need <= before + c) {
+    sm.bstar = 2 * tid + 1;
+    sm.rem = need - before - c0;
+    sm.cstar = c1;
+  }
+  __syncthreads();
+}
+
+// Maximum and minimum over the CTA (every thread gets both; NaN inputs are
+// ignored).
+__device__ __forceinline__ void block_minmax(HistSmem& sm, float& mx, float& mn) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -891,86 +953,295 @@ topk_rows_win_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq,
   }
   __syncthreads();
 #pragma unroll
-  for (int w = 0; w < kWinWarps; ++w) {
+  for (int w = 0; w < kHistWarps; ++w) {
     mx = fmaxf(mx, sm.rmax[w]);
     mn = fminf(mn, sm.rmin[w]);
   }
-  // bin = floor((max - s) * scale), 0 for the maximum, at most 255 for the minimum
+}
+
+__device__ __forceinline__ void zero_hist(HistSmem& sm) {
+  for (int b = threadIdx.x; b < kHistWarps * kHistBins / 2; b += kHistThreads) (&sm.wh[0][0])[b] = 0u;
+}
+
+__global__ void __launch_bounds__(kHistThreads)
+topk_rows_hist_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int G, int64_t q_pos0, int B,
+                      int k, int32_t* __restrict__ sel, int32_t* __restrict__ sel_count,
+                      int32_t* __restrict__ overflow, int32_t* __restrict__ list, int32_t* __restrict__ list_count) {
+  __shared__ HistSmem sm;
+  const int64_t row = blockIdx.x;  // (seq * nq + i) * G + g
+  const int64_t i = (row / G) % nq;
+  const int n = static_cast<int>((q_pos0 + i) / B);
+  const float* srow = scores + row * rpad;  // 16-byte aligned (rpad is a multiple of 128)
+  const float4* r4 = reinterpret_cast<const float4*>(srow);
+  int32_t* out = sel + row * k;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (n <= k) {
+    for (int j = tid; j < k; j += kHistThreads) out[j] = j < n ? j : -1;
+    if (tid == 0) {
+      sel_count[row] = n;
+      overflow[row] = 0;
+    }
+    return;
+  }
+  if (tid == 0) {
+    sm.nc = 0;
+    sm.nsurv = 0;
+    // the whole row (rounded up to float4s; the padded row has room) into L2
+    // while the sample is read and binned
+    tc::prefetch_l2(srow, static_cast<uint32_t>((n + 3) / 4) * 16u);
+  }
+  zero_hist(sm);
+  for (int w = tid; w < kHistMaxCand / 32; w += kHistThreads) sm.bits[w] = 0u;
+  __syncthreads();
+
+  const int nwords = (n + 31) / 32;
+  uint32_t* myh = sm.wh[warp];
+  bool use_surv = false;
+  float smax_surv = -INFINITY, smin_surv = INFINITY;
+  if (n > 4 * k && 2 * k <= kHistSurv / 2) {
+    // ---- sampled threshold: the float4s 8 j (candidates 32 j .. 32 j + 3),
+    // held in registers; samples past the row are NaN (ignored by min/max)
+    const int s4 = n / 32, s = 4 * s4;
+    float4 sv[kHistSampPer];
+#pragma unroll
+    for (int q = 0; q < kHistSampPer; ++q) {
+      const int j = tid + kHistThreads * q;
+      sv[q] = j < s4 ? __ldg(r4 + 8 * j) : make_float4(NAN, NAN, NAN, NAN);
+    }
+    float smx = -INFINITY, smn = INFINITY;
+#pragma unroll
+    for (int q = 0; q < kHistSampPer; ++q) {
+      smx = fmaxf(smx, fmaxf(fmaxf(sv[q].x, sv[q].y), fmaxf(sv[q].z, sv[q].w)));
+      smn = fminf(smn, fminf(fminf(sv[q].x, sv[q].y), fminf(sv[q].z, sv[q].w)));
+    }
+    block_minmax(sm, smx, smn);
+    const float sw = smx - smn;
+    const float sscale = sw > 0.f ? 255.5f / sw : 0.f;
+    // t = (max - x) * scale: bin b holds t in [b - 0.5, b + 0.5], sub-bin u of
+    // b holds t in b + [u - 128.5, u - 127.5] / 256 (the exact step's bins)
+    auto sbin1 = [&](float x) -> int {
+      const float y = __fmaf_rn(__fsub_rn(smx, x), sscale, kRoundBase);
+      return min(__float_as_int(y) - kRoundBits, kHistBins - 1);
+    };
+#pragma unroll
+    for (int q = 0; q < kHistSampPer; ++q) {
+      if (tid + kHistThreads * q < s4) {
+        hist_add(myh, sbin1(sv[q].x));
+        hist_add(myh, sbin1(sv[q].y));
+        hist_add(myh, sbin1(sv[q].z));
+        hist_add(myh, sbin1(sv[q].w));
+      }
+    }
+    __syncthreads();
+    // the sample rank that corresponds to about 2k candidates of the row
+    const uint32_t r = static_cast<uint32_t>(min(static_cast<int>((2 * static_cast<int64_t>(k) * s + n - 1) / n), s));
+    hist_boundary(sm, r);
+    const int sb = static_cast<int>(sm.bstar);
+    // threshold half a bin below the boundary bin's lower edge, or, when that
+    // bin holds many samples, a sub-bin below its boundary sub-bin's
+    float t_thr = static_cast<float>(sb) + 1.0f;
+    if (sm.cstar > 16u) {
+      const float sscale2 = sscale * 256.f;
+      const float sbase2 = kRoundBase + 128.f - 256.f * static_cast<float>(sb);
+      const uint32_t srem = sm.rem;
+      zero_hist(sm);
+      __syncthreads();
+      auto sadd2 = [&](float x) {
+        if (sbin1(x) == sb) {
+          const float y = __fmaf_rn(__fsub_rn(smx, x), sscale2, sbase2);
+          hist_add(myh, max(min(__float_as_int(y) - kRoundBits, kHistBins - 1), 0));
+        }
+      };
+#pragma unroll
+      for (int q = 0; q < kHistSampPer; ++q) {
+        if (tid + kHistThreads * q < s4) {
+          sadd2(sv[q].x);
+          sadd2(sv[q].y);
+          sadd2(sv[q].z);
+          sadd2(sv[q].w);
+        }
+      }
+      __syncthreads();
+      hist_boundary(sm, srem);
+      t_thr = static_cast<float>(sb) + (static_cast<float>(sm.bstar) - 126.5f) / 256.f;
+    }
+    const float thr = sscale > 0.f ? smx - t_thr / sscale : smx;
+    // ---- survivors, batch by batch: each lane's passes as a bit mask, one
+    // atomic per warp for the batch's positions
+    const int nfull = n / 4;
+    float smax = -INFINITY;  // largest survivor
+    for (int base = 0; base < nfull; base += kHistThreads * kHistBatch) {
+      float4 v[kHistBatch];
+#pragma unroll
+      for (int u = 0; u < kHistBatch; ++u) {
+        const int j = base + kHistThreads * u + tid;
+        v[u] = j < nfull ? __ldg(r4 + j) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      }
+      uint32_t mask = 0;
+#pragma unroll
+      for (int u = 0; u < kHistBatch; ++u) {
+        mask |= static_cast<uint32_t>(v[u].x >= thr) << (4 * u);
+        mask |= static_cast<uint32_t>(v[u].y >= thr) << (4 * u + 1);
+        mask |= static_cast<uint32_t>(v[u].z >= thr) << (4 * u + 2);
+        mask |= static_cast<uint32_t>(v[u].w >= thr) << (4 * u + 3);
+      }
+      const uint32_t cnt = __popc(mask);
+      uint32_t inc = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      uint32_t pos = 0;
+      if (lane == 31 && inc) pos = atomicAdd(&sm.nsurv, inc);
+      pos = __shfl_sync(0xffffffffu, pos, 31) + inc - cnt;
+      // the lane's survivors, re-read from L1 (their lines were just loaded)
+      while (mask) {
+        const int b = __ffs(mask) - 1;
+        mask &= mask - 1;
+        const int id = 4 * (base + kHistThreads * (b >> 2) + tid) + (b & 3);
+        const float x = __ldg(srow + id);
+        if (pos < static_cast<uint32_t>(kHistSurv)) sm.surv[pos] = make_uint2(__float_as_uint(x), static_cast<uint32_t>(id));
+        smax = fmaxf(smax, x);
+        ++pos;
+      }
+    }
+    for (int id = 4 * nfull + tid; id < n; id += kHistThreads) {
+      const float x = srow[id];
+      if (x >= thr) {
+        const uint32_t p = atomicAdd(&sm.nsurv, 1u);
+        if (p < static_cast<uint32_t>(kHistSurv)) sm.surv[p] = make_uint2(__float_as_uint(x), static_cast<uint32_t>(id));
+        smax = fmaxf(smax, x);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+    if (lane == 0) sm.rmax[warp] = smax;
+    __syncthreads();
+    const uint32_t total = sm.nsurv;
+    use_surv = total >= static_cast<uint32_t>(k) && total <= static_cast<uint32_t>(kHistSurv);
+    if (use_surv) {
+      // every survivor lies in [thr, largest survivor]
+      smin_surv = thr;
+      for (int w = 0; w < kHistWarps; ++w) smax_surv = fmaxf(smax_surv, sm.rmax[w]);
+    }
+    zero_hist(sm);
+    __syncthreads();
+  }
+
+  // ---- exact step over entries e < m: survivor e, or candidate e of the row
+  const int m = use_surv ? static_cast<int>(sm.nsurv) : n;
+  auto val = [&](int e) -> float { return use_surv ? __uint_as_float(sm.surv[e].x) : srow[e]; };
+  auto idx = [&](int e) -> int { return use_surv ? static_cast<int>(sm.surv[e].y) : e; };
+  float mx = smax_surv, mn = smin_surv;
+  if (!use_surv) {
+    for (int e = tid; e < m; e += kHistThreads) {
+      const float x = val(e);
+      mx = fmaxf(mx, x);
+      mn = fminf(mn, x);
+    }
+    block_minmax(sm, mx, mn);
+  }
+  // level-1 bin: round((max - s) * 255.5 / (max - min)), 0 for the maximum,
+  // at most 255; explicit roundings so every pass computes the same bin
   const float width = mx - mn;
   const float scale = width > 0.f ? 255.5f / width : 0.f;
-  auto bin_of = [&](float x) -> int { return min(static_cast<int>((mx - x) * scale), kWinBins - 1); };
-  uint32_t* myh = sm.wh[warp];
-#pragma unroll
-  for (int e = 0; e < kWinPer; ++e) {
-    if (e >= nper) break;
-    if (tid + kWinThreads * e < n) atomicAdd(&myh[bin_of(v[e])], 1u);
-  }
+  auto bin1 = [&](float x) -> int {
+    const float y = __fmaf_rn(__fsub_rn(mx, x), scale, kRoundBase);
+    return min(__float_as_int(y) - kRoundBits, kHistBins - 1);
+  };
+  for (int e = tid; e < m; e += kHistThreads) hist_add(myh, bin1(val(e)));
   __syncthreads();
-  // bin counts from the top; the bin where the running count reaches k
-  if (tid < kWinBins) {
-    uint32_t c = 0;
-#pragma unroll
-    for (int w = 0; w < kWinWarps; ++w) c += sm.wh[w][tid];
-    uint32_t inc = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += y;
-    }
-    if (lane == 31) sm.wsum[warp] = inc;
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    uint32_t before = inc - c;
-    for (int w = 0; w < warp; ++w) before += sm.wsum[w];
-    const uint32_t kk = static_cast<uint32_t>(k);
-    if (before < kk && kk <= before + c) {
-      sm.bstar = static_cast<uint32_t>(tid);
-      sm.rem = kk - before;
-    }
-  }
-  __syncthreads();
+  hist_boundary(sm, static_cast<uint32_t>(k));
   const int bstar = static_cast<int>(sm.bstar);
-  const uint32_t rem = sm.rem;
-  // higher bins straight into the bitmap; the boundary bin gathered
-  // bitmap words past the last iteration hold no candidate
-  if (tid >= nper * kWinWarps) sm.bits[tid] = 0u;
-#pragma unroll
-  for (int e = 0; e < kWinPer; ++e) {
-    if (e >= nper) break;
-    const bool real = tid + kWinThreads * e < n;
-    const int b = real ? bin_of(v[e]) : kWinBins;
-    const uint32_t above = __ballot_sync(0xffffffffu, b < bstar);
-    if (lane == 0) sm.bits[warp + kWinWarps * e] = above;
-    const bool eq = b == bstar;
-    const uint32_t bal = __ballot_sync(0xffffffffu, eq);
-    if (bal) {
+  uint32_t need = sm.rem;
+  // level 2 (boundary bin too full): 256 sub-bins of b*, the same construction
+  // with 256 times the scale; entries of b* land in [0, 256]
+  const bool lvl2 = sm.cstar > static_cast<uint32_t>(kHistBnd);
+  const float scale2 = scale * 256.f;
+  const float base2 = kRoundBase + 128.f - 256.f * static_cast<float>(bstar);
+  auto bin2 = [&](float x) -> int {
+    const float y = __fmaf_rn(__fsub_rn(mx, x), scale2, base2);
+    return max(min(__float_as_int(y) - kRoundBits, kHistBins - 1), 0);
+  };
+  int sstar = 0;
+  if (lvl2) {
+    zero_hist(sm);
+    __syncthreads();
+    for (int e = tid; e < m; e += kHistThreads) {
+      const float x = val(e);
+      if (bin1(x) == bstar) hist_add(myh, bin2(x));
+    }
+    __syncthreads();
+    hist_boundary(sm, need);
+    sstar = static_cast<int>(sm.bstar);
+    need = sm.rem;
+  }
+  // entries ranked above the boundary go straight into the selection bitmap,
+  // the boundary's are gathered as (key, id)
+  const int msteps = (m + kHistThreads - 1) / kHistThreads;
+  for (int it = 0; it < msteps; ++it) {
+    const int e = it * kHistThreads + tid;
+    const bool valid = e < m;
+    const float x = valid ? val(e) : 0.f;
+    const int id = valid ? idx(e) : 0;
+    const int b = valid ? bin1(x) : kHistBins;
+    bool above = b < bstar, eq = b == bstar;
+    if (lvl2 && eq) {
+      const int b2 = bin2(x);
+      above = b2 < sstar;
+      eq = b2 == sstar;
+    }
+    if (above) atomicOr(&sm.bits[id >> 5], 1u << (id & 31));
+    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
+    if (eb) {
       uint32_t base = 0;
-      if (lane == 0) base = atomicAdd(&sm.nc, static_cast<uint32_t>(__popc(bal)));
+      if (lane == 0) base = atomicAdd(&sm.nc, static_cast<uint32_t>(__popc(eb)));
       base = __shfl_sync(0xffffffffu, base, 0);
-      const uint32_t pos = base + __popc(bal & ((1u << lane) - 1u));
-      if (eq && pos < kWinCand) sm.cand[pos] = make_uint2(score_key(v[e]), static_cast<uint32_t>(tid + kWinThreads * e));
+      const uint32_t p = base + __popc(eb & ((1u << lane) - 1u));
+      if (eq && p < static_cast<uint32_t>(kHistBnd)) sm.bnd[p] = make_uint2(score_key(x), static_cast<uint32_t>(id));
     }
   }
   __syncthreads();
   const uint32_t nc = sm.nc;
-  if (nc > kWinCand) {
+  if (nc > static_cast<uint32_t>(kHistBnd)) {
     if (tid == 0) {
       overflow[row] = 1;
       list[atomicAdd(list_count, 1)] = static_cast<int32_t>(row);
     }
     return;
   }
-  if (warp == 0) {
+  // the `need` best of the nc boundary entries (need <= nc)
+  if (nc == need) {
+    for (uint32_t c = tid; c < nc; c += kHistThreads) {
+      const uint32_t id = sm.bnd[c].y;
+      atomicOr(&sm.bits[id >> 5], 1u << (id & 31));
+    }
+  } else if (nc <= kHistRankMax) {
+    if (static_cast<uint32_t>(tid) < nc) {
+      const uint2 q = sm.bnd[tid];
+      uint32_t r = 0;  // entries ranked ahead: larger key, or equal key and smaller id
+      for (uint32_t j = 0; j < nc; ++j) {
+        const uint2 f = sm.bnd[j];
+        r += (f.x > q.x) | ((f.x == q.x) & (f.y < q.y));
+      }
+      if (r < need) atomicOr(&sm.bits[q.y >> 5], 1u << (q.y & 31));
+    }
+  } else if (warp == 0) {
     uint32_t theta = 0, id_cut = 0xFFFFFFFFu;
-    if (nc > rem) warp_select(sm.cand, static_cast<int>(nc), static_cast<int>(rem), sm.wh[0], theta, id_cut);
+    warp_select(sm.bnd, static_cast<int>(nc), static_cast<int>(need), &sm.wh[0][0], theta, id_cut);
     for (uint32_t c = lane; c < nc; c += 32) {
-      const uint2 e = sm.cand[c];
-      if (nc <= rem || kept(e, theta, id_cut)) atomicOr(&sm.bits[e.y >> 5], 1u << (e.y & 31));
+      const uint2 q = sm.bnd[c];
+      if (kept(q, theta, id_cut)) atomicOr(&sm.bits[q.y >> 5], 1u << (q.y & 31));
     }
   }
   __syncthreads();
-  // ascending readout: thread t owns bitmap word t (ids 32 t .. 32 t + 31)
-  const uint32_t word = sm.bits[tid];
-  const uint32_t cnt = __popc(word);
+  // ascending readout: thread t owns words [t * wpt, t * wpt + wpt)
+  const int wpt = (nwords + kHistThreads - 1) / kHistThreads;
+  const int w0 = tid * wpt;
+  uint32_t cnt = 0;
+  for (int w = 0; w < wpt; ++w)
+    if (w0 + w < nwords) cnt += __popc(sm.bits[w0 + w]);
   uint32_t inc = cnt;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -981,12 +1252,15 @@ topk_rows_win_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq,
   __syncthreads();
   uint32_t pos = inc - cnt;
   for (int w = 0; w < warp; ++w) pos += sm.wsum[w];
-  uint32_t wb = word;
-  while (wb) {
-    const int bit = __ffs(wb) - 1;
-    wb &= wb - 1;
-    if (pos < static_cast<uint32_t>(k)) out[pos] = 32 * tid + bit;
-    ++pos;
+  for (int w = 0; w < wpt; ++w) {
+    if (w0 + w >= nwords) break;
+    uint32_t wb = sm.bits[w0 + w];
+    while (wb) {
+      const int bit = __ffs(wb) - 1;
+      wb &= wb - 1;
+      if (pos < static_cast<uint32_t>(k)) out[pos] = 32 * (w0 + w) + bit;
+      ++pos;
+    }
   }
   if (tid == 0) {
     sel_count[row] = k;

@@ -442,17 +442,18 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
   }
   const int nwords = static_cast<int>((std::max<int64_t>(rneed, 1) + 31) / 32);
   const size_t ssmem = (static_cast<size_t>(sgqa::kRows2Warps) * sgqa::kRows2Bins / 2 + 2 * sgqa::kRows2Cand + nwords) * 4;
-  // Rows of 2048 .. 16384 candidates: one HBM read into registers, a linear
-  // histogram and an exact boundary-bin select.  Long rows (>= 32768
-  // candidates): two passes over the row (histogram, then gather).  Rows either
-  // cannot finish (boundary-bin overflow) go to the radix kernel, which also
-  // takes the rows in between and short rows (its per-row set-up is smaller).
-  if (rneed >= 2048 && rneed <= sgqa::kWinMaxCand) {
+  // Rows of 2048 .. 16384 candidates: a sampled threshold, one pass over the
+  // row keeping the survivors, a linear histogram and an exact boundary-bin
+  // select over them.  Long rows (>= 32768 candidates): two passes over the
+  // row in HBM (histogram, then gather).  Rows either cannot finish
+  // (boundary-bin overflow) go to the radix kernel, which also takes the rows
+  // in between and short rows (its per-row set-up is smaller).
+  if (rneed >= 2048 && rneed <= sgqa::kHistMaxCand) {
     cudaError_t e = cudaMemsetAsync(list_count, 0, 4, st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(list count)");
-    sgqa::topk_rows_win_kernel<<<static_cast<unsigned>(rows), sgqa::kWinThreads, 0, st>>>(
+    sgqa::topk_rows_hist_kernel<<<static_cast<unsigned>(rows), sgqa::kHistThreads, 0, st>>>(
         scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, flags, list, list_count);
-    SGQA_LAUNCH_CHECK("topk_rows_win_kernel");
+    SGQA_LAUNCH_CHECK("topk_rows_hist_kernel");
     sgqa::topk_rows_list_kernel<<<static_cast<unsigned>(std::min<int64_t>(rows, 2 * 148)), sgqa::kSelThreads, 0, st>>>(
         scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, list, list_count);
     SGQA_LAUNCH_CHECK("topk_rows_list_kernel");

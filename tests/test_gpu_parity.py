@@ -126,28 +126,45 @@ def test_index_topk_parity(cuda_device, case):
     assert ties <= 2 * len(rows)
 
 
-@pytest.mark.parametrize("case", ["short_rows", "filtered_rows"])
+@pytest.mark.parametrize("case", ["short_rows", "filtered_rows", "dup_short", "dup_long"])
 def test_index_topk_exact_ties(cuda_device, case):
-    """Zero head weights make every score exactly 0: the only valid selection
-    is the k smallest block ids.  short_rows: 600..2903 candidates per row,
-    where rows up to 2048 resolve the tie inside one histogram bin and longer
-    rows overflow the boundary buffer and are redone by the radix kernel.
-    filtered_rows: 16384..16895 candidates, the sampled-threshold path; every
-    zero row keeps all of its candidates, overflows the kept list and is
-    recomputed for the radix kernel.  The other queries keep their weights
-    and are checked against the oracle as usual."""
-    if case == "short_rows":
+    """Exact score ties, which the selection must break toward smaller block ids.
+
+    short_rows / filtered_rows: zero head weights make every score of every
+    third row exactly 0, so the only valid selection is the k smallest ids.
+    short_rows has 600..2903 candidates per row (the shared-memory histogram
+    kernel: a zero row falls in one bin and one sub-bin, overflows the boundary
+    buffer and is redone by the radix kernel); filtered_rows has 16384..16895
+    (the sampled-threshold path: every zero row keeps all of its candidates,
+    overflows the kept list and is recomputed for the radix kernel).
+
+    dup_short / dup_long: the store repeats 211 distinct keys (block r holds
+    the codes of block r mod 211), so every row's scores come in groups of
+    equal values and the k-th position falls inside a group of about n / 211
+    equal scores: the histogram kernel resolves those ties itself (groups up
+    to 64 by ranking, larger ones by the warp radix select).  The selected
+    members of the boundary group must be its smallest ids.  dup_short has
+    600..2903 candidates per row, dup_long 15360..16383."""
+    dup = case.startswith("dup")
+    if case in ("short_rows", "dup_short"):
         wl = dataclasses.replace(WL["prefill8k"], name="ties", seq_len=24576, topk=512)
         q0, nq = 4800, 16384 + 2048  # candidates 600 .. 2903 per query (B = 8)
+    elif case == "dup_long":
+        wl = dataclasses.replace(WL["prefill8k"], name="ties_dup_long", seq_len=131072, topk=512)
+        q0, nq = 122880, 8192  # candidates 15360 .. 16383 per query
     else:
         wl = dataclasses.replace(WL["prefill8k"], name="ties_long", seq_len=139264, topk=512)
         q0, nq = 131072, 4096  # candidates 16384 .. 16895 per query
     cache, _ = Hn.make_inputs(wl, cuda_device)
     qs = I.make_queries(wl, cuda_device, q0, nq)
     zero = torch.zeros(nq, dtype=torch.bool, device=cuda_device)
-    zero[::3] = True
-    qs["idx_w"][zero] = 0.0
+    if not dup:
+        zero[::3] = True
+        qs["idx_w"][zero] = 0.0
     _, codes, keys = Hn.oracle_keys(Hn.to_np(cache["kp"][0]), Hn.to_np(cache["c"][0]), wl.block)
+    if dup:
+        codes = np.ascontiguousarray(codes[np.arange(codes.shape[0]) % 211])
+        keys = O.e4m3_decode(codes)
     store = torch.from_numpy(codes).to(cuda_device)[None].contiguous()
     p = Hn.params_for(wl)
     sel = torch.full((1, nq, wl.groups, wl.topk), -7, dtype=torch.int32, device=cuda_device)
@@ -162,11 +179,18 @@ def test_index_topk_exact_ties(cuda_device, case):
     assert np.all(sel[zero_np] == np.arange(wl.topk, dtype=np.int32))
     iq, iw = Hn.to_np(qs["idx_q"]), Hn.to_np(qs["idx_w"])
     ties = 0
-    rows = [i for i in range(1, nq, 97 if case != "short_rows" else 397) if not zero_np[i]] + [nq - 1]
+    step = 397 if case in ("short_rows", "dup_short") else 97
+    rows = [i for i in range(1, nq, step) if not zero_np[i]] + [nq - 1]
     for i in rows:
         for g in range(wl.groups):
             sc = O.index_scores(iq[i, g], iw[i, g], keys[:(q0 + i) // wl.block])
             ties += Hn.check_selection(sel[i, g], sc, wl.topk)
+            if dup:
+                order = np.lexsort((np.arange(sc.shape[0]), -sc))
+                group = np.flatnonzero(sc == sc[order[wl.topk - 1]])
+                assert group.size > 1
+                chosen = np.intersect1d(sel[i, g], group)
+                assert np.array_equal(chosen, group[:chosen.size]), (i, g)
     assert ties <= 2 * len(rows)
 
 
