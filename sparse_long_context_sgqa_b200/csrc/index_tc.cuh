@@ -562,12 +562,26 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
       int kept[2 * QW];  // filter: this warp's kept entries per query slot (the same in every lane)
 #pragma unroll
       for (int x = 0; x < 2 * QW; ++x) kept[x] = 0;
+      // FP32 outputs: slot x = (h2, qq) of this warp writes row row0 + qs * G,
+      // element c * kIdxCand + m (the sample's tile c, or candidate tile c):
+      // 32-bit offsets from one base (at most 32 * G rows of o.ld apart) and a
+      // bit per slot for the queries the call has
+      int32_t soff[2 * QW];
+      uint32_t vmask = 0;
+#pragma unroll
+      for (int x = 0; x < 2 * QW; ++x) {
+        const int qs = (64 * part + 32 * (x / QW)) / H + x % QW;
+        soff[x] = static_cast<int32_t>(static_cast<int64_t>(qs) * G * o.ld);
+        vmask |= static_cast<uint32_t>(qs < nq_here) << x;
+      }
+      float* const sbase = MODE == kScoreFilter ? nullptr : o.scores + row0 * o.ld + m;
       for (int c = 0; c < n_loop; ++c) {
         const int ab = c & 1;
         if (!tc::mbar_wait(bar(sm.acc_full[ab]), (c >> 1) & 1, abort)) break;
         tc::fence_after();
         const int64_t r = static_cast<int64_t>(tile_of(c)) * kIdxCand + m;  // candidate block id
         const bool tail = static_cast<int64_t>(tile_of(c) + 1) * kIdxCand > ncand_min;
+        float* const tb = MODE == kScoreFilter ? nullptr : sbase + static_cast<int64_t>(c) * kIdxCand;
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           const int col0 = 64 * part + 32 * h2;
@@ -600,12 +614,10 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
             }
             const float acc = __uint_as_float(static_cast<uint32_t>(acc2)) +
                               __uint_as_float(static_cast<uint32_t>(acc2 >> 32));
-            const int64_t row = row0 + static_cast<int64_t>(qs) * G;
-            if (MODE == kScoreRows) {
-              if (qs < nq_here) o.scores[row * o.ld + r] = acc;
-            } else if (MODE == kScoreSample) {
-              if (qs < nq_here) o.scores[row * o.ld + static_cast<int64_t>(c) * kIdxCand + m] = acc;
+            if (MODE != kScoreFilter) {
+              if ((vmask >> (h2 * QW + qq)) & 1u) tb[soff[h2 * QW + qq]] = acc;
             } else {
+              const int64_t row = row0 + static_cast<int64_t>(qs) * G;
               // keep the score if it reaches the row's threshold (rows past the
               // call's queries have threshold +inf); each (row, quadrant) has its
               // own list, filled in ballot order: no shared counters

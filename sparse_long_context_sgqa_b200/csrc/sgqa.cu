@@ -356,6 +356,9 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
     }
     const int64_t grid = static_cast<int64_t>(G) * S * ((nq + Q - 1) / Q);
     const size_t smem = sizeof(sgqa::IndexTcSmem) + 1024;
+    // the score kernel addresses a CTA's output rows with 32-bit offsets
+    if (static_cast<int64_t>(sgqa::kIdxCols) * G * w.rpad >= INT32_MAX)
+      return fail(SGQA_ERR_UNSUPPORTED, "context too long for the index score kernel");
     auto launch_score = [&](int mode, sgqa::ScoreOut o) {
 #define SGQA_SCORE(HH, MM)                                                                                       \
   do {                                                                                                           \
