@@ -472,8 +472,8 @@ namespace sgqa {
 // ---------------------------------------------------------------------------
 // Decode attention (few queries, long context): HBM-bound gather of the
 // selected 8-token blocks.  One CTA takes a contiguous range of one (query,
-// group)'s blocks (split-K); a single producer thread streams each block's K
-// and V (one 5-D TMA box each, 3 KB, 128-byte swizzled) into a 16-slot ring,
+// group)'s blocks (split-K); four lanes of a producer warp stream the blocks'
+// K and V (one 5-D TMA box each, 3 KB, 128-byte swizzled) into a 16-slot ring,
 // and four compute warps consume two blocks (16 tokens) per step with the
 // warp-level MMA formulation (16 heads = the m16 rows).  The splits of a row
 // form one thread-block cluster: each keeps its (max, sum, unnormalised O) in
@@ -483,9 +483,14 @@ namespace sgqa {
 // ---------------------------------------------------------------------------
 constexpr int kDecSlots = 16;
 constexpr int kDecThreads = 160;  // warp 0 producer, warps 1-4 compute
+constexpr int kDecIssuers = 4;    // producer lanes issuing TMA loads side by side
+static_assert(kDecSlots % kDecIssuers == 0 && kDecIssuers <= 32, "issuer groups tile the ring");
+
+constexpr int kDecQPad = kD + 8;  // Q rows of 400 B: ldmatrix rows fall in distinct banks
 
 struct __align__(1024) DecSmem {
   uint8_t kv[kDecSlots][2][3 * 1024];   // [slot][K|V][chunk][8 rows x 128 B]
+  __nv_bfloat16 q[kHg][kDecQPad];       // the row's 16 heads (A operand, read by ldmatrix)
   int32_t rows[2049];                   // first token row of each of this CTA's blocks
   uint64_t full[kDecSlots], empty[kDecSlots];
   int abort;
@@ -536,32 +541,55 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     const int e = b0 + b;
     sm.rows[b] = e < cnt ? ids[e] * 8 : static_cast<int32_t>(cur0);
   }
-  // per-warp attention state (warps 1..4); Q loads overlap the staging
+  // Q into shared memory (its fragments are re-read per k-step: held in
+  // registers they pushed the O accumulators into local memory)
+  {
+    const uint4* q16 = reinterpret_cast<const uint4*>(q + ((seq * nq + i) * G + g) * kHg * kD);
+    for (int x = threadIdx.x; x < kHg * kD / 8; x += kDecThreads)
+      *reinterpret_cast<uint4*>(&sm.q[x / (kD / 8)][(x % (kD / 8)) * 8]) = q16[x];
+  }
+  // per-warp attention state (compute warps)
   WarpAttn st;
-  if (warp >= 1) warp_load_q(st, q + ((seq * nq + i) * G + g) * kHg * kD, lane);
+#pragma unroll
+  for (int j = 0; j < 24; ++j) st.o[j][0] = st.o[j][1] = st.o[j][2] = st.o[j][3] = 0.f;
+  st.m[0] = st.m[1] = -INFINITY;
+  st.l[0] = st.l[1] = 0.f;
   __syncthreads();
 
   if (warp == 0) {
     if (lane == 0) {
       tc::prefetch_tmap(&kmap);
       tc::prefetch_tmap(&vmap);
-      // blocks in pairs: step s uses slots 2s, 2s+1 (mod kDecSlots); an odd tail gets a zero block
-      const int nsteps = (nb + 1) / 2;
-      int issued = 0;
-      for (int b = 0; b < 2 * nsteps; ++b) {
+    }
+    __syncwarp();
+    // blocks in pairs: step s uses slots 2s, 2s+1 (mod kDecSlots); an odd tail
+    // gets a zero block.  kDecIssuers lanes issue consecutive blocks side by
+    // side (one thread's TMA issue rate does not keep an SM's share of HBM busy).
+    const int nblocks = 2 * ((nb + 1) / 2);
+    int mine_end = 0;  // one past the last block this lane issued
+    for (int bg = 0; bg < nblocks; bg += kDecIssuers) {
+      const int b = bg + lane;
+      bool ok = true;
+      if (lane < kDecIssuers && b < nblocks) {
         const int slot = b % kDecSlots;
-        if (b >= kDecSlots && !tc::mbar_wait(bar(sm.empty[slot]), ((b / kDecSlots) - 1) & 1, abort)) break;
-        const int32_t r = b < nb ? sm.rows[b] : -64;  // -64: zero-filled tail block
-        tc::mbar_expect_tx(bar(sm.full[slot]), 2 * 3 * 1024);
-        tc::tma_load_5d(smem_u32(&sm.kv[slot][0][0]), &kmap, 0, r, 0, g, static_cast<int32_t>(seq), bar(sm.full[slot]));
-        tc::tma_load_5d(smem_u32(&sm.kv[slot][1][0]), &vmap, 0, r, 0, g, static_cast<int32_t>(seq), bar(sm.full[slot]));
-        issued = b + 1;
+        if (b >= kDecSlots) ok = tc::mbar_wait(bar(sm.empty[slot]), ((b / kDecSlots) - 1) & 1, abort);
+        if (ok) {
+          const int32_t r = b < nb ? sm.rows[b] : -64;  // -64: zero-filled tail block
+          tc::mbar_expect_tx(bar(sm.full[slot]), 2 * 3 * 1024);
+          tc::tma_load_5d(smem_u32(&sm.kv[slot][0][0]), &kmap, 0, r, 0, g, static_cast<int32_t>(seq), bar(sm.full[slot]));
+          tc::tma_load_5d(smem_u32(&sm.kv[slot][1][0]), &vmap, 0, r, 0, g, static_cast<int32_t>(seq), bar(sm.full[slot]));
+          mine_end = b + 1;
+        }
       }
-      if (*abort) {
-        for (int b = issued > kDecSlots ? issued - kDecSlots : 0; b < issued; ++b) {
-          const uint64_t t0 = globaltimer_ns();
-          while (!tc::mbar_try(bar(sm.full[b % kDecSlots]), (b / kDecSlots) & 1) && globaltimer_ns() - t0 < kWaitLimitNs) {
-          }
+      if (!__all_sync(0xffffffffu, ok)) break;
+    }
+    if (*abort && lane < kDecIssuers) {
+      // this lane's loads still in flight (at most one ring's worth) land
+      // before the CTA exits (waits bounded)
+      for (int b = lane; b < mine_end; b += kDecIssuers) {
+        if (b < mine_end - kDecSlots) continue;
+        const uint64_t t0 = globaltimer_ns();
+        while (!tc::mbar_try(bar(sm.full[b % kDecSlots]), (b / kDecSlots) & 1) && globaltimer_ns() - t0 < kWaitLimitNs) {
         }
       }
     }
@@ -569,6 +597,8 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     const int cw = warp - 1;  // compute warp 0..3
     const int nsteps = (nb + 1) / 2;
     const int mrow = lane & 7, mat = lane >> 3;
+    // ldmatrix row of this lane in the Q tile: matrices (heads 0-7 | 8-15) x (dims +0 | +8)
+    const uint32_t qrow = smem_u32(&sm.q[8 * (mat & 1) + mrow][8 * (mat >> 1)]);
     for (int s = cw; s < nsteps; s += 4) {
       const int ba = 2 * s, bb = 2 * s + 1;
       const int sa = ba % kDecSlots, sb2 = bb % kDecSlots;
@@ -597,8 +627,10 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
       for (int ks = 0; ks < 12; ++ks) {
         uint32_t bf[4];
         ldmatrix_x4(bf, kblk + blk_off(mrow, 2 * ks + (mat & 1)));
-        mma_bf16_16816(sc[0], st.qf[ks], bf[0], bf[1]);
-        mma_bf16_16816(sc[1], st.qf[ks], bf[2], bf[3]);
+        uint32_t qa[4];
+        ldmatrix_x4(qa, qrow + 2u * (16 * ks));
+        mma_bf16_16816(sc[0], qa, bf[0], bf[1]);
+        mma_bf16_16816(sc[1], qa, bf[2], bf[3]);
       }
       float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
