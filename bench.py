@@ -264,7 +264,19 @@ def cuda_arm(args, wl, rank, world, local_rank):
         step()
     e1.record(st)
     torch.cuda.synchronize()
+    # nvidia-smi samples every 200 ms: a timed region shorter than a second is
+    # followed by the same (untimed) steps until a second of load has been
+    # sampled, so that the clock record holds several samples under load
+    clock_window = "timed steps"
+    if sampler is not None and e0.elapsed_time(e1) < 1000.0:
+        clock_window = "timed steps, then the same steps untimed to 1 s"
+        t_end = time.perf_counter() + (1000.0 - e0.elapsed_time(e1)) / 1e3
+        while time.perf_counter() < t_end:
+            step()
+            torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
+    if clocks is not None:
+        clocks["window"] = clock_window
     # kernels launched in the timed region: counted by the library (a graph
     # replay launches the kernels captured once per step)
     gpu_launches = graph_launches * args.steps if graph is not None else Bd.launch_count() - n_launch0
