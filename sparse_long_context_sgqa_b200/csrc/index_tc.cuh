@@ -582,19 +582,27 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
         const int64_t r = static_cast<int64_t>(tile_of(c)) * kIdxCand + m;  // candidate block id
         const bool tail = static_cast<int64_t>(tile_of(c) + 1) * kIdxCand > ncand_min;
         float* const tb = MODE == kScoreFilter ? nullptr : sbase + static_cast<int64_t>(c) * kIdxCand;
+        // the warp's 64 columns in four chunks of 16 (SPC query slots each),
+        // the next chunk's TMEM load in flight while this one is reduced
+        constexpr int SPC = 16 / H;
+        const uint32_t tcol = tmem + ab * kIdxCols + 64 * part + lane_off;
+        uint32_t dbuf[2][16];
+        tc::tmem_ld16(tcol, dbuf[0]);
+        tc::tmem_ld_wait16(dbuf[0]);
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int col0 = 64 * part + 32 * h2;
-          uint32_t d[32];
-          tc::tmem_ld32(tmem + ab * kIdxCols + col0 + lane_off, d);
-          tc::tmem_ld_wait();
-          if (h2 == 1) {
+        for (int j = 0; j < 4; ++j) {
+          if (j < 3) {
+            tc::tmem_ld16(tcol + 16 * (j + 1), dbuf[(j + 1) & 1]);
+          } else {
+            // every column of this accumulator has been read
             tc::fence_before();
             tc::mbar_arrive(bar(sm.acc_empty[ab]));
           }
+          const uint32_t(&d)[16] = dbuf[j & 1];
 #pragma unroll
-          for (int qq = 0; qq < QW; ++qq) {
-            const int qs = col0 / H + qq;
+          for (int u = 0; u < SPC; ++u) {
+            const int x = j * SPC + u;  // slot index among the warp's 2 * QW
+            const int qs = (64 * part) / H + x;
             const float4 w0 = *reinterpret_cast<const float4*>(&sm.w[qs * H]);
             float wv[H];
             wv[0] = w0.x; wv[1] = w0.y; wv[2] = w0.z; wv[3] = w0.w;
@@ -607,15 +615,15 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
             uint64_t acc2 = 0;
 #pragma unroll
             for (int i = 0; i < H; i += 2) {
-              const uint64_t x2 = pack_f32x2(fmaxf(__uint_as_float(d[qq * H + i]), 0.f),
-                                             fmaxf(__uint_as_float(d[qq * H + i + 1]), 0.f));
+              const uint64_t x2 = pack_f32x2(fmaxf(__uint_as_float(d[u * H + i]), 0.f),
+                                             fmaxf(__uint_as_float(d[u * H + i + 1]), 0.f));
               const uint64_t w2 = pack_f32x2(wv[i], wv[i + 1]);
               asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc2) : "l"(x2), "l"(w2));
             }
             const float acc = __uint_as_float(static_cast<uint32_t>(acc2)) +
                               __uint_as_float(static_cast<uint32_t>(acc2 >> 32));
             if (MODE != kScoreFilter) {
-              if ((vmask >> (h2 * QW + qq)) & 1u) tb[soff[h2 * QW + qq]] = acc;
+              if ((vmask >> x) & 1u) tb[soff[x]] = acc;
             } else {
               const int64_t row = row0 + static_cast<int64_t>(qs) * G;
               // keep the score if it reaches the row's threshold (rows past the
@@ -625,13 +633,14 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
               if (tail) pass = pass && r < sm.ncand[qs];
               const uint32_t bal = __ballot_sync(0xffffffffu, pass);
               if (bal) {
-                const int pos = kept[h2 * QW + qq] + __popc(bal & ((1u << lane) - 1u));
+                const int pos = kept[x] + __popc(bal & ((1u << lane) - 1u));
                 if (pass && pos < o.cap)
                   o.staging[(row * 4 + quad) * o.cap + pos] = make_uint2(score_key(acc), static_cast<uint32_t>(r));
-                kept[h2 * QW + qq] += __popc(bal);
+                kept[x] += __popc(bal);
               }
             }
           }
+          if (j < 3) tc::tmem_ld_wait16(dbuf[(j + 1) & 1]);
         }
       }
       if (MODE == kScoreFilter && lane == 0) {
