@@ -194,6 +194,52 @@ def test_index_topk_exact_ties(cuda_device, case):
     assert ties <= 2 * len(rows)
 
 
+@pytest.mark.parametrize("case", ["short", "long"])
+def test_index_topk_outlier_keys(cuda_device, case):
+    """Blocks 2 and 37 of the store hold the E4M3 code of 240 in every
+    dimension, so in many rows one candidate's score lies hundreds of times
+    the typical spread away from the rest.  The linear bins of the histogram
+    top-k then crowd every other candidate into a few bins: the sample's and
+    the exact step's second histogram levels must separate them.  Block 2 is
+    in the sample (float4 0), block 37 is not.  Selections are checked against
+    the oracle (exact up to near-ties).  short: 600..2903 candidates per row,
+    long: 15360..16383."""
+    if case == "short":
+        wl = dataclasses.replace(WL["prefill8k"], name="outlier", seq_len=24576, topk=512)
+        q0, nq, step = 4800, 16384 + 2048, 397
+    else:
+        wl = dataclasses.replace(WL["prefill8k"], name="outlier_long", seq_len=131072, topk=512)
+        q0, nq, step = 122880, 8192, 97
+    cache, _ = Hn.make_inputs(wl, cuda_device)
+    qs = I.make_queries(wl, cuda_device, q0, nq)
+    _, codes, _ = Hn.oracle_keys(Hn.to_np(cache["kp"][0]), Hn.to_np(cache["c"][0]), wl.block)
+    codes = codes.copy()
+    codes[[2, 37]] = 119  # E4M3 code of 240.0
+    keys = O.e4m3_decode(codes)
+    assert keys[2, 0] == 240.0
+    store = torch.from_numpy(codes).to(cuda_device)[None].contiguous()
+    p = Hn.params_for(wl)
+    sel = torch.full((1, nq, wl.groups, wl.topk), -7, dtype=torch.int32, device=cuda_device)
+    cnt = torch.full((1, nq, wl.groups), -7, dtype=torch.int32, device=cuda_device)
+    ws = _bd().alloc_workspace(p, 1, nq, q0 + nq, cuda_device)
+    _bd().sgqa_index_topk(p, 1, q0, nq, qs["idx_q"][None].contiguous(), qs["idx_w"][None].contiguous(),
+                          wl.seq_len, store, sel, cnt, ws)
+    _bd().sgqa_check()
+    sel, cnt = sel[0].cpu().numpy(), cnt[0].cpu().numpy()
+    assert np.all(cnt == wl.topk)
+    iq, iw = Hn.to_np(qs["idx_q"]), Hn.to_np(qs["idx_w"])
+    rows = list(range(1, nq, step)) + [nq - 1]
+    ties, skewed = 0, 0
+    for i in rows:
+        for g in range(wl.groups):
+            sc = O.index_scores(iq[i, g], iw[i, g], keys[:(q0 + i) // wl.block])
+            ties += Hn.check_selection(sel[i, g], sc, wl.topk)
+            rest = np.delete(sc, [2, 37])
+            skewed += sc.max() - np.median(rest) > 100 * (np.sort(rest)[-1] - np.median(rest))
+    assert ties <= 2 * len(rows)
+    assert skewed > 0  # the planted outliers did skew some of the checked rows
+
+
 def _attn_isolated(wl, device, q_pos0, nq, rows, num_seqs=1, groups=None):
     cache, _ = Hn.make_inputs(wl, device, seqs=range(num_seqs))
     qs = [I.make_queries(wl, device, q_pos0, nq, seq=s) for s in range(num_seqs)]
