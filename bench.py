@@ -214,6 +214,29 @@ def union_stats(sel, cnt, wl):
             "inflation": per_unit / max(per_query, 1e-9)}
 
 
+def ranks_from_env(env=None):
+    """(world size, rank, local rank) as torchrun sets them; one process without."""
+    env = os.environ if env is None else env
+    return int(env.get("WORLD_SIZE", "1")), int(env.get("RANK", "0")), int(env.get("LOCAL_RANK", "0"))
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The largest of every rank's value (every rank calls it, in the same order)."""
+    dist = torch.distributed
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(elapsed_ms: float, steps: int, units_per_rank_step: int, world: int):
+    """(ms per step, whole-job units per second): every rank processes its own
+    units each step, the job's time is the slowest rank's."""
+    ms_step = elapsed_ms / steps
+    return ms_step, units_per_rank_step * world / (ms_step / 1e3)
+
+
 def cuda_arm(args, wl, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -280,16 +303,12 @@ def cuda_arm(args, wl, rank, world, local_rank):
     # kernels launched in the timed region: counted by the library (a graph
     # replay launches the kernels captured once per step)
     gpu_launches = graph_launches * args.steps if graph is not None else Bd.launch_count() - n_launch0
-    elapsed = e0.elapsed_time(e1)
+    elapsed = max_over_ranks(e0.elapsed_time(e1), dev)
     if world > 1:
-        t = torch.tensor([elapsed], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed = float(t.item())
         torch.distributed.barrier()
     Bd.sgqa_check()
-    ms_step = elapsed / args.steps
     tokens_per_step = wl.nq * wl.num_seqs
-    value = tokens_per_step * world / (ms_step / 1e3)
+    ms_step, value = job_throughput(elapsed, args.steps, tokens_per_step, world)
 
     # end to end from pinned host memory (prefill workloads)
     e2e = None
@@ -439,9 +458,7 @@ def main():
         L = args.seq_len or wl.seq_len
         qs = L - 1 if wl.n_queries == 1 else wl.q_start
         wl = dataclasses.replace(wl, seq_len=L, num_seqs=args.num_seqs or wl.num_seqs, q_start=qs)
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local_rank = ranks_from_env()
 
     if args.impl == "reference":
         if rank == 0:
