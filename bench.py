@@ -37,6 +37,7 @@ METRIC = {
     "prefill1m": ("sparse_gqa_prefill_tokens_per_s_1m", "tokens/s"),
     "prefill1m_b1": ("sparse_gqa_prefill_tokens_per_s_1m_b1", "tokens/s"),
     "decode": ("sparse_gqa_decode_tokens_per_s", "tokens/s"),
+    "prefill128k_indep": ("sparse_gqa_prefill_tokens_per_s_128k_independent_queries", "tokens/s"),
 }
 
 
@@ -202,7 +203,9 @@ def stage_times(wl, p, model, q, dev):
 
 
 def union_stats(sel, cnt, wl):
-    """Blocks per 8-query unit (the attention kernel's work) against blocks per query."""
+    """Blocks per 8-query unit (the attention kernel's work) against blocks per
+    query, and the mean Jaccard overlap |A & B| / |A | B| of adjacent queries'
+    selections (pairs 2i, 2i+1 of the chunk, every group)."""
     S, n, G, k = sel.shape
     nb = n // 8
     u = sel[:, :nb * 8].reshape(S, nb, 8, G, k).permute(0, 1, 3, 2, 4).reshape(-1, 8 * k)
@@ -210,8 +213,14 @@ def union_stats(sel, cnt, wl):
     distinct = ((u[:, 1:] != u[:, :-1]) & (u[:, 1:] >= 0)).sum(-1) + (u[:, 0] >= 0).to(torch.int64)
     per_unit = float(distinct.double().mean())
     per_query = float(cnt.double().mean())
+    npair = n // 2
+    a, b = sel[:, 0:2 * npair:2], sel[:, 1:2 * npair:2]
+    x = torch.sort(torch.cat([a, b], dim=-1), dim=-1).values
+    inter = ((x[..., 1:] == x[..., :-1]) & (x[..., 1:] >= 0)).sum(-1).double()
+    ca, cb = cnt[:, 0:2 * npair:2].double(), cnt[:, 1:2 * npair:2].double()
+    jac = float((inter / torch.clamp(ca + cb - inter, min=1.0)).mean())
     return {"blocks_per_unit": per_unit, "blocks_per_query": per_query,
-            "inflation": per_unit / max(per_query, 1e-9)}
+            "inflation": per_unit / max(per_query, 1e-9), "jaccard_adjacent": jac}
 
 
 def ranks_from_env(env=None):

@@ -19,6 +19,9 @@ rotary span; block 8, top-512 blocks):
 * ``decode``      16 sequences x 262144 cached tokens, one query each, seed 3.
 * ``prefill1m``   N=1048576 in 8192-query chunks, seed 4 (B=8, top-512);
   ``prefill1m_b1`` the same with B=1, top-2048 tokens.
+* ``prefill128k_indep`` the 128K workload with independent queries (no shared
+  segment direction): a stress case for the 8-query grouping, whose adjacent
+  queries then overlap only through the keys' topics.
 
 Planted structure (all but ``tiny``):
 
@@ -67,6 +70,7 @@ class Workload:
     seed: int = 0
     fp32_inputs: bool = False   # tiny: every input drawn as fp32 N(0,1)
     structured: bool = True     # planted topics / query segments / norms / rotary
+    query_overlap: bool = True  # queries of a 64-token segment share a direction (structured only)
 
     @property
     def nq(self) -> int:
@@ -85,6 +89,7 @@ WORKLOADS = {
     "decode": Workload("decode", 262144, num_seqs=16, q_start=262143, n_queries=1, chunk=1, seed=3),
     "prefill1m": Workload("prefill1m", 1048576, seed=4),
     "prefill1m_b1": Workload("prefill1m_b1", 1048576, block=1, topk=2048, seed=4),
+    "prefill128k_indep": Workload("prefill128k_indep", 131072, seed=2, query_overlap=False),
 }
 
 
@@ -189,12 +194,15 @@ def make_queries(wl: Workload, device, pos0: int, n: int, seq: int = 0):
         iq_ = _randn((m, G, H, Di), device, *tag, "idx")
         iw_ = _randn((m, G, H), device, *tag, "w")
         if wl.structured:
-            u = _randn((s1 - s0, G, H, Di), device, *tag, "u")
-            uw = _randn((s1 - s0, G, H), device, *tag, "uw")
-            rep = torch.arange(m, device=device) // QUERY_SEGMENT
             pos = torch.arange(s0 * QUERY_SEGMENT, s1 * QUERY_SEGMENT, device=device)
-            iq_ = _rotary(_rms(u[rep] + QUERY_NOISE * iq_), pos, 32)
-            iw_ = uw[rep] + QUERY_NOISE * iw_
+            if wl.query_overlap:
+                u = _randn((s1 - s0, G, H, Di), device, *tag, "u")
+                uw = _randn((s1 - s0, G, H), device, *tag, "uw")
+                rep = torch.arange(m, device=device) // QUERY_SEGMENT
+                iq_ = _rotary(_rms(u[rep] + QUERY_NOISE * iq_), pos, 32)
+                iw_ = uw[rep] + QUERY_NOISE * iw_
+            else:
+                iq_ = _rotary(_rms(iq_), pos, 32)
             q_ = _rotary(_rms(q_), pos, 64)
         lo, hi = a - s0 * QUERY_SEGMENT, b - s0 * QUERY_SEGMENT
         q[a - pos0:b - pos0] = q_[lo:hi].to(dt)
