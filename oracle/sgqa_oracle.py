@@ -29,6 +29,8 @@ extraction; the formulas below are the readings of the surrounding prose:
                 group g(h) = floor(h / heads_per_group); ordinary scaled dot
                 products and an exact softmax over the group's selected
                 original tokens.
+* gate       -- same section: each head's result scaled by the sigmoid of its
+                own gate logit (one per token and head).
 
 Inputs are taken exactly as the GPU sees them (BF16 or FP32 values widened to
 float64).  All accumulation is float64.
@@ -46,7 +48,7 @@ import numpy as np
 __all__ = [
     "round_fp32", "round_bf16", "round_e4m3", "e4m3_encode", "e4m3_decode",
     "merge_block", "merge_blocks", "store_codes", "index_scores",
-    "select_topk", "attended_positions", "sparse_attention",
+    "select_topk", "attended_positions", "sparse_attention", "gated_head_output",
     "forward_rows", "token_coverage", "E4M3_MAX",
 ]
 
@@ -238,6 +240,20 @@ def sparse_attention(q_heads, k_rows, v_rows, scale) -> np.ndarray:
     p = np.exp(logits)
     p /= p.sum(axis=1, keepdims=True)
     return p @ v_rows
+
+
+def gated_head_output(head_out, gate_logit) -> np.ndarray:
+    """Head-wise sigmoid gate on the attention output.
+
+    Section "Main attention still reads original K/V": the attention result of
+    a head is sigmoid-gated before the heads are concatenated and projected.
+    Reading (the section gives no shape): one gate logit per (token, head),
+    as the head-wise attention gate of the same vendor's Step 3.5 Flash
+    configuration table ("Every architecture field") states.
+    head_out [..., D], gate_logit [...] -> sigmoid(gate_logit) * head_out.
+    """
+    g = np.asarray(gate_logit, dtype=np.float64)
+    return (1.0 / (1.0 + np.exp(-g)))[..., None] * np.asarray(head_out, dtype=np.float64)
 
 
 # ---------------------------------------------------------------------------

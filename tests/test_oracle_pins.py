@@ -327,3 +327,35 @@ def test_selection_tie_goes_to_smaller_block_id():
     s = O.index_scores(rng.standard_normal((3, 16)), rng.standard_normal(3), keys)
     assert np.all(s == s[0])
     assert list(O.select_topk(s, 4)) == [0, 1, 2, 3]
+
+
+# --------------------------------------------------------------------------
+# Head-wise sigmoid output gate (section "Main attention still reads original K/V")
+# --------------------------------------------------------------------------
+
+def test_gate_closed_forms():
+    """sigmoid(0) = 1/2 exactly; sigmoid(g) + sigmoid(-g) = 1; saturation at
+    large |g| (a wrong sign or a missing gate fails one of these)."""
+    rng = np.random.default_rng(11)
+    out = rng.standard_normal((5, 3, 192))
+    assert np.array_equal(O.gated_head_output(out, np.zeros((5, 3))), 0.5 * out)
+    g = rng.standard_normal((5, 3)) * 3.0
+    np.testing.assert_allclose(O.gated_head_output(out, g) + O.gated_head_output(out, -g), out, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(O.gated_head_output(out, np.full((5, 3), 40.0)), out, rtol=1e-15, atol=0)
+    assert np.abs(O.gated_head_output(out, np.full((5, 3), -40.0))).max() < 1e-16 * np.abs(out).max()
+    # one logit scales its whole head vector, and only that head's
+    g1 = np.zeros((5, 3)); g1[2, 1] = math.log(3.0)   # sigmoid = 3/4
+    got = O.gated_head_output(out, g1)
+    np.testing.assert_allclose(got[2, 1], 0.75 * out[2, 1], rtol=1e-15)
+    mask = np.ones((5, 3), bool); mask[2, 1] = False
+    assert np.array_equal(got[mask], 0.5 * out[mask])
+
+
+def test_gate_on_single_token_attention_is_gated_value_row():
+    """Attention over one token returns that token's V row; the gate scales it."""
+    rng = np.random.default_rng(12)
+    q = rng.standard_normal((16, 192)); k = rng.standard_normal((1, 192)); v = rng.standard_normal((1, 192))
+    att = O.sparse_attention(q, k, v, 192 ** -0.5)
+    g = rng.standard_normal(16)
+    np.testing.assert_allclose(O.gated_head_output(att, g), (1 / (1 + np.exp(-g)))[:, None] * v[0][None, :],
+                               rtol=1e-13, atol=0)
