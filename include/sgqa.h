@@ -139,6 +139,26 @@ sgqa_status sgqa_sparse_attn(const sgqa_params* p, int64_t num_seqs, int64_t q_p
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * sgqa_sparse_attn followed by the head-wise sigmoid output gate, fused into
+ * the attention kernels' final normalisation.  Page section "Main attention
+ * still reads original K/V": each head's result is sigmoid-gated before the
+ * heads are concatenated and projected; one gate logit per (token, head) (the
+ * head-wise gate of the vendor's sibling-model configuration table,
+ * "Every architecture field").
+ *
+ * gate : [S, nq, G*Hg] bf16 gate logits (device, 2-byte aligned), read only;
+ *        out[s, t, h, :] = sigmoid(gate[s, t, h]) * attention[s, t, h, :].
+ *        NULL makes the call identical to sgqa_sparse_attn.
+ * Every other argument, the workspace and the errors as sgqa_sparse_attn;
+ * SGQA_ERR_INVALID_ARGUMENT for a misaligned gate.
+ */
+sgqa_status sgqa_sparse_attn_gated(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                                   const void* q, int64_t cache_cap, int64_t cache_len,
+                                   const void* k_cache, const void* v_cache,
+                                   const int32_t* sel, const int32_t* sel_count, const void* gate,
+                                   void* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * The whole hot path for one call: merge the blocks that this call's tokens
  * complete (blocks [floor(q_pos0/B), floor((q_pos0+nq)/B))), then
  * sgqa_index_topk, then sgqa_sparse_attn.  Arguments as above; the proxy keys,
@@ -154,6 +174,19 @@ sgqa_status sgqa_forward(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0,
                          float* merged_f32, uint8_t* store,
                          int32_t* sel, int32_t* sel_count, void* out,
                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * sgqa_forward with the head-wise sigmoid output gate of
+ * sgqa_sparse_attn_gated (gate: [S, nq, G*Hg] bf16 logits, or NULL).
+ */
+sgqa_status sgqa_forward_gated(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                               const void* q, const void* idx_q, const float* idx_w,
+                               int64_t cache_cap, int64_t cache_len,
+                               const void* proxy_k, const void* comp_logits,
+                               const void* k_cache, const void* v_cache,
+                               float* merged_f32, uint8_t* store,
+                               int32_t* sel, int32_t* sel_count, const void* gate, void* out,
+                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Sparse attention for decode-sized calls without a caller workspace.  The

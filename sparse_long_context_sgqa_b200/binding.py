@@ -25,8 +25,8 @@ STATUS = {0: "SGQA_OK", 1: "SGQA_ERR_INVALID_ARGUMENT", 2: "SGQA_ERR_UNSUPPORTED
           3: "SGQA_ERR_WORKSPACE", 4: "SGQA_ERR_CUDA", 5: "SGQA_ERR_TIMEOUT", 6: "SGQA_ERR_DEVICE"}
 
 EXPORTED = ["sgqa_workspace_size", "sgqa_merge_blocks", "sgqa_index_topk", "sgqa_sparse_attn",
-            "sgqa_forward", "sgqa_sparse_attn_noalloc", "sgqa_check", "sgqa_last_error", "sgqa_version",
-            "sgqa_launch_count"]
+            "sgqa_sparse_attn_gated", "sgqa_forward", "sgqa_forward_gated", "sgqa_sparse_attn_noalloc",
+            "sgqa_check", "sgqa_last_error", "sgqa_version", "sgqa_launch_count"]
 
 
 class SgqaError(RuntimeError):
@@ -66,8 +66,12 @@ _lib.sgqa_merge_blocks.argtypes = [_P, _i64, _i64, _vp, _vp, _i64, _i64, _vp, _v
 _lib.sgqa_index_topk.argtypes = [_P, _i64, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sgqa_sparse_attn.argtypes = [_P, _i64, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp,
                                   _vp, _sz, _vp]
+_lib.sgqa_sparse_attn_gated.argtypes = [_P, _i64, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
+                                        _vp, _sz, _vp]
 _lib.sgqa_forward.argtypes = [_P, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp,
                               _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.sgqa_forward_gated.argtypes = [_P, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp,
+                                    _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sgqa_sparse_attn_noalloc.argtypes = [_P, _i64, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.sgqa_check.argtypes = [_vp]
 _lib.sgqa_last_error.restype = ctypes.c_char_p
@@ -131,6 +135,26 @@ def sgqa_sparse_attn(p: Params, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k
                               _ptr(k_cache), _ptr(v_cache), _ptr(sel), _ptr(sel_count), _ptr(out),
                               _ptr(workspace), workspace.numel() if workspace is not None else 0,
                               _stream(stream)))
+
+
+def sgqa_sparse_attn_gated(p: Params, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k_cache, v_cache, sel,
+                           sel_count, gate, out, workspace, stream=None):
+    """sgqa_sparse_attn with the head-wise sigmoid output gate (gate: [S, nq, G*Hg] bf16 logits)."""
+    _ok(_lib.sgqa_sparse_attn_gated(ctypes.byref(p.c()), num_seqs, q_pos0, nq, _ptr(q), cache_cap, cache_len,
+                                    _ptr(k_cache), _ptr(v_cache), _ptr(sel), _ptr(sel_count), _ptr(gate),
+                                    _ptr(out), _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                                    _stream(stream)))
+
+
+def sgqa_forward_gated(p: Params, num_seqs, q_pos0, nq, q, idx_q, idx_w, cache_cap, cache_len, proxy_k,
+                       comp_logits, k_cache, v_cache, merged_f32, store, sel, sel_count, gate, out, workspace,
+                       stream=None):
+    """sgqa_forward with the head-wise sigmoid output gate (gate: [S, nq, G*Hg] bf16 logits)."""
+    _ok(_lib.sgqa_forward_gated(ctypes.byref(p.c()), num_seqs, q_pos0, nq, _ptr(q), _ptr(idx_q), _ptr(idx_w),
+                                cache_cap, cache_len, _ptr(proxy_k), _ptr(comp_logits), _ptr(k_cache),
+                                _ptr(v_cache), _ptr(merged_f32), _ptr(store), _ptr(sel), _ptr(sel_count),
+                                _ptr(gate), _ptr(out), _ptr(workspace),
+                                workspace.numel() if workspace is not None else 0, _stream(stream)))
 
 
 def sgqa_forward(p: Params, num_seqs, q_pos0, nq, q, idx_q, idx_w, cache_cap, cache_len, proxy_k,

@@ -288,13 +288,14 @@ __device__ __forceinline__ void warp_attend_step(WarpAttn& st, uint32_t ks, uint
 }
 
 // Final normalisation and bf16 store of one warp's 16 x 192 output.
-__device__ __forceinline__ void warp_store_out(WarpAttn& st, __nv_bfloat16* o16, int lane) {
+// g16: the 16 heads' gate logits (nullptr: no gate).
+__device__ __forceinline__ void warp_store_out(WarpAttn& st, __nv_bfloat16* o16, const __nv_bfloat16* g16, int lane) {
   float l0 = st.l[0], l1 = st.l[1];
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  const float i0 = 1.f / l0, i1 = 1.f / l1;
+  const float i0 = gate_factor(g16, lane >> 2) / l0, i1 = gate_factor(g16, (lane >> 2) + 8) / l1;
   __nv_bfloat16* ra = o16 + (lane >> 2) * kD + 2 * (lane & 3);
   __nv_bfloat16* rb = ra + 8 * kD;
 #pragma unroll
@@ -332,8 +333,8 @@ __global__ void __launch_bounds__(kGroupedThreads, 1)
 attn_grouped_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
                     const __nv_bfloat16* __restrict__ vc, const int32_t* __restrict__ plan_ids,
                     const uint8_t* __restrict__ plan_mask, const int32_t* __restrict__ plan_count,
-                    __nv_bfloat16* __restrict__ out, int64_t nq, int G, int k, int64_t q_pos0,
-                    int64_t cache_cap, int64_t cache_len, float scale_log2) {
+                    __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ gate, int64_t nq, int G,
+                    int k, int64_t q_pos0, int64_t cache_cap, int64_t cache_len, float scale_log2) {
   extern __shared__ __align__(16) __nv_bfloat16 smem[];
   __shared__ int64_t s_tok[kGroupedStages][kStepTok];
   constexpr int E = kStepTok / B;  // union entries per step
@@ -412,7 +413,9 @@ attn_grouped_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
     else __syncthreads();  // keep the barrier count uniform with issue()
     cp_async_commit();
   }
-  if (qvalid) warp_store_out(st, out + ((seq * nq + i) * G + g) * kHg * kD, lane);
+  if (qvalid)
+    warp_store_out(st, out + ((seq * nq + i) * G + g) * kHg * kD,
+                   gate == nullptr ? nullptr : gate + ((seq * nq + i) * G + g) * kHg, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -540,7 +543,8 @@ attn_decode_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
 
 // Combine nsplit partials of each (row, head) into the bf16 output.
 __global__ void attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
-                                    __nv_bfloat16* __restrict__ out, int64_t rows, int nsplit) {
+                                    __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ gate,
+                                    int64_t rows, int nsplit) {
   const int64_t rh = blockIdx.x;  // row * 16 + h
   const int64_t row = rh / kHg;
   const int h = static_cast<int>(rh % kHg);
@@ -552,7 +556,7 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o, const floa
     const float* ml = part_ml + ((row * nsplit + s) * kHg + h) * 2;
     ls += exp2f(ml[0] - mu) * ml[1];
   }
-  const float inv = 1.f / ls;
+  const float inv = gate_factor(gate, rh) / ls;  // normalisation and output gate
   for (int d = threadIdx.x; d < kD; d += blockDim.x) {
     float acc = 0.f;
     for (int s = 0; s < nsplit; ++s) {

@@ -61,6 +61,7 @@ struct __align__(1024) AttnTcSmem {
   uint64_t o_final, drain, drain_pv;
   float mchain[128];                       // running reference max after the latest tile, per row
   float lsum[2][128];                      // partial row sums of the two warps of a quadrant
+  float gfac[128];                         // output gate factor per row (1 without a gate)
   uint32_t tmem;
   int abort;
 };
@@ -73,8 +74,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUtensorMap kmap,
                const __grid_constant__ CUtensorMap vmap, const int32_t* __restrict__ plan_ids,
                const uint8_t* __restrict__ plan_mask, const int32_t* __restrict__ plan_count,
-               __nv_bfloat16* __restrict__ out, int64_t nq, int G, int k, int64_t q_pos0,
-               float scale_log2) {
+               __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ gate, int64_t nq, int G,
+               int k, int64_t q_pos0, float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
   AttnTcSmem& sm = *reinterpret_cast<AttnTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                   ~static_cast<uintptr_t>(1023));
@@ -277,6 +278,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     const int64_t cur_lo = 8 * (t / 8);
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const int64_t orow_idx = ((seq * nq + (qvalid ? qi : 0)) * G + g) * kHg + (m & 15);
+    if (half == 0) sm.gfac[m] = gate_factor(gate, orow_idx);  // read by both warps at the end
     // Q row m, dims [96 half, 96 half + 96), into TMEM columns tQ + 48 half ...
     {
       const uint4* src = reinterpret_cast<const uint4*>(q + orow_idx * kD + 96 * half);
@@ -436,7 +438,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     const float ltot = l_adj + sm.lsum[half ^ 1][m];
     if (ok) {
       tc::fence_after();
-      const float inv = 1.f / ltot;
+      const float inv = sm.gfac[m] / ltot;  // softmax normalisation and output gate
       __nv_bfloat16* orow = out + orow_idx * kD;
 #pragma unroll 1
       for (int h = 3 * half; h < 3 * half + 3; ++h) {
@@ -507,8 +509,9 @@ constexpr int kDecMaxSplit = 8;  // splits of a row = one (portable) cluster
 __global__ void __launch_bounds__(kDecThreads, 2)
 attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                        const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ sel,
-                       const int32_t* __restrict__ sel_count, __nv_bfloat16* __restrict__ out, int64_t nq, int G,
-                       int k, int64_t q_pos0, int nsplit, float scale_log2) {
+                       const int32_t* __restrict__ sel_count, __nv_bfloat16* __restrict__ out,
+                       const __nv_bfloat16* __restrict__ gate, int64_t nq, int G, int k, int64_t q_pos0, int nsplit,
+                       float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
   DecSmem& sm = *reinterpret_cast<DecSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
@@ -770,7 +773,7 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
       gf[r * kHg + h] = a;
       ls += a * cluster.map_shared_rank(pl, r)[h];
     }
-    ginv[h] = 1.f / ls;
+    ginv[h] = gate_factor(gate, row * kHg + h) / ls;  // normalisation and output gate
   }
   __syncthreads();
   {

@@ -40,6 +40,12 @@ __device__ __forceinline__ float key_score(uint32_t k) {
   return __uint_as_float(b);
 }
 
+// Head-wise output gate: the sigmoid of a head's BF16 gate logit, 1 without
+// a gate (expf of a large positive argument gives inf, hence exactly 0).
+__device__ __forceinline__ float gate_factor(const __nv_bfloat16* gate, int64_t head_row) {
+  return gate == nullptr ? 1.f : 1.f / (1.f + expf(-__bfloat162float(gate[head_row])));
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

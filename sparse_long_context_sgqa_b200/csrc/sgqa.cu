@@ -234,7 +234,8 @@ sgqa_status encode_bf16(CUtensorMap* m, const void* base, int rank, const cuuint
 
 sgqa_status launch_attn_tc(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q,
                            int64_t cap, int64_t clen, const void* kc, const void* vc, const int32_t* ids,
-                           const uint8_t* msk, const int32_t* cnt, void* out, int64_t units, cudaStream_t st) {
+                           const uint8_t* msk, const int32_t* cnt, void* out, const void* gate, int64_t units,
+                           cudaStream_t st) {
   const int G = p->num_kv_groups;
   const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
   CUtensorMap km, vm;
@@ -255,8 +256,8 @@ sgqa_status launch_attn_tc(const sgqa_params* p, int64_t S, int64_t q0, int64_t 
   auto kern = skip_pairs ? sgqa::attn_tc_kernel<true> : sgqa::attn_tc_kernel<false>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   kern<<<static_cast<unsigned>(units), sgqa::kTcThreads, smem, st>>>(
-      static_cast<const __nv_bfloat16*>(q), km, vm, ids, msk, cnt, static_cast<__nv_bfloat16*>(out), nq, G,
-      p->topk, q0, scale_log2);
+      static_cast<const __nv_bfloat16*>(q), km, vm, ids, msk, cnt, static_cast<__nv_bfloat16*>(out),
+      static_cast<const __nv_bfloat16*>(gate), nq, G, p->topk, q0, scale_log2);
   SGQA_LAUNCH_CHECK("attn_tc_kernel");
   return SGQA_OK;
 }
@@ -483,8 +484,9 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
 template <int B>
 sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q,
                         int64_t cap, int64_t clen, const void* kc, const void* vc, const int32_t* sel,
-                        const int32_t* sel_count, void* out, void* ws, cudaStream_t st) {
+                        const int32_t* sel_count, void* out, const void* gate, void* ws, cudaStream_t st) {
   const int G = p->num_kv_groups, k = p->topk;
+  const __nv_bfloat16* gb = static_cast<const __nv_bfloat16*>(gate);
   const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
   const AttnWs w = attn_ws(p, S, nq);
   const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
@@ -517,8 +519,8 @@ sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, sgqa::attn_decode_tma_kernel, km, vm, qb, sel, sel_count, ob, nq, G, k,
-                                       q0, nsplit, scale_log2);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, sgqa::attn_decode_tma_kernel, km, vm, qb, sel, sel_count, ob, gb, nq, G,
+                                       k, q0, nsplit, scale_log2);
     if (e != cudaSuccess) return cuda_fail(e, "attn_decode_tma_kernel launch");
     SGQA_LAUNCH_CHECK("attn_decode_tma_kernel");
     return SGQA_OK;
@@ -532,7 +534,7 @@ sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq,
     sgqa::attn_decode_kernel<B><<<static_cast<unsigned>(rows * w.nsplit), sgqa::kDecWarps * 32, smem, st>>>(
         qb, kb, vb, sel, sel_count, po, pml, nq, G, k, q0, cap, w.nsplit, scale_log2);
     SGQA_LAUNCH_CHECK("attn_decode_kernel");
-    sgqa::attn_combine_kernel<<<static_cast<unsigned>(rows * 16), 64, 0, st>>>(po, pml, ob, rows, w.nsplit);
+    sgqa::attn_combine_kernel<<<static_cast<unsigned>(rows * 16), 64, 0, st>>>(po, pml, ob, gb, rows, w.nsplit);
     SGQA_LAUNCH_CHECK("attn_combine_kernel");
     return SGQA_OK;
   }
@@ -557,23 +559,23 @@ sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq,
     SGQA_LAUNCH_CHECK("attn_plan_sort_kernel");
   }
   if (B == 8 && use_tc_attention())
-    return launch_attn_tc(p, S, q0, nq, q, cap, clen, kc, vc, ids, msk, cnt, out, units, st);
+    return launch_attn_tc(p, S, q0, nq, q, cap, clen, kc, vc, ids, msk, cnt, out, gate, units, st);
   const size_t smem = sgqa::kGroupedStages * 2 * sgqa::kStageElems * 2;
   cudaFuncSetAttribute(sgqa::attn_grouped_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   sgqa::attn_grouped_kernel<B><<<static_cast<unsigned>(units), sgqa::kGroupedThreads, smem, st>>>(
-      qb, kb, vb, ids, msk, cnt, ob, nq, G, k, q0, cap, clen, scale_log2);
+      qb, kb, vb, ids, msk, cnt, ob, gb, nq, G, k, q0, cap, clen, scale_log2);
   SGQA_LAUNCH_CHECK("attn_grouped_kernel");
   return SGQA_OK;
 }
 
 sgqa_status do_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q,
                     int64_t cap, int64_t clen, const void* kc, const void* vc, const int32_t* sel,
-                    const int32_t* sel_count, void* out, void* ws, cudaStream_t st) {
+                    const int32_t* sel_count, void* out, const void* gate, void* ws, cudaStream_t st) {
   switch (p->block_size) {
-    case 1: return launch_attn<1>(p, S, q0, nq, q, cap, clen, kc, vc, sel, sel_count, out, ws, st);
-    case 2: return launch_attn<2>(p, S, q0, nq, q, cap, clen, kc, vc, sel, sel_count, out, ws, st);
-    case 4: return launch_attn<4>(p, S, q0, nq, q, cap, clen, kc, vc, sel, sel_count, out, ws, st);
-    default: return launch_attn<8>(p, S, q0, nq, q, cap, clen, kc, vc, sel, sel_count, out, ws, st);
+    case 1: return launch_attn<1>(p, S, q0, nq, q, cap, clen, kc, vc, sel, sel_count, out, gate, ws, st);
+    case 2: return launch_attn<2>(p, S, q0, nq, q, cap, clen, kc, vc, sel, sel_count, out, gate, ws, st);
+    case 4: return launch_attn<4>(p, S, q0, nq, q, cap, clen, kc, vc, sel, sel_count, out, gate, ws, st);
+    default: return launch_attn<8>(p, S, q0, nq, q, cap, clen, kc, vc, sel, sel_count, out, gate, ws, st);
   }
 }
 
@@ -680,10 +682,11 @@ sgqa_status sgqa_index_topk(const sgqa_params* p, int64_t num_seqs, int64_t q_po
                   static_cast<cudaStream_t>(stream));
 }
 
-sgqa_status sgqa_sparse_attn(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
-                             const void* q, int64_t cache_cap, int64_t cache_len, const void* k_cache,
-                             const void* v_cache, const int32_t* sel, const int32_t* sel_count,
-                             void* out, void* workspace, size_t workspace_bytes, void* stream) {
+static sgqa_status sparse_attn_impl(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                                    const void* q, int64_t cache_cap, int64_t cache_len, const void* k_cache,
+                                    const void* v_cache, const int32_t* sel, const int32_t* sel_count,
+                                    const void* gate, void* out, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
   g_err.clear();
   sgqa_status s = check_common(p, num_seqs, q_pos0, nq, cache_cap);
   if (s != SGQA_OK) return s;
@@ -696,18 +699,36 @@ sgqa_status sgqa_sparse_attn(const sgqa_params* p, int64_t num_seqs, int64_t q_p
   REQUIRE_PTR(sel, 4);
   REQUIRE_PTR(sel_count, 4);
   REQUIRE_PTR(out, 16);
+  if (gate != nullptr && !aligned(gate, 2)) return fail(SGQA_ERR_INVALID_ARGUMENT, "gate must be 2-byte aligned");
   const AttnWs w = attn_ws(p, num_seqs, nq);
   if ((s = check_ws(workspace, workspace_bytes, w.bytes)) != SGQA_OK) return s;
-  return do_attn(p, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k_cache, v_cache, sel, sel_count, out,
+  return do_attn(p, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k_cache, v_cache, sel, sel_count, out, gate,
                  workspace, static_cast<cudaStream_t>(stream));
 }
 
-sgqa_status sgqa_forward(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
-                         const void* q, const void* idx_q, const float* idx_w, int64_t cache_cap,
-                         int64_t cache_len, const void* proxy_k, const void* comp_logits,
-                         const void* k_cache, const void* v_cache, float* merged_f32, uint8_t* store,
-                         int32_t* sel, int32_t* sel_count, void* out, void* workspace,
-                         size_t workspace_bytes, void* stream) {
+sgqa_status sgqa_sparse_attn(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                             const void* q, int64_t cache_cap, int64_t cache_len, const void* k_cache,
+                             const void* v_cache, const int32_t* sel, const int32_t* sel_count,
+                             void* out, void* workspace, size_t workspace_bytes, void* stream) {
+  return sparse_attn_impl(p, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k_cache, v_cache, sel, sel_count,
+                          nullptr, out, workspace, workspace_bytes, stream);
+}
+
+sgqa_status sgqa_sparse_attn_gated(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                                   const void* q, int64_t cache_cap, int64_t cache_len, const void* k_cache,
+                                   const void* v_cache, const int32_t* sel, const int32_t* sel_count,
+                                   const void* gate, void* out, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  return sparse_attn_impl(p, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k_cache, v_cache, sel, sel_count,
+                          gate, out, workspace, workspace_bytes, stream);
+}
+
+static sgqa_status forward_impl(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                                const void* q, const void* idx_q, const float* idx_w, int64_t cache_cap,
+                                int64_t cache_len, const void* proxy_k, const void* comp_logits,
+                                const void* k_cache, const void* v_cache, float* merged_f32, uint8_t* store,
+                                int32_t* sel, int32_t* sel_count, const void* gate, void* out, void* workspace,
+                                size_t workspace_bytes, void* stream) {
   g_err.clear();
   sgqa_status s = check_common(p, num_seqs, q_pos0, nq, cache_cap);
   if (s != SGQA_OK) return s;
@@ -727,6 +748,7 @@ sgqa_status sgqa_forward(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0,
   REQUIRE_PTR(out, 16);
   if (merged_f32 != nullptr && !aligned(merged_f32, 16))
     return fail(SGQA_ERR_INVALID_ARGUMENT, "merged_f32 must be 16-byte aligned");
+  if (gate != nullptr && !aligned(gate, 2)) return fail(SGQA_ERR_INVALID_ARGUMENT, "gate must be 2-byte aligned");
   size_t need = 0;
   if ((s = sgqa_workspace_size(p, num_seqs, nq, q_pos0 + nq, &need)) != SGQA_OK) return s;
   if ((s = check_ws(workspace, workspace_bytes, need)) != SGQA_OK) return s;
@@ -738,8 +760,28 @@ sgqa_status sgqa_forward(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0,
   if ((s = do_index(p, num_seqs, q_pos0, nq, idx_q, idx_w, cache_cap, store, sel, sel_count, workspace,
                     st)) != SGQA_OK)
     return s;
-  return do_attn(p, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k_cache, v_cache, sel, sel_count, out,
+  return do_attn(p, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k_cache, v_cache, sel, sel_count, out, gate,
                  workspace, st);
+}
+
+sgqa_status sgqa_forward(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                         const void* q, const void* idx_q, const float* idx_w, int64_t cache_cap,
+                         int64_t cache_len, const void* proxy_k, const void* comp_logits,
+                         const void* k_cache, const void* v_cache, float* merged_f32, uint8_t* store,
+                         int32_t* sel, int32_t* sel_count, void* out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  return forward_impl(p, num_seqs, q_pos0, nq, q, idx_q, idx_w, cache_cap, cache_len, proxy_k, comp_logits, k_cache,
+                      v_cache, merged_f32, store, sel, sel_count, nullptr, out, workspace, workspace_bytes, stream);
+}
+
+sgqa_status sgqa_forward_gated(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                               const void* q, const void* idx_q, const float* idx_w, int64_t cache_cap,
+                               int64_t cache_len, const void* proxy_k, const void* comp_logits,
+                               const void* k_cache, const void* v_cache, float* merged_f32, uint8_t* store,
+                               int32_t* sel, int32_t* sel_count, const void* gate, void* out, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  return forward_impl(p, num_seqs, q_pos0, nq, q, idx_q, idx_w, cache_cap, cache_len, proxy_k, comp_logits, k_cache,
+                      v_cache, merged_f32, store, sel, sel_count, gate, out, workspace, workspace_bytes, stream);
 }
 
 sgqa_status sgqa_sparse_attn_noalloc(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
@@ -767,7 +809,7 @@ sgqa_status sgqa_sparse_attn_noalloc(const sgqa_params* p, int64_t num_seqs, int
                 w.bytes, (unsigned)SGQA_NOALLOC_SCRATCH_BYTES);
   void* scratch = nullptr;
   if ((s = noalloc_scratch(&scratch)) != SGQA_OK) return s;
-  return do_attn(p, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k_cache, v_cache, sel, sel_count, out,
+  return do_attn(p, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k_cache, v_cache, sel, sel_count, out, nullptr,
                  scratch, static_cast<cudaStream_t>(stream));
 }
 

@@ -211,6 +211,12 @@ def make_queries(wl: Workload, device, pos0: int, n: int, seq: int = 0):
     return {"q": q, "idx_q": iq, "idx_w": iw}
 
 
+def make_gate(wl: Workload, device, pos0: int, n: int, seq: int = 0) -> torch.Tensor:
+    """Head-wise output-gate logits [n, G*Hg] (bf16) for positions [pos0, pos0+n):
+    2 * N(0,1), so that the gate's sigmoid spans most of (0, 1)."""
+    return (2.0 * _randn((n, wl.n_heads), device, wl.seed, seq, pos0, "gate")).to(torch.bfloat16)
+
+
 def make_selection(wl: Workload, device, pos0: int, n: int, num_seqs: int = 1, seed: int = 0):
     """A random valid selection input (for exercising attention on its own).
 

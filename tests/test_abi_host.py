@@ -95,6 +95,18 @@ def test_null_and_range_checks_before_any_launch(lib, bd):
                              dummy, dummy, ctypes.c_int64(64), dummy, dummy, dummy, ctypes.c_void_p(4096 + 16),
                              ctypes.c_size_t(1 << 30), st)
     assert rc == 3
+    # a misaligned gate is refused before any launch (gated attention and forward)
+    odd = ctypes.c_void_p(4096 + 1)
+    rc = lib.sgqa_sparse_attn_gated(ctypes.byref(p), ctypes.c_int64(1), ctypes.c_int64(0), ctypes.c_int64(64),
+                                    dummy, ctypes.c_int64(64), ctypes.c_int64(64), dummy, dummy, dummy, dummy, odd,
+                                    dummy, dummy, ctypes.c_size_t(1 << 30), st)
+    assert rc == 1
+    assert b"gate" in ctypes.string_at(lib.sgqa_last_error())
+    rc = lib.sgqa_forward_gated(ctypes.byref(p), ctypes.c_int64(1), ctypes.c_int64(0), ctypes.c_int64(64), dummy,
+                                dummy, dummy, ctypes.c_int64(64), ctypes.c_int64(64), dummy, dummy, dummy, dummy, None,
+                                dummy, dummy, dummy, odd, dummy, dummy, ctypes.c_size_t(1 << 30), st)
+    assert rc == 1
+    assert b"gate" in ctypes.string_at(lib.sgqa_last_error())
     # nothing to do is not an error
     rc = lib.sgqa_forward(ctypes.byref(p), ctypes.c_int64(1), ctypes.c_int64(0), ctypes.c_int64(0), None, None,
                           None, ctypes.c_int64(0), ctypes.c_int64(0), None, None, None, None, None, None, None,

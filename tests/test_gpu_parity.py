@@ -240,7 +240,7 @@ def test_index_topk_outlier_keys(cuda_device, case):
     assert skewed > 0  # the planted outliers did skew some of the checked rows
 
 
-def _attn_isolated(wl, device, q_pos0, nq, rows, num_seqs=1, groups=None):
+def _attn_isolated(wl, device, q_pos0, nq, rows, num_seqs=1, groups=None, gated=False):
     cache, _ = Hn.make_inputs(wl, device, seqs=range(num_seqs))
     qs = [I.make_queries(wl, device, q_pos0, nq, seq=s) for s in range(num_seqs)]
     q = torch.stack([x["q"] for x in qs]).to(torch.bfloat16).contiguous()
@@ -249,7 +249,13 @@ def _attn_isolated(wl, device, q_pos0, nq, rows, num_seqs=1, groups=None):
     L = wl.seq_len
     out = torch.zeros((num_seqs, nq, wl.n_heads, wl.head_dim), dtype=torch.bfloat16, device=device)
     ws = _bd().alloc_workspace(p, num_seqs, nq, q_pos0 + nq, device)
-    _bd().sgqa_sparse_attn(p, num_seqs, q_pos0, nq, q, L, L, cache["k"], cache["v"], sel, cnt, out, ws)
+    gate = None
+    if gated:
+        gate = torch.stack([I.make_gate(wl, device, q_pos0, nq, seq=s) for s in range(num_seqs)]).contiguous()
+        _bd().sgqa_sparse_attn_gated(p, num_seqs, q_pos0, nq, q, L, L, cache["k"], cache["v"], sel, cnt, gate, out,
+                                     ws)
+    else:
+        _bd().sgqa_sparse_attn(p, num_seqs, q_pos0, nq, q, L, L, cache["k"], cache["v"], sel, cnt, out, ws)
     _bd().sgqa_check()
     worst = 0.0
     for s in range(num_seqs):
@@ -264,9 +270,52 @@ def _attn_isolated(wl, device, q_pos0, nq, rows, num_seqs=1, groups=None):
                 pos = O.attended_positions(t, ids, wl.block)
                 hs = slice(g * 16, (g + 1) * 16)
                 ref = O.sparse_attention(qn[i, hs], K[pos, g], V[pos, g], Hn.scale_of(wl))
+                if gate is not None:
+                    ref = O.gated_head_output(ref, Hn.to_np(gate[s, i, hs]))
                 worst = max(worst, float(np.abs(on[i, hs] - ref).max()))
     assert worst <= Hn.ATTN_ATOL, worst
     return worst
+
+
+@pytest.mark.parametrize("case", ["prefill8k", "decode_path", "b1", "b2_decode"])
+def test_sparse_attn_gated_parity(cuda_device, case):
+    """The head-wise sigmoid output gate fused into each attention kernel's
+    normalisation: tcgen05 prefill (B = 8), TMA decode with the cluster combine
+    (B = 8), the warp-MMA prefill (B = 1) and the split-K decode with its
+    combine kernel (B = 2)."""
+    if case == "prefill8k":
+        _attn_isolated(WL["prefill8k"], cuda_device, 0, 8192, Hn.sample_rows(WL["prefill8k"], 24), gated=True)
+    elif case == "decode_path":
+        wl = dataclasses.replace(SMALL8, seq_len=20000, name="dec")
+        _attn_isolated(wl, cuda_device, 19990, 10, range(10), num_seqs=3, gated=True)
+    elif case == "b1":
+        wl = dataclasses.replace(SMALL8, block=1, topk=2048)
+        _attn_isolated(wl, cuda_device, 0, 2048, list(range(0, 2048, 97)) + [2047], gated=True)
+    else:
+        wl = dataclasses.replace(SMALL8, seq_len=20000, name="dec2", block=2, topk=100)
+        _attn_isolated(wl, cuda_device, 19990, 10, range(10), num_seqs=2, gated=True)
+
+
+def test_forward_gated_equals_gate_times_forward(cuda_device):
+    """sgqa_forward_gated = sigmoid(gate) * sgqa_forward, head by head (same
+    inputs, one 2048-token prefill chunk)."""
+    wl = SMALL8
+    run = Hn.run_forward(wl, cuda_device)
+    p = Hn.params_for(wl)
+    S, nq, L = 1, wl.nq, wl.seq_len
+    gate = I.make_gate(wl, cuda_device, wl.q_start, nq)[None].contiguous()
+    out = torch.zeros_like(run.out)
+    sel, cnt = torch.empty_like(run.sel), torch.empty_like(run.cnt)
+    store = torch.empty_like(run.store)
+    ws = _bd().alloc_workspace(p, S, nq, wl.q_start + nq, cuda_device)
+    _bd().sgqa_forward_gated(p, S, wl.q_start, nq, run.queries["q"], run.queries["idx_q"], run.queries["idx_w"], L, L,
+                             run.cache["kp"], run.cache["c"], run.cache["k"], run.cache["v"], None, store, sel, cnt,
+                             gate, out, ws)
+    _bd().sgqa_check()
+    assert torch.equal(sel, run.sel) and torch.equal(cnt, run.cnt)
+    sig = torch.sigmoid(gate.float())[..., None]
+    diff = (out.float() - sig * run.out.float()).abs().max().item()
+    assert diff <= Hn.ATTN_ATOL, diff
 
 
 @pytest.mark.parametrize("case", ["tiny", "prefill8k", "unaligned_chunk", "decode_path", "b1", "b2"])
