@@ -1,45 +1,34 @@
-// Indexer score + streaming top-k on the 5th-generation tensor cores (page
-// "Step-5-Preview: Sparse Reads Are Not a Compressed KV Cache", section
-// "Selection is a weighted ReLU score, not attention softmax").
+// Indexer scores on the 5th-generation tensor cores and the top-k kernels of
+// the prefill path (page "Step-5-Preview: Sparse Reads Are Not a Compressed KV
+// Cache", section "Selection is a weighted ReLU score, not attention softmax").
 //
 // The page's standalone code materialises a [G*N, R] FP32 score matrix (its
 // section "A configured million-token window is not a validated million-token
-// launch": 512 GiB at 1M tokens).  Here no score matrix exists: one CTA owns a
-// tile of Q queries of one group (Q * H = 256 (query, head) columns) and
-// sweeps that tile's causal candidate blocks 128 at a time:
+// launch": 512 GiB at 1M tokens).  Here scores exist per 8192-query chunk only,
+// and for long rows not at all: one CTA owns a tile of Q queries of one group
+// (Q * H = 256 (query, head) columns) and sweeps that tile's causal candidate
+// blocks 128 at a time,
 //   D[128 cand x 256 cols] = keys[128 x 64] . q[256 x 64]^T   (4 tcgen05.mma
 //   M128 N256 K16, keys = the E4M3 store widened to BF16, both TMA-fed),
-// double-buffered in TMEM.  Four epilogue warps own one candidate (TMEM lane)
-// per thread and, per query, form I = sum_i w_i * max(0, D[., (q, i)]) in
-// FP32 registers, then keep the candidate only if its order-preserving key
-// beats the query's running threshold; kept (key, id) pairs are appended to a
-// per-(query, group) staging list in global memory (warp-aggregated atomics).
-// When a list nears its capacity (4k entries), a warp radix-selects the k best
-// in place (ties to the smaller id) and raises the threshold to the k-th key.
-// topk_final_kernel then selects exactly k per list and writes them ascending.
+// double-buffered in TMEM, with the ReLU-weighted head sum in the epilogue
+// (index_score_tc_kernel).  The select kernels below take its output.
 #pragma once
 #include "common.cuh"
 #include "tc.cuh"
 
 namespace sgqa {
 
-constexpr int kIdxThreads = 192;
 constexpr int kScoreTcThreads = 576;  // score kernel: producer, MMA, 16 epilogue warps
 constexpr int kIdxStages = 4;
 constexpr int kIdxCand = 128;    // candidates per tile (MMA M)
 constexpr int kIdxCols = 256;    // (query, head) columns per CTA (MMA N)
-constexpr int kCbufEntries = 2048;  // staging entries a warp compacts in shared memory
 
 struct __align__(1024) IndexTcSmem {
   uint8_t b[kIdxCols * 128];               // queries: 256 rows x 64 bf16 (SW128)
   uint8_t a[kIdxStages][kIdxCand * 128];   // candidate keys: 128 rows x 64 bf16 (SW128)
   float w[kIdxCols];                       // head weights, column order
   uint32_t thr[kIdxCols];                  // per-query threshold key (first Q used)
-  int cnt[kIdxCols];                       // per-query staged count
   int ncand[kIdxCols];                     // per-query candidate count floor(t / B)
-  uint32_t hist[4][256];                   // per-warp radix histograms
-  uint32_t wbal[4][64];                    // per TMEM-lane quadrant: take ballot per query this tile
-  uint2 cbuf[4][kCbufEntries];             // per-warp copy of a staging list being compacted
   uint64_t b_full, a_full[kIdxStages], a_empty[kIdxStages], acc_full[2], acc_empty[2], drain;
   uint32_t tmem;
   int abort;
@@ -167,250 +156,13 @@ __device__ __noinline__ void warp_select(const uint2* buf, int n, int k, uint32_
   __syncwarp();
 }
 
-// Warp copy of n entries, eight loads in flight per lane.
-__device__ __forceinline__ void copy_list(uint2* dst, const uint2* src, int n) {
-  const int lane = threadIdx.x & 31;
-  int i = lane;
-  for (; i + 7 * 32 < n; i += 8 * 32) {
-    uint2 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = src[i + u * 32];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) dst[i + u * 32] = v[u];
-  }
-  for (; i < n; i += 32) dst[i] = src[i];
-  __syncwarp();
-}
-
 __device__ __forceinline__ bool kept(uint2 e, uint32_t theta, uint32_t id_cut) {
   return e.x > theta || (e.x == theta && e.y <= id_cut);
 }
 
-template <int H>
-__global__ void __launch_bounds__(kIdxThreads, 1)
-index_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_constant__ CUtensorMap qmap,
-                const float* __restrict__ idx_w, uint2* __restrict__ staging, int32_t* __restrict__ staged,
-                int64_t nq, int G, int64_t q_pos0, int B, int64_t rpad, int k, int cap) {
-  constexpr int Q = kIdxCols / H;  // queries per CTA
-  extern __shared__ uint8_t smem_raw[];
-  IndexTcSmem& sm = *reinterpret_cast<IndexTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                    ~static_cast<uintptr_t>(1023));
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // grid: x = group-major (g, seq, query tile) so co-resident CTAs share keys
-  const int64_t ntiles_q = (nq + Q - 1) / Q;
-  const int64_t per_group = static_cast<int64_t>(gridDim.x) / G;
-  const int g = static_cast<int>(blockIdx.x / per_group);
-  const int64_t rest = blockIdx.x % per_group;
-  const int64_t seq = rest / ntiles_q;
-  // heavier (later) query tiles first
-  const int64_t qt = ntiles_q - 1 - rest % ntiles_q;
-  const int64_t q0 = qt * Q;
-  const int nq_here = static_cast<int>(nq - q0 < Q ? nq - q0 : Q);
-  const int64_t t_last = q_pos0 + q0 + nq_here - 1;
-  const int64_t ncand_max = t_last / B;
-  const int n_tiles = static_cast<int>((ncand_max + kIdxCand - 1) / kIdxCand);
-  volatile int* abort = &sm.abort;
-  auto bar = [](uint64_t& b) { return smem_u32(&b); };
-
-  if (threadIdx.x == 0) {
-    sm.abort = 0;
-    tc::mbar_init(bar(sm.b_full), 1);
-    for (int s = 0; s < kIdxStages; ++s) {
-      tc::mbar_init(bar(sm.a_full[s]), 1);
-      tc::mbar_init(bar(sm.a_empty[s]), 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(bar(sm.acc_full[b]), 1);
-      tc::mbar_init(bar(sm.acc_empty[b]), 128);
-    }
-    tc::mbar_init(bar(sm.drain), 1);
-    tc::mbar_fence_init();
-  }
-  for (int c = threadIdx.x; c < kIdxCols; c += kIdxThreads) {
-    const int qs = c / H;
-    const int64_t qi = q0 + qs;
-    sm.w[c] = qs < nq_here ? idx_w[((seq * nq + qi) * G + g) * H + (c % H)] : 0.f;
-    sm.thr[c] = 0u;
-    sm.cnt[c] = 0;
-    // indexed by query slot (c < Q), not by column
-    sm.ncand[c] = c < nq_here ? static_cast<int>((q_pos0 + q0 + c) / B) : 0;
-  }
-  if (warp == 1) tc::tmem_alloc(smem_u32(&sm.tmem), 512);
-  __syncthreads();
-  tc::fence_after();
-  const uint32_t tmem = sm.tmem;
-
-  if (n_tiles > 0) {
-    if (warp == 0) {
-      if (lane == 0) {
-        tc::prefetch_tmap(&keymap);
-        tc::prefetch_tmap(&qmap);
-        tc::mbar_expect_tx(bar(sm.b_full), kIdxCols * 128);
-        tc::tma_load_4d(smem_u32(&sm.b[0]), &qmap, 0, 0, g, static_cast<int32_t>(seq * nq + q0), bar(sm.b_full));
-        int issued = 0;
-        for (int c = 0; c < n_tiles; ++c) {
-          const int s = c % kIdxStages;
-          if (c >= kIdxStages && !tc::mbar_wait(bar(sm.a_empty[s]), ((c / kIdxStages) - 1) & 1, abort)) break;
-          tc::mbar_expect_tx(bar(sm.a_full[s]), kIdxCand * 128);
-          tc::tma_load_2d(smem_u32(&sm.a[s][0]), &keymap, 0, static_cast<int32_t>(seq * rpad + c * kIdxCand),
-                          bar(sm.a_full[s]));
-          issued = c + 1;
-        }
-        if (*abort) {
-          const uint64_t t0 = globaltimer_ns();
-          while (!tc::mbar_try(bar(sm.b_full), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-          }
-          for (int c = issued > kIdxStages ? issued - kIdxStages : 0; c < issued; ++c) {
-            const uint64_t t1 = globaltimer_ns();
-            while (!tc::mbar_try(bar(sm.a_full[c % kIdxStages]), (c / kIdxStages) & 1) &&
-                   globaltimer_ns() - t1 < kWaitLimitNs) {
-            }
-          }
-        }
-      }
-    } else if (warp == 1) {
-      if (lane == 0) {
-        const uint32_t idesc = tc::idesc_bf16(kIdxCand, kIdxCols, false);
-        bool ok = tc::mbar_wait(bar(sm.b_full), 0, abort);
-        for (int c = 0; ok && c < n_tiles; ++c) {
-          const int s = c % kIdxStages, ab = c & 1;
-          if (!tc::mbar_wait(bar(sm.a_full[s]), (c / kIdxStages) & 1, abort)) { ok = false; break; }
-          if (c >= 2 && !tc::mbar_wait(bar(sm.acc_empty[ab]), ((c >> 1) - 1) & 1, abort)) { ok = false; break; }
-          tc::fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t a = tc::sdesc_sw128(smem_u32(&sm.a[s][0]) + kk * 32, 16, 1024);
-            const uint64_t b = tc::sdesc_sw128(smem_u32(&sm.b[0]) + kk * 32, 16, 1024);
-            tc::mma_f16(tmem + ab * kIdxCols, a, b, idesc, kk > 0 ? 1u : 0u);
-          }
-          tc::mma_commit(bar(sm.a_empty[s]));
-          tc::mma_commit(bar(sm.acc_full[ab]));
-        }
-        if (!ok) {
-          tc::mma_commit(bar(sm.drain));
-          const uint64_t t0 = globaltimer_ns();
-          while (!tc::mbar_try(bar(sm.drain), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-          }
-        }
-      }
-    } else {
-      // ---------------------------------------------------------- epilogue
-      const int quad = warp & 3;
-      const int m = quad * 32 + lane;  // candidate within the tile
-      const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-      const int ew = warp - 2;          // owns queries qs % 4 == ew (count update, compaction)
-      for (int c = 0; c < n_tiles; ++c) {
-        const int ab = c & 1;
-        // a failed wait skips the work but keeps the epilogue warps' barriers in step
-        const bool ok = tc::mbar_wait(bar(sm.acc_full[ab]), (c >> 1) & 1, abort);
-        tc::fence_after();
-        const int r = c * kIdxCand + m;
-        // phase 1: scores, keys and take-ballots of every query for this candidate
-        uint32_t keys[Q];
-#pragma unroll
-        for (int ch2 = 0; ch2 < kIdxCols / 64; ++ch2) {
-          uint32_t d2[64];
-          if (ok) {
-            tc::tmem_ld32(tmem + ab * kIdxCols + 64 * ch2 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&d2[0]));
-            tc::tmem_ld32(tmem + ab * kIdxCols + 64 * ch2 + 32 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&d2[32]));
-            tc::tmem_ld_wait();
-          }
-          if (ch2 == kIdxCols / 64 - 1 && ok) {
-            tc::fence_before();
-            tc::mbar_arrive(bar(sm.acc_empty[ab]));
-          }
-#pragma unroll
-          for (int qq = 0; qq < 64 / H; ++qq) {
-            const int qs = ch2 * (64 / H) + qq;
-            const float4 w0 = *reinterpret_cast<const float4*>(&sm.w[qs * H]);
-            float wv[H];
-            wv[0] = w0.x; wv[1] = w0.y; wv[2] = w0.z; wv[3] = w0.w;
-            if constexpr (H == 8) {
-              const float4 w1 = *reinterpret_cast<const float4*>(&sm.w[qs * H + 4]);
-              wv[4] = w1.x; wv[5] = w1.y; wv[6] = w1.z; wv[7] = w1.w;
-            }
-            float acc = 0.f;
-#pragma unroll
-            for (int i = 0; i < H; ++i) acc = fmaf(wv[i], fmaxf(__uint_as_float(d2[qq * H + i]), 0.f), acc);
-            keys[qs] = score_key(acc);
-            const bool take = ok && r < sm.ncand[qs] && keys[qs] > sm.thr[qs];
-            const uint32_t bal = __ballot_sync(0xffffffffu, take);
-            if (lane == 0) sm.wbal[quad][qs] = bal;
-          }
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        // phase 2: append in candidate order (quadrant 0..3, then lane) so every
-        // staging list stays sorted by block id
-#pragma unroll
-        for (int qs = 0; qs < Q; ++qs) {
-          const uint32_t bal = sm.wbal[quad][qs];
-          if (bal == 0u) continue;
-          int base = sm.cnt[qs];
-          for (int qd = 0; qd < quad; ++qd) base += __popc(sm.wbal[qd][qs]);
-          if ((bal >> lane) & 1u) {
-            const int pos = base + __popc(bal & ((1u << lane) - 1u));
-            staging[(((seq * nq + q0 + qs) * G + g) * static_cast<int64_t>(cap)) + pos] =
-                make_uint2(keys[qs], static_cast<uint32_t>(r));
-          }
-        }
-        __threadfence_block();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        // count update and, where the list could overflow next tile, compaction
-        for (int qs = ew; qs < nq_here; qs += 4) {
-          const int n = sm.cnt[qs] + __popc(sm.wbal[0][qs]) + __popc(sm.wbal[1][qs]) + __popc(sm.wbal[2][qs]) +
-                        __popc(sm.wbal[3][qs]);
-          __syncwarp();
-          if (n > cap - kIdxCand) {
-            uint2* st = staging + ((seq * nq + q0 + qs) * G + g) * static_cast<int64_t>(cap);
-            const uint2* src = st;
-            if (n <= kCbufEntries) {
-              copy_list(sm.cbuf[ew], st, n);
-              src = sm.cbuf[ew];
-            }
-            uint32_t theta, id_cut;
-            warp_select(src, n, k, sm.hist[ew], theta, id_cut);
-            int out = 0;
-            for (int base = 0; base < n; base += 32) {
-              const int i = base + lane;
-              const uint2 e = i < n ? src[i] : make_uint2(0u, 0u);
-              const bool keep = i < n && kept(e, theta, id_cut);
-              const uint32_t bal = __ballot_sync(0xffffffffu, keep);
-              __syncwarp();
-              if (keep) st[out + __popc(bal & ((1u << lane) - 1u))] = e;
-              out += __popc(bal);
-              __syncwarp();
-            }
-            if (lane == 0) {
-              sm.thr[qs] = theta;
-              sm.cnt[qs] = k;
-            }
-          } else if (lane == 0) {
-            sm.cnt[qs] = n;
-          }
-          __syncwarp();
-        }
-        __threadfence_block();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-      }
-      if (ew == 0)
-        for (int qs = lane; qs < nq_here; qs += 32) staged[(seq * nq + q0 + qs) * G + g] = sm.cnt[qs];
-    }
-  } else if (warp >= 2) {
-    const int ew = warp - 2;
-    if (ew == 0)
-      for (int qs = lane; qs < nq_here; qs += 32) staged[(seq * nq + q0 + qs) * G + g] = 0;
-  }
-  tc::fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc::fence_after();
-    tc::tmem_dealloc(tmem, 512);
-  }
-}
-
-// Indexer scores I[t, g, r] on the tensor cores: the same TMA/tcgen05 pipeline
-// as index_tc_kernel (one CTA = 256 (query, head) columns of one group, all
-// candidates in tiles of 128), with one of three epilogues:
+// Indexer scores I[t, g, r] on the tensor cores (one CTA = 256 (query, head)
+// columns of one group, all candidates in tiles of 128), with one of three
+// epilogues:
 //   kScoreRows    every score as FP32 rows [row, rpad] (one 128-byte store per
 //                 warp and query); a top-k kernel then selects from the rows;
 //   kScoreSample  only every kSampleStride-th candidate tile, compacted into
@@ -477,7 +229,6 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
   if (MODE == kScoreFilter) {
     for (int qs = threadIdx.x; qs < Q; qs += kScoreTcThreads) {
       const bool real = qs < nq_here;
-      sm.cnt[qs] = 0;
       sm.thr[qs] = __float_as_uint(real ? o.thr[(seq * nq + q0 + qs) * G + g] : INFINITY);
       sm.ncand[qs] = real ? static_cast<int>((q_pos0 + q0 + qs) / B) : 0;
     }
@@ -818,58 +569,6 @@ topk_rows2_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, in
     if (pos != k) report(kDevBounds);
   }
 }
-
-// Exact top-k of each staging list.  A list is sorted by block id and the
-// selection is a stable filter, so the output comes out ascending.  One warp
-// per (query, group) row.
-constexpr int kFinalWarps = 4;
-
-__global__ void __launch_bounds__(kFinalWarps * 32)
-topk_final_kernel(const uint2* __restrict__ staging, const int32_t* __restrict__ staged, int64_t rows,
-                  int64_t nq, int G, int64_t q_pos0, int B, int k, int cap, int buf_entries,
-                  int32_t* __restrict__ sel, int32_t* __restrict__ sel_count) {
-  extern __shared__ uint2 fbuf[];  // [kFinalWarps][buf_entries]
-  __shared__ uint32_t hist[kFinalWarps][256];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * kFinalWarps + warp;  // (seq * nq + i) * G + g
-  if (row >= rows) return;
-  const int64_t i = (row / G) % nq;
-  const int64_t ncand = (q_pos0 + i) / B;
-  const int want = static_cast<int>(ncand < k ? ncand : k);
-  const int n = min(max(staged[row], 0), cap);
-  const uint2* st = staging + row * static_cast<int64_t>(cap);
-  int32_t* out = sel + row * k;
-  int have;
-  if (n <= k) {
-    for (int j = lane; j < k; j += 32) out[j] = j < n ? static_cast<int32_t>(st[j].y) : -1;
-    have = n;
-  } else {
-    const uint2* src = st;
-    if (n <= buf_entries) {
-      uint2* b = fbuf + static_cast<int64_t>(warp) * buf_entries;
-      copy_list(b, st, n);
-      src = b;
-    }
-    uint32_t theta, id_cut;
-    warp_select(src, n, k, hist[warp], theta, id_cut);
-    int o = 0;
-    for (int base = 0; base < n; base += 32) {
-      const int j = base + lane;
-      const uint2 e = j < n ? src[j] : make_uint2(0u, 0u);
-      const bool keep = j < n && kept(e, theta, id_cut);
-      const uint32_t bal = __ballot_sync(0xffffffffu, keep);
-      const int pos = o + __popc(bal & ((1u << lane) - 1u));
-      if (keep && pos < k) out[pos] = static_cast<int32_t>(e.y);
-      o += __popc(bal);
-    }
-    have = o < k ? o : k;
-  }
-  if (lane == 0) {
-    sel_count[row] = have;
-    if (have != want) report(kDevBounds);
-  }
-}
-
 
 // ---------------------------------------------------------------------------
 // Top-k for rows of 2048 .. kHistMaxCand candidates (every prefill row up to a

@@ -88,23 +88,11 @@ int decode_splits(int64_t rows) {
   return static_cast<int>(std::min<int64_t>(std::max<int64_t>(s, 1), 32));
 }
 
-// Prefill attention path for B = 8: tcgen05 kernel unless SGQA_ATTN_PATH=mma.
-bool use_tc_attention() {
-  const char* e = getenv("SGQA_ATTN_PATH");
-  return !(e != nullptr && strcmp(e, "mma") == 0);
-}
 
 int plan_pow2(int k) {
   int p = 1;
   while (p < 8 * k) p <<= 1;
   return std::max(p, 2);
-}
-
-// Staging capacity per (query, group) list of the streaming top-k: room for k
-// kept entries plus at least two candidate tiles of appends.
-int staging_cap(int k) {
-  const int64_t c = std::max<int64_t>(4 * static_cast<int64_t>(k), k + 2 * sgqa::kIdxCand);
-  return static_cast<int>(round_up(c, 32));
 }
 
 // Index workspace: widened keys, then one region that holds, one after the
@@ -113,7 +101,6 @@ int staging_cap(int k) {
 // per-row arrays.
 struct IndexWs {
   int64_t rpad, nsamp;
-  int cap;
   size_t keys_off, scores_off, sample_off, staging_off, flags_off, staged_off, thr_off, list_off, bytes;
 };
 IndexWs index_ws(const sgqa_params* p, int64_t S, int64_t nq, int64_t max_ctx) {
@@ -121,11 +108,10 @@ IndexWs index_ws(const sgqa_params* p, int64_t S, int64_t nq, int64_t max_ctx) {
   const int64_t rneed = std::max<int64_t>((max_ctx - 1) / p->block_size, 1);
   w.rpad = round_up(rneed, 128);
   w.nsamp = round_up(w.rpad, sgqa::kIdxCand * sgqa::kSampleStride) / sgqa::kSampleStride;
-  w.cap = staging_cap(p->topk);
   w.keys_off = 0;
   const size_t keys = align256(static_cast<size_t>(S * w.rpad * 64) * 2);
   const size_t rows = static_cast<size_t>(S * nq * p->num_kv_groups);
-  const size_t big = align256(std::max({rows * static_cast<size_t>(w.rpad) * 4, rows * static_cast<size_t>(w.cap) * 8,
+  const size_t big = align256(std::max({rows * static_cast<size_t>(w.rpad) * 4,
                                         rows * static_cast<size_t>(sgqa::kFilterCap) * 8,
                                         rows * static_cast<size_t>(w.nsamp) * 4}));
   w.scores_off = w.sample_off = w.staging_off = keys;
@@ -262,18 +248,12 @@ sgqa_status launch_attn_tc(const sgqa_params* p, int64_t S, int64_t q0, int64_t 
   return SGQA_OK;
 }
 
-// Index path for many queries: tcgen05 score rows + two-pass top-k by default;
-// SGQA_INDEX_PATH=stream selects the fused streaming top-k kernel instead.
-// Rows longer than the register-resident top-k takes (16384 candidates) use
-// the filtered path; shorter rows are cheaper to materialise and select
-// (measured at 128K and 1M contexts).  The kept lists are sized for k <= 512
-// (about 2k entries expected per row, 8k room).
+// Index path for many queries: tcgen05 score rows and a top-k kernel over
+// them.  Rows longer than the histogram top-k takes (16384 candidates) use the
+// filtered path; shorter rows are cheaper to materialise and select (measured
+// at 128K and 1M contexts).  The kept lists are sized for k <= 512 (about 1k
+// entries expected per row, 4k room).
 constexpr int64_t kFilterMinCand = 16385;
-
-bool use_stream_index() {
-  const char* e = getenv("SGQA_INDEX_PATH");
-  return e != nullptr && strcmp(e, "stream") == 0;
-}
 
 sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* idx_q,
                      const float* idx_w, int64_t cap, const uint8_t* store, int32_t* sel,
@@ -289,49 +269,6 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
     SGQA_LAUNCH_CHECK("widen_store_kernel");
   }
   const __nv_bfloat16* iq = static_cast<const __nv_bfloat16*>(idx_q);
-  if (nq > kDecodeMaxNq && use_stream_index()) {
-    uint2* staging = ws_at<uint2>(ws, w.staging_off);
-    int32_t* staged = ws_at<int32_t>(ws, w.staged_off);
-    const int Q = sgqa::kIdxCols / H;
-    sgqa_status s;
-    CUtensorMap km, qm;
-    {
-      cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(S * w.rpad)};
-      cuuint64_t strides[1] = {128};
-      cuuint32_t box[2] = {64, static_cast<cuuint32_t>(sgqa::kIdxCand)};
-      if ((s = encode_bf16(&km, keys, 2, dims, strides, box, "indexer keys")) != SGQA_OK) return s;
-    }
-    {
-      cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(G),
-                            static_cast<cuuint64_t>(S * nq)};
-      cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(H) * 128, static_cast<cuuint64_t>(G) * H * 128};
-      cuuint32_t box[4] = {64, static_cast<cuuint32_t>(H), 1, static_cast<cuuint32_t>(Q)};
-      if ((s = encode_bf16(&qm, iq, 4, dims, strides, box, "idx_q")) != SGQA_OK) return s;
-    }
-    const int64_t ntq = (nq + Q - 1) / Q;
-    const int64_t grid = static_cast<int64_t>(G) * S * ntq;
-    static_assert(sizeof(sgqa::IndexTcSmem) + 1024 <= 232448, "index tile exceeds shared memory");
-    const size_t smem = sizeof(sgqa::IndexTcSmem) + 1024;
-    if (H == 8) {
-      cudaFuncSetAttribute(sgqa::index_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      sgqa::index_tc_kernel<8><<<static_cast<unsigned>(grid), sgqa::kIdxThreads, smem, st>>>(
-          km, qm, idx_w, staging, staged, nq, G, q0, B, w.rpad, p->topk, w.cap);
-    } else {
-      cudaFuncSetAttribute(sgqa::index_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      sgqa::index_tc_kernel<4><<<static_cast<unsigned>(grid), sgqa::kIdxThreads, smem, st>>>(
-          km, qm, idx_w, staging, staged, nq, G, q0, B, w.rpad, p->topk, w.cap);
-    }
-    SGQA_LAUNCH_CHECK("index_tc_kernel");
-    const int buf_entries = std::min(w.cap, 2048);
-    const size_t fsmem = static_cast<size_t>(sgqa::kFinalWarps) * buf_entries * 8;
-    cudaFuncSetAttribute(sgqa::topk_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem);
-    const int64_t rows = S * nq * G;
-    sgqa::topk_final_kernel<<<static_cast<unsigned>((rows + sgqa::kFinalWarps - 1) / sgqa::kFinalWarps),
-                              sgqa::kFinalWarps * 32, fsmem, st>>>(staging, staged, rows, nq, G, q0, B, p->topk,
-                                                                   w.cap, buf_entries, sel, sel_count);
-    SGQA_LAUNCH_CHECK("topk_final_kernel");
-    return SGQA_OK;
-  }
   float* scores = ws_at<float>(ws, w.scores_off);
   int32_t* flags = ws_at<int32_t>(ws, w.flags_off);
   // rows a select kernel could not settle, for the radix kernel (count after the list)
@@ -558,14 +495,16 @@ sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq,
         sel, sel_count, nq, G, k, pow2, ids, msk, cnt);
     SGQA_LAUNCH_CHECK("attn_plan_sort_kernel");
   }
-  if (B == 8 && use_tc_attention())
+  if constexpr (B == 8) {
     return launch_attn_tc(p, S, q0, nq, q, cap, clen, kc, vc, ids, msk, cnt, out, gate, units, st);
-  const size_t smem = sgqa::kGroupedStages * 2 * sgqa::kStageElems * 2;
-  cudaFuncSetAttribute(sgqa::attn_grouped_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  sgqa::attn_grouped_kernel<B><<<static_cast<unsigned>(units), sgqa::kGroupedThreads, smem, st>>>(
-      qb, kb, vb, ids, msk, cnt, ob, gb, nq, G, k, q0, cap, clen, scale_log2);
-  SGQA_LAUNCH_CHECK("attn_grouped_kernel");
-  return SGQA_OK;
+  } else {
+    const size_t smem = sgqa::kGroupedStages * 2 * sgqa::kStageElems * 2;
+    cudaFuncSetAttribute(sgqa::attn_grouped_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    sgqa::attn_grouped_kernel<B><<<static_cast<unsigned>(units), sgqa::kGroupedThreads, smem, st>>>(
+        qb, kb, vb, ids, msk, cnt, ob, gb, nq, G, k, q0, cap, clen, scale_log2);
+    SGQA_LAUNCH_CHECK("attn_grouped_kernel");
+    return SGQA_OK;
+  }
 }
 
 sgqa_status do_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q,
