@@ -39,14 +39,17 @@ constexpr int kPlanThreads = 512;
 // The candidate ids of a unit are < floor(t_last / B); a bitmap over that range
 // (one bit per block, in shared memory) turns the union into set-bit order:
 // set bits, prefix-popcount the words, then every (query, id) finds its union
-// position from the prefix and ORs its query bit into that entry's mask.
+// position from the prefix and ORs its query bit into that entry's mask, in
+// shared memory; the masks go out with 8-byte stores.
 __global__ void __launch_bounds__(kPlanThreads)
 attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ sel_count,
                  int64_t nq, int G, int k, int nwords, int32_t* __restrict__ plan_ids,
                  uint8_t* __restrict__ plan_mask, int32_t* __restrict__ plan_count) {
-  extern __shared__ uint32_t sm_words[];      // [nwords] bitmap, then [nwords] prefix
+  // [nwords] bitmap, [nwords] prefix, then the union's masks (8k bytes)
+  extern __shared__ __align__(16) uint32_t sm_words[];
   uint32_t* bm = sm_words;
   uint32_t* pre = sm_words + nwords;
+  uint32_t* msk = sm_words + 2 * nwords;  // 8-byte aligned
   __shared__ int warp_sums[kPlanThreads / 32];
   __shared__ int s_total;
   const int64_t nqb = (nq + 7) / 8;
@@ -56,6 +59,7 @@ attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ se
   const int64_t seq = unit / (G * nqb);
   const int tid = threadIdx.x;
   for (int w = tid; w < nwords; w += kPlanThreads) bm[w] = 0;
+  for (int w = tid; w < 2 * k; w += kPlanThreads) msk[w] = 0;  // 8k bytes
   __syncthreads();
   const int nq_here = static_cast<int>(nq - qb * 8 < 8 ? nq - qb * 8 : 8);
   const int64_t row0 = (seq * nq + qb * 8) * G + g;
@@ -97,13 +101,11 @@ attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ se
       const int b = __ffs(bits) - 1;
       bits &= bits - 1;
       plan_ids[obase + pos] = w * 32 + b;
-      plan_mask[obase + pos] = 0;
       ++pos;
     }
     run = pos;
   }
   __syncthreads();
-  uint32_t* mask32 = reinterpret_cast<uint32_t*>(plan_mask + obase);  // 8k-byte aligned per unit
   for (int q = 0; q < nq_here; ++q) {
     const int64_t row = row0 + static_cast<int64_t>(q) * G;
     const int cnt = min(max(sel_count[row], 0), k);
@@ -111,9 +113,15 @@ attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ se
       const int id = sel[row * k + j];
       if (id < 0 || id >= nbits) continue;
       const int pos = pre[id >> 5] + __popc(bm[id >> 5] & ((1u << (id & 31)) - 1u));
-      atomicOr(&mask32[pos >> 2], (1u << q) << (8 * (pos & 3)));
+      atomicOr(&msk[pos >> 2], (1u << q) << (8 * (pos & 3)));
     }
   }
+  __syncthreads();
+  // the masks of entries [0, s_total), 8 bytes per store (a unit's 8k bytes
+  // start 8-byte aligned; bytes past s_total are zeros)
+  uint2* gm = reinterpret_cast<uint2*>(plan_mask + obase);
+  const uint2* sm2 = reinterpret_cast<const uint2*>(msk);
+  for (int x = tid; x < (s_total + 7) / 8; x += kPlanThreads) gm[x] = sm2[x];
   if (tid == 0) plan_count[unit] = s_total;
 }
 
