@@ -164,7 +164,33 @@ def setup(wl, dev, seq):
     return p, model, q, out, sel, cnt
 
 
-def stage_times(wl, p, model, q, dev):
+def make_paged(wl, model, dev):
+    """The decode caches moved into a pool of 16-token pages in a seeded
+    shuffled order: (k_pool, v_pool, page_table)."""
+    S, L, G, D = model.k.shape
+    per = (L + 15) // 16
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(wl.seed)
+    table = torch.randperm(S * per, generator=gen).to(torch.int32).view(S, per).to(dev).contiguous()
+    kp = torch.empty((S * per, 16, G, D), dtype=model.k.dtype, device=dev)
+    vp = torch.empty_like(kp)
+    idx = table.view(-1).long()
+    kp[idx] = model.k[:, :per * 16].reshape(S * per, 16, G, D)
+    vp[idx] = model.v[:, :per * 16].reshape(S * per, 16, G, D)
+    return kp.view(S * per * 16, G, D), vp.view(S * per * 16, G, D), table
+
+
+def attend(p, wl, model, q, q0, n, sel, cnt, out, paged):
+    """The attention call of one chunk: contiguous caches, or the paged pool."""
+    from sparse_long_context_sgqa_b200 import binding as Bd
+    S = wl.num_seqs
+    if paged is None:
+        Bd.sgqa_sparse_attn(p, S, q0, n, q, wl.seq_len, wl.seq_len, model.k, model.v, sel, cnt, out, model.ws)
+    else:
+        Bd.sgqa_sparse_attn_paged(p, S, q0, n, q, paged[0], paged[1], paged[2], wl.seq_len, sel, cnt, out)
+
+
+def stage_times(wl, p, model, q, dev, paged=None):
     """One step with CUDA events between the stage calls; returns per-stage ms and work."""
     from sparse_long_context_sgqa_b200 import binding as Bd
     S, B, G, k = wl.num_seqs, wl.block, wl.groups, wl.topk
@@ -185,8 +211,7 @@ def stage_times(wl, p, model, q, dev):
         ev[1].record(st)
         Bd.sgqa_index_topk(p, S, q0, n, qs["idx_q"], qs["idx_w"], wl.seq_len, model.store, sel, cnt, model.ws)
         ev[2].record(st)
-        Bd.sgqa_sparse_attn(p, S, q0, n, qs["q"], wl.seq_len, wl.seq_len, model.k, model.v, sel, cnt, out,
-                            model.ws)
+        attend(p, wl, model, qs["q"], q0, n, sel, cnt, out, paged)
         ev[3].record(st)
         torch.cuda.synchronize()
         ms["merge"] += ev[0].elapsed_time(ev[1])
@@ -253,8 +278,23 @@ def cuda_arm(args, wl, rank, world, local_rank):
     chunk = min(wl.chunk, wl.nq)
     n_chunks = (wl.nq + chunk - 1) // chunk
 
+    paged = None
+    if args.paged:
+        if wl.nq > 32:
+            raise SystemExit("--paged: decode workloads only (at most 32 queries per sequence)")
+        paged = make_paged(wl, model, dev)
+
     def eager_step():
-        if wl.nq <= 32:
+        if paged is not None:
+            # merge, index and the paged attention: sgqa_forward's three stages
+            from sparse_long_context_sgqa_b200 import binding as Bd
+            q0, B = wl.q_start, wl.block
+            Bd.sgqa_merge_blocks(p, wl.num_seqs, wl.seq_len, model.kp, model.c, q0 // B, (q0 + wl.nq) // B, None,
+                                 model.store)
+            Bd.sgqa_index_topk(p, wl.num_seqs, q0, wl.nq, q["idx_q"], q["idx_w"], wl.seq_len, model.store, sel, cnt,
+                               model.ws)
+            attend(p, wl, model, q["q"], q0, wl.nq, sel, cnt, out, paged)
+        elif wl.nq <= 32:
             model.forward(wl.q_start, q["q"], q["idx_q"], q["idx_w"], sel, cnt, out)
         else:
             model.prefill(q["q"], q["idx_q"], q["idx_w"], out, sel, cnt, q_pos0=wl.q_start)
@@ -282,7 +322,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    ms_stage, work = stage_times(wl, p, model, q, dev)
+    ms_stage, work = stage_times(wl, p, model, q, dev, paged)
 
     if world > 1:
         torch.distributed.barrier()
@@ -326,7 +366,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
 
     peaks = load_peaks()
     per_launch_ms = {k: v / max(1, work["launches"]) for k, v in ms_stage.items()}
-    traffic = TRAFFIC.get(wl.name)
+    traffic = None if paged is not None else TRAFFIC.get(wl.name)  # captured for the contiguous caches
     if wl.nq <= 32:
         achieved = work["attn_bytes"] / work["launches"] / (per_launch_ms["attention"] / 1e3) / 1e9
         roof = {"kernel": "sparse attention (decode gather: attn_decode_tma_kernel)", "bound": "hbm",
@@ -351,7 +391,8 @@ def cuda_arm(args, wl, rank, world, local_rank):
         "metric": METRIC[wl.name][0], "value": value, "unit": METRIC[wl.name][1], "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "seq_len": wl.seq_len, "num_seqs": wl.num_seqs, "queries": wl.nq,
+        "config": {"workload": wl.name + ("_paged16" if paged is not None else ""), "seq_len": wl.seq_len,
+                   "num_seqs": wl.num_seqs, "queries": wl.nq,
                    "chunk": chunk, "groups": wl.groups, "heads": wl.n_heads, "head_dim": wl.head_dim,
                    "idx_heads": wl.idx_heads, "block": wl.block, "topk": wl.topk,
                    "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (no flush)"},
@@ -458,6 +499,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="decode: launch eagerly instead of replaying a CUDA graph")
+    ap.add_argument("--paged", action="store_true",
+                    help="decode: K/V in a pool of 16-token pages in shuffled order (sgqa_sparse_attn_paged)")
     ap.add_argument("--seq-len", type=int, default=0, help="override the workload's context length")
     ap.add_argument("--num-seqs", type=int, default=0, help="override the workload's sequence count")
     args = ap.parse_args()

@@ -215,6 +215,31 @@ sgqa_status sgqa_sparse_attn_noalloc(const sgqa_params* p, int64_t num_seqs, int
                                      const int32_t* sel, const int32_t* sel_count, void* out, void* stream);
 
 /*
+ * Decode sparse attention over a paged K/V cache.  Page section "Cache
+ * capacity: 4,104 reads do not mean 4,104 stored tokens": capacity is kept in
+ * 16-token pages reached through page tables.  The computation is that of
+ * sgqa_sparse_attn_gated; only where the tokens live differs: token j of
+ * sequence s is row page_table[s][j / 16] * 16 + j % 16 of the pools.
+ *
+ * k_pool, v_pool : [num_pages * 16, G, D] bf16 (physical pages of 16 tokens)
+ * page_table     : [S, max_pages] int32, the physical page of each logical
+ *                  page; pages [0, ceil(cache_len / 16)) of every sequence
+ *                  must be mapped to pages in [0, num_pages)
+ * cache_len      : valid tokens of every sequence (q_pos0 + nq <= cache_len)
+ * q, sel, sel_count, gate (NULL = no gate), out : as sgqa_sparse_attn_gated
+ *
+ * Decode-sized calls only: nq <= 32 queries per sequence and block_size 8;
+ * others return SGQA_ERR_UNSUPPORTED.  Needs no workspace.  A page-table
+ * entry outside [0, num_pages) reads zeros and makes sgqa_check report
+ * SGQA_ERR_DEVICE.
+ */
+sgqa_status sgqa_sparse_attn_paged(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                                   const void* q, const void* k_pool, const void* v_pool, int64_t num_pages,
+                                   const int32_t* page_table, int64_t max_pages, int64_t cache_len,
+                                   const int32_t* sel, const int32_t* sel_count, const void* gate, void* out,
+                                   void* stream);
+
+/*
  * Synchronise `stream` and report the device status word that bounded waits
  * and device-side checks write (then clear it).  Returns SGQA_OK,
  * SGQA_ERR_TIMEOUT, SGQA_ERR_DEVICE or SGQA_ERR_CUDA.

@@ -505,13 +505,15 @@ __device__ __forceinline__ uint32_t blk_off(uint32_t r, uint32_t j) {
 }
 
 constexpr int kDecMaxSplit = 8;  // splits of a row = one (portable) cluster
+constexpr int kPageTokens = 16;  // tokens per page of a paged K/V cache
 
 __global__ void __launch_bounds__(kDecThreads, 2)
 attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                        const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ sel,
                        const int32_t* __restrict__ sel_count, __nv_bfloat16* __restrict__ out,
                        const __nv_bfloat16* __restrict__ gate, int64_t nq, int G, int k, int64_t q_pos0, int nsplit,
-                       float scale_log2) {
+                       float scale_log2, const int32_t* __restrict__ page_table, int64_t max_pages,
+                       int64_t num_pages) {
   extern __shared__ uint8_t smem_raw[];
   DecSmem& sm = *reinterpret_cast<DecSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
@@ -524,6 +526,7 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
   const int64_t t = q_pos0 + i;
   const int cnt = min(max(sel_count[row], 0), k);
   const int32_t* ids = sel + row * k;
+  const int32_t tseq = page_table != nullptr ? 0 : static_cast<int32_t>(seq);  // a paged pool has no sequence axis
   const int nblk = cnt + 1;  // selected blocks, then the current block
   const int per = (nblk + nsplit - 1) / nsplit;
   const int b0 = min(nblk, split * per), b1 = min(nblk, b0 + per);
@@ -542,7 +545,18 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
   // stage the block rows (one coalesced read instead of a dependent load per TMA issue)
   for (int b = threadIdx.x; b < nb; b += kDecThreads) {
     const int e = b0 + b;
-    sm.rows[b] = e < cnt ? ids[e] * 8 : static_cast<int32_t>(cur0);
+    int32_t r = e < cnt ? ids[e] * 8 : static_cast<int32_t>(cur0);  // first token of the block
+    if (page_table != nullptr) {
+      // paged cache: the block's 8 tokens lie in one 16-token page of the pool
+      const int32_t pg = page_table[seq * max_pages + (r >> 4)];
+      if (pg < 0 || pg >= num_pages) {
+        report(kDevBounds);
+        r = -64;  // outside the pool: the copy reads zeros
+      } else {
+        r = pg * kPageTokens + (r & (kPageTokens - 1));
+      }
+    }
+    sm.rows[b] = r;
   }
   // Q into shared memory (its fragments are re-read per k-step: held in
   // registers they pushed the O accumulators into local memory)
@@ -579,8 +593,8 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
         if (ok) {
           const int32_t r = b < nb ? sm.rows[b] : -64;  // -64: zero-filled tail block
           tc::mbar_expect_tx(bar(sm.full[slot]), 2 * 3 * 1024);
-          tc::tma_load_5d(smem_u32(&sm.kv[slot][0][0]), &kmap, 0, r, 0, g, static_cast<int32_t>(seq), bar(sm.full[slot]));
-          tc::tma_load_5d(smem_u32(&sm.kv[slot][1][0]), &vmap, 0, r, 0, g, static_cast<int32_t>(seq), bar(sm.full[slot]));
+          tc::tma_load_5d(smem_u32(&sm.kv[slot][0][0]), &kmap, 0, r, 0, g, tseq, bar(sm.full[slot]));
+          tc::tma_load_5d(smem_u32(&sm.kv[slot][1][0]), &vmap, 0, r, 0, g, tseq, bar(sm.full[slot]));
           mine_end = b + 1;
         }
       }

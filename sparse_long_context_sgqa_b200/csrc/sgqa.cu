@@ -457,7 +457,8 @@ sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, sgqa::attn_decode_tma_kernel, km, vm, qb, sel, sel_count, ob, gb, nq, G,
-                                       k, q0, nsplit, scale_log2);
+                                       k, q0, nsplit, scale_log2, static_cast<const int32_t*>(nullptr),
+                                       static_cast<int64_t>(0), static_cast<int64_t>(0));
     if (e != cudaSuccess) return cuda_fail(e, "attn_decode_tma_kernel launch");
     SGQA_LAUNCH_CHECK("attn_decode_tma_kernel");
     return SGQA_OK;
@@ -505,6 +506,49 @@ sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq,
     SGQA_LAUNCH_CHECK("attn_grouped_kernel");
     return SGQA_OK;
   }
+}
+
+// Decode attention over a paged K/V cache: the TMA-fed gather kernel with its
+// tensor maps over the page pool [num_pages * 16 tokens, G, D] and each
+// block's row looked up in the page table.
+sgqa_status launch_attn_decode_paged(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q,
+                                     const void* kpool, const void* vpool, int64_t num_pages,
+                                     const int32_t* page_table, int64_t max_pages, const int32_t* sel,
+                                     const int32_t* sel_count, const void* gate, void* out, cudaStream_t st) {
+  const int G = p->num_kv_groups, k = p->topk;
+  const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
+  const int64_t rows = S * nq * G;
+  const int64_t pool_rows = num_pages * sgqa::kPageTokens;
+  CUtensorMap km, vm;
+  cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(pool_rows), 3, static_cast<cuuint64_t>(G), 1};
+  // the last axis (size 1) stands where the contiguous maps have the sequence
+  cuuint64_t strides[4] = {static_cast<cuuint64_t>(G) * 384, 128, 384, static_cast<cuuint64_t>(G) * 384};
+  cuuint32_t box[5] = {64, 8, 3, 1, 1};
+  sgqa_status s;
+  if ((s = encode_bf16(&km, kpool, 5, dims, strides, box, "k_pool")) != SGQA_OK) return s;
+  if ((s = encode_bf16(&vm, vpool, 5, dims, strides, box, "v_pool")) != SGQA_OK) return s;
+  const int nsplit = std::min(decode_splits(rows), sgqa::kDecMaxSplit);
+  const size_t smem = sizeof(sgqa::DecSmem) + 1024;
+  cudaFuncSetAttribute(sgqa::attn_decode_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(rows * nsplit));
+  cfg.blockDim = dim3(sgqa::kDecThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(nsplit);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, sgqa::attn_decode_tma_kernel, km, vm, static_cast<const __nv_bfloat16*>(q),
+                                     sel, sel_count, static_cast<__nv_bfloat16*>(out),
+                                     static_cast<const __nv_bfloat16*>(gate), nq, G, k, q0, nsplit, scale_log2,
+                                     page_table, max_pages, num_pages);
+  if (e != cudaSuccess) return cuda_fail(e, "attn_decode_tma_kernel launch (paged)");
+  SGQA_LAUNCH_CHECK("attn_decode_tma_kernel");
+  return SGQA_OK;
 }
 
 sgqa_status do_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q,
@@ -721,6 +765,39 @@ sgqa_status sgqa_forward_gated(const sgqa_params* p, int64_t num_seqs, int64_t q
                                size_t workspace_bytes, void* stream) {
   return forward_impl(p, num_seqs, q_pos0, nq, q, idx_q, idx_w, cache_cap, cache_len, proxy_k, comp_logits, k_cache,
                       v_cache, merged_f32, store, sel, sel_count, gate, out, workspace, workspace_bytes, stream);
+}
+
+sgqa_status sgqa_sparse_attn_paged(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
+                                   const void* q, const void* k_pool, const void* v_pool, int64_t num_pages,
+                                   const int32_t* page_table, int64_t max_pages, int64_t cache_len,
+                                   const int32_t* sel, const int32_t* sel_count, const void* gate, void* out,
+                                   void* stream) {
+  g_err.clear();
+  sgqa_status s = check_params(p);
+  if (s != SGQA_OK) return s;
+  if (num_seqs < 1) return fail(SGQA_ERR_INVALID_ARGUMENT, "num_seqs must be >= 1");
+  if (q_pos0 < 0 || nq < 0) return fail(SGQA_ERR_INVALID_ARGUMENT, "q_pos0 and nq must be >= 0");
+  if (nq == 0) return SGQA_OK;
+  if (nq > kDecodeMaxNq)
+    return fail(SGQA_ERR_UNSUPPORTED, "sgqa_sparse_attn_paged takes at most %d queries per sequence (got %lld)",
+                (int)kDecodeMaxNq, (long long)nq);
+  if (p->block_size != 8) return fail(SGQA_ERR_UNSUPPORTED, "sgqa_sparse_attn_paged needs block_size 8");
+  if (cache_len < q_pos0 + nq) return fail(SGQA_ERR_INVALID_ARGUMENT, "need q_pos0 + nq <= cache_len");
+  if (max_pages * sgqa::kPageTokens < cache_len)
+    return fail(SGQA_ERR_INVALID_ARGUMENT, "max_pages (%lld) pages of %d tokens do not hold cache_len %lld",
+                (long long)max_pages, sgqa::kPageTokens, (long long)cache_len);
+  if (num_pages < 1 || num_pages * sgqa::kPageTokens > (int64_t(1) << 31) - 1)
+    return fail(SGQA_ERR_UNSUPPORTED, "num_pages must be in [1, 2^27)");
+  REQUIRE_PTR(q, 16);
+  REQUIRE_PTR(k_pool, 16);
+  REQUIRE_PTR(v_pool, 16);
+  REQUIRE_PTR(page_table, 4);
+  REQUIRE_PTR(sel, 4);
+  REQUIRE_PTR(sel_count, 4);
+  REQUIRE_PTR(out, 16);
+  if (gate != nullptr && !aligned(gate, 2)) return fail(SGQA_ERR_INVALID_ARGUMENT, "gate must be 2-byte aligned");
+  return launch_attn_decode_paged(p, num_seqs, q_pos0, nq, q, k_pool, v_pool, num_pages, page_table, max_pages, sel,
+                                  sel_count, gate, out, static_cast<cudaStream_t>(stream));
 }
 
 sgqa_status sgqa_sparse_attn_noalloc(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,

@@ -107,6 +107,17 @@ def test_null_and_range_checks_before_any_launch(lib, bd):
                                 dummy, dummy, dummy, odd, dummy, dummy, ctypes.c_size_t(1 << 30), st)
     assert rc == 1
     assert b"gate" in ctypes.string_at(lib.sgqa_last_error())
+    # paged decode: decode-sized calls with B = 8 only, a page table that covers cache_len
+    def paged(nq, max_pages, cache_len=4096, pt=dummy):
+        return lib.sgqa_sparse_attn_paged(ctypes.byref(p), ctypes.c_int64(1), ctypes.c_int64(4000), ctypes.c_int64(nq),
+                                          dummy, dummy, dummy, ctypes.c_int64(300), pt, ctypes.c_int64(max_pages),
+                                          ctypes.c_int64(cache_len), dummy, dummy, None, dummy, st)
+    assert paged(33, 256) == 2
+    assert paged(4, 255) == 1 and b"max_pages" in ctypes.string_at(lib.sgqa_last_error())
+    assert paged(4, 256, pt=ctypes.c_void_p(4096 + 2)) == 1
+    p.block_size = 4
+    assert paged(4, 256) == 2
+    p.block_size = 8
     # nothing to do is not an error
     rc = lib.sgqa_forward(ctypes.byref(p), ctypes.c_int64(1), ctypes.c_int64(0), ctypes.c_int64(0), None, None,
                           None, ctypes.c_int64(0), ctypes.c_int64(0), None, None, None, None, None, None, None,

@@ -296,6 +296,75 @@ def test_sparse_attn_gated_parity(cuda_device, case):
         _attn_isolated(wl, cuda_device, 19990, 10, range(10), num_seqs=2, gated=True)
 
 
+def _paged_pool(k, v, rng, spare=37):
+    """Pools of 16-token pages holding every sequence's cache in shuffled pages."""
+    S, L, G, D = k.shape
+    per = (L + 15) // 16
+    num_pages = S * per + spare
+    perm = torch.from_numpy(rng.permutation(num_pages)[:S * per].astype(np.int32)).to(k.device)
+    table = perm.view(S, per).contiguous()
+    kp = torch.zeros((num_pages, 16, G, D), dtype=k.dtype, device=k.device)
+    vp = torch.zeros_like(kp)
+    pad = per * 16 - L
+    kpad = torch.nn.functional.pad(k, (0, 0, 0, 0, 0, pad)).view(S * per, 16, G, D)
+    vpad = torch.nn.functional.pad(v, (0, 0, 0, 0, 0, pad)).view(S * per, 16, G, D)
+    kp[table.view(-1).long()] = kpad
+    vp[table.view(-1).long()] = vpad
+    return kp.view(num_pages * 16, G, D), vp.view(num_pages * 16, G, D), table
+
+
+def test_sparse_attn_paged_equals_contiguous(cuda_device):
+    """A paged cache (16-token pages in shuffled order, spare pages) gives the
+    contiguous path's output bit for bit, gated, and the oracle's."""
+    wl = dataclasses.replace(SMALL8, seq_len=20000, name="dec")
+    S, q0, nq, L = 3, 19990, 10, 20000
+    cache, _ = Hn.make_inputs(wl, cuda_device, seqs=range(S))
+    qs = [I.make_queries(wl, cuda_device, q0, nq, seq=s) for s in range(S)]
+    q = torch.stack([x["q"] for x in qs]).to(torch.bfloat16).contiguous()
+    sel, cnt = I.make_selection(wl, cuda_device, q0, nq, num_seqs=S)
+    gate = torch.stack([I.make_gate(wl, cuda_device, q0, nq, seq=s) for s in range(S)]).contiguous()
+    p = Hn.params_for(wl)
+    out_c = torch.zeros((S, nq, wl.n_heads, wl.head_dim), dtype=torch.bfloat16, device=cuda_device)
+    out_p = torch.zeros_like(out_c)
+    ws = _bd().alloc_workspace(p, S, nq, q0 + nq, cuda_device)
+    _bd().sgqa_sparse_attn_gated(p, S, q0, nq, q, L, L, cache["k"], cache["v"], sel, cnt, gate, out_c, ws)
+    kpool, vpool, table = _paged_pool(cache["k"], cache["v"], np.random.default_rng(5))
+    _bd().sgqa_sparse_attn_paged(p, S, q0, nq, q, kpool, vpool, table, L, sel, cnt, out_p, gate=gate)
+    _bd().sgqa_check()
+    assert torch.equal(out_p, out_c)
+    worst = 0.0
+    for s in range(S):
+        K, V = Hn.to_np(cache["k"][s]), Hn.to_np(cache["v"][s])
+        seln, cntn = sel[s].cpu().numpy(), cnt[s].cpu().numpy()
+        on, qn, gn = out_p[s].float().cpu().numpy(), Hn.to_np(q[s]), Hn.to_np(gate[s])
+        for i in range(nq):
+            for g in range(wl.groups):
+                pos = O.attended_positions(q0 + i, seln[i, g, :cntn[i, g]], wl.block)
+                hs = slice(g * 16, (g + 1) * 16)
+                ref = O.gated_head_output(O.sparse_attention(qn[i, hs], K[pos, g], V[pos, g], Hn.scale_of(wl)), gn[i, hs])
+                worst = max(worst, float(np.abs(on[i, hs] - ref).max()))
+    assert worst <= Hn.ATTN_ATOL, worst
+
+
+def test_sparse_attn_paged_bad_page_is_reported(cuda_device):
+    """A page-table entry outside the pool is caught by the kernel's check
+    (the copy reads zeros) and reported by sgqa_check as a device error."""
+    wl = dataclasses.replace(SMALL8, seq_len=4096, name="dec_bad")
+    S, q0, nq, L = 1, 4090, 4, 4096
+    cache, _ = Hn.make_inputs(wl, cuda_device, seqs=range(S))
+    q = I.make_queries(wl, cuda_device, q0, nq)["q"][None].to(torch.bfloat16).contiguous()
+    sel, cnt = I.make_selection(wl, cuda_device, q0, nq, num_seqs=S)
+    kpool, vpool, table = _paged_pool(cache["k"], cache["v"], np.random.default_rng(6), spare=0)
+    table[0, 255] = kpool.shape[0] // 16 + 3  # the page of the current block (tokens 4080..4095)
+    out = torch.zeros((S, nq, wl.n_heads, wl.head_dim), dtype=torch.bfloat16, device=cuda_device)
+    p = Hn.params_for(wl)
+    _bd().sgqa_sparse_attn_paged(p, S, q0, nq, q, kpool, vpool, table, L, sel, cnt, out)
+    with pytest.raises(_bd().SgqaError) as err:
+        _bd().sgqa_check()
+    assert err.value.code == 6  # SGQA_ERR_DEVICE
+    _bd().sgqa_check()  # the status word was cleared
+
+
 def test_forward_gated_equals_gate_times_forward(cuda_device):
     """sgqa_forward_gated = sigmoid(gate) * sgqa_forward, head by head (same
     inputs, one 2048-token prefill chunk)."""
