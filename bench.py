@@ -49,7 +49,7 @@ TRAFFIC = {
     "prefill8k": 396776192,      # attn_tc_kernel, one launch (one 8192-query chunk)
     "prefill128k": 2093507584,   # attn_tc_kernel, mean over the 16 chunk launches of one step
     "prefill1m": None,           # dominant stage: the index stage (several kernels, tensor/ALU bound)
-    "decode": 234788864,         # attn_decode_tma_kernel, one launch (16 sequences)
+    "decode": 234981632,         # attn_decode_tma_kernel, one launch (16 sequences)
 }
 
 
