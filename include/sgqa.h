@@ -121,7 +121,7 @@ sgqa_status sgqa_index_topk(const sgqa_params* p, int64_t num_seqs, int64_t q_po
  * Sparse attention over the selected original K/V.  Page sections "Main
  * attention still reads original K/V" and "Selection is a weighted ReLU
  * score ...": query head h uses group g = floor(h / Hg); it attends, with
- * ordinary scaled dot products and an exact softmax, to every token of the
+ * plain scaled dot-product scores and an exact softmax, to every token of the
  * blocks in sel[t, g] plus the positions B*floor(t/B) .. t of its current
  * block.  The Hg heads of a group share the selection.  The output is the
  * pre-gate head vector.

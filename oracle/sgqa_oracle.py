@@ -23,12 +23,12 @@ extraction; the formulas below are the readings of the surrounding prose:
                 Q8 = the E4M3 store value widened losslessly to BF16.  No
                 softmax, no extra scale.
 * selection  -- same section: only blocks r < floor(t/B) compete; top-k by
-                score, equal scores resolved by ascending block id; the block
-                containing t is appended, restricted to positions <= t.
+                score, equal scores resolved by ascending block id; t's own
+                block is added on top, limited to positions <= t.
 * attention  -- section "Main attention still reads original K/V": head h uses
-                group g(h) = floor(h / heads_per_group); ordinary scaled dot
-                products and an exact softmax over the group's selected
-                original tokens.
+                group g(h) = floor(h / heads_per_group); plain scaled
+                dot-product scores and an exact softmax over the group's
+                selected original tokens.
 * gate       -- same section: each head's result scaled by the sigmoid of its
                 own gate logit (one per token and head).
 
