@@ -38,8 +38,8 @@ float64).  All accumulation is float64.
 Parity pins: every function here is pinned by tests under ``tests/`` against
 closed forms, invariants, library routines (torch's BF16/E4M3 casts, torch's
 scaled_dot_product_attention, Python's sorted) or brute force.  No function is
-"parity unpinned" except ``token_coverage`` (the pages do not define the
-measure; see its docstring).
+parity unpinned; ``token_coverage`` implements this build's reading of a
+measure the pages leave undefined (see its docstring).
 """
 from __future__ import annotations
 
@@ -288,12 +288,14 @@ def forward_rows(rows, *, q, k, v, idx_q, idx_w, keys, block, topk,
 
 
 def token_coverage(q_heads, k_all, positions, scale) -> float:
-    """Dense-softmax mass that the attended positions capture (parity unpinned).
+    """Dense-softmax mass that the attended positions capture.
 
     The second page reports token coverage for B=8,k=4096 against B=1,k=2048
     without defining it.  Reading adopted here: for one query row, the mean over
     the group's heads of the causal dense softmax probability mass that falls on
-    the attended positions.  k_all holds the K rows of positions 0..t.
+    the attended positions.  k_all holds the K rows of positions 0..t.  The
+    definition is this reading; the pins check its implementation (full set,
+    complements, equal logits, torch's softmax).
     """
     q_heads = np.asarray(q_heads, dtype=np.float64)
     k_all = np.asarray(k_all, dtype=np.float64)

@@ -359,3 +359,26 @@ def test_gate_on_single_token_attention_is_gated_value_row():
     g = rng.standard_normal(16)
     np.testing.assert_allclose(O.gated_head_output(att, g), (1 / (1 + np.exp(-g)))[:, None] * v[0][None, :],
                                rtol=1e-13, atol=0)
+
+
+# --------------------------------------------------------------------------
+# Token coverage (this build's reading of the second page's undefined measure)
+# --------------------------------------------------------------------------
+
+def test_token_coverage_invariants_and_torch_softmax():
+    """All positions cover 1; a set and its complement sum to 1; equal logits
+    give |A| / (t + 1); the value matches torch's softmax mass directly."""
+    rng = np.random.default_rng(13)
+    q = rng.standard_normal((16, 192))
+    k = rng.standard_normal((40, 192))
+    scale = 192 ** -0.5
+    allpos = np.arange(40)
+    assert abs(O.token_coverage(q, k, allpos, scale) - 1.0) < 1e-14
+    a = rng.choice(40, size=17, replace=False)
+    comp = np.setdiff1d(allpos, a)
+    assert abs(O.token_coverage(q, k, a, scale) + O.token_coverage(q, k, comp, scale) - 1.0) < 1e-14
+    assert O.token_coverage(np.zeros((16, 192)), k, a, scale) == pytest.approx(17 / 40, abs=1e-15)
+    p = torch.softmax(torch.from_numpy(q @ k.T * scale), dim=1)
+    ref = float(p[:, torch.from_numpy(a)].sum(dim=1).mean())
+    assert O.token_coverage(q, k, a, scale) == pytest.approx(ref, abs=1e-13)
+
