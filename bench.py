@@ -391,11 +391,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
         "metric": METRIC[wl.name][0], "value": value, "unit": METRIC[wl.name][1], "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name + ("_paged16" if paged is not None else ""), "seq_len": wl.seq_len,
-                   "num_seqs": wl.num_seqs, "queries": wl.nq,
-                   "chunk": chunk, "groups": wl.groups, "heads": wl.n_heads, "head_dim": wl.head_dim,
-                   "idx_heads": wl.idx_heads, "block": wl.block, "topk": wl.topk,
-                   "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (no flush)"},
+        "config": workload_config(wl, world, paged is not None),
         "stages_ms_per_step": ms_stage,
         "union": work.get("union"),
         "stage_tflops": {"index": work["index_flops"] / (ms_stage["index"] / 1e3) / 1e12 if ms_stage["index"] else None,
@@ -477,14 +473,21 @@ def oracle_sample(wl, budget_s: float = 20.0, max_rows: int = 64):
                       f"tokens/s = 1/(merge_s/N + row_s/rows)"}
 
 
-def reference_arm(args, wl):
+def workload_config(wl, world: int, paged: bool = False) -> dict:
+    """The `config` object of both arms' JSON lines."""
+    return {"workload": wl.name + ("_paged16" if paged else ""), "seq_len": wl.seq_len, "num_seqs": wl.num_seqs,
+            "queries": wl.nq, "chunk": min(wl.chunk, wl.nq), "groups": wl.groups, "heads": wl.n_heads,
+            "head_dim": wl.head_dim, "idx_heads": wl.idx_heads, "block": wl.block, "topk": wl.topk,
+            "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (no flush)"}
+
+
+def reference_arm(args, wl, world: int = 1):
     cb = oracle_sample(wl, budget_s=max(5.0, 15.0 / max(1, args.steps)))
     ms = 1e3 / cb["value"]
     return {"impl": "reference", "metric": METRIC[wl.name][0], "value": cb["value"], "unit": "tokens/s",
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms * wl.nq,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": wl.name, "seq_len": wl.seq_len, "queries": wl.nq,
-                                            "block": wl.block, "topk": wl.topk},
+            "data": "synthetic", "config": workload_config(wl, world, getattr(args, "paged", False)),
             "cpu_baseline": cb,
             "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -514,7 +517,7 @@ def main():
 
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(reference_arm(args, wl)), flush=True)
+            print(json.dumps(reference_arm(args, wl, world)), flush=True)
         return
 
     if world > 1:
