@@ -336,6 +336,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
         step()
     e1.record(st)
     torch.cuda.synchronize()
+    n_launch1 = Bd.launch_count()  # before any untimed step below
     # nvidia-smi samples every 200 ms: a timed region shorter than a second is
     # followed by the same (untimed) steps until a second of load has been
     # sampled, so that the clock record holds several samples under load
@@ -351,7 +352,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
         clocks["window"] = clock_window
     # kernels launched in the timed region: counted by the library (a graph
     # replay launches the kernels captured once per step)
-    gpu_launches = graph_launches * args.steps if graph is not None else Bd.launch_count() - n_launch0
+    gpu_launches = graph_launches * args.steps if graph is not None else n_launch1 - n_launch0
     elapsed = max_over_ranks(e0.elapsed_time(e1), dev)
     if world > 1:
         torch.distributed.barrier()
