@@ -6,7 +6,6 @@ boundary; selections bit-exact except swaps between scores within 1e-5
 relative of the k-th score; attention outputs 2e-2 max-abs on bf16 outputs.
 """
 import dataclasses
-import math
 
 import numpy as np
 import pytest
