@@ -1,9 +1,10 @@
 """User-facing API: one object that owns the caches and workspace of a batch of
 sequences and runs the hot path chunk by chunk through the C ABI.
 
-``SparseGQA.prefill`` / ``decode`` take device tensors; ``forward_host`` takes
-pinned host tensors and copies them in and the result out (the end-to-end
-path).  All arithmetic runs in ``libsgqa.so``.
+``SparseGQA.forward`` (one call: a decode step or one chunk) and ``prefill``
+(all chunks) take device tensors; ``forward_host`` takes pinned host tensors
+and copies them in and the result out (the end-to-end path).  All arithmetic
+runs in ``libsgqa.so``.
 """
 from __future__ import annotations
 
@@ -31,17 +32,37 @@ class SparseGQA:
                        if keep_merged_f32 else None)
         self.ws = Bd.alloc_workspace(params, num_seqs, chunk, capacity, device)
 
-    def forward(self, q_pos0, q, idx_q, idx_w, sel, sel_count, out, cache_len=None, stream=None):
-        """One call of the hot path for queries [q_pos0, q_pos0 + nq) (nq <= chunk)."""
-        nq = q.shape[1]
-        Bd.sgqa_forward(self.p, self.S, q_pos0, nq, q, idx_q, idx_w, self.cap,
-                        self.cap if cache_len is None else cache_len, self.kp, self.c, self.k, self.v,
-                        self.merged, self.store, sel, sel_count, out, self.ws, stream)
+    def forward(self, q_pos0, q, idx_q, idx_w, sel, sel_count, out, cache_len=None, stream=None, gate=None):
+        """One call of the hot path for queries [q_pos0, q_pos0 + nq) (nq <= chunk).
 
-    def prefill(self, q, idx_q, idx_w, out, sel=None, sel_count=None, q_pos0=0, stream=None):
-        """Chunked prefill of all queries in q ([S, N, G*Hg, D]); caches already hold their K/V."""
+        Every tensor is contiguous with the layouts of include/sgqa.h; gate
+        ([S, nq, G*Hg] bf16 logits) applies the head-wise sigmoid output gate.
+        """
+        nq = q.shape[1]
+        clen = self.cap if cache_len is None else cache_len
+        if gate is None:
+            Bd.sgqa_forward(self.p, self.S, q_pos0, nq, q, idx_q, idx_w, self.cap, clen, self.kp, self.c, self.k,
+                            self.v, self.merged, self.store, sel, sel_count, out, self.ws, stream)
+        else:
+            Bd.sgqa_forward_gated(self.p, self.S, q_pos0, nq, q, idx_q, idx_w, self.cap, clen, self.kp, self.c,
+                                  self.k, self.v, self.merged, self.store, sel, sel_count, gate, out, self.ws, stream)
+
+    def prefill(self, q, idx_q, idx_w, out, sel=None, sel_count=None, q_pos0=0, stream=None, gate=None):
+        """Chunked prefill of all queries in q ([S, N, G*Hg, D]); caches already hold their K/V.
+
+        A chunk of a batch of several sequences is not contiguous in q: it is
+        copied into a contiguous tensor before the call.
+        """
         S, N = q.shape[0], q.shape[1]
         G, k = self.p.num_kv_groups, self.p.topk
+        if self.device.type != "cuda":  # host-side use (tests with a stand-in library)
+            self._prefill_chunks(q, idx_q, idx_w, out, sel, sel_count, q_pos0, stream, gate, S, N, G, k)
+            return
+        st = torch.cuda.current_stream(self.device) if stream is None else stream
+        with torch.cuda.stream(st):  # the chunk copies run on the calls' stream
+            self._prefill_chunks(q, idx_q, idx_w, out, sel, sel_count, q_pos0, st, gate, S, N, G, k)
+
+    def _prefill_chunks(self, q, idx_q, idx_w, out, sel, sel_count, q_pos0, stream, gate, S, N, G, k):
         for c0 in range(0, N, self.chunk):
             n = min(self.chunk, N - c0)
             s_sel = sel[:, c0:c0 + n] if sel is not None and S == 1 else torch.empty(
@@ -50,8 +71,9 @@ class SparseGQA:
                 (S, n, G), dtype=torch.int32, device=self.device)
             o = out[:, c0:c0 + n] if S == 1 else torch.empty((S, n) + tuple(out.shape[2:]),
                                                              dtype=out.dtype, device=self.device)
-            self.forward(q_pos0 + c0, q[:, c0:c0 + n], idx_q[:, c0:c0 + n], idx_w[:, c0:c0 + n],
-                         s_sel, s_cnt, o, stream=stream)
+            self.forward(q_pos0 + c0, q[:, c0:c0 + n].contiguous(), idx_q[:, c0:c0 + n].contiguous(),
+                         idx_w[:, c0:c0 + n].contiguous(), s_sel, s_cnt, o, stream=stream,
+                         gate=None if gate is None else gate[:, c0:c0 + n].contiguous())
             if S != 1:
                 out[:, c0:c0 + n] = o
                 if sel is not None:
@@ -95,12 +117,18 @@ class SparseGQA:
                 ready = torch.cuda.Event()
                 ready.record(h2d_s)
             cur.wait_event(ready)
-            o = out[:, c0:c0 + n] if S == 1 else torch.empty((S, n) + tuple(out.shape[2:]), dtype=out.dtype,
-                                                             device=self.device)
-            self.forward(c0, dq["q"][:, c0:c0 + n], dq["idx_q"][:, c0:c0 + n], dq["idx_w"][:, c0:c0 + n],
-                         sel[:, :n], cnt[:, :n], o, stream=cur)
-            if S != 1:
-                out[:, c0:c0 + n] = o
+            with torch.cuda.stream(cur):  # the chunk's own copies run on the calls' stream
+                o = out[:, c0:c0 + n] if S == 1 else torch.empty((S, n) + tuple(out.shape[2:]), dtype=out.dtype,
+                                                                 device=self.device)
+                if S == 1 or n == self.chunk:
+                    c_sel, c_cnt = sel[:, :n], cnt[:, :n]
+                else:  # a short last chunk of several sequences: contiguous scratch of its own
+                    c_sel = torch.empty((S, n, G, k), dtype=torch.int32, device=self.device)
+                    c_cnt = torch.empty((S, n, G), dtype=torch.int32, device=self.device)
+                self.forward(c0, dq["q"][:, c0:c0 + n].contiguous(), dq["idx_q"][:, c0:c0 + n].contiguous(),
+                             dq["idx_w"][:, c0:c0 + n].contiguous(), c_sel, c_cnt, o, stream=cur)
+                if S != 1:
+                    out[:, c0:c0 + n] = o
             done = torch.cuda.Event()
             done.record(cur)
             d2h_s.wait_event(done)
