@@ -198,15 +198,21 @@ sgqa_status sgqa_forward_gated(const sgqa_params* p, int64_t num_seqs, int64_t q
  *
  * Same computation and arguments as sgqa_sparse_attn, minus the workspace.
  * It takes only calls with nq <= 32 queries per sequence (the split-K decode
- * path) whose split partials fit the library's static scratch array of
- * SGQA_NOALLOC_SCRATCH_BYTES (16 MiB) per device; larger calls return
- * SGQA_ERR_UNSUPPORTED with a message.  The array is a file-scope __device__
- * variable that every GPU loading the library holds until exit.  The first
- * call on a device looks up the array's device address (set-up); make that
- * first call before any stream capture.  All calls share the array, so calls
- * that overlap on the GPU (other streams, other host threads) race; order
- * them on one stream.  Nothing in the array needs clearing: every call writes
- * each partial it reads.  No cudaMalloc, cudaFree or allocating routine.
+ * path); more return SGQA_ERR_UNSUPPORTED.  With block_size 8 the splits of a
+ * row combine inside their thread-block cluster and no scratch is used.  With
+ * block_size 1, 2 or 4 the split partials (S * nq * G rows, each split 16 x D
+ * FP32 values plus a max and a sum per head) live in the library's static
+ * scratch array of SGQA_NOALLOC_SCRATCH_BYTES (16 MiB) per device; calls whose
+ * partials do not fit return SGQA_ERR_UNSUPPORTED with a message.  The array
+ * is a file-scope __device__ variable that every GPU loading the library
+ * holds until exit.  The first call on a device that uses the array looks up
+ * its device address (set-up); make that first call before any stream
+ * capture.  The address is looked up once per device and process: calls
+ * after cudaDeviceReset() on that device are not supported.  All calls share
+ * the array, so calls that overlap on the GPU (other streams, other host
+ * threads) race; order them on one stream.  Nothing in the array needs
+ * clearing: every call writes each partial it reads.  No cudaMalloc, cudaFree
+ * or allocating routine.
  */
 #define SGQA_NOALLOC_SCRATCH_BYTES (16u << 20)
 sgqa_status sgqa_sparse_attn_noalloc(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
@@ -215,29 +221,34 @@ sgqa_status sgqa_sparse_attn_noalloc(const sgqa_params* p, int64_t num_seqs, int
                                      const int32_t* sel, const int32_t* sel_count, void* out, void* stream);
 
 /*
- * Decode sparse attention over a paged K/V cache.  Page section "Cache
- * capacity: 4,104 reads do not mean 4,104 stored tokens": capacity is kept in
- * 16-token pages reached through page tables.  The computation is that of
+ * Sparse attention over a paged K/V cache.  Page section "Cache capacity:
+ * 4,104 reads do not mean 4,104 stored tokens": capacity is kept in 16-token
+ * pages reached through page tables.  The computation is that of
  * sgqa_sparse_attn_gated; only where the tokens live differs: token j of
- * sequence s is row page_table[s][j / 16] * 16 + j % 16 of the pools.
+ * sequence s is row j % 16 of page page_table[s][j / 16] of the pools.  Each
+ * page holds its 16 tokens group by group, so one group's 8-token block is a
+ * contiguous 3 KB run (one copy).
  *
- * k_pool, v_pool : [num_pages * 16, G, D] bf16 (physical pages of 16 tokens)
+ * k_pool, v_pool : [num_pages, G, 16, D] bf16 (physical pages of 16 tokens)
  * page_table     : [S, max_pages] int32, the physical page of each logical
  *                  page; pages [0, ceil(cache_len / 16)) of every sequence
  *                  must be mapped to pages in [0, num_pages)
  * cache_len      : valid tokens of every sequence (q_pos0 + nq <= cache_len)
  * q, sel, sel_count, gate (NULL = no gate), out : as sgqa_sparse_attn_gated
+ * workspace      : as sgqa_sparse_attn (sgqa_workspace_size); calls of at
+ *                  most 32 queries per sequence need none (NULL, 0)
  *
- * Decode-sized calls only: nq <= 32 queries per sequence and block_size 8;
- * others return SGQA_ERR_UNSUPPORTED.  Needs no workspace.  A page-table
- * entry outside [0, num_pages) reads zeros and makes sgqa_check report
- * SGQA_ERR_DEVICE.
+ * block_size 8 only (others return SGQA_ERR_UNSUPPORTED); any number of
+ * queries (decode-sized calls take the split gather, larger ones the
+ * tensor-core prefill kernel).  A page-table entry outside [0, num_pages)
+ * is never followed: its tokens read as zeros, sgqa_check reports
+ * SGQA_ERR_DEVICE, and the outputs of the call are undefined.
  */
 sgqa_status sgqa_sparse_attn_paged(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
                                    const void* q, const void* k_pool, const void* v_pool, int64_t num_pages,
                                    const int32_t* page_table, int64_t max_pages, int64_t cache_len,
                                    const int32_t* sel, const int32_t* sel_count, const void* gate, void* out,
-                                   void* stream);
+                                   void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Synchronise `stream` and report the device status word that bounded waits
@@ -245,6 +256,25 @@ sgqa_status sgqa_sparse_attn_paged(const sgqa_params* p, int64_t num_seqs, int64
  * SGQA_ERR_TIMEOUT, SGQA_ERR_DEVICE or SGQA_ERR_CUDA.
  */
 sgqa_status sgqa_check(void* stream);
+
+/*
+ * Time limit of the kernels' pipeline waits on the current device (a
+ * consumer waiting for its data, a producer for a free buffer slot), in
+ * nanoseconds; 0 restores the default and maximum of 2 s.  The pages have no
+ * counterpart: this is a diagnostic control.  A wait that runs out makes its
+ * kernel stop early (its outputs are then undefined), after it has let the
+ * copies and MMAs it already issued complete, and sgqa_check() reports
+ * SGQA_ERR_TIMEOUT; later calls run normally once the limit is long enough.
+ * A very short limit is how the tests make those waits run out; limits
+ * below 1 ms are counted in SM clock cycles (at most the given nanoseconds
+ * at clocks up to 2 GHz), since the device's nanosecond timer advances in
+ * steps of up to a microsecond.  The new
+ * limit applies to waits that start after the call returns; do not call it
+ * while kernels of this library run on the device.  Returns
+ * SGQA_ERR_INVALID_ARGUMENT above the maximum, SGQA_ERR_CUDA if the device
+ * variable cannot be written.
+ */
+sgqa_status sgqa_set_wait_limit_ns(uint64_t ns);
 
 /* Message of the last failed call on this thread ("" if none).  The pointer
  * stays valid until the next call on this thread. */

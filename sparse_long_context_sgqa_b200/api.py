@@ -99,11 +99,13 @@ class SparseGQA:
             self._copy_streams = (torch.cuda.Stream(device=self.device), torch.cuda.Stream(device=self.device))
         h2d_s, d2h_s = self._copy_streams
         S, N = host["q"].shape[0], host["q"].shape[1]
-        dq = {n: torch.empty(host[n].shape, dtype=host[n].dtype, device=self.device) for n in ("q", "idx_q", "idx_w")}
-        out = torch.empty(out_host.shape, dtype=out_host.dtype, device=self.device)
         G, k = self.p.num_kv_groups, self.p.topk
-        sel = torch.empty((S, self.chunk, G, k), dtype=torch.int32, device=self.device)
-        cnt = torch.empty((S, self.chunk, G), dtype=torch.int32, device=self.device)
+        with torch.cuda.stream(cur):  # the buffers belong to the calls' stream (and the two copy streams below)
+            dq = {n: torch.empty(host[n].shape, dtype=host[n].dtype, device=self.device)
+                  for n in ("q", "idx_q", "idx_w")}
+            out = torch.empty(out_host.shape, dtype=out_host.dtype, device=self.device)
+            sel = torch.empty((S, self.chunk, G, k), dtype=torch.int32, device=self.device)
+            cnt = torch.empty((S, self.chunk, G), dtype=torch.int32, device=self.device)
         h2d_s.wait_stream(cur)
         d2h_s.wait_stream(cur)
         for c0 in range(0, N, self.chunk):

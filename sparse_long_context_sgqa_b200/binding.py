@@ -27,7 +27,7 @@ STATUS = {0: "SGQA_OK", 1: "SGQA_ERR_INVALID_ARGUMENT", 2: "SGQA_ERR_UNSUPPORTED
 EXPORTED = ["sgqa_workspace_size", "sgqa_merge_blocks", "sgqa_index_topk", "sgqa_sparse_attn",
             "sgqa_sparse_attn_gated", "sgqa_forward", "sgqa_forward_gated", "sgqa_sparse_attn_paged",
             "sgqa_sparse_attn_noalloc",
-            "sgqa_check", "sgqa_last_error", "sgqa_version", "sgqa_launch_count"]
+            "sgqa_set_wait_limit_ns", "sgqa_check", "sgqa_last_error", "sgqa_version", "sgqa_launch_count"]
 
 
 class SgqaError(RuntimeError):
@@ -74,8 +74,9 @@ _lib.sgqa_forward.argtypes = [_P, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _i64, _
 _lib.sgqa_forward_gated.argtypes = [_P, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp,
                                     _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sgqa_sparse_attn_paged.argtypes = [_P, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _i64, _vp, _vp, _vp,
-                                        _vp, _vp]
+                                        _vp, _vp, _sz, _vp]
 _lib.sgqa_sparse_attn_noalloc.argtypes = [_P, _i64, _i64, _i64, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.sgqa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
 _lib.sgqa_check.argtypes = [_vp]
 _lib.sgqa_last_error.restype = ctypes.c_char_p
 _lib.sgqa_version.restype = ctypes.c_char_p
@@ -171,12 +172,14 @@ def sgqa_forward(p: Params, num_seqs, q_pos0, nq, q, idx_q, idx_w, cache_cap, ca
 
 
 def sgqa_sparse_attn_paged(p: Params, num_seqs, q_pos0, nq, q, k_pool, v_pool, page_table, cache_len, sel,
-                           sel_count, out, gate=None, stream=None):
-    """Decode attention over a paged cache: pools [num_pages * 16, G, D], page_table [S, max_pages] int32."""
-    num_pages = k_pool.shape[0] // 16
+                           sel_count, out, gate=None, workspace=None, stream=None):
+    """Attention over a paged cache: pools [num_pages, G, 16, D], page_table [S, max_pages] int32;
+    a workspace only for calls of more than 32 queries per sequence."""
+    num_pages = k_pool.shape[0]
     _ok(_lib.sgqa_sparse_attn_paged(ctypes.byref(p.c()), num_seqs, q_pos0, nq, _ptr(q), _ptr(k_pool), _ptr(v_pool),
                                     num_pages, _ptr(page_table), page_table.shape[1], cache_len, _ptr(sel),
-                                    _ptr(sel_count), _ptr(gate), _ptr(out), _stream(stream)))
+                                    _ptr(sel_count), _ptr(gate), _ptr(out), _ptr(workspace),
+                                    workspace.numel() if workspace is not None else 0, _stream(stream)))
 
 
 def sgqa_sparse_attn_noalloc(p: Params, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k_cache, v_cache, sel,
@@ -186,6 +189,11 @@ def sgqa_sparse_attn_noalloc(p: Params, num_seqs, q_pos0, nq, q, cache_cap, cach
     _ok(_lib.sgqa_sparse_attn_noalloc(ctypes.byref(p.c()), num_seqs, q_pos0, nq, _ptr(q), cache_cap, cache_len,
                                       _ptr(k_cache), _ptr(v_cache), _ptr(sel), _ptr(sel_count), _ptr(out),
                                       _stream(stream)))
+
+
+def sgqa_set_wait_limit_ns(ns: int):
+    """Time limit of the kernels' pipeline waits on the current device (0: the default, 2 s)."""
+    _ok(_lib.sgqa_set_wait_limit_ns(int(ns)))
 
 
 def sgqa_check(stream=None):

@@ -43,7 +43,7 @@ constexpr int kPlanThreads = 512;
 // shared memory; the masks go out with 8-byte stores.
 __global__ void __launch_bounds__(kPlanThreads)
 attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ sel_count,
-                 int64_t nq, int G, int k, int nwords, int32_t* __restrict__ plan_ids,
+                 int64_t nq, int G, int k, int nwords, int64_t q_pos0, int B, int32_t* __restrict__ plan_ids,
                  uint8_t* __restrict__ plan_mask, int32_t* __restrict__ plan_count) {
   // [nwords] bitmap, [nwords] prefix, then the union's masks (8k bytes)
   extern __shared__ __align__(16) uint32_t sm_words[];
@@ -63,13 +63,16 @@ attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ se
   __syncthreads();
   const int nq_here = static_cast<int>(nq - qb * 8 < 8 ? nq - qb * 8 : 8);
   const int64_t row0 = (seq * nq + qb * 8) * G + g;
-  const int nbits = nwords * 32;
+  // a query at position t may only have selected blocks below floor(t / B):
+  // other ids break the call's contract, are reported and left out
+  const int64_t lim0 = q_pos0 + qb * 8;
   for (int q = 0; q < nq_here; ++q) {
     const int64_t row = row0 + static_cast<int64_t>(q) * G;
     const int cnt = min(max(sel_count[row], 0), k);
+    const int64_t lim = (lim0 + q) / B;
     for (int j = tid; j < cnt; j += kPlanThreads) {
       const int id = sel[row * k + j];
-      if (id >= 0 && id < nbits) atomicOr(&bm[id >> 5], 1u << (id & 31));
+      if (id >= 0 && id < lim) atomicOr(&bm[id >> 5], 1u << (id & 31));
       else report(kDevBounds);
     }
   }
@@ -109,9 +112,10 @@ attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ se
   for (int q = 0; q < nq_here; ++q) {
     const int64_t row = row0 + static_cast<int64_t>(q) * G;
     const int cnt = min(max(sel_count[row], 0), k);
+    const int64_t lim = (lim0 + q) / B;
     for (int j = tid; j < cnt; j += kPlanThreads) {
       const int id = sel[row * k + j];
-      if (id < 0 || id >= nbits) continue;
+      if (id < 0 || id >= lim) continue;
       const int pos = pre[id >> 5] + __popc(bm[id >> 5] & ((1u << (id & 31)) - 1u));
       atomicOr(&msk[pos >> 2], (1u << q) << (8 * (pos & 3)));
     }
@@ -131,7 +135,7 @@ constexpr int kPlanSortThreads = 1024;
 // id range is too wide for a shared-memory bitmap (B = 1 at very long contexts).
 __global__ void __launch_bounds__(kPlanSortThreads)
 attn_plan_sort_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ sel_count,
-                 int64_t nq, int G, int k, int pow2, int32_t* __restrict__ plan_ids,
+                 int64_t nq, int G, int k, int pow2, int64_t q_pos0, int B, int32_t* __restrict__ plan_ids,
                  uint8_t* __restrict__ plan_mask, int32_t* __restrict__ plan_count) {
   extern __shared__ uint32_t sk[];  // pow2 keys
   __shared__ int warp_sums[32];
@@ -148,8 +152,15 @@ attn_plan_sort_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict
     if (i >= nq) break;
     const int64_t row = (seq * nq + i) * G + g;
     const int cnt = min(max(sel_count[row], 0), k);
-    for (int j = tid; j < cnt; j += kPlanSortThreads)
-      sk[q * k + j] = (static_cast<uint32_t>(sel[row * k + j]) << 3) | q;
+    const int64_t lim = (q_pos0 + i) / B;
+    for (int j = tid; j < cnt; j += kPlanSortThreads) {
+      const int id = sel[row * k + j];
+      if (id >= 0 && id < lim) {
+        sk[q * k + j] = (static_cast<uint32_t>(id) << 3) | q;
+      } else {
+        report(kDevBounds);  // outside the query's candidates: left out
+      }
+    }
   }
   __syncthreads();
   for (int size = 2; size <= pow2; size <<= 1) {

@@ -69,13 +69,19 @@ struct __align__(1024) AttnTcSmem {
 // SKIP_PAIRS: skip the exponentials of block pairs that no row of a warp
 // attends (pays when selections cover a small part of the context); otherwise
 // all 64 exponentials of a tile run as one branch-free block.
-template <bool SKIP_PAIRS>
+// PAGED: the K/V live in a pool of 16-token pages [pages, G, 16, D] reached
+// through page_table [S, max_pages] (the tensor maps cover the pool); a
+// block's copy starts at (row 0 or 8 of its page, page).  Otherwise the maps
+// cover the contiguous caches [S, cap, G, D] and a copy starts at (token row,
+// sequence).
+template <bool SKIP_PAIRS, bool PAGED>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUtensorMap kmap,
                const __grid_constant__ CUtensorMap vmap, const int32_t* __restrict__ plan_ids,
                const uint8_t* __restrict__ plan_mask, const int32_t* __restrict__ plan_count,
                __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ gate, int64_t nq, int G,
-               int k, int64_t q_pos0, float scale_log2) {
+               int k, int64_t q_pos0, float scale_log2, const int32_t* __restrict__ page_table, int64_t max_pages,
+               int64_t num_pages) {
   extern __shared__ uint8_t smem_raw[];
   AttnTcSmem& sm = *reinterpret_cast<AttnTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                   ~static_cast<uintptr_t>(1023));
@@ -97,6 +103,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
   const int64_t t_last = q_pos0 + min(nq, qb * 8 + 8) - 1;
   const int64_t c0 = 8 * (t_first / 8);  // first token of the current segment
   volatile int* abort = &sm.abort;
+  const uint32_t wlim = tc::wait_limit();  // pipeline wait limit of this launch
 
   auto bar = [](uint64_t& b) { return smem_u32(&b); };
   if (threadIdx.x == 0) {
@@ -129,6 +136,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
   const uint32_t tS0 = tmem + 192;    // S buffers at [192, 256), [256, 320)
   const uint32_t tP0 = tmem + 320;    // P buffers at [320, 352), [352, 384)
   const uint32_t tQ = tmem + 384;     // Q at [384, 480)
+  int issued = 0;                     // producers: tiles whose copies this warp issued
 
   if (warp == 0 || warp == 10) {
     // ------------------------------------------------------------ producers
@@ -138,54 +146,60 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     const int nst = is_k ? kTcStages : kTcVStages;
     if (tc::elect_one()) tc::prefetch_tmap(is_k ? &kmap : &vmap);
     __syncwarp();
-    // Block ids of the union, one per lane in batches of four tiles (32 ids),
-    // loaded a whole batch ahead: the id fetch (an L2 round trip) never sits
-    // between two tiles' copies.  Lane 8 t + e holds block e of tile 4 b + t.
+    // Copy rows of the union's blocks, one per lane in batches of four tiles
+    // (32 blocks), loaded a whole batch ahead: the id fetch (an L2 round trip,
+    // plus the page-table read of a paged pool) never sits between two tiles'
+    // copies.  Lane 8 t + e holds block e of tile 4 b + t.  A row is a token
+    // row, or page * 16 + row within the page; negative: a zero-filled box.
+    auto page_row = [&](int64_t tok) -> int32_t {  // paged pool: the row of token tok
+      const int32_t pg = page_table[seq * max_pages + (tok >> 4)];
+      if (pg < 0 || pg >= num_pages) {
+        report(kDevBounds);
+        return -64;
+      }
+      return pg * 16 + static_cast<int32_t>(tok & 15);
+    };
     auto load_batch = [&](int bt) -> int32_t {
       const int idx = 32 * bt + lane;
-      return idx < U ? uid[idx] : -1;
+      const int32_t id = idx < U ? uid[idx] : -1;
+      if (id < 0) return -64;
+      return PAGED ? page_row(static_cast<int64_t>(id) * 8) : id * 8;
     };
-    int32_t ids_cur = load_batch(0), ids_next = n_union_tiles > 4 ? load_batch(1) : -1;
-    int issued = 0;
+    int32_t ids_cur = load_batch(0), ids_next = n_union_tiles > 4 ? load_batch(1) : -64;
+    // the current-block tile: the current block and, when the unit spans two blocks, the next
+    int32_t cur_rows = -64;
+    if (lane < 2 && (lane == 0 || c0 + 8 <= t_last))
+      cur_rows = PAGED ? page_row(c0 + 8 * lane) : static_cast<int32_t>(c0 + 8 * lane);
     for (int j = 0; j < n_tiles; ++j) {
       const int s = j % nst;
       if (j > 0 && (j & 3) == 0) {
         ids_cur = ids_next;
         if (4 * (j / 4 + 1) < n_union_tiles) ids_next = load_batch(j / 4 + 1);
       }
-      // this tile's eight token rows (-64: a zero-filled box)
+      // this tile's eight copy rows (-64: a zero-filled box)
       int32_t rows[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const int32_t id = __shfl_sync(0xffffffffu, ids_cur, 8 * (j & 3) + e);
-        if (j < n_union_tiles)
-          rows[e] = id >= 0 ? id * 8 : -64;
-        else  // the current block and, when the unit spans two blocks, the next
-          rows[e] = (e == 0 || (e == 1 && c0 + 8 <= t_last)) ? static_cast<int32_t>(c0 + 8 * e) : -64;
+        const int32_t r_union = __shfl_sync(0xffffffffu, ids_cur, 8 * (j & 3) + e);
+        const int32_t r_cur = __shfl_sync(0xffffffffu, cur_rows, e & 1);
+        rows[e] = j < n_union_tiles ? r_union : (e < 2 ? r_cur : -64);
       }
       uint64_t* empty = is_k ? &sm.k_empty[s] : &sm.v_empty[s];
       uint64_t* full = is_k ? &sm.k_full[s] : &sm.v_full[s];
-      if (j >= nst && !tc::warp_wait(bar(*empty), ((j / nst) - 1) & 1, abort)) break;
+      if (j >= nst && !tc::warp_wait(bar(*empty), ((j / nst) - 1) & 1, abort, wlim)) break;
       if (tc::elect_one()) {
         tc::mbar_expect_tx(bar(*full), 8 * 3 * 1024);
         const CUtensorMap* map = is_k ? &kmap : &vmap;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const uint32_t dst = is_k ? smem_u32(&sm.k[s][e][0][0]) : smem_u32(&sm.v[s][e][0][0]);
-          tc::tma_load_5d(dst, map, 0, rows[e], 0, g, static_cast<int32_t>(seq), bar(*full));
+          const int32_t c1 = PAGED ? (rows[e] & 15) : rows[e];
+          const int32_t c4 = PAGED ? (rows[e] >> 4) : static_cast<int32_t>(seq);
+          tc::tma_load_5d(dst, map, 0, c1, 0, g, c4, bar(*full));
         }
       }
       __syncwarp();
       issued = j + 1;
-    }
-    if (*abort) {
-      // Let the copies already issued land before the CTA's shared memory goes away.
-      for (int j = issued > nst ? issued - nst : 0; j < issued; ++j) {
-        const uint64_t t1 = globaltimer_ns();
-        uint64_t* full = is_k ? &sm.k_full[j % nst] : &sm.v_full[j % nst];
-        while (!tc::mbar_try(bar(*full), (j / nst) & 1) && globaltimer_ns() - t1 < kWaitLimitNs) {
-        }
-      }
     }
   } else if (warp == 1 || warp == 11) {
     // ------------------------------------------------------------ MMA issuers
@@ -204,12 +218,12 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     const uint64_t dv0 = tc::sdesc_sw128(smem_u32(&sm.v[0][0][0][0]), 1024, 3072);
     bool ok = true;
     if (is_qk) {
-      ok = tc::warp_wait(bar(sm.q_full), 0, abort);
+      ok = tc::warp_wait(bar(sm.q_full), 0, abort, wlim);
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int s = j % kTcStages, b = j % 2;
-        ok = tc::warp_wait(bar(sm.k_full[s]), (j / kTcStages) & 1, abort);
+        ok = tc::warp_wait(bar(sm.k_full[s]), (j / kTcStages) & 1, abort, wlim);
         // S buffer b is free once the softmax of tile j-2 has loaded it
-        if (ok && j >= 2) ok = tc::warp_wait(bar(sm.s_free[b]), ((j / 2) - 1) & 1, abort);
+        if (ok && j >= 2) ok = tc::warp_wait(bar(sm.s_free[b]), ((j / 2) - 1) & 1, abort, wlim);
         if (!ok) break;
         tc::fence_after();
         if (tc::elect_one()) {
@@ -226,8 +240,8 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     } else {
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int s = j % kTcVStages, b = j % 2;
-        ok = tc::warp_wait(bar(sm.v_full[s]), (j / kTcVStages) & 1, abort) &&
-             tc::warp_wait(bar(sm.p_full[b]), (j / 2) & 1, abort);
+        ok = tc::warp_wait(bar(sm.v_full[s]), (j / kTcVStages) & 1, abort, wlim) &&
+             tc::warp_wait(bar(sm.p_full[b]), (j / 2) & 1, abort, wlim);
         if (!ok) break;
         tc::fence_after();
         if (tc::elect_one()) {
@@ -243,15 +257,6 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       if (ok) {
         if (tc::elect_one()) tc::mma_commit(bar(sm.o_final));
         __syncwarp();
-      }
-    }
-    if (!ok) {
-      // Let this warp's MMAs already issued finish before TMEM is released.
-      uint64_t& d = is_qk ? sm.drain : sm.drain_pv;
-      if (tc::elect_one()) tc::mma_commit(bar(d));
-      __syncwarp();
-      const uint64_t t0 = globaltimer_ns();
-      while (!tc::mbar_try(bar(d), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
       }
     }
   } else {
@@ -321,7 +326,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       } else {
         bmask = 3u;
       }
-      ok = ok && tc::mbar_wait(bar(sm.s_full[b]), (j / 2) & 1, abort);
+      ok = ok && tc::mbar_wait(bar(sm.s_full[b]), (j / 2) & 1, abort, wlim);
       tc::fence_after();
       uint32_t sr[64];
       tc::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
@@ -371,7 +376,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       if (j + 1 < n_tiles) asm volatile("bar.arrive %0, 64;" ::"r"(pub_mine) : "memory");
       if (__any_sync(0xffffffffu, need)) {
         // O must hold P(j-1) V(j-1) before it is rescaled
-        ok = ok && tc::mbar_wait(bar(sm.pv_done[(j - 1) % 2]), ((j - 1) / 2) & 1, abort);
+        ok = ok && tc::mbar_wait(bar(sm.pv_done[(j - 1) % 2]), ((j - 1) / 2) & 1, abort, wlim);
         tc::fence_after();
         const float alpha = need ? exp2f(m_prev - m_use) : 1.f;
 #pragma unroll 1
@@ -420,7 +425,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       }
       const float lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       // P buffer b is free once O += P(j-2) V(j-2) has read it
-      if (j >= 2) ok = ok && tc::mbar_wait(bar(sm.pv_done[b]), ((j / 2) - 1) & 1, abort);
+      if (j >= 2) ok = ok && tc::mbar_wait(bar(sm.pv_done[b]), ((j / 2) - 1) & 1, abort, wlim);
       tc::fence_after();
       tc::tmem_st32(tP, pk);
       l += lsum;
@@ -428,7 +433,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       tc::fence_before();
       tc::mbar_arrive(bar(sm.p_full[b]));
     }
-    ok = ok && tc::mbar_wait(bar(sm.o_final), 0, abort);
+    ok = ok && tc::mbar_wait(bar(sm.o_final), 0, abort, wlim);
     // both loops done: the final reference is in mchain; combine the two partial sums
     asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
     const float m_fin = sm.mchain[m];
@@ -457,6 +462,24 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
           }
         }
       }
+    }
+  }
+  // Every role has left its loop, so the abort flag is final.  After a
+  // failed wait, copies and MMAs already issued may still be in flight: the
+  // producers wait for their last ring's worth of copies and each MMA warp for
+  // its own MMAs (full time bound) before shared memory and TMEM are released.
+  __syncthreads();
+  if (sm.abort) {
+    if (warp == 0 || warp == 10) {
+      const bool is_k = warp == 0;
+      const int nst = is_k ? kTcStages : kTcVStages;
+      for (int j = issued > nst ? issued - nst : 0; j < issued; ++j)
+        tc::mbar_drain(bar(is_k ? sm.k_full[j % nst] : sm.v_full[j % nst]), (j / nst) & 1);
+    } else if (warp == 1 || warp == 11) {
+      uint64_t& d = warp == 1 ? sm.drain : sm.drain_pv;
+      if (tc::elect_one()) tc::mma_commit(bar(d));
+      __syncwarp();
+      tc::mbar_drain(bar(d), 0);
     }
   }
   tc::fence_before();
@@ -526,13 +549,17 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
   const int64_t t = q_pos0 + i;
   const int cnt = min(max(sel_count[row], 0), k);
   const int32_t* ids = sel + row * k;
-  const int32_t tseq = page_table != nullptr ? 0 : static_cast<int32_t>(seq);  // a paged pool has no sequence axis
+  // A block's copy coordinates: contiguous caches (token row, sequence); a
+  // paged pool [pages, G, 16, D] (row within its page, page), packed in the
+  // staged row value as page * 16 + row (negative: a zero block)
+  const bool paged = page_table != nullptr;
   const int nblk = cnt + 1;  // selected blocks, then the current block
   const int per = (nblk + nsplit - 1) / nsplit;
   const int b0 = min(nblk, split * per), b1 = min(nblk, b0 + per);
   const int nb = b1 - b0;
   const int64_t cur0 = 8 * (t / 8);
   volatile int* abort = &sm.abort;
+  const uint32_t wlim = tc::wait_limit();  // pipeline wait limit of this launch
   auto bar = [](uint64_t& b) { return smem_u32(&b); };
   if (threadIdx.x == 0) {
     sm.abort = 0;
@@ -542,10 +569,22 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     }
     tc::mbar_fence_init();
   }
-  // stage the block rows (one coalesced read instead of a dependent load per TMA issue)
+  // stage the block rows (one coalesced read instead of a dependent load per TMA issue);
+  // a selected id outside [0, floor(t/8)) breaks the call's contract: it is
+  // reported, read as zeros and masked out (row -64)
+  const int64_t nhist = t / 8;
   for (int b = threadIdx.x; b < nb; b += kDecThreads) {
     const int e = b0 + b;
-    int32_t r = e < cnt ? ids[e] * 8 : static_cast<int32_t>(cur0);  // first token of the block
+    int32_t r = static_cast<int32_t>(cur0);  // first token of the block
+    if (e < cnt) {
+      const int32_t id = ids[e];
+      if (id < 0 || id >= nhist) {
+        report(kDevBounds);
+        sm.rows[b] = -64;
+        continue;
+      }
+      r = id * 8;
+    }
     if (page_table != nullptr) {
       // paged cache: the block's 8 tokens lie in one 16-token page of the pool
       const int32_t pg = page_table[seq * max_pages + (r >> 4)];
@@ -565,6 +604,7 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     for (int x = threadIdx.x; x < kHg * kD / 8; x += kDecThreads)
       *reinterpret_cast<uint4*>(&sm.q[x / (kD / 8)][(x % (kD / 8)) * 8]) = q16[x];
   }
+  int mine_end = 0;  // producer lanes: one past the last block this lane issued
   // per-warp attention state (compute warps)
   WarpAttn st;
 #pragma unroll
@@ -583,32 +623,22 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     // gets a zero block.  kDecIssuers lanes issue consecutive blocks side by
     // side (one thread's TMA issue rate does not keep an SM's share of HBM busy).
     const int nblocks = 2 * ((nb + 1) / 2);
-    int mine_end = 0;  // one past the last block this lane issued
     for (int bg = 0; bg < nblocks; bg += kDecIssuers) {
       const int b = bg + lane;
       bool ok = true;
       if (lane < kDecIssuers && b < nblocks) {
         const int slot = b % kDecSlots;
-        if (b >= kDecSlots) ok = tc::mbar_wait(bar(sm.empty[slot]), ((b / kDecSlots) - 1) & 1, abort);
+        if (b >= kDecSlots) ok = tc::mbar_wait(bar(sm.empty[slot]), ((b / kDecSlots) - 1) & 1, abort, wlim);
         if (ok) {
           const int32_t r = b < nb ? sm.rows[b] : -64;  // -64: zero-filled tail block
           tc::mbar_expect_tx(bar(sm.full[slot]), 2 * 3 * 1024);
-          tc::tma_load_5d(smem_u32(&sm.kv[slot][0][0]), &kmap, 0, r, 0, g, tseq, bar(sm.full[slot]));
-          tc::tma_load_5d(smem_u32(&sm.kv[slot][1][0]), &vmap, 0, r, 0, g, tseq, bar(sm.full[slot]));
+          const int32_t c1 = paged ? (r & 15) : r, c4 = paged ? (r >> 4) : static_cast<int32_t>(seq);
+          tc::tma_load_5d(smem_u32(&sm.kv[slot][0][0]), &kmap, 0, c1, 0, g, c4, bar(sm.full[slot]));
+          tc::tma_load_5d(smem_u32(&sm.kv[slot][1][0]), &vmap, 0, c1, 0, g, c4, bar(sm.full[slot]));
           mine_end = b + 1;
         }
       }
       if (!__all_sync(0xffffffffu, ok)) break;
-    }
-    if (*abort && lane < kDecIssuers) {
-      // this lane's loads still in flight (at most one ring's worth) land
-      // before the CTA exits (waits bounded)
-      for (int b = lane; b < mine_end; b += kDecIssuers) {
-        if (b < mine_end - kDecSlots) continue;
-        const uint64_t t0 = globaltimer_ns();
-        while (!tc::mbar_try(bar(sm.full[b % kDecSlots]), (b / kDecSlots) & 1) && globaltimer_ns() - t0 < kWaitLimitNs) {
-        }
-      }
     }
   } else {
     const int cw = warp - 1;  // compute warp 0..3
@@ -619,14 +649,14 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     for (int s = cw; s < nsteps; s += 4) {
       const int ba = 2 * s, bb = 2 * s + 1;
       const int sa = ba % kDecSlots, sb2 = bb % kDecSlots;
-      if (!tc::mbar_wait(bar(sm.full[sa]), (ba / kDecSlots) & 1, abort)) break;
-      if (!tc::mbar_wait(bar(sm.full[sb2]), (bb / kDecSlots) & 1, abort)) break;
+      if (!tc::mbar_wait(bar(sm.full[sa]), (ba / kDecSlots) & 1, abort, wlim)) break;
+      if (!tc::mbar_wait(bar(sm.full[sb2]), (bb / kDecSlots) & 1, abort, wlim)) break;
       // token mask: 8 tokens per block; the current block only up to t; zero blocks none
       uint32_t tm = 0;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int b = 2 * s + h;
-        if (b < nb) {
+        if (b < nb && sm.rows[b] >= 0) {  // -64: a zero block (bad id or page), attended by no one
           const int e = b0 + b;
           uint32_t m8 = 0xFFu;
           if (e >= cnt) m8 = (t - cur0 >= 7) ? 0xFFu : ((1u << (t - cur0 + 1)) - 1u);
@@ -714,6 +744,14 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
         tc::mbar_arrive(bar(sm.empty[sb2]));
       }
     }
+  }
+  __syncthreads();
+  // Every role has left its loop, so the abort flag is final.  After a failed
+  // wait, this lane's loads still in flight (at most one ring's worth) land
+  // (full time bound) before the ring's memory is reused below.
+  if (sm.abort && warp == 0 && lane < kDecIssuers) {
+    for (int b = lane; b < mine_end; b += kDecIssuers)
+      if (b >= mine_end - kDecSlots) tc::mbar_drain(bar(sm.full[b % kDecSlots]), (b / kDecSlots) & 1);
   }
   __syncthreads();
   // combine the four compute warps into this split's partial (shared memory

@@ -144,6 +144,132 @@ index_score_kernel(const __nv_bfloat16* __restrict__ idx_q, const float* __restr
   }
 }
 
+// Warp-level exact selection over buf[0, n) (n > k): the k-th largest key
+// theta and, among entries whose key equals theta, the largest id to keep
+// (id_cut), so that {key > theta} + {key == theta, id <= id_cut} is exactly k
+// entries -- every key above the k-th and the smallest ids among its ties.
+// Radix select on the 32-bit order-preserving keys, 8 bits per pass from the
+// top; ties by a second radix select on the (distinct) ids.  The passes start
+// at the highest byte in which the entries differ: the bits above it are
+// common to all of them, so the passes over those would pick them with the
+// count unchanged.
+__device__ __forceinline__ void common_high_bits(uint32_t and_all, uint32_t or_all, uint32_t& prefix,
+                                                 uint32_t& mask, int& shift) {
+  const uint32_t diff = and_all ^ or_all;
+  shift = diff ? (31 - __clz(static_cast<int>(diff))) / 8 * 8 : -8;
+  mask = shift >= 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+  prefix = and_all & mask;
+}
+__device__ __noinline__ void warp_select(const uint2* buf, int n, int k, uint32_t* hist, uint32_t& theta,
+                                         uint32_t& id_cut) {
+  const int lane = threadIdx.x & 31;
+  uint32_t prefix = 0, mask = 0, rem = static_cast<uint32_t>(k);
+  int shift0;
+  {
+    uint32_t a = 0xFFFFFFFFu, o = 0u;
+    for (int i = lane; i < n; i += 32) {
+      a &= buf[i].x;
+      o |= buf[i].x;
+    }
+    a = __reduce_and_sync(0xffffffffu, a);
+    o = __reduce_or_sync(0xffffffffu, o);
+    common_high_bits(a, o, prefix, mask, shift0);
+  }
+  for (int shift = shift0; shift >= 0; shift -= 8) {
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int i = lane; i < n; i += 32) {
+      const uint32_t key = buf[i].x;
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    uint32_t loc[8], sum = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) { loc[q] = hist[255 - (lane * 8 + q)]; sum += loc[q]; }
+    uint32_t inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) { uint32_t y = __shfl_up_sync(0xffffffffu, inc, o); if (lane >= o) inc += y; }
+    const uint32_t before = inc - sum;
+    const bool mine = before < rem && rem <= inc;
+    uint32_t pick = 0, newrem = 0;
+    if (mine) {
+      uint32_t acc = before;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (acc < rem && rem <= acc + loc[q]) { pick = 255 - (lane * 8 + q); newrem = rem - acc; }
+        acc += loc[q];
+      }
+    }
+    const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+    pick = __shfl_sync(0xffffffffu, pick, src);
+    rem = __shfl_sync(0xffffffffu, newrem, src);
+    prefix |= pick << shift;
+    mask |= 255u << shift;
+    __syncwarp();
+  }
+  theta = prefix;
+  int ties = 0;
+  for (int i = lane; i < n; i += 32) ties += buf[i].x == theta;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ties += __shfl_xor_sync(0xffffffffu, ties, o);
+  id_cut = 0xFFFFFFFFu;
+  if (static_cast<uint32_t>(ties) > rem) {
+    uint32_t ipre = 0, imask = 0, irem = rem;
+    int ishift0;
+    {
+      uint32_t a = 0xFFFFFFFFu, o = 0u;
+      for (int i = lane; i < n; i += 32) {
+        const uint2 e = buf[i];
+        if (e.x == theta) {
+          a &= e.y;
+          o |= e.y;
+        }
+      }
+      a = __reduce_and_sync(0xffffffffu, a);
+      o = __reduce_or_sync(0xffffffffu, o);
+      common_high_bits(a, o, ipre, imask, ishift0);
+    }
+    for (int shift = ishift0; shift >= 0; shift -= 8) {
+      for (int b = lane; b < 256; b += 32) hist[b] = 0;
+      __syncwarp();
+      for (int i = lane; i < n; i += 32) {
+        const uint2 e = buf[i];
+        if (e.x == theta && (e.y & imask) == ipre) atomicAdd(&hist[(e.y >> shift) & 255u], 1u);
+      }
+      __syncwarp();
+      uint32_t loc[8], sum = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) { loc[q] = hist[lane * 8 + q]; sum += loc[q]; }
+      uint32_t inc = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) { uint32_t y = __shfl_up_sync(0xffffffffu, inc, o); if (lane >= o) inc += y; }
+      const uint32_t before = inc - sum;
+      const bool mine = before < irem && irem <= inc;
+      uint32_t pick = 0, newrem = 0;
+      if (mine) {
+        uint32_t acc = before;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (acc < irem && irem <= acc + loc[q]) { pick = lane * 8 + q; newrem = irem - acc; }
+          acc += loc[q];
+        }
+      }
+      const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+      pick = __shfl_sync(0xffffffffu, pick, src);
+      irem = __shfl_sync(0xffffffffu, newrem, src);
+      ipre |= pick << shift;
+      imask |= 255u << shift;
+      __syncwarp();
+    }
+    id_cut = ipre;
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ bool kept(uint2 e, uint32_t theta, uint32_t id_cut) {
+  return e.x > theta || (e.x == theta && e.y <= id_cut);
+}
+
 constexpr int kSelThreads = 512;
 
 // Block-wide exclusive scan of one int per thread; returns the total.
@@ -178,11 +304,12 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int& total, int* warp
 // passes read SRAM instead of HBM.
 constexpr int kSelStageMax = 40960;
 
-// The selection of one row by the whole CTA (every thread calls it with the same row).
+// The selection of one row by the whole CTA (every thread calls it with the
+// same row); srow holds the row's scores.
 template <bool STAGE>
-__device__ __forceinline__ void topk_row_radix(int64_t row, const float* __restrict__ scores, int64_t rpad,
-                                               int64_t nq, int G, int64_t q_pos0, int B, int k,
-                                               int32_t* __restrict__ sel, int32_t* __restrict__ sel_count) {
+__device__ __forceinline__ void topk_row_radix_at(int64_t row, const float* __restrict__ srow, int64_t nq, int G,
+                                                  int64_t q_pos0, int B, int k, int32_t* __restrict__ sel,
+                                                  int32_t* __restrict__ sel_count) {
   extern __shared__ float staged_row[];
   __shared__ uint32_t hist[2048];
   __shared__ int warp_sums[32];
@@ -190,7 +317,6 @@ __device__ __forceinline__ void topk_row_radix(int64_t row, const float* __restr
   const int64_t i = (row / G) % nq;
   const int64_t t = q_pos0 + i;
   const int64_t n = t / B;
-  const float* srow = scores + row * rpad;
   int32_t* out = sel + row * k;
   const int tid = threadIdx.x;
   if (STAGE && n > k) {
@@ -268,6 +394,13 @@ __device__ __forceinline__ void topk_row_radix(int64_t row, const float* __restr
   if (tid == 0) sel_count[row] = k;
 }
 
+template <bool STAGE>
+__device__ __forceinline__ void topk_row_radix(int64_t row, const float* __restrict__ scores, int64_t rpad,
+                                               int64_t nq, int G, int64_t q_pos0, int B, int k,
+                                               int32_t* __restrict__ sel, int32_t* __restrict__ sel_count) {
+  topk_row_radix_at<STAGE>(row, scores + row * rpad, nq, G, q_pos0, B, k, sel, sel_count);
+}
+
 // one CTA per row; only_if (optional) restricts the work to flagged rows
 template <bool STAGE>
 __global__ void __launch_bounds__(kSelThreads)
@@ -297,80 +430,144 @@ topk_rows_list_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq
 
 namespace sgqa {
 
-// Decode scores: one CTA per (sequence, 128 candidates) scores that query's
-// four groups at once (B operand = 4 groups x 8 heads = 32 columns, resident in
-// registers), reading the E4M3 store directly; each warp takes 32 candidates.
-constexpr int kDecScoreWarps = 4;
+// Exact E4M3 -> BF16 widening of two codes by integer operations: the
+// hardware conversion to FP16 is exact, and every E4M3 value is an FP16
+// normal (or zero) whose 10-bit mantissa has only its top 3 bits set, so the
+// BF16 pattern is the FP16 one with the exponent rebiased (15 -> 127) and the
+// mantissa shifted to 7 bits.  (Store codes are finite: the merge saturates.)
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2_int(uint16_t v) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v), __NV_E4M3);
+  const uint32_t x = static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+  const uint32_t mag = x & 0x7FFF7FFFu;
+  const uint32_t r = ((mag >> 3) & 0x0FFF0FFFu) + 0x38003800u;
+  return (r & __vcmpne2(mag, 0u)) | (x & 0x80008000u);
+}
 
-__global__ void __launch_bounds__(kDecScoreWarps * 32)
+// Decode scores: one CTA per (sequence and query, 512 candidates) scores the
+// query's four groups at once (B operand = 4 groups x 8 heads = 32 columns,
+// resident in registers), reading the E4M3 store directly.  The MMA's k index
+// is permuted (the same permutation on both operands leaves every dot product
+// unchanged) so that each lane's A fragments for all four k-steps come from
+// one contiguous 16-byte piece of a key row: logical k = 16 s + 8 h + 2 j + e
+// is dimension 16 j + 4 s + 2 h + e (lane j = lane % 4).  A warp's strip of
+// 16 candidates is then two fully used 512-byte runs of the store, and each
+// warp issues the loads of its four strips before any MMA.
+constexpr int kDecScoreThreads = 256;
+constexpr int kDecScoreCand = 512;  // candidates per CTA: 8 warps x 4 strips of 16
+
+__global__ void __launch_bounds__(kDecScoreThreads)
 index_score_decode_kernel(const __nv_bfloat16* __restrict__ idx_q, const float* __restrict__ idx_w,
                           const uint8_t* __restrict__ store, float* __restrict__ scores, int64_t nq,
                           int64_t q_pos0, int B, int64_t rpad, int64_t key_rows) {
-  constexpr int G = 4, H = 8, Di = 64;
+  constexpr int G = 4, H = 8, Di = 64, STRIPS = kDecScoreCand / 16 / (kDecScoreThreads / 32);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int j = lane & 3, rl = lane >> 2;
   const int64_t sq = blockIdx.y;  // seq * nq + i
   const int64_t i = sq % nq, seq = sq / nq;
   const int64_t ncand = (q_pos0 + i) / B;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 128 + 32 * warp;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kDecScoreCand;
   if (c0 >= ncand) return;
-  // B fragments: column n = 8g + head (lane/4 within an n-tile)
-  uint32_t bf[G][4][2];
+  // the key rows of this warp's strips, 16 bytes per lane and row, all in flight
+  const uint8_t* kb = store + seq * key_rows * Di + 16 * j;
+  uint4 ka[STRIPS], kbb[STRIPS];
+#pragma unroll
+  for (int st = 0; st < STRIPS; ++st) {
+    const int64_t ra = c0 + 16 * (warp + (kDecScoreThreads / 32) * st) + rl, rb = ra + 8;
+    ka[st] = ra < key_rows ? __ldg(reinterpret_cast<const uint4*>(kb + ra * Di)) : make_uint4(0u, 0u, 0u, 0u);
+    kbb[st] = rb < key_rows ? __ldg(reinterpret_cast<const uint4*>(kb + rb * Di)) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  // B fragments (column n = head lane / 4 of group g): 16 consecutive query
+  // values 16 j .. 16 j + 15 of that head; k-step s takes pairs 2 s and 2 s + 1
+  uint32_t bf[G][8];
   float wv[G][2];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const __nv_bfloat16* row = idx_q + ((sq * G + g) * H + (lane >> 2)) * Di;
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      const int k0 = 16 * s + 2 * (lane & 3);
-      bf[g][s][0] = *reinterpret_cast<const uint32_t*>(row + k0);
-      bf[g][s][1] = *reinterpret_cast<const uint32_t*>(row + k0 + 8);
-    }
-    const float* wr = idx_w + (sq * G + g) * H + 2 * (lane & 3);
-    wv[g][0] = wr[0];
-    wv[g][1] = wr[1];
+    const uint4* qrow = reinterpret_cast<const uint4*>(idx_q + ((sq * G + g) * H + rl) * Di + 16 * j);
+    const uint4 q0 = __ldg(qrow), q1 = __ldg(qrow + 1);
+    bf[g][0] = q0.x; bf[g][1] = q0.y; bf[g][2] = q0.z; bf[g][3] = q0.w;
+    bf[g][4] = q1.x; bf[g][5] = q1.y; bf[g][6] = q1.z; bf[g][7] = q1.w;
+    const float2 w2 = __ldg(reinterpret_cast<const float2*>(idx_w + (sq * G + g) * H + 2 * j));
+    wv[g][0] = w2.x;
+    wv[g][1] = w2.y;
   }
-  const uint8_t* kb = store + seq * key_rows * Di;
 #pragma unroll
-  for (int strip = 0; strip < 2; ++strip) {
-    const int64_t r0 = c0 + 16 * strip;
-    const int64_t ra_row = r0 + (lane >> 2), rb_row = ra_row + 8;
-    const bool oka = ra_row < key_rows, okb = rb_row < key_rows;
-    const uint8_t* ra = kb + ra_row * Di + 2 * (lane & 3);
-    const uint8_t* rb = kb + rb_row * Di + 2 * (lane & 3);
-    uint32_t af[4][4];
+  for (int st = 0; st < STRIPS; ++st) {
+    const int64_t ra = c0 + 16 * (warp + (kDecScoreThreads / 32) * st) + rl, rb = ra + 8;
+    // A fragments: pair m of the lane's 16 codes = dimensions 16 j + 2 m, + 1
+    uint32_t pa[8], pb[8];
+    const uint32_t wa[4] = {ka[st].x, ka[st].y, ka[st].z, ka[st].w};
+    const uint32_t wb[4] = {kbb[st].x, kbb[st].y, kbb[st].z, kbb[st].w};
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      af[s][0] = oka ? e4m3x2_to_bf16x2(*reinterpret_cast<const uint16_t*>(ra + 16 * s)) : 0u;
-      af[s][1] = okb ? e4m3x2_to_bf16x2(*reinterpret_cast<const uint16_t*>(rb + 16 * s)) : 0u;
-      af[s][2] = oka ? e4m3x2_to_bf16x2(*reinterpret_cast<const uint16_t*>(ra + 16 * s + 8)) : 0u;
-      af[s][3] = okb ? e4m3x2_to_bf16x2(*reinterpret_cast<const uint16_t*>(rb + 16 * s + 8)) : 0u;
+    for (int m = 0; m < 4; ++m) {
+      pa[2 * m] = e4m3x2_to_bf16x2_int(static_cast<uint16_t>(wa[m] & 0xFFFFu));
+      pa[2 * m + 1] = e4m3x2_to_bf16x2_int(static_cast<uint16_t>(wa[m] >> 16));
+      pb[2 * m] = e4m3x2_to_bf16x2_int(static_cast<uint16_t>(wb[m] & 0xFFFFu));
+      pb[2 * m + 1] = e4m3x2_to_bf16x2_int(static_cast<uint16_t>(wb[m] >> 16));
     }
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int s = 0; s < 4; ++s) mma_bf16_16816(acc, af[s], bf[g][s][0], bf[g][s][1]);
-      float pa = wv[g][0] * fmaxf(acc[0], 0.f) + wv[g][1] * fmaxf(acc[1], 0.f);
-      float pb = wv[g][0] * fmaxf(acc[2], 0.f) + wv[g][1] * fmaxf(acc[3], 0.f);
-      pa += __shfl_xor_sync(0xffffffffu, pa, 1);
-      pa += __shfl_xor_sync(0xffffffffu, pa, 2);
-      pb += __shfl_xor_sync(0xffffffffu, pb, 1);
-      pb += __shfl_xor_sync(0xffffffffu, pb, 2);
-      if ((lane & 3) == 0) {
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint32_t af[4] = {pa[2 * ks], pb[2 * ks], pa[2 * ks + 1], pb[2 * ks + 1]};
+        mma_bf16_16816(acc, af, bf[g][2 * ks], bf[g][2 * ks + 1]);
+      }
+      float sa = wv[g][0] * fmaxf(acc[0], 0.f) + wv[g][1] * fmaxf(acc[1], 0.f);
+      float sb = wv[g][0] * fmaxf(acc[2], 0.f) + wv[g][1] * fmaxf(acc[3], 0.f);
+      sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+      sa += __shfl_xor_sync(0xffffffffu, sa, 2);
+      sb += __shfl_xor_sync(0xffffffffu, sb, 1);
+      sb += __shfl_xor_sync(0xffffffffu, sb, 2);
+      if (j == 0) {
         float* srow = scores + (sq * G + g) * rpad;
-        srow[ra_row] = pa;
-        srow[rb_row] = pb;
+        if (ra < rpad) srow[ra] = sa;
+        if (rb < rpad) srow[rb] = sb;
       }
     }
   }
 }
 
 // Exact top-k of rows of at most 32768 scores: 1024 threads hold 32 keys each
-// in registers; four 8-bit radix passes with a private histogram per warp
-// (no cross-warp contention on the few bins that clustered keys share); the
-// kept ids are marked in a bitmap and read out in id order (ascending).
+// in registers.  Fast path: one linear histogram of 2048 bins between the
+// row's smallest and largest score finds the bin holding the k-th largest;
+// every score of a better bin is kept, and the boundary bin's entries (a few
+// dozen on typical rows) are ranked exactly -- score, then smaller id -- by
+// one warp.  The bin function rounds monotonically, so a better score never
+// lands in a worse bin.  A boundary bin larger than its buffer (massive near
+// or exact ties) falls back to four 8-bit radix passes over the keys, with a
+// private histogram per warp, and ties taken in id order.  The kept ids are
+// marked in a bitmap and read out in id order (ascending).
 constexpr int kRegSelThreads = 1024;
 constexpr int kRegSelPer = 32;
+constexpr int kRegSelBins = 2048;
+constexpr int kRegSelBnd = 1024;  // boundary entries the fast path ranks
+
+// The kept bits (thread t owns word t) read out in id order by the whole CTA.
+__device__ __forceinline__ void topk_reg_readout(const uint32_t* keep_bits, int* sums, int tid, int lane, int warp,
+                                                 int k, int32_t* __restrict__ out, int32_t* __restrict__ sel_count,
+                                                 int64_t row) {
+  const uint32_t kb = keep_bits[tid];
+  const uint32_t cnt = __popc(kb);
+  uint32_t x = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) { uint32_t y = __shfl_up_sync(0xffffffffu, x, o); if (lane >= o) x += y; }
+  __syncthreads();
+  if (lane == 31) sums[warp] = static_cast<int>(x);
+  __syncthreads();
+  uint32_t pos = x - cnt;
+  for (int w = 0; w < warp; ++w) pos += sums[w];
+  uint32_t b = kb;
+  while (b) {
+    const int t = __ffs(b) - 1;
+    b &= b - 1;
+    if (pos < static_cast<uint32_t>(k)) out[pos] = tid * 32 + t;
+    ++pos;
+  }
+  if (tid == kRegSelThreads - 1) {
+    sel_count[row] = k;
+    if (pos != static_cast<uint32_t>(k)) report(kDevBounds);
+  }
+}
 
 __global__ void __launch_bounds__(kRegSelThreads)
 topk_rows_reg_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int G, int64_t q_pos0, int B,
@@ -399,6 +596,98 @@ topk_rows_reg_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq,
   }
   keep_bits[tid] = 0;
   tie_bits[tid] = 0;
+  // ---- fast path: linear histogram between the row's extreme scores
+  __shared__ float fmx[32], fmn[32];
+  __shared__ uint32_t s_cnt, s_nb;
+  uint32_t* hall = &wh[0][0];  // 4 copies x 2048 bins, then reused for the boundary list
+  {
+    float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+    for (int u = 0; u < kRegSelPer; ++u) {
+      if (tid + u * kRegSelThreads < n) {
+        const float v = key_score(key[u]);
+        mx = fmaxf(mx, v);
+        mn = fminf(mn, v);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    }
+    if (lane == 0) {
+      fmx[warp] = mx;
+      fmn[warp] = mn;
+    }
+    for (int b = tid; b < 4 * kRegSelBins; b += kRegSelThreads) hall[b] = 0u;
+    if (tid == 0) s_nb = 0;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < 32; ++w) {
+      mx = fmaxf(mx, fmx[w]);
+      mn = fminf(mn, fmn[w]);
+    }
+    const float width = mx - mn;
+    const float scale = width > 0.f ? (kRegSelBins - 0.5f) / width : 0.f;
+    // bins best first; both steps round monotonically
+    auto bin_of = [&](uint32_t kk) -> int {
+      return min(static_cast<int>(__fmul_rn(__fsub_rn(mx, key_score(kk)), scale)), kRegSelBins - 1);
+    };
+    uint32_t* myh = hall + (warp & 3) * kRegSelBins;
+#pragma unroll
+    for (int u = 0; u < kRegSelPer; ++u)
+      if (tid + u * kRegSelThreads < n) atomicAdd(&myh[bin_of(key[u])], 1u);
+    __syncthreads();
+    // thread t owns bins 2t, 2t + 1: the bin in which the running count reaches k
+    const uint32_t c0 = hall[2 * tid] + hall[kRegSelBins + 2 * tid] + hall[2 * kRegSelBins + 2 * tid] +
+                        hall[3 * kRegSelBins + 2 * tid];
+    const uint32_t c1 = hall[2 * tid + 1] + hall[kRegSelBins + 2 * tid + 1] + hall[2 * kRegSelBins + 2 * tid + 1] +
+                        hall[3 * kRegSelBins + 2 * tid + 1];
+    uint32_t x = c0 + c1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) { uint32_t y = __shfl_up_sync(0xffffffffu, x, o); if (lane >= o) x += y; }
+    if (lane == 31) sums[warp] = static_cast<int>(x);
+    __syncthreads();
+    uint32_t before = x - c0 - c1;
+    for (int w = 0; w < warp; ++w) before += sums[w];
+    const uint32_t kk = static_cast<uint32_t>(k);
+    if (before < kk && kk <= before + c0) {
+      s_pick = 2 * tid; s_rem = kk - before; s_cnt = c0;
+    } else if (before + c0 < kk && kk <= before + c0 + c1) {
+      s_pick = 2 * tid + 1; s_rem = kk - before - c0; s_cnt = c1;
+    }
+    __syncthreads();
+    if (s_cnt <= kRegSelBnd) {
+      const int bstar = static_cast<int>(s_pick);
+      const uint32_t rem = s_rem;
+      uint2* bnd = reinterpret_cast<uint2*>(hall);  // [kRegSelBnd], the histogram is consumed
+      uint32_t* scratch = hall + 2 * kRegSelBnd;     // warp_select's 256 counters
+#pragma unroll
+      for (int u = 0; u < kRegSelPer; ++u) {
+        const int j = tid + u * kRegSelThreads;
+        if (j < n) {
+          const int b = bin_of(key[u]);
+          if (b < bstar) atomicOr(&keep_bits[j >> 5], 1u << (j & 31));
+          else if (b == bstar) bnd[atomicAdd(&s_nb, 1u)] = make_uint2(key[u], static_cast<uint32_t>(j));
+        }
+      }
+      __syncthreads();
+      if (warp == 0) {
+        const uint32_t nb = s_nb;
+        uint32_t theta = 0, id_cut = 0xFFFFFFFFu;
+        if (nb > rem) warp_select(bnd, static_cast<int>(nb), static_cast<int>(rem), scratch, theta, id_cut);
+        for (uint32_t c = lane; c < nb; c += 32) {
+          const uint2 e = bnd[c];
+          if (nb <= rem || kept(e, theta, id_cut)) atomicOr(&keep_bits[e.y >> 5], 1u << (e.y & 31));
+        }
+      }
+      __syncthreads();
+      topk_reg_readout(keep_bits, sums, tid, lane, warp, k, out, sel_count, row);
+      return;
+    }
+    __syncthreads();
+  }
+  // ---- fallback: radix passes (every thread takes this branch together)
   uint32_t prefix = 0, mask = 0, rem = static_cast<uint32_t>(k);
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int b = lane; b < 256; b += 32) wh[warp][b] = 0;
@@ -461,28 +750,7 @@ topk_rows_reg_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq,
     keep_bits[tid] |= take;
     __syncthreads();
   }
-  // read out in id order
-  const uint32_t kb = keep_bits[tid];
-  const uint32_t cnt = __popc(kb);
-  uint32_t x = cnt;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) { uint32_t y = __shfl_up_sync(0xffffffffu, x, o); if (lane >= o) x += y; }
-  __syncthreads();
-  if (lane == 31) sums[warp] = static_cast<int>(x);
-  __syncthreads();
-  uint32_t pos = x - cnt;
-  for (int w = 0; w < warp; ++w) pos += sums[w];
-  uint32_t b = kb;
-  while (b) {
-    const int t = __ffs(b) - 1;
-    b &= b - 1;
-    if (pos < static_cast<uint32_t>(k)) out[pos] = tid * 32 + t;
-    ++pos;
-  }
-  if (tid == kRegSelThreads - 1) {
-    sel_count[row] = k;
-    if (pos != static_cast<uint32_t>(k)) report(kDevBounds);
-  }
+  topk_reg_readout(keep_bits, sums, tid, lane, warp, k, out, sel_count, row);
 }
 
 }  // namespace sgqa

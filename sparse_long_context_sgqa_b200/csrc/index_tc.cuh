@@ -14,6 +14,7 @@
 // (index_score_tc_kernel).  The select kernels below take its output.
 #pragma once
 #include "common.cuh"
+#include "index_rows.cuh"
 #include "tc.cuh"
 
 namespace sgqa {
@@ -34,149 +35,26 @@ struct __align__(1024) IndexTcSmem {
   int abort;
 };
 
-// Warp-level exact selection over buf[0, n) (n > k): the k-th largest key
-// theta and, among entries whose key equals theta, the largest id to keep
-// (id_cut), so that {key > theta} + {key == theta, id <= id_cut} is exactly k
-// entries -- every key above the k-th and the smallest ids among its ties.
-// Radix select on the 32-bit order-preserving keys, 8 bits per pass from the
-// top; ties by a second radix select on the (distinct) ids.  The passes start
-// at the highest byte in which the entries differ: the bits above it are
-// common to all of them, so the passes over those would pick them with the
-// count unchanged.
-__device__ __forceinline__ void common_high_bits(uint32_t and_all, uint32_t or_all, uint32_t& prefix,
-                                                 uint32_t& mask, int& shift) {
-  const uint32_t diff = and_all ^ or_all;
-  shift = diff ? (31 - __clz(static_cast<int>(diff))) / 8 * 8 : -8;
-  mask = shift >= 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
-  prefix = and_all & mask;
-}
-__device__ __noinline__ void warp_select(const uint2* buf, int n, int k, uint32_t* hist, uint32_t& theta,
-                                         uint32_t& id_cut) {
-  const int lane = threadIdx.x & 31;
-  uint32_t prefix = 0, mask = 0, rem = static_cast<uint32_t>(k);
-  int shift0;
-  {
-    uint32_t a = 0xFFFFFFFFu, o = 0u;
-    for (int i = lane; i < n; i += 32) {
-      a &= buf[i].x;
-      o |= buf[i].x;
-    }
-    a = __reduce_and_sync(0xffffffffu, a);
-    o = __reduce_or_sync(0xffffffffu, o);
-    common_high_bits(a, o, prefix, mask, shift0);
-  }
-  for (int shift = shift0; shift >= 0; shift -= 8) {
-    for (int b = lane; b < 256; b += 32) hist[b] = 0;
-    __syncwarp();
-    for (int i = lane; i < n; i += 32) {
-      const uint32_t key = buf[i].x;
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
-    }
-    __syncwarp();
-    uint32_t loc[8], sum = 0;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) { loc[q] = hist[255 - (lane * 8 + q)]; sum += loc[q]; }
-    uint32_t inc = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) { uint32_t y = __shfl_up_sync(0xffffffffu, inc, o); if (lane >= o) inc += y; }
-    const uint32_t before = inc - sum;
-    const bool mine = before < rem && rem <= inc;
-    uint32_t pick = 0, newrem = 0;
-    if (mine) {
-      uint32_t acc = before;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (acc < rem && rem <= acc + loc[q]) { pick = 255 - (lane * 8 + q); newrem = rem - acc; }
-        acc += loc[q];
-      }
-    }
-    const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
-    pick = __shfl_sync(0xffffffffu, pick, src);
-    rem = __shfl_sync(0xffffffffu, newrem, src);
-    prefix |= pick << shift;
-    mask |= 255u << shift;
-    __syncwarp();
-  }
-  theta = prefix;
-  int ties = 0;
-  for (int i = lane; i < n; i += 32) ties += buf[i].x == theta;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ties += __shfl_xor_sync(0xffffffffu, ties, o);
-  id_cut = 0xFFFFFFFFu;
-  if (static_cast<uint32_t>(ties) > rem) {
-    uint32_t ipre = 0, imask = 0, irem = rem;
-    int ishift0;
-    {
-      uint32_t a = 0xFFFFFFFFu, o = 0u;
-      for (int i = lane; i < n; i += 32) {
-        const uint2 e = buf[i];
-        if (e.x == theta) {
-          a &= e.y;
-          o |= e.y;
-        }
-      }
-      a = __reduce_and_sync(0xffffffffu, a);
-      o = __reduce_or_sync(0xffffffffu, o);
-      common_high_bits(a, o, ipre, imask, ishift0);
-    }
-    for (int shift = ishift0; shift >= 0; shift -= 8) {
-      for (int b = lane; b < 256; b += 32) hist[b] = 0;
-      __syncwarp();
-      for (int i = lane; i < n; i += 32) {
-        const uint2 e = buf[i];
-        if (e.x == theta && (e.y & imask) == ipre) atomicAdd(&hist[(e.y >> shift) & 255u], 1u);
-      }
-      __syncwarp();
-      uint32_t loc[8], sum = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) { loc[q] = hist[lane * 8 + q]; sum += loc[q]; }
-      uint32_t inc = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) { uint32_t y = __shfl_up_sync(0xffffffffu, inc, o); if (lane >= o) inc += y; }
-      const uint32_t before = inc - sum;
-      const bool mine = before < irem && irem <= inc;
-      uint32_t pick = 0, newrem = 0;
-      if (mine) {
-        uint32_t acc = before;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (acc < irem && irem <= acc + loc[q]) { pick = lane * 8 + q; newrem = irem - acc; }
-          acc += loc[q];
-        }
-      }
-      const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
-      pick = __shfl_sync(0xffffffffu, pick, src);
-      irem = __shfl_sync(0xffffffffu, newrem, src);
-      ipre |= pick << shift;
-      imask |= 255u << shift;
-      __syncwarp();
-    }
-    id_cut = ipre;
-  }
-  __syncwarp();
-}
-
-__device__ __forceinline__ bool kept(uint2 e, uint32_t theta, uint32_t id_cut) {
-  return e.x > theta || (e.x == theta && e.y <= id_cut);
-}
 
 // Indexer scores I[t, g, r] on the tensor cores (one CTA = 256 (query, head)
 // columns of one group, all candidates in tiles of 128), with one of three
 // epilogues:
 //   kScoreRows    every score as FP32 rows [row, rpad] (one 128-byte store per
 //                 warp and query); a top-k kernel then selects from the rows;
-//   kScoreSample  only every kSampleStride-th candidate tile, compacted into
-//                 rows [row, ld] (for the per-row threshold estimate);
+//   kScoreSample  only every o.samp-th candidate tile, compacted into rows
+//                 [row, ld] (for the per-row threshold estimate);
 //   kScoreFilter  every score, but only those at or above the row's threshold
 //                 are kept, as (order-preserving key, block id) pairs in the
 //                 row's staging list; the row's count (which may exceed the
 //                 list's capacity) is written at the end.  A CTA owns its rows,
 //                 so the counters live in shared memory.
 constexpr int kScoreRows = 0, kScoreSample = 1, kScoreFilter = 2;
-constexpr int kSampleStride = 16;
+constexpr int kSampleStride = 16;   // the smallest sample stride (in candidate tiles)
+constexpr int kSampleTilesMax = 64; // sampled tiles per row: at most 8192 samples
 struct ScoreOut {
   float* scores;            // kScoreRows: [rows, ld] = [rows, rpad]; kScoreSample: [rows, ld]
   int64_t ld;
+  int samp;                 // kScoreSample: every samp-th candidate tile is scored
   const float* thr;         // kScoreFilter: per-row threshold
   uint2* staging;           // kScoreFilter: [rows, 4, cap] (key, id), one list per TMEM lane quadrant
   int32_t* staged;          // kScoreFilter: [rows, 4] scores at or above the threshold per list
@@ -204,9 +82,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
   const int64_t ncand_max = (q_pos0 + q0 + nq_here - 1) / B;
   const int n_tiles = static_cast<int>((ncand_max + kIdxCand - 1) / kIdxCand);
   // tiles this launch computes (the sample takes every kSampleStride-th) and the tile behind loop index c
-  const int n_loop = MODE == kScoreSample ? (n_tiles + kSampleStride - 1) / kSampleStride : n_tiles;
-  auto tile_of = [](int c) { return MODE == kScoreSample ? c * kSampleStride : c; };
+  const int samp = o.samp;
+  const int n_loop = MODE == kScoreSample ? (n_tiles + samp - 1) / samp : n_tiles;
+  auto tile_of = [samp](int c) { return MODE == kScoreSample ? c * samp : c; };
   volatile int* abort = &sm.abort;
+  const uint32_t wlim = tc::wait_limit();  // pipeline wait limit of this launch
   auto bar = [](uint64_t& b) { return smem_u32(&b); };
   if (threadIdx.x == 0) {
     sm.abort = 0;
@@ -237,6 +117,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
   __syncthreads();
   tc::fence_after();
   const uint32_t tmem = sm.tmem;
+  int issued = 0;  // producer: key tiles whose copies were issued
   if (n_tiles > 0) {
     if (warp == 0) {
       // producer: queries once, then the candidate tiles through the ring (converged warp, one elected issuer)
@@ -247,10 +128,9 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
         tc::tma_load_4d(smem_u32(&sm.b[0]), &qmap, 0, 0, g, static_cast<int32_t>(seq * nq + q0), bar(sm.b_full));
       }
       __syncwarp();
-      int issued = 0;
       for (int c = 0; c < n_loop; ++c) {
         const int s = c % kIdxStages;
-        if (c >= kIdxStages && !tc::warp_wait(bar(sm.a_empty[s]), ((c / kIdxStages) - 1) & 1, abort)) break;
+        if (c >= kIdxStages && !tc::warp_wait(bar(sm.a_empty[s]), ((c / kIdxStages) - 1) & 1, abort, wlim)) break;
         if (tc::elect_one()) {
           tc::mbar_expect_tx(bar(sm.a_full[s]), kIdxCand * 128);
           tc::tma_load_2d(smem_u32(&sm.a[s][0]), &keymap, 0,
@@ -260,28 +140,17 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
         __syncwarp();
         issued = c + 1;
       }
-      if (*abort) {
-        const uint64_t t0 = globaltimer_ns();
-        while (!tc::mbar_try(bar(sm.b_full), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-        }
-        for (int c = issued > kIdxStages ? issued - kIdxStages : 0; c < issued; ++c) {
-          const uint64_t t1 = globaltimer_ns();
-          while (!tc::mbar_try(bar(sm.a_full[c % kIdxStages]), (c / kIdxStages) & 1) &&
-                 globaltimer_ns() - t1 < kWaitLimitNs) {
-          }
-        }
-      }
     } else if (warp == 1) {
       // MMA issuer (converged warp, one elected issuer per tile)
       const uint32_t idesc = tc::idesc_bf16(kIdxCand, kIdxCols, false);
       const uint64_t da0 = tc::sdesc_sw128(smem_u32(&sm.a[0][0]), 16, 1024);
       const uint64_t db0 = tc::sdesc_sw128(smem_u32(&sm.b[0]), 16, 1024);
       constexpr uint32_t kStageUnits = kIdxCand * 128 / 16;  // one key stage in 16-byte units
-      bool ok = tc::warp_wait(bar(sm.b_full), 0, abort);
+      bool ok = tc::warp_wait(bar(sm.b_full), 0, abort, wlim);
       for (int c = 0; ok && c < n_loop; ++c) {
         const int s = c % kIdxStages, ab = c & 1;
-        if (!tc::warp_wait(bar(sm.a_full[s]), (c / kIdxStages) & 1, abort)) { ok = false; break; }
-        if (c >= 2 && !tc::warp_wait(bar(sm.acc_empty[ab]), ((c >> 1) - 1) & 1, abort)) { ok = false; break; }
+        if (!tc::warp_wait(bar(sm.a_full[s]), (c / kIdxStages) & 1, abort, wlim)) { ok = false; break; }
+        if (c >= 2 && !tc::warp_wait(bar(sm.acc_empty[ab]), ((c >> 1) - 1) & 1, abort, wlim)) { ok = false; break; }
         tc::fence_after();
         if (tc::elect_one()) {
 #pragma unroll
@@ -291,13 +160,6 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
           tc::mma_commit(bar(sm.acc_full[ab]));
         }
         __syncwarp();
-      }
-      if (!ok) {
-        if (tc::elect_one()) tc::mma_commit(bar(sm.drain));
-        __syncwarp();
-        const uint64_t t0 = globaltimer_ns();
-        while (!tc::mbar_try(bar(sm.drain), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-        }
       }
     } else {
       // epilogue: sixteen warps, four per TMEM lane quadrant (= 32 candidates),
@@ -328,7 +190,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
       float* const sbase = MODE == kScoreFilter ? nullptr : o.scores + row0 * o.ld + m;
       for (int c = 0; c < n_loop; ++c) {
         const int ab = c & 1;
-        if (!tc::mbar_wait(bar(sm.acc_full[ab]), (c >> 1) & 1, abort)) break;
+        if (!tc::mbar_wait(bar(sm.acc_full[ab]), (c >> 1) & 1, abort, wlim)) break;
         tc::fence_after();
         const int64_t r = static_cast<int64_t>(tile_of(c)) * kIdxCand + m;  // candidate block id
         const bool tail = static_cast<int64_t>(tile_of(c) + 1) * kIdxCand > ncand_min;
@@ -406,6 +268,22 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
     }
   } else if (MODE == kScoreFilter && warp >= 2 && warp < 6) {
     for (int qs = lane; qs < nq_here; qs += 32) o.staged[((seq * nq + q0 + qs) * G + g) * 4 + (warp & 3)] = 0;
+  }
+  // Every role has left its loop, so the abort flag is final.  After a
+  // failed wait, the producer lets its copies still in flight land and the
+  // MMA warp waits for its own MMAs (full time bound) before shared memory and
+  // TMEM are released.
+  __syncthreads();
+  if (sm.abort && n_tiles > 0) {
+    if (warp == 0) {
+      tc::mbar_drain(bar(sm.b_full), 0);
+      for (int c = issued > kIdxStages ? issued - kIdxStages : 0; c < issued; ++c)
+        tc::mbar_drain(bar(sm.a_full[c % kIdxStages]), (c / kIdxStages) & 1);
+    } else if (warp == 1) {
+      if (tc::elect_one()) tc::mma_commit(bar(sm.drain));
+      __syncwarp();
+      tc::mbar_drain(bar(sm.drain), 0);
+    }
   }
   tc::fence_before();
   __syncthreads();
@@ -991,24 +869,25 @@ topk_rows_hist_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq
 
 // ---------------------------------------------------------------------------
 // Filtered selection for long rows (no FP32 score rows in HBM).  A sample of
-// the scores (every kSampleStride-th candidate tile) gives each row a
-// threshold below its kThrRank-th largest sampled score, so about
-// kThrRank * kSampleStride candidates are expected to reach it; the full
-// score pass then keeps only the (key, id) pairs at or above the threshold.
-// The selection stays exact: every candidate at or above the threshold is in
-// the list, so if at least k are, the k largest are among them.  A row with
-// fewer than k or more than kFilterCap kept entries is flagged and redone from
-// recomputed scores by the radix kernel.
+// the scores (every samp-th candidate tile) gives each row a threshold below
+// its rank-th largest sampled score, so about rank * samp candidates are
+// expected to reach it; the full score pass then keeps only the (key, id)
+// pairs at or above the threshold.  The selection stays exact: every
+// candidate at or above the threshold is in the list, so if at least k are,
+// the k largest are among them.  A row with fewer than k or more than its
+// lists hold is flagged and redone from recomputed scores by the radix
+// kernel.  Sizes (host side): k <= 512 keeps about 2k candidates in four
+// lists of 1024; larger k about 3k in four lists of 2k.
 // ---------------------------------------------------------------------------
-constexpr int kThrRank = 64;
-constexpr int kFilterCap = 4096;             // kept entries per row: four lists of kFilterCap / 4
+constexpr int kThrRank = 64;                 // rank at the smallest sample stride, k <= 512
+constexpr int kFilterCap = 4096;             // kept entries per row for k <= 512: four lists of kFilterCap / 4
 constexpr int kFilterSubCap = kFilterCap / 4;
 constexpr int kThrThreads = 256;
-constexpr int kThrPer = 32;  // samples per thread: rows of up to 131072 candidates
+constexpr int kThrPer = 32;  // samples per thread (kSampleTilesMax tiles of 128)
 
 __global__ void __launch_bounds__(kThrThreads)
 index_threshold_kernel(const float* __restrict__ sample, int64_t ld, int64_t nq, int G, int64_t q_pos0, int B,
-                       float* __restrict__ thr) {
+                       int samp, int thr_rank, float* __restrict__ thr) {
   __shared__ uint32_t wh[kThrThreads / 32][256];
   __shared__ float rmax[kThrThreads / 32], rmin[kThrThreads / 32];
   __shared__ uint32_t wsum[kThrThreads / 32];
@@ -1018,9 +897,9 @@ index_threshold_kernel(const float* __restrict__ sample, int64_t ld, int64_t nq,
   const int64_t n = (q_pos0 + i) / B;
   const float* srow = sample + row * ld;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // sample entry j = c * 128 + m is candidate (c * kSampleStride) * 128 + m
-  auto cand_of = [](int j) -> int64_t { return static_cast<int64_t>(j / kIdxCand) * kSampleStride * kIdxCand + j % kIdxCand; };
-  const int nsamp_tiles = static_cast<int>(((n + kIdxCand - 1) / kIdxCand + kSampleStride - 1) / kSampleStride);
+  // sample entry j = c * 128 + m is candidate (c * samp) * 128 + m
+  auto cand_of = [samp](int j) -> int64_t { return static_cast<int64_t>(j / kIdxCand) * samp * kIdxCand + j % kIdxCand; };
+  const int nsamp_tiles = static_cast<int>(((n + kIdxCand - 1) / kIdxCand + samp - 1) / samp);
   const int nj_all = nsamp_tiles * kIdxCand;
   // rows with more samples than the registers hold (contexts beyond 1M) use every step-th one
   const int step = (nj_all + kThrThreads * kThrPer - 1) / (kThrThreads * kThrPer);
@@ -1060,8 +939,8 @@ index_threshold_kernel(const float* __restrict__ sample, int64_t ld, int64_t nq,
     mn = fminf(mn, rmin[w]);
     total += static_cast<int>(wsum[w]);
   }
-  // the threshold sits below the (kThrRank / step)-th largest of the samples read
-  const int rank = max(kThrRank / step, 1);
+  // the threshold sits below the (thr_rank / step)-th largest of the samples read
+  const int rank = max(thr_rank / step, 1);
   if (total <= rank) {  // too few samples to estimate: keep everything
     if (tid == 0) thr[row] = -INFINITY;
     return;
@@ -1258,11 +1137,201 @@ topk_staged_kernel(const uint2* __restrict__ staging, const int32_t* __restrict_
   }
 }
 
-// One flagged row's scores, recomputed by the whole CTA.
+// Exact top-k of a row's staged (key, id) lists for k > 512 (up to 2048),
+// from up to four lists of 4096 entries: 1024 threads hold 16 entries each.
+// A linear 256-bin histogram between the kept scores' minimum and maximum
+// finds the bin holding the k-th largest; entries of higher bins are taken,
+// the boundary bin's entries are ranked exactly (score, then smaller id) by
+// one warp.  The taken ids are collected unordered and sorted ascending
+// (bitonic) in shared memory, so the output does not need a bitmap over the
+// whole candidate range (rows reach 1M candidates).  Rows with fewer than k
+// kept entries, an overflowing list or a boundary bin larger than its buffer
+// (massive exact ties) are flagged and listed for the fallback.
+constexpr int kStagedBigThreads = 1024;
+constexpr int kStagedBigPer = 16;
+constexpr int kStagedBigBnd = 4096;  // boundary entries resolved in the kernel
+constexpr int kStagedBigWarps = kStagedBigThreads / 32;
+struct StagedBigSmem {
+  uint2 cand[kStagedBigBnd];
+  uint32_t ids[2048];
+  uint32_t wh[kStagedBigWarps][256];
+  float rmax[kStagedBigWarps], rmin[kStagedBigWarps];
+  uint32_t wsum[kStagedBigWarps];
+  uint32_t bstar, rem, nc, nsel, cstar;
+};
+
+__global__ void __launch_bounds__(kStagedBigThreads)
+topk_staged_sort_kernel(const uint2* __restrict__ staging, const int32_t* __restrict__ staged, int64_t nq, int G,
+                        int64_t q_pos0, int B, int k, int cap, int32_t* __restrict__ sel,
+                        int32_t* __restrict__ sel_count, int32_t* __restrict__ flags, int32_t* __restrict__ list,
+                        int32_t* __restrict__ list_count) {
+  extern __shared__ __align__(16) uint8_t dyn_raw[];
+  StagedBigSmem& sm = *reinterpret_cast<StagedBigSmem*>(dyn_raw);
+  const int64_t row = blockIdx.x;
+  const int64_t i = (row / G) % nq;
+  const int64_t n = (q_pos0 + i) / B;
+  int32_t* out = sel + row * k;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (n <= k) {
+    for (int j = tid; j < k; j += kStagedBigThreads) out[j] = j < n ? j : -1;
+    if (tid == 0) {
+      sel_count[row] = static_cast<int32_t>(n);
+      flags[row] = 0;
+    }
+    return;
+  }
+  const int4 c4 = *reinterpret_cast<const int4*>(staged + row * 4);
+  const int cnt = c4.x + c4.y + c4.z + c4.w;
+  auto flag_row = [&]() {
+    if (tid == 0) {
+      flags[row] = 1;
+      list[atomicAdd(list_count, 1)] = static_cast<int32_t>(row);
+    }
+  };
+  if (cnt < k || c4.x > cap || c4.y > cap || c4.z > cap || c4.w > cap || cnt > kStagedBigThreads * kStagedBigPer) {
+    flag_row();
+    return;
+  }
+  const int p1 = c4.x, p2 = p1 + c4.y, p3 = p2 + c4.z;
+  const uint2* lists = staging + row * 4 * static_cast<int64_t>(cap);
+  auto entry = [&](int j) -> uint2 {
+    const int q = (j >= p1) + (j >= p2) + (j >= p3);
+    const int off = j - (q == 0 ? 0 : q == 1 ? p1 : q == 2 ? p2 : p3);
+    return lists[q * static_cast<int64_t>(cap) + off];
+  };
+  for (int b = tid; b < kStagedBigWarps * 256; b += kStagedBigThreads) (&sm.wh[0][0])[b] = 0u;
+  if (tid == 0) {
+    sm.nc = 0;
+    sm.nsel = 0;
+  }
+  uint2 e[kStagedBigPer];  // (key, id); the score is key_score(key)
+  float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+  for (int x = 0; x < kStagedBigPer; ++x) {
+    const int j = tid + kStagedBigThreads * x;
+    e[x] = j < cnt ? entry(j) : make_uint2(0u, 0xFFFFFFFFu);
+    if (j < cnt) {
+      const float v = key_score(e[x].x);
+      mx = fmaxf(mx, v);
+      mn = fminf(mn, v);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+  }
+  if (lane == 0) {
+    sm.rmax[warp] = mx;
+    sm.rmin[warp] = mn;
+  }
+  __syncthreads();
+  for (int w = 0; w < kStagedBigWarps; ++w) {
+    mx = fmaxf(mx, sm.rmax[w]);
+    mn = fminf(mn, sm.rmin[w]);
+  }
+  const float width = mx - mn;
+  const float scale = width > 0.f ? 255.5f / width : 0.f;
+  // bins ordered best first; the product rounds monotonically, so a higher
+  // score never falls in a later bin
+  auto bin_of = [&](float x) -> int { return min(static_cast<int>(__fmul_rn(__fsub_rn(mx, x), scale)), 255); };
+#pragma unroll
+  for (int x = 0; x < kStagedBigPer; ++x)
+    if (tid + kStagedBigThreads * x < cnt) atomicAdd(&sm.wh[warp][bin_of(key_score(e[x].x))], 1u);
+  __syncthreads();
+  if (warp == 0) {
+    // 256 bins, 8 per lane: the bin in which the running count reaches k
+    uint32_t loc[8], sum = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      uint32_t c = 0;
+      for (int w = 0; w < kStagedBigWarps; ++w) c += sm.wh[w][lane * 8 + q];
+      loc[q] = c;
+      sum += c;
+    }
+    uint32_t inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    uint32_t acc = inc - sum;
+    const uint32_t kk = static_cast<uint32_t>(k);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (acc < kk && kk <= acc + loc[q]) {
+        sm.bstar = lane * 8 + q;
+        sm.rem = kk - acc;
+        sm.cstar = loc[q];
+      }
+      acc += loc[q];
+    }
+  }
+  __syncthreads();
+  if (sm.cstar > kStagedBigBnd) {  // the boundary does not fit its buffer
+    flag_row();
+    return;
+  }
+  const int bstar = static_cast<int>(sm.bstar);
+  const uint32_t rem = sm.rem;
+#pragma unroll
+  for (int x = 0; x < kStagedBigPer; ++x) {
+    if (tid + kStagedBigThreads * x >= cnt) continue;
+    const int b = bin_of(key_score(e[x].x));
+    if (b < bstar) {
+      sm.ids[atomicAdd(&sm.nsel, 1u)] = e[x].y;
+    } else if (b == bstar) {
+      sm.cand[atomicAdd(&sm.nc, 1u)] = e[x];
+    }
+  }
+  __syncthreads();
+  const uint32_t nc = sm.nc;
+  if (warp == 0) {
+    uint32_t theta = 0, id_cut = 0xFFFFFFFFu;
+    if (nc > rem) warp_select(sm.cand, static_cast<int>(nc), static_cast<int>(rem), sm.wh[0], theta, id_cut);
+    const uint32_t base = sm.nsel;  // k - rem entries above the boundary bin
+    uint32_t taken = 0;
+    for (uint32_t c0 = 0; c0 < nc; c0 += 32) {
+      const uint32_t c = c0 + lane;
+      const bool take = c < nc && (nc <= rem || kept(sm.cand[c], theta, id_cut));
+      const uint32_t bal = __ballot_sync(0xffffffffu, take);
+      if (take) sm.ids[base + taken + __popc(bal & ((1u << lane) - 1u))] = sm.cand[c].y;
+      taken += __popc(bal);
+    }
+  }
+  __syncthreads();
+  // ascending ids: bitonic sort of the k taken ids (padded to a power of two)
+  int pow2 = 1;
+  while (pow2 < k) pow2 <<= 1;
+  for (int j = k + tid; j < pow2; j += kStagedBigThreads) sm.ids[j] = 0xFFFFFFFFu;
+  __syncthreads();
+  for (int size = 2; size <= pow2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int c = tid; c < pow2 / 2; c += kStagedBigThreads) {
+        const int lo = 2 * stride * (c / stride) + (c % stride);
+        const int hi = lo + stride;
+        const bool asc = (lo & size) == 0;
+        const uint32_t a = sm.ids[lo], b = sm.ids[hi];
+        if ((a > b) == asc) {
+          sm.ids[lo] = b;
+          sm.ids[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int j = tid; j < k; j += kStagedBigThreads) out[j] = static_cast<int32_t>(sm.ids[j]);
+  if (tid == 0) {
+    sel_count[row] = k;
+    flags[row] = 0;
+  }
+}
+
+// One flagged row's scores, recomputed by the whole CTA into srow.
 __device__ __forceinline__ void index_score_fallback_row(int64_t row, const __nv_bfloat16* __restrict__ idx_q,
                                                          const float* __restrict__ idx_w,
                                                          const __nv_bfloat16* __restrict__ keys,
-                                                         float* __restrict__ scores, int64_t nq, int G, int H,
+                                                         float* __restrict__ srow, int64_t nq, int G, int H,
                                                          int64_t q_pos0, int B, int64_t rpad, float (*qf)[64],
                                                          float* wf) {
   const int64_t i = (row / G) % nq;
@@ -1292,24 +1361,31 @@ __device__ __forceinline__ void index_score_fallback_row(int64_t row, const __nv
       for (int x = 0; x < 64; ++x) d = fmaf(qf[h][x], kv[x], d);
       acc = fmaf(wf[h], fmaxf(d, 0.f), acc);
     }
-    scores[row * rpad + r] = acc;
+    srow[r] = acc;
   }
 }
 
-// Listed rows only: the row's scores recomputed on the CUDA cores (FP32 dot
-// products of the row's indexer queries with the widened keys) into the score
-// rows, for the radix kernel; a fixed grid strides over the list.
-__global__ void __launch_bounds__(256)
-index_score_fallback_kernel(const __nv_bfloat16* __restrict__ idx_q, const float* __restrict__ idx_w,
-                            const __nv_bfloat16* __restrict__ keys, const int32_t* __restrict__ list,
-                            const int32_t* __restrict__ list_count, float* __restrict__ scores, int64_t nq, int G,
-                            int H, int64_t q_pos0, int B, int64_t rpad) {
+// Listed rows only (the rows the filtered path could not settle): each CTA
+// recomputes a row's scores on the CUDA cores (FP32 dot products of the row's
+// indexer queries with the widened keys) into its own slot of rpad floats,
+// then radix-selects the row from it; a fixed grid strides over the list, so
+// the scratch is grid x rpad floats whatever the number of rows.
+__global__ void __launch_bounds__(kSelThreads)
+index_fallback_select_kernel(const __nv_bfloat16* __restrict__ idx_q, const float* __restrict__ idx_w,
+                             const __nv_bfloat16* __restrict__ keys, const int32_t* __restrict__ list,
+                             const int32_t* __restrict__ list_count, float* __restrict__ slots, int64_t nq, int G,
+                             int H, int64_t q_pos0, int B, int64_t rpad, int k, int32_t* __restrict__ sel,
+                             int32_t* __restrict__ sel_count) {
   __shared__ float qf[8][64];
   __shared__ float wf[8];
+  float* slot = slots + static_cast<int64_t>(blockIdx.x) * rpad;
   const int nlist = *list_count;
   for (int x = blockIdx.x; x < nlist; x += gridDim.x) {
-    __syncthreads();  // qf / wf of the previous row are no longer read
-    index_score_fallback_row(list[x], idx_q, idx_w, keys, scores, nq, G, H, q_pos0, B, rpad, qf, wf);
+    __syncthreads();  // the previous row's scores, qf and wf are no longer read
+    const int64_t row = list[x];
+    index_score_fallback_row(row, idx_q, idx_w, keys, slot, nq, G, H, q_pos0, B, rpad, qf, wf);
+    __syncthreads();  // the slot holds the row's scores
+    topk_row_radix_at<false>(row, slot, nq, G, q_pos0, B, k, sel, sel_count);
   }
 }
 

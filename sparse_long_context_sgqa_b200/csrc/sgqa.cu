@@ -95,32 +95,80 @@ int plan_pow2(int k) {
   return std::max(p, 2);
 }
 
-// Index workspace: widened keys, then one region that holds, one after the
-// other within a call, the sampled scores, the filtered staging lists and the
-// FP32 score rows (the stages that use them run in that order), then three
-// per-row arrays.
+// Index path for many queries: tcgen05 score rows and a top-k kernel over
+// them.  Rows longer than the histogram top-k takes (16384 candidates) use the
+// filtered path; shorter rows are cheaper to materialise and select (measured
+// at 128K and 1M contexts).
+constexpr int64_t kFilterMinCand = 16385;
+
+// Sizes of the filtered path for rows of up to rneed candidates and top-k k:
+// every samp-th tile of 128 candidates is sampled (at most kSampleTilesMax
+// tiles per row); the threshold sits below the rank-th largest sample, so
+// about rank * samp candidates -- 2k for k <= 512, 3k above -- are expected to
+// pass; each row keeps four lists of subcap (key, id) pairs.
+struct FilterSizes {
+  int samp, rank, subcap;
+  int64_t nsamp;
+};
+FilterSizes filter_sizes(int64_t rneed, int k) {
+  FilterSizes f;
+  const int64_t ntiles = (rneed + sgqa::kIdxCand - 1) / sgqa::kIdxCand;
+  f.samp = static_cast<int>(std::max<int64_t>(sgqa::kSampleStride,
+                                              (ntiles + sgqa::kSampleTilesMax - 1) / sgqa::kSampleTilesMax));
+  f.nsamp = (ntiles + f.samp - 1) / f.samp * sgqa::kIdxCand;
+  const int64_t target = k <= 512 ? 2 * static_cast<int64_t>(k) : 3 * static_cast<int64_t>(k);
+  f.rank = static_cast<int>(std::max<int64_t>(16, (target + f.samp - 1) / f.samp));
+  f.subcap = k <= 512 ? sgqa::kFilterSubCap : 2 * k;
+  return f;
+}
+
+// CTAs of the fallback kernel (each owns one row-sized scratch slot).
+constexpr int64_t kFallbackGrid = 2 * 148;
+
+// Index workspace: widened keys, then one region used by the call's path --
+// the FP32 score rows [rows, rpad] (rows of fewer than kFilterMinCand
+// candidates, and decode), or in turn the sampled scores, the filtered
+// (key, id) lists and the fallback's per-CTA score slots (the stages that use
+// them run in that order) -- then four per-row arrays.
 struct IndexWs {
-  int64_t rpad, nsamp;
-  size_t keys_off, scores_off, sample_off, staging_off, flags_off, staged_off, thr_off, list_off, bytes;
+  int64_t rpad;
+  bool filtered;
+  FilterSizes f;
+  int64_t fb_grid;
+  size_t keys_off, region_off, flags_off, staged_off, thr_off, list_off, bytes;
 };
 IndexWs index_ws(const sgqa_params* p, int64_t S, int64_t nq, int64_t max_ctx) {
   IndexWs w;
   const int64_t rneed = std::max<int64_t>((max_ctx - 1) / p->block_size, 1);
   w.rpad = round_up(rneed, 128);
-  w.nsamp = round_up(w.rpad, sgqa::kIdxCand * sgqa::kSampleStride) / sgqa::kSampleStride;
   w.keys_off = 0;
   const size_t keys = align256(static_cast<size_t>(S * w.rpad * 64) * 2);
   const size_t rows = static_cast<size_t>(S * nq * p->num_kv_groups);
-  const size_t big = align256(std::max({rows * static_cast<size_t>(w.rpad) * 4,
-                                        rows * static_cast<size_t>(sgqa::kFilterCap) * 8,
-                                        rows * static_cast<size_t>(w.nsamp) * 4}));
-  w.scores_off = w.sample_off = w.staging_off = keys;
-  w.flags_off = keys + big;
+  w.filtered = nq > kDecodeMaxNq && rneed >= kFilterMinCand;
+  w.f = filter_sizes(rneed, p->topk);
+  w.fb_grid = std::min<int64_t>(static_cast<int64_t>(rows), kFallbackGrid);
+  size_t region;
+  if (w.filtered) {
+    region = std::max({rows * static_cast<size_t>(w.f.nsamp) * 4, rows * 4 * static_cast<size_t>(w.f.subcap) * 8,
+                       static_cast<size_t>(w.fb_grid) * static_cast<size_t>(w.rpad) * 4});
+  } else {
+    region = rows * static_cast<size_t>(w.rpad) * 4;
+  }
+  w.region_off = keys;
+  w.flags_off = keys + align256(region);
   w.staged_off = w.flags_off + align256(rows * 4);
   w.thr_off = w.staged_off + align256(rows * 4 * 4);  // staged: [rows, 4] counts
   w.list_off = w.thr_off + align256(rows * 4);       // unsettled rows [rows], then their count
   w.bytes = w.list_off + align256(rows * 4) + 256;
   return w;
+}
+
+// Workspace for every call with q_pos0 + nq <= max_ctx: the largest call of
+// each path (score rows, filtered).
+size_t index_ws_bytes_upto(const sgqa_params* p, int64_t S, int64_t nq, int64_t max_ctx) {
+  const int64_t rows_max_ctx = (kFilterMinCand - 1) * p->block_size + 1;  // longest context on the score-rows path
+  return std::max(index_ws(p, S, nq, max_ctx).bytes,
+                  index_ws(p, S, nq, std::min(max_ctx, rows_max_ctx)).bytes);
 }
 
 struct AttnWs {
@@ -218,42 +266,62 @@ sgqa_status encode_bf16(CUtensorMap* m, const void* base, int rank, const cuuint
   return SGQA_OK;
 }
 
+// Where the K/V of an attention call live: the contiguous caches
+// [S, cap, G, D], or a pool of 16-token pages [pages, G, 16, D] with a page
+// table [S, max_pages].
+struct KvSource {
+  const void* k;
+  const void* v;
+  int64_t cap, clen;                    // contiguous
+  const int32_t* page_table = nullptr;  // paged
+  int64_t max_pages = 0, num_pages = 0;
+  bool paged() const { return page_table != nullptr; }
+};
+
+// Tensor maps over K and V with 8-token boxes of all 192 dims (three 128-byte
+// column chunks, SW128): contiguous caches as (64 elements, token row, chunk,
+// group, sequence); a page pool as (64 elements, row in page, chunk, group,
+// page), where one group's 8-token block is a contiguous 3 KB run.
+sgqa_status kv_maps(const KvSource& kv, int G, int64_t S, CUtensorMap* km, CUtensorMap* vm) {
+  cuuint32_t box[5] = {64, 8, 3, 1, 1};
+  sgqa_status s;
+  if (kv.paged()) {
+    cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(sgqa::kPageTokens), 3, static_cast<cuuint64_t>(G),
+                          static_cast<cuuint64_t>(kv.num_pages)};
+    cuuint64_t strides[4] = {384, 128, static_cast<cuuint64_t>(sgqa::kPageTokens) * 384,
+                             static_cast<cuuint64_t>(G) * sgqa::kPageTokens * 384};
+    if ((s = encode_bf16(km, kv.k, 5, dims, strides, box, "k_pool")) != SGQA_OK) return s;
+    return encode_bf16(vm, kv.v, 5, dims, strides, box, "v_pool");
+  }
+  cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(kv.clen), 3, static_cast<cuuint64_t>(G), static_cast<cuuint64_t>(S)};
+  cuuint64_t strides[4] = {static_cast<cuuint64_t>(G) * 384, 128, 384, static_cast<cuuint64_t>(kv.cap) * G * 384};
+  if ((s = encode_bf16(km, kv.k, 5, dims, strides, box, "k_cache")) != SGQA_OK) return s;
+  return encode_bf16(vm, kv.v, 5, dims, strides, box, "v_cache");
+}
+
 sgqa_status launch_attn_tc(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q,
-                           int64_t cap, int64_t clen, const void* kc, const void* vc, const int32_t* ids,
-                           const uint8_t* msk, const int32_t* cnt, void* out, const void* gate, int64_t units,
-                           cudaStream_t st) {
+                           const KvSource& kv, const int32_t* ids, const uint8_t* msk, const int32_t* cnt, void* out,
+                           const void* gate, int64_t units, cudaStream_t st) {
   const int G = p->num_kv_groups;
   const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
   CUtensorMap km, vm;
   sgqa_status s;
-  {
-    // (64 elements, token rows < cache_len, 3 column chunks, group, sequence)
-    cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(clen), 3, static_cast<cuuint64_t>(G), static_cast<cuuint64_t>(S)};
-    cuuint64_t strides[4] = {static_cast<cuuint64_t>(G) * 384, 128, 384, static_cast<cuuint64_t>(cap) * G * 384};
-    cuuint32_t box[5] = {64, 8, 3, 1, 1};
-    if ((s = encode_bf16(&km, kc, 5, dims, strides, box, "k_cache")) != SGQA_OK) return s;
-    if ((s = encode_bf16(&vm, vc, 5, dims, strides, box, "v_cache")) != SGQA_OK) return s;
-  }
+  if ((s = kv_maps(kv, G, S, &km, &vm)) != SGQA_OK) return s;
   static_assert(sizeof(sgqa::AttnTcSmem) + 1024 <= 232448, "attention tile exceeds shared memory");
   const size_t smem = sizeof(sgqa::AttnTcSmem) + 1024;
   // Selections covering under a quarter of the candidates leave many block
   // pairs unattended by both queries of a warp: skip their exponentials.
   const bool skip_pairs = (q0 + nq - 1) / p->block_size > 4 * static_cast<int64_t>(p->topk);
-  auto kern = skip_pairs ? sgqa::attn_tc_kernel<true> : sgqa::attn_tc_kernel<false>;
+  auto kern = kv.paged() ? (skip_pairs ? sgqa::attn_tc_kernel<true, true> : sgqa::attn_tc_kernel<false, true>)
+                         : (skip_pairs ? sgqa::attn_tc_kernel<true, false> : sgqa::attn_tc_kernel<false, false>);
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   kern<<<static_cast<unsigned>(units), sgqa::kTcThreads, smem, st>>>(
       static_cast<const __nv_bfloat16*>(q), km, vm, ids, msk, cnt, static_cast<__nv_bfloat16*>(out),
-      static_cast<const __nv_bfloat16*>(gate), nq, G, p->topk, q0, scale_log2);
+      static_cast<const __nv_bfloat16*>(gate), nq, G, p->topk, q0, scale_log2, kv.page_table, kv.max_pages,
+      kv.num_pages);
   SGQA_LAUNCH_CHECK("attn_tc_kernel");
   return SGQA_OK;
 }
-
-// Index path for many queries: tcgen05 score rows and a top-k kernel over
-// them.  Rows longer than the histogram top-k takes (16384 candidates) use the
-// filtered path; shorter rows are cheaper to materialise and select (measured
-// at 128K and 1M contexts).  The kept lists are sized for k <= 512 (about 1k
-// entries expected per row, 4k room).
-constexpr int64_t kFilterMinCand = 16385;
 
 sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* idx_q,
                      const float* idx_w, int64_t cap, const uint8_t* store, int32_t* sel,
@@ -269,7 +337,7 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
     SGQA_LAUNCH_CHECK("widen_store_kernel");
   }
   const __nv_bfloat16* iq = static_cast<const __nv_bfloat16*>(idx_q);
-  float* scores = ws_at<float>(ws, w.scores_off);
+  float* scores = ws_at<float>(ws, w.region_off);
   int32_t* flags = ws_at<int32_t>(ws, w.flags_off);
   // rows a select kernel could not settle, for the radix kernel (count after the list)
   int32_t* list = ws_at<int32_t>(ws, w.list_off);
@@ -315,47 +383,53 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
       }
 #undef SGQA_SCORE
     };
-    if (rneed >= kFilterMinCand && p->topk * 8 <= sgqa::kFilterCap) {
+    if (w.filtered) {
       // Long rows: sampled threshold, filtered score pass, exact select from the
-      // kept lists; rows the filter could not settle are recomputed and go to
-      // the radix kernel.  No FP32 score row is written for the others.
+      // kept lists; rows the filter could not settle are recomputed and
+      // radix-selected by the fallback kernel.  No FP32 score row is written.
       const int64_t rows = S * nq * G;
-      float* sample = ws_at<float>(ws, w.sample_off);
+      float* sample = ws_at<float>(ws, w.region_off);
       float* thr = ws_at<float>(ws, w.thr_off);
-      uint2* staging = ws_at<uint2>(ws, w.staging_off);
+      uint2* staging = ws_at<uint2>(ws, w.region_off);
+      float* slots = ws_at<float>(ws, w.region_off);
       int32_t* staged = ws_at<int32_t>(ws, w.staged_off);
-      launch_score(sgqa::kScoreSample, sgqa::ScoreOut{sample, w.nsamp, nullptr, nullptr, nullptr, 0});
+      launch_score(sgqa::kScoreSample, sgqa::ScoreOut{sample, w.f.nsamp, w.f.samp, nullptr, nullptr, nullptr, 0});
       SGQA_LAUNCH_CHECK("index_score_tc_kernel (sample)");
-      sgqa::index_threshold_kernel<<<static_cast<unsigned>(rows), sgqa::kThrThreads, 0, st>>>(sample, w.nsamp, nq, G,
-                                                                                           q0, B, thr);
+      sgqa::index_threshold_kernel<<<static_cast<unsigned>(rows), sgqa::kThrThreads, 0, st>>>(
+          sample, w.f.nsamp, nq, G, q0, B, w.f.samp, w.f.rank, thr);
       SGQA_LAUNCH_CHECK("index_threshold_kernel");
-      launch_score(sgqa::kScoreFilter, sgqa::ScoreOut{nullptr, 0, thr, staging, staged, sgqa::kFilterSubCap});
+      launch_score(sgqa::kScoreFilter, sgqa::ScoreOut{nullptr, 0, 0, thr, staging, staged, w.f.subcap});
       SGQA_LAUNCH_CHECK("index_score_tc_kernel (filter)");
-      const int nwords_max = static_cast<int>((rneed + 31) / 32);
-      const size_t dsmem = static_cast<size_t>(2 * sgqa::kFilterCap + nwords_max) * 4;
-      cudaFuncSetAttribute(sgqa::topk_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsmem);
       cudaError_t e = cudaMemsetAsync(list_count, 0, 4, st);
       if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(list count)");
-      sgqa::topk_staged_kernel<<<static_cast<unsigned>(rows), sgqa::kStagedThreads, dsmem, st>>>(
-          staging, staged, nq, G, q0, B, p->topk, sgqa::kFilterSubCap, nwords_max, sel, sel_count, flags, list,
-          list_count);
-      SGQA_LAUNCH_CHECK("topk_staged_kernel");
-      const unsigned fb_grid = static_cast<unsigned>(std::min<int64_t>(rows, 2 * 148));
-      sgqa::index_score_fallback_kernel<<<fb_grid, 256, 0, st>>>(iq, idx_w, keys, list, list_count, scores, nq, G, H,
-                                                                 q0, B, w.rpad);
-      SGQA_LAUNCH_CHECK("index_score_fallback_kernel");
-      sgqa::topk_rows_list_kernel<<<fb_grid, sgqa::kSelThreads, 0, st>>>(scores, w.rpad, nq, G, q0, B, p->topk, sel,
-                                                                         sel_count, list, list_count);
-      SGQA_LAUNCH_CHECK("topk_rows_list_kernel");
+      if (p->topk <= 512) {
+        const int nwords_max = static_cast<int>((rneed + 31) / 32);
+        const size_t dsmem = static_cast<size_t>(2 * sgqa::kFilterCap + nwords_max) * 4;
+        if (dsmem > 227 * 1024) return fail(SGQA_ERR_UNSUPPORTED, "context too long for the staged top-k kernel");
+        cudaFuncSetAttribute(sgqa::topk_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsmem);
+        sgqa::topk_staged_kernel<<<static_cast<unsigned>(rows), sgqa::kStagedThreads, dsmem, st>>>(
+            staging, staged, nq, G, q0, B, p->topk, w.f.subcap, nwords_max, sel, sel_count, flags, list, list_count);
+        SGQA_LAUNCH_CHECK("topk_staged_kernel");
+      } else {
+        const size_t dsmem = sizeof(sgqa::StagedBigSmem);
+        cudaFuncSetAttribute(sgqa::topk_staged_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsmem);
+        sgqa::topk_staged_sort_kernel<<<static_cast<unsigned>(rows), sgqa::kStagedBigThreads, dsmem, st>>>(
+            staging, staged, nq, G, q0, B, p->topk, w.f.subcap, sel, sel_count, flags, list, list_count);
+        SGQA_LAUNCH_CHECK("topk_staged_sort_kernel");
+      }
+      sgqa::index_fallback_select_kernel<<<static_cast<unsigned>(w.fb_grid), sgqa::kSelThreads, 0, st>>>(
+          iq, idx_w, keys, list, list_count, slots, nq, G, H, q0, B, w.rpad, p->topk, sel, sel_count);
+      SGQA_LAUNCH_CHECK("index_fallback_select_kernel");
       return SGQA_OK;
     }
-    launch_score(sgqa::kScoreRows, sgqa::ScoreOut{scores, w.rpad, nullptr, nullptr, nullptr, 0});
+    launch_score(sgqa::kScoreRows, sgqa::ScoreOut{scores, w.rpad, 0, nullptr, nullptr, nullptr, 0});
     SGQA_LAUNCH_CHECK("index_score_tc_kernel");
   } else if (rneed > 0 && G == 4 && H == 8) {
     // few queries: one CTA per (query, 128 candidates) scores all four groups from the E4M3 store
-    dim3 grid(static_cast<unsigned>((rneed + 127) / 128), static_cast<unsigned>(S * nq));
-    sgqa::index_score_decode_kernel<<<grid, sgqa::kDecScoreWarps * 32, 0, st>>>(iq, idx_w, store, scores, nq, q0, B,
-                                                                                 w.rpad, cap / B);
+    dim3 grid(static_cast<unsigned>((rneed + sgqa::kDecScoreCand - 1) / sgqa::kDecScoreCand),
+              static_cast<unsigned>(S * nq));
+    sgqa::index_score_decode_kernel<<<grid, sgqa::kDecScoreThreads, 0, st>>>(iq, idx_w, store, scores, nq, q0, B,
+                                                                              w.rpad, cap / B);
     SGQA_LAUNCH_CHECK("index_score_decode_kernel");
   } else if (rneed > 0) {
     // few queries: warp-MMA scores straight from the E4M3 store
@@ -389,7 +463,7 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
   // row in HBM (histogram, then gather).  Rows either cannot finish
   // (boundary-bin overflow) go to the radix kernel, which also takes the rows
   // in between and short rows (its per-row set-up is smaller).
-  if (rneed >= 2048 && rneed <= sgqa::kHistMaxCand) {
+  if (rneed >= 2048 && rneed <= sgqa::kHistMaxCand && p->topk <= 512) {
     cudaError_t e = cudaMemsetAsync(list_count, 0, 4, st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(list count)");
     sgqa::topk_rows_hist_kernel<<<static_cast<unsigned>(rows), sgqa::kHistThreads, 0, st>>>(
@@ -419,29 +493,25 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
 }
 
 template <int B>
-sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q,
-                        int64_t cap, int64_t clen, const void* kc, const void* vc, const int32_t* sel,
-                        const int32_t* sel_count, void* out, const void* gate, void* ws, cudaStream_t st) {
+sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q, const KvSource& kv,
+                        const int32_t* sel, const int32_t* sel_count, void* out, const void* gate, void* ws,
+                        cudaStream_t st) {
   const int G = p->num_kv_groups, k = p->topk;
   const __nv_bfloat16* gb = static_cast<const __nv_bfloat16*>(gate);
   const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
   const AttnWs w = attn_ws(p, S, nq);
   const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
-  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(kc);
-  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(vc);
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(kv.k);
+  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(kv.v);
   __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(out);
   if (nq <= kDecodeMaxNq && B == 8) {
     // TMA-fed gather, the splits of a row combined inside their cluster
     const int64_t rows = S * nq * G;
     CUtensorMap km, vm;
-    cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(clen), 3, static_cast<cuuint64_t>(G), static_cast<cuuint64_t>(S)};
-    cuuint64_t strides[4] = {static_cast<cuuint64_t>(G) * 384, 128, 384, static_cast<cuuint64_t>(cap) * G * 384};
-    cuuint32_t box[5] = {64, 8, 3, 1, 1};
     sgqa_status s;
-    if ((s = encode_bf16(&km, kc, 5, dims, strides, box, "k_cache")) != SGQA_OK) return s;
-    if ((s = encode_bf16(&vm, vc, 5, dims, strides, box, "v_cache")) != SGQA_OK) return s;
+    if ((s = kv_maps(kv, G, S, &km, &vm)) != SGQA_OK) return s;
     // the splits of a row run as one cluster (combined through distributed shared memory)
-    const int nsplit = std::min(w.nsplit, sgqa::kDecMaxSplit);
+    const int nsplit = std::min(decode_splits(rows), sgqa::kDecMaxSplit);
     const size_t smem = sizeof(sgqa::DecSmem) + 1024;
     cudaFuncSetAttribute(sgqa::attn_decode_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     cudaLaunchConfig_t cfg = {};
@@ -457,12 +527,12 @@ sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, sgqa::attn_decode_tma_kernel, km, vm, qb, sel, sel_count, ob, gb, nq, G,
-                                       k, q0, nsplit, scale_log2, static_cast<const int32_t*>(nullptr),
-                                       static_cast<int64_t>(0), static_cast<int64_t>(0));
+                                       k, q0, nsplit, scale_log2, kv.page_table, kv.max_pages, kv.num_pages);
     if (e != cudaSuccess) return cuda_fail(e, "attn_decode_tma_kernel launch");
     SGQA_LAUNCH_CHECK("attn_decode_tma_kernel");
     return SGQA_OK;
   }
+  if (kv.paged() && B != 8) return fail(SGQA_ERR_UNSUPPORTED, "paged K/V needs block_size 8");
   if (nq <= kDecodeMaxNq) {
     const int64_t rows = S * nq * G;
     const size_t smem = sgqa::kDecWarps * sgqa::kDecStages * 2 * sgqa::kStageElems * 2;
@@ -470,7 +540,7 @@ sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq,
     float* po = ws_at<float>(ws, w.po_off);
     float* pml = ws_at<float>(ws, w.pml_off);
     sgqa::attn_decode_kernel<B><<<static_cast<unsigned>(rows * w.nsplit), sgqa::kDecWarps * 32, smem, st>>>(
-        qb, kb, vb, sel, sel_count, po, pml, nq, G, k, q0, cap, w.nsplit, scale_log2);
+        qb, kb, vb, sel, sel_count, po, pml, nq, G, k, q0, kv.cap, w.nsplit, scale_log2);
     SGQA_LAUNCH_CHECK("attn_decode_kernel");
     sgqa::attn_combine_kernel<<<static_cast<unsigned>(rows * 16), 64, 0, st>>>(po, pml, ob, gb, rows, w.nsplit);
     SGQA_LAUNCH_CHECK("attn_combine_kernel");
@@ -486,80 +556,48 @@ sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq,
   if (psmem <= 96 * 1024) {
     cudaFuncSetAttribute(sgqa::attn_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
     sgqa::attn_plan_kernel<<<static_cast<unsigned>(units), sgqa::kPlanThreads, psmem, st>>>(
-        sel, sel_count, nq, G, k, nwords, ids, msk, cnt);
+        sel, sel_count, nq, G, k, nwords, q0, B, ids, msk, cnt);
     SGQA_LAUNCH_CHECK("attn_plan_kernel");
   } else {
     const int pow2 = plan_pow2(k);
     const size_t ssmem = static_cast<size_t>(pow2) * 4;
     cudaFuncSetAttribute(sgqa::attn_plan_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
     sgqa::attn_plan_sort_kernel<<<static_cast<unsigned>(units), sgqa::kPlanSortThreads, ssmem, st>>>(
-        sel, sel_count, nq, G, k, pow2, ids, msk, cnt);
+        sel, sel_count, nq, G, k, pow2, q0, B, ids, msk, cnt);
     SGQA_LAUNCH_CHECK("attn_plan_sort_kernel");
   }
   if constexpr (B == 8) {
-    return launch_attn_tc(p, S, q0, nq, q, cap, clen, kc, vc, ids, msk, cnt, out, gate, units, st);
+    return launch_attn_tc(p, S, q0, nq, q, kv, ids, msk, cnt, out, gate, units, st);
   } else {
     const size_t smem = sgqa::kGroupedStages * 2 * sgqa::kStageElems * 2;
     cudaFuncSetAttribute(sgqa::attn_grouped_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     sgqa::attn_grouped_kernel<B><<<static_cast<unsigned>(units), sgqa::kGroupedThreads, smem, st>>>(
-        qb, kb, vb, ids, msk, cnt, ob, gb, nq, G, k, q0, cap, clen, scale_log2);
+        qb, kb, vb, ids, msk, cnt, ob, gb, nq, G, k, q0, kv.cap, kv.clen, scale_log2);
     SGQA_LAUNCH_CHECK("attn_grouped_kernel");
     return SGQA_OK;
   }
 }
 
-// Decode attention over a paged K/V cache: the TMA-fed gather kernel with its
-// tensor maps over the page pool [num_pages * 16 tokens, G, D] and each
-// block's row looked up in the page table.
-sgqa_status launch_attn_decode_paged(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q,
-                                     const void* kpool, const void* vpool, int64_t num_pages,
-                                     const int32_t* page_table, int64_t max_pages, const int32_t* sel,
-                                     const int32_t* sel_count, const void* gate, void* out, cudaStream_t st) {
-  const int G = p->num_kv_groups, k = p->topk;
-  const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
-  const int64_t rows = S * nq * G;
-  const int64_t pool_rows = num_pages * sgqa::kPageTokens;
-  CUtensorMap km, vm;
-  cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(pool_rows), 3, static_cast<cuuint64_t>(G), 1};
-  // the last axis (size 1) stands where the contiguous maps have the sequence
-  cuuint64_t strides[4] = {static_cast<cuuint64_t>(G) * 384, 128, 384, static_cast<cuuint64_t>(G) * 384};
-  cuuint32_t box[5] = {64, 8, 3, 1, 1};
-  sgqa_status s;
-  if ((s = encode_bf16(&km, kpool, 5, dims, strides, box, "k_pool")) != SGQA_OK) return s;
-  if ((s = encode_bf16(&vm, vpool, 5, dims, strides, box, "v_pool")) != SGQA_OK) return s;
-  const int nsplit = std::min(decode_splits(rows), sgqa::kDecMaxSplit);
-  const size_t smem = sizeof(sgqa::DecSmem) + 1024;
-  cudaFuncSetAttribute(sgqa::attn_decode_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(rows * nsplit));
-  cfg.blockDim = dim3(sgqa::kDecThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(nsplit);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, sgqa::attn_decode_tma_kernel, km, vm, static_cast<const __nv_bfloat16*>(q),
-                                     sel, sel_count, static_cast<__nv_bfloat16*>(out),
-                                     static_cast<const __nv_bfloat16*>(gate), nq, G, k, q0, nsplit, scale_log2,
-                                     page_table, max_pages, num_pages);
-  if (e != cudaSuccess) return cuda_fail(e, "attn_decode_tma_kernel launch (paged)");
-  SGQA_LAUNCH_CHECK("attn_decode_tma_kernel");
-  return SGQA_OK;
+sgqa_status do_attn_kv(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q, const KvSource& kv,
+                       const int32_t* sel, const int32_t* sel_count, void* out, const void* gate, void* ws,
+                       cudaStream_t st) {
+  switch (p->block_size) {
+    case 1: return launch_attn<1>(p, S, q0, nq, q, kv, sel, sel_count, out, gate, ws, st);
+    case 2: return launch_attn<2>(p, S, q0, nq, q, kv, sel, sel_count, out, gate, ws, st);
+    case 4: return launch_attn<4>(p, S, q0, nq, q, kv, sel, sel_count, out, gate, ws, st);
+    default: return launch_attn<8>(p, S, q0, nq, q, kv, sel, sel_count, out, gate, ws, st);
+  }
 }
 
 sgqa_status do_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q,
                     int64_t cap, int64_t clen, const void* kc, const void* vc, const int32_t* sel,
                     const int32_t* sel_count, void* out, const void* gate, void* ws, cudaStream_t st) {
-  switch (p->block_size) {
-    case 1: return launch_attn<1>(p, S, q0, nq, q, cap, clen, kc, vc, sel, sel_count, out, gate, ws, st);
-    case 2: return launch_attn<2>(p, S, q0, nq, q, cap, clen, kc, vc, sel, sel_count, out, gate, ws, st);
-    case 4: return launch_attn<4>(p, S, q0, nq, q, cap, clen, kc, vc, sel, sel_count, out, gate, ws, st);
-    default: return launch_attn<8>(p, S, q0, nq, q, cap, clen, kc, vc, sel, sel_count, out, gate, ws, st);
-  }
+  KvSource kv;
+  kv.k = kc;
+  kv.v = vc;
+  kv.cap = cap;
+  kv.clen = clen;
+  return do_attn_kv(p, S, q0, nq, q, kv, sel, sel_count, out, gate, ws, st);
 }
 
 sgqa_status check_common(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, int64_t cap) {
@@ -620,9 +658,9 @@ sgqa_status sgqa_workspace_size(const sgqa_params* p, int64_t num_seqs, int64_t 
   if (s != SGQA_OK) return s;
   if (bytes == nullptr) return fail(SGQA_ERR_INVALID_ARGUMENT, "bytes is NULL");
   if (num_seqs < 1 || nq < 0 || max_ctx < nq) return fail(SGQA_ERR_INVALID_ARGUMENT, "bad sizes");
-  const IndexWs iw = index_ws(p, num_seqs, nq, std::max<int64_t>(max_ctx, 1));
+  const size_t iw = index_ws_bytes_upto(p, num_seqs, nq, std::max<int64_t>(max_ctx, 1));
   const AttnWs aw = attn_ws(p, num_seqs, nq);
-  *bytes = std::max(iw.bytes, aw.bytes);
+  *bytes = std::max(iw, aw.bytes);
   return SGQA_OK;
 }
 
@@ -771,16 +809,13 @@ sgqa_status sgqa_sparse_attn_paged(const sgqa_params* p, int64_t num_seqs, int64
                                    const void* q, const void* k_pool, const void* v_pool, int64_t num_pages,
                                    const int32_t* page_table, int64_t max_pages, int64_t cache_len,
                                    const int32_t* sel, const int32_t* sel_count, const void* gate, void* out,
-                                   void* stream) {
+                                   void* workspace, size_t workspace_bytes, void* stream) {
   g_err.clear();
   sgqa_status s = check_params(p);
   if (s != SGQA_OK) return s;
   if (num_seqs < 1) return fail(SGQA_ERR_INVALID_ARGUMENT, "num_seqs must be >= 1");
   if (q_pos0 < 0 || nq < 0) return fail(SGQA_ERR_INVALID_ARGUMENT, "q_pos0 and nq must be >= 0");
   if (nq == 0) return SGQA_OK;
-  if (nq > kDecodeMaxNq)
-    return fail(SGQA_ERR_UNSUPPORTED, "sgqa_sparse_attn_paged takes at most %d queries per sequence (got %lld)",
-                (int)kDecodeMaxNq, (long long)nq);
   if (p->block_size != 8) return fail(SGQA_ERR_UNSUPPORTED, "sgqa_sparse_attn_paged needs block_size 8");
   if (cache_len < q_pos0 + nq) return fail(SGQA_ERR_INVALID_ARGUMENT, "need q_pos0 + nq <= cache_len");
   if (max_pages * sgqa::kPageTokens < cache_len)
@@ -796,8 +831,19 @@ sgqa_status sgqa_sparse_attn_paged(const sgqa_params* p, int64_t num_seqs, int64
   REQUIRE_PTR(sel_count, 4);
   REQUIRE_PTR(out, 16);
   if (gate != nullptr && !aligned(gate, 2)) return fail(SGQA_ERR_INVALID_ARGUMENT, "gate must be 2-byte aligned");
-  return launch_attn_decode_paged(p, num_seqs, q_pos0, nq, q, k_pool, v_pool, num_pages, page_table, max_pages, sel,
-                                  sel_count, gate, out, static_cast<cudaStream_t>(stream));
+  if (nq > kDecodeMaxNq) {  // the union plan of the prefill kernel lives in the workspace
+    const AttnWs w = attn_ws(p, num_seqs, nq);
+    if ((s = check_ws(workspace, workspace_bytes, w.bytes)) != SGQA_OK) return s;
+  }
+  KvSource kv;
+  kv.k = k_pool;
+  kv.v = v_pool;
+  kv.cap = kv.clen = cache_len;
+  kv.page_table = page_table;
+  kv.max_pages = max_pages;
+  kv.num_pages = num_pages;
+  return do_attn_kv(p, num_seqs, q_pos0, nq, q, kv, sel, sel_count, out, gate, workspace,
+                    static_cast<cudaStream_t>(stream));
 }
 
 sgqa_status sgqa_sparse_attn_noalloc(const sgqa_params* p, int64_t num_seqs, int64_t q_pos0, int64_t nq,
@@ -819,14 +865,30 @@ sgqa_status sgqa_sparse_attn_noalloc(const sgqa_params* p, int64_t num_seqs, int
   REQUIRE_PTR(sel, 4);
   REQUIRE_PTR(sel_count, 4);
   REQUIRE_PTR(out, 16);
-  const AttnWs w = attn_ws(p, num_seqs, nq);
-  if (w.bytes > SGQA_NOALLOC_SCRATCH_BYTES)
-    return fail(SGQA_ERR_UNSUPPORTED, "call needs %zu bytes of scratch; the static array holds %u",
-                w.bytes, (unsigned)SGQA_NOALLOC_SCRATCH_BYTES);
+  // Block size 8 takes the cluster-combined decode kernel, which keeps its
+  // split partials in shared memory: no scratch.  Other block sizes write
+  // split partials, which live in the static array.
   void* scratch = nullptr;
-  if ((s = noalloc_scratch(&scratch)) != SGQA_OK) return s;
+  if (p->block_size != 8) {
+    const AttnWs w = attn_ws(p, num_seqs, nq);
+    if (w.bytes > SGQA_NOALLOC_SCRATCH_BYTES)
+      return fail(SGQA_ERR_UNSUPPORTED, "call needs %zu bytes of scratch; the static array holds %u",
+                  w.bytes, (unsigned)SGQA_NOALLOC_SCRATCH_BYTES);
+    if ((s = noalloc_scratch(&scratch)) != SGQA_OK) return s;
+  }
   return do_attn(p, num_seqs, q_pos0, nq, q, cache_cap, cache_len, k_cache, v_cache, sel, sel_count, out, nullptr,
                  scratch, static_cast<cudaStream_t>(stream));
+}
+
+sgqa_status sgqa_set_wait_limit_ns(uint64_t ns) {
+  g_err.clear();
+  if (ns > sgqa::kWaitLimitNs)
+    return fail(SGQA_ERR_INVALID_ARGUMENT, "wait limit %llu ns is above the maximum of %llu ns",
+                (unsigned long long)ns, (unsigned long long)sgqa::kWaitLimitNs);
+  const uint64_t v = ns == 0 ? sgqa::kWaitLimitNs : ns;
+  cudaError_t e = cudaMemcpyToSymbol(sgqa::g_wait_limit_ns, &v, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "set wait limit");
+  return SGQA_OK;
 }
 
 sgqa_status sgqa_check(void* stream) {

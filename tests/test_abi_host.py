@@ -107,12 +107,13 @@ def test_null_and_range_checks_before_any_launch(lib, bd):
                                 dummy, dummy, dummy, odd, dummy, dummy, ctypes.c_size_t(1 << 30), st)
     assert rc == 1
     assert b"gate" in ctypes.string_at(lib.sgqa_last_error())
-    # paged decode: decode-sized calls with B = 8 only, a page table that covers cache_len
+    # paged: B = 8 only, a page table that covers cache_len, a workspace for more than 32 queries
     def paged(nq, max_pages, cache_len=4096, pt=dummy):
         return lib.sgqa_sparse_attn_paged(ctypes.byref(p), ctypes.c_int64(1), ctypes.c_int64(4000), ctypes.c_int64(nq),
                                           dummy, dummy, dummy, ctypes.c_int64(300), pt, ctypes.c_int64(max_pages),
-                                          ctypes.c_int64(cache_len), dummy, dummy, None, dummy, st)
-    assert paged(33, 256) == 2
+                                          ctypes.c_int64(cache_len), dummy, dummy, None, dummy, None,
+                                          ctypes.c_size_t(0), st)
+    assert paged(33, 256, cache_len=4033) == 3 and b"workspace" in ctypes.string_at(lib.sgqa_last_error())
     assert paged(4, 255) == 1 and b"max_pages" in ctypes.string_at(lib.sgqa_last_error())
     assert paged(4, 256, pt=ctypes.c_void_p(4096 + 2)) == 1
     p.block_size = 4
@@ -123,3 +124,22 @@ def test_null_and_range_checks_before_any_launch(lib, bd):
                           None, ctypes.c_int64(0), ctypes.c_int64(0), None, None, None, None, None, None, None,
                           None, None, None, ctypes.c_size_t(0), st)
     assert rc == 0
+
+
+def test_wait_limit_above_the_maximum_is_rejected(bd):
+    """Validated on the host before the device variable is touched (no GPU needed)."""
+    with pytest.raises(bd.SgqaError) as err:
+        bd.sgqa_set_wait_limit_ns(3_000_000_000)
+    assert err.value.code == 1
+
+
+def test_workspace_stays_bounded_at_1m_context(bd):
+    """Long rows never materialise FP32 score rows: the index workspace of an
+    8192-query chunk at a 1M-token context is the filtered path's lists, the
+    sample and the fallback's per-CTA rows, or the score rows of the longest
+    chunk that still takes them (16384 candidates), whichever is larger."""
+    b8 = bd.sgqa_workspace_size(bd.Params(), 1, 8192, 1 << 20)
+    rows_path = 8192 * 4 * 16384 * 4  # score rows of 16384 candidates
+    assert rows_path <= b8 < rows_path + (1 << 30), b8
+    b1 = bd.sgqa_workspace_size(bd.Params(block_size=1, topk=2048), 1, 8192, 1 << 20)
+    assert b1 < 6 * (1 << 30), b1
