@@ -46,10 +46,10 @@ METRIC = {
 # profiles/ give the commands and figures); None where no capture of the
 # current kernel exists.
 TRAFFIC = {
-    "prefill8k": 396776192,      # attn_tc_kernel, one launch (one 8192-query chunk)
-    "prefill128k": 2093507584,   # attn_tc_kernel, mean over the 16 chunk launches of one step
+    "prefill128k": 2101091360,   # attn_tc_kernel, mean over the 16 chunk launches of one step
+    "prefill8k": None,           # not captured for the current kernel
     "prefill1m": None,           # dominant stage: the index stage (several kernels, tensor/ALU bound)
-    "decode": 234981632,         # attn_decode_tma_kernel, one launch (16 sequences)
+    "decode": None,              # not captured for the current kernel
 }
 
 

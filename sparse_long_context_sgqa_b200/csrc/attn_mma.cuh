@@ -235,15 +235,17 @@ __device__ __forceinline__ void warp_load_q(WarpAttn& st, const __nv_bfloat16* q
   st.l[0] = st.l[1] = 0.f;
 }
 
-// tokmask bit p: token p of the staged step is attended by this warp's query.
-__device__ __forceinline__ void warp_attend_step(WarpAttn& st, uint32_t ks, uint32_t vs,
-                                                 uint32_t tokmask, float scale_log2, int lane) {
+// One 16-token step.  kaddr / vaddr: this lane's ldmatrix row addresses (K:
+// token 8 (mat >> 1) + mrow of the step, dims + 8 (mat & 1); V: token
+// 8 (mat & 1) + mrow, dims + 8 (mat >> 1)), so a step's 16 tokens may be any
+// staged rows.  tokmask bit p: token p of the step is attended by this warp's
+// query.
+__device__ __forceinline__ void warp_attend_at(WarpAttn& st, uint32_t kaddr, uint32_t vaddr,
+                                               uint32_t tokmask, float scale_log2, int lane) {
   float s[2][4];
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-  const int mrow = lane & 7, mat = lane >> 3;
   // QK^T: matrices (tok 0-7|8-15) x (dims 16s | 16s+8)
-  const uint32_t kaddr = ks + ((8 * (mat >> 1) + mrow) * kRowPad + 8 * (mat & 1)) * 2;
 #pragma unroll
   for (int kstep = 0; kstep < 12; ++kstep) {
     uint32_t b[4];
@@ -296,7 +298,6 @@ __device__ __forceinline__ void warp_attend_step(WarpAttn& st, uint32_t ks, uint
   pa[2] = pack_bf16x2(p[1][0], p[1][1]);
   pa[3] = pack_bf16x2(p[1][2], p[1][3]);
   // PV: trans matrices (tok 0-7 | 8-15) x (dims 16jj | 16jj+8)
-  const uint32_t vaddr = vs + ((8 * (mat & 1) + mrow) * kRowPad + 8 * (mat >> 1)) * 2;
 #pragma unroll
   for (int jj = 0; jj < 12; ++jj) {
     uint32_t b[4];
@@ -304,6 +305,14 @@ __device__ __forceinline__ void warp_attend_step(WarpAttn& st, uint32_t ks, uint
     mma_bf16_16816(st.o[2 * jj], pa, b[0], b[1]);
     mma_bf16_16816(st.o[2 * jj + 1], pa, b[2], b[3]);
   }
+}
+
+// The step over 16 consecutive staged tokens at ks / vs.
+__device__ __forceinline__ void warp_attend_step(WarpAttn& st, uint32_t ks, uint32_t vs,
+                                                 uint32_t tokmask, float scale_log2, int lane) {
+  const int mrow = lane & 7, mat = lane >> 3;
+  warp_attend_at(st, ks + ((8 * (mat >> 1) + mrow) * kRowPad + 8 * (mat & 1)) * 2,
+                 vs + ((8 * (mat & 1) + mrow) * kRowPad + 8 * (mat >> 1)) * 2, tokmask, scale_log2, lane);
 }
 
 // Final normalisation and bf16 store of one warp's 16 x 192 output.
@@ -324,14 +333,14 @@ __device__ __forceinline__ void warp_store_out(WarpAttn& st, __nv_bfloat16* o16,
   }
 }
 
-// Stage the K and V rows of 16 tokens (tok[p] < 0: zero row).  The calling
-// threads [0, nthreads) share the 2 x 16 x 24 sixteen-byte chunks.
+// Stage the K and V rows of ntok tokens (tok[p] < 0: zero row).  The calling
+// threads [0, nthreads) share the 2 x ntok x 24 sixteen-byte chunks.
 __device__ __forceinline__ void stage_tokens(uint32_t ks, uint32_t vs, const __nv_bfloat16* kc,
                                              const __nv_bfloat16* vc, const int64_t* tokbase,
-                                             int tid, int nthreads) {
-  for (int c = tid; c < 2 * kStepTok * 24; c += nthreads) {
-    const int which = c / (kStepTok * 24);
-    const int cc = c % (kStepTok * 24);
+                                             int tid, int nthreads, int ntok = kStepTok) {
+  for (int c = tid; c < 2 * ntok * 24; c += nthreads) {
+    const int which = c / (ntok * 24);
+    const int cc = c % (ntok * 24);
     const int p = cc / 24, part = cc % 24;
     const int64_t base = tokbase[p];
     const bool ok = base >= 0;
@@ -342,9 +351,16 @@ __device__ __forceinline__ void stage_tokens(uint32_t ks, uint32_t vs, const __n
 }
 
 // ---------------------------------------------------------------------------
-// Prefill: 8 warps = 8 adjacent queries sharing the union of their blocks.
+// Prefill for B in {1, 2, 4}: 8 warps = 8 adjacent queries share the union
+// of their selections, staged once per window of kWinTok tokens.  Each warp
+// compacts the window positions its own query selected (at B = 1 about a
+// fifth of a window) and runs its 16-token MMA steps over those rows only,
+// addressing them through ldmatrix's per-lane row pointers, so the MMA work
+// follows the query's own tokens instead of the union.
 // ---------------------------------------------------------------------------
-constexpr int kGroupedStages = 4;
+constexpr int kWinTok = 64;
+constexpr int kWinStages = 3;
+constexpr int kWinElems = kWinTok * kRowPad;  // one K or V window
 constexpr int kGroupedThreads = 256;
 
 template <int B>
@@ -355,9 +371,11 @@ attn_grouped_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
                     __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ gate, int64_t nq, int G,
                     int k, int64_t q_pos0, int64_t cache_cap, int64_t cache_len, float scale_log2) {
   extern __shared__ __align__(16) __nv_bfloat16 smem[];
-  __shared__ int64_t s_tok[kGroupedStages][kStepTok];
-  constexpr int E = kStepTok / B;  // union entries per step
+  __shared__ int64_t s_tok[kWinStages][kWinTok];
+  __shared__ uint8_t s_own[8][kWinTok];  // per warp: the window positions its query attends, compacted
+  constexpr int E = kWinTok / B;         // union entries per window
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int mrow = lane & 7, mat = lane >> 3;
   const int64_t nqb = (nq + 7) / 8;
   const int64_t unit = blockIdx.x;
   const int g = static_cast<int>(unit % G);
@@ -367,12 +385,12 @@ attn_grouped_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
   const bool qvalid = i < nq;
   const int64_t t = q_pos0 + (qvalid ? i : qb * 8);
   const int64_t t_first = q_pos0 + qb * 8;
-  const int64_t c0 = B * (t_first / B);  // current segment start
+  const int64_t c0 = B * (t_first / B);  // current segment start (the unit's current tokens lie in c0 .. c0 + 15)
   const int U = plan_count[unit];
   const int32_t* uid = plan_ids + unit * (8 * static_cast<int64_t>(k));
   const uint8_t* umask = plan_mask + unit * (8 * static_cast<int64_t>(k));
-  const int n_union_steps = (U + E - 1) / E;
-  const int n_steps = n_union_steps + 1;
+  const int n_union_win = (U + E - 1) / E;
+  const int n_win = n_union_win + 1;
   const int64_t row_stride = static_cast<int64_t>(G) * kD;
   const __nv_bfloat16* kseq = kc + seq * cache_cap * row_stride + g * kD;
   const __nv_bfloat16* vseq = vc + seq * cache_cap * row_stride + g * kD;
@@ -380,55 +398,70 @@ attn_grouped_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
   WarpAttn st;
   warp_load_q(st, q + ((seq * nq + (qvalid ? i : 0)) * G + g) * kHg * kD, lane);
 
-  auto token_of = [&](int step, int p) -> int64_t {
-    if (step < n_union_steps) {
-      const int e = step * E + p / B;
+  auto token_of = [&](int win, int p) -> int64_t {
+    if (win < n_union_win) {
+      const int e = win * E + p / B;
       if (e >= U) return -1;
       const int64_t tk = static_cast<int64_t>(uid[e]) * B + (p % B);
       return (tk >= 0 && tk < cache_len) ? tk : -1;
     }
     const int64_t s = c0 + p;
-    return s < cache_len ? s : -1;
+    return (p < 16 && s < cache_len) ? s : -1;
   };
-  auto issue = [&](int step) {
-    const int stage = step % kGroupedStages;
-    if (tid < kStepTok) {
-      const int64_t tk = token_of(step, tid);
+  auto issue = [&](int win) {
+    const int stage = win % kWinStages;
+    if (tid < kWinTok) {
+      const int64_t tk = token_of(win, tid);
       s_tok[stage][tid] = tk >= 0 ? tk * row_stride : -1;
     }
     __syncthreads();
-    const uint32_t ks = smem_u32(smem + (2 * stage) * kStageElems);
-    const uint32_t vs = smem_u32(smem + (2 * stage + 1) * kStageElems);
-    stage_tokens(ks, vs, kseq, vseq, s_tok[stage], tid, kGroupedThreads);
+    const uint32_t ks = smem_u32(smem + (2 * stage) * kWinElems);
+    const uint32_t vs = smem_u32(smem + (2 * stage + 1) * kWinElems);
+    stage_tokens(ks, vs, kseq, vseq, s_tok[stage], tid, kGroupedThreads, kWinTok);
   };
   // prologue
-  for (int sidx = 0; sidx < kGroupedStages - 1; ++sidx) {
-    if (sidx < n_steps) issue(sidx);
+  for (int w = 0; w < kWinStages - 1; ++w) {
+    if (w < n_win) issue(w);
     cp_async_commit();
   }
   const int64_t tcur0 = B * (t / B);
-  for (int step = 0; step < n_steps; ++step) {
-    cp_async_wait<kGroupedStages - 2>();
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int win = 0; win < n_win; ++win) {
+    cp_async_wait<kWinStages - 2>();
     __syncthreads();
-    // token mask for this warp's query
-    uint32_t tm = 0;
-    if (step < n_union_steps) {
-      if (lane < kStepTok) {
-        const int e = step * E + lane / B;
-        tm = (e < U && ((umask[e] >> warp) & 1u)) ? 1u : 0u;
+    // the window positions this warp's query attends (lane and lane + 32)
+    bool own0, own1;
+    if (win < n_union_win) {
+      const int e0 = win * E + lane / B, e1 = win * E + (lane + 32) / B;
+      own0 = e0 < U && ((umask[e0] >> warp) & 1u);
+      own1 = e1 < U && ((umask[e1] >> warp) & 1u);
+    } else {
+      const int64_t s0 = c0 + lane;
+      own0 = lane < 16 && s0 >= tcur0 && s0 <= t;
+      own1 = false;
+    }
+    const uint32_t m0 = __ballot_sync(0xffffffffu, own0), m1 = __ballot_sync(0xffffffffu, own1);
+    const int n0 = __popc(m0), n_own = n0 + __popc(m1);
+    if (own0) s_own[warp][__popc(m0 & lt)] = static_cast<uint8_t>(lane);
+    if (own1) s_own[warp][n0 + __popc(m1 & lt)] = static_cast<uint8_t>(lane + 32);
+    __syncwarp();
+    if (qvalid) {
+      const int stage = win % kWinStages;
+      const uint32_t ks = smem_u32(smem + (2 * stage) * kWinElems);
+      const uint32_t vs = smem_u32(smem + (2 * stage + 1) * kWinElems);
+      for (int sub = 0; sub < n_own; sub += kStepTok) {
+        const int left = n_own - sub;
+        const uint32_t tm = left >= kStepTok ? 0xFFFFu : ((1u << left) - 1u);
+        // rows past the compacted list repeat its last row; their scores are masked
+        const int rk = s_own[warp][sub + min(8 * (mat >> 1) + mrow, left - 1)];
+        const int rv = s_own[warp][sub + min(8 * (mat & 1) + mrow, left - 1)];
+        warp_attend_at(st, ks + (rk * kRowPad + 8 * (mat & 1)) * 2, vs + (rv * kRowPad + 8 * (mat >> 1)) * 2, tm,
+                       scale_log2, lane);
       }
-    } else if (lane < kStepTok) {
-      const int64_t s = c0 + lane;
-      tm = (s >= tcur0 && s <= t) ? 1u : 0u;
     }
-    tm = __ballot_sync(0xffffffffu, tm) & 0xFFFFu;
-    if (qvalid && tm != 0) {
-      const int stage = step % kGroupedStages;
-      warp_attend_step(st, smem_u32(smem + (2 * stage) * kStageElems),
-                       smem_u32(smem + (2 * stage + 1) * kStageElems), tm, scale_log2, lane);
-    }
-    const int nxt = step + kGroupedStages - 1;
-    if (nxt < n_steps) issue(nxt);
+    __syncwarp();  // s_own is rewritten for the next window
+    const int nxt = win + kWinStages - 1;
+    if (nxt < n_win) issue(nxt);
     else __syncthreads();  // keep the barrier count uniform with issue()
     cp_async_commit();
   }

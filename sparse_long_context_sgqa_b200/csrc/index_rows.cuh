@@ -19,6 +19,8 @@
 // This form suits decode (one query per sequence, a few MB of scores) and is
 // the general fallback; long prefill uses the fused streaming kernel.
 #pragma once
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 
 namespace sgqa {
@@ -430,98 +432,137 @@ topk_rows_list_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq
 
 namespace sgqa {
 
-// Exact E4M3 -> BF16 widening of two codes by integer operations: the
-// hardware conversion to FP16 is exact, and every E4M3 value is an FP16
-// normal (or zero) whose 10-bit mantissa has only its top 3 bits set, so the
-// BF16 pattern is the FP16 one with the exponent rebiased (15 -> 127) and the
-// mantissa shifted to 7 bits.  (Store codes are finite: the merge saturates.)
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2_int(uint16_t v) {
+// Two E4M3 codes widened to FP16 (exact: every E4M3 value is an FP16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
   const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v), __NV_E4M3);
-  const uint32_t x = static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
-  const uint32_t mag = x & 0x7FFF7FFFu;
-  const uint32_t r = ((mag >> 3) & 0x0FFF0FFFu) + 0x38003800u;
-  return (r & __vcmpne2(mag, 0u)) | (x & 0x80008000u);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
 }
+
+// 2^e as a float, e in [-126, 127].
+__device__ __forceinline__ float exp2i(int e) { return __uint_as_float(static_cast<uint32_t>(127 + e) << 23); }
 
 // Decode scores: one CTA per (sequence and query, 512 candidates) scores the
 // query's four groups at once (B operand = 4 groups x 8 heads = 32 columns,
-// resident in registers), reading the E4M3 store directly.  The MMA's k index
-// is permuted (the same permutation on both operands leaves every dot product
-// unchanged) so that each lane's A fragments for all four k-steps come from
-// one contiguous 16-byte piece of a key row: logical k = 16 s + 8 h + 2 j + e
-// is dimension 16 j + 4 s + 2 h + e (lane j = lane % 4).  A warp's strip of
-// 16 candidates is then two fully used 512-byte runs of the store, and each
-// warp issues the loads of its four strips before any MMA.
+// resident in registers), reading the E4M3 store directly.
+//
+// The MMA runs in FP16: the E4M3 codes convert to FP16 exactly with one
+// instruction per pair.  Each head's query row is scaled by a power of two
+// 2^s_h that brings its largest magnitude into [2^14, 2^15) and rounded to
+// FP16, which is exact (a BF16 value has 8 significant bits, FP16 11) for
+// every element down to 2^-28 of the head's largest; the head's weight
+// carries 2^-s_h, so sum_h w_h * ReLU(dot_h) is unchanged (the scale is a
+// power of two and positive).
+//
+// The MMA's k index is permuted (the same permutation on both operands leaves
+// every dot product unchanged) so that each lane's A fragments for all four
+// k-steps come from one contiguous 16-byte piece of a key row: logical
+// k = 16 s + 8 h + 2 j + e is dimension 16 j + 4 s + 2 h + e (lane j =
+// lane % 4).  A warp's strip of 16 candidates is then two fully used
+// 512-byte runs of the store, and each warp issues the loads of its four
+// strips before any MMA.
 constexpr int kDecScoreThreads = 256;
-constexpr int kDecScoreCand = 512;  // candidates per CTA: 8 warps x 4 strips of 16
+constexpr int kDecScoreDepth = 4;  // strips of 16 candidates each warp has in flight
 
-__global__ void __launch_bounds__(kDecScoreThreads)
+// One (sequence and query) per blockIdx.y; blockIdx.x takes a contiguous
+// range of `per_cta` candidates, which its warps walk strip by strip (warp w:
+// strips w, w + 8, ...), the key rows of the next kDecScoreDepth strips always
+// in flight while the current one is computed.
+__global__ void __launch_bounds__(kDecScoreThreads, 2)
 index_score_decode_kernel(const __nv_bfloat16* __restrict__ idx_q, const float* __restrict__ idx_w,
                           const uint8_t* __restrict__ store, float* __restrict__ scores, int64_t nq,
-                          int64_t q_pos0, int B, int64_t rpad, int64_t key_rows) {
-  constexpr int G = 4, H = 8, Di = 64, STRIPS = kDecScoreCand / 16 / (kDecScoreThreads / 32);
+                          int64_t q_pos0, int B, int64_t rpad, int64_t key_rows, int64_t per_cta,
+                          int32_t* __restrict__ list_count) {
+  constexpr int G = 4, H = 8, Di = 64, W = kDecScoreThreads / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int j = lane & 3, rl = lane >> 2;
+  // the select kernel that follows lists the rows it leaves to the radix kernel
+  if (list_count != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *list_count = 0;
   const int64_t sq = blockIdx.y;  // seq * nq + i
   const int64_t i = sq % nq, seq = sq / nq;
   const int64_t ncand = (q_pos0 + i) / B;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kDecScoreCand;
-  if (c0 >= ncand) return;
-  // the key rows of this warp's strips, 16 bytes per lane and row, all in flight
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * per_cta;
+  const int64_t c1 = min(ncand, c0 + per_cta);
+  if (c0 >= c1) return;
+  const int nstrips = static_cast<int>((c1 - c0 + 15) / 16);
+  const int mine = nstrips > warp ? (nstrips - warp + W - 1) / W : 0;  // strips of this warp
+  // key rows of this warp's strip number s (s-th of its own): 16 bytes per lane and row
   const uint8_t* kb = store + seq * key_rows * Di + 16 * j;
-  uint4 ka[STRIPS], kbb[STRIPS];
+  auto load_strip = [&](int s, uint4& a, uint4& b) {
+    const int64_t ra = c0 + 16 * (warp + static_cast<int64_t>(W) * s) + rl, rb = ra + 8;
+    a = (s < mine && ra < key_rows) ? __ldg(reinterpret_cast<const uint4*>(kb + ra * Di)) : make_uint4(0u, 0u, 0u, 0u);
+    b = (s < mine && rb < key_rows) ? __ldg(reinterpret_cast<const uint4*>(kb + rb * Di)) : make_uint4(0u, 0u, 0u, 0u);
+  };
+  uint4 ka[kDecScoreDepth], kbb[kDecScoreDepth];
 #pragma unroll
-  for (int st = 0; st < STRIPS; ++st) {
-    const int64_t ra = c0 + 16 * (warp + (kDecScoreThreads / 32) * st) + rl, rb = ra + 8;
-    ka[st] = ra < key_rows ? __ldg(reinterpret_cast<const uint4*>(kb + ra * Di)) : make_uint4(0u, 0u, 0u, 0u);
-    kbb[st] = rb < key_rows ? __ldg(reinterpret_cast<const uint4*>(kb + rb * Di)) : make_uint4(0u, 0u, 0u, 0u);
-  }
-  // B fragments (column n = head lane / 4 of group g): 16 consecutive query
-  // values 16 j .. 16 j + 15 of that head; k-step s takes pairs 2 s and 2 s + 1
+  for (int d = 0; d < kDecScoreDepth; ++d) load_strip(d, ka[d], kbb[d]);
+  // B fragments (column n = head rl of group g): the scaled FP16 values of
+  // dimensions 16 j .. 16 j + 15 of that head; k-step s takes pairs 2 s, 2 s + 1
   uint32_t bf[G][8];
   float wv[G][2];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     const uint4* qrow = reinterpret_cast<const uint4*>(idx_q + ((sq * G + g) * H + rl) * Di + 16 * j);
     const uint4 q0 = __ldg(qrow), q1 = __ldg(qrow + 1);
-    bf[g][0] = q0.x; bf[g][1] = q0.y; bf[g][2] = q0.z; bf[g][3] = q0.w;
-    bf[g][4] = q1.x; bf[g][5] = q1.y; bf[g][6] = q1.z; bf[g][7] = q1.w;
-    const float2 w2 = __ldg(reinterpret_cast<const float2*>(idx_w + (sq * G + g) * H + 2 * j));
-    wv[g][0] = w2.x;
-    wv[g][1] = w2.y;
-  }
+    const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    float mx = 0.f;
 #pragma unroll
-  for (int st = 0; st < STRIPS; ++st) {
-    const int64_t ra = c0 + 16 * (warp + (kDecScoreThreads / 32) * st) + rl, rb = ra + 8;
-    // A fragments: pair m of the lane's 16 codes = dimensions 16 j + 2 m, + 1
-    uint32_t pa[8], pb[8];
-    const uint32_t wa[4] = {ka[st].x, ka[st].y, ka[st].z, ka[st].w};
-    const uint32_t wb[4] = {kbb[st].x, kbb[st].y, kbb[st].z, kbb[st].w};
+    for (int m = 0; m < 8; ++m)
+      mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(qw[m] << 16)), fabsf(__uint_as_float(qw[m] & 0xFFFF0000u))));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    // s_h = 141 - biased exponent of the head's largest magnitude (clamped)
+    const int eb = static_cast<int>((__float_as_uint(mx) >> 23) & 0xFFu);
+    const int sh = min(max(141 - eb, -110), 110);
+    const float up = exp2i(sh), down = exp2i(-sh);
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      pa[2 * m] = e4m3x2_to_bf16x2_int(static_cast<uint16_t>(wa[m] & 0xFFFFu));
-      pa[2 * m + 1] = e4m3x2_to_bf16x2_int(static_cast<uint16_t>(wa[m] >> 16));
-      pb[2 * m] = e4m3x2_to_bf16x2_int(static_cast<uint16_t>(wb[m] & 0xFFFFu));
-      pb[2 * m + 1] = e4m3x2_to_bf16x2_int(static_cast<uint16_t>(wb[m] >> 16));
+    for (int m = 0; m < 8; ++m) {
+      const __half2 h2 = __floats2half2_rn(__uint_as_float(qw[m] << 16) * up, __uint_as_float(qw[m] & 0xFFFF0000u) * up);
+      bf[g][m] = *reinterpret_cast<const uint32_t*>(&h2);
     }
+    // this lane's accumulator columns are heads 2 j and 2 j + 1: their weights carry 2^-s
+    const float d0 = __shfl_sync(0xffffffffu, down, 8 * j), d1 = __shfl_sync(0xffffffffu, down, 8 * j + 4);
+    const float2 w2 = __ldg(reinterpret_cast<const float2*>(idx_w + (sq * G + g) * H + 2 * j));
+    wv[g][0] = w2.x * d0;
+    wv[g][1] = w2.y * d1;
+  }
+  for (int s0 = 0; s0 < mine; s0 += kDecScoreDepth) {
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int d = 0; d < kDecScoreDepth; ++d) {
+      const int s = s0 + d;
+      if (s < mine) {
+        const int64_t ra = c0 + 16 * (warp + static_cast<int64_t>(W) * s) + rl, rb = ra + 8;
+        // A fragments: pair m of the lane's 16 codes = dimensions 16 j + 2 m, + 1
+        uint32_t pa[8], pb[8];
+        const uint32_t wa[4] = {ka[d].x, ka[d].y, ka[d].z, ka[d].w};
+        const uint32_t wb[4] = {kbb[d].x, kbb[d].y, kbb[d].z, kbb[d].w};
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        const uint32_t af[4] = {pa[2 * ks], pb[2 * ks], pa[2 * ks + 1], pb[2 * ks + 1]};
-        mma_bf16_16816(acc, af, bf[g][2 * ks], bf[g][2 * ks + 1]);
-      }
-      float sa = wv[g][0] * fmaxf(acc[0], 0.f) + wv[g][1] * fmaxf(acc[1], 0.f);
-      float sb = wv[g][0] * fmaxf(acc[2], 0.f) + wv[g][1] * fmaxf(acc[3], 0.f);
-      sa += __shfl_xor_sync(0xffffffffu, sa, 1);
-      sa += __shfl_xor_sync(0xffffffffu, sa, 2);
-      sb += __shfl_xor_sync(0xffffffffu, sb, 1);
-      sb += __shfl_xor_sync(0xffffffffu, sb, 2);
-      if (j == 0) {
-        float* srow = scores + (sq * G + g) * rpad;
-        if (ra < rpad) srow[ra] = sa;
-        if (rb < rpad) srow[rb] = sb;
+        for (int m = 0; m < 4; ++m) {
+          pa[2 * m] = e4m3x2_to_f16x2(static_cast<uint16_t>(wa[m] & 0xFFFFu));
+          pa[2 * m + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(wa[m] >> 16));
+          pb[2 * m] = e4m3x2_to_f16x2(static_cast<uint16_t>(wb[m] & 0xFFFFu));
+          pb[2 * m + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(wb[m] >> 16));
+        }
+        load_strip(s + kDecScoreDepth, ka[d], kbb[d]);  // the strip that reuses this slot
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint32_t af[4] = {pa[2 * ks], pb[2 * ks], pa[2 * ks + 1], pb[2 * ks + 1]};
+            mma_f16_16816(acc, af, bf[g][2 * ks], bf[g][2 * ks + 1]);
+          }
+          float sa = wv[g][0] * fmaxf(acc[0], 0.f) + wv[g][1] * fmaxf(acc[1], 0.f);
+          float sb = wv[g][0] * fmaxf(acc[2], 0.f) + wv[g][1] * fmaxf(acc[3], 0.f);
+          sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+          sa += __shfl_xor_sync(0xffffffffu, sa, 2);
+          sb += __shfl_xor_sync(0xffffffffu, sb, 1);
+          sb += __shfl_xor_sync(0xffffffffu, sb, 2);
+          if (j == 0) {
+            float* srow = scores + (sq * G + g) * rpad;
+            if (ra < rpad) srow[ra] = sa;
+            if (rb < rpad) srow[rb] = sb;
+          }
+        }
       }
     }
   }
@@ -751,6 +792,336 @@ topk_rows_reg_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq,
     __syncthreads();
   }
   topk_reg_readout(keep_bits, sums, tid, lane, warp, k, out, sel_count, row);
+}
+
+// ---------------------------------------------------------------------------
+// Exact top-k of decode rows (at most kDecSelCtas * 4096 candidates) by a
+// thread-block cluster of kDecSelCtas CTAs per row, so that a few long rows
+// use many SMs.  CTA c owns candidates [4096 c, 4096 c + 4096), 16 per thread
+// in registers.  The cluster agrees on the row's extreme scores, builds one
+// linear 2048-bin histogram between them (each CTA its own, summed through
+// distributed shared memory), and finds the bin holding the k-th largest;
+// better bins are taken, the boundary bin's entries are gathered to CTA 0 and
+// ranked exactly (score, then smaller id) by one warp, or -- when they all
+// share one score -- taken in id order.  Each CTA writes its taken ids in
+// ascending order at the offset the lower CTAs' counts give.  A boundary
+// with more distinct entries than the gather buffer holds lists the row for
+// the radix kernel (topk_rows_list_kernel), which then rewrites it.
+// ---------------------------------------------------------------------------
+constexpr int kDecSelCtas = 8;
+constexpr int kDecSelThreads = 256;
+constexpr int kDecSelPer = 16;
+constexpr int kDecSelSlice = kDecSelThreads * kDecSelPer;  // 4096 candidates per CTA
+constexpr int kDecSelBins = 2048;
+constexpr int kDecSelBnd = 512;                            // boundary entries one CTA holds
+constexpr int kDecSelGather = 2048;                        // boundary entries CTA 0 ranks
+
+struct DecSelSmem {
+  uint32_t hist[kDecSelBins];    // this CTA's histogram (later warp_select's scratch in CTA 0)
+  uint32_t slot[kDecSelBins / kDecSelCtas];  // the cluster's total of bins [256 c, 256 c + 256)
+  uint32_t tot[kDecSelBins];     // the cluster's total histogram
+  uint2 bnd[kDecSelBnd];         // this CTA's boundary entries (key, id)
+  uint2 gath[kDecSelGather];     // CTA 0: every CTA's boundary entries
+  uint32_t bits[kDecSelSlice / 32];
+  uint32_t wsum[kDecSelThreads / 32];
+  float wmx[kDecSelThreads / 32], wmn[kDecSelThreads / 32];
+  float mx, mn, gmx, gmn;
+  uint32_t nb, nabove, bstar, rem, cstar;
+  // written by CTA 0 into every CTA: how to treat the boundary and where this CTA's ids go
+  uint32_t mode, theta, id_cut, take, off;
+};
+
+__global__ void __launch_bounds__(kDecSelThreads)
+topk_decode_cluster_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int G, int64_t q_pos0, int B,
+                           int k, int32_t* __restrict__ sel, int32_t* __restrict__ sel_count,
+                           int32_t* __restrict__ list, int32_t* __restrict__ list_count) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  __shared__ DecSelSmem sm;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = static_cast<int>(cluster.block_rank());
+  const int64_t row = blockIdx.x / kDecSelCtas;
+  const int64_t i = (row / G) % nq;
+  const int n = static_cast<int>((q_pos0 + i) / B);
+  int32_t* out = sel + row * k;
+  if (n <= k) {  // every CTA of the cluster leaves here together
+    if (c == 0) {
+      for (int x = tid; x < k; x += kDecSelThreads) out[x] = x < n ? x : -1;
+      if (tid == 0) sel_count[row] = n;
+    }
+    return;
+  }
+  const int base = c * kDecSelSlice;
+  const float* srow = scores + row * rpad + base;
+  float v[kDecSelPer];
+  float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+  for (int u = 0; u < kDecSelPer; ++u) {
+    const int jl = tid + kDecSelThreads * u;
+    v[u] = base + jl < n ? srow[jl] : -INFINITY;
+    if (base + jl < n) {
+      mx = fmaxf(mx, v[u]);
+      mn = fminf(mn, v[u]);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+  }
+  if (lane == 0) {
+    sm.wmx[warp] = mx;
+    sm.wmn[warp] = mn;
+  }
+  for (int b = tid; b < kDecSelBins; b += kDecSelThreads) sm.hist[b] = 0u;
+  for (int w = tid; w < kDecSelSlice / 32; w += kDecSelThreads) sm.bits[w] = 0u;
+  if (tid == 0) {
+    sm.nb = 0;
+    sm.nabove = 0;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float a = lane < kDecSelThreads / 32 ? sm.wmx[lane] : -INFINITY;
+    float b = lane < kDecSelThreads / 32 ? sm.wmn[lane] : INFINITY;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      b = fminf(b, __shfl_xor_sync(0xffffffffu, b, o));
+    }
+    if (lane == 0) {
+      sm.mx = a;
+      sm.mn = b;
+    }
+  }
+  cluster.sync();  // (1) every CTA's extremes
+  if (warp == 0) {  // one round trip: lane r reads CTA r's
+    float a = -INFINITY, b = INFINITY;
+    if (lane < kDecSelCtas) {
+      const DecSelSmem* o = cluster.map_shared_rank(&sm, lane);
+      a = o->mx;
+      b = o->mn;
+    }
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) {
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      b = fminf(b, __shfl_xor_sync(0xffffffffu, b, o));
+    }
+    if (lane == 0) {
+      sm.gmx = a;
+      sm.gmn = b;
+    }
+  }
+  __syncthreads();
+  const float gmx = sm.gmx, width = gmx - sm.gmn;
+  const float scale = width > 0.f ? (kDecSelBins - 0.5f) / width : 0.f;
+  // bins best first; both steps round monotonically
+  auto bin_of = [&](float x) -> int { return min(static_cast<int>(__fmul_rn(__fsub_rn(gmx, x), scale)), kDecSelBins - 1); };
+#pragma unroll
+  for (int u = 0; u < kDecSelPer; ++u)
+    if (base + tid + kDecSelThreads * u < n) atomicAdd(&sm.hist[bin_of(v[u])], 1u);
+  cluster.sync();  // (2) every CTA's histogram
+  {  // CTA c sums its slot of bins over the cluster (independent loads)
+    constexpr int per = kDecSelBins / kDecSelCtas;
+    uint32_t h[kDecSelCtas];
+#pragma unroll
+    for (int r = 0; r < kDecSelCtas; ++r) h[r] = cluster.map_shared_rank(&sm, r)->hist[per * c + tid];
+    uint32_t t = 0;
+#pragma unroll
+    for (int r = 0; r < kDecSelCtas; ++r) t += h[r];
+    sm.slot[tid] = t;
+  }
+  cluster.sync();  // (3) every slot
+  {
+    uint32_t h[kDecSelCtas];
+#pragma unroll
+    for (int r = 0; r < kDecSelCtas; ++r) h[r] = cluster.map_shared_rank(&sm, r)->slot[tid];
+#pragma unroll
+    for (int r = 0; r < kDecSelCtas; ++r) sm.tot[(kDecSelBins / kDecSelCtas) * r + tid] = h[r];
+  }
+  __syncthreads();
+  {  // thread t owns bins 8 t .. 8 t + 7: the bin in which the running count reaches k
+    uint32_t loc[8], sum = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      loc[q] = sm.tot[8 * tid + q];
+      sum += loc[q];
+    }
+    uint32_t x = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) sm.wsum[warp] = x;
+    __syncthreads();
+    uint32_t acc = x - sum;
+    for (int w = 0; w < warp; ++w) acc += sm.wsum[w];
+    const uint32_t kk = static_cast<uint32_t>(k);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (acc < kk && kk <= acc + loc[q]) {
+        sm.bstar = 8 * tid + q;
+        sm.rem = kk - acc;
+        sm.cstar = loc[q];
+      }
+      acc += loc[q];
+    }
+  }
+  __syncthreads();
+  const int bstar = static_cast<int>(sm.bstar);
+  const uint32_t rem = sm.rem, cstar = sm.cstar;
+  // better bins are taken (counted); the boundary bin's entries are collected
+  uint32_t above = 0;
+#pragma unroll
+  for (int u = 0; u < kDecSelPer; ++u) {
+    const int jl = tid + kDecSelThreads * u;
+    if (base + jl < n) {
+      const int b = bin_of(v[u]);
+      if (b < bstar) {
+        atomicOr(&sm.bits[jl >> 5], 1u << (jl & 31));
+        ++above;
+      } else if (b == bstar) {
+        const uint32_t pos = atomicAdd(&sm.nb, 1u);
+        if (pos < kDecSelBnd) sm.bnd[pos] = make_uint2(score_key(v[u]), static_cast<uint32_t>(base + jl));
+      }
+    }
+  }
+  above = __reduce_add_sync(0xffffffffu, above);
+  if (lane == 0 && above) atomicAdd(&sm.nabove, above);
+  cluster.sync();  // (4) every CTA's counts and boundary entries
+  if (c == 0 && warp == 0) {
+    // CTA 0 decides the boundary and every CTA's output offset, one round trip per step
+    uint32_t nbr = 0, nab = 0;
+    if (lane < kDecSelCtas) {
+      const DecSelSmem* o = cluster.map_shared_rank(&sm, lane);
+      nbr = o->nb;
+      nab = o->nabove;
+    }
+    const bool overflow = __any_sync(0xffffffffu, nbr > static_cast<uint32_t>(kDecSelBnd));
+    const uint32_t nbc = min(nbr, static_cast<uint32_t>(kDecSelBnd));
+    uint32_t bstart = nbc;  // exclusive prefix of the stored boundary counts over CTAs 0..lane-1
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, bstart, o);
+      if (lane >= o) bstart += y;
+    }
+    const uint32_t total = __shfl_sync(0xffffffffu, bstart, kDecSelCtas - 1);
+    bstart -= nbc;
+    uint32_t mode = 0;  // 0: ranked (or all taken); 1: equal scores, taken in id order; 2: the radix kernel
+    uint32_t theta = 0, id_cut = 0xFFFFFFFFu;
+    if (overflow) {
+      mode = 2;  // a CTA's boundary entries did not fit its buffer
+    } else if (cstar > rem) {
+      if (total > kDecSelGather) {
+        mode = 2;
+      } else {
+        // gather: entry e < total lives in the CTA r whose [bstart, bstart + nbc) holds it
+        for (uint32_t e0 = 0; e0 < total; e0 += 32) {
+          const uint32_t e = e0 + lane;
+          int r = 0;
+#pragma unroll
+          for (int q = 1; q < kDecSelCtas; ++q) r += e >= __shfl_sync(0xffffffffu, bstart, q) ? 1 : 0;
+          const uint32_t rs = __shfl_sync(0xffffffffu, bstart, r);
+          if (e < total) sm.gath[e] = cluster.map_shared_rank(&sm, r)->bnd[e - rs];
+        }
+        __syncwarp();
+        uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+        for (uint32_t e = lane; e < total; e += 32) {
+          kmin = min(kmin, sm.gath[e].x);
+          kmax = max(kmax, sm.gath[e].x);
+        }
+        kmin = __reduce_min_sync(0xffffffffu, kmin);
+        kmax = __reduce_max_sync(0xffffffffu, kmax);
+        if (kmin == kmax) {
+          mode = 1;
+        } else {
+          warp_select(sm.gath, static_cast<int>(total), static_cast<int>(rem), sm.hist, theta, id_cut);
+        }
+      }
+    }
+    // boundary entries each CTA keeps: all, the first rem in CTA order (mode 1), or by (theta, id_cut)
+    uint32_t take = 0;
+    if (mode == 1 || cstar <= rem) {
+      take = bstart >= rem ? 0u : min(nbc, rem - bstart);
+    } else if (mode == 0) {
+      for (uint32_t e0 = 0; e0 < total; e0 += 32) {
+        const uint32_t e = e0 + lane;
+        const bool kp = e < total && kept(sm.gath[e], theta, id_cut);
+        int r = 0;
+#pragma unroll
+        for (int q = 1; q < kDecSelCtas; ++q) r += e >= __shfl_sync(0xffffffffu, bstart, q) ? 1 : 0;
+        // count kept entries per CTA: lane r sums the ballots of entries of CTA r
+#pragma unroll
+        for (int q = 0; q < kDecSelCtas; ++q) {
+          const uint32_t bq = __ballot_sync(0xffffffffu, kp && r == q);
+          if (lane == q) take += __popc(bq);
+        }
+      }
+    }
+    uint32_t cnt = nab + take, off = cnt;  // ids this CTA writes; exclusive prefix = its offset
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, off, o);
+      if (lane >= o) off += y;
+    }
+    off -= cnt;
+    if (lane < kDecSelCtas) {
+      DecSelSmem* o = cluster.map_shared_rank(&sm, lane);
+      o->mode = mode;
+      o->theta = theta;
+      o->id_cut = id_cut;
+      o->take = take;
+      o->off = off;
+    }
+    if (mode == 2 && lane == 0) list[atomicAdd(list_count, 1)] = static_cast<int32_t>(row);
+  }
+  cluster.sync();  // (5) the decision is in every CTA; nothing reads another CTA's memory after this
+  if (sm.mode == 2) return;  // every CTA of the cluster leaves here together; the radix kernel writes the row
+  {
+    const uint32_t mine = min(sm.nb, static_cast<uint32_t>(kDecSelBnd));
+    if (sm.mode == 0 && cstar > rem) {
+      const uint32_t theta = sm.theta, id_cut = sm.id_cut;
+      for (uint32_t e = tid; e < mine; e += kDecSelThreads) {
+        const uint2 x = sm.bnd[e];
+        if (kept(x, theta, id_cut)) atomicOr(&sm.bits[(x.y - base) >> 5], 1u << ((x.y - base) & 31));
+      }
+    } else {
+      // all boundary entries, or the `take` smallest ids of this CTA's (equal scores)
+      const uint32_t take = sm.take;
+      for (uint32_t e = tid; e < mine; e += kDecSelThreads) {
+        const uint32_t id = sm.bnd[e].y;
+        uint32_t rank = 0;
+        if (take < mine)
+          for (uint32_t f = 0; f < mine; ++f) rank += sm.bnd[f].y < id;
+        if (rank < take) atomicOr(&sm.bits[(id - base) >> 5], 1u << ((id - base) & 31));
+      }
+    }
+  }
+  __syncthreads();
+  // ascending readout: thread t < 128 owns bitmap word t
+  const uint32_t wb = tid < kDecSelSlice / 32 ? sm.bits[tid] : 0u;
+  const uint32_t cw = __popc(wb);
+  uint32_t x = cw;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sm.wsum[warp] = x;
+  __syncthreads();
+  uint32_t pos = x - cw + sm.off;
+  for (int w = 0; w < warp; ++w) pos += sm.wsum[w];
+  uint32_t bw = wb;
+  while (bw) {
+    const int b = __ffs(bw) - 1;
+    bw &= bw - 1;
+    if (pos < static_cast<uint32_t>(k)) out[pos] = base + 32 * tid + b;
+    ++pos;
+  }
+  if (c == kDecSelCtas - 1 && tid == kDecSelThreads - 1) {
+    sel_count[row] = k;
+    if (pos != static_cast<uint32_t>(k)) report(kDevBounds);
+  }
 }
 
 }  // namespace sgqa

@@ -76,6 +76,9 @@ float softmax_scale(const sgqa_params* p) {
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Streaming multiprocessors of a B200 (grid sizing).
+constexpr int64_t kSmCount = 148;
+
 // Queries per sequence below which attention runs split-K per query.
 constexpr int64_t kDecodeMaxNq = 32;
 
@@ -425,12 +428,42 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
     launch_score(sgqa::kScoreRows, sgqa::ScoreOut{scores, w.rpad, 0, nullptr, nullptr, nullptr, 0});
     SGQA_LAUNCH_CHECK("index_score_tc_kernel");
   } else if (rneed > 0 && G == 4 && H == 8) {
-    // few queries: one CTA per (query, 128 candidates) scores all four groups from the E4M3 store
-    dim3 grid(static_cast<unsigned>((rneed + sgqa::kDecScoreCand - 1) / sgqa::kDecScoreCand),
-              static_cast<unsigned>(S * nq));
+    // few queries: the (query, candidate range) CTAs score all four groups from the E4M3 store; two
+    // CTAs per SM over the whole launch, each range at least 1024 candidates and a whole number of strips
+    const int64_t qrows = S * nq;
+    if (qrows > 65535) return fail(SGQA_ERR_UNSUPPORTED, "decode index grid too large");
+    const int64_t want = std::max<int64_t>(1, (2 * kSmCount + qrows - 1) / qrows);
+    int64_t per_cta = (rneed + want - 1) / want;
+    per_cta = std::max<int64_t>(1024, (per_cta + 15) / 16 * 16);
+    dim3 grid(static_cast<unsigned>((rneed + per_cta - 1) / per_cta), static_cast<unsigned>(qrows));
     sgqa::index_score_decode_kernel<<<grid, sgqa::kDecScoreThreads, 0, st>>>(iq, idx_w, store, scores, nq, q0, B,
-                                                                              w.rpad, cap / B);
+                                                                              w.rpad, cap / B, per_cta, list_count);
     SGQA_LAUNCH_CHECK("index_score_decode_kernel");
+    if (rneed <= static_cast<int64_t>(sgqa::kDecSelCtas) * sgqa::kDecSelSlice) {
+      // each row selected by a cluster of CTAs; rows whose boundary the cluster cannot rank are listed
+      const int64_t rows = S * nq * G;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(rows * sgqa::kDecSelCtas));
+      cfg.blockDim = dim3(sgqa::kDecSelThreads);
+      cfg.dynamicSmemBytes = 0;
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = sgqa::kDecSelCtas;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      cudaError_t e = cudaLaunchKernelEx(&cfg, sgqa::topk_decode_cluster_kernel, static_cast<const float*>(scores),
+                                         w.rpad, nq, G, q0, B, static_cast<int>(p->topk), sel, sel_count, list,
+                                         list_count);
+      if (e != cudaSuccess) return cuda_fail(e, "topk_decode_cluster_kernel launch");
+      SGQA_LAUNCH_CHECK("topk_decode_cluster_kernel");
+      sgqa::topk_rows_list_kernel<<<static_cast<unsigned>(std::min<int64_t>(rows, 148)), sgqa::kSelThreads, 0, st>>>(
+          scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, list, list_count);
+      SGQA_LAUNCH_CHECK("topk_rows_list_kernel");
+      return SGQA_OK;
+    }
   } else if (rneed > 0) {
     // few queries: warp-MMA scores straight from the E4M3 store
     const int qpc = 64 / H;
@@ -569,7 +602,7 @@ sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq,
   if constexpr (B == 8) {
     return launch_attn_tc(p, S, q0, nq, q, kv, ids, msk, cnt, out, gate, units, st);
   } else {
-    const size_t smem = sgqa::kGroupedStages * 2 * sgqa::kStageElems * 2;
+    const size_t smem = sgqa::kWinStages * 2 * sgqa::kWinElems * 2;
     cudaFuncSetAttribute(sgqa::attn_grouped_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     sgqa::attn_grouped_kernel<B><<<static_cast<unsigned>(units), sgqa::kGroupedThreads, smem, st>>>(
         qb, kb, vb, ids, msk, cnt, ob, gb, nq, G, k, q0, kv.cap, kv.clen, scale_log2);

@@ -125,7 +125,8 @@ def test_index_topk_parity(cuda_device, case):
     assert ties <= 2 * len(rows)
 
 
-@pytest.mark.parametrize("case", ["short_rows", "filtered_rows", "filtered_rows_65k", "dup_short", "dup_long"])
+@pytest.mark.parametrize("case", ["short_rows", "filtered_rows", "filtered_rows_65k", "dup_short", "dup_long",
+                                  "decode_rows", "dup_decode"])
 def test_index_topk_exact_ties(cuda_device, case):
     """Exact score ties, which the selection must break toward smaller block ids.
 
@@ -137,7 +138,10 @@ def test_index_topk_exact_ties(cuda_device, case):
     (the sampled-threshold path: every zero row keeps all of its candidates,
     overflows the kept list and is recomputed for the radix kernel);
     filtered_rows_65k has 65536..66559, rows of the length a 512K-token context
-    reaches (the filtered path and its fallback at 1M-context row lengths).
+    reaches (the filtered path and its fallback at 1M-context row lengths);
+    decode_rows has 32 queries at 32762..32765 candidates (the decode path:
+    each row selected by a cluster of CTAs; a zero row's single boundary bin
+    overflows the cluster's buffers and goes to the radix kernel).
 
     dup_short / dup_long: the store repeats 211 distinct keys (block r holds
     the codes of block r mod 211), so every row's scores come in groups of
@@ -145,9 +149,13 @@ def test_index_topk_exact_ties(cuda_device, case):
     equal scores: the histogram kernel resolves those ties itself (groups up
     to 64 by ranking, larger ones by the warp radix select).  The selected
     members of the boundary group must be its smallest ids.  dup_short has
-    600..2903 candidates per row, dup_long 15360..16383."""
+    600..2903 candidates per row, dup_long 15360..16383, dup_decode 32762..32765
+    (the cluster select ranks each boundary group itself)."""
     dup = case.startswith("dup")
-    if case in ("short_rows", "dup_short"):
+    if case in ("decode_rows", "dup_decode"):
+        wl = dataclasses.replace(WL["prefill8k"], name="ties_decode", seq_len=262144, topk=512)
+        q0, nq = 262100, 32  # candidates 32762 .. 32765 per query, the decode path
+    elif case in ("short_rows", "dup_short"):
         wl = dataclasses.replace(WL["prefill8k"], name="ties", seq_len=24576, topk=512)
         q0, nq = 4800, 16384 + 2048  # candidates 600 .. 2903 per query (B = 8)
     elif case == "dup_long":
@@ -183,7 +191,7 @@ def test_index_topk_exact_ties(cuda_device, case):
     assert np.all(sel[zero_np] == np.arange(wl.topk, dtype=np.int32))
     iq, iw = Hn.to_np(qs["idx_q"]), Hn.to_np(qs["idx_w"])
     ties = 0
-    step = 397 if case in ("short_rows", "dup_short", "filtered_rows_65k") else 97
+    step = {"short_rows": 397, "dup_short": 397, "filtered_rows_65k": 397, "decode_rows": 2, "dup_decode": 2}.get(case, 97)
     rows = [i for i in range(1, nq, step) if not zero_np[i]] + [nq - 1]
     for i in rows:
         for g in range(wl.groups):
