@@ -441,9 +441,9 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
 // 2^e as a float, e in [-126, 127].
 __device__ __forceinline__ float exp2i(int e) { return __uint_as_float(static_cast<uint32_t>(127 + e) << 23); }
 
-// Decode scores: one CTA per (sequence and query, 512 candidates) scores the
-// query's four groups at once (B operand = 4 groups x 8 heads = 32 columns,
-// resident in registers), reading the E4M3 store directly.
+// Decode scores: a warp scores strips of 16 candidates for the query's four
+// groups at once (B operand = 4 groups x 8 heads = 32 columns, resident in
+// registers), straight from the E4M3 store.
 //
 // The MMA runs in FP16: the E4M3 codes convert to FP16 exactly with one
 // instruction per pair.  Each head's query row is scaled by a power of two
@@ -458,47 +458,18 @@ __device__ __forceinline__ float exp2i(int e) { return __uint_as_float(static_ca
 // k-steps come from one contiguous 16-byte piece of a key row: logical
 // k = 16 s + 8 h + 2 j + e is dimension 16 j + 4 s + 2 h + e (lane j =
 // lane % 4).  A warp's strip of 16 candidates is then two fully used
-// 512-byte runs of the store, and each warp issues the loads of its four
-// strips before any MMA.
-constexpr int kDecScoreThreads = 256;
-constexpr int kDecScoreDepth = 4;  // strips of 16 candidates each warp has in flight
+// 512-byte runs of the store.
 
-// One (sequence and query) per blockIdx.y; blockIdx.x takes a contiguous
-// range of `per_cta` candidates, which its warps walk strip by strip (warp w:
-// strips w, w + 8, ...), the key rows of the next kDecScoreDepth strips always
-// in flight while the current one is computed.
-__global__ void __launch_bounds__(kDecScoreThreads, 2)
-index_score_decode_kernel(const __nv_bfloat16* __restrict__ idx_q, const float* __restrict__ idx_w,
-                          const uint8_t* __restrict__ store, float* __restrict__ scores, int64_t nq,
-                          int64_t q_pos0, int B, int64_t rpad, int64_t key_rows, int64_t per_cta,
-                          int32_t* __restrict__ list_count) {
-  constexpr int G = 4, H = 8, Di = 64, W = kDecScoreThreads / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// B fragments of one (sequence and query) sq for all four groups (column n =
+// head lane / 4 of group g): the scaled FP16 values of dimensions
+// 16 j .. 16 j + 15 of that head (j = lane % 4), k-step s taking pairs 2 s,
+// 2 s + 1; wv: the weights of the lane's accumulator columns (heads 2 j and
+// 2 j + 1), which carry the heads' 2^-s.
+__device__ __forceinline__ void dec_query_frags(const __nv_bfloat16* __restrict__ idx_q,
+                                                const float* __restrict__ idx_w, int64_t sq, int lane,
+                                                uint32_t (&bf)[4][8], float (&wv)[4][2]) {
+  constexpr int G = 4, H = 8, Di = 64;
   const int j = lane & 3, rl = lane >> 2;
-  // the select kernel that follows lists the rows it leaves to the radix kernel
-  if (list_count != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *list_count = 0;
-  const int64_t sq = blockIdx.y;  // seq * nq + i
-  const int64_t i = sq % nq, seq = sq / nq;
-  const int64_t ncand = (q_pos0 + i) / B;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * per_cta;
-  const int64_t c1 = min(ncand, c0 + per_cta);
-  if (c0 >= c1) return;
-  const int nstrips = static_cast<int>((c1 - c0 + 15) / 16);
-  const int mine = nstrips > warp ? (nstrips - warp + W - 1) / W : 0;  // strips of this warp
-  // key rows of this warp's strip number s (s-th of its own): 16 bytes per lane and row
-  const uint8_t* kb = store + seq * key_rows * Di + 16 * j;
-  auto load_strip = [&](int s, uint4& a, uint4& b) {
-    const int64_t ra = c0 + 16 * (warp + static_cast<int64_t>(W) * s) + rl, rb = ra + 8;
-    a = (s < mine && ra < key_rows) ? __ldg(reinterpret_cast<const uint4*>(kb + ra * Di)) : make_uint4(0u, 0u, 0u, 0u);
-    b = (s < mine && rb < key_rows) ? __ldg(reinterpret_cast<const uint4*>(kb + rb * Di)) : make_uint4(0u, 0u, 0u, 0u);
-  };
-  uint4 ka[kDecScoreDepth], kbb[kDecScoreDepth];
-#pragma unroll
-  for (int d = 0; d < kDecScoreDepth; ++d) load_strip(d, ka[d], kbb[d]);
-  // B fragments (column n = head rl of group g): the scaled FP16 values of
-  // dimensions 16 j .. 16 j + 15 of that head; k-step s takes pairs 2 s, 2 s + 1
-  uint32_t bf[G][8];
-  float wv[G][2];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     const uint4* qrow = reinterpret_cast<const uint4*>(idx_q + ((sq * G + g) * H + rl) * Di + 16 * j);
@@ -519,53 +490,127 @@ index_score_decode_kernel(const __nv_bfloat16* __restrict__ idx_q, const float* 
       const __half2 h2 = __floats2half2_rn(__uint_as_float(qw[m] << 16) * up, __uint_as_float(qw[m] & 0xFFFF0000u) * up);
       bf[g][m] = *reinterpret_cast<const uint32_t*>(&h2);
     }
-    // this lane's accumulator columns are heads 2 j and 2 j + 1: their weights carry 2^-s
     const float d0 = __shfl_sync(0xffffffffu, down, 8 * j), d1 = __shfl_sync(0xffffffffu, down, 8 * j + 4);
     const float2 w2 = __ldg(reinterpret_cast<const float2*>(idx_w + (sq * G + g) * H + 2 * j));
     wv[g][0] = w2.x * d0;
     wv[g][1] = w2.y * d1;
   }
-  for (int s0 = 0; s0 < mine; s0 += kDecScoreDepth) {
+}
+
+// Scores of one strip of 16 candidates: ka / kb are the lane's 16-byte pieces
+// (piece j) of key rows rl and rl + 8 of the strip.  Every lane of a quad
+// computes all four groups' sums (bit-identical across the quad); lane j
+// returns group j's, for rows rl (sa) and rl + 8 (sb).
+__device__ __forceinline__ void dec_strip_scores(uint4 ka, uint4 kb, const uint32_t (&bf)[4][8],
+                                                 const float (&wv)[4][2], int j, float& sa_out, float& sb_out) {
+  // A fragments: pair m of the lane's 16 codes = dimensions 16 j + 2 m, + 1
+  uint32_t pa[8], pb[8];
+  const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
+  const uint32_t wb[4] = {kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
-    for (int d = 0; d < kDecScoreDepth; ++d) {
-      const int s = s0 + d;
-      if (s < mine) {
-        const int64_t ra = c0 + 16 * (warp + static_cast<int64_t>(W) * s) + rl, rb = ra + 8;
-        // A fragments: pair m of the lane's 16 codes = dimensions 16 j + 2 m, + 1
-        uint32_t pa[8], pb[8];
-        const uint32_t wa[4] = {ka[d].x, ka[d].y, ka[d].z, ka[d].w};
-        const uint32_t wb[4] = {kbb[d].x, kbb[d].y, kbb[d].z, kbb[d].w};
+  for (int m = 0; m < 4; ++m) {
+    pa[2 * m] = e4m3x2_to_f16x2(static_cast<uint16_t>(wa[m] & 0xFFFFu));
+    pa[2 * m + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(wa[m] >> 16));
+    pb[2 * m] = e4m3x2_to_f16x2(static_cast<uint16_t>(wb[m] & 0xFFFFu));
+    pb[2 * m + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(wb[m] >> 16));
+  }
+  sa_out = 0.f;
+  sb_out = 0.f;
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          pa[2 * m] = e4m3x2_to_f16x2(static_cast<uint16_t>(wa[m] & 0xFFFFu));
-          pa[2 * m + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(wa[m] >> 16));
-          pb[2 * m] = e4m3x2_to_f16x2(static_cast<uint16_t>(wb[m] & 0xFFFFu));
-          pb[2 * m + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(wb[m] >> 16));
-        }
-        load_strip(s + kDecScoreDepth, ka[d], kbb[d]);  // the strip that reuses this slot
+  for (int g = 0; g < 4; ++g) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint32_t af[4] = {pa[2 * ks], pb[2 * ks], pa[2 * ks + 1], pb[2 * ks + 1]};
-            mma_f16_16816(acc, af, bf[g][2 * ks], bf[g][2 * ks + 1]);
-          }
-          float sa = wv[g][0] * fmaxf(acc[0], 0.f) + wv[g][1] * fmaxf(acc[1], 0.f);
-          float sb = wv[g][0] * fmaxf(acc[2], 0.f) + wv[g][1] * fmaxf(acc[3], 0.f);
-          sa += __shfl_xor_sync(0xffffffffu, sa, 1);
-          sa += __shfl_xor_sync(0xffffffffu, sa, 2);
-          sb += __shfl_xor_sync(0xffffffffu, sb, 1);
-          sb += __shfl_xor_sync(0xffffffffu, sb, 2);
-          if (j == 0) {
-            float* srow = scores + (sq * G + g) * rpad;
-            if (ra < rpad) srow[ra] = sa;
-            if (rb < rpad) srow[rb] = sb;
-          }
-        }
-      }
+    for (int ks = 0; ks < 4; ++ks) {
+      const uint32_t af[4] = {pa[2 * ks], pb[2 * ks], pa[2 * ks + 1], pb[2 * ks + 1]};
+      mma_f16_16816(acc, af, bf[g][2 * ks], bf[g][2 * ks + 1]);
+    }
+    float sa = wv[g][0] * fmaxf(acc[0], 0.f) + wv[g][1] * fmaxf(acc[1], 0.f);
+    float sb = wv[g][0] * fmaxf(acc[2], 0.f) + wv[g][1] * fmaxf(acc[3], 0.f);
+    sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+    sa += __shfl_xor_sync(0xffffffffu, sa, 2);
+    sb += __shfl_xor_sync(0xffffffffu, sb, 1);
+    sb += __shfl_xor_sync(0xffffffffu, sb, 2);
+    if (j == g) {
+      sa_out = sa;
+      sb_out = sb;
     }
   }
+}
+
+// One (sequence and query) per blockIdx.y; blockIdx.x takes a contiguous
+// range of `per_cta` candidates, which its warps walk strip by strip (warp w:
+// strips w, w + 8, ...).  Each warp streams its strips' key rows through a
+// private ring of cp.async copies, kDecScoreRing strips in flight; every lane
+// copies exactly the two 16-byte pieces it later reads, so the ring needs no
+// warp barrier.  Writes FP32 score rows (lane j: group j) and, per row, the
+// largest score of every strip of 16 candidates (smax [rows, rpad / 16]),
+// from which topk_rows_bound_kernel bounds the row's k-th largest score.
+constexpr int kDecScoreThreads = 256;
+constexpr int kDecScoreRing = 8;
+constexpr size_t kDecScoreSmem = static_cast<size_t>(kDecScoreThreads / 32) * kDecScoreRing * 1024;
+
+__global__ void __launch_bounds__(kDecScoreThreads, 2)
+index_score_decode_kernel(const __nv_bfloat16* __restrict__ idx_q, const float* __restrict__ idx_w,
+                          const uint8_t* __restrict__ store, float* __restrict__ scores, int64_t nq,
+                          int64_t q_pos0, int B, int64_t rpad, int64_t key_rows, int64_t per_cta,
+                          float* __restrict__ smax, int32_t* __restrict__ list_count) {
+  constexpr int Di = 64, W = kDecScoreThreads / 32;
+  extern __shared__ __align__(16) uint8_t ring[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int j = lane & 3, rl = lane >> 2;
+  // the select kernel that follows lists the rows it leaves to the radix kernel
+  if (list_count != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *list_count = 0;
+  const int64_t sq = blockIdx.y;  // seq * nq + i
+  const int64_t i = sq % nq, seq = sq / nq;
+  const int64_t ncand = (q_pos0 + i) / B;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * per_cta;
+  const int64_t c1 = min(ncand, c0 + per_cta);
+  if (c0 >= c1) return;
+  const int nstrips = static_cast<int>((c1 - c0 + 15) / 16);
+  const int mine = nstrips > warp ? (nstrips - warp + W - 1) / W : 0;  // strips of this warp
+  const uint8_t* kseq = store + seq * key_rows * Di;
+  const uint32_t wring = smem_u32(ring + static_cast<size_t>(warp) * kDecScoreRing * 1024);
+  // strip s of this warp into slot s % ring: rows 8 h + rl, the lane's piece j, at h * 512 + 16 lane
+  auto issue = [&](int s) {
+    if (s < mine) {
+      const int64_t row0 = c0 + 16 * (warp + static_cast<int64_t>(W) * s);
+      const uint32_t dst = wring + (s % kDecScoreRing) * 1024 + 16 * lane;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t r = row0 + 8 * h + rl;
+        const bool ok = r < key_rows;
+        cp_async16_zfill(dst + 512 * h, kseq + (ok ? r * Di + 16 * j : 0), ok);
+      }
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int s = 0; s < kDecScoreRing - 1; ++s) issue(s);
+  uint32_t bf[4][8];
+  float wv[4][2];
+  dec_query_frags(idx_q, idx_w, sq, lane, bf, wv);
+  float* srow = scores + (sq * 4 + j) * rpad;
+  for (int s = 0; s < mine; ++s) {
+    cp_async_wait<kDecScoreRing - 2>();
+    const uint32_t src = wring + (s % kDecScoreRing) * 1024 + 16 * lane;
+    uint4 ka, kb;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n" : "=r"(ka.x), "=r"(ka.y), "=r"(ka.z), "=r"(ka.w) : "r"(src));
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n" : "=r"(kb.x), "=r"(kb.y), "=r"(kb.z), "=r"(kb.w)
+                 : "r"(src + 512));
+    issue(s + kDecScoreRing - 1);  // into the slot this lane emptied in the previous strip
+    float sa, sb;
+    dec_strip_scores(ka, kb, bf, wv, j, sa, sb);
+    const int64_t r0 = c0 + 16 * (warp + static_cast<int64_t>(W) * s), ra = r0 + rl, rb = ra + 8;
+    if (ra < rpad) srow[ra] = sa;
+    if (rb < rpad) srow[rb] = sb;
+    // the strip's largest score of group j over its real candidates (the first always is one)
+    float m = fmaxf(ra < ncand ? sa : -INFINITY, rb < ncand ? sb : -INFINITY);
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+    if (rl == 0) smax[(sq * 4 + j) * (rpad / 16) + r0 / 16] = m;
+  }
+  cp_async_wait<0>();
 }
 
 // Exact top-k of rows of at most 32768 scores: 1024 threads hold 32 keys each
@@ -795,333 +840,242 @@ topk_rows_reg_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq,
 }
 
 // ---------------------------------------------------------------------------
-// Exact top-k of decode rows (at most kDecSelCtas * 4096 candidates) by a
-// thread-block cluster of kDecSelCtas CTAs per row, so that a few long rows
-// use many SMs.  CTA c owns candidates [4096 c, 4096 c + 4096), 16 per thread
-// in registers.  The cluster agrees on the row's extreme scores, builds one
-// linear 2048-bin histogram between them (each CTA its own, summed through
-// distributed shared memory), and finds the bin holding the k-th largest;
-// better bins are taken, the boundary bin's entries are gathered to CTA 0 and
-// ranked exactly (score, then smaller id) by one warp, or -- when they all
-// share one score -- taken in id order.  Each CTA writes its taken ids in
-// ascending order at the offset the lower CTAs' counts give.  A boundary
-// with more distinct entries than the gather buffer holds lists the row for
-// the radix kernel (topk_rows_list_kernel), which then rewrites it.
+// Exact top-k of decode rows (at most 32768 candidates) from a lower bound on
+// the k-th largest score.  Each strip of 16 candidates has one largest score
+// (the score kernel writes them); if k strip maxima are >= L, then at least k
+// candidates are >= L, so L <= the row's k-th largest score and every member
+// of the top k -- ties at the k-th included -- scores >= L.  The kernel takes
+// as L the smallest strip maximum among the best bins of a linear 2048-bin
+// histogram of the strip maxima that hold k of them (at least k maxima are
+// >= L, and L sits close above the k-th largest maximum, a little below the
+// row's k-th largest score), collects the candidates >= L (a few more than k
+// on typical rows), and ranks them exactly (score, then smaller id): a linear
+// histogram of their scores finds the bin of the k-th largest, and one warp
+// ranks that bin's few entries.  A row with fewer strips than k has no such bound and keeps every
+// candidate for the exact rank (the launch sends rows of fewer than 16 k + 128
+// candidates to topk_rows_reg_kernel).  Ids are marked in a bitmap and read out ascending.  A row with more
+// than kBndSelCap such candidates, or a boundary bin of more than 1024 (massive
+// ties), is listed for topk_rows_list_kernel, which ranks the full row.
 // ---------------------------------------------------------------------------
-constexpr int kDecSelCtas = 8;
-constexpr int kDecSelThreads = 256;
-constexpr int kDecSelPer = 16;
-constexpr int kDecSelSlice = kDecSelThreads * kDecSelPer;  // 4096 candidates per CTA
-constexpr int kDecSelBins = 2048;
-constexpr int kDecSelBnd = 512;                            // boundary entries one CTA holds
-constexpr int kDecSelGather = 2048;                        // boundary entries CTA 0 ranks
+constexpr int kBndSelThreads = 1024;
+constexpr int kBndSelPer = 32;      // scores of the row each thread holds
+constexpr int kBndSelCap = 4096;    // candidates >= L the exact rank takes
+constexpr int kBndSelBins = 2048;
 
-struct DecSelSmem {
-  uint32_t hist[kDecSelBins];    // this CTA's histogram (later warp_select's scratch in CTA 0)
-  uint32_t slot[kDecSelBins / kDecSelCtas];  // the cluster's total of bins [256 c, 256 c + 256)
-  uint32_t tot[kDecSelBins];     // the cluster's total histogram
-  uint2 bnd[kDecSelBnd];         // this CTA's boundary entries (key, id)
-  uint2 gath[kDecSelGather];     // CTA 0: every CTA's boundary entries
-  uint32_t bits[kDecSelSlice / 32];
-  uint32_t wsum[kDecSelThreads / 32];
-  float wmx[kDecSelThreads / 32], wmn[kDecSelThreads / 32];
-  float mx, mn, gmx, gmn;
-  uint32_t nb, nabove, bstar, rem, cstar;
-  // written by CTA 0 into every CTA: how to treat the boundary and where this CTA's ids go
-  uint32_t mode, theta, id_cut, take, off;
-};
-
-__global__ void __launch_bounds__(kDecSelThreads)
-topk_decode_cluster_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq, int G, int64_t q_pos0, int B,
-                           int k, int32_t* __restrict__ sel, int32_t* __restrict__ sel_count,
-                           int32_t* __restrict__ list, int32_t* __restrict__ list_count) {
-  namespace cg = cooperative_groups;
-  cg::cluster_group cluster = cg::this_cluster();
-  __shared__ DecSelSmem sm;
+__global__ void __launch_bounds__(kBndSelThreads)
+topk_rows_bound_kernel(const float* __restrict__ scores, int64_t rpad, const float* __restrict__ smax, int64_t nq,
+                       int G, int64_t q_pos0, int B, int k, int32_t* __restrict__ sel,
+                       int32_t* __restrict__ sel_count, int32_t* __restrict__ list, int32_t* __restrict__ list_count) {
+  __shared__ uint32_t hist[kBndSelBins];
+  __shared__ uint2 surv[kBndSelCap];
+  __shared__ uint32_t keep_bits[kBndSelThreads];
+  __shared__ int sums[32];
+  __shared__ float fmx[32], fmn[32];
+  __shared__ uint32_t s_nsurv, s_lkey, s_bstar, s_rem, s_cnt, s_nb, s_kmin, s_kmax;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int c = static_cast<int>(cluster.block_rank());
-  const int64_t row = blockIdx.x / kDecSelCtas;
+  const int64_t row = blockIdx.x;
   const int64_t i = (row / G) % nq;
   const int n = static_cast<int>((q_pos0 + i) / B);
   int32_t* out = sel + row * k;
-  if (n <= k) {  // every CTA of the cluster leaves here together
-    if (c == 0) {
-      for (int x = tid; x < k; x += kDecSelThreads) out[x] = x < n ? x : -1;
-      if (tid == 0) sel_count[row] = n;
-    }
+  if (n <= k) {
+    for (int j = tid; j < k; j += kBndSelThreads) out[j] = j < n ? j : -1;
+    if (tid == 0) sel_count[row] = n;
     return;
   }
-  const int base = c * kDecSelSlice;
-  const float* srow = scores + row * rpad + base;
-  float v[kDecSelPer];
-  float mx = -INFINITY, mn = INFINITY;
-#pragma unroll
-  for (int u = 0; u < kDecSelPer; ++u) {
-    const int jl = tid + kDecSelThreads * u;
-    v[u] = base + jl < n ? srow[jl] : -INFINITY;
-    if (base + jl < n) {
-      mx = fmaxf(mx, v[u]);
-      mn = fminf(mn, v[u]);
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-  }
-  if (lane == 0) {
-    sm.wmx[warp] = mx;
-    sm.wmn[warp] = mn;
-  }
-  for (int b = tid; b < kDecSelBins; b += kDecSelThreads) sm.hist[b] = 0u;
-  for (int w = tid; w < kDecSelSlice / 32; w += kDecSelThreads) sm.bits[w] = 0u;
-  if (tid == 0) {
-    sm.nb = 0;
-    sm.nabove = 0;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    float a = lane < kDecSelThreads / 32 ? sm.wmx[lane] : -INFINITY;
-    float b = lane < kDecSelThreads / 32 ? sm.wmn[lane] : INFINITY;
+  const float* srow = scores + row * rpad;
+  // the row's strip maxima, two per thread
+  const int ns = (n + 15) / 16;
+  const float* mrow = smax + row * (rpad / 16);
+  const float m0 = tid < ns ? mrow[tid] : -INFINITY;
+  const float m1 = tid + kBndSelThreads < ns ? mrow[tid + kBndSelThreads] : -INFINITY;
+  {
+    float mx = fmaxf(m0, m1);
+    float mn = fminf(tid < ns ? m0 : INFINITY, tid + kBndSelThreads < ns ? m1 : INFINITY);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-      b = fminf(b, __shfl_xor_sync(0xffffffffu, b, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     }
     if (lane == 0) {
-      sm.mx = a;
-      sm.mn = b;
+      fmx[warp] = mx;
+      fmn[warp] = mn;
     }
   }
-  cluster.sync();  // (1) every CTA's extremes
-  if (warp == 0) {  // one round trip: lane r reads CTA r's
-    float a = -INFINITY, b = INFINITY;
-    if (lane < kDecSelCtas) {
-      const DecSelSmem* o = cluster.map_shared_rank(&sm, lane);
-      a = o->mx;
-      b = o->mn;
-    }
-#pragma unroll
-    for (int o = 4; o > 0; o >>= 1) {
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-      b = fminf(b, __shfl_xor_sync(0xffffffffu, b, o));
-    }
-    if (lane == 0) {
-      sm.gmx = a;
-      sm.gmn = b;
-    }
+  for (int b = tid; b < kBndSelBins; b += kBndSelThreads) hist[b] = 0u;
+  keep_bits[tid] = 0u;
+  if (tid == 0) {
+    s_nsurv = 0;
+    s_lkey = ns >= k ? 0xFFFFFFFFu : 0u;  // fewer strips than k: no bound, every candidate is kept
+    s_bstar = 0;
+    s_kmin = 0xFFFFFFFFu;
+    s_kmax = 0u;
   }
   __syncthreads();
-  const float gmx = sm.gmx, width = gmx - sm.gmn;
-  const float scale = width > 0.f ? (kDecSelBins - 0.5f) / width : 0.f;
+  float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+  for (int w = 0; w < 32; ++w) {
+    mx = fmaxf(mx, fmx[w]);
+    mn = fminf(mn, fmn[w]);
+  }
+  const float width = mx - mn;
+  const float scale = width > 0.f ? (kBndSelBins - 0.5f) / width : 0.f;
   // bins best first; both steps round monotonically
-  auto bin_of = [&](float x) -> int { return min(static_cast<int>(__fmul_rn(__fsub_rn(gmx, x), scale)), kDecSelBins - 1); };
-#pragma unroll
-  for (int u = 0; u < kDecSelPer; ++u)
-    if (base + tid + kDecSelThreads * u < n) atomicAdd(&sm.hist[bin_of(v[u])], 1u);
-  cluster.sync();  // (2) every CTA's histogram
-  {  // CTA c sums its slot of bins over the cluster (independent loads)
-    constexpr int per = kDecSelBins / kDecSelCtas;
-    uint32_t h[kDecSelCtas];
-#pragma unroll
-    for (int r = 0; r < kDecSelCtas; ++r) h[r] = cluster.map_shared_rank(&sm, r)->hist[per * c + tid];
-    uint32_t t = 0;
-#pragma unroll
-    for (int r = 0; r < kDecSelCtas; ++r) t += h[r];
-    sm.slot[tid] = t;
-  }
-  cluster.sync();  // (3) every slot
-  {
-    uint32_t h[kDecSelCtas];
-#pragma unroll
-    for (int r = 0; r < kDecSelCtas; ++r) h[r] = cluster.map_shared_rank(&sm, r)->slot[tid];
-#pragma unroll
-    for (int r = 0; r < kDecSelCtas; ++r) sm.tot[(kDecSelBins / kDecSelCtas) * r + tid] = h[r];
-  }
+  auto bin_of = [&](float x) -> int { return min(static_cast<int>(__fmul_rn(__fsub_rn(mx, x), scale)), kBndSelBins - 1); };
+  if (ns >= k) {  // (uniform over the CTA)
+  if (tid < ns) atomicAdd(&hist[bin_of(m0)], 1u);
+  if (tid + kBndSelThreads < ns) atomicAdd(&hist[bin_of(m1)], 1u);
   __syncthreads();
-  {  // thread t owns bins 8 t .. 8 t + 7: the bin in which the running count reaches k
-    uint32_t loc[8], sum = 0;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      loc[q] = sm.tot[8 * tid + q];
-      sum += loc[q];
-    }
-    uint32_t x = sum;
+  {  // thread t owns bins 2 t, 2 t + 1: the bin in which the running count of maxima reaches k
+    const uint32_t c0 = hist[2 * tid], c1 = hist[2 * tid + 1];
+    uint32_t x = c0 + c1;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
       if (lane >= o) x += y;
     }
-    if (lane == 31) sm.wsum[warp] = x;
+    if (lane == 31) sums[warp] = static_cast<int>(x);
     __syncthreads();
-    uint32_t acc = x - sum;
-    for (int w = 0; w < warp; ++w) acc += sm.wsum[w];
+    uint32_t before = x - c0 - c1;
+    for (int w = 0; w < warp; ++w) before += sums[w];
     const uint32_t kk = static_cast<uint32_t>(k);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      if (acc < kk && kk <= acc + loc[q]) {
-        sm.bstar = 8 * tid + q;
-        sm.rem = kk - acc;
-        sm.cstar = loc[q];
-      }
-      acc += loc[q];
-    }
+    if (before < kk && kk <= before + c0) s_bstar = 2 * tid;
+    else if (before + c0 < kk && kk <= before + c0 + c1) s_bstar = 2 * tid + 1;
   }
   __syncthreads();
-  const int bstar = static_cast<int>(sm.bstar);
-  const uint32_t rem = sm.rem, cstar = sm.cstar;
-  // better bins are taken (counted); the boundary bin's entries are collected
-  uint32_t above = 0;
+  {  // L: the smallest maximum of the bins up to the boundary bin
+    const int bstar = static_cast<int>(s_bstar);
+    uint32_t lk = 0xFFFFFFFFu;
+    if (tid < ns && bin_of(m0) <= bstar) lk = score_key(m0);
+    if (tid + kBndSelThreads < ns && bin_of(m1) <= bstar) lk = min(lk, score_key(m1));
+    lk = __reduce_min_sync(0xffffffffu, lk);
+    if (lane == 0 && lk != 0xFFFFFFFFu) atomicMin(&s_lkey, lk);
+  }
+  }
+  __syncthreads();
+  const uint32_t lkey = s_lkey;
+  {  // the candidates >= L (thread t reads scores 4 t .. 4 t + 3 of every 4096, twice from L2):
+     // counted per thread, placed by one shared atomic per warp
+    constexpr int kChunks = kBndSelPer / 4;
+    uint32_t c = 0, kmin = 0xFFFFFFFFu, kmax = 0u;
 #pragma unroll
-  for (int u = 0; u < kDecSelPer; ++u) {
-    const int jl = tid + kDecSelThreads * u;
-    if (base + jl < n) {
-      const int b = bin_of(v[u]);
-      if (b < bstar) {
-        atomicOr(&sm.bits[jl >> 5], 1u << (jl & 31));
-        ++above;
-      } else if (b == bstar) {
-        const uint32_t pos = atomicAdd(&sm.nb, 1u);
-        if (pos < kDecSelBnd) sm.bnd[pos] = make_uint2(score_key(v[u]), static_cast<uint32_t>(base + jl));
+    for (int u = 0; u < kChunks; ++u) {
+      const int j0 = 4 * tid + 4 * kBndSelThreads * u;
+      if (j0 < n) {
+        const float4 v = *reinterpret_cast<const float4*>(srow + j0);
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t kk = score_key(vv[e]);
+          if (j0 + e < n && kk >= lkey) {
+            ++c;
+            kmin = min(kmin, kk);
+            kmax = max(kmax, kk);
+          }
+        }
+      }
+    }
+    uint32_t x = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    uint32_t wbase = 0;
+    if (lane == 31 && x) {
+      wbase = atomicAdd(&s_nsurv, x);
+      atomicMin(&s_kmin, kmin);
+      atomicMax(&s_kmax, kmax);
+    }
+    uint32_t pos = __shfl_sync(0xffffffffu, wbase, 31) + x - c;
+#pragma unroll
+    for (int u = 0; u < kChunks; ++u) {
+      const int j0 = 4 * tid + 4 * kBndSelThreads * u;
+      if (c != 0 && j0 < n) {
+        const float4 v = *reinterpret_cast<const float4*>(srow + j0);
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t kk = score_key(vv[e]);
+          if (j0 + e < n && kk >= lkey) {
+            if (pos < static_cast<uint32_t>(kBndSelCap)) surv[pos] = make_uint2(kk, static_cast<uint32_t>(j0 + e));
+            ++pos;
+          }
+        }
       }
     }
   }
-  above = __reduce_add_sync(0xffffffffu, above);
-  if (lane == 0 && above) atomicAdd(&sm.nabove, above);
-  cluster.sync();  // (4) every CTA's counts and boundary entries
-  if (c == 0 && warp == 0) {
-    // CTA 0 decides the boundary and every CTA's output offset, one round trip per step
-    uint32_t nbr = 0, nab = 0;
-    if (lane < kDecSelCtas) {
-      const DecSelSmem* o = cluster.map_shared_rank(&sm, lane);
-      nbr = o->nb;
-      nab = o->nabove;
-    }
-    const bool overflow = __any_sync(0xffffffffu, nbr > static_cast<uint32_t>(kDecSelBnd));
-    const uint32_t nbc = min(nbr, static_cast<uint32_t>(kDecSelBnd));
-    uint32_t bstart = nbc;  // exclusive prefix of the stored boundary counts over CTAs 0..lane-1
+  for (int b = tid; b < kBndSelBins; b += kBndSelThreads) hist[b] = 0u;
+  __syncthreads();
+  const uint32_t nsurv = s_nsurv;
+  if (nsurv > static_cast<uint32_t>(kBndSelCap)) {  // every thread leaves here together
+    if (tid == 0) list[atomicAdd(list_count, 1)] = static_cast<int32_t>(row);
+    return;
+  }
+  // the exact rank among them: a linear histogram of their scores finds the
+  // bin holding the k-th largest; better bins are kept, that bin's entries
+  // (typically one or two) are ranked by one warp
+  const float hi = key_score(s_kmax), lo = key_score(s_kmin);
+  const float scale2 = hi > lo ? (kBndSelBins - 0.5f) / (hi - lo) : 0.f;
+  auto bin2 = [&](uint32_t kk) -> int {
+    return min(static_cast<int>(__fmul_rn(__fsub_rn(hi, key_score(kk)), scale2)), kBndSelBins - 1);
+  };
+  for (uint32_t e = tid; e < nsurv; e += kBndSelThreads) atomicAdd(&hist[bin2(surv[e].x)], 1u);
+  __syncthreads();
+  {  // thread t owns bins 2 t, 2 t + 1
+    const uint32_t c0 = hist[2 * tid], c1 = hist[2 * tid + 1];
+    uint32_t x = c0 + c1;
 #pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, bstart, o);
-      if (lane >= o) bstart += y;
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
     }
-    const uint32_t total = __shfl_sync(0xffffffffu, bstart, kDecSelCtas - 1);
-    bstart -= nbc;
-    uint32_t mode = 0;  // 0: ranked (or all taken); 1: equal scores, taken in id order; 2: the radix kernel
+    if (lane == 31) sums[warp] = static_cast<int>(x);
+    __syncthreads();
+    uint32_t before = x - c0 - c1;
+    for (int w = 0; w < warp; ++w) before += sums[w];
+    const uint32_t kk = static_cast<uint32_t>(k);
+    if (before < kk && kk <= before + c0) {
+      s_bstar = 2 * tid;
+      s_rem = kk - before;
+      s_cnt = c0;
+    } else if (before + c0 < kk && kk <= before + c0 + c1) {
+      s_bstar = 2 * tid + 1;
+      s_rem = kk - before - c0;
+      s_cnt = c1;
+    }
+    if (tid == 0) s_nb = 0;
+  }
+  __syncthreads();
+  const int bstar = static_cast<int>(s_bstar);
+  const uint32_t rem = s_rem, cstar = s_cnt;
+  if (cstar > static_cast<uint32_t>(kBndSelBins / 2)) {  // a huge group of near-equal scores: the radix kernel
+    if (tid == 0) list[atomicAdd(list_count, 1)] = static_cast<int32_t>(row);
+    return;
+  }
+  uint2* bnd = reinterpret_cast<uint2*>(hist);  // [kBndSelBins / 2]; the histogram is consumed
+  __syncthreads();
+  for (uint32_t e = tid; e < nsurv; e += kBndSelThreads) {
+    const uint2 x = surv[e];
+    const int b = bin2(x.x);
+    if (b < bstar) atomicOr(&keep_bits[x.y >> 5], 1u << (x.y & 31));
+    else if (b == bstar) bnd[atomicAdd(&s_nb, 1u)] = x;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t nb = s_nb;
     uint32_t theta = 0, id_cut = 0xFFFFFFFFu;
-    if (overflow) {
-      mode = 2;  // a CTA's boundary entries did not fit its buffer
-    } else if (cstar > rem) {
-      if (total > kDecSelGather) {
-        mode = 2;
-      } else {
-        // gather: entry e < total lives in the CTA r whose [bstart, bstart + nbc) holds it
-        for (uint32_t e0 = 0; e0 < total; e0 += 32) {
-          const uint32_t e = e0 + lane;
-          int r = 0;
-#pragma unroll
-          for (int q = 1; q < kDecSelCtas; ++q) r += e >= __shfl_sync(0xffffffffu, bstart, q) ? 1 : 0;
-          const uint32_t rs = __shfl_sync(0xffffffffu, bstart, r);
-          if (e < total) sm.gath[e] = cluster.map_shared_rank(&sm, r)->bnd[e - rs];
-        }
-        __syncwarp();
-        uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-        for (uint32_t e = lane; e < total; e += 32) {
-          kmin = min(kmin, sm.gath[e].x);
-          kmax = max(kmax, sm.gath[e].x);
-        }
-        kmin = __reduce_min_sync(0xffffffffu, kmin);
-        kmax = __reduce_max_sync(0xffffffffu, kmax);
-        if (kmin == kmax) {
-          mode = 1;
-        } else {
-          warp_select(sm.gath, static_cast<int>(total), static_cast<int>(rem), sm.hist, theta, id_cut);
-        }
-      }
-    }
-    // boundary entries each CTA keeps: all, the first rem in CTA order (mode 1), or by (theta, id_cut)
-    uint32_t take = 0;
-    if (mode == 1 || cstar <= rem) {
-      take = bstart >= rem ? 0u : min(nbc, rem - bstart);
-    } else if (mode == 0) {
-      for (uint32_t e0 = 0; e0 < total; e0 += 32) {
-        const uint32_t e = e0 + lane;
-        const bool kp = e < total && kept(sm.gath[e], theta, id_cut);
-        int r = 0;
-#pragma unroll
-        for (int q = 1; q < kDecSelCtas; ++q) r += e >= __shfl_sync(0xffffffffu, bstart, q) ? 1 : 0;
-        // count kept entries per CTA: lane r sums the ballots of entries of CTA r
-#pragma unroll
-        for (int q = 0; q < kDecSelCtas; ++q) {
-          const uint32_t bq = __ballot_sync(0xffffffffu, kp && r == q);
-          if (lane == q) take += __popc(bq);
-        }
-      }
-    }
-    uint32_t cnt = nab + take, off = cnt;  // ids this CTA writes; exclusive prefix = its offset
-#pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, off, o);
-      if (lane >= o) off += y;
-    }
-    off -= cnt;
-    if (lane < kDecSelCtas) {
-      DecSelSmem* o = cluster.map_shared_rank(&sm, lane);
-      o->mode = mode;
-      o->theta = theta;
-      o->id_cut = id_cut;
-      o->take = take;
-      o->off = off;
-    }
-    if (mode == 2 && lane == 0) list[atomicAdd(list_count, 1)] = static_cast<int32_t>(row);
-  }
-  cluster.sync();  // (5) the decision is in every CTA; nothing reads another CTA's memory after this
-  if (sm.mode == 2) return;  // every CTA of the cluster leaves here together; the radix kernel writes the row
-  {
-    const uint32_t mine = min(sm.nb, static_cast<uint32_t>(kDecSelBnd));
-    if (sm.mode == 0 && cstar > rem) {
-      const uint32_t theta = sm.theta, id_cut = sm.id_cut;
-      for (uint32_t e = tid; e < mine; e += kDecSelThreads) {
-        const uint2 x = sm.bnd[e];
-        if (kept(x, theta, id_cut)) atomicOr(&sm.bits[(x.y - base) >> 5], 1u << ((x.y - base) & 31));
-      }
-    } else {
-      // all boundary entries, or the `take` smallest ids of this CTA's (equal scores)
-      const uint32_t take = sm.take;
-      for (uint32_t e = tid; e < mine; e += kDecSelThreads) {
-        const uint32_t id = sm.bnd[e].y;
-        uint32_t rank = 0;
-        if (take < mine)
-          for (uint32_t f = 0; f < mine; ++f) rank += sm.bnd[f].y < id;
-        if (rank < take) atomicOr(&sm.bits[(id - base) >> 5], 1u << ((id - base) & 31));
-      }
+    // warp_select's 256 counters live in the consumed candidate list
+    if (nb > rem) warp_select(bnd, static_cast<int>(nb), static_cast<int>(rem), reinterpret_cast<uint32_t*>(surv), theta,
+                              id_cut);
+    for (uint32_t e = lane; e < nb; e += 32) {
+      const uint2 x = bnd[e];
+      if (nb <= rem || kept(x, theta, id_cut)) atomicOr(&keep_bits[x.y >> 5], 1u << (x.y & 31));
     }
   }
   __syncthreads();
-  // ascending readout: thread t < 128 owns bitmap word t
-  const uint32_t wb = tid < kDecSelSlice / 32 ? sm.bits[tid] : 0u;
-  const uint32_t cw = __popc(wb);
-  uint32_t x = cw;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) sm.wsum[warp] = x;
-  __syncthreads();
-  uint32_t pos = x - cw + sm.off;
-  for (int w = 0; w < warp; ++w) pos += sm.wsum[w];
-  uint32_t bw = wb;
-  while (bw) {
-    const int b = __ffs(bw) - 1;
-    bw &= bw - 1;
-    if (pos < static_cast<uint32_t>(k)) out[pos] = base + 32 * tid + b;
-    ++pos;
-  }
-  if (c == kDecSelCtas - 1 && tid == kDecSelThreads - 1) {
-    sel_count[row] = k;
-    if (pos != static_cast<uint32_t>(k)) report(kDevBounds);
-  }
+  topk_reg_readout(keep_bits, sums, tid, lane, warp, k, out, sel_count, row);
 }
 
 }  // namespace sgqa

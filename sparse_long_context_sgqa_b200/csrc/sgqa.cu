@@ -132,7 +132,8 @@ constexpr int64_t kFallbackGrid = 2 * 148;
 // the FP32 score rows [rows, rpad] (rows of fewer than kFilterMinCand
 // candidates, and decode), or in turn the sampled scores, the filtered
 // (key, id) lists and the fallback's per-CTA score slots (the stages that use
-// them run in that order) -- then four per-row arrays.
+// them run in that order); decode adds each row's strip maxima
+// [rows, rpad / 16] after its score rows -- then four per-row arrays.
 struct IndexWs {
   int64_t rpad;
   bool filtered;
@@ -156,6 +157,8 @@ IndexWs index_ws(const sgqa_params* p, int64_t S, int64_t nq, int64_t max_ctx) {
                        static_cast<size_t>(w.fb_grid) * static_cast<size_t>(w.rpad) * 4});
   } else {
     region = rows * static_cast<size_t>(w.rpad) * 4;
+    // decode: the largest score of every 16-candidate strip, after the rows
+    if (nq <= kDecodeMaxNq) region = align256(region) + rows * static_cast<size_t>(w.rpad / 16) * 4;
   }
   w.region_off = keys;
   w.flags_off = keys + align256(region);
@@ -432,35 +435,25 @@ sgqa_status do_index(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, co
     // CTAs per SM over the whole launch, each range at least 1024 candidates and a whole number of strips
     const int64_t qrows = S * nq;
     if (qrows > 65535) return fail(SGQA_ERR_UNSUPPORTED, "decode index grid too large");
-    const int64_t want = std::max<int64_t>(1, (2 * kSmCount + qrows - 1) / qrows);
+    float* smax = ws_at<float>(ws, w.region_off + align256(static_cast<size_t>(qrows * G) * w.rpad * 4));
+    const int64_t want = std::max<int64_t>(1, (2 * kSmCount) / qrows);
     int64_t per_cta = (rneed + want - 1) / want;
     per_cta = std::max<int64_t>(1024, (per_cta + 15) / 16 * 16);
     dim3 grid(static_cast<unsigned>((rneed + per_cta - 1) / per_cta), static_cast<unsigned>(qrows));
-    sgqa::index_score_decode_kernel<<<grid, sgqa::kDecScoreThreads, 0, st>>>(iq, idx_w, store, scores, nq, q0, B,
-                                                                              w.rpad, cap / B, per_cta, list_count);
+    cudaError_t ea = cudaFuncSetAttribute(sgqa::index_score_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(sgqa::kDecScoreSmem));
+    if (ea != cudaSuccess) return cuda_fail(ea, "cudaFuncSetAttribute(index_score_decode_kernel)");
+    sgqa::index_score_decode_kernel<<<grid, sgqa::kDecScoreThreads, sgqa::kDecScoreSmem, st>>>(
+        iq, idx_w, store, scores, nq, q0, B, w.rpad, cap / B, per_cta, smax, list_count);
     SGQA_LAUNCH_CHECK("index_score_decode_kernel");
-    if (rneed <= static_cast<int64_t>(sgqa::kDecSelCtas) * sgqa::kDecSelSlice) {
-      // each row selected by a cluster of CTAs; rows whose boundary the cluster cannot rank are listed
+    if (rneed <= static_cast<int64_t>(sgqa::kBndSelThreads) * sgqa::kBndSelPer && rneed >= 16 * p->topk + 128) {
+      // each row ranked from the bound its strip maxima give; rows with massive ties are listed
       const int64_t rows = S * nq * G;
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(static_cast<unsigned>(rows * sgqa::kDecSelCtas));
-      cfg.blockDim = dim3(sgqa::kDecSelThreads);
-      cfg.dynamicSmemBytes = 0;
-      cfg.stream = st;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = sgqa::kDecSelCtas;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      cudaError_t e = cudaLaunchKernelEx(&cfg, sgqa::topk_decode_cluster_kernel, static_cast<const float*>(scores),
-                                         w.rpad, nq, G, q0, B, static_cast<int>(p->topk), sel, sel_count, list,
-                                         list_count);
-      if (e != cudaSuccess) return cuda_fail(e, "topk_decode_cluster_kernel launch");
-      SGQA_LAUNCH_CHECK("topk_decode_cluster_kernel");
-      sgqa::topk_rows_list_kernel<<<static_cast<unsigned>(std::min<int64_t>(rows, 148)), sgqa::kSelThreads, 0, st>>>(
-          scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, list, list_count);
+      sgqa::topk_rows_bound_kernel<<<static_cast<unsigned>(rows), sgqa::kBndSelThreads, 0, st>>>(
+          scores, w.rpad, smax, nq, G, q0, B, static_cast<int>(p->topk), sel, sel_count, list, list_count);
+      SGQA_LAUNCH_CHECK("topk_rows_bound_kernel");
+      sgqa::topk_rows_list_kernel<<<static_cast<unsigned>(std::min<int64_t>(rows, kSmCount)), sgqa::kSelThreads, 0,
+                                    st>>>(scores, w.rpad, nq, G, q0, B, p->topk, sel, sel_count, list, list_count);
       SGQA_LAUNCH_CHECK("topk_rows_list_kernel");
       return SGQA_OK;
     }

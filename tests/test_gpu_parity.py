@@ -109,9 +109,18 @@ def _index_isolated(wl, device, q_pos0, nq, rows):
     return ties
 
 
-@pytest.mark.parametrize("case", ["tiny", "prefill8k", "unaligned_chunk", "b1", "b4_k64"])
+@pytest.mark.parametrize("case", ["tiny", "prefill8k", "unaligned_chunk", "b1", "b4_k64", "decode_short",
+                                  "decode_mid"])
 def test_index_topk_parity(cuda_device, case):
-    if case == "tiny":
+    """decode_short / decode_mid: calls of at most 32 queries (the decode path,
+    one cluster per query scoring and selecting on chip) with 512..515 and
+    9000..9002 candidates: rows just above k, where the last CTAs of a cluster
+    own no candidate, and rows that split unevenly over the cluster."""
+    if case == "decode_short":
+        wl = dataclasses.replace(SMALL8, name="dec_short", seq_len=4224); q0, nq = 4100, 24; rows = range(nq)
+    elif case == "decode_mid":
+        wl = dataclasses.replace(SMALL8, name="dec_mid", seq_len=72192); q0, nq = 72000, 24; rows = range(nq)
+    elif case == "tiny":
         wl = WL["tiny"]; q0, nq = 0, 256; rows = range(256)
     elif case == "prefill8k":
         wl = WL["prefill8k"]; q0, nq = 0, 8192; rows = Hn.sample_rows(wl, 48)
