@@ -9,15 +9,12 @@
 // accumulator tiles.  K/V rows are staged in shared memory with cp.async
 // (rows padded to 400 B so ldmatrix is conflict-free).
 //
-// Two kernels use it:
-//  * attn_grouped_kernel  (prefill) -- page "What gets cheaper ..." and the
-//    second page: adjacent queries' selections overlap, so the 8 queries of a
-//    query block share one pass over the UNION of their selected blocks; each
-//    16-token tile is loaded once for 8 warps and a warp skips tiles its
-//    query did not select.  The union is built by attn_plan_kernel.
-//  * attn_decode_kernel   (few queries, long context) -- split-K over the
-//    query's tokens, 4 warps per CTA, partial (m, l, O) combined by
-//    attn_combine_kernel.
+// It serves attn_decode_kernel (few queries, blocks under 8 tokens) --
+// split-K over the query's tokens, 4 warps per CTA, partial (m, l, O)
+// combined by attn_combine_kernel.  This file also holds the union planners
+// (attn_plan_kernel, attn_plan_sort_kernel) of the prefill kernel in
+// attn_tc.cuh: adjacent queries' selections overlap (the second page), so the
+// 8 queries of a query block share one pass over the union of their blocks.
 #pragma once
 #include "common.cuh"
 
@@ -348,126 +345,6 @@ __device__ __forceinline__ void stage_tokens(uint32_t ks, uint32_t vs, const __n
     const uint32_t dst = (which ? vs : ks) + (p * kRowPad + part * 8) * 2;
     cp_async16_zfill(dst, src, ok);
   }
-}
-
-// ---------------------------------------------------------------------------
-// Prefill for B in {1, 2, 4}: 8 warps = 8 adjacent queries share the union
-// of their selections, staged once per window of kWinTok tokens.  Each warp
-// compacts the window positions its own query selected (at B = 1 about a
-// fifth of a window) and runs its 16-token MMA steps over those rows only,
-// addressing them through ldmatrix's per-lane row pointers, so the MMA work
-// follows the query's own tokens instead of the union.
-// ---------------------------------------------------------------------------
-constexpr int kWinTok = 64;
-constexpr int kWinStages = 3;
-constexpr int kWinElems = kWinTok * kRowPad;  // one K or V window
-constexpr int kGroupedThreads = 256;
-
-template <int B>
-__global__ void __launch_bounds__(kGroupedThreads, 1)
-attn_grouped_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
-                    const __nv_bfloat16* __restrict__ vc, const int32_t* __restrict__ plan_ids,
-                    const uint8_t* __restrict__ plan_mask, const int32_t* __restrict__ plan_count,
-                    __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ gate, int64_t nq, int G,
-                    int k, int64_t q_pos0, int64_t cache_cap, int64_t cache_len, float scale_log2) {
-  extern __shared__ __align__(16) __nv_bfloat16 smem[];
-  __shared__ int64_t s_tok[kWinStages][kWinTok];
-  __shared__ uint8_t s_own[8][kWinTok];  // per warp: the window positions its query attends, compacted
-  constexpr int E = kWinTok / B;         // union entries per window
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int mrow = lane & 7, mat = lane >> 3;
-  const int64_t nqb = (nq + 7) / 8;
-  const int64_t unit = blockIdx.x;
-  const int g = static_cast<int>(unit % G);
-  const int64_t qb = (unit / G) % nqb;
-  const int64_t seq = unit / (G * nqb);
-  const int64_t i = qb * 8 + warp;
-  const bool qvalid = i < nq;
-  const int64_t t = q_pos0 + (qvalid ? i : qb * 8);
-  const int64_t t_first = q_pos0 + qb * 8;
-  const int64_t c0 = B * (t_first / B);  // current segment start (the unit's current tokens lie in c0 .. c0 + 15)
-  const int U = plan_count[unit];
-  const int32_t* uid = plan_ids + unit * (8 * static_cast<int64_t>(k));
-  const uint8_t* umask = plan_mask + unit * (8 * static_cast<int64_t>(k));
-  const int n_union_win = (U + E - 1) / E;
-  const int n_win = n_union_win + 1;
-  const int64_t row_stride = static_cast<int64_t>(G) * kD;
-  const __nv_bfloat16* kseq = kc + seq * cache_cap * row_stride + g * kD;
-  const __nv_bfloat16* vseq = vc + seq * cache_cap * row_stride + g * kD;
-
-  WarpAttn st;
-  warp_load_q(st, q + ((seq * nq + (qvalid ? i : 0)) * G + g) * kHg * kD, lane);
-
-  auto token_of = [&](int win, int p) -> int64_t {
-    if (win < n_union_win) {
-      const int e = win * E + p / B;
-      if (e >= U) return -1;
-      const int64_t tk = static_cast<int64_t>(uid[e]) * B + (p % B);
-      return (tk >= 0 && tk < cache_len) ? tk : -1;
-    }
-    const int64_t s = c0 + p;
-    return (p < 16 && s < cache_len) ? s : -1;
-  };
-  auto issue = [&](int win) {
-    const int stage = win % kWinStages;
-    if (tid < kWinTok) {
-      const int64_t tk = token_of(win, tid);
-      s_tok[stage][tid] = tk >= 0 ? tk * row_stride : -1;
-    }
-    __syncthreads();
-    const uint32_t ks = smem_u32(smem + (2 * stage) * kWinElems);
-    const uint32_t vs = smem_u32(smem + (2 * stage + 1) * kWinElems);
-    stage_tokens(ks, vs, kseq, vseq, s_tok[stage], tid, kGroupedThreads, kWinTok);
-  };
-  // prologue
-  for (int w = 0; w < kWinStages - 1; ++w) {
-    if (w < n_win) issue(w);
-    cp_async_commit();
-  }
-  const int64_t tcur0 = B * (t / B);
-  const uint32_t lt = (1u << lane) - 1u;
-  for (int win = 0; win < n_win; ++win) {
-    cp_async_wait<kWinStages - 2>();
-    __syncthreads();
-    // the window positions this warp's query attends (lane and lane + 32)
-    bool own0, own1;
-    if (win < n_union_win) {
-      const int e0 = win * E + lane / B, e1 = win * E + (lane + 32) / B;
-      own0 = e0 < U && ((umask[e0] >> warp) & 1u);
-      own1 = e1 < U && ((umask[e1] >> warp) & 1u);
-    } else {
-      const int64_t s0 = c0 + lane;
-      own0 = lane < 16 && s0 >= tcur0 && s0 <= t;
-      own1 = false;
-    }
-    const uint32_t m0 = __ballot_sync(0xffffffffu, own0), m1 = __ballot_sync(0xffffffffu, own1);
-    const int n0 = __popc(m0), n_own = n0 + __popc(m1);
-    if (own0) s_own[warp][__popc(m0 & lt)] = static_cast<uint8_t>(lane);
-    if (own1) s_own[warp][n0 + __popc(m1 & lt)] = static_cast<uint8_t>(lane + 32);
-    __syncwarp();
-    if (qvalid) {
-      const int stage = win % kWinStages;
-      const uint32_t ks = smem_u32(smem + (2 * stage) * kWinElems);
-      const uint32_t vs = smem_u32(smem + (2 * stage + 1) * kWinElems);
-      for (int sub = 0; sub < n_own; sub += kStepTok) {
-        const int left = n_own - sub;
-        const uint32_t tm = left >= kStepTok ? 0xFFFFu : ((1u << left) - 1u);
-        // rows past the compacted list repeat its last row; their scores are masked
-        const int rk = s_own[warp][sub + min(8 * (mat >> 1) + mrow, left - 1)];
-        const int rv = s_own[warp][sub + min(8 * (mat & 1) + mrow, left - 1)];
-        warp_attend_at(st, ks + (rk * kRowPad + 8 * (mat & 1)) * 2, vs + (rv * kRowPad + 8 * (mat >> 1)) * 2, tm,
-                       scale_log2, lane);
-      }
-    }
-    __syncwarp();  // s_own is rewritten for the next window
-    const int nxt = win + kWinStages - 1;
-    if (nxt < n_win) issue(nxt);
-    else __syncthreads();  // keep the barrier count uniform with issue()
-    cp_async_commit();
-  }
-  if (qvalid)
-    warp_store_out(st, out + ((seq * nq + i) * G + g) * kHg * kD,
-                   gate == nullptr ? nullptr : gate + ((seq * nq + i) * G + g) * kHg, lane);
 }
 
 // ---------------------------------------------------------------------------

@@ -7,8 +7,11 @@
 // One CTA takes one unit = (sequence, block of 8 adjacent queries, KV group).
 // The MMA M dimension is the 8 queries x 16 heads = 128 rows, all sharing the
 // group's K/V; the unit walks the sorted union of the 8 queries' selected
-// 8-token blocks (built by attn_plan_kernel) 64 tokens (8 blocks) at a time,
-// then one tile holding the current-block tokens.
+// blocks (built by attn_plan_kernel) 64 tokens at a time (8 blocks of 8, or
+// 64 / BS blocks of BS < 8 tokens), then one tile holding the current-block
+// tokens.  Blocks of 8 tokens arrive by TMA, one box per block; smaller
+// blocks by cp.async row gathers into the same swizzled layout, their masks
+// applied per token.
 //
 // Tensor memory (512 columns, one row per TMEM lane):
 //   [0, 192)    O accumulator, FP32
@@ -74,14 +77,18 @@ struct __align__(1024) AttnTcSmem {
 // block's copy starts at (row 0 or 8 of its page, page).  Otherwise the maps
 // cover the contiguous caches [S, cap, G, D] and a copy starts at (token row,
 // sequence).
-template <bool SKIP_PAIRS, bool PAGED>
+template <bool SKIP_PAIRS, bool PAGED, int BS>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUtensorMap kmap,
                const __grid_constant__ CUtensorMap vmap, const int32_t* __restrict__ plan_ids,
                const uint8_t* __restrict__ plan_mask, const int32_t* __restrict__ plan_count,
                __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ gate, int64_t nq, int G,
                int k, int64_t q_pos0, float scale_log2, const int32_t* __restrict__ page_table, int64_t max_pages,
-               int64_t num_pages) {
+               int64_t num_pages, const __nv_bfloat16* __restrict__ kc, const __nv_bfloat16* __restrict__ vc,
+               int64_t cache_cap, int64_t cache_len) {
+  static_assert(BS == 1 || BS == 2 || BS == 4 || BS == 8, "block size");
+  static_assert(BS == 8 || (!PAGED && !SKIP_PAIRS), "paged pools and pair skipping are for 8-token blocks");
+  constexpr int E = kTcTileTok / BS;  // union entries (blocks) per 64-token tile
   extern __shared__ uint8_t smem_raw[];
   AttnTcSmem& sm = *reinterpret_cast<AttnTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                   ~static_cast<uintptr_t>(1023));
@@ -97,7 +104,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
   const int U = plan_count[unit];
   const int32_t* uid = plan_ids + unit * (8 * static_cast<int64_t>(k));
   const uint8_t* umask = plan_mask + unit * (8 * static_cast<int64_t>(k));
-  const int n_union_tiles = (U + 7) / 8;
+  const int n_union_tiles = (U + E - 1) / E;
   const int n_tiles = n_union_tiles + 1;
   const int64_t t_first = q_pos0 + qb * 8;
   const int64_t t_last = q_pos0 + min(nq, qb * 8 + 8) - 1;
@@ -109,12 +116,14 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
   if (threadIdx.x == 0) {
     sm.abort = 0;
     tc::mbar_init(bar(sm.q_full), 256);
+    // a full K/V stage: one TMA transaction count (8-token blocks) or the
+    // 32 lanes of the copying warp (smaller blocks)
     for (int s = 0; s < kTcStages; ++s) {
-      tc::mbar_init(bar(sm.k_full[s]), 1);
+      tc::mbar_init(bar(sm.k_full[s]), BS == 8 ? 1 : 32);
       tc::mbar_init(bar(sm.k_empty[s]), 1);
     }
     for (int s = 0; s < kTcVStages; ++s) {
-      tc::mbar_init(bar(sm.v_full[s]), 1);
+      tc::mbar_init(bar(sm.v_full[s]), BS == 8 ? 1 : 32);
       tc::mbar_init(bar(sm.v_empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -144,62 +153,134 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     // (K after QK^T, V after PV), so each gets its own issuer.
     const bool is_k = warp == 0;
     const int nst = is_k ? kTcStages : kTcVStages;
-    if (tc::elect_one()) tc::prefetch_tmap(is_k ? &kmap : &vmap);
-    __syncwarp();
-    // Copy rows of the union's blocks, one per lane in batches of four tiles
-    // (32 blocks), loaded a whole batch ahead: the id fetch (an L2 round trip,
-    // plus the page-table read of a paged pool) never sits between two tiles'
-    // copies.  Lane 8 t + e holds block e of tile 4 b + t.  A row is a token
-    // row, or page * 16 + row within the page; negative: a zero-filled box.
-    auto page_row = [&](int64_t tok) -> int32_t {  // paged pool: the row of token tok
-      const int32_t pg = page_table[seq * max_pages + (tok >> 4)];
-      if (pg < 0 || pg >= num_pages) {
-        report(kDevBounds);
-        return -64;
-      }
-      return pg * 16 + static_cast<int32_t>(tok & 15);
-    };
-    auto load_batch = [&](int bt) -> int32_t {
-      const int idx = 32 * bt + lane;
-      const int32_t id = idx < U ? uid[idx] : -1;
-      if (id < 0) return -64;
-      return PAGED ? page_row(static_cast<int64_t>(id) * 8) : id * 8;
-    };
-    int32_t ids_cur = load_batch(0), ids_next = n_union_tiles > 4 ? load_batch(1) : -64;
-    // the current-block tile: the current block and, when the unit spans two blocks, the next
-    int32_t cur_rows = -64;
-    if (lane < 2 && (lane == 0 || c0 + 8 <= t_last))
-      cur_rows = PAGED ? page_row(c0 + 8 * lane) : static_cast<int32_t>(c0 + 8 * lane);
-    for (int j = 0; j < n_tiles; ++j) {
-      const int s = j % nst;
-      if (j > 0 && (j & 3) == 0) {
-        ids_cur = ids_next;
-        if (4 * (j / 4 + 1) < n_union_tiles) ids_next = load_batch(j / 4 + 1);
-      }
-      // this tile's eight copy rows (-64: a zero-filled box)
-      int32_t rows[8];
+    if constexpr (BS < 8) {
+      // Blocks of fewer than 8 tokens: the 32 lanes gather the tile's 64
+      // token rows with cp.async into the layout the TMA boxes produce
+      // (8-row slots, 128-byte swizzle).  Piece L = 32 it + lane of the
+      // tile's 64 x 24 sixteen-byte pieces is piece L % 24 of token L / 24,
+      // so consecutive lanes read consecutive bytes of a row.  Row offsets
+      // are 32-bit counts of 16-byte pieces (a sequence's K of one group up
+      // to 2^31 pieces: 178 M tokens at 4 groups).
+      const uint4* src0 = reinterpret_cast<const uint4*>((is_k ? kc : vc) + (seq * cache_cap * G + g) * static_cast<int64_t>(kD));
+      const uint32_t rstride16 = static_cast<uint32_t>(G) * (kD / 8);  // 16-byte pieces between token rows
+      // this lane's row offsets (16-byte units) of tile positions lane and
+      // lane + 32, -1: a zero row; the union ids are fetched a tile before
+      // they are needed (id_of), the offsets formed from them (row_of)
+      auto id_of = [&](int j, int p) -> int32_t {
+        const int idx = j * E + p / BS;
+        return (j < n_union_tiles && idx < U) ? __ldg(uid + idx) : -1;
+      };
+      auto row_of = [&](int j, int p, int32_t id) -> int32_t {
+        int64_t tk = -1;
+        if (j < n_union_tiles) {
+          if (id >= 0) tk = static_cast<int64_t>(id) * BS + p % BS;
+          if (tk >= cache_len) tk = -1;
+        } else if (p < 16 && c0 + p < cache_len) {
+          tk = c0 + p;
+        }
+        return tk < 0 ? -1 : static_cast<int32_t>(tk * rstride16);
+      };
+      // Iteration it = 3 a + r copies piece c_r of token 4 a + p_r, where
+      // 32 r + lane = 24 p_r + c_r; its destination is the same for every a
+      // of one parity, plus (a >> 1) slots.
+      uint32_t dstc[3][2];
+      int pr[3], cr[3];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int32_t r_union = __shfl_sync(0xffffffffu, ids_cur, 8 * (j & 3) + e);
-        const int32_t r_cur = __shfl_sync(0xffffffffu, cur_rows, e & 1);
-        rows[e] = j < n_union_tiles ? r_union : (e < 2 ? r_cur : -64);
-      }
-      uint64_t* empty = is_k ? &sm.k_empty[s] : &sm.v_empty[s];
-      uint64_t* full = is_k ? &sm.k_full[s] : &sm.v_full[s];
-      if (j >= nst && !tc::warp_wait(bar(*empty), ((j / nst) - 1) & 1, abort, wlim)) break;
-      if (tc::elect_one()) {
-        tc::mbar_expect_tx(bar(*full), 8 * 3 * 1024);
-        const CUtensorMap* map = is_k ? &kmap : &vmap;
+      for (int r = 0; r < 3; ++r) {
+        pr[r] = (32 * r + lane) / 24;
+        cr[r] = (32 * r + lane) % 24;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint32_t dst = is_k ? smem_u32(&sm.k[s][e][0][0]) : smem_u32(&sm.v[s][e][0][0]);
-          const int32_t c1 = PAGED ? (rows[e] & 15) : rows[e];
-          const int32_t c4 = PAGED ? (rows[e] >> 4) : static_cast<int32_t>(seq);
-          tc::tma_load_5d(dst, map, 0, c1, 0, g, c4, bar(*full));
+        for (int par = 0; par < 2; ++par) {
+          const int row = 4 * par + pr[r];  // row within the 8-row slot
+          dstc[r][par] = (cr[r] >> 3) * 1024 + row * 128 + (((cr[r] & 7) ^ row) << 4);
         }
       }
+      int32_t ra = row_of(0, lane, id_of(0, lane)), rb = row_of(0, lane + 32, id_of(0, lane + 32));
+      int32_t na = id_of(1, lane), nb = id_of(1, lane + 32);  // the next tile's ids
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % nst;
+        uint64_t* empty = is_k ? &sm.k_empty[s] : &sm.v_empty[s];
+        uint64_t* full = is_k ? &sm.k_full[s] : &sm.v_full[s];
+        if (j >= nst && !tc::warp_wait(bar(*empty), ((j / nst) - 1) & 1, abort, wlim)) break;
+        const uint32_t dst0 = is_k ? smem_u32(&sm.k[s][0][0][0]) : smem_u32(&sm.v[s][0][0][0]);
+#pragma unroll
+        for (int a = 0; a < 16; ++a) {
+#pragma unroll
+          for (int r = 0; r < 3; ++r) {
+            const int32_t off = __shfl_sync(0xffffffffu, a < 8 ? ra : rb, (4 * a + pr[r]) & 31);
+            cp_async16_zfill(dst0 + (a >> 1) * 3072 + dstc[r][a & 1], src0 + (off >= 0 ? off + cr[r] : 0), off >= 0);
+          }
+        }
+        // the stage is full once every lane has arrived and its copies have
+        // landed (the asynchronous arrive fires when they complete)
+        cp_async_mbar_arrive(bar(*full));
+        tc::mbar_arrive(bar(*full));
+        issued = j + 1;
+        ra = row_of(j + 1, lane, na);
+        rb = row_of(j + 1, lane + 32, nb);
+        na = id_of(j + 2, lane);
+        nb = id_of(j + 2, lane + 32);
+      }
+      cp_async_commit();
+      cp_async_wait<0>();  // nothing may land after the CTA's shared memory is released
+    } else {
+      if (tc::elect_one()) tc::prefetch_tmap(is_k ? &kmap : &vmap);
       __syncwarp();
-      issued = j + 1;
+      // Copy rows of the union's blocks, one per lane in batches of four tiles
+      // (32 blocks), loaded a whole batch ahead: the id fetch (an L2 round trip,
+      // plus the page-table read of a paged pool) never sits between two tiles'
+      // copies.  Lane 8 t + e holds block e of tile 4 b + t.  A row is a token
+      // row, or page * 16 + row within the page; negative: a zero-filled box.
+      auto page_row = [&](int64_t tok) -> int32_t {  // paged pool: the row of token tok
+        const int32_t pg = page_table[seq * max_pages + (tok >> 4)];
+        if (pg < 0 || pg >= num_pages) {
+          report(kDevBounds);
+          return -64;
+        }
+        return pg * 16 + static_cast<int32_t>(tok & 15);
+      };
+      auto load_batch = [&](int bt) -> int32_t {
+        const int idx = 32 * bt + lane;
+        const int32_t id = idx < U ? uid[idx] : -1;
+        if (id < 0) return -64;
+        return PAGED ? page_row(static_cast<int64_t>(id) * 8) : id * 8;
+      };
+      int32_t ids_cur = load_batch(0), ids_next = n_union_tiles > 4 ? load_batch(1) : -64;
+      // the current-block tile: the current block and, when the unit spans two blocks, the next
+      int32_t cur_rows = -64;
+      if (lane < 2 && (lane == 0 || c0 + 8 <= t_last))
+        cur_rows = PAGED ? page_row(c0 + 8 * lane) : static_cast<int32_t>(c0 + 8 * lane);
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % nst;
+        if (j > 0 && (j & 3) == 0) {
+          ids_cur = ids_next;
+          if (4 * (j / 4 + 1) < n_union_tiles) ids_next = load_batch(j / 4 + 1);
+        }
+        // this tile's eight copy rows (-64: a zero-filled box)
+        int32_t rows[8];
+  #pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int32_t r_union = __shfl_sync(0xffffffffu, ids_cur, 8 * (j & 3) + e);
+          const int32_t r_cur = __shfl_sync(0xffffffffu, cur_rows, e & 1);
+          rows[e] = j < n_union_tiles ? r_union : (e < 2 ? r_cur : -64);
+        }
+        uint64_t* empty = is_k ? &sm.k_empty[s] : &sm.v_empty[s];
+        uint64_t* full = is_k ? &sm.k_full[s] : &sm.v_full[s];
+        if (j >= nst && !tc::warp_wait(bar(*empty), ((j / nst) - 1) & 1, abort, wlim)) break;
+        if (tc::elect_one()) {
+          tc::mbar_expect_tx(bar(*full), 8 * 3 * 1024);
+          const CUtensorMap* map = is_k ? &kmap : &vmap;
+  #pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t dst = is_k ? smem_u32(&sm.k[s][e][0][0]) : smem_u32(&sm.v[s][e][0][0]);
+            const int32_t c1 = PAGED ? (rows[e] & 15) : rows[e];
+            const int32_t c4 = PAGED ? (rows[e] >> 4) : static_cast<int32_t>(seq);
+            tc::tma_load_5d(dst, map, 0, c1, 0, g, c4, bar(*full));
+          }
+        }
+        __syncwarp();
+        issued = j + 1;
+      }
     }
   } else if (warp == 1 || warp == 11) {
     // ------------------------------------------------------------ MMA issuers
@@ -280,7 +361,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     const int64_t qi = qb * 8 + qs;
     const bool qvalid = qi < nq;
     const int64_t t = q_pos0 + (qvalid ? qi : qb * 8);
-    const int64_t cur_lo = 8 * (t / 8);
+    const int64_t cur_lo = BS * (t / BS);
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const int64_t orow_idx = ((seq * nq + (qvalid ? qi : 0)) * G + g) * kHg + (m & 15);
     if (half == 0) sm.gfac[m] = gate_factor(gate, orow_idx);  // read by both warps at the end
@@ -307,17 +388,39 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     float m_l = -INFINITY, l = 0.f;          // this warp's partial row sum, relative to 2^m_l
     bool ok = true;
     // mask bytes of this warp's next tile, loaded one own tile (two tiles) ahead
-    uint2 mb_next = half < n_union_tiles ? *reinterpret_cast<const uint2*>(umask + 8 * half) : make_uint2(0u, 0u);
+    uint2 mb_next = make_uint2(0u, 0u);
+    // blocks under 8 tokens: the mask bytes of tile positions lane and lane + 32
+    auto tok_bytes = [&](int jj) -> uint2 {
+      const int i0 = jj * E + lane / BS, i1 = jj * E + (lane + 32) / BS;
+      return make_uint2(jj < n_union_tiles && i0 < U ? umask[i0] : 0u, jj < n_union_tiles && i1 < U ? umask[i1] : 0u);
+    };
+    if (BS == 8) {
+      if (half < n_union_tiles) mb_next = *reinterpret_cast<const uint2*>(umask + 8 * half);
+    } else {
+      mb_next = tok_bytes(half);
+    }
     for (int j = half; j < n_tiles; j += 2) {
       const int b = j % 2;
       const uint32_t tS = tS0 + 64 * b + lane_off;
       const uint32_t tP = tP0 + 32 * b + lane_off;
       const uint2 mb = mb_next;
-      if (j + 2 < n_union_tiles) mb_next = *reinterpret_cast<const uint2*>(umask + 8 * (j + 2));
+      if (BS == 8) {
+        if (j + 2 < n_union_tiles) mb_next = *reinterpret_cast<const uint2*>(umask + 8 * (j + 2));
+      } else {
+        mb_next = tok_bytes(j + 2);
+      }
       // blocks (8 tokens each) of this tile the row attends: the row's query
-      // selected the block, or (current tile) causal positions of its own block
-      uint32_t bmask = 0;
-      if (j < n_union_tiles) {
+      // selected the block, or (current tile) causal positions of its own block;
+      // blocks under 8 tokens: a token mask (bit p: tile position p)
+      uint32_t bmask = 0, tlo = 0, thi = 0;
+      if (BS < 8 && j < n_union_tiles) {
+        const int qa = 2 * quad, qb2 = 2 * quad + 1;
+        const uint32_t la = __ballot_sync(0xffffffffu, (mb.x >> qa) & 1u), ha = __ballot_sync(0xffffffffu, (mb.y >> qa) & 1u);
+        const uint32_t lb = __ballot_sync(0xffffffffu, (mb.x >> qb2) & 1u), hb = __ballot_sync(0xffffffffu, (mb.y >> qb2) & 1u);
+        tlo = (lane >> 4) ? lb : la;
+        thi = (lane >> 4) ? hb : ha;
+        bmask = 0xFFu;
+      } else if (j < n_union_tiles) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const uint32_t byte = ((e < 4 ? mb.x : mb.y) >> (8 * (e & 3))) & 0xFFu;
@@ -338,7 +441,19 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       // with max).  Union tiles mask whole blocks: a block the row does not
       // attend gets the exponent offset -inf below instead of masked scores.
       float bm[8];
-      if (j < n_union_tiles) {
+      if (BS < 8 && j < n_union_tiles) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          bm[e] = -INFINITY;
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            const bool keep = (((e < 4 ? tlo : thi) >> (8 * (e & 3) + x)) & 1u) != 0u;
+            const float v = keep ? __uint_as_float(sr[8 * e + x]) : -INFINITY;
+            sr[8 * e + x] = __float_as_uint(v);
+            bm[e] = fmaxf(bm[e], v);
+          }
+        }
+      } else if (j < n_union_tiles) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const float* x = reinterpret_cast<const float*>(&sr[8 * e]);
@@ -470,7 +585,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
   // its own MMAs (full time bound) before shared memory and TMEM are released.
   __syncthreads();
   if (sm.abort) {
-    if (warp == 0 || warp == 10) {
+    if ((warp == 0 || warp == 10) && BS == 8) {  // (smaller blocks: the copies landed before the loop's end)
       const bool is_k = warp == 0;
       const int nst = is_k ? kTcStages : kTcVStages;
       for (int j = issued > nst ? issued - nst : 0; j < issued; ++j)

@@ -305,6 +305,7 @@ sgqa_status kv_maps(const KvSource& kv, int G, int64_t S, CUtensorMap* km, CUten
   return encode_bf16(vm, kv.v, 5, dims, strides, box, "v_cache");
 }
 
+template <int BS>
 sgqa_status launch_attn_tc(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q,
                            const KvSource& kv, const int32_t* ids, const uint8_t* msk, const int32_t* cnt, void* out,
                            const void* gate, int64_t units, cudaStream_t st) {
@@ -317,14 +318,17 @@ sgqa_status launch_attn_tc(const sgqa_params* p, int64_t S, int64_t q0, int64_t 
   const size_t smem = sizeof(sgqa::AttnTcSmem) + 1024;
   // Selections covering under a quarter of the candidates leave many block
   // pairs unattended by both queries of a warp: skip their exponentials.
+  // (Blocks under 8 tokens: pools are not paged here, and no pairs are skipped.)
   const bool skip_pairs = (q0 + nq - 1) / p->block_size > 4 * static_cast<int64_t>(p->topk);
-  auto kern = kv.paged() ? (skip_pairs ? sgqa::attn_tc_kernel<true, true> : sgqa::attn_tc_kernel<false, true>)
-                         : (skip_pairs ? sgqa::attn_tc_kernel<true, false> : sgqa::attn_tc_kernel<false, false>);
+  auto kern = BS < 8 ? sgqa::attn_tc_kernel<false, false, BS>
+              : kv.paged()
+                  ? (skip_pairs ? sgqa::attn_tc_kernel<BS == 8, BS == 8, BS> : sgqa::attn_tc_kernel<false, BS == 8, BS>)
+                  : (skip_pairs ? sgqa::attn_tc_kernel<BS == 8, false, BS> : sgqa::attn_tc_kernel<false, false, BS>);
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   kern<<<static_cast<unsigned>(units), sgqa::kTcThreads, smem, st>>>(
       static_cast<const __nv_bfloat16*>(q), km, vm, ids, msk, cnt, static_cast<__nv_bfloat16*>(out),
       static_cast<const __nv_bfloat16*>(gate), nq, G, p->topk, q0, scale_log2, kv.page_table, kv.max_pages,
-      kv.num_pages);
+      kv.num_pages, static_cast<const __nv_bfloat16*>(kv.k), static_cast<const __nv_bfloat16*>(kv.v), kv.cap, kv.clen);
   SGQA_LAUNCH_CHECK("attn_tc_kernel");
   return SGQA_OK;
 }
@@ -592,16 +596,7 @@ sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq,
         sel, sel_count, nq, G, k, pow2, q0, B, ids, msk, cnt);
     SGQA_LAUNCH_CHECK("attn_plan_sort_kernel");
   }
-  if constexpr (B == 8) {
-    return launch_attn_tc(p, S, q0, nq, q, kv, ids, msk, cnt, out, gate, units, st);
-  } else {
-    const size_t smem = sgqa::kWinStages * 2 * sgqa::kWinElems * 2;
-    cudaFuncSetAttribute(sgqa::attn_grouped_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    sgqa::attn_grouped_kernel<B><<<static_cast<unsigned>(units), sgqa::kGroupedThreads, smem, st>>>(
-        qb, kb, vb, ids, msk, cnt, ob, gb, nq, G, k, q0, kv.cap, kv.clen, scale_log2);
-    SGQA_LAUNCH_CHECK("attn_grouped_kernel");
-    return SGQA_OK;
-  }
+  return launch_attn_tc<B>(p, S, q0, nq, q, kv, ids, msk, cnt, out, gate, units, st);
 }
 
 sgqa_status do_attn_kv(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq, const void* q, const KvSource& kv,
