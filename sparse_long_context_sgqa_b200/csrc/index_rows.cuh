@@ -516,16 +516,20 @@ __device__ __forceinline__ void dec_strip_scores(uint4 ka, uint4 kb, const uint3
   }
   sa_out = 0.f;
   sb_out = 0.f;
+  // k-steps outside, groups inside: four independent accumulations in flight
+  float acc[4][4];
+#pragma unroll
+  for (int g = 0; g < 4; ++g) acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) {
+    const uint32_t af[4] = {pa[2 * ks], pb[2 * ks], pa[2 * ks + 1], pb[2 * ks + 1]};
+#pragma unroll
+    for (int g = 0; g < 4; ++g) mma_f16_16816(acc[g], af, bf[g][2 * ks], bf[g][2 * ks + 1]);
+  }
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      const uint32_t af[4] = {pa[2 * ks], pb[2 * ks], pa[2 * ks + 1], pb[2 * ks + 1]};
-      mma_f16_16816(acc, af, bf[g][2 * ks], bf[g][2 * ks + 1]);
-    }
-    float sa = wv[g][0] * fmaxf(acc[0], 0.f) + wv[g][1] * fmaxf(acc[1], 0.f);
-    float sb = wv[g][0] * fmaxf(acc[2], 0.f) + wv[g][1] * fmaxf(acc[3], 0.f);
+    float sa = wv[g][0] * fmaxf(acc[g][0], 0.f) + wv[g][1] * fmaxf(acc[g][1], 0.f);
+    float sb = wv[g][0] * fmaxf(acc[g][2], 0.f) + wv[g][1] * fmaxf(acc[g][3], 0.f);
     sa += __shfl_xor_sync(0xffffffffu, sa, 1);
     sa += __shfl_xor_sync(0xffffffffu, sa, 2);
     sb += __shfl_xor_sync(0xffffffffu, sb, 1);
@@ -849,17 +853,20 @@ topk_rows_reg_kernel(const float* __restrict__ scores, int64_t rpad, int64_t nq,
 // histogram of the strip maxima that hold k of them (at least k maxima are
 // >= L, and L sits close above the k-th largest maximum, a little below the
 // row's k-th largest score), collects the candidates >= L (a few more than k
-// on typical rows), and ranks them exactly (score, then smaller id): a linear
+// on typical rows) in one pass over the row, each warp into its own part of
+// the list, and ranks them exactly (score, then smaller id): a linear
 // histogram of their scores finds the bin of the k-th largest, and one warp
-// ranks that bin's few entries.  A row with fewer strips than k has no such bound and keeps every
+// ranks that bin's few entries (by counting when there are at most 64).  A row with fewer strips than k has no such bound and keeps every
 // candidate for the exact rank (the launch sends rows of fewer than 16 k + 128
 // candidates to topk_rows_reg_kernel).  Ids are marked in a bitmap and read out ascending.  A row with more
-// than kBndSelCap such candidates, or a boundary bin of more than 1024 (massive
-// ties), is listed for topk_rows_list_kernel, which ranks the full row.
+// than kBndSelWarpCap such candidates in one warp's share, or a boundary bin of
+// more than 1024 (massive ties), is listed for topk_rows_list_kernel, which
+// ranks the full row.
 // ---------------------------------------------------------------------------
 constexpr int kBndSelThreads = 1024;
 constexpr int kBndSelPer = 32;      // scores of the row each thread holds
 constexpr int kBndSelCap = 4096;    // candidates >= L the exact rank takes
+constexpr int kBndSelWarpCap = kBndSelCap / (kBndSelThreads / 32);  // of them, per warp
 constexpr int kBndSelBins = 2048;
 
 __global__ void __launch_bounds__(kBndSelThreads)
@@ -871,7 +878,8 @@ topk_rows_bound_kernel(const float* __restrict__ scores, int64_t rpad, const flo
   __shared__ uint32_t keep_bits[kBndSelThreads];
   __shared__ int sums[32];
   __shared__ float fmx[32], fmn[32];
-  __shared__ uint32_t s_nsurv, s_lkey, s_bstar, s_rem, s_cnt, s_nb, s_kmin, s_kmax;
+  __shared__ uint32_t s_nsurv, s_lkey, s_bstar, s_rem, s_cnt, s_nb, s_kmin, s_kmax, s_over;
+  __shared__ uint32_t wcount[kBndSelThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t row = blockIdx.x;
   const int64_t i = (row / G) % nq;
@@ -909,6 +917,7 @@ topk_rows_bound_kernel(const float* __restrict__ scores, int64_t rpad, const flo
     s_bstar = 0;
     s_kmin = 0xFFFFFFFFu;
     s_kmax = 0u;
+    s_over = 0;
   }
   __syncthreads();
   float mx = -INFINITY, mn = INFINITY;
@@ -953,75 +962,62 @@ topk_rows_bound_kernel(const float* __restrict__ scores, int64_t rpad, const flo
   }
   __syncthreads();
   const uint32_t lkey = s_lkey;
-  {  // the candidates >= L (thread t reads scores 4 t .. 4 t + 3 of every 4096, twice from L2):
-     // counted per thread, placed by one shared atomic per warp
+  {  // the candidates >= L, one pass (thread t reads scores 4 t .. 4 t + 3 of
+     // every 4096): each warp appends to its own region of the list (no
+     // shared counter), a region that fills up sends the row to the radix kernel
     constexpr int kChunks = kBndSelPer / 4;
-    uint32_t c = 0, kmin = 0xFFFFFFFFu, kmax = 0u;
+    uint2* mine = surv + warp * kBndSelWarpCap;
+    uint32_t cnt = 0, kmin = 0xFFFFFFFFu, kmax = 0u;
 #pragma unroll
     for (int u = 0; u < kChunks; ++u) {
       const int j0 = 4 * tid + 4 * kBndSelThreads * u;
-      if (j0 < n) {
-        const float4 v = *reinterpret_cast<const float4*>(srow + j0);
-        const float vv[4] = {v.x, v.y, v.z, v.w};
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j0 < n) v = *reinterpret_cast<const float4*>(srow + j0);
+      const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t kk = score_key(vv[e]);
-          if (j0 + e < n && kk >= lkey) {
-            ++c;
-            kmin = min(kmin, kk);
-            kmax = max(kmax, kk);
-          }
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t kk = score_key(vv[e]);
+        const bool in = j0 + e < n && kk >= lkey;
+        const uint32_t bal = __ballot_sync(0xffffffffu, in);
+        const uint32_t pos = cnt + __popc(bal & ((1u << lane) - 1u));
+        if (in) {
+          if (pos < static_cast<uint32_t>(kBndSelWarpCap)) mine[pos] = make_uint2(kk, static_cast<uint32_t>(j0 + e));
+          kmin = min(kmin, kk);
+          kmax = max(kmax, kk);
         }
+        cnt += __popc(bal);
       }
-    }
-    uint32_t x = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
     }
     kmin = __reduce_min_sync(0xffffffffu, kmin);
     kmax = __reduce_max_sync(0xffffffffu, kmax);
-    uint32_t wbase = 0;
-    if (lane == 31 && x) {
-      wbase = atomicAdd(&s_nsurv, x);
-      atomicMin(&s_kmin, kmin);
-      atomicMax(&s_kmax, kmax);
-    }
-    uint32_t pos = __shfl_sync(0xffffffffu, wbase, 31) + x - c;
-#pragma unroll
-    for (int u = 0; u < kChunks; ++u) {
-      const int j0 = 4 * tid + 4 * kBndSelThreads * u;
-      if (c != 0 && j0 < n) {
-        const float4 v = *reinterpret_cast<const float4*>(srow + j0);
-        const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t kk = score_key(vv[e]);
-          if (j0 + e < n && kk >= lkey) {
-            if (pos < static_cast<uint32_t>(kBndSelCap)) surv[pos] = make_uint2(kk, static_cast<uint32_t>(j0 + e));
-            ++pos;
-          }
-        }
+    if (lane == 0) {
+      wcount[warp] = cnt;
+      if (cnt) {
+        atomicAdd(&s_nsurv, cnt);
+        atomicMin(&s_kmin, kmin);
+        atomicMax(&s_kmax, kmax);
       }
+      if (cnt > static_cast<uint32_t>(kBndSelWarpCap)) s_over = 1;
     }
   }
   for (int b = tid; b < kBndSelBins; b += kBndSelThreads) hist[b] = 0u;
   __syncthreads();
-  const uint32_t nsurv = s_nsurv;
-  if (nsurv > static_cast<uint32_t>(kBndSelCap)) {  // every thread leaves here together
+  if (s_over) {  // every thread leaves here together
     if (tid == 0) list[atomicAdd(list_count, 1)] = static_cast<int32_t>(row);
     return;
   }
+  // slot x of the list is entry x % cap of warp x / cap's region
+  auto live = [&](int x) { return static_cast<uint32_t>(x % kBndSelWarpCap) < wcount[x / kBndSelWarpCap]; };
   // the exact rank among them: a linear histogram of their scores finds the
   // bin holding the k-th largest; better bins are kept, that bin's entries
-  // (typically one or two) are ranked by one warp
+  // (typically a few) are ranked by one warp
   const float hi = key_score(s_kmax), lo = key_score(s_kmin);
   const float scale2 = hi > lo ? (kBndSelBins - 0.5f) / (hi - lo) : 0.f;
   auto bin2 = [&](uint32_t kk) -> int {
     return min(static_cast<int>(__fmul_rn(__fsub_rn(hi, key_score(kk)), scale2)), kBndSelBins - 1);
   };
-  for (uint32_t e = tid; e < nsurv; e += kBndSelThreads) atomicAdd(&hist[bin2(surv[e].x)], 1u);
+  for (int x = tid; x < kBndSelCap; x += kBndSelThreads)
+    if (live(x)) atomicAdd(&hist[bin2(surv[x].x)], 1u);
   __syncthreads();
   {  // thread t owns bins 2 t, 2 t + 1
     const uint32_t c0 = hist[2 * tid], c1 = hist[2 * tid + 1];
@@ -1055,23 +1051,39 @@ topk_rows_bound_kernel(const float* __restrict__ scores, int64_t rpad, const flo
     return;
   }
   uint2* bnd = reinterpret_cast<uint2*>(hist);  // [kBndSelBins / 2]; the histogram is consumed
-  __syncthreads();
-  for (uint32_t e = tid; e < nsurv; e += kBndSelThreads) {
-    const uint2 x = surv[e];
-    const int b = bin2(x.x);
-    if (b < bstar) atomicOr(&keep_bits[x.y >> 5], 1u << (x.y & 31));
-    else if (b == bstar) bnd[atomicAdd(&s_nb, 1u)] = x;
+  for (int x = tid; x < kBndSelCap; x += kBndSelThreads) {
+    if (!live(x)) continue;
+    const uint2 e = surv[x];
+    const int b = bin2(e.x);
+    if (b < bstar) atomicOr(&keep_bits[e.y >> 5], 1u << (e.y & 31));
+    else if (b == bstar) bnd[atomicAdd(&s_nb, 1u)] = e;
   }
   __syncthreads();
   if (warp == 0) {
     const uint32_t nb = s_nb;
-    uint32_t theta = 0, id_cut = 0xFFFFFFFFu;
-    // warp_select's 256 counters live in the consumed candidate list
-    if (nb > rem) warp_select(bnd, static_cast<int>(nb), static_cast<int>(rem), reinterpret_cast<uint32_t*>(surv), theta,
-                              id_cut);
-    for (uint32_t e = lane; e < nb; e += 32) {
-      const uint2 x = bnd[e];
-      if (nb <= rem || kept(x, theta, id_cut)) atomicOr(&keep_bits[x.y >> 5], 1u << (x.y & 31));
+    if (nb <= rem) {
+      for (uint32_t e = lane; e < nb; e += 32) atomicOr(&keep_bits[bnd[e].y >> 5], 1u << (bnd[e].y & 31));
+    } else if (nb <= 64) {
+      // rank by counting: an entry is kept if fewer than rem entries beat it (score, then smaller id)
+      const uint2 e0 = lane < static_cast<int>(nb) ? bnd[lane] : make_uint2(0u, 0xFFFFFFFFu);
+      const uint2 e1 = lane + 32 < static_cast<int>(nb) ? bnd[lane + 32] : make_uint2(0u, 0xFFFFFFFFu);
+      uint32_t r0 = 0, r1 = 0;
+      for (int q = 0; q < 32; ++q) {
+        const uint2 f0 = make_uint2(__shfl_sync(0xffffffffu, e0.x, q), __shfl_sync(0xffffffffu, e0.y, q));
+        const uint2 f1 = make_uint2(__shfl_sync(0xffffffffu, e1.x, q), __shfl_sync(0xffffffffu, e1.y, q));
+        auto beats = [](uint2 f, uint2 e) { return f.x > e.x || (f.x == e.x && f.y < e.y); };
+        const bool v0 = q < static_cast<int>(nb), v1 = q + 32 < static_cast<int>(nb);
+        r0 += (v0 && beats(f0, e0)) + (v1 && beats(f1, e0));
+        r1 += (v0 && beats(f0, e1)) + (v1 && beats(f1, e1));
+      }
+      if (lane < static_cast<int>(nb) && r0 < rem) atomicOr(&keep_bits[e0.y >> 5], 1u << (e0.y & 31));
+      if (lane + 32 < static_cast<int>(nb) && r1 < rem) atomicOr(&keep_bits[e1.y >> 5], 1u << (e1.y & 31));
+    } else {
+      uint32_t theta = 0, id_cut = 0xFFFFFFFFu;
+      // warp_select's 256 counters live in the consumed candidate list
+      warp_select(bnd, static_cast<int>(nb), static_cast<int>(rem), reinterpret_cast<uint32_t*>(surv), theta, id_cut);
+      for (uint32_t e = lane; e < nb; e += 32)
+        if (kept(bnd[e], theta, id_cut)) atomicOr(&keep_bits[bnd[e].y >> 5], 1u << (bnd[e].y & 31));
     }
   }
   __syncthreads();

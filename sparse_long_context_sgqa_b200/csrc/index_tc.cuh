@@ -891,7 +891,7 @@ index_threshold_kernel(const float* __restrict__ sample, int64_t ld, int64_t nq,
   __shared__ uint32_t wh[kThrThreads / 32][256];
   __shared__ float rmax[kThrThreads / 32], rmin[kThrThreads / 32];
   __shared__ uint32_t wsum[kThrThreads / 32];
-  __shared__ int s_bstar;
+  __shared__ int s_bstar, s_before, s_sub;
   const int64_t row = blockIdx.x;
   const int64_t i = (row / G) % nq;
   const int64_t n = (q_pos0 + i) / B;
@@ -967,12 +967,51 @@ index_threshold_kernel(const float* __restrict__ sample, int64_t ld, int64_t nq,
     __syncthreads();
     uint32_t before = inc - c;
     for (int w = 0; w < warp; ++w) before += wsum[w];
-    if (before < static_cast<uint32_t>(rank) && static_cast<uint32_t>(rank) <= before + c) s_bstar = tid;
+    if (before < static_cast<uint32_t>(rank) && static_cast<uint32_t>(rank) <= before + c) {
+      s_bstar = tid;
+      s_before = static_cast<int>(before);
+    }
+  }
+  __syncthreads();
+  // Second level: the boundary bin's samples in 256 sub-bins, so that the
+  // threshold sits close below the rank-th largest sample even where one bin
+  // of the first level holds many samples (the kept count, about
+  // rank * samp, would otherwise grow by that bin's samples times samp).
+  const int bstar = s_bstar;
+  for (int b = tid; b < (kThrThreads / 32) * 256; b += kThrThreads) (&wh[0][0])[b] = 0u;
+  __syncthreads();
+  const float scale2 = scale * 256.f;
+  auto sub_of = [&](float x) -> int {
+    return min(max(static_cast<int>((mx - x) * scale2) - 256 * bstar, 0), 255);
+  };
+#pragma unroll
+  for (int e = 0; e < kThrPer; ++e)
+    if (v[e] != -INFINITY && bin_of(v[e]) == bstar) atomicAdd(&wh[warp][sub_of(v[e])], 1u);
+  __syncthreads();
+  {
+    const uint32_t rank2 = static_cast<uint32_t>(rank - s_before);
+    uint32_t c = 0;
+#pragma unroll
+    for (int w = 0; w < kThrThreads / 32; ++w) c += wh[w][tid];
+    uint32_t inc = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    __syncthreads();
+    if (lane == 31) wsum[warp] = inc;
+    __syncthreads();
+    uint32_t before = inc - c;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    // the last sub-bin takes the samples the clamp moved there (rounding)
+    if ((before < rank2 && rank2 <= before + c) || (tid == 255 && before + c < rank2)) s_sub = tid;
   }
   __syncthreads();
   if (tid == 0) {
-    // every sample of bin b* (and above) lies strictly above mx - (b* + 1) / scale
-    float t = scale > 0.f ? mx - static_cast<float>(s_bstar + 1) / scale : mx;
+    // every sample of bin b*, sub-bin s* (and above) lies above about
+    // mx - (256 b* + s* + 1) / scale2; a small margin covers the rounding
+    float t = scale > 0.f ? mx - static_cast<float>(256 * bstar + s_sub + 1) / scale2 : mx;
     t -= fabsf(t) * 1e-6f + 1e-30f;
     thr[row] = t;
   }
