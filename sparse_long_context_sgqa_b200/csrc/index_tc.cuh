@@ -179,15 +179,20 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
       // element c * kIdxCand + m (the sample's tile c, or candidate tile c):
       // 32-bit offsets from one base (at most 32 * G rows of o.ld apart) and a
       // bit per slot for the queries the call has
+      // (filter: soff[x] is instead the offset of slot x's (row, quadrant)
+      // list from the CTA's first one, in entries: at most 32 * G * 4 * cap)
       int32_t soff[2 * QW];
       uint32_t vmask = 0;
 #pragma unroll
       for (int x = 0; x < 2 * QW; ++x) {
         const int qs = (64 * part + 32 * (x / QW)) / H + x % QW;
-        soff[x] = static_cast<int32_t>(static_cast<int64_t>(qs) * G * o.ld);
+        soff[x] = MODE == kScoreFilter ? static_cast<int32_t>(qs * G * 4 * o.cap)
+                                       : static_cast<int32_t>(static_cast<int64_t>(qs) * G * o.ld);
         vmask |= static_cast<uint32_t>(qs < nq_here) << x;
       }
       float* const sbase = MODE == kScoreFilter ? nullptr : o.scores + row0 * o.ld + m;
+      uint2* const lbase = MODE == kScoreFilter ? o.staging + (row0 * 4 + quad) * o.cap : nullptr;
+      const uint32_t lt_mask = (1u << lane) - 1u;
       for (int c = 0; c < n_loop; ++c) {
         const int ab = c & 1;
         if (!tc::mbar_wait(bar(sm.acc_full[ab]), (c >> 1) & 1, abort, wlim)) break;
@@ -238,17 +243,15 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
             if (MODE != kScoreFilter) {
               if ((vmask >> x) & 1u) tb[soff[x]] = acc;
             } else {
-              const int64_t row = row0 + static_cast<int64_t>(qs) * G;
               // keep the score if it reaches the row's threshold (rows past the
               // call's queries have threshold +inf); each (row, quadrant) has its
               // own list, filled in ballot order: no shared counters
               bool pass = acc >= __uint_as_float(sm.thr[qs]);
               if (tail) pass = pass && r < sm.ncand[qs];
               const uint32_t bal = __ballot_sync(0xffffffffu, pass);
-              if (bal) {
-                const int pos = kept[x] + __popc(bal & ((1u << lane) - 1u));
-                if (pass && pos < o.cap)
-                  o.staging[(row * 4 + quad) * o.cap + pos] = make_uint2(score_key(acc), static_cast<uint32_t>(r));
+              if (bal) {  // (long rows: most strips of 32 candidates have none)
+                const int pos = kept[x] + __popc(bal & lt_mask);
+                if (pass && pos < o.cap) lbase[soff[x] + pos] = make_uint2(score_key(acc), static_cast<uint32_t>(r));
                 kept[x] += __popc(bal);
               }
             }
@@ -1178,25 +1181,33 @@ topk_staged_kernel(const uint2* __restrict__ staging, const int32_t* __restrict_
 
 // Exact top-k of a row's staged (key, id) lists for k > 512 (up to 2048),
 // from up to four lists of 4096 entries: 1024 threads hold 16 entries each.
-// A linear 256-bin histogram between the kept scores' minimum and maximum
+// A linear 2048-bin histogram between the kept scores' minimum and maximum
 // finds the bin holding the k-th largest; entries of higher bins are taken,
 // the boundary bin's entries are ranked exactly (score, then smaller id) by
-// one warp.  The taken ids are collected unordered and sorted ascending
-// (bitonic) in shared memory, so the output does not need a bitmap over the
-// whole candidate range (rows reach 1M candidates).  Rows with fewer than k
-// kept entries, an overflowing list or a boundary bin larger than its buffer
-// (massive exact ties) are flagged and listed for the fallback.
+// one warp (by counting when there are at most 64).  Each list holds its ids
+// ascending (the score kernel appends candidate tiles in order), so the taken
+// entries of a list stay ascending: the output is the merge of four sorted
+// runs -- each taken entry's place is its rank in its own run plus, in each
+// other run, the number of taken ids below its own (a binary search).  Rows
+// with fewer than k kept entries, an overflowing list or a boundary bin
+// larger than its buffer (massive exact ties) are flagged and listed for the
+// fallback.
 constexpr int kStagedBigThreads = 1024;
 constexpr int kStagedBigPer = 16;
 constexpr int kStagedBigBnd = 4096;  // boundary entries resolved in the kernel
+constexpr int kStagedBigBins = 2048;
 constexpr int kStagedBigWarps = kStagedBigThreads / 32;
+constexpr int kStagedBigEntries = kStagedBigThreads * kStagedBigPer;
 struct StagedBigSmem {
-  uint2 cand[kStagedBigBnd];
-  uint32_t ids[2048];
-  uint32_t wh[kStagedBigWarps][256];
+  uint2 bnd[kStagedBigBnd];                   // boundary entries (key, id)
+  uint32_t bj[kStagedBigBnd];                 // their entry indices
+  uint32_t hist[kStagedBigBins];              // (then warp_select's counters)
+  uint32_t tbits[kStagedBigEntries / 32];     // taken entries, bit j = entry j
+  uint32_t wpre[kStagedBigEntries / 32];      // taken entries before each word
+  uint32_t T[2048];                           // taken ids, the four runs one after the other
   float rmax[kStagedBigWarps], rmin[kStagedBigWarps];
   uint32_t wsum[kStagedBigWarps];
-  uint32_t bstar, rem, nc, nsel, cstar;
+  uint32_t bstar, rem, cstar, nb, runs[5];
 };
 
 __global__ void __launch_bounds__(kStagedBigThreads)
@@ -1227,22 +1238,21 @@ topk_staged_sort_kernel(const uint2* __restrict__ staging, const int32_t* __rest
       list[atomicAdd(list_count, 1)] = static_cast<int32_t>(row);
     }
   };
-  if (cnt < k || c4.x > cap || c4.y > cap || c4.z > cap || c4.w > cap || cnt > kStagedBigThreads * kStagedBigPer) {
+  if (cnt < k || c4.x > cap || c4.y > cap || c4.z > cap || c4.w > cap || cnt > kStagedBigEntries) {
     flag_row();
     return;
   }
   const int p1 = c4.x, p2 = p1 + c4.y, p3 = p2 + c4.z;
   const uint2* lists = staging + row * 4 * static_cast<int64_t>(cap);
+  auto run_of = [&](int j) { return (j >= p1) + (j >= p2) + (j >= p3); };
   auto entry = [&](int j) -> uint2 {
-    const int q = (j >= p1) + (j >= p2) + (j >= p3);
+    const int q = run_of(j);
     const int off = j - (q == 0 ? 0 : q == 1 ? p1 : q == 2 ? p2 : p3);
     return lists[q * static_cast<int64_t>(cap) + off];
   };
-  for (int b = tid; b < kStagedBigWarps * 256; b += kStagedBigThreads) (&sm.wh[0][0])[b] = 0u;
-  if (tid == 0) {
-    sm.nc = 0;
-    sm.nsel = 0;
-  }
+  for (int b = tid; b < kStagedBigBins; b += kStagedBigThreads) sm.hist[b] = 0u;
+  for (int w = tid; w < kStagedBigEntries / 32; w += kStagedBigThreads) sm.tbits[w] = 0u;
+  if (tid == 0) sm.nb = 0;
   uint2 e[kStagedBigPer];  // (key, id); the score is key_score(key)
   float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
@@ -1270,40 +1280,37 @@ topk_staged_sort_kernel(const uint2* __restrict__ staging, const int32_t* __rest
     mn = fminf(mn, sm.rmin[w]);
   }
   const float width = mx - mn;
-  const float scale = width > 0.f ? 255.5f / width : 0.f;
+  const float scale = width > 0.f ? (kStagedBigBins - 0.5f) / width : 0.f;
   // bins ordered best first; the product rounds monotonically, so a higher
   // score never falls in a later bin
-  auto bin_of = [&](float x) -> int { return min(static_cast<int>(__fmul_rn(__fsub_rn(mx, x), scale)), 255); };
+  auto bin_of = [&](float x) -> int {
+    return min(static_cast<int>(__fmul_rn(__fsub_rn(mx, x), scale)), kStagedBigBins - 1);
+  };
 #pragma unroll
   for (int x = 0; x < kStagedBigPer; ++x)
-    if (tid + kStagedBigThreads * x < cnt) atomicAdd(&sm.wh[warp][bin_of(key_score(e[x].x))], 1u);
+    if (tid + kStagedBigThreads * x < cnt) atomicAdd(&sm.hist[bin_of(key_score(e[x].x))], 1u);
   __syncthreads();
-  if (warp == 0) {
-    // 256 bins, 8 per lane: the bin in which the running count reaches k
-    uint32_t loc[8], sum = 0;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      uint32_t c = 0;
-      for (int w = 0; w < kStagedBigWarps; ++w) c += sm.wh[w][lane * 8 + q];
-      loc[q] = c;
-      sum += c;
-    }
-    uint32_t inc = sum;
+  {  // thread t owns bins 2 t, 2 t + 1: the bin in which the running count reaches k
+    const uint32_t c0 = sm.hist[2 * tid], c1 = sm.hist[2 * tid + 1];
+    uint32_t x = c0 + c1;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += y;
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
     }
-    uint32_t acc = inc - sum;
+    if (lane == 31) sm.wsum[warp] = x;
+    __syncthreads();
+    uint32_t before = x - c0 - c1;
+    for (int w = 0; w < warp; ++w) before += sm.wsum[w];
     const uint32_t kk = static_cast<uint32_t>(k);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      if (acc < kk && kk <= acc + loc[q]) {
-        sm.bstar = lane * 8 + q;
-        sm.rem = kk - acc;
-        sm.cstar = loc[q];
-      }
-      acc += loc[q];
+    if (before < kk && kk <= before + c0) {
+      sm.bstar = 2 * tid;
+      sm.rem = kk - before;
+      sm.cstar = c0;
+    } else if (before + c0 < kk && kk <= before + c0 + c1) {
+      sm.bstar = 2 * tid + 1;
+      sm.rem = kk - before - c0;
+      sm.cstar = c1;
     }
   }
   __syncthreads();
@@ -1315,51 +1322,103 @@ topk_staged_sort_kernel(const uint2* __restrict__ staging, const int32_t* __rest
   const uint32_t rem = sm.rem;
 #pragma unroll
   for (int x = 0; x < kStagedBigPer; ++x) {
-    if (tid + kStagedBigThreads * x >= cnt) continue;
+    const int j = tid + kStagedBigThreads * x;
+    if (j >= cnt) continue;
     const int b = bin_of(key_score(e[x].x));
     if (b < bstar) {
-      sm.ids[atomicAdd(&sm.nsel, 1u)] = e[x].y;
+      atomicOr(&sm.tbits[j >> 5], 1u << (j & 31));
     } else if (b == bstar) {
-      sm.cand[atomicAdd(&sm.nc, 1u)] = e[x];
+      const uint32_t pos = atomicAdd(&sm.nb, 1u);
+      sm.bnd[pos] = e[x];
+      sm.bj[pos] = static_cast<uint32_t>(j);
     }
   }
   __syncthreads();
-  const uint32_t nc = sm.nc;
   if (warp == 0) {
-    uint32_t theta = 0, id_cut = 0xFFFFFFFFu;
-    if (nc > rem) warp_select(sm.cand, static_cast<int>(nc), static_cast<int>(rem), sm.wh[0], theta, id_cut);
-    const uint32_t base = sm.nsel;  // k - rem entries above the boundary bin
-    uint32_t taken = 0;
-    for (uint32_t c0 = 0; c0 < nc; c0 += 32) {
-      const uint32_t c = c0 + lane;
-      const bool take = c < nc && (nc <= rem || kept(sm.cand[c], theta, id_cut));
-      const uint32_t bal = __ballot_sync(0xffffffffu, take);
-      if (take) sm.ids[base + taken + __popc(bal & ((1u << lane) - 1u))] = sm.cand[c].y;
-      taken += __popc(bal);
-    }
-  }
-  __syncthreads();
-  // ascending ids: bitonic sort of the k taken ids (padded to a power of two)
-  int pow2 = 1;
-  while (pow2 < k) pow2 <<= 1;
-  for (int j = k + tid; j < pow2; j += kStagedBigThreads) sm.ids[j] = 0xFFFFFFFFu;
-  __syncthreads();
-  for (int size = 2; size <= pow2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int c = tid; c < pow2 / 2; c += kStagedBigThreads) {
-        const int lo = 2 * stride * (c / stride) + (c % stride);
-        const int hi = lo + stride;
-        const bool asc = (lo & size) == 0;
-        const uint32_t a = sm.ids[lo], b = sm.ids[hi];
-        if ((a > b) == asc) {
-          sm.ids[lo] = b;
-          sm.ids[hi] = a;
-        }
+    const uint32_t nb = sm.nb;
+    auto take = [&](uint32_t c) { atomicOr(&sm.tbits[sm.bj[c] >> 5], 1u << (sm.bj[c] & 31)); };
+    if (nb <= rem) {
+      for (uint32_t c = lane; c < nb; c += 32) take(c);
+    } else if (nb <= 64) {
+      // rank by counting: an entry is taken if fewer than rem entries beat it (score, then smaller id)
+      const uint2 e0 = lane < static_cast<int>(nb) ? sm.bnd[lane] : make_uint2(0u, 0xFFFFFFFFu);
+      const uint2 e1 = lane + 32 < static_cast<int>(nb) ? sm.bnd[lane + 32] : make_uint2(0u, 0xFFFFFFFFu);
+      uint32_t r0 = 0, r1 = 0;
+      for (int q = 0; q < 32; ++q) {
+        const uint2 f0 = make_uint2(__shfl_sync(0xffffffffu, e0.x, q), __shfl_sync(0xffffffffu, e0.y, q));
+        const uint2 f1 = make_uint2(__shfl_sync(0xffffffffu, e1.x, q), __shfl_sync(0xffffffffu, e1.y, q));
+        auto beats = [](uint2 f, uint2 g) { return f.x > g.x || (f.x == g.x && f.y < g.y); };
+        const bool v0 = q < static_cast<int>(nb), v1 = q + 32 < static_cast<int>(nb);
+        r0 += (v0 && beats(f0, e0)) + (v1 && beats(f1, e0));
+        r1 += (v0 && beats(f0, e1)) + (v1 && beats(f1, e1));
       }
-      __syncthreads();
+      if (lane < static_cast<int>(nb) && r0 < rem) take(lane);
+      if (lane + 32 < static_cast<int>(nb) && r1 < rem) take(lane + 32);
+    } else {
+      uint32_t theta = 0, id_cut = 0xFFFFFFFFu;
+      warp_select(sm.bnd, static_cast<int>(nb), static_cast<int>(rem), sm.hist, theta, id_cut);
+      for (uint32_t c = lane; c < nb; c += 32)
+        if (kept(sm.bnd[c], theta, id_cut)) take(c);
     }
   }
-  for (int j = tid; j < k; j += kStagedBigThreads) out[j] = static_cast<int32_t>(sm.ids[j]);
+  __syncthreads();
+  // taken entries before each bitmap word (exclusive scan over 512 words)
+  if (tid < kStagedBigEntries / 32) {
+    const uint32_t c = __popc(sm.tbits[tid]);
+    uint32_t x = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) sm.wsum[warp] = x;
+    sm.wpre[tid] = x - c;  // within the warp; the earlier warps' totals are added below
+  }
+  __syncthreads();
+  if (tid < kStagedBigEntries / 32) {
+    uint32_t add = 0;
+    for (int w = 0; w < warp; ++w) add += sm.wsum[w];
+    sm.wpre[tid] += add;
+  }
+  __syncthreads();
+  auto rank_all = [&](int j) -> uint32_t {  // taken entries before entry j
+    return sm.wpre[j >> 5] + __popc(sm.tbits[j >> 5] & ((1u << (j & 31)) - 1u));
+  };
+  if (tid == 0) {  // (a run that starts at cnt is empty: every taken entry lies before it)
+    sm.runs[0] = 0;
+    sm.runs[1] = p1 < cnt ? rank_all(p1) : static_cast<uint32_t>(k);
+    sm.runs[2] = p2 < cnt ? rank_all(p2) : static_cast<uint32_t>(k);
+    sm.runs[3] = p3 < cnt ? rank_all(p3) : static_cast<uint32_t>(k);
+    sm.runs[4] = static_cast<uint32_t>(k);
+  }
+#pragma unroll
+  for (int x = 0; x < kStagedBigPer; ++x) {
+    const int j = tid + kStagedBigThreads * x;
+    if (j < cnt && ((sm.tbits[j >> 5] >> (j & 31)) & 1u)) sm.T[rank_all(j)] = e[x].y;
+  }
+  __syncthreads();
+  // merge of the four ascending runs: place = own rank + taken ids below it in the other runs
+#pragma unroll
+  for (int x = 0; x < kStagedBigPer; ++x) {
+    const int j = tid + kStagedBigThreads * x;
+    if (j >= cnt || !((sm.tbits[j >> 5] >> (j & 31)) & 1u)) continue;
+    const int q = run_of(j);
+    const uint32_t id = e[x].y;
+    uint32_t pos = rank_all(j) - sm.runs[q];
+#pragma unroll
+    for (int q2 = 0; q2 < 4; ++q2) {
+      if (q2 == q) continue;
+      uint32_t lo = sm.runs[q2], hi = sm.runs[q2 + 1];  // first taken id >= id in [lo, hi)
+      const uint32_t base = lo;
+      while (lo < hi) {
+        const uint32_t mid = (lo + hi) >> 1;
+        if (sm.T[mid] < id) lo = mid + 1;
+        else hi = mid;
+      }
+      pos += lo - base;
+    }
+    if (pos < static_cast<uint32_t>(k)) out[pos] = static_cast<int32_t>(id);
+  }
   if (tid == 0) {
     sel_count[row] = k;
     flags[row] = 0;

@@ -135,7 +135,7 @@ def test_index_topk_parity(cuda_device, case):
 
 
 @pytest.mark.parametrize("case", ["short_rows", "filtered_rows", "filtered_rows_65k", "dup_short", "dup_long",
-                                  "decode_rows", "dup_decode"])
+                                  "decode_rows", "dup_decode", "filtered_k2048", "dup_k2048"])
 def test_index_topk_exact_ties(cuda_device, case):
     """Exact score ties, which the selection must break toward smaller block ids.
 
@@ -159,9 +159,17 @@ def test_index_topk_exact_ties(cuda_device, case):
     to 64 by ranking, larger ones by the warp radix select).  The selected
     members of the boundary group must be its smallest ids.  dup_short has
     600..2903 candidates per row, dup_long 15360..16383, dup_decode 32762..32765
-    (the cluster select ranks each boundary group itself)."""
+    (the cluster select ranks each boundary group itself).
+
+    filtered_k2048 / dup_k2048: B = 1 and top-2048 (the 1M-context B = 1
+    variant's selection) at 32768..33023 candidates: the filtered path with
+    kept lists of 2k and the select for k above 512, which merges the four
+    ascending lists' taken ids."""
     dup = case.startswith("dup")
-    if case in ("decode_rows", "dup_decode"):
+    if case in ("filtered_k2048", "dup_k2048"):
+        wl = dataclasses.replace(WL["prefill8k"], name="ties_k2048", seq_len=40960, block=1, topk=2048)
+        q0, nq = 32768, 256  # candidates 32768 .. 33023 per query (B = 1)
+    elif case in ("decode_rows", "dup_decode"):
         wl = dataclasses.replace(WL["prefill8k"], name="ties_decode", seq_len=262144, topk=512)
         q0, nq = 262100, 32  # candidates 32762 .. 32765 per query, the decode path
     elif case in ("short_rows", "dup_short"):
@@ -200,7 +208,8 @@ def test_index_topk_exact_ties(cuda_device, case):
     assert np.all(sel[zero_np] == np.arange(wl.topk, dtype=np.int32))
     iq, iw = Hn.to_np(qs["idx_q"]), Hn.to_np(qs["idx_w"])
     ties = 0
-    step = {"short_rows": 397, "dup_short": 397, "filtered_rows_65k": 397, "decode_rows": 2, "dup_decode": 2}.get(case, 97)
+    step = {"short_rows": 397, "dup_short": 397, "filtered_rows_65k": 397, "decode_rows": 2, "dup_decode": 2,
+            "filtered_k2048": 19, "dup_k2048": 19}.get(case, 97)
     rows = [i for i in range(1, nq, step) if not zero_np[i]] + [nq - 1]
     for i in rows:
         for g in range(wl.groups):
