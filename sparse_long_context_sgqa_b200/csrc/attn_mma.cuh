@@ -35,18 +35,21 @@ constexpr int kPlanThreads = 512;
 
 // The candidate ids of a unit are < floor(t_last / B); a bitmap over that range
 // (one bit per block, in shared memory) turns the union into set-bit order:
-// set bits, prefix-popcount the words, then every (query, id) finds its union
-// position from the prefix and ORs its query bit into that entry's mask, in
+// set bits, prefix-popcount the words (the prefix kept for every eighth word,
+// so a 1M-token range at B = 1 fits: 128 KB of bitmap, 16 KB of prefix), then
+// every (query, id) finds its union position from the prefix and the counts
+// of at most eight words, and ORs its query bit into that entry's mask, in
 // shared memory; the masks go out with 8-byte stores.
 __global__ void __launch_bounds__(kPlanThreads)
 attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ sel_count,
                  int64_t nq, int G, int k, int nwords, int64_t q_pos0, int B, int32_t* __restrict__ plan_ids,
                  uint8_t* __restrict__ plan_mask, int32_t* __restrict__ plan_count) {
-  // [nwords] bitmap, [nwords] prefix, then the union's masks (8k bytes)
+  // [nwords] bitmap, [ngroups] prefix of every eighth word, then the union's masks (8k bytes)
   extern __shared__ __align__(16) uint32_t sm_words[];
+  const int ngroups = (nwords + 7) / 8;
   uint32_t* bm = sm_words;
   uint32_t* pre = sm_words + nwords;
-  uint32_t* msk = sm_words + 2 * nwords;  // 8-byte aligned
+  uint32_t* msk = sm_words + nwords + ngroups + ((nwords + ngroups) & 1);  // 8-byte aligned
   __shared__ int warp_sums[kPlanThreads / 32];
   __shared__ int s_total;
   const int64_t nqb = (nq + 7) / 8;
@@ -94,7 +97,7 @@ attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ se
   int run = (warp > 0 ? warp_sums[warp - 1] : 0) + x - local;
   const int64_t obase = unit * (8 * static_cast<int64_t>(k));
   for (int w = w0; w < w1; ++w) {
-    pre[w] = run;
+    if ((w & 7) == 0) pre[w >> 3] = run;
     uint32_t bits = bm[w];
     int pos = run;
     while (bits) {
@@ -113,7 +116,9 @@ attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ se
     for (int j = tid; j < cnt; j += kPlanThreads) {
       const int id = sel[row * k + j];
       if (id < 0 || id >= lim) continue;
-      const int pos = pre[id >> 5] + __popc(bm[id >> 5] & ((1u << (id & 31)) - 1u));
+      const int w = id >> 5;
+      int pos = pre[w >> 3] + __popc(bm[w] & ((1u << (id & 31)) - 1u));
+      for (int v = w & ~7; v < w; ++v) pos += __popc(bm[v]);
       atomicOr(&msk[pos >> 2], (1u << q) << (8 * (pos & 3)));
     }
   }

@@ -576,6 +576,17 @@ def test_forward_prefill1m_last_chunk(cuda_device):
     _e2e(wl, cuda_device, Hn.sample_rows(wl, 64))
 
 
+def test_forward_prefill1m_b1_last_chunk(cuda_device):
+    """The last 8192-query chunk of the 1M-token prefill with B = 1 and
+    top-2048 tokens (the pages' comparison variant): rows of
+    1040384..1048575 candidates take the filtered path with kept lists of 2k
+    and the select for k above 512; the union of 8 queries' tokens spans a
+    1M-token range (the bitmap planner with its compact prefix) and the
+    attention gathers token rows by cp.async."""
+    wl = dataclasses.replace(WL["prefill1m_b1"], q_start=1048576 - 8192)
+    _e2e(wl, cuda_device, Hn.sample_rows(wl, 24))
+
+
 def test_forward_prefill1m_mid_chunk(cuda_device):
     """A chunk in the middle of the 1M-token prefill: queries 327680..335871,
     rows of 40960..41983 candidates."""
