@@ -35,18 +35,19 @@ constexpr int kPlanThreads = 512;
 
 // The candidate ids of a unit are < floor(t_last / B); a bitmap over that range
 // (one bit per block, in shared memory) turns the union into set-bit order:
-// set bits, prefix-popcount the words (the prefix kept for every eighth word,
-// so a 1M-token range at B = 1 fits: 128 KB of bitmap, 16 KB of prefix), then
-// every (query, id) finds its union position from the prefix and the counts
-// of at most eight words, and ORs its query bit into that entry's mask, in
-// shared memory; the masks go out with 8-byte stores.
+// set bits, prefix-popcount the words (the prefix kept for every word, or --
+// pshift = 3, wide ranges -- for every eighth word, so that a 1M-token range
+// at B = 1 fits: 128 KB of bitmap, 16 KB of prefix), then every (query, id)
+// finds its union position from the prefix and the counts of the words since,
+// and ORs its query bit into that entry's mask, in shared memory; the masks
+// go out with 8-byte stores.
 __global__ void __launch_bounds__(kPlanThreads)
 attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ sel_count,
-                 int64_t nq, int G, int k, int nwords, int64_t q_pos0, int B, int32_t* __restrict__ plan_ids,
-                 uint8_t* __restrict__ plan_mask, int32_t* __restrict__ plan_count) {
-  // [nwords] bitmap, [ngroups] prefix of every eighth word, then the union's masks (8k bytes)
+                 int64_t nq, int G, int k, int nwords, int pshift, int64_t q_pos0, int B,
+                 int32_t* __restrict__ plan_ids, uint8_t* __restrict__ plan_mask, int32_t* __restrict__ plan_count) {
+  // [nwords] bitmap, [ngroups] prefix of every (1 << pshift)-th word, then the union's masks (8k bytes)
   extern __shared__ __align__(16) uint32_t sm_words[];
-  const int ngroups = (nwords + 7) / 8;
+  const int ngroups = ((nwords - 1) >> pshift) + 1;
   uint32_t* bm = sm_words;
   uint32_t* pre = sm_words + nwords;
   uint32_t* msk = sm_words + nwords + ngroups + ((nwords + ngroups) & 1);  // 8-byte aligned
@@ -97,7 +98,7 @@ attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ se
   int run = (warp > 0 ? warp_sums[warp - 1] : 0) + x - local;
   const int64_t obase = unit * (8 * static_cast<int64_t>(k));
   for (int w = w0; w < w1; ++w) {
-    if ((w & 7) == 0) pre[w >> 3] = run;
+    if ((w & ((1 << pshift) - 1)) == 0) pre[w >> pshift] = run;
     uint32_t bits = bm[w];
     int pos = run;
     while (bits) {
@@ -117,8 +118,8 @@ attn_plan_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ se
       const int id = sel[row * k + j];
       if (id < 0 || id >= lim) continue;
       const int w = id >> 5;
-      int pos = pre[w >> 3] + __popc(bm[w] & ((1u << (id & 31)) - 1u));
-      for (int v = w & ~7; v < w; ++v) pos += __popc(bm[v]);
+      int pos = pre[w >> pshift] + __popc(bm[w] & ((1u << (id & 31)) - 1u));
+      for (int v = (w >> pshift) << pshift; v < w; ++v) pos += __popc(bm[v]);
       atomicOr(&msk[pos >> 2], (1u << q) << (8 * (pos & 3)));
     }
   }

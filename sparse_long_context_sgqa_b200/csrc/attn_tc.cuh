@@ -110,7 +110,6 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
   const int64_t t_last = q_pos0 + min(nq, qb * 8 + 8) - 1;
   const int64_t c0 = 8 * (t_first / 8);  // first token of the current segment
   volatile int* abort = &sm.abort;
-  const uint32_t wlim = tc::wait_limit();  // pipeline wait limit of this launch
 
   auto bar = [](uint64_t& b) { return smem_u32(&b); };
   if (threadIdx.x == 0) {
@@ -201,7 +200,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
         const int s = j % nst;
         uint64_t* empty = is_k ? &sm.k_empty[s] : &sm.v_empty[s];
         uint64_t* full = is_k ? &sm.k_full[s] : &sm.v_full[s];
-        if (j >= nst && !tc::warp_wait(bar(*empty), ((j / nst) - 1) & 1, abort, wlim)) break;
+        if (j >= nst && !tc::warp_wait(bar(*empty), ((j / nst) - 1) & 1, abort)) break;
         const uint32_t dst0 = is_k ? smem_u32(&sm.k[s][0][0][0]) : smem_u32(&sm.v[s][0][0][0]);
 #pragma unroll
         for (int a = 0; a < 16; ++a) {
@@ -239,17 +238,17 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
         }
         return pg * 16 + static_cast<int32_t>(tok & 15);
       };
+      // contiguous caches: the raw ids (a row is id * 8); a paged pool: the rows
       auto load_batch = [&](int bt) -> int32_t {
         const int idx = 32 * bt + lane;
         const int32_t id = idx < U ? uid[idx] : -1;
-        if (id < 0) return -64;
-        return PAGED ? page_row(static_cast<int64_t>(id) * 8) : id * 8;
+        if (!PAGED) return id;
+        return id < 0 ? -64 : page_row(static_cast<int64_t>(id) * 8);
       };
-      int32_t ids_cur = load_batch(0), ids_next = n_union_tiles > 4 ? load_batch(1) : -64;
+      int32_t ids_cur = load_batch(0), ids_next = n_union_tiles > 4 ? load_batch(1) : -1;
       // the current-block tile: the current block and, when the unit spans two blocks, the next
       int32_t cur_rows = -64;
-      if (lane < 2 && (lane == 0 || c0 + 8 <= t_last))
-        cur_rows = PAGED ? page_row(c0 + 8 * lane) : static_cast<int32_t>(c0 + 8 * lane);
+      if (PAGED && lane < 2 && (lane == 0 || c0 + 8 <= t_last)) cur_rows = page_row(c0 + 8 * lane);
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % nst;
         if (j > 0 && (j & 3) == 0) {
@@ -258,19 +257,25 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
         }
         // this tile's eight copy rows (-64: a zero-filled box)
         int32_t rows[8];
-  #pragma unroll
+#pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const int32_t r_union = __shfl_sync(0xffffffffu, ids_cur, 8 * (j & 3) + e);
-          const int32_t r_cur = __shfl_sync(0xffffffffu, cur_rows, e & 1);
-          rows[e] = j < n_union_tiles ? r_union : (e < 2 ? r_cur : -64);
+          const int32_t id = __shfl_sync(0xffffffffu, ids_cur, 8 * (j & 3) + e);
+          if (PAGED) {
+            const int32_t r_cur = __shfl_sync(0xffffffffu, cur_rows, e & 1);
+            rows[e] = j < n_union_tiles ? id : (e < 2 ? r_cur : -64);
+          } else if (j < n_union_tiles) {
+            rows[e] = id >= 0 ? id * 8 : -64;
+          } else {  // the current block and, when the unit spans two blocks, the next
+            rows[e] = (e == 0 || (e == 1 && c0 + 8 <= t_last)) ? static_cast<int32_t>(c0 + 8 * e) : -64;
+          }
         }
         uint64_t* empty = is_k ? &sm.k_empty[s] : &sm.v_empty[s];
         uint64_t* full = is_k ? &sm.k_full[s] : &sm.v_full[s];
-        if (j >= nst && !tc::warp_wait(bar(*empty), ((j / nst) - 1) & 1, abort, wlim)) break;
+        if (j >= nst && !tc::warp_wait(bar(*empty), ((j / nst) - 1) & 1, abort)) break;
         if (tc::elect_one()) {
           tc::mbar_expect_tx(bar(*full), 8 * 3 * 1024);
           const CUtensorMap* map = is_k ? &kmap : &vmap;
-  #pragma unroll
+#pragma unroll
           for (int e = 0; e < 8; ++e) {
             const uint32_t dst = is_k ? smem_u32(&sm.k[s][e][0][0]) : smem_u32(&sm.v[s][e][0][0]);
             const int32_t c1 = PAGED ? (rows[e] & 15) : rows[e];
@@ -299,12 +304,12 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     const uint64_t dv0 = tc::sdesc_sw128(smem_u32(&sm.v[0][0][0][0]), 1024, 3072);
     bool ok = true;
     if (is_qk) {
-      ok = tc::warp_wait(bar(sm.q_full), 0, abort, wlim);
+      ok = tc::warp_wait(bar(sm.q_full), 0, abort);
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int s = j % kTcStages, b = j % 2;
-        ok = tc::warp_wait(bar(sm.k_full[s]), (j / kTcStages) & 1, abort, wlim);
+        ok = tc::warp_wait(bar(sm.k_full[s]), (j / kTcStages) & 1, abort);
         // S buffer b is free once the softmax of tile j-2 has loaded it
-        if (ok && j >= 2) ok = tc::warp_wait(bar(sm.s_free[b]), ((j / 2) - 1) & 1, abort, wlim);
+        if (ok && j >= 2) ok = tc::warp_wait(bar(sm.s_free[b]), ((j / 2) - 1) & 1, abort);
         if (!ok) break;
         tc::fence_after();
         if (tc::elect_one()) {
@@ -321,8 +326,8 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
     } else {
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int s = j % kTcVStages, b = j % 2;
-        ok = tc::warp_wait(bar(sm.v_full[s]), (j / kTcVStages) & 1, abort, wlim) &&
-             tc::warp_wait(bar(sm.p_full[b]), (j / 2) & 1, abort, wlim);
+        ok = tc::warp_wait(bar(sm.v_full[s]), (j / kTcVStages) & 1, abort) &&
+             tc::warp_wait(bar(sm.p_full[b]), (j / 2) & 1, abort);
         if (!ok) break;
         tc::fence_after();
         if (tc::elect_one()) {
@@ -429,7 +434,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       } else {
         bmask = 3u;
       }
-      ok = ok && tc::mbar_wait(bar(sm.s_full[b]), (j / 2) & 1, abort, wlim);
+      ok = ok && tc::mbar_wait(bar(sm.s_full[b]), (j / 2) & 1, abort);
       tc::fence_after();
       uint32_t sr[64];
       tc::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
@@ -491,7 +496,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       if (j + 1 < n_tiles) asm volatile("bar.arrive %0, 64;" ::"r"(pub_mine) : "memory");
       if (__any_sync(0xffffffffu, need)) {
         // O must hold P(j-1) V(j-1) before it is rescaled
-        ok = ok && tc::mbar_wait(bar(sm.pv_done[(j - 1) % 2]), ((j - 1) / 2) & 1, abort, wlim);
+        ok = ok && tc::mbar_wait(bar(sm.pv_done[(j - 1) % 2]), ((j - 1) / 2) & 1, abort);
         tc::fence_after();
         const float alpha = need ? exp2f(m_prev - m_use) : 1.f;
 #pragma unroll 1
@@ -540,7 +545,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       }
       const float lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       // P buffer b is free once O += P(j-2) V(j-2) has read it
-      if (j >= 2) ok = ok && tc::mbar_wait(bar(sm.pv_done[b]), ((j / 2) - 1) & 1, abort, wlim);
+      if (j >= 2) ok = ok && tc::mbar_wait(bar(sm.pv_done[b]), ((j / 2) - 1) & 1, abort);
       tc::fence_after();
       tc::tmem_st32(tP, pk);
       l += lsum;
@@ -548,7 +553,7 @@ attn_tc_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUte
       tc::fence_before();
       tc::mbar_arrive(bar(sm.p_full[b]));
     }
-    ok = ok && tc::mbar_wait(bar(sm.o_final), 0, abort, wlim);
+    ok = ok && tc::mbar_wait(bar(sm.o_final), 0, abort);
     // both loops done: the final reference is in mchain; combine the two partial sums
     asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
     const float m_fin = sm.mchain[m];
@@ -674,7 +679,6 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
   const int nb = b1 - b0;
   const int64_t cur0 = 8 * (t / 8);
   volatile int* abort = &sm.abort;
-  const uint32_t wlim = tc::wait_limit();  // pipeline wait limit of this launch
   auto bar = [](uint64_t& b) { return smem_u32(&b); };
   if (threadIdx.x == 0) {
     sm.abort = 0;
@@ -743,7 +747,7 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
       bool ok = true;
       if (lane < kDecIssuers && b < nblocks) {
         const int slot = b % kDecSlots;
-        if (b >= kDecSlots) ok = tc::mbar_wait(bar(sm.empty[slot]), ((b / kDecSlots) - 1) & 1, abort, wlim);
+        if (b >= kDecSlots) ok = tc::mbar_wait(bar(sm.empty[slot]), ((b / kDecSlots) - 1) & 1, abort);
         if (ok) {
           const int32_t r = b < nb ? sm.rows[b] : -64;  // -64: zero-filled tail block
           tc::mbar_expect_tx(bar(sm.full[slot]), 2 * 3 * 1024);
@@ -764,8 +768,8 @@ attn_decode_tma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
     for (int s = cw; s < nsteps; s += 4) {
       const int ba = 2 * s, bb = 2 * s + 1;
       const int sa = ba % kDecSlots, sb2 = bb % kDecSlots;
-      if (!tc::mbar_wait(bar(sm.full[sa]), (ba / kDecSlots) & 1, abort, wlim)) break;
-      if (!tc::mbar_wait(bar(sm.full[sb2]), (bb / kDecSlots) & 1, abort, wlim)) break;
+      if (!tc::mbar_wait(bar(sm.full[sa]), (ba / kDecSlots) & 1, abort)) break;
+      if (!tc::mbar_wait(bar(sm.full[sb2]), (bb / kDecSlots) & 1, abort)) break;
       // token mask: 8 tokens per block; the current block only up to t; zero blocks none
       uint32_t tm = 0;
 #pragma unroll

@@ -18,11 +18,11 @@ __device__ int g_status;
 
 // Every spin-wait gives up after this many nanoseconds of %globaltimer.  The
 // pipeline waits (a consumer waiting for data, a producer for a free slot)
-// read the limit from g_wait_limit_ns, which sgqa_set_wait_limit_ns() may
-// lower; the drains that let in-flight copies and MMAs land before a kernel
+// read the limit from g_wait_limit_ns (constant memory: a cached read), which
+// sgqa_set_wait_limit_ns() may lower between launches; the drains that let in-flight copies and MMAs land before a kernel
 // exits always use the full kWaitLimitNs.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-__device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
+__constant__ uint64_t g_wait_limit_ns = kWaitLimitNs;
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;

@@ -86,7 +86,6 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
   const int n_loop = MODE == kScoreSample ? (n_tiles + samp - 1) / samp : n_tiles;
   auto tile_of = [samp](int c) { return MODE == kScoreSample ? c * samp : c; };
   volatile int* abort = &sm.abort;
-  const uint32_t wlim = tc::wait_limit();  // pipeline wait limit of this launch
   auto bar = [](uint64_t& b) { return smem_u32(&b); };
   if (threadIdx.x == 0) {
     sm.abort = 0;
@@ -130,7 +129,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
       __syncwarp();
       for (int c = 0; c < n_loop; ++c) {
         const int s = c % kIdxStages;
-        if (c >= kIdxStages && !tc::warp_wait(bar(sm.a_empty[s]), ((c / kIdxStages) - 1) & 1, abort, wlim)) break;
+        if (c >= kIdxStages && !tc::warp_wait(bar(sm.a_empty[s]), ((c / kIdxStages) - 1) & 1, abort)) break;
         if (tc::elect_one()) {
           tc::mbar_expect_tx(bar(sm.a_full[s]), kIdxCand * 128);
           tc::tma_load_2d(smem_u32(&sm.a[s][0]), &keymap, 0,
@@ -146,11 +145,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
       const uint64_t da0 = tc::sdesc_sw128(smem_u32(&sm.a[0][0]), 16, 1024);
       const uint64_t db0 = tc::sdesc_sw128(smem_u32(&sm.b[0]), 16, 1024);
       constexpr uint32_t kStageUnits = kIdxCand * 128 / 16;  // one key stage in 16-byte units
-      bool ok = tc::warp_wait(bar(sm.b_full), 0, abort, wlim);
+      bool ok = tc::warp_wait(bar(sm.b_full), 0, abort);
       for (int c = 0; ok && c < n_loop; ++c) {
         const int s = c % kIdxStages, ab = c & 1;
-        if (!tc::warp_wait(bar(sm.a_full[s]), (c / kIdxStages) & 1, abort, wlim)) { ok = false; break; }
-        if (c >= 2 && !tc::warp_wait(bar(sm.acc_empty[ab]), ((c >> 1) - 1) & 1, abort, wlim)) { ok = false; break; }
+        if (!tc::warp_wait(bar(sm.a_full[s]), (c / kIdxStages) & 1, abort)) { ok = false; break; }
+        if (c >= 2 && !tc::warp_wait(bar(sm.acc_empty[ab]), ((c >> 1) - 1) & 1, abort)) { ok = false; break; }
         tc::fence_after();
         if (tc::elect_one()) {
 #pragma unroll
@@ -195,7 +194,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap keymap, const __grid_c
       const uint32_t lt_mask = (1u << lane) - 1u;
       for (int c = 0; c < n_loop; ++c) {
         const int ab = c & 1;
-        if (!tc::mbar_wait(bar(sm.acc_full[ab]), (c >> 1) & 1, abort, wlim)) break;
+        if (!tc::mbar_wait(bar(sm.acc_full[ab]), (c >> 1) & 1, abort)) break;
         tc::fence_after();
         const int64_t r = static_cast<int64_t>(tile_of(c)) * kIdxCand + m;  // candidate block id
         const bool tail = static_cast<int64_t>(tile_of(c) + 1) * kIdxCand > ncand_min;

@@ -582,13 +582,17 @@ sgqa_status launch_attn(const sgqa_params* p, int64_t S, int64_t q0, int64_t nq,
   int32_t* ids = ws_at<int32_t>(ws, w.ids_off);
   uint8_t* msk = ws_at<uint8_t>(ws, w.mask_off);
   int32_t* cnt = ws_at<int32_t>(ws, w.cnt_off);
-  // bitmap, prefix of every eighth word, masks
-  const size_t psmem = static_cast<size_t>(nwords) * 4 + static_cast<size_t>((nwords + 7) / 8 + 1) * 4 +
-                       static_cast<size_t>(k) * 8;
+  // bitmap, prefix of every word (or, for wide id ranges, of every eighth), masks
+  auto plan_smem = [&](int pshift) {
+    return static_cast<size_t>(nwords) * 4 + static_cast<size_t>(((nwords - 1) >> pshift) + 2) * 4 +
+           static_cast<size_t>(k) * 8;
+  };
+  const int pshift = plan_smem(0) <= 96 * 1024 ? 0 : 3;
+  const size_t psmem = plan_smem(pshift);
   if (psmem <= 200 * 1024) {
     cudaFuncSetAttribute(sgqa::attn_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
     sgqa::attn_plan_kernel<<<static_cast<unsigned>(units), sgqa::kPlanThreads, psmem, st>>>(
-        sel, sel_count, nq, G, k, nwords, q0, B, ids, msk, cnt);
+        sel, sel_count, nq, G, k, nwords, pshift, q0, B, ids, msk, cnt);
     SGQA_LAUNCH_CHECK("attn_plan_kernel");
   } else {
     const int pow2 = plan_pow2(k);

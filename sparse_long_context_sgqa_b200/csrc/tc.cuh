@@ -8,10 +8,6 @@ namespace sgqa {
 namespace tc {
 
 // ---- mbarrier -------------------------------------------------------------
-// Limits below kFineWaitNs are counted in SM clock cycles (%globaltimer
-// advances in steps of up to a microsecond; at most 2 GHz, `limit` cycles take
-// at most `limit` ns).
-constexpr uint32_t kFineWaitNs = 1000000u;
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
@@ -45,18 +41,6 @@ __device__ __forceinline__ uint32_t mbar_test(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok;
 }
-// The pipeline wait limit of this launch (read once per kernel).
-__device__ __forceinline__ uint32_t wait_limit() {
-  return static_cast<uint32_t>(*reinterpret_cast<volatile uint64_t*>(&g_wait_limit_ns));
-}
-// One completion test under a wait limit: the plain try_wait (which may
-// suspend the thread for a while) at limits of a millisecond or more; below
-// that the non-blocking test_wait, so that a short limit is noticed as soon
-// as the phase is late.
-__device__ __forceinline__ bool mbar_try_lim(uint32_t bar, uint32_t parity, uint32_t limit) {
-  return limit >= kFineWaitNs ? mbar_try(bar, parity) : mbar_test(bar, parity) != 0u;
-}
-
 // Three completion tests issued back to back (one shared-memory round trip
 // instead of three); bit i of the result is barrier i's test.
 __device__ __forceinline__ uint32_t mbar_test3(uint32_t b0, uint32_t p0, uint32_t b1, uint32_t p1, uint32_t b2,
@@ -95,28 +79,33 @@ __device__ __forceinline__ uint32_t mbar_test6(const uint32_t (&b)[6], const uin
       : "memory");
   return ok;
 }
-// Wait for the phase with the given parity to complete; gives up after
-// `limit` ns (the launch's wait_limit()), records kDevTimeout and returns
-// false.  `abort` (shared)
+// Wait for the phase with the given parity to complete; gives up after the
+// pipeline wait limit (g_wait_limit_ns, constant memory), records kDevTimeout
+// and returns false.  `abort` (shared)
 // short-cuts every later wait of the CTA once one has given up.
 // A wait also gives up at once when any CTA of any kernel has already
 // recorded a failure (device status word set), so a broken launch ends after
 // one bounded wait instead of one per CTA.
-__device__ __forceinline__ uint64_t wait_clock(bool fine) {
-  return fine ? static_cast<uint64_t>(clock64()) : globaltimer_ns();
-}
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint32_t limit) {
-  if (mbar_try_lim(bar, parity, limit)) return true;
+// The hot path is one try_wait (which may suspend the thread until the phase
+// completes).  Limits under a millisecond (a diagnostic setting) use the
+// non-blocking test_wait instead, timed by the SM clock (%globaltimer's ticks
+// are up to a microsecond apart; at most 2 GHz, `limit` cycles take at most
+// `limit` ns), so that a short limit is noticed as soon as the phase is late.
+constexpr uint64_t kFineWaitNs = 1000000u;
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  const uint64_t limit = g_wait_limit_ns;
   const bool fine = limit < kFineWaitNs;
-  const uint64_t t0 = wait_clock(fine);
+  if (fine ? mbar_test(bar, parity) != 0u : mbar_try(bar, parity)) return true;
+  auto now = [fine]() -> uint64_t { return fine ? static_cast<uint64_t>(clock64()) : globaltimer_ns(); };
+  const uint64_t t0 = now();
   for (uint32_t it = 0;; ++it) {
-    if (mbar_try_lim(bar, parity, limit)) return true;
+    if (fine ? mbar_test(bar, parity) != 0u : mbar_try(bar, parity)) return true;
     if (*abort) return false;
     if ((it & 1023u) == 1023u && *reinterpret_cast<volatile int*>(&g_status) != 0) {
       *abort = 1;
       return false;
     }
-    if (wait_clock(fine) - t0 > limit) {
+    if (now() - t0 > limit) {
       *abort = 1;
       report(kDevTimeout);
       return false;
@@ -136,8 +125,8 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
 // mbar_wait by every lane of a converged warp, with one result for the whole
 // warp (a lane whose wait gave up makes every lane see false), so the warp
 // stays converged for the elect/sync steps that follow.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint32_t limit) {
-  const bool r = mbar_wait(bar, parity, abort, limit);
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  const bool r = mbar_wait(bar, parity, abort);
   return __all_sync(0xffffffffu, r);
 }
 // One lane of a converged warp (the lowest active one) returns true.
