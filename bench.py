@@ -262,8 +262,9 @@ def stage_times(wl, p, model, q, dev, paged=None, cov_rows_per_chunk=0):
 
 def union_stats(sel, cnt, wl):
     """Blocks per 8-query unit (the attention kernel's work) against blocks per
-    query, and the mean Jaccard overlap |A & B| / |A | B| of adjacent queries'
-    selections (pairs 2i, 2i+1 of the chunk, every group)."""
+    query, the mean Jaccard overlap |A & B| / |A | B| of adjacent queries'
+    selections (pairs 2i, 2i+1 of the chunk, every group), and distinct blocks
+    per 64-query segment."""
     S, n, G, k = sel.shape
     nb = n // 8
     u = sel[:, :nb * 8].reshape(S, nb, 8, G, k).permute(0, 1, 3, 2, 4).reshape(-1, 8 * k)
@@ -277,8 +278,18 @@ def union_stats(sel, cnt, wl):
     inter = ((x[..., 1:] == x[..., :-1]) & (x[..., 1:] >= 0)).sum(-1).double()
     ca, cb = cnt[:, 0:2 * npair:2].double(), cnt[:, 1:2 * npair:2].double()
     jac = float((inter / torch.clamp(ca + cb - inter, min=1.0)).mean())
+    # distinct blocks over each 64-query segment (8 units): the K/V a segment's
+    # units read between them, which adjacent units share through L2
+    nseg = n // 64
+    seg = 0.0
+    if nseg > 0:
+        v = sel[:, :nseg * 64].reshape(S, nseg, 64, G, k).permute(0, 1, 3, 2, 4).reshape(-1, 64 * k)
+        v = torch.sort(v, dim=-1).values
+        dv = ((v[:, 1:] != v[:, :-1]) & (v[:, 1:] >= 0)).sum(-1) + (v[:, 0] >= 0).to(torch.int64)
+        seg = float(dv.double().mean())
     return {"blocks_per_unit": per_unit, "blocks_per_query": per_query,
-            "inflation": per_unit / max(per_query, 1e-9), "jaccard_adjacent": jac}
+            "inflation": per_unit / max(per_query, 1e-9), "jaccard_adjacent": jac,
+            "blocks_per_segment64": seg}
 
 
 def ranks_from_env(env=None):

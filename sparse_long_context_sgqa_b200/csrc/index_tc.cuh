@@ -1183,14 +1183,15 @@ topk_staged_kernel(const uint2* __restrict__ staging, const int32_t* __restrict_
 // A linear 2048-bin histogram between the kept scores' minimum and maximum
 // finds the bin holding the k-th largest; entries of higher bins are taken,
 // the boundary bin's entries are ranked exactly (score, then smaller id) by
-// one warp (by counting when there are at most 64).  Each list holds its ids
+// one warp (by counting when there are at most 64); a boundary bin too full
+// for its buffer is split once more into 2048 sub-bins, and a sub-bin still
+// too full (exact ties) is resolved by key and id threshold searches.  Each list holds its ids
 // ascending (the score kernel appends candidate tiles in order), so the taken
 // entries of a list stay ascending: the output is the merge of four sorted
 // runs -- each taken entry's place is its rank in its own run plus, in each
 // other run, the number of taken ids below its own (a binary search).  Rows
-// with fewer than k kept entries, an overflowing list or a boundary bin
-// larger than its buffer (massive exact ties) are flagged and listed for the
-// fallback.
+// with fewer than k kept entries or an overflowing list are flagged and
+// listed for the fallback.
 constexpr int kStagedBigThreads = 1024;
 constexpr int kStagedBigPer = 16;
 constexpr int kStagedBigBnd = 4096;  // boundary entries resolved in the kernel
@@ -1206,8 +1207,105 @@ struct StagedBigSmem {
   uint32_t T[2048];                           // taken ids, the four runs one after the other
   float rmax[kStagedBigWarps], rmin[kStagedBigWarps];
   uint32_t wsum[kStagedBigWarps];
+  uint32_t wk[4][kStagedBigWarps];            // per-warp key / id ranges
+  uint2 cut;                                  // (key, id) thresholds of a tied sub-bin
   uint32_t bstar, rem, cstar, nb, runs[5];
 };
+
+// Bin of a score: bins ordered best first, 2048 across [mn, mx]; the product
+// rounds monotonically, so a higher score never falls in a later bin.
+__device__ __forceinline__ int staged_bin(float mx, float scale, float x) {
+  return min(static_cast<int>(__fmul_rn(__fsub_rn(mx, x), scale)), kStagedBigBins - 1);
+}
+// Sub-bin of a score of bin bstar: the fractional part of the same scaled
+// distance (scaling by 2048 is exact), so the order stays monotone across levels.
+__device__ __forceinline__ int staged_sub(float mx, float scale2, int bstar, float x) {
+  return min(max(static_cast<int>(__fmul_rn(__fsub_rn(mx, x), scale2)) - kStagedBigBins * bstar, 0),
+             kStagedBigBins - 1);
+}
+
+// The rem best entries (score, then smaller id) of sub-bin sstar of bin bstar,
+// when there are more of them than the boundary buffer holds: the largest key
+// K with at least rem entries at or above it, then the smallest id X with
+// enough entries of key K at or below it.  Entries above K, and those of key K
+// with id <= X, are the ones taken (ids are distinct, so exactly rem).
+// Returns (K, X).  Called by every thread of the block.
+__device__ __forceinline__ uint2 staged_tie_cut(StagedBigSmem& sm, const uint2* __restrict__ lists, int cap, int p1,
+                                               int p2, int p3, int cnt, float mx, float scale, float scale2,
+                                               int bstar, int sstar, uint32_t rem) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // entry x of this thread, if it lies in the boundary sub-bin (else key 0);
+  // read again from the lists (L2) on every pass, which keeps registers free
+  auto load = [&](int x) -> uint2 {
+    const int j = tid + kStagedBigThreads * x;
+    if (j >= cnt) return make_uint2(0u, 0u);
+    const int q = (j >= p1) + (j >= p2) + (j >= p3);
+    const uint2 en = lists[q * static_cast<int64_t>(cap) + (j - (q == 0 ? 0 : q == 1 ? p1 : q == 2 ? p2 : p3))];
+    const float v = key_score(en.x);
+    const bool in = staged_bin(mx, scale, v) == bstar && staged_sub(mx, scale2, bstar, v) == sstar;
+    return in ? en : make_uint2(0u, 0u);
+  };
+  uint32_t k0 = 0xFFFFFFFFu, k1 = 0u, i0 = 0xFFFFFFFFu, i1 = 0u;
+#pragma unroll 4
+  for (int x = 0; x < kStagedBigPer; ++x) {
+    const uint2 en = load(x);
+    if (en.x != 0u) {  // every real key is above 0
+      k0 = min(k0, en.x);
+      k1 = max(k1, en.x);
+      i0 = min(i0, en.y);
+      i1 = max(i1, en.y);
+    }
+  }
+  k0 = __reduce_min_sync(0xffffffffu, k0);
+  k1 = __reduce_max_sync(0xffffffffu, k1);
+  i0 = __reduce_min_sync(0xffffffffu, i0);
+  i1 = __reduce_max_sync(0xffffffffu, i1);
+  __syncthreads();  // every thread has read the previous scan's totals
+  if (lane == 0) {
+    sm.wk[0][warp] = k0;
+    sm.wk[1][warp] = k1;
+    sm.wk[2][warp] = i0;
+    sm.wk[3][warp] = i1;
+  }
+  __syncthreads();
+  for (int w = 0; w < kStagedBigWarps; ++w) {
+    k0 = min(k0, sm.wk[0][w]);
+    k1 = max(k1, sm.wk[1][w]);
+    i0 = min(i0, sm.wk[2][w]);
+    i1 = max(i1, sm.wk[3][w]);
+  }
+  // number of boundary entries with key >= kmin and (key > kmax or id <= xmax), over the block
+  auto block_count = [&](uint32_t kmin, uint32_t kmax, uint32_t xmax) -> uint32_t {
+    uint32_t c = 0;
+#pragma unroll 4
+    for (int x = 0; x < kStagedBigPer; ++x) {
+      const uint2 en = load(x);
+      c += en.x != 0u && en.x >= kmin && (en.x > kmax || en.y <= xmax);
+    }
+    c = __reduce_add_sync(0xffffffffu, c);
+    __syncthreads();  // every thread has read the previous counts
+    if (lane == 0) sm.wsum[warp] = c;
+    __syncthreads();
+    uint32_t t = 0;
+    for (int w = 0; w < kStagedBigWarps; ++w) t += sm.wsum[w];
+    return t;
+  };
+  uint32_t lo = k0, hi = k1;  // every boundary entry has key >= k0, and there are >= rem of them
+  while (lo < hi) {
+    const uint32_t mid = lo + (hi - lo + 1) / 2;
+    if (block_count(mid, 0u, 0xFFFFFFFFu) >= rem) lo = mid;  // key >= mid
+    else hi = mid - 1;
+  }
+  const uint32_t kcut = lo;
+  lo = i0;
+  hi = i1;  // key > K, or key == K and id <= i1: all entries at or above K, >= rem
+  while (lo < hi) {
+    const uint32_t mid = lo + (hi - lo) / 2;
+    if (block_count(kcut, kcut, mid) >= rem) hi = mid;
+    else lo = mid + 1;
+  }
+  return make_uint2(kcut, lo);
+}
 
 __global__ void __launch_bounds__(kStagedBigThreads)
 topk_staged_sort_kernel(const uint2* __restrict__ staging, const int32_t* __restrict__ staged, int64_t nq, int G,
@@ -1280,11 +1378,7 @@ topk_staged_sort_kernel(const uint2* __restrict__ staging, const int32_t* __rest
   }
   const float width = mx - mn;
   const float scale = width > 0.f ? (kStagedBigBins - 0.5f) / width : 0.f;
-  // bins ordered best first; the product rounds monotonically, so a higher
-  // score never falls in a later bin
-  auto bin_of = [&](float x) -> int {
-    return min(static_cast<int>(__fmul_rn(__fsub_rn(mx, x), scale)), kStagedBigBins - 1);
-  };
+  auto bin_of = [&](float x) -> int { return staged_bin(mx, scale, x); };
 #pragma unroll
   for (int x = 0; x < kStagedBigPer; ++x)
     if (tid + kStagedBigThreads * x < cnt) atomicAdd(&sm.hist[bin_of(key_score(e[x].x))], 1u);
@@ -1313,17 +1407,77 @@ topk_staged_sort_kernel(const uint2* __restrict__ staging, const int32_t* __rest
     }
   }
   __syncthreads();
-  if (sm.cstar > kStagedBigBnd) {  // the boundary does not fit its buffer
-    flag_row();
-    return;
-  }
   const int bstar = static_cast<int>(sm.bstar);
-  const uint32_t rem = sm.rem;
+  uint32_t rem = sm.rem;
+  // A boundary bin too full for its buffer (a few outlying scores stretch the
+  // bins) is split once more: its entries in 2048 sub-bins of its own width.
+  const float scale2 = scale * static_cast<float>(kStagedBigBins);
+  auto sub_of = [&](float x) -> int { return staged_sub(mx, scale2, bstar, x); };
+  const bool split = sm.cstar > kStagedBigBnd;  // (uniform)
+  int sstar = -1;
+  if (split) {
+    __syncthreads();  // the first level's scan has read the histogram
+    for (int b = tid; b < kStagedBigBins; b += kStagedBigThreads) sm.hist[b] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int x = 0; x < kStagedBigPer; ++x) {
+      const int j = tid + kStagedBigThreads * x;
+      if (j < cnt) {
+        const float v = key_score(e[x].x);
+        if (bin_of(v) == bstar) atomicAdd(&sm.hist[sub_of(v)], 1u);
+      }
+    }
+    __syncthreads();
+    {
+      const uint32_t c0 = sm.hist[2 * tid], c1 = sm.hist[2 * tid + 1];
+      uint32_t x = c0 + c1;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane == 31) sm.wsum[warp] = x;
+      __syncthreads();
+      uint32_t before = x - c0 - c1;
+      for (int w = 0; w < warp; ++w) before += sm.wsum[w];
+      if (before < rem && rem <= before + c0) {
+        sm.bstar = 2 * tid;  // (reused: the sub-bin)
+        sm.rem = rem - before;
+        sm.cstar = c0;
+      } else if (before + c0 < rem && rem <= before + c0 + c1) {
+        sm.bstar = 2 * tid + 1;
+        sm.rem = rem - before - c0;
+        sm.cstar = c1;
+      }
+    }
+    __syncthreads();
+    sstar = static_cast<int>(sm.bstar);
+    rem = sm.rem;
+  }
+  // A sub-bin still too full for the buffer holds (nearly) equal scores, e.g.
+  // many exact zeros: its rem best entries are found by threshold searches
+  // (on entries it reads again from the lists, so that the registers holding
+  // this thread's own stay untouched).
+  const bool wide = split && sm.cstar > kStagedBigBnd;  // (uniform)
+  if (wide) {
+    const uint2 cut = staged_tie_cut(sm, lists, cap, p1, p2, p3, cnt, mx, scale, scale2, bstar, sstar, rem);
+    if (tid == 0) sm.cut = cut;
+    __syncthreads();
+  }
 #pragma unroll
   for (int x = 0; x < kStagedBigPer; ++x) {
     const int j = tid + kStagedBigThreads * x;
     if (j >= cnt) continue;
-    const int b = bin_of(key_score(e[x].x));
+    const float v = key_score(e[x].x);
+    int b = bin_of(v);
+    if (split && b == bstar) {  // order within the boundary bin by sub-bin
+      const int sb = sub_of(v);
+      b = sb < sstar ? bstar - 1 : (sb == sstar ? bstar : bstar + 1);
+      if (wide && b == bstar) {  // resolved by the thresholds
+        const uint2 cut = sm.cut;
+        b = (e[x].x > cut.x || (e[x].x == cut.x && e[x].y <= cut.y)) ? bstar - 1 : bstar + 1;
+      }
+    }
     if (b < bstar) {
       atomicOr(&sm.tbits[j >> 5], 1u << (j & 31));
     } else if (b == bstar) {

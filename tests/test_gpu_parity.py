@@ -135,7 +135,7 @@ def test_index_topk_parity(cuda_device, case):
 
 
 @pytest.mark.parametrize("case", ["short_rows", "filtered_rows", "filtered_rows_65k", "dup_short", "dup_long",
-                                  "decode_rows", "dup_decode", "filtered_k2048", "dup_k2048"])
+                                  "decode_rows", "dup_decode", "filtered_k2048", "dup_k2048", "zeros_k2048"])
 def test_index_topk_exact_ties(cuda_device, case):
     """Exact score ties, which the selection must break toward smaller block ids.
 
@@ -164,9 +164,17 @@ def test_index_topk_exact_ties(cuda_device, case):
     filtered_k2048 / dup_k2048: B = 1 and top-2048 (the 1M-context B = 1
     variant's selection) at 32768..33023 candidates: the filtered path with
     kept lists of 2k and the select for k above 512, which merges the four
-    ascending lists' taken ids."""
-    dup = case.startswith("dup")
-    if case in ("filtered_k2048", "dup_k2048"):
+    ascending lists' taken ids.
+
+    zeros_k2048: the same rows over the 211-key store, with head weights
+    (-1, -1, 0, ...) in every third row: every score is <= 0 and a candidate
+    scores exactly 0 when both weighted heads' ReLU inputs are <= 0, about a
+    quarter of them (5k..12k per row).  The k-th best falls inside that group
+    of exact zeros, which fills one histogram bin and one sub-bin beyond the
+    boundary buffer, and is resolved by the key / id threshold searches; the
+    selection must be the group's 2048 smallest ids."""
+    dup = case.startswith("dup") or case == "zeros_k2048"
+    if case in ("filtered_k2048", "dup_k2048", "zeros_k2048"):
         wl = dataclasses.replace(WL["prefill8k"], name="ties_k2048", seq_len=40960, block=1, topk=2048)
         q0, nq = 32768, 256  # candidates 32768 .. 33023 per query (B = 1)
     elif case in ("decode_rows", "dup_decode"):
@@ -187,9 +195,14 @@ def test_index_topk_exact_ties(cuda_device, case):
     cache, _ = Hn.make_inputs(wl, cuda_device)
     qs = I.make_queries(wl, cuda_device, q0, nq)
     zero = torch.zeros(nq, dtype=torch.bool, device=cuda_device)
+    neg = torch.zeros(nq, dtype=torch.bool, device=cuda_device)
     if not dup:
         zero[::3] = True
         qs["idx_w"][zero] = 0.0
+    if case == "zeros_k2048":
+        neg[::3] = True
+        qs["idx_w"][neg] = 0.0
+        qs["idx_w"][neg, :, :2] = -1.0
     _, codes, keys = Hn.oracle_keys(Hn.to_np(cache["kp"][0]), Hn.to_np(cache["c"][0]), wl.block)
     if dup:
         codes = np.ascontiguousarray(codes[np.arange(codes.shape[0]) % 211])
@@ -209,8 +222,25 @@ def test_index_topk_exact_ties(cuda_device, case):
     iq, iw = Hn.to_np(qs["idx_q"]), Hn.to_np(qs["idx_w"])
     ties = 0
     step = {"short_rows": 397, "dup_short": 397, "filtered_rows_65k": 397, "decode_rows": 2, "dup_decode": 2,
-            "filtered_k2048": 19, "dup_k2048": 19}.get(case, 97)
+            "filtered_k2048": 19, "dup_k2048": 19, "zeros_k2048": 19}.get(case, 97)
     rows = [i for i in range(1, nq, step) if not zero_np[i]] + [nq - 1]
+    if case == "zeros_k2048":
+        rows = list(range(0, nq, 3 * 7))  # weight-(-1, -1) rows only
+        wide = 0
+        for i in rows:
+            for g in range(wl.groups):
+                cand = keys[:(q0 + i) // wl.block]
+                dots = cand.astype(np.float64) @ iq[i, g, :2].astype(np.float64).T
+                if np.abs(dots).min() < 1e-3:  # a sign the fp32 sums might not share
+                    continue
+                grp = np.flatnonzero(np.all(dots <= 0.0, axis=1))
+                if grp.size < wl.topk:  # the zeros and the best of the rest
+                    ties += Hn.check_selection(sel[i, g], O.index_scores(iq[i, g], iw[i, g], cand), wl.topk)
+                    continue
+                wide += grp.size > 4096
+                assert np.array_equal(sel[i, g], grp[:wl.topk]), (i, g)
+        assert wide > 0 and ties <= 2 * len(rows)
+        return
     for i in rows:
         for g in range(wl.groups):
             sc = O.index_scores(iq[i, g], iw[i, g], keys[:(q0 + i) // wl.block])
