@@ -46,10 +46,11 @@ METRIC = {
 # profiles/ give the commands and figures); None where no capture of the
 # current kernel exists.
 TRAFFIC = {
-    "prefill128k": 2101091360,   # attn_tc_kernel, mean over the 16 chunk launches of one step
+    "prefill128k": 2089586144,   # attn_tc_kernel, mean over the 16 chunk launches of one step
     "prefill8k": None,           # not captured for the current kernel
     "prefill1m": None,           # dominant stage: the index stage (several kernels, tensor/ALU bound)
-    "decode": None,              # not captured for the current kernel
+    "prefill1m_b1": None,        # dominant stage: the index stage
+    "decode": 236356608,         # attn_decode_tma_kernel: a 4-sequence launch (59089152 B) scaled to 16 sequences
 }
 
 
@@ -411,7 +412,10 @@ def cuda_arm(args, wl, rank, world, local_rank):
 
     peaks = load_peaks()
     per_launch_ms = {k: v / max(1, work["launches"]) for k, v in ms_stage.items()}
-    traffic = None if paged is not None else TRAFFIC.get(wl.name)  # captured for the contiguous caches
+    # captured for the contiguous caches at the workload's own sizes
+    base = I.WORKLOADS.get(wl.name)
+    same = base is not None and (base.seq_len, base.num_seqs) == (wl.seq_len, wl.num_seqs)
+    traffic = TRAFFIC.get(wl.name) if paged is None and same else None
     if wl.nq <= 32:
         achieved = work["attn_bytes"] / work["launches"] / (per_launch_ms["attention"] / 1e3) / 1e9
         roof = {"kernel": "sparse attention (decode gather: attn_decode_tma_kernel)", "bound": "hbm",
