@@ -54,6 +54,14 @@ TRAFFIC = {
 }
 
 
+def captured_traffic(wl, paged: bool):
+    """The TRAFFIC figure for this run, or None: the captures cover the
+    contiguous caches at each workload's own sizes only."""
+    base = I.WORKLOADS.get(wl.name)
+    same = base is not None and (base.seq_len, base.num_seqs) == (wl.seq_len, wl.num_seqs)
+    return TRAFFIC.get(wl.name) if same and not paged else None
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -412,10 +420,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
 
     peaks = load_peaks()
     per_launch_ms = {k: v / max(1, work["launches"]) for k, v in ms_stage.items()}
-    # captured for the contiguous caches at the workload's own sizes
-    base = I.WORKLOADS.get(wl.name)
-    same = base is not None and (base.seq_len, base.num_seqs) == (wl.seq_len, wl.num_seqs)
-    traffic = TRAFFIC.get(wl.name) if paged is None and same else None
+    traffic = captured_traffic(wl, paged is not None)
     if wl.nq <= 32:
         achieved = work["attn_bytes"] / work["launches"] / (per_launch_ms["attention"] / 1e3) / 1e9
         roof = {"kernel": "sparse attention (decode gather: attn_decode_tma_kernel)", "bound": "hbm",

@@ -1,4 +1,5 @@
-"""The JSON line of bench.py's reference arm (CPU oracle), as the driver reads it."""
+"""The JSON line of bench.py's reference arm (CPU oracle), as the driver reads it, and the
+bench's host-side rules."""
 import importlib.util
 import json
 import os
@@ -35,3 +36,18 @@ def test_reference_arm_json_line():
     assert d["value"] > 0 and d["cpu_baseline"]["value"] == d["value"]
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_traffic_only_at_the_captured_sizes():
+    """roofline.traffic comes from captures of each workload at its own sizes
+    on contiguous caches: a run with other sizes or a paged pool reports null."""
+    import dataclasses
+    bench = _load_bench()
+    wl = bench.I.WORKLOADS["decode"]
+    assert bench.captured_traffic(wl, False) == bench.TRAFFIC["decode"] is not None
+    assert bench.captured_traffic(wl, True) is None
+    assert bench.captured_traffic(dataclasses.replace(wl, num_seqs=4), False) is None
+    assert bench.captured_traffic(dataclasses.replace(wl, seq_len=32768, q_start=32767), False) is None
+    big = bench.I.WORKLOADS["prefill128k"]
+    assert bench.captured_traffic(big, False) == bench.TRAFFIC["prefill128k"] is not None
+    assert bench.captured_traffic(bench.I.WORKLOADS["prefill1m"], False) is None
